@@ -1,0 +1,191 @@
+"""Seeded synthetic inputs for the block-quantized matmul y = x . dequant(Wq)^T.
+
+This module is the one place that both the CUDA path's tests/benchmarks and
+the CPU oracle take their inputs from.  It draws random numbers and packs
+them into the block formats' byte layouts; it never decodes a block and never
+computes a product, so it holds none of the matmul's arithmetic.
+
+Formats (the llama.cpp "legacy" and "K-quant" families that "Llamas na Web"
+names in its problem statement and in "3. Design de Shader Consciente de
+Quantizacao"):
+
+* Q8_0 -- 32 weights per 34-byte block: little-endian fp16 ``d`` then 32
+  int8 codes ``q``; the weight is ``q*d``.
+* Q4_0 -- 32 weights per 18-byte block: fp16 ``d`` then 16 bytes; byte ``i``
+  holds element ``i`` in its low nibble and element ``i+16`` in its high
+  nibble; the weight is ``(nibble-8)*d``.
+* Q4_K -- 256 weights per 144-byte superblock: fp16 ``d``, fp16 ``dmin``,
+  12 bytes holding eight 6-bit (scale, min) pairs, 128 bytes of nibbles.
+
+Draw order for one tensor: a fresh ``numpy.random.default_rng(seed)``
+(PCG64) draws the weight tensor first (row-major [N][K]) and then the
+activations ([M][K]).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+QK = 32          # weights per Q8_0 / Q4_0 block
+QK_K = 256       # weights per Q4_K superblock
+BLOCK_BYTES = {"q8_0": 34, "q4_0": 18, "q4_k": 144}
+BLOCK_WEIGHTS = {"q8_0": QK, "q4_0": QK, "q4_k": QK_K}
+
+
+def row_bytes(fmt: str, K: int) -> int:
+    """Bytes of one packed weight row of K weights."""
+    bw = BLOCK_WEIGHTS[fmt]
+    if K % bw:
+        raise ValueError(f"K={K} is not a multiple of the {fmt} block ({bw})")
+    return K // bw * BLOCK_BYTES[fmt]
+
+
+def rng(seed: int) -> np.random.Generator:
+    return np.random.default_rng(seed)
+
+
+def normal_weights(g: np.random.Generator, N: int, K: int, std: float = 0.02) -> np.ndarray:
+    """fp32 weights ~ N(0, std^2), row-major [N][K]."""
+    return (g.standard_normal((N, K), dtype=np.float32) * np.float32(std)).astype(np.float32)
+
+
+def _f16_bits(a: np.ndarray) -> np.ndarray:
+    """Round fp32 to fp16 (nearest-even, numpy's cast) and return the 16-bit codes."""
+    return np.ascontiguousarray(a.astype(np.float16)).view(np.uint16)
+
+
+def _round_half_away(v: np.ndarray) -> np.ndarray:
+    return (np.sign(v) * np.floor(np.abs(v) + np.float32(0.5))).astype(np.float32)
+
+
+def quantize_q8_0(w: np.ndarray) -> np.ndarray:
+    """Pack fp32 weights [N][K] into Q8_0 bytes [N][K/32*34].
+
+    Per block of 32: d32 = max|w| / 127 in fp32, stored as fp16(d32);
+    q = round(w / d32), halves away from zero, clamped to [-127, 127];
+    an all-zero block stores d = 0, q = 0.
+    """
+    N, K = w.shape
+    nb = K // QK
+    wb = w.reshape(N, nb, QK).astype(np.float32)
+    amax = np.abs(wb).max(axis=-1)
+    d32 = (amax / np.float32(127.0)).astype(np.float32)
+    safe = np.where(d32 > 0, d32, np.float32(1.0))
+    q = _round_half_away(wb / safe[..., None])
+    q = np.clip(q, -127, 127)
+    q = np.where(d32[..., None] > 0, q, 0).astype(np.int8)
+    out = np.empty((N, nb, 34), dtype=np.uint8)
+    out[..., 0:2] = _f16_bits(d32).view(np.uint8).reshape(N, nb, 2)
+    out[..., 2:34] = q.view(np.uint8)
+    return out.reshape(N, nb * 34)
+
+
+def quantize_q4_0(w: np.ndarray) -> np.ndarray:
+    """Pack fp32 weights [N][K] into Q4_0 bytes [N][K/32*18].
+
+    Per block of 32: amax = the signed weight of largest magnitude (first
+    index wins a tie); d32 = amax / -8 in fp32, stored as fp16(d32);
+    q = min(15, round(w/d32 + 8)) with halves rounded up, floored at 0;
+    an all-zero block stores d = 0 and every code 8.
+    """
+    N, K = w.shape
+    nb = K // QK
+    wb = w.reshape(N, nb, QK).astype(np.float32)
+    idx = np.abs(wb).argmax(axis=-1)
+    amax = np.take_along_axis(wb, idx[..., None], axis=-1)[..., 0]
+    d32 = (amax / np.float32(-8.0)).astype(np.float32)
+    safe = np.where(d32 != 0, d32, np.float32(1.0))
+    v = (wb / safe[..., None] + np.float32(8.0)).astype(np.float32)
+    q = np.floor(v + np.float32(0.5))
+    q = np.clip(q, 0, 15)
+    q = np.where(d32[..., None] != 0, q, 8).astype(np.uint8)
+    packed = (q[..., :16] | (q[..., 16:] << 4)).astype(np.uint8)
+    out = np.empty((N, nb, 18), dtype=np.uint8)
+    out[..., 0:2] = _f16_bits(d32).view(np.uint8).reshape(N, nb, 2)
+    out[..., 2:18] = packed
+    return out.reshape(N, nb * 18)
+
+
+def random_q4_k(g: np.random.Generator, N: int, K: int) -> np.ndarray:
+    """Random Q4_K bytes [N][K/256*144].
+
+    d and dmin ~ U(0, 0.01) drawn in fp32 and rounded to fp16; the 12
+    scale/min bytes and the 128 nibble bytes are uniform random bytes (every
+    bit of the 12 bytes belongs to exactly one 6-bit field, so uniform bytes
+    give uniform 6-bit scales and mins).  Draw order: d[N][nb], dmin[N][nb],
+    scale bytes[N][nb][12], nibble bytes[N][nb][128].
+    """
+    nb = K // QK_K
+    if K % QK_K:
+        raise ValueError("Q4_K needs K % 256 == 0")
+    d = g.uniform(0.0, 0.01, size=(N, nb)).astype(np.float32)
+    dmin = g.uniform(0.0, 0.01, size=(N, nb)).astype(np.float32)
+    sc = g.integers(0, 256, size=(N, nb, 12), dtype=np.uint8)
+    qs = g.integers(0, 256, size=(N, nb, 128), dtype=np.uint8)
+    out = np.empty((N, nb, 144), dtype=np.uint8)
+    out[..., 0:2] = _f16_bits(d).view(np.uint8).reshape(N, nb, 2)
+    out[..., 2:4] = _f16_bits(dmin).view(np.uint8).reshape(N, nb, 2)
+    out[..., 4:16] = sc
+    out[..., 16:144] = qs
+    return out.reshape(N, nb * 144)
+
+
+def activations(g: np.random.Generator, M: int, K: int, act: str) -> np.ndarray:
+    """x ~ N(0,1) drawn in fp32 [M][K], then stored in ``act``.
+
+    Returns float32 for "f32", float16 for "f16" and the uint16 bit codes of
+    bf16 (round to nearest even) for "bf16".
+    """
+    x = g.standard_normal((M, K), dtype=np.float32)
+    if act == "f32":
+        return np.ascontiguousarray(x)
+    if act == "f16":
+        return np.ascontiguousarray(x.astype(np.float16))
+    if act == "bf16":
+        return f32_to_bf16_bits(x)
+    raise ValueError(act)
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 codes, round to nearest even (finite inputs)."""
+    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    lsb = (b >> 16) & 1
+    r = (b + 0x7FFF + lsb) >> 16
+    return r.astype(np.uint16)
+
+
+def make_weights(fmt: str, g: np.random.Generator, N: int, K: int) -> np.ndarray:
+    """Packed weights for one tensor, drawn from ``g`` as each format's workload specifies."""
+    if fmt == "q8_0":
+        return quantize_q8_0(normal_weights(g, N, K))
+    if fmt == "q4_0":
+        return quantize_q4_0(normal_weights(g, N, K))
+    if fmt == "q4_k":
+        return random_q4_k(g, N, K)
+    raise ValueError(fmt)
+
+
+def make_problem(fmt: str, act: str, M: int, N: int, K: int, seed: int = 0):
+    """(Wq bytes [N][row_bytes], x [M][K] in ``act``) from one seeded stream: W first, then x."""
+    g = rng(seed)
+    Wq = make_weights(fmt, g, N, K)
+    x = activations(g, M, K, act)
+    return Wq, x
+
+
+# The workloads, by what they are (format, activation dtype, shapes, seed).
+WORKLOADS = {
+    "q8_0_gemv_4096x4096": dict(fmt="q8_0", act="f32", Ms=[1], shapes=[(4096, 4096)], seeds=[0]),
+    "q4_0_gemv_11008x4096": dict(fmt="q4_0", act="f32", Ms=[1, 4, 8], shapes=[(11008, 4096)], seeds=[0]),
+    "q4_k_7b_layer_decode": dict(
+        fmt="q4_k", act="f16", Ms=[1],
+        # (N, K) of q, k, v, o, gate, up, down
+        shapes=[(4096, 4096)] * 4 + [(11008, 4096), (11008, 4096), (4096, 11008)],
+        seeds=[0, 1, 2, 3, 4, 5, 6]),
+    "q4_0_prefill_gemm": dict(fmt="q4_0", act="bf16", Ms=[512, 2048],
+                              shapes=[(11008, 4096), (4096, 11008)], seeds=[0, 0]),
+}
+
+SWEEP_FMTS = ["q8_0", "q4_0", "q4_k"]
+SWEEP_MS = [1, 2, 4, 8, 16, 64, 256, 1024]
+SWEEP_SHAPES_KN = [(4096, 4096), (4096, 14336), (14336, 4096), (4096, 32000)]

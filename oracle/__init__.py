@@ -1,0 +1,186 @@
+"""CPU oracle for the block-quantized matmul -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+leg may import this package.  The library under
+``block_quantized_matmul_lwq_b200`` never does, and shares no code with it.
+
+The arithmetic lives in ``lwq_oracle.c`` (plain C, fp64 accumulation, one
+OpenMP loop over output rows); this module only builds it with gcc and
+marshals numpy arrays through ctypes.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "lwq_oracle.c")
+_LIB = os.path.join(_HERE, "liblwq_oracle.so")
+
+FMT = {"q8_0": 1, "q4_0": 2, "q4_k": 3}
+ACT = {"f32": 0, "f16": 1, "bf16": 2}
+
+CFLAGS = ["-O2", "-fopenmp", "-ffp-contract=off", "-shared", "-fPIC", "-std=c11"]
+
+
+def build(out: str = _LIB, extra: list[str] | None = None) -> str:
+    """Compile the oracle with gcc (no-op when the .so is newer than the source)."""
+    if extra is None and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(_SRC):
+        return out
+    cmd = ["gcc", *CFLAGS, *(extra or []), _SRC, "-o", out + ".tmp", "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(out + ".tmp", out)
+    return out
+
+
+_lib = None
+
+
+def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
+    c = ctypes
+    lib.lwq_oracle_f16.restype = c.c_double
+    lib.lwq_oracle_f16.argtypes = [c.c_uint16]
+    lib.lwq_oracle_bf16.restype = c.c_double
+    lib.lwq_oracle_bf16.argtypes = [c.c_uint16]
+    lib.lwq_oracle_row_bytes.restype = c.c_long
+    lib.lwq_oracle_row_bytes.argtypes = [c.c_int, c.c_long]
+    lib.lwq_oracle_q4k_scale_min.restype = None
+    lib.lwq_oracle_q4k_scale_min.argtypes = [c.c_void_p, c.c_int, c.POINTER(c.c_int), c.POINTER(c.c_int)]
+    lib.lwq_oracle_dequant_row.restype = c.c_int
+    lib.lwq_oracle_dequant_row.argtypes = [c.c_int, c.c_void_p, c.c_long, c.c_void_p]
+    lib.lwq_oracle_matmul.restype = c.c_int
+    lib.lwq_oracle_matmul.argtypes = [c.c_int, c.c_int, c.c_void_p, c.c_void_p, c.c_long, c.c_long,
+                                      c.c_long, c.c_void_p, c.c_void_p, c.c_int]
+    lib.lwq_oracle_matmul_sampled.restype = c.c_int
+    lib.lwq_oracle_matmul_sampled.argtypes = [c.c_int, c.c_int, c.c_void_p, c.c_void_p, c.c_long,
+                                              c.c_long, c.c_long, c.c_void_p, c.c_void_p, c.c_long,
+                                              c.c_void_p, c.c_void_p, c.c_int]
+    lib.lwq_oracle_max_threads.restype = c.c_int
+    lib.lwq_oracle_max_threads.argtypes = []
+    return lib
+
+
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load (building first if needed) the oracle library; ``path`` loads another build."""
+    global _lib
+    if path is not None:
+        return _bind(ctypes.CDLL(path))
+    if _lib is None:
+        _lib = _bind(ctypes.CDLL(build()))
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    return a.ctypes.data
+
+
+def _act_of(x: np.ndarray, act: str | None) -> str:
+    if act is not None:
+        return act
+    if x.dtype == np.float32:
+        return "f32"
+    if x.dtype == np.float16:
+        return "f16"
+    raise ValueError("uint16 activations are ambiguous: pass act='bf16' or 'f16'")
+
+
+def f16(code: int, lib=None) -> float:
+    return (lib or load()).lwq_oracle_f16(code)
+
+
+def bf16(code: int, lib=None) -> float:
+    return (lib or load()).lwq_oracle_bf16(code)
+
+
+def row_bytes(fmt: str, K: int, lib=None) -> int:
+    return (lib or load()).lwq_oracle_row_bytes(FMT[fmt], K)
+
+
+def q4k_scale_min(scales12: np.ndarray, j: int, lib=None) -> tuple[int, int]:
+    s = np.ascontiguousarray(scales12, dtype=np.uint8)
+    assert s.size == 12
+    sc, m = ctypes.c_int(), ctypes.c_int()
+    (lib or load()).lwq_oracle_q4k_scale_min(_ptr(s), j, ctypes.byref(sc), ctypes.byref(m))
+    return sc.value, m.value
+
+
+def dequant(fmt: str, Wq: np.ndarray, K: int, lib=None) -> np.ndarray:
+    """Decode packed rows [N][row_bytes] to fp32 [N][K]."""
+    lib = lib or load()
+    Wq = np.ascontiguousarray(Wq, dtype=np.uint8)
+    rb = lib.lwq_oracle_row_bytes(FMT[fmt], K)
+    if rb < 0:
+        raise ValueError(f"bad K={K} for {fmt}")
+    Wq = Wq.reshape(-1, rb)
+    out = np.empty((Wq.shape[0], K), dtype=np.float32)
+    for n in range(Wq.shape[0]):
+        rc = lib.lwq_oracle_dequant_row(FMT[fmt], _ptr(Wq[n]), K, _ptr(out[n]))
+        if rc:
+            raise ValueError("dequant failed")
+    return out
+
+
+def matmul(fmt: str, Wq: np.ndarray, x: np.ndarray, K: int | None = None, act: str | None = None,
+           nthreads: int = 0, lib=None):
+    """(y, den): fp64 [M][N] reference output and sum_k |x*w|."""
+    lib = lib or load()
+    act = _act_of(x, act)
+    x = np.ascontiguousarray(x)
+    M = x.shape[0]
+    K = x.shape[1] if K is None else K
+    rb = lib.lwq_oracle_row_bytes(FMT[fmt], K)
+    Wq = np.ascontiguousarray(Wq, dtype=np.uint8).reshape(-1, rb)
+    N = Wq.shape[0]
+    y = np.empty((M, N), dtype=np.float64)
+    den = np.empty((M, N), dtype=np.float64)
+    rc = lib.lwq_oracle_matmul(FMT[fmt], ACT[act], _ptr(Wq), _ptr(x), M, N, K, _ptr(y), _ptr(den), nthreads)
+    if rc:
+        raise ValueError("oracle matmul failed")
+    return y, den
+
+
+def matmul_sampled(fmt: str, Wq: np.ndarray, x: np.ndarray, ms, ns, K: int | None = None,
+                   act: str | None = None, nthreads: int = 0, lib=None):
+    """(y, den) fp64 for the listed outputs (ms[i], ns[i])."""
+    lib = lib or load()
+    act = _act_of(x, act)
+    x = np.ascontiguousarray(x)
+    M = x.shape[0]
+    K = x.shape[1] if K is None else K
+    rb = lib.lwq_oracle_row_bytes(FMT[fmt], K)
+    Wq = np.ascontiguousarray(Wq, dtype=np.uint8).reshape(-1, rb)
+    N = Wq.shape[0]
+    ms = np.ascontiguousarray(ms, dtype=np.int64)
+    ns = np.ascontiguousarray(ns, dtype=np.int64)
+    y = np.empty(ms.shape[0], dtype=np.float64)
+    den = np.empty(ms.shape[0], dtype=np.float64)
+    rc = lib.lwq_oracle_matmul_sampled(FMT[fmt], ACT[act], _ptr(Wq), _ptr(x), M, N, K, _ptr(ms), _ptr(ns),
+                                       ms.shape[0], _ptr(y), _ptr(den), nthreads)
+    if rc:
+        raise ValueError("oracle sampled matmul failed")
+    return y, den
+
+
+def max_threads(lib=None) -> int:
+    return (lib or load()).lwq_oracle_max_threads()
+
+
+def normalised_error(y_gpu: np.ndarray, y_ref: np.ndarray, den: np.ndarray) -> float:
+    """max |y - y_ref| / den over all outputs; where den == 0 the output must be exactly 0.
+
+    Returns +inf if any output with den == 0 is nonzero or any value is not finite.
+    """
+    y_gpu = np.asarray(y_gpu, dtype=np.float64)
+    if not np.all(np.isfinite(y_gpu)):
+        return float("inf")
+    zero = den == 0
+    if np.any(y_gpu[zero] != 0):
+        return float("inf")
+    if np.all(zero):
+        return 0.0
+    err = np.abs(y_gpu[~zero] - y_ref[~zero]) / den[~zero]
+    return float(err.max()) if err.size else 0.0

@@ -1,0 +1,319 @@
+"""Checks that pin the CPU oracle to facts outside itself.
+
+Each ``pin_*`` function takes a loaded oracle library handle and raises
+AssertionError when the oracle disagrees with a fact fixed by the block
+layouts, by IEEE-754, by mathematics, or by an independent library routine.
+``test_oracle_pins.py`` runs them against the real oracle (all must pass);
+``test_oracle_mutants.py`` runs them against copies of the oracle with one
+planted mistake each (each copy must fail at least one).
+"""
+
+from __future__ import annotations
+
+import os
+
+import numpy as np
+import torch
+
+import oracle
+from block_quantized_matmul_lwq_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+# ---------------------------------------------------------------- fixtures
+
+def _parse_bytes(spec: str) -> bytes:
+    out = bytearray()
+    for piece in spec.split("."):
+        if "*" in piece:
+            b, n = piece.split("*")
+            out += bytes([int(b, 16)]) * int(n)
+        else:
+            out += bytes.fromhex(piece)
+    return bytes(out)
+
+
+def _parse_values(spec: str) -> list[float]:
+    vals: list[float] = []
+    for tok in spec.split(","):
+        tok = tok.strip()
+        if "*" in tok:
+            v, n = tok.rsplit("*", 1)
+            vals += [float(v)] * int(n)
+        else:
+            vals.append(float(tok))
+    return vals
+
+
+def hand_blocks():
+    """(name, fmt, K, block bytes, expected weights) from tests/golden/hand_blocks.txt."""
+    rows = []
+    with open(os.path.join(GOLDEN, "hand_blocks.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            head, vals = line.split(":")
+            name, fmt, K, spec = head.split()
+            rows.append((name, fmt, int(K), _parse_bytes(spec), _parse_values(vals)))
+    return rows
+
+
+# ------------------------------------------------- independent decoders
+# Written separately from the oracle's C code, vectorised, from the layouts.
+
+def indep_f16(codes: np.ndarray) -> np.ndarray:
+    return np.asarray(codes, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
+def indep_bf16(codes: np.ndarray) -> np.ndarray:
+    t = torch.from_numpy(np.asarray(codes, dtype=np.uint16).view(np.int16).copy())
+    return t.view(torch.bfloat16).to(torch.float64).numpy()
+
+
+def indep_decode(fmt: str, Wq: np.ndarray, K: int) -> np.ndarray:
+    """Decode packed rows with numpy only; returns fp64 exact values [N][K]."""
+    rb = inputs.row_bytes(fmt, K)
+    W = np.asarray(Wq, dtype=np.uint8).reshape(-1, rb)
+    N = W.shape[0]
+    if fmt == "q8_0":
+        b = W.reshape(N, K // 32, 34)
+        d = indep_f16(b[..., 0:2].copy().view(np.uint16)[..., 0])
+        q = b[..., 2:].view(np.int8).astype(np.float64)
+        return (q * d[..., None]).reshape(N, K)
+    if fmt == "q4_0":
+        b = W.reshape(N, K // 32, 18)
+        d = indep_f16(b[..., 0:2].copy().view(np.uint16)[..., 0])
+        nib = b[..., 2:]
+        q = np.concatenate([(nib & 15), (nib >> 4)], axis=-1).astype(np.float64) - 8.0
+        return (q * d[..., None]).reshape(N, K)
+    if fmt == "q4_k":
+        b = W.reshape(N, K // 256, 144)
+        d = indep_f16(b[..., 0:2].copy().view(np.uint16)[..., 0])
+        dmin = indep_f16(b[..., 2:4].copy().view(np.uint16)[..., 0])
+        s = b[..., 4:16].astype(np.int64)
+        sc = np.empty(s.shape[:-1] + (8,), dtype=np.int64)
+        mn = np.empty_like(sc)
+        sc[..., :4] = s[..., 0:4] & 63
+        mn[..., :4] = s[..., 4:8] & 63
+        sc[..., 4:] = (s[..., 8:12] & 15) | ((s[..., 0:4] >> 6) << 4)
+        mn[..., 4:] = (s[..., 8:12] >> 4) | ((s[..., 4:8] >> 6) << 4)
+        qs = b[..., 16:].reshape(N, K // 256, 4, 32).astype(np.int64)
+        q = np.stack([qs & 15, qs >> 4], axis=3).reshape(N, K // 256, 8, 32)  # sub-block j = 2g + half
+        w = d[..., None, None] * sc[..., None] * q - dmin[..., None, None] * mn[..., None]
+        return w.reshape(N, K)
+    raise ValueError(fmt)
+
+
+def pack_q4k_scales(sc: list[int], m: list[int]) -> np.ndarray:
+    """12 bytes holding eight 6-bit scales and mins (inverse of the unpack rule)."""
+    s = np.zeros(12, dtype=np.uint8)
+    for j in range(4):
+        s[j] = (sc[j] & 63) | ((sc[j + 4] >> 4) << 6)
+        s[j + 4] = (m[j] & 63) | ((m[j + 4] >> 4) << 6)
+        s[j + 8] = (sc[j + 4] & 15) | ((m[j + 4] & 15) << 4)
+    return s
+
+
+# ------------------------------------------------------------------ pins
+
+def pin_hand_blocks(lib):
+    """Hand-built blocks decode to their hand-derived values."""
+    for name, fmt, K, raw, expect in hand_blocks():
+        got = oracle.dequant(fmt, np.frombuffer(raw, dtype=np.uint8), K, lib=lib)[0]
+        assert got.shape[0] == len(expect), name
+        np.testing.assert_array_equal(got.astype(np.float64), np.array(expect), err_msg=name)
+
+
+def pin_f16_exhaustive(lib):
+    """All 65,536 fp16 codes decode as numpy's IEEE binary16 does."""
+    codes = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = indep_f16(codes)
+    got = np.array([lib.lwq_oracle_f16(int(c)) for c in codes])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan]))
+
+
+def pin_bf16_exhaustive(lib):
+    """All 65,536 bf16 codes decode as torch.bfloat16 does."""
+    codes = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = indep_bf16(codes)
+    got = np.array([lib.lwq_oracle_bf16(int(c)) for c in codes])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def pin_q4k_scale_roundtrip(lib):
+    """pack(sc, m) -> 12 bytes -> unpack returns (sc, m): all-0, all-63, single bits, random."""
+    cases = [([0] * 8, [0] * 8), ([63] * 8, [63] * 8)]
+    for j in range(8):
+        for bit in range(6):
+            sc = [0] * 8
+            mm = [0] * 8
+            sc[j] = 1 << bit
+            cases.append((sc, [0] * 8))
+            mm[j] = 1 << bit
+            cases.append(([0] * 8, mm))
+    g = np.random.default_rng(1234)
+    for _ in range(2000):
+        cases.append((list(g.integers(0, 64, 8)), list(g.integers(0, 64, 8))))
+    for sc, mm in cases:
+        s = pack_q4k_scales(sc, mm)
+        for j in range(8):
+            assert oracle.q4k_scale_min(s, j, lib=lib) == (sc[j], mm[j]), (sc, mm, j)
+
+
+def pin_roundtrip_q8_0(lib):
+    """Quantize -> oracle decode stays within the Q8_0 rounding bound on 10^5 random blocks."""
+    g = np.random.default_rng(7)
+    w = (g.standard_normal((3125, 1024), dtype=np.float32) * np.float32(0.02)).astype(np.float32)
+    Wq = inputs.quantize_q8_0(w)
+    got = oracle.dequant("q8_0", Wq, 1024, lib=lib).astype(np.float64)
+    wb = w.reshape(-1, 32).astype(np.float64)
+    d32 = np.abs(w.reshape(-1, 32)).max(axis=1).astype(np.float32) / np.float32(127)
+    d16 = d32.astype(np.float16).astype(np.float64)
+    d32 = d32.astype(np.float64)
+    # |w - q d| <= |w - q d32| + |q| |d32 - d| <= d32/2 + 127 |d32 - d|  (+ fp32 slop)
+    bound = d32 / 2 + 127 * np.abs(d32 - d16) + 4 * np.spacing(np.abs(wb).max(axis=1).astype(np.float32))
+    err = np.abs(got.reshape(-1, 32) - wb).max(axis=1)
+    assert np.all(err <= bound), float((err - bound).max())
+
+
+def pin_roundtrip_q4_0(lib):
+    """Quantize -> oracle decode stays within the Q4_0 rounding bound on 10^5 random blocks."""
+    g = np.random.default_rng(8)
+    w = (g.standard_normal((3125, 1024), dtype=np.float32) * np.float32(0.02)).astype(np.float32)
+    Wq = inputs.quantize_q4_0(w)
+    got = oracle.dequant("q4_0", Wq, 1024, lib=lib).astype(np.float64).reshape(-1, 32)
+    wb = w.reshape(-1, 32).astype(np.float64)
+    idx = np.abs(wb).argmax(axis=1)
+    amax = wb[np.arange(wb.shape[0]), idx]
+    d32 = (amax.astype(np.float32) / np.float32(-8)).astype(np.float64)
+    d16 = d32.astype(np.float16).astype(np.float64)
+    slop = 4 * np.spacing(np.abs(wb).max(axis=1).astype(np.float32))
+    # codes within [0, 15]: |w - (q-8)d| <= |d32|/2 + 8|d32 - d|; the clamped code 16 -> 15 adds |d32|/2
+    bound = np.abs(d32) + 8 * np.abs(d32 - d16) + slop
+    err = np.abs(got - wb).max(axis=1)
+    assert np.all(err <= bound), float((err - bound).max())
+    # the element equal to amax decodes to -8 d exactly
+    got_amax = got[np.arange(wb.shape[0]), idx]
+    np.testing.assert_array_equal(got_amax, (-8.0 * d16).astype(np.float32).astype(np.float64))
+
+
+def pin_bruteforce_one_block(lib):
+    """K = one block, N, M <= 3: oracle y equals Python-loop sums over an independent decode."""
+    g = np.random.default_rng(99)
+    for fmt, K in (("q8_0", 32), ("q4_0", 32), ("q4_k", 256)):
+        for act in ("f32", "f16", "bf16"):
+            for M, N in ((1, 1), (2, 3), (3, 2)):
+                Wq = inputs.make_weights(fmt, g, N, K)
+                x = inputs.activations(g, M, K, act)
+                y, den = oracle.matmul(fmt, Wq, x, K=K, act=act, lib=lib)
+                W = indep_decode(fmt, Wq, K)
+                W32 = W.astype(np.float32).astype(np.float64)  # the oracle rounds w once to fp32
+                xd = {"f32": lambda a: a.astype(np.float64), "f16": lambda a: a.astype(np.float64),
+                      "bf16": indep_bf16}[act](x)
+                for m in range(M):
+                    for n in range(N):
+                        acc = 0.0
+                        acc_abs = 0.0
+                        for k in range(K):
+                            p = float(xd[m, k]) * float(W32[n, k])
+                            acc += p
+                            acc_abs += abs(p)
+                        assert y[m, n] == acc, (fmt, act, m, n, y[m, n], acc)
+                        assert den[m, n] == acc_abs, (fmt, act, m, n)
+
+
+def pin_library_matmul(lib):
+    """Oracle y equals torch.matmul (fp64) of the independently decoded W, to 1e-12 relative to den."""
+    g = np.random.default_rng(5)
+    for fmt, K in (("q8_0", 512), ("q4_0", 512), ("q4_k", 512)):
+        for act in ("f32", "f16", "bf16"):
+            M, N = 5, 37
+            Wq = inputs.make_weights(fmt, g, N, K)
+            x = inputs.activations(g, M, K, act)
+            y, den = oracle.matmul(fmt, Wq, x, act=act, lib=lib)
+            W = torch.from_numpy(indep_decode(fmt, Wq, K).astype(np.float32).astype(np.float64))
+            xd = torch.from_numpy(indep_bf16(x) if act == "bf16" else x.astype(np.float64))
+            ref = (xd @ W.T).numpy()
+            ref_den = (xd.abs() @ W.abs().T).numpy()
+            assert np.all(np.abs(y - ref) <= 1e-12 * ref_den), fmt
+            assert np.all(np.abs(den - ref_den) <= 1e-12 * ref_den), fmt
+
+
+def pin_linearity(lib):
+    """y(a x1 + b x2) == a y(x1) + b y(x2) exactly when every sum is exact (dyadic grid)."""
+    g = np.random.default_rng(11)
+    K, N = 256, 9
+    # blocks with power-of-two d and small-integer x: every partial sum is exact in fp64
+    for fmt in ("q8_0", "q4_0", "q4_k"):
+        Wq = inputs.make_weights(fmt, g, N, K).reshape(N, -1).copy()
+        bb, bw = inputs.BLOCK_BYTES[fmt], inputs.BLOCK_WEIGHTS[fmt]
+        blk = Wq.reshape(N, K // bw, bb)
+        e = g.integers(-8, -2, size=blk.shape[:2])
+        dcode = (np.exp2(e).astype(np.float16)).view(np.uint16)
+        blk[..., 0:2] = dcode.view(np.uint8).reshape(blk.shape[:2] + (2,))
+        if fmt == "q4_k":
+            blk[..., 2:4] = (np.exp2(e - 1).astype(np.float16)).view(np.uint16).view(np.uint8).reshape(blk.shape[:2] + (2,))
+        Wq = blk.reshape(N, -1)
+        x1 = g.integers(-8, 9, size=(3, K)).astype(np.float32)
+        x2 = g.integers(-8, 9, size=(3, K)).astype(np.float32)
+        a, b = np.float32(2.0), np.float32(-0.5)
+        y1, _ = oracle.matmul(fmt, Wq, x1, lib=lib)
+        y2, _ = oracle.matmul(fmt, Wq, x2, lib=lib)
+        y12, _ = oracle.matmul(fmt, Wq, (a * x1 + b * x2).astype(np.float32), lib=lib)
+        np.testing.assert_array_equal(y12, 2.0 * y1 - 0.5 * y2, err_msg=fmt)
+        # a unit vector picks out one decoded weight: y(e_k)[n] == w_hat[n][k]
+        W = oracle.dequant(fmt, Wq, K, lib=lib)
+        ks = [0, 1, 15, 16, 17, 31, 32, 100, 255]
+        eye = np.zeros((len(ks), K), dtype=np.float32)
+        eye[np.arange(len(ks)), ks] = 1.0
+        ye, _ = oracle.matmul(fmt, Wq, eye, lib=lib)
+        np.testing.assert_array_equal(ye, W[:, ks].T.astype(np.float64), err_msg=fmt)
+
+
+def pin_zero_denominator(lib):
+    """All-eight Q4_0 rows and zero activations give y == 0 and den == 0 exactly."""
+    K, N = 128, 4
+    blk = np.zeros((N, K // 32, 18), dtype=np.uint8)
+    blk[..., 0:2] = np.frombuffer(bytes.fromhex("003c"), dtype=np.uint8)
+    blk[..., 2:] = 0x88
+    x = np.random.default_rng(3).standard_normal((2, K)).astype(np.float32)
+    y, den = oracle.matmul("q4_0", blk.reshape(N, -1), x, lib=lib)
+    assert np.all(y == 0) and np.all(den == 0)
+    Wq = inputs.make_weights("q4_k", np.random.default_rng(4), N, 256)
+    y, den = oracle.matmul("q4_k", Wq, np.zeros((2, 256), dtype=np.float16), lib=lib)
+    assert np.all(y == 0) and np.all(den == 0)
+
+
+def pin_sampled_equals_full(lib):
+    """The sampled entry point returns bit-identical values to the full product."""
+    g = np.random.default_rng(21)
+    for fmt, K in (("q8_0", 256), ("q4_0", 288), ("q4_k", 512)):
+        M, N = 3, 23
+        Wq = inputs.make_weights(fmt, g, N, K)
+        x = inputs.activations(g, M, K, "f16")
+        y, den = oracle.matmul(fmt, Wq, x, lib=lib)
+        ms = g.integers(0, M, 40)
+        ns = g.integers(0, N, 40)
+        ys, dens = oracle.matmul_sampled(fmt, Wq, x, ms, ns, lib=lib)
+        np.testing.assert_array_equal(ys, y[ms, ns])
+        np.testing.assert_array_equal(dens, den[ms, ns])
+
+
+def pin_row_bytes(lib):
+    for fmt, K, rb in (("q8_0", 4096, 4352), ("q4_0", 4096, 2304), ("q4_k", 4096, 2304),
+                       ("q4_0", 11008, 6192), ("q4_k", 11008, 6192), ("q8_0", 14336, 15232)):
+        assert lib.lwq_oracle_row_bytes(oracle.FMT[fmt], K) == rb
+    assert lib.lwq_oracle_row_bytes(oracle.FMT["q4_k"], 128) == -1
+    assert lib.lwq_oracle_row_bytes(oracle.FMT["q4_0"], 48) == -1
+
+
+ALL_PINS = [pin_hand_blocks, pin_f16_exhaustive, pin_bf16_exhaustive, pin_q4k_scale_roundtrip,
+            pin_roundtrip_q8_0, pin_roundtrip_q4_0, pin_bruteforce_one_block, pin_library_matmul,
+            pin_linearity, pin_zero_denominator, pin_sampled_equals_full, pin_row_bytes]
