@@ -1,0 +1,546 @@
+"""Benchmark of the block-quantized matmul on B200.
+
+One step = one pass of the decode hot path over one batch of synthetic input:
+the Q4_0 GEMV y = x . dequant(Wq)^T with N=11008, K=4096 and fp32
+activations, at M = 1, 4 and 8 (three calls).  `value` is the whole-job
+throughput in GB/s of packed weights + activations + outputs, timed on the
+device with CUDA events, inputs resident in HBM, each call reading a
+different copy of the weights from a rotation larger than 4x L2.  The other
+workloads (Q8_0 4096x4096, the Q4_K 7B decode layer and the Q4_0 prefill
+GEMMs) are measured in the same run and reported under "workloads".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lwq|reference]
+
+Under torchrun every rank runs the same workload on its own GPU (the path
+has no exchange step: replicas, weak scaling) and rank 0 prints one JSON line
+with the max-over-ranks time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from block_quantized_matmul_lwq_b200 import inputs  # noqa: E402
+
+METRIC = "quantized matmul: decode GEMV weight GB/s (% of HBM); prefill GEMM TFLOP/s"
+HEADLINE = "q4_0_gemv_11008x4096"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ helpers
+
+def load_peaks() -> tuple[dict, str]:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def step_calls(workload: str):
+    """[(fmt, act, M, N, K, seed)] of one step of a workload."""
+    spec = inputs.WORKLOADS[workload]
+    calls = []
+    if workload == "q4_k_7b_layer_decode":
+        for (N, K), seed in zip(spec["shapes"], spec["seeds"]):
+            calls.append((spec["fmt"], spec["act"], 1, N, K, seed))
+    elif workload == "q4_0_prefill_gemm":
+        for M, (N, K), seed in zip(spec["Ms"], spec["shapes"], spec["seeds"]):
+            calls.append((spec["fmt"], spec["act"], M, N, K, seed))
+    else:
+        (N, K), = spec["shapes"]
+        for M in spec["Ms"]:
+            calls.append((spec["fmt"], spec["act"], M, N, K, spec["seeds"][0]))
+    return calls
+
+
+def call_bytes(fmt, act, M, N, K) -> int:
+    xe = 4 if act == "f32" else 2
+    return N * inputs.row_bytes(fmt, K) + M * K * xe + M * N * 4
+
+
+def call_flops(M, N, K) -> int:
+    return 2 * M * N * K
+
+
+def reduce_max(value: float, dist_on: bool, device=None) -> float:
+    """Max of a float over all ranks (identity without torch.distributed)."""
+    if not dist_on:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(value: float, dist_on: bool, device=None) -> float:
+    if not dist_on:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while active."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="lwq_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) == len(self.FIELDS):
+                        rows.append(parts)
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(r[0]) for r in rows if num(r[0]) is not None]
+        smax = [num(r[1]) for r in rows if num(r[1]) is not None]
+        power = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+class Problem:
+    """Device-resident inputs of one workload: rotating weight copies, x, y per call."""
+
+    def __init__(self, workload: str, dev, rotate_min_bytes: int):
+        import torch
+        self.calls = step_calls(workload)
+        self.host = []
+        self.dev_calls = []
+        cache = {}
+        for fmt, act, M, N, K, seed in self.calls:
+            key = (fmt, N, K, seed)
+            if key not in cache:
+                g = inputs.rng(seed)
+                cache[key] = (inputs.make_weights(fmt, g, N, K), g)
+            Wq, _ = cache[key]
+            x = inputs.activations(inputs.rng(seed + 1000003), M, K, act)
+            self.host.append((Wq, x))
+        self.step_weight_bytes = sum(N * inputs.row_bytes(f, K) for f, a, M, N, K, s in self.calls)
+        # every call of a step reads its own weight copy; R steps cycle through
+        # all copies, so a copy is re-read only after >= rotate_min_bytes of other weights
+        self.R = max(3, -(-rotate_min_bytes // max(1, self.step_weight_bytes)))
+        uses = {}
+        self.use_index = []
+        for fmt, act, M, N, K, seed in self.calls:
+            key = (fmt, N, K, seed)
+            self.use_index.append(uses.get(key, 0))
+            uses[key] = uses.get(key, 0) + 1
+        self.uses = uses
+        self.weights = {}
+        for (fmt, act, M, N, K, seed), (Wq, x) in zip(self.calls, self.host):
+            key = (fmt, N, K, seed)
+            if key not in self.weights:
+                base = torch.from_numpy(Wq).to(dev)
+                self.weights[key] = [base] + [base.clone() for _ in range(self.R * uses[key] - 1)]
+            xd = torch.from_numpy(x.view(np.int16) if x.dtype == np.uint16 else x).to(dev)
+            yd = torch.empty((M, N), dtype=torch.float32, device=dev)
+            self.dev_calls.append((fmt, act, M, N, K, seed, xd, yd))
+        self.copies_bytes = sum(len(v) * v[0].numel() for v in self.weights.values())
+        self.bytes_per_step = sum(call_bytes(f, a, M, N, K) for f, a, M, N, K, s in self.calls)
+        self.flops_per_step = sum(call_flops(M, N, K) for f, a, M, N, K, s in self.calls)
+
+    def enqueue_call(self, lwq, i: int, r: int, stream) -> int:
+        """Enqueue call i of the step on `stream`, reading weight copy r; returns launches enqueued."""
+        fmt, act, M, N, K, seed, xd, yd = self.dev_calls[i]
+        key = (fmt, N, K, seed)
+        W = self.weights[key][(r * self.uses[key] + self.use_index[i]) % len(self.weights[key])]
+        lwq.lwq_matmul(lwq.fmt_code(fmt, act), W, xd, yd, M, N, K, stream=stream)
+        return lwq.lwq_last_launch_count()
+
+    def enqueue_step(self, lwq, r: int, stream) -> int:
+        """Enqueue one step on `stream`, reading weight copy r; returns launches enqueued."""
+        return sum(self.enqueue_call(lwq, i, r, stream) for i in range(len(self.dev_calls)))
+
+
+def time_workload(lwq, workload: str, dev, steps: int, warmup: int, dist_on: bool, per_call: bool = True):
+    """Device time of `steps` steps (graph-replayed, rotating weights), max over ranks."""
+    import torch
+    import torch.distributed as dist
+    prob = Problem(workload, dev, rotate_min_bytes=4 * L2_BYTES)
+    stream = torch.cuda.Stream(device=dev)
+    graphs = []
+    launches_per_step = 0
+    with torch.cuda.stream(stream):
+        for r in range(prob.R):   # eager warm-up of every copy, then one graph per copy
+            prob.enqueue_step(lwq, r, stream)
+        stream.synchronize()
+        for r in range(prob.R):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                launches_per_step = prob.enqueue_step(lwq, r, stream)
+            graphs.append(g)
+    stream.synchronize()
+    for i in range(warmup):
+        with torch.cuda.stream(stream):
+            graphs[i % prob.R].replay()
+    stream.synchronize()
+    if dist_on:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for i in range(steps):
+            graphs[i % prob.R].replay()
+        end.record(stream)
+    stream.synchronize()
+    torch.cuda.synchronize(dev)
+    if dist_on:
+        dist.barrier()
+    ms = start.elapsed_time(end)
+    ms_max = reduce_max(ms, dist_on, dev)
+
+    # per-call device durations: one graph per call running it on every weight copy
+    per = None
+    if per_call:
+        per = []
+        for i, c in enumerate(prob.calls):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                with torch.cuda.graph(g, stream=stream):
+                    for r in range(prob.R):
+                        prob.enqueue_call(lwq, i, r, stream)
+                g.replay()
+            stream.synchronize()
+            reps = max(2, min(50, steps // (4 * prob.R) or 2))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for _ in range(reps):
+                    g.replay()
+                e1.record(stream)
+            stream.synchronize()
+            per.append({"call": c, "ms_mean": e0.elapsed_time(e1) / (reps * prob.R)})
+            del g
+    return prob, ms, ms_max, launches_per_step, per
+
+
+def e2e_workload(lwq, workload: str, dev, steps: int, dist_on: bool):
+    """End to end through the public API: pinned host inputs -> device -> lwq_matmul -> host result."""
+    import torch
+    import torch.distributed as dist
+    calls = step_calls(workload)
+    host = []
+    for fmt, act, M, N, K, seed in calls:
+        g = inputs.rng(seed)
+        Wq = inputs.make_weights(fmt, g, N, K)
+        x = inputs.activations(inputs.rng(seed + 1000003), M, K, act)
+        Wp = torch.from_numpy(Wq).pin_memory()
+        xp = torch.from_numpy(x.view(np.int16) if x.dtype == np.uint16 else x).pin_memory()
+        yp = torch.empty((M, N), dtype=torch.float32).pin_memory()
+        Wd = torch.empty_like(Wp, device=dev)
+        xd = torch.empty_like(xp, device=dev)
+        yd = torch.empty((M, N), dtype=torch.float32, device=dev)
+        host.append((fmt, act, M, N, K, Wp, xp, yp, Wd, xd, yd))
+    stream = torch.cuda.Stream(device=dev)
+    h2d = sum(h[5].numel() * h[5].element_size() + h[6].numel() * h[6].element_size() for h in host)
+    d2h = sum(h[7].numel() * 4 for h in host)
+
+    def one_step():
+        for fmt, act, M, N, K, Wp, xp, yp, Wd, xd, yd in host:
+            Wd.copy_(Wp, non_blocking=True)
+            xd.copy_(xp, non_blocking=True)
+            lwq.lwq_matmul(lwq.fmt_code(fmt, act), Wd, xd, yd, M, N, K, stream=stream)
+            yp.copy_(yd, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            one_step()
+    stream.synchronize()
+    if dist_on:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(steps):
+            one_step()
+        end.record(stream)
+    stream.synchronize()
+    if dist_on:
+        dist.barrier()
+    ms = reduce_max(start.elapsed_time(end), dist_on, dev)
+    nbytes = sum(call_bytes(c[0], c[1], c[2], c[3], c[4]) for c in calls)
+    return ms, nbytes, h2d, d2h
+
+
+def cpu_baseline(workload: str, budget_s: float = 15.0) -> dict:
+    """The oracle as it stands, on the host cores, over a bounded row sample of one step."""
+    import oracle
+    calls = step_calls(workload)
+    threads = oracle.max_threads()
+    # calibrate on a small row sample, then size the sample to the budget
+    rows = 64
+    t_rows = None
+    total_bytes = 0.0
+    total_s = 0.0
+    for attempt in range(2):
+        total_bytes = 0.0
+        total_s = 0.0
+        for fmt, act, M, N, K, seed in calls:
+            g = inputs.rng(seed)
+            n = min(rows, N)
+            Wq = inputs.make_weights(fmt, g, n, K)
+            x = inputs.activations(inputs.rng(seed + 1000003), M, K, act)
+            t0 = time.perf_counter()
+            oracle.matmul(fmt, Wq, x, act=act)
+            total_s += time.perf_counter() - t0
+            total_bytes += call_bytes(fmt, act, M, n, K)
+        if attempt == 0:
+            t_rows = total_s / rows
+            rows = max(16, int(budget_s / max(t_rows, 1e-9) / 2))
+            rows = min(rows, max(c[3] for c in calls))
+    return {"value": total_bytes / total_s / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"first {rows} weight rows of every call of one step (fp64 C oracle, OpenMP)",
+            "seconds": total_s}
+
+
+def run_gpu_arm(args):
+    import torch
+    import torch.distributed as dist
+    import block_quantized_matmul_lwq_b200 as lwq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist_on = world > 1
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if dist_on:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    peaks, peak_src = load_peaks()
+    ws_bytes = 0
+    for wl in [HEADLINE] + args.extra:
+        for fmt, act, M, N, K, seed in step_calls(wl):
+            ws_bytes = max(ws_bytes, lwq.lwq_workspace_size(lwq.fmt_code(fmt, act), M, N, K))
+    ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    lwq.lwq_init(ws, ws.numel())
+
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else local
+    sampler = ClockSampler(gpu_index)
+    with sampler:
+        prob, ms_local, ms, lps, per = time_workload(lwq, HEADLINE, dev, args.steps, args.warmup, dist_on)
+    clocks = sampler.summary()
+
+    bytes_all = reduce_sum(float(prob.bytes_per_step * args.steps), dist_on, dev)
+    value = bytes_all / (ms / 1e3) / 1e9
+    # roofline: every launch in the timed region is the headline kernel (tensor-core GEMV,
+    # Q4_0 x fp32); achieved = algorithmic bytes per step / device time per step on this rank
+    achieved = prob.bytes_per_step / (ms_local / args.steps / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": args.traffic,
+                "peak_source": peak_src, "kernel": "lwq::gemv_tc_kernel<Q4_0, fp32 x, NT=1>",
+                "per_call_ms": [{"M": p["call"][2], "ms": round(p["ms_mean"], 5),
+                                 "GB/s": round(call_bytes(*p["call"][:5]) / p["ms_mean"] / 1e6, 1)} for p in per]}
+
+    e2e_ms, e2e_bytes, h2d, d2h = e2e_workload(lwq, HEADLINE, dev, args.e2e_steps, dist_on)
+    e2e_all = reduce_sum(float(e2e_bytes * args.e2e_steps), dist_on, dev)
+    e2e = {"value": round(e2e_all / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+
+    extra = {}
+    for wl in args.extra:
+        p2, _, ms2, lps2, per2 = time_workload(lwq, wl, dev, args.extra_steps, 3, dist_on)
+        rec = {"steps": args.extra_steps, "ms_per_step": round(ms2 / args.extra_steps, 5),
+               "launches_per_step": lps2}
+        if wl == "q4_0_prefill_gemm":
+            tflops = p2.flops_per_step * args.extra_steps / (ms2 / 1e3) / 1e12
+            rec.update({"value": round(tflops, 2), "unit": "TFLOP/s",
+                        "frac_of_bf16_peak": round(tflops / peaks["bf16_tflops"], 4),
+                        "per_call": [{"M": p["call"][2], "N": p["call"][3], "K": p["call"][4],
+                                      "ms": round(p["ms_mean"], 4),
+                                      "TFLOP/s": round(call_flops(*p["call"][2:5]) / p["ms_mean"] / 1e9, 1)}
+                                     for p in per2]})
+        else:
+            gbs = p2.bytes_per_step * args.extra_steps / (ms2 / 1e3) / 1e9
+            rec.update({"value": round(gbs, 1), "unit": "GB/s", "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                        "per_call": [{"M": p["call"][2], "N": p["call"][3], "K": p["call"][4],
+                                      "ms": round(p["ms_mean"], 5),
+                                      "GB/s": round(call_bytes(*p["call"][:5]) / p["ms_mean"] / 1e6, 1)}
+                                     for p in per2]})
+        extra[wl] = rec
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(HEADLINE, budget_s=args.cpu_budget)
+
+    torch.cuda.synchronize(dev)
+    err = lwq.lwq_get_device_error()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": HEADLINE, "weights": "q4_0", "activations": "f32 (split into bf16 hi+lo)",
+                       "accumulate": "f32", "M": [1, 4, 8], "N": 11008, "K": 4096, "seed": 0,
+                       "l2": f"inputs larger than L2: every call reads its own weight copy, "
+                             f"{prob.copies_bytes / 1e6:.0f} MB of copies in rotation",
+                       "parallelism": f"replicas x{world}", "timing": "CUDA graphs of one step, CUDA events"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": lps * args.steps, "clocks": clocks, "workloads": extra,
+            "device_error": err,
+        }
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        dist.barrier()
+        dist.destroy_process_group()
+    lwq.lwq_shutdown()
+
+
+def run_reference_arm(args):
+    """The oracle (the deliberately slow CPU definition) on the host cores, rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    calls = step_calls(HEADLINE)
+    threads = oracle.max_threads()
+    # size each step's row sample so that warmup + steps fit the budget
+    budget = args.reference_budget
+    probe_rows = 32
+    t0 = time.perf_counter()
+    data = []
+    for fmt, act, M, N, K, seed in calls:
+        g = inputs.rng(seed)
+        Wq = inputs.make_weights(fmt, g, probe_rows, K)
+        x = inputs.activations(inputs.rng(seed + 1000003), M, K, act)
+        data.append((fmt, act, M, K, Wq, x))
+    t_probe = time.perf_counter()
+    for fmt, act, M, K, Wq, x in data:
+        oracle.matmul(fmt, Wq, x, act=act)
+    per_row = (time.perf_counter() - t_probe) / probe_rows
+    rows = int(budget / max(1, args.steps + args.warmup) / max(per_row, 1e-9))
+    rows = max(1, min(rows, 11008))
+    data = []
+    for fmt, act, M, N, K, seed in calls:
+        g = inputs.rng(seed)
+        Wq = inputs.make_weights(fmt, g, rows, K)
+        x = inputs.activations(inputs.rng(seed + 1000003), M, K, act)
+        data.append((fmt, act, M, K, Wq, x))
+    for _ in range(args.warmup):
+        for fmt, act, M, K, Wq, x in data:
+            oracle.matmul(fmt, Wq, x, act=act)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        for fmt, act, M, K, Wq, x in data:
+            oracle.matmul(fmt, Wq, x, act=act)
+    dt = time.perf_counter() - t0
+    step_bytes = sum(call_bytes(fmt, act, M, rows, K) for fmt, act, M, K, Wq, x in data)
+    value = step_bytes * args.steps / dt / 1e9
+    sample = f"first {rows} of 11008 weight rows of every call of a step (M=1,4,8; K=4096)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus":
+            int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": HEADLINE, "weights": "q4_0", "activations": "f32", "M": [1, 4, 8], "N": 11008,
+                   "K": 4096, "seed": 0},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=60)
+    ap.add_argument("--impl", choices=["lwq", "reference"], default="lwq")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--extra-steps", type=int, default=400)
+    ap.add_argument("--extra", nargs="*", default=["q8_0_gemv_4096x4096", "q4_k_7b_layer_decode",
+                                                   "q4_0_prefill_gemm"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--reference-budget", type=float, default=60.0)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu dram bytes per launch of the roofline kernel, when measured for this build")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    return args
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference_arm(args)
+    else:
+        run_gpu_arm(args)
+
+
+if __name__ == "__main__":
+    main()

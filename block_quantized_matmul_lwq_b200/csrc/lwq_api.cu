@@ -1,0 +1,555 @@
+// C ABI of the block-quantized matmul library (see include/lwq.h).
+//
+// Host side of the path: argument checks, the per-device workspace registry
+// (one caller-owned arena per device, registered once), TMA descriptor
+// encoding, the per-shape configuration table and the kernel launches.
+// Nothing here allocates device memory or synchronizes the host inside
+// lwq_matmul.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/lwq.h"
+#include "lwq_gemm.cuh"
+#include "lwq_gemv.cuh"
+#include "lwq_gemv_simple.cuh"
+
+namespace lwq {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr size_t kSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory per block on sm_100
+constexpr unsigned long long kTimeoutNs = 2000000000ull;  // bounded waits give up after 2 s
+
+struct DeviceState {
+    void *ws = nullptr;
+    size_t ws_bytes = 0;
+    bool registered = false;
+    int sms = 0;
+};
+
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mu;
+thread_local int t_last_launches = 0;
+
+// ------------------------------------------------------- driver entry point
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+int current_device(int *dev) {
+    if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= kMaxDevices) return LWQ_ERR_CUDA;
+    return LWQ_OK;
+}
+
+int sm_count(int dev) {
+    if (g_dev[dev].sms == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+        g_dev[dev].sms = v;
+    }
+    return g_dev[dev].sms;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int block_weights(int wf) { return wf == LWQ_Q4_K ? 256 : (wf == LWQ_Q8_0 || wf == LWQ_Q4_0 ? 32 : 0); }
+int block_bytes(int wf) { return wf == LWQ_Q4_K ? 144 : (wf == LWQ_Q8_0 ? 34 : (wf == LWQ_Q4_0 ? 18 : 0)); }
+int act_code(int fmt) {
+    switch (fmt & LWQ_ACT_MASK) {
+    case LWQ_ACT_F32: return X_F32;
+    case LWQ_ACT_F16: return X_F16;
+    case LWQ_ACT_BF16: return X_BF16;
+    default: return -1;
+    }
+}
+
+int check_fmt_k(int fmt, long K) {
+    const int wf = fmt & LWQ_FMT_MASK;
+    if (fmt & ~(LWQ_FMT_MASK | LWQ_ACT_MASK)) return LWQ_ERR_UNSUPPORTED;
+    if (block_weights(wf) == 0 || act_code(fmt) < 0) return LWQ_ERR_UNSUPPORTED;
+    if (K <= 0 || K % block_weights(wf)) return LWQ_ERR_INVALID_ARG;
+    return LWQ_OK;
+}
+
+// ---------------------------------------------------------- configuration
+struct Plan {
+    lwq_config cfg;
+    int nt;          // GEMV n8 tiles (1: <= 8 activation rows per pass, 2: <= 16)
+    int m_group;     // activation rows per pass
+    size_t smem;
+    size_t ws_need;  // workspace bytes for one pass
+};
+
+size_t gemv_smem(int wf, int nw, int stages, int nt) {
+    const int cb = (wf == LWQ_Q8_0) ? 272 : 144;
+    return (size_t)stages * nw * GEMV_ROWS * cb + (size_t)stages * nw * GEMV_ROWS * 8 * nt * 4 +
+           (size_t)3 * stages * 8;
+}
+
+bool tc_gemv_eligible(int wf, int xt, long K) {
+    if (K % 256) return false;
+    if (wf == LWQ_Q4_K) return xt == X_F16;
+    return true;
+}
+
+// Workspace layout: [kCounterBytes of per-row-tile arrival counters][fp32
+// split-K partials].  The counter region has a fixed size so that no call's
+// partials ever overlap another call's counters (counters return to zero at
+// the end of every call).
+constexpr size_t kCounterBytes = 64 * 1024;
+constexpr int kMaxSplitTiles = (int)(kCounterBytes / 4);
+
+size_t splitk_ws(int S, int m, int N) {
+    if (S <= 1) return 0;
+    return kCounterBytes + (size_t)S * m * N * 4;
+}
+
+int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Plan *p) {
+    const int wf = fmt & LWQ_FMT_MASK, xt = act_code(fmt);
+    memset(p, 0, sizeof(*p));
+    int path = force && force->path ? force->path : 0;
+    if (!path) {
+        if (M > 16 && xt != X_F32 && gemm_eligible(wf, xt, K))
+            path = 2;
+        else if (tc_gemv_eligible(wf, xt, K))
+            path = 1;
+        else
+            path = 3;
+    }
+    p->cfg.path = path;
+    if (path == 2) {
+        if (!gemm_eligible(wf, xt, K)) return LWQ_ERR_UNSUPPORTED;
+        GemmPlan gp;
+        int rc = gemm_plan(wf, xt, M, N, K, force, sms, &gp);
+        if (rc) return rc;
+        p->cfg.warps = gp.warps;
+        p->cfg.stages = gp.stages;
+        p->cfg.splits = 1;
+        p->cfg.ctas = gp.ctas;
+        p->cfg.tile_n = gp.tile_n;
+        p->cfg.tile_m = gp.tile_m;
+        p->smem = gp.smem;
+        p->m_group = M;
+        p->ws_need = 0;
+        return LWQ_OK;
+    }
+    if (path == 3) {
+        p->m_group = M < 16 ? M : 16;
+        p->cfg.warps = 8;
+        p->cfg.ctas = (N + 7) / 8;
+        p->cfg.splits = 1;
+        return LWQ_OK;
+    }
+    if (path != 1 || !tc_gemv_eligible(wf, xt, K)) return LWQ_ERR_UNSUPPORTED;
+    const int mmax = (xt == X_F32) ? 8 : 16;
+    p->m_group = M < mmax ? M : mmax;
+    p->nt = p->m_group <= 8 ? 1 : 2;
+    const int nchunks = K / 256;
+    const int nw_max = p->nt == 1 ? 16 : 14;   // register budget (see gemv_tc_kernel)
+    int nw = force && force->warps ? force->warps : (wf == LWQ_Q8_0 ? 8 : nw_max);
+    if (nw > nw_max || nw < 1) return LWQ_ERR_UNSUPPORTED;
+    if (nw > nchunks) nw = nchunks;
+    int S = force && force->splits ? force->splits : (nchunks + nw - 1) / nw;
+    if (S < 1) return LWQ_ERR_UNSUPPORTED;
+    const int cps = (nchunks + S - 1) / S;
+    if (cps > nw) return LWQ_ERR_UNSUPPORTED;  // every chunk of a split needs a warp
+    S = (nchunks + cps - 1) / cps;               // drop empty splits
+    int stages = force && force->stages ? force->stages : 4;
+    while (stages > 2 && gemv_smem(wf, nw, stages, p->nt) > kSmemLimit) --stages;
+    if (stages < 2 || gemv_smem(wf, nw, stages, p->nt) > kSmemLimit) return LWQ_ERR_UNSUPPORTED;
+    const int row_tiles = (N + GEMV_ROWS - 1) / GEMV_ROWS;
+    if (S > 1 && row_tiles > kMaxSplitTiles) return LWQ_ERR_UNSUPPORTED;
+    int groups = force && force->ctas ? force->ctas / S : sms / S;
+    if (groups < 1) groups = 1;
+    if (groups > row_tiles) groups = row_tiles;
+    p->cfg.warps = nw;
+    p->cfg.stages = stages;
+    p->cfg.splits = S;
+    p->cfg.ctas = S * groups;
+    p->smem = gemv_smem(wf, nw, stages, p->nt);
+    p->ws_need = splitk_ws(S, p->m_group, N);
+    return LWQ_OK;
+}
+
+// --------------------------------------------------------------- launches
+// Raise a kernel's dynamic shared-memory limit once per (device, kernel), so
+// that launches captured into CUDA graphs make no attribute calls.
+cudaError_t ensure_smem(const void *kern, size_t smem) {
+    struct Entry {
+        int dev;
+        const void *kern;
+        size_t smem;
+    };
+    static Entry cache[256];
+    static int n = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_mu);
+    for (int i = 0; i < n; ++i)
+        if (cache[i].dev == dev && cache[i].kern == kern && cache[i].smem >= smem) return cudaSuccess;
+    const size_t want = kSmemLimit;  // set the maximum once; any smaller launch fits
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)want);
+    if (e != cudaSuccess) return e;
+    if (n < 256) cache[n++] = Entry{dev, kern, want};
+    return cudaSuccess;
+}
+
+template <int FMT, int XT, int NT>
+cudaError_t launch_gemv_tc(const CUtensorMap &map, const GemvArgs &a, int ctas, int nw, size_t smem,
+                           cudaStream_t st) {
+    auto kern = gemv_tc_kernel<FMT, XT, NT>;
+    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), smem);
+    if (e != cudaSuccess) return e;
+    kern<<<ctas, (nw + 2) * 32, smem, st>>>(map, a);
+    return cudaGetLastError();
+}
+
+template <int FMT, int XT>
+cudaError_t launch_gemv_tc_nt(int nt, const CUtensorMap &map, const GemvArgs &a, int ctas, int nw, size_t smem,
+                              cudaStream_t st) {
+    if (nt == 1) return launch_gemv_tc<FMT, XT, 1>(map, a, ctas, nw, smem, st);
+    if constexpr (XT != X_F32) return launch_gemv_tc<FMT, XT, 2>(map, a, ctas, nw, smem, st);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t dispatch_gemv_tc(int wf, int xt, int nt, const CUtensorMap &map, const GemvArgs &a, int ctas, int nw,
+                             size_t smem, cudaStream_t st) {
+    switch (wf) {
+    case LWQ_Q4_0:
+        if (xt == X_F32) return launch_gemv_tc_nt<F_Q4_0, X_F32>(nt, map, a, ctas, nw, smem, st);
+        if (xt == X_F16) return launch_gemv_tc_nt<F_Q4_0, X_F16>(nt, map, a, ctas, nw, smem, st);
+        return launch_gemv_tc_nt<F_Q4_0, X_BF16>(nt, map, a, ctas, nw, smem, st);
+    case LWQ_Q8_0:
+        if (xt == X_F32) return launch_gemv_tc_nt<F_Q8_0, X_F32>(nt, map, a, ctas, nw, smem, st);
+        if (xt == X_F16) return launch_gemv_tc_nt<F_Q8_0, X_F16>(nt, map, a, ctas, nw, smem, st);
+        return launch_gemv_tc_nt<F_Q8_0, X_BF16>(nt, map, a, ctas, nw, smem, st);
+    case LWQ_Q4_K:
+        if (xt == X_F16) return launch_gemv_tc_nt<F_Q4_K, X_F16>(nt, map, a, ctas, nw, smem, st);
+        return cudaErrorInvalidValue;
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <int FMT, int XT>
+cudaError_t launch_simple(const uint8_t *W, const void *x, float *y, int M, int N, int K, long rb,
+                          cudaStream_t st) {
+    gemv_simple_kernel<FMT, XT><<<(N + 7) / 8, 256, 0, st>>>(W, x, y, M, N, K, rb);
+    return cudaGetLastError();
+}
+
+cudaError_t dispatch_simple(int wf, int xt, const uint8_t *W, const void *x, float *y, int M, int N, int K, long rb,
+                            cudaStream_t st) {
+#define LWQ_SIMPLE(F)                                                                        \
+    if (xt == X_F32) return launch_simple<F, X_F32>(W, x, y, M, N, K, rb, st);              \
+    if (xt == X_F16) return launch_simple<F, X_F16>(W, x, y, M, N, K, rb, st);              \
+    return launch_simple<F, X_BF16>(W, x, y, M, N, K, rb, st);
+    switch (wf) {
+    case LWQ_Q8_0: { LWQ_SIMPLE(F_Q8_0) }
+    case LWQ_Q4_0: { LWQ_SIMPLE(F_Q4_0) }
+    case LWQ_Q4_K: { LWQ_SIMPLE(F_Q4_K) }
+    }
+#undef LWQ_SIMPLE
+    return cudaErrorInvalidValue;
+}
+
+int encode_weight_map(CUtensorMap *map, const void *Wq, int wf, int N, long rb) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return LWQ_ERR_CUDA;
+    const int cb = (wf == LWQ_Q8_0) ? 272 : 144;
+    cuuint64_t dims[2] = {(cuuint64_t)(rb / 2), (cuuint64_t)N};
+    cuuint64_t strides[1] = {(cuuint64_t)rb};
+    cuuint32_t box[2] = {(cuuint32_t)(cb / 2), (cuuint32_t)GEMV_ROWS};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(Wq), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? LWQ_OK : LWQ_ERR_CUDA;
+}
+
+// ------------------------------------------------------------- prefill GEMM
+template <int FMT, int XT, int BN>
+cudaError_t launch_gemm_tc(const CUtensorMap &wm, const CUtensorMap &xm, const GemmArgs &a, int ctas,
+                           size_t smem, cudaStream_t st) {
+    auto kern = gemm_tc_kernel<FMT, XT, BN>;
+    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), smem);
+    if (e != cudaSuccess) return e;
+    kern<<<ctas, GEMM_THREADS, smem, st>>>(wm, xm, a);
+    return cudaGetLastError();
+}
+
+template <int FMT, int XT>
+cudaError_t launch_gemm_bn(int bn, const CUtensorMap &wm, const CUtensorMap &xm, const GemmArgs &a, int ctas,
+                           size_t smem, cudaStream_t st) {
+    if (bn == 64) return launch_gemm_tc<FMT, XT, 64>(wm, xm, a, ctas, smem, st);
+    if (bn == 128) return launch_gemm_tc<FMT, XT, 128>(wm, xm, a, ctas, smem, st);
+    return launch_gemm_tc<FMT, XT, 256>(wm, xm, a, ctas, smem, st);
+}
+
+template <int FMT>
+cudaError_t launch_gemm_xt(int xt, int bn, const CUtensorMap &wm, const CUtensorMap &xm, const GemmArgs &a,
+                           int ctas, size_t smem, cudaStream_t st) {
+    if (xt == X_F16) return launch_gemm_bn<FMT, X_F16>(bn, wm, xm, a, ctas, smem, st);
+    return launch_gemm_bn<FMT, X_BF16>(bn, wm, xm, a, ctas, smem, st);
+}
+
+int gemm_launch(int wf, int xt, const void *Wq, const void *x, float *y, int M, int N, int K, long rb,
+                const lwq_config &cfg, size_t smem, unsigned long long timeout_ns, cudaStream_t st) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return LWQ_ERR_CUDA;
+    const int cb = gemm_chunk_bytes(wf);
+    const int bn = cfg.tile_m;
+    CUtensorMap wm, xm;
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)(rb / 2), (cuuint64_t)N};
+        cuuint64_t strides[1] = {(cuuint64_t)rb};
+        cuuint32_t box[2] = {(cuuint32_t)(cb / 2), (cuuint32_t)GEMM_WROWS};
+        cuuint32_t estr[2] = {1, 1};
+        if (enc(&wm, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(Wq), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return LWQ_ERR_CUDA;
+    }
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        cuuint32_t box[2] = {(cuuint32_t)GEMM_BK, (cuuint32_t)bn};
+        cuuint32_t estr[2] = {1, 1};
+        if (enc(&xm, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(x), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return LWQ_ERR_CUDA;
+    }
+    GemmArgs a;
+    a.y = y;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.nchunks = K / 256;
+    a.n_wtiles = (N + GEMM_WROWS - 1) / GEMM_WROWS;
+    a.n_ttiles = (M + bn - 1) / bn;
+    a.ab_stages = cfg.stages;
+    a.p_stages = 2;
+    a.timeout_ns = timeout_ns;
+    cudaError_t e;
+    switch (wf) {
+    case LWQ_Q4_0: e = launch_gemm_xt<F_Q4_0>(xt, bn, wm, xm, a, cfg.ctas, smem, st); break;
+    case LWQ_Q8_0: e = launch_gemm_xt<F_Q8_0>(xt, bn, wm, xm, a, cfg.ctas, smem, st); break;
+    default: e = launch_gemm_xt<F_Q4_K>(xt, bn, wm, xm, a, cfg.ctas, smem, st); break;
+    }
+    return e == cudaSuccess ? LWQ_OK : LWQ_ERR_CUDA;
+}
+
+int run(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, const lwq_config *force,
+        void *stream) {
+    t_last_launches = 0;
+    if (!Wq || !x || !y) return LWQ_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || K <= 0) return LWQ_ERR_INVALID_ARG;
+    int rc = check_fmt_k(fmt, K);
+    if (rc) return rc;
+    if (!aligned16(Wq) || !aligned16(x) || !aligned16(y)) return LWQ_ERR_MISALIGNED;
+    int dev;
+    if ((rc = current_device(&dev))) return rc;
+    const int wf = fmt & LWQ_FMT_MASK, xt = act_code(fmt);
+    Plan p;
+    if ((rc = make_plan(fmt, M, N, K, force, sm_count(dev), &p))) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const long rb = (long)K / block_weights(wf) * block_bytes(wf);
+    const size_t xelem = (xt == X_F32) ? 4 : 2;
+    int launches = 0;
+
+    if (p.cfg.path == 2) {
+        rc = gemm_launch(wf, xt, Wq, x, y, M, N, K, rb, p.cfg, p.smem, kTimeoutNs, st);
+        if (rc) return rc;
+        t_last_launches = 1;
+        return LWQ_OK;
+    }
+    if (p.cfg.path == 3) {
+        for (int m0 = 0; m0 < M; m0 += 16) {
+            const int mg = (M - m0) < 16 ? (M - m0) : 16;
+            cudaError_t e = dispatch_simple(wf, xt, static_cast<const uint8_t *>(Wq),
+                                            static_cast<const uint8_t *>(x) + (size_t)m0 * K * xelem,
+                                            y + (size_t)m0 * N, mg, N, K, rb, st);
+            if (e != cudaSuccess) return LWQ_ERR_CUDA;
+            ++launches;
+        }
+        t_last_launches = launches;
+        return LWQ_OK;
+    }
+
+    // tensor-core GEMV, in passes of m_group activation rows
+    DeviceState &ds = g_dev[dev];
+    if (p.ws_need > 0) {
+        if (!ds.registered) return LWQ_ERR_NOT_INITIALIZED;
+        if (ds.ws_bytes < p.ws_need) return LWQ_ERR_WORKSPACE_TOO_SMALL;
+    }
+    CUtensorMap map;
+    if ((rc = encode_weight_map(&map, Wq, wf, N, rb))) return rc;
+    const int nchunks = K / 256;
+    const int S = p.cfg.splits;
+    const int cps = (nchunks + S - 1) / S;
+    const int row_tiles = (N + GEMV_ROWS - 1) / GEMV_ROWS;
+    for (int m0 = 0; m0 < M; m0 += p.m_group) {
+        const int mg = (M - m0) < p.m_group ? (M - m0) : p.m_group;
+        GemvArgs a;
+        a.x = static_cast<const uint8_t *>(x) + (size_t)m0 * K * xelem;
+        a.y = y + (size_t)m0 * N;
+        a.counters = static_cast<unsigned *>(ds.ws);
+        a.partial = reinterpret_cast<float *>(static_cast<uint8_t *>(ds.ws) + kCounterBytes);
+        a.M = mg;
+        a.N = N;
+        a.K = K;
+        a.nchunks = nchunks;
+        a.splits = S;
+        a.chunks_per_split = cps;
+        a.row_tiles = row_tiles;
+        a.stages = p.cfg.stages;
+        a.timeout_ns = kTimeoutNs;
+        const int nt = mg <= 8 ? 1 : 2;
+        cudaError_t e = dispatch_gemv_tc(wf, xt, nt, map, a, p.cfg.ctas, p.cfg.warps,
+                                         gemv_smem(wf, p.cfg.warps, p.cfg.stages, nt), st);
+        if (e != cudaSuccess) return LWQ_ERR_CUDA;
+        ++launches;
+    }
+    t_last_launches = launches;
+    return LWQ_OK;
+}
+
+__global__ void selftest_timeout_kernel(unsigned long long timeout_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        // nothing arrives on `bar`: the bounded wait must give up and report
+        if (!mbar_wait(&bar, 0, timeout_ns, DEVERR_SELFTEST)) return;
+    }
+}
+
+}  // namespace
+}  // namespace lwq
+
+using namespace lwq;
+
+extern "C" {
+
+size_t lwq_row_bytes(int fmt, int64_t K) {
+    const int wf = fmt & LWQ_FMT_MASK;
+    if (block_weights(wf) == 0 || K <= 0 || K % block_weights(wf)) return 0;
+    return (size_t)(K / block_weights(wf)) * block_bytes(wf);
+}
+
+size_t lwq_workspace_size(int fmt, int max_M, int max_N, int max_K) {
+    if (max_M <= 0 || max_N <= 0 || max_K <= 0) return 0;
+    if (check_fmt_k(fmt, max_K)) return 0;
+    int dev = 0;
+    int sms = 148;
+    if (current_device(&dev) == LWQ_OK) sms = sm_count(dev);
+    // the need grows with M (up to one pass), N and K: evaluate at the maxima
+    // and at every pass size the M loop can use
+    size_t need = 0;
+    for (int m = 1; m <= max_M && m <= 16; ++m) {
+        Plan p;
+        if (make_plan(fmt, m, max_N, max_K, nullptr, sms, &p) == LWQ_OK && p.ws_need > need) need = p.ws_need;
+    }
+    if (need < 256) need = 256;
+    return need;
+}
+
+int lwq_init(void *d_workspace, size_t bytes) {
+    int dev;
+    int rc = current_device(&dev);
+    if (rc) return rc;
+    if (bytes > 0 && (!d_workspace || !aligned16(d_workspace))) return d_workspace ? LWQ_ERR_MISALIGNED : LWQ_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (bytes > 0 && cudaMemset(d_workspace, 0, bytes) != cudaSuccess) return LWQ_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return LWQ_ERR_CUDA;
+    g_dev[dev].ws = bytes ? d_workspace : nullptr;
+    g_dev[dev].ws_bytes = bytes;
+    g_dev[dev].registered = true;
+    return LWQ_OK;
+}
+
+int lwq_shutdown(void) {
+    int dev;
+    if (current_device(&dev) == LWQ_OK) {
+        std::lock_guard<std::mutex> lk(g_mu);
+        g_dev[dev] = DeviceState{};
+    }
+    return LWQ_OK;
+}
+
+int lwq_matmul(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, void *stream) {
+    return run(fmt, Wq, x, y, M, N, K, nullptr, stream);
+}
+
+int lwq_matmul_config(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, const lwq_config *cfg,
+                      void *stream) {
+    return run(fmt, Wq, x, y, M, N, K, cfg, stream);
+}
+
+int lwq_select_config(int fmt, int M, int N, int K, lwq_config *cfg) {
+    if (!cfg || M <= 0 || N <= 0 || K <= 0) return LWQ_ERR_INVALID_ARG;
+    int rc = check_fmt_k(fmt, K);
+    if (rc) return rc;
+    int dev = 0, sms = 148;
+    if (current_device(&dev) == LWQ_OK) sms = sm_count(dev);
+    Plan p;
+    if ((rc = make_plan(fmt, M, N, K, nullptr, sms, &p))) return rc;
+    *cfg = p.cfg;
+    return LWQ_OK;
+}
+
+const char *lwq_status_string(int s) {
+    switch (s) {
+    case LWQ_OK: return "ok";
+    case LWQ_ERR_INVALID_ARG: return "invalid argument";
+    case LWQ_ERR_UNSUPPORTED: return "unsupported format, dtype or configuration";
+    case LWQ_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case LWQ_ERR_NOT_INITIALIZED: return "workspace not registered (call lwq_init)";
+    case LWQ_ERR_WORKSPACE_TOO_SMALL: return "workspace too small (see lwq_workspace_size)";
+    case LWQ_ERR_CUDA: return "CUDA error";
+    case LWQ_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
+    default: return "unknown status";
+    }
+}
+
+int lwq_get_device_error(void) {
+    unsigned v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_dev_error, sizeof(v)) != cudaSuccess) return LWQ_ERR_CUDA;
+    if (v == 0) return LWQ_OK;
+    unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_dev_error, &zero, sizeof(zero)) != cudaSuccess) return LWQ_ERR_CUDA;
+    return LWQ_ERR_DEVICE_TIMEOUT;
+}
+
+int lwq_selftest_timeout(unsigned timeout_us, void *stream) {
+    selftest_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        (unsigned long long)timeout_us * 1000ull);
+    return cudaGetLastError() == cudaSuccess ? LWQ_OK : LWQ_ERR_CUDA;
+}
+
+int lwq_last_launch_count(void) { return t_last_launches; }
+
+int lwq_version(void) { return 0x000100; }
+
+}  // extern "C"

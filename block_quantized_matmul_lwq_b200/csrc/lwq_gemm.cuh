@@ -1,0 +1,452 @@
+// Prefill GEMM (M > 16 activation rows): y[M,N] = x[M,K] . dequant(Wq)^T
+// on the 5th-generation tensor cores (tcgen05, accumulators in TMEM).
+//
+// This is the matrix-matrix half of the co-designed dequantization in
+// "Resumo Tecnico: Llamas na Web", "3. Design de Shader Consciente de
+// Quantizacao": quantized tiles are loaded, dequantized in shared memory and
+// reused across rows; here they are reused across up to 256 activation rows
+// per MMA, so the decode work per flop shrinks with the token tile.
+//
+// Roles (one persistent CTA per SM, warp-specialized):
+//   warp 0      TMA producer: packed weight chunks [128 rows][256 weights]
+//               and activation tiles [BN tokens][64 k] (128-byte swizzle)
+//   warp 1      TMEM allocator and single-thread UMMA issuer
+//   warps 2..9  dequantizers: packed chunk -> bf16/fp16 weight tile
+//               [128 rows][64 k] in the UMMA K-major 128-byte-swizzle layout
+//   warps 10-13 epilogue: TMEM -> registers -> y (fp32), coalesced along N
+// UMMA shape: M = 128 weight rows, N = BN tokens (64/128/256), K = 16;
+// accumulators double-buffered in TMEM so the epilogue of one tile overlaps
+// the main loop of the next.  Every wait is bounded (device error word).
+#pragma once
+
+#include "../../include/lwq.h"
+#include "lwq_gemv.cuh"
+#include "lwq_ptx.cuh"
+
+namespace lwq {
+
+constexpr int GEMM_WROWS = 128;       // weight rows per tile (UMMA M)
+constexpr int GEMM_BK = 64;           // k per k-block (one 128-byte swizzle atom of 16-bit values)
+constexpr int GEMM_KB_PER_CHUNK = 4;  // k-blocks per packed 256-weight chunk
+constexpr int GEMM_DQ_WARPS = 8;
+constexpr int GEMM_EPI_WARPS = 4;
+constexpr int GEMM_THREADS = (2 + GEMM_DQ_WARPS + GEMM_EPI_WARPS) * 32;
+
+struct GemmPlan {
+    int warps, stages, ctas, tile_n, tile_m;
+    size_t smem;
+};
+
+struct GemmArgs {
+    float *y;
+    int M, N, K;
+    int nchunks;      // K / 256
+    int n_wtiles;     // ceil(N / 128)
+    int n_ttiles;     // ceil(M / BN)
+    int ab_stages;
+    int p_stages;
+    unsigned long long timeout_ns;
+};
+
+template <int FMT>
+struct GemmFmt;
+template <>
+struct GemmFmt<F_Q4_0> { static constexpr int chunk_bytes = 144; };
+template <>
+struct GemmFmt<F_Q8_0> { static constexpr int chunk_bytes = 272; };
+template <>
+struct GemmFmt<F_Q4_K> { static constexpr int chunk_bytes = 144; };
+
+__host__ __device__ constexpr size_t gemm_a_bytes() { return (size_t)GEMM_WROWS * 128; }
+__host__ __device__ constexpr size_t gemm_b_bytes(int bn) { return (size_t)bn * 128; }
+
+// Shared memory: [ab stages x (A 16 KB | B bn*128 B)] [p stages x 128*CB] [barriers] [tmem addr]
+__host__ __device__ inline size_t gemm_smem_bytes(int cb, int bn, int ab_stages, int p_stages) {
+    size_t s = (size_t)ab_stages * (gemm_a_bytes() + gemm_b_bytes(bn));
+    s += (size_t)p_stages * GEMM_WROWS * cb;
+    s = (s + 7) & ~(size_t)7;
+    s += (size_t)(2 * ab_stages + 2 * p_stages + 4 + 1) * 8 + 16;
+    return s + 1024;  // slack to align the base to 1024 B
+}
+
+// Byte offset of 16-bit element (row r, k) inside a [rows][64] K-major tile
+// in the 128-byte swizzle layout: row r at r*128, 16-byte chunk j = k/8 stored
+// at chunk position j ^ (r % 8).
+__device__ __forceinline__ uint32_t sw128_chunk_offset(int r, int j) {
+    return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4));
+}
+
+// ------------------------------------------------------------- dequantizers
+// One thread writes the four 16-byte chunks (32 weights) of unit (row, h) of
+// a k-block: h selects the first or second 32 weights of the block's 64.
+
+// exact (q - 8) pairs in the target type for the low nibbles of bytes b0, b1
+// at bits 0-3 and 16-19 of `v`
+template <int XT>
+__device__ __forceinline__ uint32_t q4_pair(uint32_t v) {
+    if constexpr (XT == X_F16)
+        return hfma2_f16(and_or(v, 0x000F000Fu, H2_MAGIC), H2_ONE, H2_M1032);
+    else
+        return hfma2_bf16(and_or(v, 0x000F000Fu, B2_MAGIC), B2_ONE, B2_M136);
+}
+
+// w = d * (q - 8), rounded once to the 16-bit type.
+// fp16: d is exact in fp16, one rounding in the multiply.
+// bf16: d = d_hi + d_lo with both parts exact in bf16 and (q-8)*d_lo exact,
+//       so fma((q-8), d_hi, (q-8)*d_lo) rounds the exact product once.
+template <int XT>
+__device__ __forceinline__ uint32_t scale_pair(uint32_t qm8, uint32_t dh2, uint32_t dl2) {
+    if constexpr (XT == X_F16)
+        return hmul2_f16(qm8, dh2);
+    else
+        return hfma2_bf16(qm8, dh2, hmul2_bf16(qm8, dl2));
+}
+
+template <int XT>
+__device__ __forceinline__ void split_scale(float d, uint32_t &dh2, uint32_t &dl2) {
+    if constexpr (XT == X_F16) {
+        const uint32_t h = __half_as_ushort(__float2half_rn(d));  // d came from fp16: exact
+        dh2 = h | (h << 16);
+        dl2 = 0;
+    } else {
+        const __nv_bfloat16 hi = __float2bfloat16_rn(d);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(d - __bfloat162float(hi));  // exact (<= 4 bits)
+        const uint32_t a = __bfloat16_as_ushort(hi), b = __bfloat16_as_ushort(lo);
+        dh2 = a | (a << 16);
+        dl2 = b | (b << 16);
+    }
+}
+
+template <int FMT, int XT>
+struct Dequant;
+
+// Q4_0: k-block kb of a chunk = blocks 2kb (h=0) and 2kb+1 (h=1).
+template <int XT>
+struct Dequant<F_Q4_0, XT> {
+    static __device__ __forceinline__ void run(const uint8_t *prow, int kb, int h, uint32_t a_row_base, int r) {
+        const uint32_t *w = reinterpret_cast<const uint32_t *>(prow) + 9 * kb + 4 * h;
+        uint32_t W[5];
+#pragma unroll
+        for (int i = 0; i < 5; ++i) W[i] = w[i];
+        const uint32_t s = h ? 32u : 16u;
+        uint32_t q[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) q[i] = __funnelshift_rc(W[i], W[i + 1], s);
+        const float d = f16_bits_to_float(h ? (W[0] >> 16) : W[0]);
+        uint32_t dh2, dl2;
+        split_scale<XT>(d, dh2, dl2);
+        // chunk c (0..3): elements 8c..8c+7 of the block
+        //   c=0: low nibbles of bytes 0-7, c=1: low of 8-15, c=2: high of 0-7, c=3: high of 8-15
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const uint32_t qa = q[(c & 1) * 2], qb = q[(c & 1) * 2 + 1];
+            const uint32_t sh = (c >> 1) * 4;
+            uint32_t o[4];
+            const uint32_t src[2] = {qa, qb};
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                const uint32_t v01 = prmt(src[p], 0u, 0x4140u) >> sh;  // bytes 0,1 -> halves
+                const uint32_t v23 = prmt(src[p], 0u, 0x4342u) >> sh;  // bytes 2,3 -> halves
+                o[2 * p] = scale_pair<XT>(q4_pair<XT>(v01), dh2, dl2);
+                o[2 * p + 1] = scale_pair<XT>(q4_pair<XT>(v23), dh2, dl2);
+            }
+            st_shared_v4(a_row_base + sw128_chunk_offset(r, 4 * h + c), o[0], o[1], o[2], o[3]);
+        }
+    }
+};
+
+// Q8_0: k-block kb = blocks 2kb (h=0) and 2kb+1 (h=1); 34-byte blocks.
+template <int XT>
+struct Dequant<F_Q8_0, XT> {
+    static __device__ __forceinline__ void run(const uint8_t *prow, int kb, int h, uint32_t a_row_base, int r) {
+        const uint32_t *w = reinterpret_cast<const uint32_t *>(prow) + 17 * kb + 8 * h;
+        uint32_t W[9];
+#pragma unroll
+        for (int i = 0; i < 9; ++i) W[i] = w[i];
+        const uint32_t s = h ? 32u : 16u;
+        const float d = f16_bits_to_float(h ? (W[0] >> 16) : W[0]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const uint32_t q0 = __funnelshift_rc(W[2 * c], W[2 * c + 1], s) ^ 0x80808080u;
+            const uint32_t q1 = __funnelshift_rc(W[2 * c + 1], W[2 * c + 2], s) ^ 0x80808080u;
+            uint32_t o[4];
+            if constexpr (XT == X_F16) {
+                const uint32_t h16 = __half_as_ushort(__float2half_rn(d));
+                const uint32_t d2 = h16 | (h16 << 16);
+                o[0] = hmul2_f16(hfma2_f16(prmt(q0, 0x6400u, 0x5150u), H2_ONE, H2_M1152), d2);
+                o[1] = hmul2_f16(hfma2_f16(prmt(q0, 0x6400u, 0x5352u), H2_ONE, H2_M1152), d2);
+                o[2] = hmul2_f16(hfma2_f16(prmt(q1, 0x6400u, 0x5150u), H2_ONE, H2_M1152), d2);
+                o[3] = hmul2_f16(hfma2_f16(prmt(q1, 0x6400u, 0x5352u), H2_ONE, H2_M1152), d2);
+            } else {
+                const float bias = 8388736.0f;  // 2^23 + 128
+                float f[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    f[i] = (__uint_as_float(prmt(q0, 0x4B000000u, 0x7440u + i)) - bias) * d;
+                    f[4 + i] = (__uint_as_float(prmt(q1, 0x4B000000u, 0x7440u + i)) - bias) * d;
+                }
+                o[0] = pack_bf16x2(f[0], f[1]);
+                o[1] = pack_bf16x2(f[2], f[3]);
+                o[2] = pack_bf16x2(f[4], f[5]);
+                o[3] = pack_bf16x2(f[6], f[7]);
+            }
+            st_shared_v4(a_row_base + sw128_chunk_offset(r, 4 * h + c), o[0], o[1], o[2], o[3]);
+        }
+    }
+};
+
+// Q4_K: chunk = one superblock; k-block kb = nibble group kb: h=0 sub-block
+// 2kb (low nibbles), h=1 sub-block 2kb+1 (high nibbles).
+template <int XT>
+struct Dequant<F_Q4_K, XT> {
+    static __device__ __forceinline__ void run(const uint8_t *prow, int kb, int h, uint32_t a_row_base, int r) {
+        const uint4 hd = *reinterpret_cast<const uint4 *>(prow);
+        const uint4 qa = *reinterpret_cast<const uint4 *>(prow + 16 + 32 * kb);
+        const uint4 qb = *reinterpret_cast<const uint4 *>(prow + 32 + 32 * kb);
+        const int j = 2 * kb + h;
+        const uint32_t s0 = hd.y, s1 = hd.z, s2 = hd.w;
+        uint32_t scw, mw;
+        if (j < 4) {
+            scw = s0 & 0x3F3F3F3Fu;
+            mw = s1 & 0x3F3F3F3Fu;
+        } else {
+            scw = (s2 & 0x0F0F0F0Fu) | ((s0 >> 2) & 0x30303030u);
+            mw = ((s2 >> 4) & 0x0F0F0F0Fu) | ((s1 >> 2) & 0x30303030u);
+        }
+        const int sc = (scw >> (8 * (j & 3))) & 63, m = (mw >> (8 * (j & 3))) & 63;
+        const float ds = f16_bits_to_float(hd.x) * (float)sc;           // exact in fp32
+        const float dm = f16_bits_to_float(hd.x >> 16) * (float)m;      // exact in fp32
+        const uint32_t qw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+        const uint32_t sh = 4u * h;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            float f[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t byte = (qw[2 * c + (i >> 2)] >> (8 * (i & 3) + sh)) & 15u;
+                f[i] = fmaf(ds, __uint_as_float(0x4B000000u | byte) - 8388608.0f, -dm);
+            }
+            uint32_t o[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+                o[p] = (XT == X_F16) ? pack_f16x2(f[2 * p], f[2 * p + 1]) : pack_bf16x2(f[2 * p], f[2 * p + 1]);
+            st_shared_v4(a_row_base + sw128_chunk_offset(r, 4 * h + c), o[0], o[1], o[2], o[3]);
+        }
+    }
+};
+
+// -------------------------------------------------------------------- kernel
+template <int FMT, int XT, int BN>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap,
+                   const GemmArgs a) {
+    constexpr int CB = GemmFmt<FMT>::chunk_bytes;
+    constexpr uint32_t A_BYTES = (uint32_t)gemm_a_bytes();
+    constexpr uint32_t B_BYTES = (uint32_t)gemm_b_bytes(BN);
+    constexpr uint32_t AB_BYTES = A_BYTES + B_BYTES;
+    constexpr uint32_t P_BYTES = (uint32_t)GEMM_WROWS * CB;
+    constexpr uint32_t TMEM_COLS = 2 * BN;
+    constexpr uint32_t IDESC = umma_idesc_f16(XT == X_F16 ? 0 : 1, GEMM_WROWS, BN);
+
+    extern __shared__ uint8_t smem_raw[];
+    // 1024-byte aligned base (128-byte swizzle atoms)
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+    const int S = a.ab_stages, P = a.p_stages;
+    uint8_t *ab = smem;
+    uint8_t *pk = ab + (size_t)S * AB_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(pk + (((size_t)P * P_BYTES + 7) & ~(size_t)7));
+    uint64_t *ab_full = bars, *ab_empty = bars + S;
+    uint64_t *p_full = bars + 2 * S, *p_empty = bars + 2 * S + P;
+    uint64_t *acc_full = bars + 2 * S + 2 * P, *acc_empty = acc_full + 2;
+    uint64_t *mma_done = acc_full + 4;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_tiles = a.n_wtiles * a.n_ttiles;
+    const int kblocks = a.nchunks * GEMM_KB_PER_CHUNK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&ab_full[s], 1 + GEMM_DQ_WARPS);
+            mbar_init(&ab_empty[s], 1);
+        }
+        for (int s = 0; s < P; ++s) {
+            mbar_init(&p_full[s], 1);
+            mbar_init(&p_empty[s], GEMM_DQ_WARPS);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&acc_full[s], 1);
+            mbar_init(&acc_empty[s], GEMM_EPI_WARPS);
+        }
+        mbar_init(mma_done, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&wmap);
+            tma_prefetch_desc(&xmap);
+            int kbi = 0, ci = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
+                const int tt = tile % a.n_ttiles, wt = tile / a.n_ttiles;
+                for (int c = 0; ok && c < a.nchunks; ++c, ++ci) {
+                    const int ps = ci % P;
+                    if (ci >= P && !(ok = mbar_wait(&p_empty[ps], ((ci / P) - 1) & 1, a.timeout_ns, DEVERR_GEMM_WAIT)))
+                        break;
+                    mbar_arrive_expect_tx(&p_full[ps], P_BYTES);
+                    tma_load_2d(pk + (size_t)ps * P_BYTES, &wmap, &p_full[ps], c * (CB / 2), wt * GEMM_WROWS);
+                    for (int kb = 0; kb < GEMM_KB_PER_CHUNK; ++kb, ++kbi) {
+                        const int s = kbi % S;
+                        if (kbi >= S &&
+                            !(ok = mbar_wait(&ab_empty[s], ((kbi / S) - 1) & 1, a.timeout_ns, DEVERR_GEMM_WAIT)))
+                            break;
+                        mbar_arrive_expect_tx(&ab_full[s], B_BYTES);
+                        tma_load_2d(ab + (size_t)s * AB_BYTES + A_BYTES, &xmap, &ab_full[s],
+                                    (c * GEMM_KB_PER_CHUNK + kb) * GEMM_BK, tt * BN);
+                    }
+                }
+            }
+            // drain: the last loads land before the CTA may exit
+            for (int j = max(0, kbi - S); j < kbi; ++j)
+                mbar_wait(&ab_full[j % S], (j / S) & 1, a.timeout_ns, DEVERR_GEMM_WAIT);
+            for (int j = max(0, ci - P); j < ci; ++j)
+                mbar_wait(&p_full[j % P], (j / P) & 1, a.timeout_ns, DEVERR_GEMM_WAIT);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------- UMMA issuer
+        if (lane == 0) {
+            int kbi = 0, ti = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++ti) {
+                const int as = ti & 1;
+                if (ti >= 2 && !(ok = mbar_wait(&acc_empty[as], ((ti >> 1) - 1) & 1, a.timeout_ns, DEVERR_GEMM_WAIT)))
+                    break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(as * BN);
+                for (int k = 0; k < kblocks; ++k, ++kbi) {
+                    const int s = kbi % S;
+                    if (!(ok = mbar_wait(&ab_full[s], (kbi / S) & 1, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(ab + (size_t)s * AB_BYTES);
+                    const uint32_t b_addr = a_addr + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < GEMM_BK / 16; ++kk)
+                        umma_f16(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32), IDESC,
+                                 (k | kk) ? 1u : 0u);
+                    umma_commit(&ab_empty[s]);
+                }
+                if (!ok) break;
+                umma_commit(&acc_full[as]);
+            }
+            // every issued MMA completes before TMEM is released
+            umma_commit(mma_done);
+            mbar_wait(mma_done, 0, a.timeout_ns, DEVERR_GEMM_WAIT);
+        }
+    } else if (warp < 2 + GEMM_DQ_WARPS) {
+        // ------------------------------------------------------ dequantizers
+        const int t = threadIdx.x - 64;          // 0..255
+        const int r = t & (GEMM_WROWS - 1);      // weight row within the tile
+        const int h = t >> 7;                    // which 32 of the k-block's 64 weights
+        int kbi = 0, ci = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
+            for (int c = 0; ok && c < a.nchunks; ++c, ++ci) {
+                const int ps = ci % P;
+                if (!(ok = mbar_wait(&p_full[ps], (ci / P) & 1, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
+                const uint8_t *prow = pk + (size_t)ps * P_BYTES + (size_t)r * CB;
+                for (int kb = 0; kb < GEMM_KB_PER_CHUNK; ++kb, ++kbi) {
+                    const int s = kbi % S;
+                    if (kbi >= S &&
+                        !(ok = mbar_wait(&ab_empty[s], ((kbi / S) - 1) & 1, a.timeout_ns, DEVERR_GEMM_WAIT)))
+                        break;
+                    Dequant<FMT, XT>::run(prow, kb, h, smem_u32(ab + (size_t)s * AB_BYTES), r);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ab_full[s]);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_empty[ps]);
+            }
+        }
+    } else {
+        // --------------------------------------------------------- epilogue
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int N = a.N, M = a.M;
+        int ti = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++ti) {
+            const int tt = tile % a.n_ttiles, wt = tile / a.n_ttiles;
+            const int as = ti & 1;
+            if (!mbar_wait(&acc_full[as], (ti >> 1) & 1, a.timeout_ns, DEVERR_GEMM_WAIT)) break;
+            tc_fence_after();
+            const int n = wt * GEMM_WROWS + q * 32 + lane;
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(as * BN);
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(taddr + c0, v);
+                tmem_wait_ld();
+                const int m0 = tt * BN + c0;
+                if (n < N) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (m0 + j < M) a.y[(size_t)(m0 + j) * N + n] = __uint_as_float(v[j]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[as]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+inline bool gemm_eligible(int wf, int xt, long K) {
+    (void)wf;
+    return (xt == X_F16 || xt == X_BF16) && K % 256 == 0;
+}
+
+inline int gemm_chunk_bytes(int wf) { return wf == LWQ_Q8_0 ? 272 : 144; }
+
+inline int gemm_plan(int wf, int xt, int M, int N, int K, const lwq_config *force, int sms, GemmPlan *g) {
+    (void)xt;
+    (void)K;
+    int bn = force && force->tile_m ? force->tile_m : (M <= 64 ? 64 : (M <= 128 ? 128 : 256));
+    if (bn != 64 && bn != 128 && bn != 256) return LWQ_ERR_UNSUPPORTED;
+    const int cb = gemm_chunk_bytes(wf);
+    int p_stages = 2;
+    int ab = force && force->stages ? force->stages : 4;
+    const size_t limit = 232448;
+    while (ab > 2 && gemm_smem_bytes(cb, bn, ab, p_stages) > limit) --ab;
+    if (gemm_smem_bytes(cb, bn, ab, p_stages) > limit) return LWQ_ERR_UNSUPPORTED;
+    const int tiles = ((N + GEMM_WROWS - 1) / GEMM_WROWS) * ((M + bn - 1) / bn);
+    int ctas = force && force->ctas ? force->ctas : sms;
+    if (ctas > tiles) ctas = tiles;
+    if (ctas < 1) ctas = 1;
+    g->warps = GEMM_DQ_WARPS;
+    g->stages = ab;
+    g->ctas = ctas;
+    g->tile_n = GEMM_WROWS;
+    g->tile_m = bn;
+    g->smem = gemm_smem_bytes(cb, bn, ab, p_stages);
+    return LWQ_OK;
+}
+
+}  // namespace lwq

@@ -1,0 +1,171 @@
+/*
+ * lwq.h -- block-quantized matmul for NVIDIA B200 (sm_100a).
+ *
+ *     y[M,N] = x[M,K] . dequant(Wq[N,K])^T
+ *
+ * The weights Wq are stored in llama.cpp-style blocks (the "legacy" and
+ * "K-quant" families named in "Resumo Tecnico: Llamas na Web",
+ * "Declaracao do Problema" item 3, and in its "3. Design de Shader Consciente
+ * de Quantizacao", which co-designs dequantization with the matmul kernels:
+ * decoded in registers for the matrix-vector (decode) case and in shared
+ * memory, reused across rows, for the matrix-matrix (prefill) case).
+ *
+ * Paths (chosen per call by a per-shape configuration table, the analogue of
+ * the tunable tile sizes in "2. Biblioteca de Kernels Portatil em
+ * Desempenho", "Parametros Ajustaveis"):
+ *   M <= 16  decode GEMV: packed rows staged by TMA into shared memory,
+ *            decoded in registers, multiplied on the tensor cores with
+ *            warp-level MMAs, split-K partials reduced deterministically;
+ *   M >  16  prefill GEMM: packed tiles staged by TMA, dequantized to
+ *            bf16/fp16 in shared memory, tcgen05 MMAs accumulating in TMEM.
+ *
+ * Everything is plain C: pointers and sizes, no C++ or framework types.
+ */
+#ifndef LWQ_H
+#define LWQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ------------------------------------------------------------ status codes */
+typedef enum {
+    LWQ_OK = 0,
+    LWQ_ERR_INVALID_ARG = 1,        /* a size is <= 0, K is not a multiple of the block, NULL pointer */
+    LWQ_ERR_UNSUPPORTED = 2,        /* unknown format / activation code, or a shape no path handles */
+    LWQ_ERR_MISALIGNED = 3,         /* Wq, x, y or the workspace is not 16-byte aligned */
+    LWQ_ERR_NOT_INITIALIZED = 4,    /* a call needs the workspace and lwq_init was not called on this device */
+    LWQ_ERR_WORKSPACE_TOO_SMALL = 5,/* the registered workspace is smaller than this call needs */
+    LWQ_ERR_CUDA = 6,               /* a CUDA runtime/driver call failed (launch error, bad device) */
+    LWQ_ERR_DEVICE_TIMEOUT = 7      /* a kernel gave up a bounded wait (see lwq_get_device_error) */
+} lwq_status;
+
+/* ------------------------------------------------- format and dtype codes
+ * fmt = weight format | activation dtype.
+ *
+ * LWQ_Q8_0: 32 weights per 34-byte block: fp16 d (little endian), int8 q[32];
+ *           w = d*q.
+ * LWQ_Q4_0: 32 weights per 18-byte block: fp16 d, 16 bytes b[16]; byte i
+ *           holds element i in its low nibble and element i+16 in its high
+ *           nibble; w = (nibble - 8)*d.
+ * LWQ_Q4_K: 256 weights per 144-byte superblock: fp16 d, fp16 dmin, 12 bytes
+ *           of eight 6-bit (scale, min) pairs (for j < 4: sc_j = s[j]&63,
+ *           m_j = s[j+4]&63; for j >= 4: sc_j = (s[j+4]&15)|((s[j-4]>>6)<<4),
+ *           m_j = (s[j+4]>>4)|((s[j]>>6)<<4)), 128 bytes of nibbles in 4
+ *           groups of 32 (group g: low nibbles are sub-block 2g, high
+ *           nibbles sub-block 2g+1); w = d*sc_j*q - dmin*m_j.
+ * Activations x: fp32, fp16 or bf16, row-major [M][K].
+ */
+#define LWQ_Q8_0 1
+#define LWQ_Q4_0 2
+#define LWQ_Q4_K 3
+#define LWQ_FMT_MASK 0xFF
+#define LWQ_ACT_F32 0x000
+#define LWQ_ACT_F16 0x100
+#define LWQ_ACT_BF16 0x200
+#define LWQ_ACT_MASK 0xF00
+
+/* Bytes of one packed row of K weights (K/32*34, K/32*18, K/256*144), or 0
+ * when fmt is unknown or K is not a positive multiple of the block size. */
+size_t lwq_row_bytes(int fmt, int64_t K);
+
+/* Device workspace bytes that lwq_matmul needs for every call with
+ * M <= max_M, N <= max_N, K <= max_K in this format.  The workspace holds the
+ * split-K partial sums (fp32) and the per-row-tile arrival counters that the
+ * deterministic split-K reduction uses; it is the library's one static arena,
+ * sized once at start-up ("1. Inferencia Local Eficiente em Memoria",
+ * "Alocacao Estatica de Memoria" and "Arena de Buffer de Parametros").
+ * Returns 0 for invalid arguments. */
+size_t lwq_workspace_size(int fmt, int max_M, int max_N, int max_K);
+
+/* Register the caller-owned device workspace for the CURRENT device.
+ * d_workspace: device pointer, 16-byte aligned (NULL with bytes == 0 is
+ * allowed: calls that need no workspace still run).  The library keeps the
+ * pointer until lwq_shutdown or the next lwq_init on this device; it never
+ * allocates, frees or reads it outside lwq_matmul.  This call zeroes the
+ * arrival-counter region with a synchronous cudaMemset, so call it before any
+ * stream capture.  Errors: LWQ_ERR_MISALIGNED, LWQ_ERR_CUDA. */
+int lwq_init(void *d_workspace, size_t bytes);
+
+/* Forget the workspace registered for the current device.  Always LWQ_OK. */
+int lwq_shutdown(void);
+
+/*
+ * y[M,N] (fp32, row-major) = x[M,K] . dequant(Wq)^T.
+ *
+ *   fmt     weight format | activation dtype (codes above)
+ *   Wq      device pointer, N packed rows of lwq_row_bytes(fmt, K) bytes each
+ *   x       device pointer, row-major [M][K] in the activation dtype
+ *   y       device pointer, row-major [M][N] fp32, fully overwritten
+ *   M, N, K sizes (> 0); K a multiple of 32 (Q8_0, Q4_0) or 256 (Q4_K)
+ *   stream  a cudaStream_t (NULL = the legacy default stream)
+ *
+ * Ownership: the caller owns Wq, x, y and the workspace.  The call is
+ * asynchronous: it validates the arguments on the host, enqueues one or two
+ * kernels on `stream` and returns; it never allocates and never synchronizes
+ * the host.  Kernel faults surface at the caller's next synchronization, as
+ * with any CUDA launch.  Wq, x and y must be 16-byte aligned
+ * (LWQ_ERR_MISALIGNED).  Calls that use split-K (see lwq_workspace_size) need
+ * a registered workspace (LWQ_ERR_NOT_INITIALIZED,
+ * LWQ_ERR_WORKSPACE_TOO_SMALL); calls sharing one workspace must be ordered
+ * (one stream, or events), since their partial sums share the arena.
+ * M > 16 with fp32 activations runs the GEMV path over groups of rows of x.
+ */
+int lwq_matmul(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, void *stream);
+
+/* ------------------------------------------------ configuration table
+ * The per-shape configuration lwq_matmul would use, and a way to force one
+ * (used by the sweep that fills the table and by tests). */
+typedef struct {
+    int path;        /* 1 = GEMV (tensor-core MMA), 2 = GEMM (tcgen05), 3 = simple GEMV */
+    int warps;       /* GEMV: compute warps per CTA, each owning 256 weights of K */
+    int stages;      /* pipeline depth (shared-memory ring stages) */
+    int splits;      /* GEMV: split-K factor (1 = none) */
+    int ctas;        /* CTAs launched (persistent grid) */
+    int tile_n;      /* GEMM: output columns per tile (weights rows) */
+    int tile_m;      /* GEMM: output rows per tile (activation rows) */
+    int reserved[5];
+} lwq_config;
+
+/* Fill *cfg with the configuration lwq_matmul(fmt, ., ., ., M, N, K) would
+ * use on the current device.  Errors as lwq_matmul's argument checks. */
+int lwq_select_config(int fmt, int M, int N, int K, lwq_config *cfg);
+
+/* lwq_matmul with a forced configuration.  Fields set to 0 take the table's
+ * value; an impossible configuration returns LWQ_ERR_UNSUPPORTED. */
+int lwq_matmul_config(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K,
+                      const lwq_config *cfg, void *stream);
+
+/* ------------------------------------------------ errors and diagnostics */
+
+/* Static description of a status code. */
+const char *lwq_status_string(int status);
+
+/* Device-side error word of the current device: every wait in the kernels
+ * (on an mbarrier, a split-K counter or a TMEM handoff) is bounded; a kernel
+ * that gives up sets a bit here and returns instead of hanging.  The caller
+ * must synchronize first.  Returns LWQ_OK, LWQ_ERR_DEVICE_TIMEOUT (and clears
+ * the word), or LWQ_ERR_CUDA. */
+int lwq_get_device_error(void);
+
+/* Launch a one-CTA kernel on `stream` that waits on an mbarrier nothing ever
+ * arrives at, with a wait bound of timeout_us microseconds, so that callers
+ * can check that bounded waits end and report LWQ_ERR_DEVICE_TIMEOUT through
+ * lwq_get_device_error.  Faults nothing and hangs nothing. */
+int lwq_selftest_timeout(unsigned timeout_us, void *stream);
+
+/* Number of kernels the last successful lwq_matmul / lwq_matmul_config call
+ * on this thread enqueued. */
+int lwq_last_launch_count(void);
+
+/* Library version, e.g. 0x000100 for 0.1.0. */
+int lwq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LWQ_H */

@@ -1,0 +1,105 @@
+"""Host-side checks of the C-ABI library: it loads, exports every symbol the
+header declares, and its argument checks / configuration table behave.  No
+call here reaches a GPU (every checked call returns before any device work)."""
+
+import os
+import re
+
+import pytest
+
+import block_quantized_matmul_lwq_b200 as lwq
+from block_quantized_matmul_lwq_b200 import build as lwq_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    lwq_build.build()
+
+
+def header_functions():
+    with open(os.path.join(ROOT, "include", "lwq.h")) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(lwq_[a-z_]+)\s*\(", src)))
+
+
+def test_exports_every_header_symbol():
+    names = header_functions()
+    assert len(names) >= 10
+    lib = lwq.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(lwq.EXPORTS) == names
+
+
+def test_row_bytes():
+    f = lwq.fmt_code
+    assert lwq.lwq_row_bytes(f("q8_0", "f32"), 4096) == 4352
+    assert lwq.lwq_row_bytes(f("q4_0", "f32"), 4096) == 2304
+    assert lwq.lwq_row_bytes(f("q4_k", "f16"), 11008) == 6192
+    assert lwq.lwq_row_bytes(f("q4_k", "f16"), 128) == 0
+    assert lwq.lwq_row_bytes(f("q4_0", "f32"), 48) == 0
+    assert lwq.lwq_row_bytes(f("q4_0", "f32"), -32) == 0
+    assert lwq.lwq_row_bytes(0x7, 4096) == 0
+
+
+FAKE = 0x10000  # 16-byte aligned host integer; never dereferenced by the checks below
+
+
+@pytest.mark.parametrize("args,status", [
+    ((lwq.fmt_code("q4_0", "f32"), FAKE, FAKE, FAKE, 0, 8, 64), 1),
+    ((lwq.fmt_code("q4_0", "f32"), FAKE, FAKE, FAKE, 1, -8, 64), 1),
+    ((lwq.fmt_code("q4_0", "f32"), FAKE, FAKE, FAKE, 1, 8, 48), 1),
+    ((lwq.fmt_code("q4_k", "f16"), FAKE, FAKE, FAKE, 1, 8, 128), 1),
+    ((0x9, FAKE, FAKE, FAKE, 1, 8, 64), 2),
+    ((lwq.LWQ_Q4_0 | 0x300, FAKE, FAKE, FAKE, 1, 8, 64), 2),
+    ((lwq.LWQ_Q4_0 | 0x10000, FAKE, FAKE, FAKE, 1, 8, 64), 2),
+    ((lwq.fmt_code("q4_0", "f32"), FAKE + 2, FAKE, FAKE, 1, 8, 64), 3),
+    ((lwq.fmt_code("q4_0", "f32"), FAKE, FAKE + 4, FAKE, 1, 8, 64), 3),
+    ((lwq.fmt_code("q4_0", "f32"), FAKE, FAKE, FAKE + 8, 1, 8, 64), 3),
+    ((lwq.fmt_code("q4_0", "f32"), 0, FAKE, FAKE, 1, 8, 64), 1),
+])
+def test_argument_checks(args, status):
+    fmt, W, x, y, M, N, K = args
+    rc = lwq.lib().lwq_matmul(fmt, W, x, y, M, N, K, None)
+    assert rc == status, (rc, lwq.lwq_status_string(rc))
+
+
+def test_status_strings():
+    for s in range(8):
+        assert lwq.lwq_status_string(s)
+    assert "unknown" in lwq.lwq_status_string(99)
+
+
+@pytest.mark.parametrize("w,a", [("q4_0", "f32"), ("q8_0", "f32"), ("q4_k", "f16"), ("q4_0", "bf16"),
+                                 ("q8_0", "f16"), ("q4_k", "bf16")])
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (8, 11008, 4096), (1, 4096, 11008), (16, 32000, 4096),
+                                   (4, 4096, 14336), (1, 5, 256), (3, 70, 512), (16, 4096, 14336)])
+def test_config_table(w, a, M, N, K):
+    fmt = lwq.fmt_code(w, a)
+    cfg = lwq.lwq_select_config(fmt, M, N, K).as_dict()
+    assert cfg["path"] in (1, 2, 3)
+    if cfg["path"] == 1:
+        assert 1 <= cfg["warps"] <= 16 and cfg["stages"] >= 2 and cfg["splits"] >= 1
+        nchunks = K // 256
+        cps = -(-nchunks // cfg["splits"])
+        assert cps <= cfg["warps"]            # every chunk of a split has a compute warp
+        assert cfg["ctas"] % cfg["splits"] == 0
+        ws = lwq.lwq_workspace_size(fmt, M, N, K)
+        assert ws >= 256
+        if cfg["splits"] > 1:
+            m_group = min(M, 8 if a == "f32" else 16)   # activation rows per GEMV pass
+            assert ws >= cfg["splits"] * m_group * N * 4
+    if w == "q4_k" and a != "f16":
+        assert cfg["path"] != 1
+
+
+def test_workspace_size_monotone():
+    fmt = lwq.fmt_code("q4_k", "f16")
+    a = lwq.lwq_workspace_size(fmt, 1, 4096, 11008)
+    b = lwq.lwq_workspace_size(fmt, 16, 11008, 14336)
+    assert 0 < a <= b
+    assert lwq.lwq_workspace_size(fmt, 0, 1, 256) == 0
+    assert lwq.lwq_workspace_size(fmt, 1, 1, 100) == 0

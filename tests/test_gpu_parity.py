@@ -1,0 +1,176 @@
+"""GPU path vs the CPU oracle, element by element, on the same seeded inputs.
+
+Small cases span several row tiles, K chunks and split-K slices and end in
+ragged tails; the full workload sizes are checked on sampled outputs (plus
+every tile edge) in the configuration the benchmark times.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import block_quantized_matmul_lwq_b200 as lwq
+import oracle
+from block_quantized_matmul_lwq_b200 import inputs
+from gpu_util import TOL_GEMV, check_full, check_sampled, run_gpu, to_device
+
+pytestmark = pytest.mark.gpu
+
+WS_BYTES = 256 << 20
+
+
+@pytest.fixture(scope="module")
+def dev():
+    d = torch.device("cuda:0")
+    torch.cuda.set_device(d)
+    ws = torch.zeros(WS_BYTES, dtype=torch.uint8, device=d)
+    lwq.lwq_init(ws, WS_BYTES)
+    yield d
+    torch.cuda.synchronize(d)
+    assert lwq.lwq_get_device_error() == lwq.LWQ_OK
+    lwq.lwq_shutdown()
+    del ws
+
+
+FAST = [("q4_0", "f32"), ("q4_0", "f16"), ("q4_0", "bf16"), ("q8_0", "f32"), ("q8_0", "f16"), ("q8_0", "bf16"),
+        ("q4_k", "f16")]
+SIMPLE_ONLY = [("q4_k", "f32"), ("q4_k", "bf16")]
+
+
+@pytest.mark.parametrize("w,a", FAST + SIMPLE_ONLY)
+@pytest.mark.parametrize("M,N,K", [(1, 1, 256), (1, 37, 512), (3, 100, 1024), (8, 333, 4096), (5, 61, 2816),
+                                   (16, 50, 768), (12, 130, 4352), (1, 17, 6144)])
+def test_small_shapes(dev, w, a, M, N, K):
+    check_full(w, a, M, N, K, dev, seed=M * 1000 + N)
+
+
+@pytest.mark.parametrize("w,a", [("q4_0", "f32"), ("q8_0", "f16"), ("q4_0", "bf16")])
+@pytest.mark.parametrize("M,N,K", [(1, 9, 32), (2, 40, 96), (4, 7, 320), (17, 33, 480)])
+def test_k_not_multiple_of_256(dev, w, a, M, N, K):
+    check_full(w, a, M, N, K, dev, seed=7)
+
+
+@pytest.mark.parametrize("w,a", FAST)
+@pytest.mark.parametrize("M", [20, 33])
+def test_many_activation_rows(dev, w, a, M):
+    check_full(w, a, M, 70, 1024, dev, seed=M)
+
+
+@pytest.mark.parametrize("w,a", FAST)
+@pytest.mark.parametrize("warps,splits,stages", [(1, 0, 2), (2, 0, 3), (4, 3, 2), (8, 2, 4), (3, 4, 2)])
+def test_forced_gemv_configs(dev, w, a, warps, splits, stages):
+    cfg = lwq.lwq_config()
+    cfg.path, cfg.warps, cfg.splits, cfg.stages = 1, warps, splits, stages
+    M, N, K = 5, 211, 3072
+    nchunks = K // 256
+    S = splits or -(-nchunks // warps)
+    if -(-nchunks // S) > warps:
+        pytest.skip("configuration leaves a chunk without a warp")
+    check_full(w, a, M, N, K, dev, seed=11, cfg=cfg)
+
+
+@pytest.mark.parametrize("w,a,M", [("q4_0", "f32", 1), ("q4_k", "f16", 1), ("q8_0", "f16", 16)])
+def test_split_k_deterministic(dev, w, a, M):
+    """Repeated calls (split-K with arrival counters) give bitwise identical results."""
+    N, K = 300, 11008
+    Wq, x = inputs.make_problem(w, a, M, N, K, seed=3)
+    assert lwq.lwq_select_config(lwq.fmt_code(w, a), M, N, K).splits > 1
+    ys = [run_gpu(w, a, Wq, x, M, N, K, dev).cpu().numpy() for _ in range(3)]
+    assert np.array_equal(ys[0], ys[1]) and np.array_equal(ys[1], ys[2])
+    y_ref, den = oracle.matmul(w, Wq, x, act=a)
+    assert oracle.normalised_error(ys[0], y_ref, den) <= TOL_GEMV
+
+
+# ----------------------------------------------------------- full workloads
+
+def test_q8_0_gemv_4096x4096(dev):
+    """Q8_0 decode GEMV, M=1, K=N=4096, fp32 activations, seed 0 -- every output."""
+    check_full("q8_0", "f32", 1, 4096, 4096, dev, seed=0)
+
+
+@pytest.mark.parametrize("M", [1, 4, 8])
+def test_q4_0_gemv_11008x4096(dev, M):
+    """Q4_0 decode GEMV, M in {1,4,8}, N=11008, K=4096, fp32 activations -- every output."""
+    check_full("q4_0", "f32", M, 11008, 4096, dev, seed=0)
+
+
+def test_q4_k_7b_layer_decode(dev):
+    """Q4_K decode over the seven projections of a 7B layer, fp16 activations -- every output."""
+    spec = inputs.WORKLOADS["q4_k_7b_layer_decode"]
+    for (N, K), seed in zip(spec["shapes"], spec["seeds"]):
+        check_full("q4_k", "f16", 1, N, K, dev, seed=seed)
+
+
+@pytest.mark.parametrize("M,N,K", [(512, 11008, 4096), (2048, 4096, 11008)])
+def test_q4_0_prefill_gemm(dev, M, N, K):
+    """Q4_0 prefill GEMM, bf16 activations -- sampled outputs plus every tile edge."""
+    check_sampled("q4_0", "bf16", M, N, K, dev, seed=0, count=1500)
+
+
+@pytest.mark.parametrize("w", ["q8_0", "q4_0", "q4_k"])
+@pytest.mark.parametrize("M", [1, 16, 64])
+@pytest.mark.parametrize("K,N", [(4096, 32000), (14336, 4096)])
+def test_sweep_points_sampled(dev, w, M, K, N):
+    check_sampled(w, "f16", M, N, K, dev, seed=M + K, count=600)
+
+
+# ------------------------------------------------------------ error paths
+
+def test_misaligned_pointers(dev):
+    fmt = lwq.fmt_code("q4_0", "f32")
+    W = torch.zeros(64 * 2304 + 16, dtype=torch.uint8, device=dev)
+    x = torch.zeros(4096 + 4, dtype=torch.float32, device=dev)
+    y = torch.zeros(64 + 4, dtype=torch.float32, device=dev)
+    rc = lwq.lib().lwq_matmul(fmt, W.data_ptr() + 1, x.data_ptr(), y.data_ptr(), 1, 64, 4096, None)
+    assert rc == 3
+    rc = lwq.lib().lwq_matmul(fmt, W.data_ptr(), x.data_ptr() + 4, y.data_ptr(), 1, 64, 4096, None)
+    assert rc == 3
+
+
+def test_workspace_errors(dev):
+    """A split-K call needs the workspace: missing -> NOT_INITIALIZED, small -> TOO_SMALL."""
+    w, a, M, N, K = "q4_k", "f16", 1, 256, 11008
+    fmt = lwq.fmt_code(w, a)
+    assert lwq.lwq_select_config(fmt, M, N, K).splits > 1
+    Wq, x = inputs.make_problem(w, a, M, N, K, seed=1)
+    Wd, xd = to_device(Wq, dev), to_device(x, dev)
+    y = torch.zeros((M, N), dtype=torch.float32, device=dev)
+    lwq.lwq_shutdown()
+    try:
+        assert lwq.lib().lwq_matmul(fmt, Wd.data_ptr(), xd.data_ptr(), y.data_ptr(), M, N, K, None) == 4
+        small = torch.zeros(256, dtype=torch.uint8, device=dev)
+        lwq.lwq_init(small, 256)
+        assert lwq.lib().lwq_matmul(fmt, Wd.data_ptr(), xd.data_ptr(), y.data_ptr(), M, N, K, None) == 5
+    finally:
+        ws = torch.zeros(WS_BYTES, dtype=torch.uint8, device=dev)
+        lwq.lwq_init(ws, WS_BYTES)
+        dev_ws_keepalive.append(ws)
+
+
+dev_ws_keepalive = []
+
+
+def test_bounded_wait_reports_timeout(dev):
+    """A wait on an mbarrier that nothing arrives at ends after its bound and reports."""
+    torch.cuda.synchronize(dev)
+    assert lwq.lwq_get_device_error() == lwq.LWQ_OK
+    lwq.lwq_selftest_timeout(2000)
+    torch.cuda.synchronize(dev)
+    assert lwq.lwq_get_device_error() == lwq.LWQ_ERR_DEVICE_TIMEOUT
+    assert lwq.lwq_get_device_error() == lwq.LWQ_OK
+    # the context is still usable
+    check_full("q4_0", "f32", 1, 64, 512, dev, seed=5)
+
+
+def test_stream_argument(dev):
+    """Calls honour the caller's stream."""
+    w, a, M, N, K = "q4_0", "f16", 2, 500, 4096
+    Wq, x = inputs.make_problem(w, a, M, N, K, seed=9)
+    Wd, xd = to_device(Wq, dev), to_device(x, dev)
+    y = torch.zeros((M, N), dtype=torch.float32, device=dev)
+    s = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(s):
+        lwq.lwq_matmul(lwq.fmt_code(w, a), Wd, xd, y, M, N, K, stream=s)
+    s.synchronize()
+    y_ref, den = oracle.matmul(w, Wq, x, act=a)
+    assert oracle.normalised_error(y.cpu().numpy(), y_ref, den) <= TOL_GEMV
