@@ -31,7 +31,7 @@ ACT_DTYPES = {"f32": LWQ_ACT_F32, "f16": LWQ_ACT_F16, "bf16": LWQ_ACT_BF16}
 # every symbol the header declares
 EXPORTS = ["lwq_row_bytes", "lwq_workspace_size", "lwq_init", "lwq_shutdown", "lwq_matmul",
            "lwq_select_config", "lwq_matmul_config", "lwq_status_string", "lwq_get_device_error",
-           "lwq_selftest_timeout", "lwq_last_launch_count", "lwq_version"]
+           "lwq_selftest_timeout", "lwq_last_launch_count", "lwq_version", "lwq_matmul_noalloc"]
 
 
 class LwqError(RuntimeError):
@@ -70,6 +70,7 @@ def _load() -> ctypes.CDLL:
     lib.lwq_selftest_timeout.restype, lib.lwq_selftest_timeout.argtypes = i, [c.c_uint, vp]
     lib.lwq_last_launch_count.restype, lib.lwq_last_launch_count.argtypes = i, []
     lib.lwq_version.restype, lib.lwq_version.argtypes = i, []
+    lib.lwq_matmul_noalloc.restype, lib.lwq_matmul_noalloc.argtypes = i, [i, vp, vp, vp, i, i, i, vp]
     return lib
 
 
@@ -168,3 +169,9 @@ def lwq_last_launch_count() -> int:
 
 def lwq_version() -> int:
     return _lib.lwq_version()
+
+
+def lwq_matmul_noalloc(fmt: int, Wq, x, y, M: int, N: int, K: int, stream=None) -> None:
+    """lwq_matmul for callers that cannot allocate: no workspace, static 4 MiB scratch (see include/lwq.h)."""
+    _check(_lib.lwq_matmul_noalloc(fmt, _ptr(Wq), _ptr(x), _ptr(y), M, N, K, _stream(stream)),
+           "lwq_matmul_noalloc")

@@ -1,0 +1,196 @@
+// lwq_matmul_noalloc: the decode GEMV for callers that cannot allocate device
+// memory.
+//
+// The regular entry point takes its split-K scratch from a workspace that the
+// caller allocates and registers with lwq_init.  Some callers cannot do that:
+// code running where the CUDA allocator may not be called (inside a custom
+// allocator's own callbacks, in a process whose memory pool is fixed and fully
+// handed out at start-up, or in a plugin that receives only input and output
+// pointers from its host).  This variant needs nothing from them but Wq, x
+// and y: its scratch is one static device array in this file, created when
+// the library is loaded on a device and held until the process exits.
+//
+// Limits and behaviour:
+//  * The scratch is kScratchBytes (4 MiB): 64 KiB of per-row-tile arrival
+//    counters and the rest for fp32 split-K partial sums.  A call whose
+//    configuration needs more (lwq_workspace_size(fmt, M, N, K) bytes) is
+//    rejected with LWQ_ERR_WORKSPACE_TOO_SMALL; so is a call with more row
+//    tiles than the counter region holds.
+//  * Only the tensor-core GEMV is offered (M <= 16 and the shapes it takes);
+//    other shapes return LWQ_ERR_UNSUPPORTED.
+//  * The device address of the array is looked up once per device, with that
+//    device current, on the first call made on it.  Make that first call
+//    before any stream capture on the device.
+//  * Every call shares the one array and it keeps the previous call's
+//    contents.  Each call clears the counters it uses (an asynchronous memset
+//    on the caller's stream) before its kernels run; partial sums are written
+//    before they are read.  Calls whose kernels overlap on the GPU (different
+//    streams without ordering between them) race on the array.
+//  * Nothing here calls cudaMalloc, cudaFree or any allocating routine.
+//  * A bounded wait that gives up in these kernels sets the device error word
+//    of this file's own module, which lwq_get_device_error does not read; the
+//    call's outputs are then not all written.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/lwq.h"
+#include "lwq_gemv.cuh"
+
+namespace lwq_noalloc {
+
+using namespace lwq;
+
+constexpr size_t kScratchBytes = 4u << 20;
+constexpr size_t kCounterBytes = 64u << 10;
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kTimeoutNs = 2000000000ull;
+
+static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
+
+struct DevSlot {
+    void *ptr = nullptr;
+    bool ready = false;
+};
+static DevSlot g_slots[kMaxDevices];
+static std::mutex g_mu;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encoder() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Device address of g_scratch on the current device (looked up once per device).
+static int scratch_ptr(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LWQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_slots[dev].ready) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return LWQ_ERR_CUDA;
+        g_slots[dev].ptr = p;
+        g_slots[dev].ready = true;
+    }
+    *out = g_slots[dev].ptr;
+    return LWQ_OK;
+}
+
+template <int FMT, int XT, int NT>
+static cudaError_t launch(const CUtensorMap &map, const GemvArgs &a, int ctas, int nw, size_t smem,
+                          cudaStream_t st) {
+    auto kern = gemv_tc_kernel<FMT, XT, NT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<ctas, (nw + 2) * 32, smem, st>>>(map, a);
+    return cudaGetLastError();
+}
+
+static cudaError_t dispatch(int wf, int xt, int nt, const CUtensorMap &map, const GemvArgs &a, int ctas, int nw,
+                            size_t smem, cudaStream_t st) {
+    if (wf == LWQ_Q4_0) {
+        if (xt == X_F32) return nt == 1 ? launch<F_Q4_0, X_F32, 1>(map, a, ctas, nw, smem, st) : cudaErrorInvalidValue;
+        if (xt == X_F16)
+            return nt == 1 ? launch<F_Q4_0, X_F16, 1>(map, a, ctas, nw, smem, st)
+                           : launch<F_Q4_0, X_F16, 2>(map, a, ctas, nw, smem, st);
+        return nt == 1 ? launch<F_Q4_0, X_BF16, 1>(map, a, ctas, nw, smem, st)
+                       : launch<F_Q4_0, X_BF16, 2>(map, a, ctas, nw, smem, st);
+    }
+    if (wf == LWQ_Q8_0) {
+        if (xt == X_F32) return nt == 1 ? launch<F_Q8_0, X_F32, 1>(map, a, ctas, nw, smem, st) : cudaErrorInvalidValue;
+        if (xt == X_F16)
+            return nt == 1 ? launch<F_Q8_0, X_F16, 1>(map, a, ctas, nw, smem, st)
+                           : launch<F_Q8_0, X_F16, 2>(map, a, ctas, nw, smem, st);
+        return nt == 1 ? launch<F_Q8_0, X_BF16, 1>(map, a, ctas, nw, smem, st)
+                       : launch<F_Q8_0, X_BF16, 2>(map, a, ctas, nw, smem, st);
+    }
+    if (wf == LWQ_Q4_K && xt == X_F16)
+        return nt == 1 ? launch<F_Q4_K, X_F16, 1>(map, a, ctas, nw, smem, st)
+                       : launch<F_Q4_K, X_F16, 2>(map, a, ctas, nw, smem, st);
+    return cudaErrorInvalidValue;
+}
+
+static size_t smem_bytes(int wf, int nw, int stages, int nt) {
+    const int cb = (wf == LWQ_Q8_0) ? 272 : 144;
+    return (size_t)stages * nw * GEMV_ROWS * cb + (size_t)stages * nw * GEMV_ROWS * 8 * nt * 4 +
+           (size_t)3 * stages * 8;
+}
+
+}  // namespace lwq_noalloc
+
+extern "C" int lwq_matmul_noalloc(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K,
+                                  void *stream) {
+    using namespace lwq_noalloc;
+    if (!Wq || !x || !y || M <= 0 || N <= 0 || K <= 0) return LWQ_ERR_INVALID_ARG;
+    if (((uintptr_t)Wq | (uintptr_t)x | (uintptr_t)y) & 15u) return LWQ_ERR_MISALIGNED;
+    lwq_config cfg;
+    int rc = lwq_select_config(fmt, M, N, K, &cfg);  // argument checks and the configuration table
+    if (rc) return rc;
+    if (cfg.path != 1 || M > 16) return LWQ_ERR_UNSUPPORTED;
+    const int wf = fmt & LWQ_FMT_MASK;
+    const int xt = (fmt & LWQ_ACT_MASK) == LWQ_ACT_F32 ? X_F32 : ((fmt & LWQ_ACT_MASK) == LWQ_ACT_F16 ? X_F16 : X_BF16);
+    const int m_group = (xt == X_F32) ? (M < 8 ? M : 8) : M;
+    const int S = cfg.splits;
+    const int row_tiles = (N + GEMV_ROWS - 1) / GEMV_ROWS;
+    if (S > 1) {
+        if ((size_t)row_tiles * 4 > kCounterBytes) return LWQ_ERR_WORKSPACE_TOO_SMALL;
+        if (kCounterBytes + (size_t)S * m_group * N * 4 > kScratchBytes) return LWQ_ERR_WORKSPACE_TOO_SMALL;
+    }
+    void *scratch = nullptr;
+    if ((rc = scratch_ptr(&scratch))) return rc;
+    EncodeTiledFn enc = encoder();
+    if (!enc) return LWQ_ERR_CUDA;
+    const long rb = (long)lwq_row_bytes(fmt, K);
+    CUtensorMap map;
+    {
+        const int cb = (wf == LWQ_Q8_0) ? 272 : 144;
+        cuuint64_t dims[2] = {(cuuint64_t)(rb / 2), (cuuint64_t)N};
+        cuuint64_t strides[1] = {(cuuint64_t)rb};
+        cuuint32_t box[2] = {(cuuint32_t)(cb / 2), (cuuint32_t)GEMV_ROWS};
+        cuuint32_t estr[2] = {1, 1};
+        if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(Wq), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return LWQ_ERR_CUDA;
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t xelem = (xt == X_F32) ? 4 : 2;
+    const int nchunks = K / 256;
+    const int cps = (nchunks + S - 1) / S;
+    for (int m0 = 0; m0 < M; m0 += m_group) {
+        const int mg = (M - m0) < m_group ? (M - m0) : m_group;
+        if (S > 1 && cudaMemsetAsync(scratch, 0, (size_t)row_tiles * 4, st) != cudaSuccess) return LWQ_ERR_CUDA;
+        GemvArgs a;
+        a.x = static_cast<const uint8_t *>(x) + (size_t)m0 * K * xelem;
+        a.y = y + (size_t)m0 * N;
+        a.counters = static_cast<unsigned *>(scratch);
+        a.partial = reinterpret_cast<float *>(static_cast<uint8_t *>(scratch) + kCounterBytes);
+        a.M = mg;
+        a.N = N;
+        a.K = K;
+        a.nchunks = nchunks;
+        a.splits = S;
+        a.chunks_per_split = cps;
+        a.row_tiles = row_tiles;
+        a.stages = cfg.stages;
+        a.timeout_ns = kTimeoutNs;
+        const int nt = mg <= 8 ? 1 : 2;
+        cudaError_t e = dispatch(wf, xt, nt, map, a, cfg.ctas, cfg.warps, smem_bytes(wf, cfg.warps, cfg.stages, nt), st);
+        if (e != cudaSuccess) return LWQ_ERR_CUDA;
+    }
+    return LWQ_OK;
+}

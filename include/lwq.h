@@ -116,6 +116,25 @@ int lwq_shutdown(void);
  */
 int lwq_matmul(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, void *stream);
 
+/* lwq_matmul for callers that cannot allocate device memory: code that may
+ * not call the CUDA allocator (an allocator's own callbacks, a process whose
+ * memory pool is fixed and fully handed out at start-up, a plugin given only
+ * input and output pointers).  It needs no workspace and no lwq_init: its
+ * split-K scratch is a static 4 MiB device array inside the library, held on
+ * every device that loads the library until the process exits.  The pages
+ * this library follows have no counterpart of this entry point.
+ *
+ * Arguments, layouts and results are those of lwq_matmul.  Only the decode
+ * GEMV is offered: M <= 16 and the shapes lwq_select_config sends to path 1,
+ * else LWQ_ERR_UNSUPPORTED.  A shape whose split-K scratch
+ * (lwq_workspace_size bytes) exceeds 4 MiB, or with more than 16384 row tiles
+ * of 16 weight rows when split, returns LWQ_ERR_WORKSPACE_TOO_SMALL.  The
+ * first call on a device looks up the array's device address (make it before
+ * any stream capture).  Calls share the array: each clears its counters on
+ * `stream` first, and calls whose kernels overlap on the GPU race.  Nothing
+ * is allocated or freed. */
+int lwq_matmul_noalloc(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, void *stream);
+
 /* ------------------------------------------------ configuration table
  * The per-shape configuration lwq_matmul would use, and a way to force one
  * (used by the sweep that fills the table and by tests). */
