@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_HERE, "liblwq.so")
 # codes (include/lwq.h)
 LWQ_Q8_0, LWQ_Q4_0, LWQ_Q4_K = 1, 2, 3
 LWQ_ACT_F32, LWQ_ACT_F16, LWQ_ACT_BF16 = 0x000, 0x100, 0x200
+LWQ_FLAG_OVERLAP = 0x1000   # weights constant: allow programmatic dependent launch
 LWQ_OK = 0
 LWQ_ERR_DEVICE_TIMEOUT = 7
 STATUS = {0: "LWQ_OK", 1: "LWQ_ERR_INVALID_ARG", 2: "LWQ_ERR_UNSUPPORTED", 3: "LWQ_ERR_MISALIGNED",

@@ -12,6 +12,7 @@
 #include <string.h>
 
 #include <mutex>
+#include <utility>
 
 #include "../../include/lwq.h"
 #include "lwq_gemm.cuh"
@@ -83,7 +84,7 @@ int act_code(int fmt) {
 
 int check_fmt_k(int fmt, long K) {
     const int wf = fmt & LWQ_FMT_MASK;
-    if (fmt & ~(LWQ_FMT_MASK | LWQ_ACT_MASK)) return LWQ_ERR_UNSUPPORTED;
+    if (fmt & ~(LWQ_FMT_MASK | LWQ_ACT_MASK | LWQ_FLAG_OVERLAP)) return LWQ_ERR_UNSUPPORTED;
     if (block_weights(wf) == 0 || act_code(fmt) < 0) return LWQ_ERR_UNSUPPORTED;
     if (K <= 0 || K % block_weights(wf)) return LWQ_ERR_INVALID_ARG;
     return LWQ_OK;
@@ -98,6 +99,7 @@ struct Plan {
     size_t ws_need;  // workspace bytes for one pass
 };
 
+// packed boxes + fp32 partials + full/empty/reduced mbarriers
 size_t gemv_smem(int wf, int nw, int stages, int nt) {
     const int cb = (wf == LWQ_Q8_0) ? 272 : 144;
     return (size_t)stages * nw * GEMV_ROWS * cb + (size_t)stages * nw * GEMV_ROWS * 8 * nt * 4 +
@@ -105,9 +107,9 @@ size_t gemv_smem(int wf, int nw, int stages, int nt) {
 }
 
 bool tc_gemv_eligible(int wf, int xt, long K) {
-    if (K % 256) return false;
-    if (wf == LWQ_Q4_K) return xt == X_F16;
-    return true;
+    (void)wf;
+    (void)xt;
+    return K % 256 == 0;
 }
 
 // Workspace layout: [kCounterBytes of per-row-tile arrival counters][fp32
@@ -190,6 +192,27 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
 }
 
 // --------------------------------------------------------------- launches
+// Launch on `st`; with `overlap`, as a programmatic dependent launch, so that
+// the kernel may start (and prefetch weights) before the preceding kernel on
+// the stream completes -- its other warps wait for that completion in-kernel.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), int ctas, int threads, size_t smem, cudaStream_t st, bool overlap,
+                     Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)ctas);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    if (overlap) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // Raise a kernel's dynamic shared-memory limit once per (device, kernel), so
 // that launches captured into CUDA graphs make no attribute calls.
 cudaError_t ensure_smem(const void *kern, size_t smem) {
@@ -212,39 +235,41 @@ cudaError_t ensure_smem(const void *kern, size_t smem) {
     return cudaSuccess;
 }
 
-template <int FMT, int XT, int NT>
+template <int FMT, int XT, int NT, bool ONE>
 cudaError_t launch_gemv_tc(const CUtensorMap &map, const GemvArgs &a, int ctas, int nw, size_t smem,
                            cudaStream_t st) {
-    auto kern = gemv_tc_kernel<FMT, XT, NT>;
+    auto kern = gemv_tc_kernel<FMT, XT, NT, ONE>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), smem);
     if (e != cudaSuccess) return e;
-    kern<<<ctas, (nw + 2) * 32, smem, st>>>(map, a);
-    return cudaGetLastError();
+    return launch_k(kern, ctas, (nw + 2) * 32, smem, st, a.overlap != 0, map, a);
 }
 
+// NT = n8 tiles of activation rows (2 only for 16-bit activations); the
+// one-row mapping serves passes with a single activation row (Q4_0, Q8_0).
 template <int FMT, int XT>
-cudaError_t launch_gemv_tc_nt(int nt, const CUtensorMap &map, const GemvArgs &a, int ctas, int nw, size_t smem,
-                              cudaStream_t st) {
-    if (nt == 1) return launch_gemv_tc<FMT, XT, 1>(map, a, ctas, nw, smem, st);
-    if constexpr (XT != X_F32) return launch_gemv_tc<FMT, XT, 2>(map, a, ctas, nw, smem, st);
+cudaError_t launch_gemv_tc_nt(int nt, bool one, const CUtensorMap &map, const GemvArgs &a, int ctas, int nw,
+                              size_t smem, cudaStream_t st) {
+    if (nt == 1) {
+        if constexpr (FMT != F_Q4_K)
+            if (one) return launch_gemv_tc<FMT, XT, 1, true>(map, a, ctas, nw, smem, st);
+        return launch_gemv_tc<FMT, XT, 1, false>(map, a, ctas, nw, smem, st);
+    }
+    if constexpr (XT != X_F32) return launch_gemv_tc<FMT, XT, 2, false>(map, a, ctas, nw, smem, st);
     return cudaErrorInvalidValue;
 }
 
-cudaError_t dispatch_gemv_tc(int wf, int xt, int nt, const CUtensorMap &map, const GemvArgs &a, int ctas, int nw,
-                             size_t smem, cudaStream_t st) {
+cudaError_t dispatch_gemv_tc(int wf, int xt, int nt, bool one, const CUtensorMap &map, const GemvArgs &a, int ctas,
+                             int nw, size_t smem, cudaStream_t st) {
+#define LWQ_TC(F)                                                                                      \
+    if (xt == X_F32) return launch_gemv_tc_nt<F, X_F32>(nt, one, map, a, ctas, nw, smem, st);         \
+    if (xt == X_F16) return launch_gemv_tc_nt<F, X_F16>(nt, one, map, a, ctas, nw, smem, st);         \
+    return launch_gemv_tc_nt<F, X_BF16>(nt, one, map, a, ctas, nw, smem, st);
     switch (wf) {
-    case LWQ_Q4_0:
-        if (xt == X_F32) return launch_gemv_tc_nt<F_Q4_0, X_F32>(nt, map, a, ctas, nw, smem, st);
-        if (xt == X_F16) return launch_gemv_tc_nt<F_Q4_0, X_F16>(nt, map, a, ctas, nw, smem, st);
-        return launch_gemv_tc_nt<F_Q4_0, X_BF16>(nt, map, a, ctas, nw, smem, st);
-    case LWQ_Q8_0:
-        if (xt == X_F32) return launch_gemv_tc_nt<F_Q8_0, X_F32>(nt, map, a, ctas, nw, smem, st);
-        if (xt == X_F16) return launch_gemv_tc_nt<F_Q8_0, X_F16>(nt, map, a, ctas, nw, smem, st);
-        return launch_gemv_tc_nt<F_Q8_0, X_BF16>(nt, map, a, ctas, nw, smem, st);
-    case LWQ_Q4_K:
-        if (xt == X_F16) return launch_gemv_tc_nt<F_Q4_K, X_F16>(nt, map, a, ctas, nw, smem, st);
-        return cudaErrorInvalidValue;
+    case LWQ_Q4_0: { LWQ_TC(F_Q4_0) }
+    case LWQ_Q8_0: { LWQ_TC(F_Q8_0) }
+    case LWQ_Q4_K: { LWQ_TC(F_Q4_K) }
     }
+#undef LWQ_TC
     return cudaErrorInvalidValue;
 }
 
@@ -285,33 +310,24 @@ int encode_weight_map(CUtensorMap *map, const void *Wq, int wf, int N, long rb) 
 }
 
 // ------------------------------------------------------------- prefill GEMM
-template <int FMT, int XT, int BN>
-cudaError_t launch_gemm_tc(const CUtensorMap &wm, const CUtensorMap &xm, const GemmArgs &a, int ctas,
-                           size_t smem, cudaStream_t st) {
-    auto kern = gemm_tc_kernel<FMT, XT, BN>;
+template <int FMT, int XT>
+cudaError_t launch_gemm_tc(const CUtensorMap &wm, const CUtensorMap &xm, const GemmArgs &a, int ctas, size_t smem,
+                           cudaStream_t st) {
+    auto kern = gemm_tc_kernel<FMT, XT>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), smem);
     if (e != cudaSuccess) return e;
-    kern<<<ctas, GEMM_THREADS, smem, st>>>(wm, xm, a);
-    return cudaGetLastError();
-}
-
-template <int FMT, int XT>
-cudaError_t launch_gemm_bn(int bn, const CUtensorMap &wm, const CUtensorMap &xm, const GemmArgs &a, int ctas,
-                           size_t smem, cudaStream_t st) {
-    if (bn == 64) return launch_gemm_tc<FMT, XT, 64>(wm, xm, a, ctas, smem, st);
-    if (bn == 128) return launch_gemm_tc<FMT, XT, 128>(wm, xm, a, ctas, smem, st);
-    return launch_gemm_tc<FMT, XT, 256>(wm, xm, a, ctas, smem, st);
+    return launch_k(kern, ctas, GEMM_THREADS, smem, st, a.overlap != 0, wm, xm, a);
 }
 
 template <int FMT>
-cudaError_t launch_gemm_xt(int xt, int bn, const CUtensorMap &wm, const CUtensorMap &xm, const GemmArgs &a,
-                           int ctas, size_t smem, cudaStream_t st) {
-    if (xt == X_F16) return launch_gemm_bn<FMT, X_F16>(bn, wm, xm, a, ctas, smem, st);
-    return launch_gemm_bn<FMT, X_BF16>(bn, wm, xm, a, ctas, smem, st);
+cudaError_t launch_gemm_xt(int xt, const CUtensorMap &wm, const CUtensorMap &xm, const GemmArgs &a, int ctas,
+                           size_t smem, cudaStream_t st) {
+    if (xt == X_F16) return launch_gemm_tc<FMT, X_F16>(wm, xm, a, ctas, smem, st);
+    return launch_gemm_tc<FMT, X_BF16>(wm, xm, a, ctas, smem, st);
 }
 
 int gemm_launch(int wf, int xt, const void *Wq, const void *x, float *y, int M, int N, int K, long rb,
-                const lwq_config &cfg, size_t smem, unsigned long long timeout_ns, cudaStream_t st) {
+                const lwq_config &cfg, size_t smem, unsigned long long timeout_ns, int overlap, cudaStream_t st) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return LWQ_ERR_CUDA;
     const int cb = gemm_chunk_bytes(wf);
@@ -345,14 +361,16 @@ int gemm_launch(int wf, int xt, const void *Wq, const void *x, float *y, int M, 
     a.nchunks = K / 256;
     a.n_wtiles = (N + GEMM_WROWS - 1) / GEMM_WROWS;
     a.n_ttiles = (M + bn - 1) / bn;
+    a.bn = bn;
     a.ab_stages = cfg.stages;
     a.p_stages = 2;
     a.timeout_ns = timeout_ns;
+    a.overlap = overlap;
     cudaError_t e;
     switch (wf) {
-    case LWQ_Q4_0: e = launch_gemm_xt<F_Q4_0>(xt, bn, wm, xm, a, cfg.ctas, smem, st); break;
-    case LWQ_Q8_0: e = launch_gemm_xt<F_Q8_0>(xt, bn, wm, xm, a, cfg.ctas, smem, st); break;
-    default: e = launch_gemm_xt<F_Q4_K>(xt, bn, wm, xm, a, cfg.ctas, smem, st); break;
+    case LWQ_Q4_0: e = launch_gemm_xt<F_Q4_0>(xt, wm, xm, a, cfg.ctas, smem, st); break;
+    case LWQ_Q8_0: e = launch_gemm_xt<F_Q8_0>(xt, wm, xm, a, cfg.ctas, smem, st); break;
+    default: e = launch_gemm_xt<F_Q4_K>(xt, wm, xm, a, cfg.ctas, smem, st); break;
     }
     return e == cudaSuccess ? LWQ_OK : LWQ_ERR_CUDA;
 }
@@ -368,6 +386,7 @@ int run(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, c
     int dev;
     if ((rc = current_device(&dev))) return rc;
     const int wf = fmt & LWQ_FMT_MASK, xt = act_code(fmt);
+    const int overlap = (fmt & LWQ_FLAG_OVERLAP) ? 1 : 0;
     Plan p;
     if ((rc = make_plan(fmt, M, N, K, force, sm_count(dev), &p))) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -376,7 +395,7 @@ int run(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, c
     int launches = 0;
 
     if (p.cfg.path == 2) {
-        rc = gemm_launch(wf, xt, Wq, x, y, M, N, K, rb, p.cfg, p.smem, kTimeoutNs, st);
+        rc = gemm_launch(wf, xt, Wq, x, y, M, N, K, rb, p.cfg, p.smem, kTimeoutNs, overlap, st);
         if (rc) return rc;
         t_last_launches = 1;
         return LWQ_OK;
@@ -422,8 +441,9 @@ int run(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, c
         a.row_tiles = row_tiles;
         a.stages = p.cfg.stages;
         a.timeout_ns = kTimeoutNs;
+        a.overlap = overlap;
         const int nt = mg <= 8 ? 1 : 2;
-        cudaError_t e = dispatch_gemv_tc(wf, xt, nt, map, a, p.cfg.ctas, p.cfg.warps,
+        cudaError_t e = dispatch_gemv_tc(wf, xt, nt, mg == 1, map, a, p.cfg.ctas, p.cfg.warps,
                                          gemv_smem(wf, p.cfg.warps, p.cfg.stages, nt), st);
         if (e != cudaSuccess) return LWQ_ERR_CUDA;
         ++launches;

@@ -11,10 +11,11 @@
 //   warp 0      TMA producer: packed weight chunks [128 rows][256 weights]
 //               and activation tiles [BN tokens][64 k] (128-byte swizzle)
 //   warp 1      TMEM allocator and single-thread UMMA issuer
-//   warps 2..9  dequantizers: packed chunk -> bf16/fp16 weight tile
+//   warps 2..17 dequantizers: packed chunk -> bf16/fp16 weight tile
 //               [128 rows][64 k] in the UMMA K-major 128-byte-swizzle layout
-//   warps 10-13 epilogue: TMEM -> registers -> y (fp32), coalesced along N
-// UMMA shape: M = 128 weight rows, N = BN tokens (64/128/256), K = 16;
+//   warps 18-21 epilogue: TMEM -> registers -> y (fp32), coalesced along N
+// UMMA shape: M = 128 weight rows, N = BN tokens (a multiple of 16 from 32
+// to 256, chosen per shape to balance the persistent grid's waves), K = 16;
 // accumulators double-buffered in TMEM so the epilogue of one tile overlaps
 // the main loop of the next.  Every wait is bounded (device error word).
 #pragma once
@@ -28,7 +29,7 @@ namespace lwq {
 constexpr int GEMM_WROWS = 128;       // weight rows per tile (UMMA M)
 constexpr int GEMM_BK = 64;           // k per k-block (one 128-byte swizzle atom of 16-bit values)
 constexpr int GEMM_KB_PER_CHUNK = 4;  // k-blocks per packed 256-weight chunk
-constexpr int GEMM_DQ_WARPS = 8;
+constexpr int GEMM_DQ_WARPS = 16;
 constexpr int GEMM_EPI_WARPS = 4;
 constexpr int GEMM_THREADS = (2 + GEMM_DQ_WARPS + GEMM_EPI_WARPS) * 32;
 
@@ -43,9 +44,11 @@ struct GemmArgs {
     int nchunks;      // K / 256
     int n_wtiles;     // ceil(N / 128)
     int n_ttiles;     // ceil(M / BN)
+    int bn;           // token tile (UMMA N)
     int ab_stages;
     int p_stages;
     unsigned long long timeout_ns;
+    int overlap;      // host side: launch with programmatic stream serialization
 };
 
 template <int FMT>
@@ -59,10 +62,14 @@ struct GemmFmt<F_Q4_K> { static constexpr int chunk_bytes = 144; };
 
 __host__ __device__ constexpr size_t gemm_a_bytes() { return (size_t)GEMM_WROWS * 128; }
 __host__ __device__ constexpr size_t gemm_b_bytes(int bn) { return (size_t)bn * 128; }
+// one A+B stage, rounded up to the 1024-byte alignment of 128-byte-swizzle atoms
+__host__ __device__ constexpr size_t gemm_ab_bytes(int bn) { return (gemm_a_bytes() + gemm_b_bytes(bn) + 1023) & ~(size_t)1023; }
+// TMEM columns for two fp32 accumulators of bn columns (a power of two >= 32)
+__host__ __device__ constexpr uint32_t gemm_tmem_cols(int bn) { return 2 * bn <= 128 ? 128u : (2 * bn <= 256 ? 256u : 512u); }
 
 // Shared memory: [ab stages x (A 16 KB | B bn*128 B)] [p stages x 128*CB] [barriers] [tmem addr]
 __host__ __device__ inline size_t gemm_smem_bytes(int cb, int bn, int ab_stages, int p_stages) {
-    size_t s = (size_t)ab_stages * (gemm_a_bytes() + gemm_b_bytes(bn));
+    size_t s = (size_t)ab_stages * gemm_ab_bytes(bn);
     s += (size_t)p_stages * GEMM_WROWS * cb;
     s = (s + 7) & ~(size_t)7;
     s += (size_t)(2 * ab_stages + 2 * p_stages + 4 + 1) * 8 + 16;
@@ -120,53 +127,53 @@ __device__ __forceinline__ void split_scale(float d, uint32_t &dh2, uint32_t &dl
 template <int FMT, int XT>
 struct Dequant;
 
-// Q4_0: k-block kb of a chunk = blocks 2kb (h=0) and 2kb+1 (h=1).
+// One dequant thread produces 16 weights of a k-block for one weight row r:
+// h selects the first or second 32 weights of the k-block's 64, v the 16-B
+// output chunks {2v, 2v+1} of those 32 (the chunk pairs are chosen so that a
+// thread's two chunks come from the same packed bytes).
+
+// Q4_0: k-block kb of a chunk = blocks 2kb (h=0) and 2kb+1 (h=1).  Block
+// bytes 8v..8v+7 hold elements 8v..8v+7 (low nibbles, output chunk v) and
+// 16+8v..16+8v+7 (high nibbles, output chunk 2+v).
 template <int XT>
 struct Dequant<F_Q4_0, XT> {
-    static __device__ __forceinline__ void run(const uint8_t *prow, int kb, int h, uint32_t a_row_base, int r) {
-        const uint32_t *w = reinterpret_cast<const uint32_t *>(prow) + 9 * kb + 4 * h;
-        uint32_t W[5];
-#pragma unroll
-        for (int i = 0; i < 5; ++i) W[i] = w[i];
+    static __device__ __forceinline__ void run(uint32_t prow, int kb, int h, int v, uint32_t a_base, int r) {
+        // block 2kb+h starts at byte 36kb + 18h; its nibbles at +2, so bytes 8v..8v+7 are at 36kb+18h+2+8v
+        const uint32_t w = prow + 4 * (9 * kb + 4 * h + 2 * v);   // word-aligned start (2 bytes early when h=0)
+        const uint32_t W0 = lds32(w), W1 = lds32(w + 4), W2 = lds32(w + 8);
         const uint32_t s = h ? 32u : 16u;
-        uint32_t q[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) q[i] = __funnelshift_rc(W[i], W[i + 1], s);
-        const float d = f16_bits_to_float(h ? (W[0] >> 16) : W[0]);
+        const uint32_t q0 = __funnelshift_rc(W0, W1, s), q1 = __funnelshift_rc(W1, W2, s);
+        const uint32_t dw = lds32(prow + 4 * (9 * kb + 4 * h));
+        const float d = f16_bits_to_float(h ? (dw >> 16) : dw);
         uint32_t dh2, dl2;
         split_scale<XT>(d, dh2, dl2);
-        // chunk c (0..3): elements 8c..8c+7 of the block
-        //   c=0: low nibbles of bytes 0-7, c=1: low of 8-15, c=2: high of 0-7, c=3: high of 8-15
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const uint32_t qa = q[(c & 1) * 2], qb = q[(c & 1) * 2 + 1];
-            const uint32_t sh = (c >> 1) * 4;
-            uint32_t o[4];
-            const uint32_t src[2] = {qa, qb};
-#pragma unroll
-            for (int p = 0; p < 2; ++p) {
-                const uint32_t v01 = prmt(src[p], 0u, 0x4140u) >> sh;  // bytes 0,1 -> halves
-                const uint32_t v23 = prmt(src[p], 0u, 0x4342u) >> sh;  // bytes 2,3 -> halves
-                o[2 * p] = scale_pair<XT>(q4_pair<XT>(v01), dh2, dl2);
-                o[2 * p + 1] = scale_pair<XT>(q4_pair<XT>(v23), dh2, dl2);
-            }
-            st_shared_v4(a_row_base + sw128_chunk_offset(r, 4 * h + c), o[0], o[1], o[2], o[3]);
-        }
+        // bytes (0,1), (2,3) of q0 and q1 as 16-bit halves, shared by the low and high chunks
+        const uint32_t p0 = prmt(q0, 0u, 0x4140u), p1 = prmt(q0, 0u, 0x4342u);
+        const uint32_t p2 = prmt(q1, 0u, 0x4140u), p3 = prmt(q1, 0u, 0x4342u);
+        st_shared_v4(a_base + sw128_chunk_offset(r, 4 * h + v),
+                     scale_pair<XT>(q4_pair<XT>(p0), dh2, dl2), scale_pair<XT>(q4_pair<XT>(p1), dh2, dl2),
+                     scale_pair<XT>(q4_pair<XT>(p2), dh2, dl2), scale_pair<XT>(q4_pair<XT>(p3), dh2, dl2));
+        st_shared_v4(a_base + sw128_chunk_offset(r, 4 * h + 2 + v),
+                     scale_pair<XT>(q4_pair<XT>(p0 >> 4), dh2, dl2), scale_pair<XT>(q4_pair<XT>(p1 >> 4), dh2, dl2),
+                     scale_pair<XT>(q4_pair<XT>(p2 >> 4), dh2, dl2), scale_pair<XT>(q4_pair<XT>(p3 >> 4), dh2, dl2));
     }
 };
 
-// Q8_0: k-block kb = blocks 2kb (h=0) and 2kb+1 (h=1); 34-byte blocks.
+// Q8_0: k-block kb = blocks 2kb (h=0) and 2kb+1 (h=1); codes 16v..16v+15
+// of the block become output chunks 4h+2v and 4h+2v+1.
 template <int XT>
 struct Dequant<F_Q8_0, XT> {
-    static __device__ __forceinline__ void run(const uint8_t *prow, int kb, int h, uint32_t a_row_base, int r) {
-        const uint32_t *w = reinterpret_cast<const uint32_t *>(prow) + 17 * kb + 8 * h;
-        uint32_t W[9];
+    static __device__ __forceinline__ void run(uint32_t prow, int kb, int h, int v, uint32_t a_base, int r) {
+        // block 2kb+h starts at byte 68kb + 34h; its codes at +2
+        const uint32_t w = prow + 4 * (17 * kb + 8 * h + 4 * v);
+        uint32_t W[5];
 #pragma unroll
-        for (int i = 0; i < 9; ++i) W[i] = w[i];
+        for (int i = 0; i < 5; ++i) W[i] = lds32(w + 4 * i);
         const uint32_t s = h ? 32u : 16u;
-        const float d = f16_bits_to_float(h ? (W[0] >> 16) : W[0]);
+        const uint32_t dw = lds32(prow + 4 * (17 * kb + 8 * h));
+        const float d = f16_bits_to_float(h ? (dw >> 16) : dw);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
             const uint32_t q0 = __funnelshift_rc(W[2 * c], W[2 * c + 1], s) ^ 0x80808080u;
             const uint32_t q1 = __funnelshift_rc(W[2 * c + 1], W[2 * c + 2], s) ^ 0x80808080u;
             uint32_t o[4];
@@ -190,19 +197,19 @@ struct Dequant<F_Q8_0, XT> {
                 o[2] = pack_bf16x2(f[4], f[5]);
                 o[3] = pack_bf16x2(f[6], f[7]);
             }
-            st_shared_v4(a_row_base + sw128_chunk_offset(r, 4 * h + c), o[0], o[1], o[2], o[3]);
+            st_shared_v4(a_base + sw128_chunk_offset(r, 4 * h + 2 * v + c), o[0], o[1], o[2], o[3]);
         }
     }
 };
 
 // Q4_K: chunk = one superblock; k-block kb = nibble group kb: h=0 sub-block
-// 2kb (low nibbles), h=1 sub-block 2kb+1 (high nibbles).
+// 2kb (low nibbles), h=1 sub-block 2kb+1 (high nibbles); elements 16v..16v+15
+// of the sub-block (bytes 32kb+16v..+15) become output chunks 4h+2v, 4h+2v+1.
 template <int XT>
 struct Dequant<F_Q4_K, XT> {
-    static __device__ __forceinline__ void run(const uint8_t *prow, int kb, int h, uint32_t a_row_base, int r) {
-        const uint4 hd = *reinterpret_cast<const uint4 *>(prow);
-        const uint4 qa = *reinterpret_cast<const uint4 *>(prow + 16 + 32 * kb);
-        const uint4 qb = *reinterpret_cast<const uint4 *>(prow + 32 + 32 * kb);
+    static __device__ __forceinline__ void run(uint32_t prow, int kb, int h, int v, uint32_t a_base, int r) {
+        const uint4 hd = lds128(prow);
+        const uint4 qv = lds128(prow + 16 + 32 * kb + 16 * v);
         const int j = 2 * kb + h;
         const uint32_t s0 = hd.y, s1 = hd.z, s2 = hd.w;
         uint32_t scw, mw;
@@ -216,10 +223,10 @@ struct Dequant<F_Q4_K, XT> {
         const int sc = (scw >> (8 * (j & 3))) & 63, m = (mw >> (8 * (j & 3))) & 63;
         const float ds = f16_bits_to_float(hd.x) * (float)sc;           // exact in fp32
         const float dm = f16_bits_to_float(hd.x >> 16) * (float)m;      // exact in fp32
-        const uint32_t qw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
         const uint32_t sh = 4u * h;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
             float f[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -230,23 +237,24 @@ struct Dequant<F_Q4_K, XT> {
 #pragma unroll
             for (int p = 0; p < 4; ++p)
                 o[p] = (XT == X_F16) ? pack_f16x2(f[2 * p], f[2 * p + 1]) : pack_bf16x2(f[2 * p], f[2 * p + 1]);
-            st_shared_v4(a_row_base + sw128_chunk_offset(r, 4 * h + c), o[0], o[1], o[2], o[3]);
+            st_shared_v4(a_base + sw128_chunk_offset(r, 4 * h + 2 * v + c), o[0], o[1], o[2], o[3]);
         }
     }
 };
 
 // -------------------------------------------------------------------- kernel
-template <int FMT, int XT, int BN>
+template <int FMT, int XT>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap,
                    const GemmArgs a) {
     constexpr int CB = GemmFmt<FMT>::chunk_bytes;
     constexpr uint32_t A_BYTES = (uint32_t)gemm_a_bytes();
-    constexpr uint32_t B_BYTES = (uint32_t)gemm_b_bytes(BN);
-    constexpr uint32_t AB_BYTES = A_BYTES + B_BYTES;
+    const int BN = a.bn;
+    const uint32_t B_BYTES = (uint32_t)gemm_b_bytes(BN);
+    const uint32_t AB_BYTES = (uint32_t)gemm_ab_bytes(BN);
     constexpr uint32_t P_BYTES = (uint32_t)GEMM_WROWS * CB;
-    constexpr uint32_t TMEM_COLS = 2 * BN;
-    constexpr uint32_t IDESC = umma_idesc_f16(XT == X_F16 ? 0 : 1, GEMM_WROWS, BN);
+    const uint32_t TMEM_COLS = gemm_tmem_cols(BN);
+    const uint32_t IDESC = umma_idesc_f16(XT == X_F16 ? 0 : 1, GEMM_WROWS, BN);
 
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned base (128-byte swizzle atoms)
@@ -281,6 +289,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
         mbar_init(mma_done, 1);
         fence_mbar_init();
+        pdl_launch_dependents();
     }
     if (warp == 1) {
         tmem_alloc(tmem_holder, TMEM_COLS);
@@ -297,7 +306,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             tma_prefetch_desc(&wmap);
             tma_prefetch_desc(&xmap);
             int kbi = 0, ci = 0;
-            bool ok = true;
+            bool ok = true, waited = false;
             for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
                 const int tt = tile % a.n_ttiles, wt = tile / a.n_ttiles;
                 for (int c = 0; ok && c < a.nchunks; ++c, ++ci) {
@@ -306,6 +315,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         break;
                     mbar_arrive_expect_tx(&p_full[ps], P_BYTES);
                     tma_load_2d(pk + (size_t)ps * P_BYTES, &wmap, &p_full[ps], c * (CB / 2), wt * GEMM_WROWS);
+                    if (!waited) {   // x may be the preceding kernel's output
+                        pdl_wait();
+                        waited = true;
+                    }
                     for (int kb = 0; kb < GEMM_KB_PER_CHUNK; ++kb, ++kbi) {
                         const int s = kbi % S;
                         if (kbi >= S &&
@@ -333,7 +346,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 if (ti >= 2 && !(ok = mbar_wait(&acc_empty[as], ((ti >> 1) - 1) & 1, a.timeout_ns, DEVERR_GEMM_WAIT)))
                     break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(as * BN);
+                const uint32_t d_tmem = tmem_base + (uint32_t)as * (TMEM_COLS / 2);
                 for (int k = 0; k < kblocks; ++k, ++kbi) {
                     const int s = kbi % S;
                     if (!(ok = mbar_wait(&ab_full[s], (kbi / S) & 1, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
@@ -355,22 +368,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
     } else if (warp < 2 + GEMM_DQ_WARPS) {
         // ------------------------------------------------------ dequantizers
-        const int t = threadIdx.x - 64;          // 0..255
+        const int t = threadIdx.x - 64;          // 0..511
         const int r = t & (GEMM_WROWS - 1);      // weight row within the tile
-        const int h = t >> 7;                    // which 32 of the k-block's 64 weights
+        const int h = (t >> 7) & 1;              // which 32 of the k-block's 64 weights
+        const int v = t >> 8;                    // which 16 of those 32
         int kbi = 0, ci = 0;
         bool ok = true;
         for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
             for (int c = 0; ok && c < a.nchunks; ++c, ++ci) {
                 const int ps = ci % P;
                 if (!(ok = mbar_wait(&p_full[ps], (ci / P) & 1, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
-                const uint8_t *prow = pk + (size_t)ps * P_BYTES + (size_t)r * CB;
+                const uint32_t prow = smem_u32(pk) + (uint32_t)(ps * P_BYTES + r * CB);
                 for (int kb = 0; kb < GEMM_KB_PER_CHUNK; ++kb, ++kbi) {
                     const int s = kbi % S;
                     if (kbi >= S &&
                         !(ok = mbar_wait(&ab_empty[s], ((kbi / S) - 1) & 1, a.timeout_ns, DEVERR_GEMM_WAIT)))
                         break;
-                    Dequant<FMT, XT>::run(prow, kb, h, smem_u32(ab + (size_t)s * AB_BYTES), r);
+                    Dequant<FMT, XT>::run(prow, kb, h, v, smem_u32(ab + (size_t)s * AB_BYTES), r);
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&ab_full[s]);
@@ -381,6 +395,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
     } else {
         // --------------------------------------------------------- epilogue
+        pdl_wait();              // y only after the preceding work completed
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const int N = a.N, M = a.M;
         int ti = 0;
@@ -390,17 +405,24 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             if (!mbar_wait(&acc_full[as], (ti >> 1) & 1, a.timeout_ns, DEVERR_GEMM_WAIT)) break;
             tc_fence_after();
             const int n = wt * GEMM_WROWS + q * 32 + lane;
-            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(as * BN);
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)as * (TMEM_COLS / 2);
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 uint32_t v[32];
-                tmem_ld_32x32b_x32(taddr + c0, v);
+                if (BN - c0 >= 32) {
+                    tmem_ld_32x32b_x32(taddr + c0, v);
+                } else {
+                    tmem_ld_32x32b_x16(taddr + c0, *reinterpret_cast<uint32_t(*)[16]>(v));
+#pragma unroll
+                    for (int j = 16; j < 32; ++j) v[j] = 0u;
+                }
                 tmem_wait_ld();
                 const int m0 = tt * BN + c0;
+                const int mcols = min(32, BN - c0);
                 if (n < N) {
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        if (m0 + j < M) a.y[(size_t)(m0 + j) * N + n] = __uint_as_float(v[j]);
+                        if (j < mcols && m0 + j < M) a.y[(size_t)(m0 + j) * N + n] = __uint_as_float(v[j]);
                 }
             }
             tc_fence_before();
@@ -428,15 +450,32 @@ inline int gemm_chunk_bytes(int wf) { return wf == LWQ_Q8_0 ? 272 : 144; }
 inline int gemm_plan(int wf, int xt, int M, int N, int K, const lwq_config *force, int sms, GemmPlan *g) {
     (void)xt;
     (void)K;
-    int bn = force && force->tile_m ? force->tile_m : (M <= 64 ? 64 : (M <= 128 ? 128 : 256));
-    if (bn != 64 && bn != 128 && bn != 256) return LWQ_ERR_UNSUPPORTED;
+    const int n_wtiles = (N + GEMM_WROWS - 1) / GEMM_WROWS;
+    int bn = force && force->tile_m ? force->tile_m : 0;
+    if (!bn) {
+        // token tile: the persistent grid runs ceil(tiles / sms) rounds of BN-wide tiles; pick the multiple of 16
+        // that minimizes rounds * (BN + 48) (the constant stands for a tile's decode and pipeline fill overhead),
+        // preferring larger tiles on ties
+        long best = -1;
+        const int hi = M < 256 ? ((M + 15) / 16) * 16 : 256;
+        for (int c = hi; c >= 32; c -= 16) {
+            const long tiles = (long)n_wtiles * ((M + c - 1) / c);
+            const long rounds = (tiles + sms - 1) / sms;
+            const long cost = rounds * (c + 48);
+            if (best < 0 || cost < best) {
+                best = cost;
+                bn = c;
+            }
+        }
+    }
+    if (bn < 32 || bn > 256 || bn % 16) return LWQ_ERR_UNSUPPORTED;
     const int cb = gemm_chunk_bytes(wf);
     int p_stages = 2;
     int ab = force && force->stages ? force->stages : 4;
     const size_t limit = 232448;
     while (ab > 2 && gemm_smem_bytes(cb, bn, ab, p_stages) > limit) --ab;
     if (gemm_smem_bytes(cb, bn, ab, p_stages) > limit) return LWQ_ERR_UNSUPPORTED;
-    const int tiles = ((N + GEMM_WROWS - 1) / GEMM_WROWS) * ((M + bn - 1) / bn);
+    const int tiles = n_wtiles * ((M + bn - 1) / bn);
     int ctas = force && force->ctas ? force->ctas : sms;
     if (ctas > tiles) ctas = tiles;
     if (ctas < 1) ctas = 1;

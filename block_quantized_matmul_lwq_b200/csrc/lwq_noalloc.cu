@@ -90,37 +90,40 @@ static int scratch_ptr(void **out) {
     return LWQ_OK;
 }
 
-template <int FMT, int XT, int NT>
+template <int FMT, int XT, int NT, bool ONE>
 static cudaError_t launch(const CUtensorMap &map, const GemvArgs &a, int ctas, int nw, size_t smem,
                           cudaStream_t st) {
-    auto kern = gemv_tc_kernel<FMT, XT, NT>;
+    auto kern = gemv_tc_kernel<FMT, XT, NT, ONE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<ctas, (nw + 2) * 32, smem, st>>>(map, a);
     return cudaGetLastError();
 }
 
-static cudaError_t dispatch(int wf, int xt, int nt, const CUtensorMap &map, const GemvArgs &a, int ctas, int nw,
-                            size_t smem, cudaStream_t st) {
-    if (wf == LWQ_Q4_0) {
-        if (xt == X_F32) return nt == 1 ? launch<F_Q4_0, X_F32, 1>(map, a, ctas, nw, smem, st) : cudaErrorInvalidValue;
-        if (xt == X_F16)
-            return nt == 1 ? launch<F_Q4_0, X_F16, 1>(map, a, ctas, nw, smem, st)
-                           : launch<F_Q4_0, X_F16, 2>(map, a, ctas, nw, smem, st);
-        return nt == 1 ? launch<F_Q4_0, X_BF16, 1>(map, a, ctas, nw, smem, st)
-                       : launch<F_Q4_0, X_BF16, 2>(map, a, ctas, nw, smem, st);
+template <int FMT, int XT>
+static cudaError_t launch_nt(int nt, bool one, const CUtensorMap &map, const GemvArgs &a, int ctas, int nw,
+                             size_t smem, cudaStream_t st) {
+    if (nt == 1) {
+        if constexpr (FMT != F_Q4_K)
+            if (one) return launch<FMT, XT, 1, true>(map, a, ctas, nw, smem, st);
+        return launch<FMT, XT, 1, false>(map, a, ctas, nw, smem, st);
     }
-    if (wf == LWQ_Q8_0) {
-        if (xt == X_F32) return nt == 1 ? launch<F_Q8_0, X_F32, 1>(map, a, ctas, nw, smem, st) : cudaErrorInvalidValue;
-        if (xt == X_F16)
-            return nt == 1 ? launch<F_Q8_0, X_F16, 1>(map, a, ctas, nw, smem, st)
-                           : launch<F_Q8_0, X_F16, 2>(map, a, ctas, nw, smem, st);
-        return nt == 1 ? launch<F_Q8_0, X_BF16, 1>(map, a, ctas, nw, smem, st)
-                       : launch<F_Q8_0, X_BF16, 2>(map, a, ctas, nw, smem, st);
+    if constexpr (XT != X_F32) return launch<FMT, XT, 2, false>(map, a, ctas, nw, smem, st);
+    return cudaErrorInvalidValue;
+}
+
+static cudaError_t dispatch(int wf, int xt, int nt, bool one, const CUtensorMap &map, const GemvArgs &a, int ctas,
+                            int nw, size_t smem, cudaStream_t st) {
+#define LWQ_NA(F)                                                                             \
+    if (xt == X_F32) return launch_nt<F, X_F32>(nt, one, map, a, ctas, nw, smem, st);        \
+    if (xt == X_F16) return launch_nt<F, X_F16>(nt, one, map, a, ctas, nw, smem, st);        \
+    return launch_nt<F, X_BF16>(nt, one, map, a, ctas, nw, smem, st);
+    switch (wf) {
+    case LWQ_Q4_0: { LWQ_NA(F_Q4_0) }
+    case LWQ_Q8_0: { LWQ_NA(F_Q8_0) }
+    case LWQ_Q4_K: { LWQ_NA(F_Q4_K) }
     }
-    if (wf == LWQ_Q4_K && xt == X_F16)
-        return nt == 1 ? launch<F_Q4_K, X_F16, 1>(map, a, ctas, nw, smem, st)
-                       : launch<F_Q4_K, X_F16, 2>(map, a, ctas, nw, smem, st);
+#undef LWQ_NA
     return cudaErrorInvalidValue;
 }
 
@@ -188,8 +191,9 @@ extern "C" int lwq_matmul_noalloc(int fmt, const void *Wq, const void *x, float 
         a.row_tiles = row_tiles;
         a.stages = cfg.stages;
         a.timeout_ns = kTimeoutNs;
+        a.overlap = 0;
         const int nt = mg <= 8 ? 1 : 2;
-        cudaError_t e = dispatch(wf, xt, nt, map, a, cfg.ctas, cfg.warps, smem_bytes(wf, cfg.warps, cfg.stages, nt), st);
+        cudaError_t e = dispatch(wf, xt, nt, mg == 1, map, a, cfg.ctas, cfg.warps, smem_bytes(wf, cfg.warps, cfg.stages, nt), st);
         if (e != cudaSuccess) return LWQ_ERR_CUDA;
     }
     return LWQ_OK;

@@ -67,6 +67,14 @@ typedef enum {
 #define LWQ_ACT_F16 0x100
 #define LWQ_ACT_BF16 0x200
 #define LWQ_ACT_MASK 0xF00
+/* Optional flag, or-ed into fmt: the caller promises that Wq is not written
+ * by any work still running on the stream when the call is made (weights are
+ * constant, as in a decode loop).  The call's kernels are then launched as
+ * programmatic dependent launches: they may start, and begin streaming Wq,
+ * before the preceding kernel on the stream has finished; they still wait for
+ * it to complete before reading x or writing y and the workspace.  This hides
+ * launch latency between back-to-back calls. */
+#define LWQ_FLAG_OVERLAP 0x1000
 
 /* Bytes of one packed row of K weights (K/32*34, K/32*18, K/256*144), or 0
  * when fmt is unknown or K is not a positive multiple of the block size. */

@@ -174,3 +174,33 @@ def test_stream_argument(dev):
     s.synchronize()
     y_ref, den = oracle.matmul(w, Wq, x, act=a)
     assert oracle.normalised_error(y.cpu().numpy(), y_ref, den) <= TOL_GEMV
+
+
+def test_overlap_flag_chains(dev):
+    """LWQ_FLAG_OVERLAP (programmatic dependent launch) gives bitwise the same results as plain
+    launches, for a chain where each call reads the previous call's output (read after write)
+    and later calls overwrite a buffer an earlier call read (write after read)."""
+    g = np.random.default_rng(17)
+    K = 4096
+    W1 = to_device(inputs.make_weights("q4_0", g, 4096, K), dev)
+    W2 = to_device(inputs.make_weights("q8_0", g, 4096, K), dev)
+    W3 = to_device(inputs.make_weights("q4_k", g, 2048, K), dev)
+    x0 = torch.from_numpy(inputs.activations(g, 4, K, "f32")).to(dev)
+
+    def chain(flag):
+        a = x0.clone()
+        b = torch.full((4, 4096), float("nan"), device=dev)
+        c = torch.full((4, 2048), float("nan"), device=dev)
+        lwq.lwq_matmul(lwq.fmt_code("q4_0", "f32") | flag, W1, a, b, 4, 4096, K)    # b = f(a)
+        lwq.lwq_matmul(lwq.fmt_code("q8_0", "f32") | flag, W2, b, a, 4, 4096, K)    # a = f(b): RAW on b, WAR on a
+        lwq.lwq_matmul(lwq.fmt_code("q4_k", "f32") | flag, W3, a, c, 4, 2048, K)    # c = f(a): RAW on a
+        lwq.lwq_matmul(lwq.fmt_code("q4_0", "f32") | flag, W1, a, b, 1, 4096, K)    # one-row kernel, RAW on a
+        torch.cuda.synchronize(dev)
+        return a.cpu().numpy(), b.cpu().numpy(), c.cpu().numpy()
+
+    plain = chain(0)
+    for _ in range(3):
+        over = chain(lwq.LWQ_FLAG_OVERLAP)
+        for p_, o_ in zip(plain, over):
+            assert np.array_equal(p_, o_)
+    assert all(np.all(np.isfinite(p_)) for p_ in plain)
