@@ -305,13 +305,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (lane == 0) {
             tma_prefetch_desc(&wmap);
             tma_prefetch_desc(&xmap);
-            int kbi = 0, ci = 0;
+            // ring positions (s, ps) and phase parities tracked incrementally
+            int kbi = 0, ci = 0, s = 0, ps = 0;
+            uint32_t ph = 0, pph = 0;
             bool ok = true, waited = false;
             for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
                 const int tt = tile % a.n_ttiles, wt = tile / a.n_ttiles;
                 for (int c = 0; ok && c < a.nchunks; ++c, ++ci) {
-                    const int ps = ci % P;
-                    if (ci >= P && !(ok = mbar_wait(&p_empty[ps], ((ci / P) - 1) & 1, a.timeout_ns, DEVERR_GEMM_WAIT)))
+                    if (ci >= P && !(ok = mbar_wait(&p_empty[ps], pph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT)))
                         break;
                     mbar_arrive_expect_tx(&p_full[ps], P_BYTES);
                     tma_load_2d(pk + (size_t)ps * P_BYTES, &wmap, &p_full[ps], c * (CB / 2), wt * GEMM_WROWS);
@@ -319,18 +320,24 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         pdl_wait();
                         waited = true;
                     }
+                    if (++ps == P) {
+                        ps = 0;
+                        pph ^= 1u;
+                    }
                     for (int kb = 0; kb < GEMM_KB_PER_CHUNK; ++kb, ++kbi) {
-                        const int s = kbi % S;
-                        if (kbi >= S &&
-                            !(ok = mbar_wait(&ab_empty[s], ((kbi / S) - 1) & 1, a.timeout_ns, DEVERR_GEMM_WAIT)))
+                        if (kbi >= S && !(ok = mbar_wait(&ab_empty[s], ph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT)))
                             break;
                         mbar_arrive_expect_tx(&ab_full[s], B_BYTES);
                         tma_load_2d(ab + (size_t)s * AB_BYTES + A_BYTES, &xmap, &ab_full[s],
                                     (c * GEMM_KB_PER_CHUNK + kb) * GEMM_BK, tt * BN);
+                        if (++s == S) {
+                            s = 0;
+                            ph ^= 1u;
+                        }
                     }
                 }
             }
-            // drain: the last loads land before the CTA may exit
+            // drain: the last loads land before the CTA may exit (runs once; divisions are fine here)
             for (int j = max(0, kbi - S); j < kbi; ++j)
                 mbar_wait(&ab_full[j % S], (j / S) & 1, a.timeout_ns, DEVERR_GEMM_WAIT);
             for (int j = max(0, ci - P); j < ci; ++j)
@@ -339,7 +346,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------- UMMA issuer
         if (lane == 0) {
-            int kbi = 0, ti = 0;
+            int ti = 0, s = 0;
+            uint32_t ph = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++ti) {
                 const int as = ti & 1;
@@ -347,9 +355,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)as * (TMEM_COLS / 2);
-                for (int k = 0; k < kblocks; ++k, ++kbi) {
-                    const int s = kbi % S;
-                    if (!(ok = mbar_wait(&ab_full[s], (kbi / S) & 1, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
+                for (int k = 0; k < kblocks; ++k) {
+                    if (!(ok = mbar_wait(&ab_full[s], ph, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(ab + (size_t)s * AB_BYTES);
                     const uint32_t b_addr = a_addr + A_BYTES;
@@ -358,6 +365,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         umma_f16(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32), IDESC,
                                  (k | kk) ? 1u : 0u);
                     umma_commit(&ab_empty[s]);
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
                 if (!ok) break;
                 umma_commit(&acc_full[as]);
@@ -372,25 +383,30 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         const int r = t & (GEMM_WROWS - 1);      // weight row within the tile
         const int h = (t >> 7) & 1;              // which 32 of the k-block's 64 weights
         const int v = t >> 8;                    // which 16 of those 32
-        int kbi = 0, ci = 0;
+        int kbi = 0, s = 0, ps = 0;
+        uint32_t ph = 0, pph = 0;
         bool ok = true;
         for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
-            for (int c = 0; ok && c < a.nchunks; ++c, ++ci) {
-                const int ps = ci % P;
-                if (!(ok = mbar_wait(&p_full[ps], (ci / P) & 1, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
+            for (int c = 0; ok && c < a.nchunks; ++c) {
+                if (!(ok = mbar_wait(&p_full[ps], pph, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
                 const uint32_t prow = smem_u32(pk) + (uint32_t)(ps * P_BYTES + r * CB);
                 for (int kb = 0; kb < GEMM_KB_PER_CHUNK; ++kb, ++kbi) {
-                    const int s = kbi % S;
-                    if (kbi >= S &&
-                        !(ok = mbar_wait(&ab_empty[s], ((kbi / S) - 1) & 1, a.timeout_ns, DEVERR_GEMM_WAIT)))
-                        break;
+                    if (kbi >= S && !(ok = mbar_wait(&ab_empty[s], ph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
                     Dequant<FMT, XT>::run(prow, kb, h, v, smem_u32(ab + (size_t)s * AB_BYTES), r);
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&ab_full[s]);
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&p_empty[ps]);
+                if (++ps == P) {
+                    ps = 0;
+                    pph ^= 1u;
+                }
             }
         }
     } else {

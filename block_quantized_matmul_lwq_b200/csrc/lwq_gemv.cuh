@@ -179,7 +179,7 @@ struct Q40 {
     uint32_t xf[NT][8][2][2][P];   // [nt][block][step][reg][part]
     float inv;
 
-    __device__ __forceinline__ void load_x(const void *x, int M, int K, long k0, int lane) {
+    __device__ __forceinline__ void load_x(const void *x, int M, int K, long k0, int lane, uint32_t, uint32_t) {
         const int g = lane >> 2, t = lane & 3;
         float mx = 0.f, s;
 #pragma unroll
@@ -258,137 +258,219 @@ struct Q40 {
 };
 
 // --------------------------------------------------- one activation row (M = 1)
-// Lane (g, t) owns blocks 2t and 2t+1 of the chunk for weight rows g and g+8.
-// k-step s (0..15) takes four weights of block 2t + s/8 from every lane t;
-// the B operand is block-diagonal: column c holds the activations of block c
-// in the k-slots of the lane that owns block c, zeros elsewhere.  So C[r][c]
-// is block c's partial dot product for row r, and lane (g, t) holds exactly
-// its own two blocks (columns 2t, 2t+1).  The activation registers of lane
-// (g, t) are non-zero only when g is 2t or 2t+1 (then they hold block g).
+// Lane (g, t) owns blocks 2t and 2t+1 of the chunk for weight rows g and g+8
+// and runs them one after the other, 8 k-steps each.  Every k-slot of lane t
+// holds a weight of its own block, so the B operand is block-diagonal: column
+// 2t+p carries part p of the activations of lane t's current block in lane
+// t's k-slots and zeros elsewhere (p = 0: the fp16 activation, or the hi half
+// of an fp32 one; p = 1: the lo half, zero for fp16/bf16 activations).  Then
+// C[r][2t+p] is part p of the block's dot product for row r, held by lane
+// (g, t) itself, and fp32 activations take no extra MMAs.
+//
+// Codes enter the MMA as fp16 subnormals: the bit pattern of an unsigned code
+// u is the fp16 value u * 2^-24 (exact, as is every product with an fp16
+// activation), so one LOP3 (Q4_0: a nibble of each half, the high nibble left
+// in place as 16u * 2^-24) or one PRMT (Q8_0: a byte of each half) makes two
+// weights with no arithmetic.  The codes' offset o (8 for Q4_0; 128 for Q8_0,
+// whose int8 codes are read as u = q + 128) is removed once per block:
+// sum (u - o) x = sum u x - o * sum x.
+//
+// Code words: lane t's two blocks span CB/16 words per row.  Block 2t starts
+// 2 bytes into the first word, so its codes are read as word 0 = (last two
+// code bytes, first two code bytes) and words 1.. as they lie; block 2t+1's
+// codes are word-aligned.  Byte b of code word j is code byte cb(hb, j) + b
+// for b = 0, 1 and cb2(hb, j) + b - 2 for b = 2, 3.
 template <int FMT, int XT>
 struct OneRow {
     static constexpr int P = XFrag<XT>::parts;
-    uint32_t xf[16][2][P];   // [k-step][reg][part]
+    static constexpr int NC = (FMT == F_Q4_0) ? 16 : 32;   // code bytes per block
+    static constexpr int NWB = NC / 4;                       // code words per block and row
+    static constexpr float OFFSET = (FMT == F_Q4_0) ? 8.f : 128.f;
+    uint32_t xb[2][8][2];   // [block 2t + hb][k-step][reg]: this lane's column of B
+    float corr[2];          // -OFFSET * (sum of the block's scaled activations)
     float inv;
 
-    __device__ __forceinline__ void load_x(const void *x, int M, int K, long k0, int lane) {
-        const int g = lane >> 2, t = lane & 3;
-        const int h = g - 2 * t;                  // which half of the k-steps this lane's B feeds
-        const bool own = (h == 0 || h == 1);
-        float4 v[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            // Q4_0: v[0..3] = elements 4i..4i+3 (low nibbles), v[4..7] = 16+4i.. (high)
-            // Q8_0: v[i] = elements 4i..4i+3
-            const int e = (FMT == F_Q4_0) ? ((i < 4) ? 4 * i : 16 + 4 * (i - 4)) : 4 * i;
-            v[i] = own ? load4<XT>(x, M, K, 0, k0, 32 * g + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+    __device__ static __forceinline__ int cb0(int hb, int j) { return hb ? 4 * j : (j ? 4 * j - 2 : NC - 2); }
+    __device__ static __forceinline__ int cb2(int hb, int j) { return hb ? 4 * j + 2 : 4 * j; }
+
+    // Element pairs (e, e+1) of activation row 0 as fp32.
+    __device__ static __forceinline__ float2 load2(const void *x, long k0, int e) {
+        if constexpr (XT == X_F32) {
+            return __ldg(reinterpret_cast<const float2 *>(static_cast<const float *>(x) + k0 + e));
+        } else {
+            const uint32_t u = __ldg(reinterpret_cast<const uint32_t *>(static_cast<const uint16_t *>(x) + k0 + e));
+            if constexpr (XT == X_F16)
+                return make_float2(f16_bits_to_float(u), f16_bits_to_float(u >> 16));
+            else
+                return make_float2(bf16_bits_to_float(u), bf16_bits_to_float(u >> 16));
         }
-        float mx = 0.f, s;
+    }
+
+    // Part p (0: hi, 1: lo) of the fp16 pair (a, b), a in the low half.
+    __device__ static __forceinline__ uint32_t part(float a, float b, int p) {
+        const uint32_t hi = pack_f16x2(a, b);
+        if (P == 1 || p == 0) return hi;
+        return pack_f16x2(a - f16_bits_to_float(hi), b - f16_bits_to_float(hi >> 16));
+    }
+
+    // Each lane packs 8 activations (two k-steps of one block) into the warp's
+    // staging area [p][t][hb][k-step][reg] (slot p at stage0 + p * pstride),
+    // then the owner lanes (g >> 1 == t) read their column of B from it.
+    __device__ __forceinline__ void load_x(const void *x, int M, int K, long k0, int lane, uint32_t stage0,
+                                           uint32_t pstride) {
+        (void)M;
+        (void)K;
+        const int blk = lane >> 2, q = lane & 3;   // block of the chunk and quarter of it
+        const int hb = blk & 1, tb = blk >> 1;
+        // Q4_0: code word q, k-steps 2q (low nibbles) and 2q+1 (high nibbles);
+        // Q8_0: code words 2q and 2q+1, one k-step each
+        float2 v[4];
+        if constexpr (FMT == F_Q4_0) {
+            const int e0 = cb0(hb, q), e2 = cb2(hb, q);
+            v[0] = load2(x, k0 + 32 * blk, e0);
+            v[1] = load2(x, k0 + 32 * blk, e2);
+            v[2] = load2(x, k0 + 32 * blk, 16 + e0);
+            v[3] = load2(x, k0 + 32 * blk, 16 + e2);
+        } else {
+            v[0] = load2(x, k0 + 32 * blk, cb0(hb, 2 * q));
+            v[1] = load2(x, k0 + 32 * blk, cb2(hb, 2 * q));
+            v[2] = load2(x, k0 + 32 * blk, cb0(hb, 2 * q + 1));
+            v[3] = load2(x, k0 + 32 * blk, cb2(hb, 2 * q + 1));
+        }
+        float mx = 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx = fmaxf(mx, absmax4(v[i]));
+        for (int i = 0; i < 4; ++i) mx = fmaxf(mx, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
+        float s;
         warp_scale<XT>(mx, s, inv);
-        // pack the lane's own half (8 k-steps) once, then place it in half h
-        uint32_t pk[8][2][P];
+        float sum = 0.f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            // Q4_0: word j/2, low (j even) or high (j odd) nibbles; Q8_0: word j
-            const int vi = (FMT == F_Q4_0) ? ((j >> 1) + 4 * (j & 1)) : j;
+        for (int i = 0; i < 4; ++i) {
+            v[i].x *= s;
+            v[i].y *= s;
+            sum += v[i].x + v[i].y;
+        }
+        // the block's sum over its four lanes
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+#pragma unroll
+        for (int p = 0; p < P; ++p) {
+            uint32_t r[4];
             if constexpr (FMT == F_Q4_0) {
-                pack2<XT>(pk[j][0], v[vi].x, v[vi].z, s);
-                pack2<XT>(pk[j][1], v[vi].y, v[vi].w, s);
+                // k-step 2q: reg 0 = code bytes (0, 2) of word q, reg 1 = bytes (1, 3); low nibbles
+                r[0] = part(v[0].x, v[1].x, p);
+                r[1] = part(v[0].y, v[1].y, p);
+                r[2] = part(v[2].x, v[3].x, p);   // k-step 2q+1: the high nibbles (elements + 16)
+                r[3] = part(v[2].y, v[3].y, p);
             } else {
-                pack2<XT>(pk[j][0], v[vi].x, v[vi].y, s);
-                pack2<XT>(pk[j][1], v[vi].z, v[vi].w, s);
+                // k-step j: reg 0 = code bytes (0, 1) of word j, reg 1 = bytes (2, 3)
+                r[0] = part(v[0].x, v[0].y, p);
+                r[1] = part(v[1].x, v[1].y, p);
+                r[2] = part(v[2].x, v[2].y, p);
+                r[3] = part(v[3].x, v[3].y, p);
             }
+            // k-steps 2q and 2q+1 of block (tb, hb): 4 consecutive words
+            st_shared_v4(stage0 + p * pstride + (uint32_t)(((tb * 2 + hb) * 16 + 4 * q) * 4), r[0], r[1], r[2], r[3]);
         }
+        __syncwarp();
+        const int g = lane >> 2, t = lane & 3;
+        corr[0] = -OFFSET * __shfl_sync(0xffffffffu, sum, 8 * t);
+        corr[1] = -OFFSET * __shfl_sync(0xffffffffu, sum, 8 * t + 4);
+        if ((g >> 1) == t && (g & 1) < P) {
+            const uint32_t src = stage0 + (g & 1) * pstride + (uint32_t)(t * 128);
 #pragma unroll
-        for (int st = 0; st < 16; ++st) {
-            const bool live = own && ((st >> 3) == h);
+            for (int i = 0; i < 8; ++i) {
+                const uint4 u = lds128(src + 16 * i);
+                xb[i >> 2][(i & 3) * 2][0] = u.x;
+                xb[i >> 2][(i & 3) * 2][1] = u.y;
+                xb[i >> 2][(i & 3) * 2 + 1][0] = u.z;
+                xb[i >> 2][(i & 3) * 2 + 1][1] = u.w;
+            }
+        } else {
 #pragma unroll
-            for (int r = 0; r < 2; ++r)
+            for (int h = 0; h < 2; ++h)
 #pragma unroll
-                for (int q = 0; q < P; ++q) xf[st][r][q] = live ? pk[st & 7][r][q] : 0u;
+                for (int j = 0; j < 8; ++j) xb[h][j][0] = xb[h][j][1] = 0u;
         }
+        __syncwarp();
     }
 
     __device__ __forceinline__ void compute(uint32_t tb, float (&acc)[1][4], int lane) const {
         const int g = lane >> 2, t = lane & 3;
         constexpr int CB = FmtInfo<FMT>::chunk_bytes;
-        const uint32_t r0 = tb + g * CB, r1 = tb + (g + 8) * CB;   // shared addresses of rows g, g+8
-        // four independent chains: [block of the pair][even / odd k-step]
-        float c[2][2][4];
+        constexpr int PW = CB / 16;   // words of lane t's block pair per row (2 * NWB + 1)
+        const uint32_t r0 = tb + g * CB + 4 * PW * t, r1 = r0 + 8 * CB;   // rows g, g+8
+        float y0 = 0.f, y1 = 0.f;
 #pragma unroll
-        for (int a = 0; a < 2; ++a)
+        for (int hb = 0; hb < 2; ++hb) {
+            uint32_t u0[NWB], u1[NWB];   // code words of the block, rows g and g+8
+            float d0, d1;
+            if (hb == 0) {
+                const uint32_t a0 = lds32(r0), a1 = lds32(r1);
+                const uint32_t b0 = lds32(r0 + 4 * NWB), b1 = lds32(r1 + 4 * NWB);
+                u0[0] = prmt(a0, b0, 0x3254u);
+                u1[0] = prmt(a1, b1, 0x3254u);
 #pragma unroll
-            for (int b = 0; b < 2; ++b)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) c[a][b][j] = 0.f;
-        float d[2][2];   // [block][row]
-        if constexpr (FMT == F_Q4_0) {
-            // lane t's block pair: 36 bytes (9 words) at word 9t of each row;
-            // block 2t: d in word 0 (low half), nibbles at bytes 2..17;
-            // block 2t+1: d in word 4 (high half), nibbles in words 5..8
-#pragma unroll
-            for (int hb = 0; hb < 2; ++hb) {
-                uint32_t W0[5], W1[5];
-#pragma unroll
-                for (int i = 0; i < 5; ++i) {
-                    W0[i] = lds32(r0 + 4 * (9 * t + 4 * hb + i));
-                    W1[i] = lds32(r1 + 4 * (9 * t + 4 * hb + i));
+                for (int j = 1; j < NWB; ++j) {
+                    u0[j] = lds32(r0 + 4 * j);
+                    u1[j] = lds32(r1 + 4 * j);
                 }
-                d[hb][0] = f16_bits_to_float(hb ? (W0[0] >> 16) : W0[0]);
-                d[hb][1] = f16_bits_to_float(hb ? (W1[0] >> 16) : W1[0]);
+                d0 = f16_bits_to_float(a0);
+                d1 = f16_bits_to_float(a1);
+            } else {
+                const uint32_t b0 = lds32(r0 + 4 * NWB), b1 = lds32(r1 + 4 * NWB);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t n0 = hb ? W0[1 + i] : __funnelshift_r(W0[i], W0[i + 1], 16);
-                    const uint32_t n1 = hb ? W1[1 + i] : __funnelshift_r(W1[i], W1[i + 1], 16);
-                    const uint32_t n0s = n0 >> 8, n1s = n1 >> 8;
-                    const uint32_t al[4] = {nib_lo(n0), nib_lo(n1), nib_lo(n0s), nib_lo(n1s)};
-                    const uint32_t ah[4] = {nib_hi(n0), nib_hi(n1), nib_hi(n0s), nib_hi(n1s)};
-                    const int st = 8 * hb + 2 * i;
-#pragma unroll
-                    for (int q = 0; q < P; ++q) {
-                        mma(c[hb][0], al, xf[st][0][q], xf[st][1][q]);
-                        mma(c[hb][1], ah, xf[st + 1][0][q], xf[st + 1][1][q]);
-                    }
+                for (int j = 0; j < NWB; ++j) {
+                    u0[j] = lds32(r0 + 4 * (NWB + 1 + j));
+                    u1[j] = lds32(r1 + 4 * (NWB + 1 + j));
                 }
+                d0 = f16_bits_to_float(b0 >> 16);
+                d1 = f16_bits_to_float(b1 >> 16);
             }
-        } else {
-            // lane t's block pair: 68 bytes (17 words) at word 17t of each row;
-            // block 2t: d in word 0 (low half), codes at bytes 2..33;
-            // block 2t+1: d in word 8 (high half), codes in words 9..16
+            float c[2][4];   // two independent chains
 #pragma unroll
-            for (int hb = 0; hb < 2; ++hb) {
-                uint32_t W0[9], W1[9];
+            for (int i = 0; i < 2; ++i)
 #pragma unroll
-                for (int i = 0; i < 9; ++i) {
-                    W0[i] = lds32(r0 + 4 * (17 * t + 8 * hb + i));
-                    W1[i] = lds32(r1 + 4 * (17 * t + 8 * hb + i));
+                for (int j = 0; j < 4; ++j) c[i][j] = 0.f;
+            float S0, S1;
+            if constexpr (FMT == F_Q4_0) {
+                // chain 0: low nibbles (u * 2^-24), chain 1: high nibbles (16u * 2^-24)
+#pragma unroll
+                for (int j = 0; j < NWB; ++j) {
+                    const uint32_t s0 = u0[j] >> 8, s1 = u1[j] >> 8;
+                    const uint32_t al[4] = {u0[j] & 0x000F000Fu, u1[j] & 0x000F000Fu, s0 & 0x000F000Fu,
+                                            s1 & 0x000F000Fu};
+                    const uint32_t ah[4] = {u0[j] & 0x00F000F0u, u1[j] & 0x00F000F0u, s0 & 0x00F000F0u,
+                                            s1 & 0x00F000F0u};
+                    mma(c[0], al, xb[hb][2 * j][0], xb[hb][2 * j][1]);
+                    mma(c[1], ah, xb[hb][2 * j + 1][0], xb[hb][2 * j + 1][1]);
                 }
-                d[hb][0] = f16_bits_to_float(hb ? (W0[0] >> 16) : W0[0]);
-                d[hb][1] = f16_bits_to_float(hb ? (W1[0] >> 16) : W1[0]);
+                const float lo0 = (P == 2) ? c[0][0] + c[0][1] : c[0][0];
+                const float lo1 = (P == 2) ? c[0][2] + c[0][3] : c[0][2];
+                const float hi0 = (P == 2) ? c[1][0] + c[1][1] : c[1][0];
+                const float hi1 = (P == 2) ? c[1][2] + c[1][3] : c[1][2];
+                S0 = fmaf(hi0, 0.0625f, lo0);
+                S1 = fmaf(hi1, 0.0625f, lo1);
+            } else {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint32_t q0 = hb ? W0[1 + i] : __funnelshift_r(W0[i], W0[i + 1], 16);
-                    const uint32_t q1 = hb ? W1[1 + i] : __funnelshift_r(W1[i], W1[i + 1], 16);
-                    uint32_t a[4];
-                    q8_pairs(q0, a[0], a[2]);
-                    q8_pairs(q1, a[1], a[3]);
-                    const int st = 8 * hb + i;
-#pragma unroll
-                    for (int q = 0; q < P; ++q) mma(c[hb][i & 1], a, xf[st][0][q], xf[st][1][q]);
+                for (int j = 0; j < NWB; ++j) {
+                    const uint32_t v0 = u0[j] ^ 0x80808080u, v1 = u1[j] ^ 0x80808080u;
+                    const uint32_t a[4] = {prmt(v0, 0u, 0x4140u), prmt(v1, 0u, 0x4140u), prmt(v0, 0u, 0x4342u),
+                                           prmt(v1, 0u, 0x4342u)};
+                    mma(c[j & 1], a, xb[hb][j][0], xb[hb][j][1]);
                 }
+                S0 = (P == 2) ? (c[0][0] + c[1][0]) + (c[0][1] + c[1][1]) : c[0][0] + c[1][0];
+                S1 = (P == 2) ? (c[0][2] + c[1][2]) + (c[0][3] + c[1][3]) : c[0][2] + c[1][2];
             }
+            // block value in scaled-activation units: d * (2^24 S - OFFSET * sum x)
+            y0 = fmaf(d0, fmaf(S0, 16777216.f, corr[hb]), y0);
+            y1 = fmaf(d1, fmaf(S1, 16777216.f, corr[hb]), y1);
         }
-        // column 2t (block 2t) lives in c[0][*], column 2t+1 (block 2t+1) in c[1][*]
-        float yg = d[0][0] * (c[0][0][0] + c[0][1][0]) + d[1][0] * (c[1][0][1] + c[1][1][1]);
-        float yg8 = d[0][1] * (c[0][0][2] + c[0][1][2]) + d[1][1] * (c[1][0][3] + c[1][1][3]);
-        yg += __shfl_xor_sync(0xffffffffu, yg, 1);
-        yg8 += __shfl_xor_sync(0xffffffffu, yg8, 1);
-        yg += __shfl_xor_sync(0xffffffffu, yg, 2);
-        yg8 += __shfl_xor_sync(0xffffffffu, yg8, 2);
-        acc[0][0] += yg;
-        acc[0][2] += yg8;
+        y0 += __shfl_xor_sync(0xffffffffu, y0, 1);
+        y1 += __shfl_xor_sync(0xffffffffu, y1, 1);
+        y0 += __shfl_xor_sync(0xffffffffu, y0, 2);
+        y1 += __shfl_xor_sync(0xffffffffu, y1, 2);
+        acc[0][0] += y0;
+        acc[0][2] += y1;
     }
 };
 
@@ -401,7 +483,7 @@ struct Q80 {
     uint32_t xf[NT][8][2][2][P];
     float inv;
 
-    __device__ __forceinline__ void load_x(const void *x, int M, int K, long k0, int lane) {
+    __device__ __forceinline__ void load_x(const void *x, int M, int K, long k0, int lane, uint32_t, uint32_t) {
         const int g = lane >> 2, t = lane & 3;
         float mx = 0.f, s;
 #pragma unroll
@@ -492,7 +574,7 @@ struct Q4K {
     uint32_t xs[NT][2];            // scaled sub-block sums (X_2t, X_2t+1) of column g: hi, lo
     float inv;
 
-    __device__ __forceinline__ void load_x(const void *x, int M, int K, long k0, int lane) {
+    __device__ __forceinline__ void load_x(const void *x, int M, int K, long k0, int lane, uint32_t, uint32_t) {
         const int g = lane >> 2, t = lane & 3;
         float mx = 0.f, s;
 #pragma unroll
@@ -671,15 +753,19 @@ __global__ void __maxnreg__(NT == 1 ? 96 : 128)
         // overlap promise is not written by the preceding work
         if (lane == 0) {
             tma_prefetch_desc(&wmap);
-            int it = 0;
+            // stage index and phase parity tracked incrementally (no division per tile)
+            int it = 0, s = 0;
+            uint32_t ph = 0;
             for (int tile = rgrp; tile < a.row_tiles; tile += G, ++it) {
-                const int s = it % stages;
-                if (it >= stages && !mbar_wait(&empty[s], ((it / stages) - 1) & 1, a.timeout_ns, DEVERR_GEMV_WAIT))
-                    break;
+                if (it >= stages && !mbar_wait(&empty[s], ph ^ 1u, a.timeout_ns, DEVERR_GEMV_WAIT)) break;
                 mbar_arrive_expect_tx(&full[s], (uint32_t)(nact * BOX));
                 for (int w = 0; w < nact; ++w)
                     tma_load_2d(boxes + ((size_t)s * NW + w) * BOX, &wmap, &full[s], (c_begin + w) * (CB / 2),
                                 tile * GEMV_ROWS);
+                if (++s == stages) {
+                    s = 0;
+                    ph ^= 1u;
+                }
             }
             // drain: every issued stage's load lands before the CTA may exit
             const int issued = it;
@@ -694,10 +780,10 @@ __global__ void __maxnreg__(NT == 1 ? 96 : 128)
         pdl_wait();
         const int M = a.M, N = a.N;
         const int nout = GEMV_ROWS * M;  // outputs per tile: 16 rows x M columns
-        int it = 0;
-        for (int tile = rgrp; tile < a.row_tiles; tile += G, ++it) {
-            const int s = it % stages;
-            if (!mbar_wait(&redfull[s], (it / stages) & 1, a.timeout_ns, DEVERR_GEMV_WAIT)) break;
+        int s = 0;
+        uint32_t ph = 0;
+        for (int tile = rgrp; tile < a.row_tiles; tile += G) {
+            if (!mbar_wait(&redfull[s], ph, a.timeout_ns, DEVERR_GEMV_WAIT)) break;
             const uint32_t rs = smem_u32(red) + (uint32_t)(s * NW * RED * 4);
             for (int o = lane; o < nout; o += 32) {
                 const int r = o % GEMV_ROWS, b = o / GEMV_ROWS;
@@ -735,6 +821,10 @@ __global__ void __maxnreg__(NT == 1 ? 96 : 128)
                     if (lane == 0) a.counters[tile] = 0u;
                 }
             }
+            if (++s == stages) {
+                s = 0;
+                ph ^= 1u;
+            }
         }
         return;
     }
@@ -743,12 +833,15 @@ __global__ void __maxnreg__(NT == 1 ? 96 : 128)
     if (warp >= nact) return;
     GemvImpl<FMT, XT, NT, ONE> impl;
     pdl_wait();   // x may be the preceding kernel's output
-    impl.load_x(a.x, a.M, a.K, (long)(c_begin + warp) * CHUNK, lane);
+    // staging for the activation layout: this warp's partial-sum slots of stages 0 and 1,
+    // which it first writes after its first tile
+    impl.load_x(a.x, a.M, a.K, (long)(c_begin + warp) * CHUNK, lane, smem_u32(red) + (uint32_t)(warp * RED * 4),
+                (uint32_t)(NW * RED * 4));
     const int g = lane >> 2, t = lane & 3;
-    int it = 0;
-    for (int tile = rgrp; tile < a.row_tiles; tile += G, ++it) {
-        const int s = it % stages;
-        if (!mbar_wait(&full[s], (it / stages) & 1, a.timeout_ns, DEVERR_GEMV_WAIT)) break;
+    int s = 0;
+    uint32_t ph = 0;
+    for (int tile = rgrp; tile < a.row_tiles; tile += G) {
+        if (!mbar_wait(&full[s], ph, a.timeout_ns, DEVERR_GEMV_WAIT)) break;
         float acc[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
@@ -769,6 +862,10 @@ __global__ void __maxnreg__(NT == 1 ? 96 : 128)
         if (lane == 0) {
             mbar_arrive(&redfull[s]);
             mbar_arrive(&empty[s]);
+        }
+        if (++s == stages) {
+            s = 0;
+            ph ^= 1u;
         }
     }
 }
