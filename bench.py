@@ -399,7 +399,8 @@ def run_gpu_arm(args):
     achieved = prob.bytes_per_step / (ms_local / args.steps / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": args.traffic,
-                "peak_source": peak_src, "kernel": "lwq::gemv_tc_kernel<Q4_0, fp32 x, NT=1>",
+                "peak_source": peak_src,
+                "kernel": "lwq::gemv_tc_kernel<Q4_0, fp32 x> (M=1 one-row, M=4 one tile, M=8 two tiles)",
                 "per_call_ms": [{"M": p["call"][2], "ms": round(p["ms_mean"], 5),
                                  "GB/s": round(call_bytes(*p["call"][:5]) / p["ms_mean"] / 1e6, 1)} for p in per]}
 
@@ -440,9 +441,10 @@ def run_gpu_arm(args):
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16",
             "data": "synthetic",
-            "config": {"workload": HEADLINE, "weights": "q4_0", "activations": "f32 (split into bf16 hi+lo)",
+            "config": {"workload": HEADLINE, "weights": "q4_0", "activations": "f32, held as fp16 hi + lo (22 significant bits)",
+                       "mma": "fp16 x fp16 products, f32 accumulation",
                        "accumulate": "f32", "M": [1, 4, 8], "N": 11008, "K": 4096, "seed": 0,
                        "l2": f"inputs larger than L2: every call reads its own weight copy, "
                              f"{prob.copies_bytes / 1e6:.0f} MB of copies in rotation",

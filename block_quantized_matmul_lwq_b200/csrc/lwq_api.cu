@@ -100,11 +100,22 @@ struct Plan {
 };
 
 // packed boxes + fp32 partials + full/empty/reduced mbarriers
-size_t gemv_smem(int wf, int nw, int stages, int nt) {
+// (ot: output tiles of 8 activation columns; fp32 activations always use one)
+size_t gemv_smem(int wf, int nw, int stages, int ot) {
     const int cb = (wf == LWQ_Q8_0) ? 272 : 144;
-    return (size_t)stages * nw * GEMV_ROWS * cb + (size_t)stages * nw * GEMV_ROWS * 8 * nt * 4 +
+    return (size_t)stages * nw * GEMV_ROWS * cb + (size_t)stages * nw * GEMV_ROWS * 8 * ot * 4 +
            (size_t)3 * stages * 8;
 }
+
+// n8 column tiles of the GEMV for a pass of mg activation rows: 16-bit
+// activations, 8 rows per tile; fp32 Q4_0, one tile of 4 rows x 2 fp16 parts
+// up to 4 rows and two tiles (one per part) up to 8; other fp32 formats, one
+// tile (parts in separate MMAs).
+inline int gemv_nt(int wf, int xt, int mg) {
+    if (xt == X_F32) return (wf == LWQ_Q4_0 && mg > 4) ? 2 : 1;
+    return mg <= 8 ? 1 : 2;
+}
+inline int gemv_ot(int xt, int nt) { return xt == X_F32 ? 1 : nt; }
 
 bool tc_gemv_eligible(int wf, int xt, long K) {
     (void)wf;
@@ -163,9 +174,9 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
     if (path != 1 || !tc_gemv_eligible(wf, xt, K)) return LWQ_ERR_UNSUPPORTED;
     const int mmax = (xt == X_F32) ? 8 : 16;
     p->m_group = M < mmax ? M : mmax;
-    p->nt = p->m_group <= 8 ? 1 : 2;
+    p->nt = gemv_nt(wf, xt, p->m_group);
     const int nchunks = K / 256;
-    const int nw_max = p->nt == 1 ? 16 : 14;   // register budget (see gemv_tc_kernel)
+    const int nw_max = gemv_max_regs(wf, xt, p->nt) == 96 ? 16 : 14;   // register budget (see gemv_tc_kernel)
     int nw = force && force->warps ? force->warps : (wf == LWQ_Q8_0 ? 8 : nw_max);
     if (nw > nw_max || nw < 1) return LWQ_ERR_UNSUPPORTED;
     if (nw > nchunks) nw = nchunks;
@@ -175,8 +186,8 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
     if (cps > nw) return LWQ_ERR_UNSUPPORTED;  // every chunk of a split needs a warp
     S = (nchunks + cps - 1) / cps;               // drop empty splits
     int stages = force && force->stages ? force->stages : 4;
-    while (stages > 2 && gemv_smem(wf, nw, stages, p->nt) > kSmemLimit) --stages;
-    if (stages < 2 || gemv_smem(wf, nw, stages, p->nt) > kSmemLimit) return LWQ_ERR_UNSUPPORTED;
+    while (stages > 2 && gemv_smem(wf, nw, stages, gemv_ot(xt, p->nt)) > kSmemLimit) --stages;
+    if (stages < 2 || gemv_smem(wf, nw, stages, gemv_ot(xt, p->nt)) > kSmemLimit) return LWQ_ERR_UNSUPPORTED;
     const int row_tiles = (N + GEMV_ROWS - 1) / GEMV_ROWS;
     if (S > 1 && row_tiles > kMaxSplitTiles) return LWQ_ERR_UNSUPPORTED;
     int groups = force && force->ctas ? force->ctas / S : sms / S;
@@ -186,7 +197,7 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
     p->cfg.stages = stages;
     p->cfg.splits = S;
     p->cfg.ctas = S * groups;
-    p->smem = gemv_smem(wf, nw, stages, p->nt);
+    p->smem = gemv_smem(wf, nw, stages, gemv_ot(xt, p->nt));
     p->ws_need = splitk_ws(S, p->m_group, N);
     return LWQ_OK;
 }
@@ -244,17 +255,17 @@ cudaError_t launch_gemv_tc(const CUtensorMap &map, const GemvArgs &a, int ctas, 
     return launch_k(kern, ctas, (nw + 2) * 32, smem, st, a.overlap != 0, map, a);
 }
 
-// NT = n8 tiles of activation rows (2 only for 16-bit activations); the
+// NT = n8 column tiles (gemv_nt: 2 for 16-bit activations beyond 8 rows, and
+// for fp32 Q4_0 beyond 4 rows); the
 // one-row mapping serves passes with a single activation row (Q4_0, Q8_0).
 template <int FMT, int XT>
 cudaError_t launch_gemv_tc_nt(int nt, bool one, const CUtensorMap &map, const GemvArgs &a, int ctas, int nw,
                               size_t smem, cudaStream_t st) {
     if (nt == 1) {
-        if constexpr (FMT != F_Q4_K)
-            if (one) return launch_gemv_tc<FMT, XT, 1, true>(map, a, ctas, nw, smem, st);
+        if (one) return launch_gemv_tc<FMT, XT, 1, true>(map, a, ctas, nw, smem, st);
         return launch_gemv_tc<FMT, XT, 1, false>(map, a, ctas, nw, smem, st);
     }
-    if constexpr (XT != X_F32) return launch_gemv_tc<FMT, XT, 2, false>(map, a, ctas, nw, smem, st);
+    if constexpr (XT != X_F32 || FMT == F_Q4_0) return launch_gemv_tc<FMT, XT, 2, false>(map, a, ctas, nw, smem, st);
     return cudaErrorInvalidValue;
 }
 
@@ -442,9 +453,9 @@ int run(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, c
         a.stages = p.cfg.stages;
         a.timeout_ns = kTimeoutNs;
         a.overlap = overlap;
-        const int nt = mg <= 8 ? 1 : 2;
+        const int nt = gemv_nt(wf, xt, mg);
         cudaError_t e = dispatch_gemv_tc(wf, xt, nt, mg == 1, map, a, p.cfg.ctas, p.cfg.warps,
-                                         gemv_smem(wf, p.cfg.warps, p.cfg.stages, nt), st);
+                                         gemv_smem(wf, p.cfg.warps, p.cfg.stages, gemv_ot(xt, nt)), st);
         if (e != cudaSuccess) return LWQ_ERR_CUDA;
         ++launches;
     }

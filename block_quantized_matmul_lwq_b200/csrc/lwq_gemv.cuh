@@ -14,11 +14,11 @@
 //    1024 + q: one LOP3 and one packed FMA per two weights, no conversion
 //    instructions) and issues mma.sync m16n8k16 with the weight rows as the
 //    MMA's M dimension.
-//  * Activations: fp16 as they are; bf16 and fp32 scaled by one power of two
-//    per warp so that the warp's largest |x| lands in [2^13, 2^14), then fp16
-//    (bf16's 8-bit significand fits fp16's 11) or an fp16 hi + lo pair (22
-//    significant bits) for fp32.  The scale is undone exactly on the fp32
-//    results.
+//  * Activations are scaled by one power of two per warp so that the warp's
+//    largest |x| lands in [2^13, 2^14), then held as fp16 (fp16 and bf16
+//    inputs: exact, bf16's 8-bit significand fits fp16's 11) or as an fp16
+//    hi + lo pair (22 significant bits) for fp32.  The scale is undone exactly
+//    on the fp32 results.
 //  * Two lane mappings.  Several activation rows (M >= 2): the MMA's N
 //    dimension carries the activation rows; the four lanes of a weight row
 //    share a block per k-step, and block scales multiply the fp32 MMA
@@ -118,14 +118,16 @@ __device__ __forceinline__ float absmax4(float4 v) {
 }
 
 // Power-of-two scale s (and 1/s) that puts the warp's largest |x| in
-// [2^13, 2^14); fp16 activations are used as they are (s = 1).
+// [2^13, 2^14).  Exact for fp16 and bf16 activations (bar elements that fall
+// below fp16's normal range, 2^-27 of the largest), and it keeps x / 16 (the
+// high-nibble k-steps) in the normal range too.
 template <int XT>
 __device__ __forceinline__ void warp_scale(float local_max, float &s, float &inv) {
     float m = local_max;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     s = inv = 1.f;
-    if (XT == X_F16 || !(m > 0.f) || !(m <= 3.0e38f)) return;
+    if (!(m > 0.f) || !(m <= 3.0e38f)) return;
     const int e = (int)((__float_as_uint(m) >> 23) & 0xFF) - 127;
     int es = 13 - e;
     es = es > 126 ? 126 : (es < -126 ? -126 : es);
@@ -133,7 +135,7 @@ __device__ __forceinline__ void warp_scale(float local_max, float &s, float &inv
     inv = __uint_as_float((uint32_t)(127 - es) << 23);
 }
 
-// Two scaled activations as fp16 pair(s): exact for fp16 (s = 1) and for
+// Two scaled activations as fp16 pair(s): exact for fp16 and
 // bf16 (8 significant bits); fp32 splits into hi + lo (22 bits together).
 template <int XT>
 __device__ __forceinline__ void pack2(uint32_t (&out)[XFrag<XT>::parts], float a, float b, float s) {
@@ -170,89 +172,233 @@ __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint3
 }
 
 // ------------------------------------------------- Q4_0, several activation rows
-// Per block (32 weights, 2 k-steps), lane t (= lane % 4) of weight row g
-// (= lane / 4) takes nibble bytes 4t..4t+3: k-step A uses elements
-// (4t, 4t+2 | 4t+1, 4t+3), k-step B (4t+16, 4t+18 | 4t+17, 4t+19).
+// The MMA's N dimension carries activation columns; lane (g, t) of weight
+// rows g, g+8 takes code word t of every block (4 code bytes, 8 weights), and
+// each block is two k-steps: its low nibbles, then its high nibbles.  Word t
+// of an odd block (word-aligned in the 36-byte block pair) is read as it
+// lies; word t of an even block holds code bytes 4t-2..4t+1 (t > 0) or
+// (14, 15, 0, 1) (t = 0).  A register of code bytes (b0, b2) or (b1, b3) of
+// the word feeds k-slots (2t, 2t+1) or (2t+8, 2t+9).
+//
+// Codes enter the MMA as fp16 subnormals (see the one-row mapping below): the
+// low nibble u is u * 2^-24 and the high nibble, left in place, 16u * 2^-24,
+// so the high-nibble k-step takes its activations divided by 16.  Per block,
+// C_b = sum_k u_k x_k * 2^-24 and y += d_b C_b; the offset 8 comes off once
+// per tile through one more MMA: A = the block scales d (fp16, exact),
+// B = the block sums of x / 64 as an fp16 hi + lo pair, so
+// y = 2^24 sum_b d_b C_b - 8 * 64 * sum_b d_b (X_b / 64).
+//
+// Column tiles (NT): 16-bit activations: tile nt holds activation rows
+// 8nt..8nt+7.  fp32 activations (hi + lo fp16 parts): NT = 1 holds up to 4
+// rows, column g = part g >> 2 of row g & 3 (the reducer adds columns b and
+// b + 4); NT = 2 holds up to 8 rows with the two parts in the two tiles, both
+// accumulated into one result (so only the first output tile is written).
 template <int XT, int NT>
 struct Q40 {
     static constexpr int P = XFrag<XT>::parts;
-    uint32_t xf[NT][8][2][2][P];   // [nt][block][step][reg][part]
+    static constexpr bool MERGED = (XT == X_F32 && NT == 1);
+    static constexpr bool PART_TILES = (XT == X_F32 && NT == 2);
+    uint32_t xf[NT][8][2][2];   // [tile][block][k-step][reg]
+    uint32_t xs[NT][2];         // correction B: block sums / 64 of blocks (2t, 2t+1), hi and lo
     float inv;
 
-    __device__ __forceinline__ void load_x(const void *x, int M, int K, long k0, int lane, uint32_t, uint32_t) {
-        const int g = lane >> 2, t = lane & 3;
-        float mx = 0.f, s;
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int blk = 0; blk < 8; ++blk) {
-                mx = fmaxf(mx, absmax4(load4<XT>(x, M, K, g + 8 * nt, k0, blk * 32 + 4 * t)));
-                mx = fmaxf(mx, absmax4(load4<XT>(x, M, K, g + 8 * nt, k0, blk * 32 + 16 + 4 * t)));
-            }
-        warp_scale<XT>(mx, s, inv);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int blk = 0; blk < 8; ++blk)
-#pragma unroll
-                for (int st = 0; st < 2; ++st) {
-                    const float4 v = load4<XT>(x, M, K, g + 8 * nt, k0, blk * 32 + 16 * st + 4 * t);
-                    pack2<XT>(xf[nt][blk][st][0], v.x, v.z, s);
-                    pack2<XT>(xf[nt][blk][st][1], v.y, v.w, s);
-                }
+    __device__ static __forceinline__ int cb0(int hb, int j) { return hb ? 4 * j : (j ? 4 * j - 2 : 14); }
+    __device__ static __forceinline__ int cb2(int hb, int j) { return hb ? 4 * j + 2 : 4 * j; }
+
+    __device__ static __forceinline__ float2 load2(const void *x, long off) {
+        if constexpr (XT == X_F32) {
+            return __ldg(reinterpret_cast<const float2 *>(static_cast<const float *>(x) + off));
+        } else {
+            const uint32_t u = __ldg(reinterpret_cast<const uint32_t *>(static_cast<const uint16_t *>(x) + off));
+            if constexpr (XT == X_F16)
+                return make_float2(f16_bits_to_float(u), f16_bits_to_float(u >> 16));
+            else
+                return make_float2(bf16_bits_to_float(u), bf16_bits_to_float(u >> 16));
+        }
     }
 
-    // tb: this warp's [16 rows][144 B] box.  acc[nt][4] accumulates (scaled).
-    __device__ __forceinline__ void compute(uint32_t tb, float (&acc)[NT][4], int lane) const {
+    // Part p of the fp16 pair (a, b).
+    __device__ static __forceinline__ uint32_t part(float a, float b, int p) {
+        const uint32_t hi = pack_f16x2(a, b);
+        if (P == 1 || p == 0) return hi;
+        return pack_f16x2(a - f16_bits_to_float(hi), b - f16_bits_to_float(hi >> 16));
+    }
+
+    // Activation rows in this pass's column tiles, and writer units per lane:
+    // a unit is (row m, code word t, nibble half h) of one block, 4 elements.
+    static constexpr int ROWS = MERGED ? 4 : (PART_TILES ? 8 : 8 * NT);
+    static constexpr int UPL = ROWS * 8 / 32;   // units per lane per block
+    static constexpr int OT = PART_TILES ? 1 : NT;
+
+    // Tile nt of a block's B in the staging area: [lane][h][reg], 512 bytes.
+    __device__ static __forceinline__ uint32_t stage_addr(uint32_t stage0, uint32_t pstride, int nt) {
+        return (OT == NT) ? stage0 + 512u * nt : stage0 + pstride * nt;
+    }
+    // Column tile and column of part p of row m.
+    __device__ static __forceinline__ void place(int m, int p, int &nt, int &g) {
+        if (MERGED) {
+            nt = 0;
+            g = m + 4 * p;
+        } else if (PART_TILES) {
+            nt = p;
+            g = m;
+        } else {
+            nt = m >> 3;
+            g = m & 7;
+        }
+    }
+
+    // One block at a time, every lane packs UPL units (each element of the
+    // pass's rows once, both fp16 parts) into the warp's staging area, then
+    // reads back its own B fragments; the block sums ride along for the offset
+    // correction.
+    __device__ __forceinline__ void load_x(const void *x, int M, int K, long k0, int lane, uint32_t stage0,
+                                           uint32_t pstride) {
         const int g = lane >> 2, t = lane & 3;
-        const uint32_t r0 = tb + g * 144, r1 = tb + (g + 8) * 144;   // shared addresses of rows g, g+8
+        // pass 1: the warp's largest |x|
+        float mx = 0.f;
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            uint32_t nw[2][2];   // [block in pair][row]
-            float dd[2][2];
-            {
-                const uint32_t b = 36 * p;
-                const uint32_t a0 = lds32(r0 + b + 4 * t), a1 = lds32(r0 + b + 4 * t + 4);
-                const uint32_t c0 = lds32(r1 + b + 4 * t), c1 = lds32(r1 + b + 4 * t + 4);
-                nw[0][0] = __funnelshift_r(a0, a1, 16);
-                nw[0][1] = __funnelshift_r(c0, c1, 16);
-                nw[1][0] = lds32(r0 + b + 20 + 4 * t);
-                nw[1][1] = lds32(r1 + b + 20 + 4 * t);
-                dd[0][0] = f16_bits_to_float(lds32(r0 + b));
-                dd[0][1] = f16_bits_to_float(lds32(r1 + b));
-                dd[1][0] = f16_bits_to_float(lds32(r0 + b + 16) >> 16);
-                dd[1][1] = f16_bits_to_float(lds32(r1 + b + 16) >> 16);
-            }
-            uint32_t aA[2][4], aB[2][4];
+        for (int k = 0; k < UPL; ++k) {
+            const int u = lane + 32 * k, m = u >> 3, tu = (u >> 1) & 3, h = u & 1;
+            if (m < M) {
+                const long base = (long)m * K + k0 + 16 * h;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint32_t w0 = nw[h][0], w1 = nw[h][1];
-                const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
-                aA[h][0] = nib_lo(w0);
-                aA[h][1] = nib_lo(w1);
-                aA[h][2] = nib_lo(w0s);
-                aA[h][3] = nib_lo(w1s);
-                aB[h][0] = nib_hi(w0);
-                aB[h][1] = nib_hi(w1);
-                aB[h][2] = nib_hi(w0s);
-                aB[h][3] = nib_hi(w1s);
+                for (int b = 0; b < 8; ++b) {
+                    const float2 p = load2(x, base + 32 * b + cb0(b & 1, tu));
+                    const float2 q = load2(x, base + 32 * b + cb2(b & 1, tu));
+                    mx = fmaxf(mx, fmaxf(fmaxf(fabsf(p.x), fabsf(p.y)), fmaxf(fabsf(q.x), fabsf(q.y))));
+                }
             }
+        }
+        float s;
+        warp_scale<XT>(mx, s, inv);
+        // correction sums of blocks (2t, 2t+1) for each tile's column g (part 0 only)
+        float cs[NT][2];
+        int crow[NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            cs[nt][0] = cs[nt][1] = 0.f;
+            const int row = MERGED ? (g & 3) : (PART_TILES ? g : g + 8 * nt);
+            const bool part0 = MERGED ? (g < 4) : (PART_TILES ? nt == 0 : true);
+            crow[nt] = (part0 && row < M) ? row : -1;
+        }
+        // pass 2, one block per round
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+#pragma unroll
+            for (int k = 0; k < UPL; ++k) {
+                const int u = lane + 32 * k, m = u >> 3, tu = (u >> 1) & 3, h = u & 1;
+                float2 p = make_float2(0.f, 0.f), q = make_float2(0.f, 0.f);
+                if (m < M) {
+                    const long e = (long)m * K + k0 + 32 * b + 16 * h;
+                    p = load2(x, e + cb0(b & 1, tu));
+                    q = load2(x, e + cb2(b & 1, tu));
+                }
+                // high-nibble step: x / 16 (exact: a power of two)
+                const float sc = h ? s * 0.0625f : s;
+                p.x *= sc;
+                p.y *= sc;
+                q.x *= sc;
+                q.y *= sc;
+                float bs = h ? 16.f * ((p.x + p.y) + (q.x + q.y)) : (p.x + p.y) + (q.x + q.y);
+                // the block sum of row m: its 8 units sit in lanes 8(m & 3) .. 8(m & 3) + 7
+                bs += __shfl_xor_sync(0xffffffffu, bs, 1);
+                bs += __shfl_xor_sync(0xffffffffu, bs, 2);
+                bs += __shfl_xor_sync(0xffffffffu, bs, 4);
+#pragma unroll
+                for (int pp = 0; pp < P; ++pp) {
+                    int nt, gg;
+                    place(m, pp, nt, gg);
+                    const uint32_t dst = stage_addr(stage0, pstride, nt) + (uint32_t)((4 * gg + tu) * 16 + 8 * h);
+                    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(dst), "r"(part(p.x, q.x, pp)),
+                                 "r"(part(p.y, q.y, pp))
+                                 : "memory");
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int r = crow[nt] < 0 ? 0 : crow[nt];
+                    const float v = __shfl_sync(0xffffffffu, bs, 8 * (r & 3));
+                    if (crow[nt] >= 0 && (crow[nt] >> 2) == k && (b >> 1) == t) cs[nt][b & 1] = v;
+                }
+            }
+            __syncwarp();
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                // two independent chains (one per block), each over both parts
-                float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int q = 0; q < P; ++q) {
-                    mma(c0, aA[0], xf[nt][2 * p][0][0][q], xf[nt][2 * p][0][1][q]);
-                    mma(c1, aA[1], xf[nt][2 * p + 1][0][0][q], xf[nt][2 * p + 1][0][1][q]);
-                    mma(c0, aB[0], xf[nt][2 * p][1][0][q], xf[nt][2 * p][1][1][q]);
-                    mma(c1, aB[1], xf[nt][2 * p + 1][1][0][q], xf[nt][2 * p + 1][1][1][q]);
-                }
-                acc[nt][0] = fmaf(dd[0][0], c0[0], fmaf(dd[1][0], c1[0], acc[nt][0]));
-                acc[nt][1] = fmaf(dd[0][0], c0[1], fmaf(dd[1][0], c1[1], acc[nt][1]));
-                acc[nt][2] = fmaf(dd[0][1], c0[2], fmaf(dd[1][1], c1[2], acc[nt][2]));
-                acc[nt][3] = fmaf(dd[0][1], c0[3], fmaf(dd[1][1], c1[3], acc[nt][3]));
+                const uint4 v = lds128(stage_addr(stage0, pstride, nt) + (uint32_t)(lane * 16));
+                xf[nt][b][0][0] = v.x;
+                xf[nt][b][0][1] = v.y;
+                xf[nt][b][1][0] = v.z;
+                xf[nt][b][1][1] = v.w;
             }
+            __syncwarp();
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const float s0 = cs[nt][0] * 0.015625f, s1 = cs[nt][1] * 0.015625f;
+            const uint32_t hh = pack_f16x2(s0, s1);
+            xs[nt][0] = hh;
+            xs[nt][1] = pack_f16x2(s0 - f16_bits_to_float(hh), s1 - f16_bits_to_float(hh >> 16));
+        }
+    }
+
+    // tb: this warp's [16 rows][144 B] box.
+    __device__ __forceinline__ void compute(uint32_t tb, float (&acc)[NT][4], int lane) const {
+        const int g = lane >> 2, t = lane & 3;
+        const uint32_t r0 = tb + g * 144, r1 = r0 + 8 * 144;   // rows g, g+8
+        const uint32_t sel = t ? 0x3210u : 0x3254u;            // word t of an even block
+        float m[OT][4];
+#pragma unroll
+        for (int o = 0; o < OT; ++o)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) m[o][j] = 0.f;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const uint32_t pb = 36 * p;
+            const uint32_t w00 = lds32(r0 + pb), w10 = lds32(r1 + pb);             // d(2p), codes
+            const uint32_t w04 = lds32(r0 + pb + 16), w14 = lds32(r1 + pb + 16);   // codes, d(2p+1)
+            uint32_t u[2][2];   // [block of the pair][row]
+            u[0][0] = prmt(lds32(r0 + pb + 4 * t), w04, sel);
+            u[0][1] = prmt(lds32(r1 + pb + 4 * t), w14, sel);
+            u[1][0] = lds32(r0 + pb + 20 + 4 * t);
+            u[1][1] = lds32(r1 + pb + 20 + 4 * t);
+            const float d[2][2] = {{f16_bits_to_float(w00), f16_bits_to_float(w10)},
+                                   {f16_bits_to_float(w04 >> 16), f16_bits_to_float(w14 >> 16)}};
+#pragma unroll
+            for (int hb = 0; hb < 2; ++hb) {
+                const uint32_t a0 = u[hb][0], a1 = u[hb][1], s0 = a0 >> 8, s1 = a1 >> 8;
+                const uint32_t al[4] = {a0 & 0x000F000Fu, a1 & 0x000F000Fu, s0 & 0x000F000Fu, s1 & 0x000F000Fu};
+                const uint32_t ah[4] = {a0 & 0x00F000F0u, a1 & 0x00F000F0u, s0 & 0x00F000F0u, s1 & 0x00F000F0u};
+                const int b = 2 * p + hb;
+                float c[OT][4];
+#pragma unroll
+                for (int o = 0; o < OT; ++o)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) c[o][j] = 0.f;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int o = PART_TILES ? 0 : nt;
+                    mma(c[o], al, xf[nt][b][0][0], xf[nt][b][0][1]);
+                    mma(c[o], ah, xf[nt][b][1][0], xf[nt][b][1][1]);
+                }
+#pragma unroll
+                for (int o = 0; o < OT; ++o) {
+                    m[o][0] = fmaf(d[hb][0], c[o][0], m[o][0]);
+                    m[o][1] = fmaf(d[hb][0], c[o][1], m[o][1]);
+                    m[o][2] = fmaf(d[hb][1], c[o][2], m[o][2]);
+                    m[o][3] = fmaf(d[hb][1], c[o][3], m[o][3]);
+                }
+            }
+        }
+        // offset correction: A = (d(2t), d(2t+1)) of rows g, g+8, twice (hi and lo sums)
+        const uint32_t q0 = prmt(lds32(r0 + 36 * t), lds32(r0 + 36 * t + 16), 0x7610u);
+        const uint32_t q1 = prmt(lds32(r1 + 36 * t), lds32(r1 + 36 * t + 16), 0x7610u);
+        const uint32_t ad[4] = {q0, q1, q0, q1};
+#pragma unroll
+        for (int o = 0; o < OT; ++o) {
+            float cm[4] = {0.f, 0.f, 0.f, 0.f};
+            mma(cm, ad, xs[o][0], xs[o][1]);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[o][j] += fmaf(m[o][j], 16777216.f, -512.f * cm[j]);
         }
     }
 };
@@ -684,6 +830,169 @@ struct Q4K {
     }
 };
 
+// ------------------------------------------------- Q4_K, one activation row
+// The one-row mapping for superblocks: lane (g, t) owns nibble group t (32
+// code bytes: sub-block 2t in the low nibbles, 2t+1 in the high nibbles) of
+// weight rows g, g+8, and B is block-diagonal as in the Q4_0/Q8_0 one-row
+// mapping (column 2t+p = part p of lane t's activations), so C[r][2t+p] is a
+// plain dot product of codes and activations per sub-block.  Two chains per
+// nibble half keep the low-nibble (sub-block 2t) and high-nibble (2t+1)
+// results apart; the high-nibble k-steps take x / 16, matching their
+// in-place codes (16u * 2^-24).  Per row, in fp32:
+//   y = d * 2^24 * (sc_2t C_2t + sc_2t+1 C_2t+1) - dmin * (m_2t X_2t + m_2t+1 X_2t+1)
+// with X_j the sub-block sums of the scaled activations.  k-slots (2t, 2t+1)
+// and (2t+8, 2t+9) of k-step (word i, half h) hold code bytes (0, 2) and
+// (1, 3) of word i, i.e. elements (4i, 4i+2) and (4i+1, 4i+3) of sub-block
+// 2t+h.
+template <int XT>
+struct OneRowK {
+    static constexpr int P = XFrag<XT>::parts;
+    uint32_t xb[8][2][2];   // [code word][nibble half][reg]: this lane's column of B
+    float xsum[2];          // X_2t, X_2t+1
+    float inv;
+
+    __device__ static __forceinline__ float2 load2(const void *x, long e) {
+        if constexpr (XT == X_F32) {
+            return __ldg(reinterpret_cast<const float2 *>(static_cast<const float *>(x) + e));
+        } else {
+            const uint32_t u = __ldg(reinterpret_cast<const uint32_t *>(static_cast<const uint16_t *>(x) + e));
+            if constexpr (XT == X_F16)
+                return make_float2(f16_bits_to_float(u), f16_bits_to_float(u >> 16));
+            else
+                return make_float2(bf16_bits_to_float(u), bf16_bits_to_float(u >> 16));
+        }
+    }
+    __device__ static __forceinline__ uint32_t part(float a, float b, int p) {
+        const uint32_t hi = pack_f16x2(a, b);
+        if (P == 1 || p == 0) return hi;
+        return pack_f16x2(a - f16_bits_to_float(hi), b - f16_bits_to_float(hi >> 16));
+    }
+
+    // Each lane packs 8 activations (code words 2q, 2q+1 of sub-block j) into
+    // the staging area [p][t][h][word][reg]; owner lanes then read their column.
+    __device__ __forceinline__ void load_x(const void *x, int M, int K, long k0, int lane, uint32_t stage0,
+                                           uint32_t pstride) {
+        (void)M;
+        (void)K;
+        const int j = lane >> 2, q = lane & 3;   // sub-block, quarter
+        float2 v[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = load2(x, k0 + 32 * j + 8 * q + 2 * i);
+        float mx = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mx = fmaxf(mx, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
+        float s;
+        warp_scale<XT>(mx, s, inv);
+        float sum = 0.f;
+        const float sb = (j & 1) ? s * 0.0625f : s;   // high-nibble sub-blocks: x / 16
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            sum += v[i].x * s + v[i].y * s;
+            v[i].x *= sb;
+            v[i].y *= sb;
+        }
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+#pragma unroll
+        for (int p = 0; p < P; ++p) {
+            // word 2q: elements 8q..8q+3 -> reg 0 = (e0, e2), reg 1 = (e1, e3); word 2q+1 likewise
+            const uint32_t r0 = part(v[0].x, v[1].x, p), r1 = part(v[0].y, v[1].y, p);
+            const uint32_t r2 = part(v[2].x, v[3].x, p), r3 = part(v[2].y, v[3].y, p);
+            st_shared_v4(stage0 + p * pstride + (uint32_t)((((j >> 1) * 2 + (j & 1)) * 8 + 2 * q) * 2 * 4), r0, r1, r2,
+                         r3);
+        }
+        __syncwarp();
+        const int g = lane >> 2, t = lane & 3;
+        xsum[0] = __shfl_sync(0xffffffffu, sum, 8 * t);
+        xsum[1] = __shfl_sync(0xffffffffu, sum, 8 * t + 4);
+        if ((g >> 1) == t && (g & 1) < P) {
+            const uint32_t src = stage0 + (g & 1) * pstride + (uint32_t)(t * 128);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {   // [h][word pair]
+                const uint4 u = lds128(src + 16 * i);
+                const int h = i >> 2, w = 2 * (i & 3);
+                xb[w][h][0] = u.x;
+                xb[w][h][1] = u.y;
+                xb[w + 1][h][0] = u.z;
+                xb[w + 1][h][1] = u.w;
+            }
+        } else {
+#pragma unroll
+            for (int w = 0; w < 8; ++w)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) xb[w][h][0] = xb[w][h][1] = 0u;
+        }
+        __syncwarp();
+    }
+
+    // Byte k of w as an exact float (0..255): 2^23 + b, minus 2^23.
+    __device__ static __forceinline__ float byte_f(uint32_t w, uint32_t sel) {
+        return __uint_as_float(prmt(w, 0x4B000000u, sel)) - 8388608.f;
+    }
+
+    __device__ __forceinline__ void compute(uint32_t tb, float (&acc)[1][4], int lane) const {
+        const int g = lane >> 2, t = lane & 3;
+        const uint32_t r0 = tb + g * 144, r1 = r0 + 8 * 144;   // rows g, g+8
+        uint32_t w[2][8];
+        {
+            const uint4 a0 = lds128(r0 + 16 + 32 * t), b0 = lds128(r0 + 32 + 32 * t);
+            const uint4 a1 = lds128(r1 + 16 + 32 * t), b1 = lds128(r1 + 32 + 32 * t);
+            w[0][0] = a0.x; w[0][1] = a0.y; w[0][2] = a0.z; w[0][3] = a0.w;
+            w[0][4] = b0.x; w[0][5] = b0.y; w[0][6] = b0.z; w[0][7] = b0.w;
+            w[1][0] = a1.x; w[1][1] = a1.y; w[1][2] = a1.z; w[1][3] = a1.w;
+            w[1][4] = b1.x; w[1][5] = b1.y; w[1][6] = b1.z; w[1][7] = b1.w;
+        }
+        float c[2][2][4];   // [nibble half][word parity]
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) c[h][e][j] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t s0 = w[0][i] >> 8, s1 = w[1][i] >> 8;
+            const uint32_t al[4] = {w[0][i] & 0x000F000Fu, w[1][i] & 0x000F000Fu, s0 & 0x000F000Fu, s1 & 0x000F000Fu};
+            const uint32_t ah[4] = {w[0][i] & 0x00F000F0u, w[1][i] & 0x00F000F0u, s0 & 0x00F000F0u, s1 & 0x00F000F0u};
+            mma(c[0][i & 1], al, xb[i][0][0], xb[i][0][1]);
+            mma(c[1][i & 1], ah, xb[i][1][0], xb[i][1][1]);
+        }
+        // sub-block results per row (units of 2^-24): columns 2t (part 0) and 2t+1 (part 1)
+        float C[2][2];   // [row][half]
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            C[0][h] = (c[h][0][0] + c[h][1][0]);
+            C[1][h] = (c[h][0][2] + c[h][1][2]);
+            if (P == 2) {
+                C[0][h] += (c[h][0][1] + c[h][1][1]);
+                C[1][h] += (c[h][0][3] + c[h][1][3]);
+            }
+        }
+        // scales and mins of sub-blocks 2t, 2t+1 (6-bit, packed as in the format)
+        const uint32_t sel_lo = 0x7540u | (uint32_t)(2 * (t & 1)), sel_hi = sel_lo + 1u;
+        float y[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const uint4 hd = lds128(r ? r1 : r0);
+            const uint32_t s0 = hd.y, s1 = hd.z, s2 = hd.w;
+            const uint32_t sc_w = (t < 2) ? (s0 & 0x3F3F3F3Fu) : ((s2 & 0x0F0F0F0Fu) | ((s0 >> 2) & 0x30303030u));
+            const uint32_t m_w = (t < 2) ? (s1 & 0x3F3F3F3Fu) : (((s2 >> 4) & 0x0F0F0F0Fu) | ((s1 >> 2) & 0x30303030u));
+            const float sc0 = byte_f(sc_w, sel_lo), sc1 = byte_f(sc_w, sel_hi);
+            const float m0 = byte_f(m_w, sel_lo), m1 = byte_f(m_w, sel_hi);
+            const float d = f16_bits_to_float(hd.x) * 16777216.f, dmin = f16_bits_to_float(hd.x >> 16);
+            const float a = fmaf(sc1, C[r][1], sc0 * C[r][0]);
+            const float b = fmaf(m1, xsum[1], m0 * xsum[0]);
+            y[r] = fmaf(d, a, -dmin * b);
+        }
+        y[0] += __shfl_xor_sync(0xffffffffu, y[0], 1);
+        y[1] += __shfl_xor_sync(0xffffffffu, y[1], 1);
+        y[0] += __shfl_xor_sync(0xffffffffu, y[0], 2);
+        y[1] += __shfl_xor_sync(0xffffffffu, y[1], 2);
+        acc[0][0] += y[0];
+        acc[0][2] += y[1];
+    }
+};
+
 // FMT x activation type x n8 tiles x one-row mapping
 template <int FMT, int XT, int NT, bool ONE>
 struct GemvImpl;
@@ -697,8 +1006,16 @@ template <int XT>
 struct GemvImpl<F_Q8_0, XT, 1, true> : OneRow<F_Q8_0, XT> {};
 template <int XT, int NT>
 struct GemvImpl<F_Q4_K, XT, NT, false> : Q4K<XT, NT> {};
+template <int XT>
+struct GemvImpl<F_Q4_K, XT, 1, true> : OneRowK<XT> {};
 
 // ------------------------------------------------------------------ kernel
+// Registers per thread: 96 lets a CTA run 16 compute warps (+ producer and
+// reducer); kernels whose activation fragments need more take 128 and at most
+// 14 compute warps.  fp32 Q4_0 with two column tiles fits 96 (a few bytes of
+// prologue spill).
+constexpr int gemv_max_regs(int fmt, int xt, int nt) { return (nt == 1 || (fmt == F_Q4_0 && xt == X_F32)) ? 96 : 128; }
+
 // blockDim = (NW + 2) * 32: warps 0..NW-1 compute, warp NW produces (TMA),
 // warp NW+1 reduces.  A dedicated producer refills a stage the moment its
 // consumers release it, and a dedicated reducer keeps the per-tile reduction
@@ -711,11 +1028,15 @@ struct GemvImpl<F_Q4_K, XT, NT, false> : Q4K<XT, NT> {};
 // Shared memory: stages * NW * 16 * CB bytes of packed boxes, stages * NW *
 // 16 * 8NT fp32 partials, then 3 * stages mbarriers.
 template <int FMT, int XT, int NT, bool ONE>
-__global__ void __maxnreg__(NT == 1 ? 96 : 128)
+__global__ void __maxnreg__(gemv_max_regs(FMT, XT, NT))
     gemv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const GemvArgs a) {
     constexpr int CB = FmtInfo<FMT>::chunk_bytes;
     constexpr int BOX = GEMV_ROWS * CB;
-    constexpr int RED = GEMV_ROWS * 8 * NT;  // floats per warp per stage
+    // fp32 activations keep one output tile (their two fp16 parts are merged
+    // before the reducer: in the MMA chain for NT = 2, by the reducer for NT = 1)
+    constexpr int OT = (XT == X_F32) ? 1 : NT;
+    constexpr bool MERGED = (XT == X_F32 && NT == 1 && !ONE && FMT == F_Q4_0);
+    constexpr int RED = GEMV_ROWS * 8 * OT;  // floats per warp per stage
     extern __shared__ __align__(128) uint8_t smem[];
 
     const int NW = blockDim.x / 32 - 2;
@@ -788,7 +1109,10 @@ __global__ void __maxnreg__(NT == 1 ? 96 : 128)
             for (int o = lane; o < nout; o += 32) {
                 const int r = o % GEMV_ROWS, b = o / GEMV_ROWS;
                 float sum = 0.f;
-                for (int w = 0; w < nact; ++w) sum += ldsf(rs + 4 * (w * RED + r * (8 * NT) + b));
+                for (int w = 0; w < nact; ++w) {
+                    sum += ldsf(rs + 4 * (w * RED + r * (8 * OT) + b));
+                    if (MERGED) sum += ldsf(rs + 4 * (w * RED + r * (8 * OT) + b + 4));
+                }
                 const int row = tile * GEMV_ROWS + r;
                 if (row < N) {
                     if (S == 1)
@@ -849,14 +1173,14 @@ __global__ void __maxnreg__(NT == 1 ? 96 : 128)
             for (int j = 0; j < 4; ++j) acc[nt][j] = 0.f;
         impl.compute(smem_u32(boxes) + (uint32_t)((s * NW + warp) * BOX), acc, lane);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+        for (int nt = 0; nt < OT; ++nt)
 #pragma unroll
             for (int j = 0; j < 4; ++j) acc[nt][j] *= impl.inv;   // undo the activation scale (exact)
         const uint32_t rw = smem_u32(red) + (uint32_t)(((s * NW + warp) * RED) * 4);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            sts_f2(rw + 4 * (g * (8 * NT) + 8 * nt + 2 * t), acc[nt][0], acc[nt][1]);
-            sts_f2(rw + 4 * ((g + 8) * (8 * NT) + 8 * nt + 2 * t), acc[nt][2], acc[nt][3]);
+        for (int nt = 0; nt < OT; ++nt) {
+            sts_f2(rw + 4 * (g * (8 * OT) + 8 * nt + 2 * t), acc[nt][0], acc[nt][1]);
+            sts_f2(rw + 4 * ((g + 8) * (8 * OT) + 8 * nt + 2 * t), acc[nt][2], acc[nt][3]);
         }
         __syncwarp();
         if (lane == 0) {

@@ -104,11 +104,10 @@ template <int FMT, int XT>
 static cudaError_t launch_nt(int nt, bool one, const CUtensorMap &map, const GemvArgs &a, int ctas, int nw,
                              size_t smem, cudaStream_t st) {
     if (nt == 1) {
-        if constexpr (FMT != F_Q4_K)
-            if (one) return launch<FMT, XT, 1, true>(map, a, ctas, nw, smem, st);
+        if (one) return launch<FMT, XT, 1, true>(map, a, ctas, nw, smem, st);
         return launch<FMT, XT, 1, false>(map, a, ctas, nw, smem, st);
     }
-    if constexpr (XT != X_F32) return launch<FMT, XT, 2, false>(map, a, ctas, nw, smem, st);
+    if constexpr (XT != X_F32 || FMT == F_Q4_0) return launch<FMT, XT, 2, false>(map, a, ctas, nw, smem, st);
     return cudaErrorInvalidValue;
 }
 
@@ -127,9 +126,9 @@ static cudaError_t dispatch(int wf, int xt, int nt, bool one, const CUtensorMap 
     return cudaErrorInvalidValue;
 }
 
-static size_t smem_bytes(int wf, int nw, int stages, int nt) {
+static size_t smem_bytes(int wf, int nw, int stages, int ot) {
     const int cb = (wf == LWQ_Q8_0) ? 272 : 144;
-    return (size_t)stages * nw * GEMV_ROWS * cb + (size_t)stages * nw * GEMV_ROWS * 8 * nt * 4 +
+    return (size_t)stages * nw * GEMV_ROWS * cb + (size_t)stages * nw * GEMV_ROWS * 8 * ot * 4 +
            (size_t)3 * stages * 8;
 }
 
@@ -192,8 +191,11 @@ extern "C" int lwq_matmul_noalloc(int fmt, const void *Wq, const void *x, float 
         a.stages = cfg.stages;
         a.timeout_ns = kTimeoutNs;
         a.overlap = 0;
-        const int nt = mg <= 8 ? 1 : 2;
-        cudaError_t e = dispatch(wf, xt, nt, mg == 1, map, a, cfg.ctas, cfg.warps, smem_bytes(wf, cfg.warps, cfg.stages, nt), st);
+        // n8 column tiles, as lwq_matmul picks them; fp32 activations keep one output tile
+        const int nt = (xt == X_F32) ? ((wf == LWQ_Q4_0 && mg > 4) ? 2 : 1) : (mg <= 8 ? 1 : 2);
+        const int ot = (xt == X_F32) ? 1 : nt;
+        cudaError_t e = dispatch(wf, xt, nt, mg == 1, map, a, cfg.ctas, cfg.warps,
+                                 smem_bytes(wf, cfg.warps, cfg.stages, ot), st);
         if (e != cudaSuccess) return LWQ_ERR_CUDA;
     }
     return LWQ_OK;

@@ -44,6 +44,41 @@ def test_small_shapes(dev, w, a, M, N, K):
     check_full(w, a, M, N, K, dev, seed=M * 1000 + N)
 
 
+@pytest.mark.parametrize("w,a", FAST)
+@pytest.mark.parametrize("M", [2, 4, 5, 6, 7, 9, 15])
+def test_every_column_layout(dev, w, a, M):
+    # row counts at and around the boundaries of the GEMV's column layouts
+    # (fp32: 4 rows x 2 parts in one tile, then one tile per part; 16-bit: 8 rows per tile)
+    check_full(w, a, M, 45, 1024, dev, seed=100 + M)
+
+
+def _scaled_problem(w, a, M, N, K, seed, e):
+    """make_problem with the activations multiplied by 2**e (exact in every activation type)."""
+    Wq, x = inputs.make_problem(w, a, M, N, K, seed=seed)
+    if a == "f32":
+        return Wq, (x * np.float32(2.0 ** e)).astype(np.float32)
+    if a == "f16":
+        v = x.view(np.float16).astype(np.float32) * np.float32(2.0 ** e)
+        assert np.all(np.isfinite(v.astype(np.float16)))
+        return Wq, v.astype(np.float16).view(np.uint16)
+    v = (x.astype(np.uint32) << 16).view(np.float32) * np.float32(2.0 ** e)
+    return Wq, (v.view(np.uint32) >> 16).astype(np.uint16)
+
+
+@pytest.mark.parametrize("w,a,e", [("q4_0", "f32", -40), ("q4_0", "f32", 40), ("q4_0", "f16", -12),
+                                   ("q4_0", "f16", 12), ("q8_0", "f16", -12), ("q4_k", "f16", 12),
+                                   ("q4_0", "bf16", -60), ("q8_0", "f32", 30)])
+@pytest.mark.parametrize("M", [1, 3, 8])
+def test_activation_magnitudes(dev, w, a, e, M):
+    # the per-warp power-of-two activation scale must hold tiny and huge inputs
+    N, K = 40, 1024
+    Wq, x = _scaled_problem(w, a, M, N, K, 11 + M, e)
+    y = run_gpu(w, a, Wq, x, M, N, K, dev).cpu().numpy()
+    y_ref, den = oracle.matmul(w, Wq, x, act=a)
+    err = oracle.normalised_error(y, y_ref, den)
+    assert err <= TOL_GEMV, f"{w}/{a} x*2^{e} M={M}: err {err:.3e}"
+
+
 @pytest.mark.parametrize("w,a", [("q4_0", "f32"), ("q8_0", "f16"), ("q4_0", "bf16")])
 @pytest.mark.parametrize("M,N,K", [(1, 9, 32), (2, 40, 96), (4, 7, 320), (17, 33, 480)])
 def test_k_not_multiple_of_256(dev, w, a, M, N, K):
