@@ -306,15 +306,18 @@ cudaError_t dispatch_simple(int wf, int xt, const uint8_t *W, const void *x, flo
     return cudaErrorInvalidValue;
 }
 
-int encode_weight_map(CUtensorMap *map, const void *Wq, int wf, int N, long rb) {
+// The GEMV's view of Wq: 3-D, (8-byte word of a 256-weight chunk, weight row,
+// chunk), strides (row_bytes, chunk_bytes); a box of (all words, 16 rows, cps
+// chunks) lands as cps consecutive [16 rows][chunk] boxes.
+int encode_weight_map(CUtensorMap *map, const void *Wq, int wf, int N, long rb, int cps) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return LWQ_ERR_CUDA;
     const int cb = (wf == LWQ_Q8_0) ? 272 : 144;
-    cuuint64_t dims[2] = {(cuuint64_t)(rb / 2), (cuuint64_t)N};
-    cuuint64_t strides[1] = {(cuuint64_t)rb};
-    cuuint32_t box[2] = {(cuuint32_t)(cb / 2), (cuuint32_t)GEMV_ROWS};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(Wq), dims, strides, box, estr,
+    cuuint64_t dims[3] = {(cuuint64_t)(cb / 8), (cuuint64_t)N, (cuuint64_t)(rb / cb)};
+    cuuint64_t strides[2] = {(cuuint64_t)rb, (cuuint64_t)cb};
+    cuuint32_t box[3] = {(cuuint32_t)(cb / 8), (cuuint32_t)GEMV_ROWS, (cuuint32_t)cps};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, const_cast<void *>(Wq), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? LWQ_OK : LWQ_ERR_CUDA;
@@ -430,11 +433,11 @@ int run(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, c
         if (!ds.registered) return LWQ_ERR_NOT_INITIALIZED;
         if (ds.ws_bytes < p.ws_need) return LWQ_ERR_WORKSPACE_TOO_SMALL;
     }
-    CUtensorMap map;
-    if ((rc = encode_weight_map(&map, Wq, wf, N, rb))) return rc;
     const int nchunks = K / 256;
     const int S = p.cfg.splits;
     const int cps = (nchunks + S - 1) / S;
+    CUtensorMap map;
+    if ((rc = encode_weight_map(&map, Wq, wf, N, rb, cps))) return rc;
     const int row_tiles = (N + GEMV_ROWS - 1) / GEMV_ROWS;
     for (int m0 = 0; m0 < M; m0 += p.m_group) {
         const int mg = (M - m0) < p.m_group ? (M - m0) : p.m_group;

@@ -4,9 +4,13 @@
 //  * A persistent grid.  CTA (split s, row group r) owns a fixed slice of K
 //    (split-K factor S) and walks the row tiles r, r+G, r+2G, ... (16 weight
 //    rows per tile).
-//  * One producer warp stages, per row tile, one [16 rows][256 weights]
-//    packed box per compute warp with 2-D TMA loads into a ring of shared
-//    memory stages (mbarrier full/empty pairs).
+//  * One producer warp stages, per row tile, the tile's packed rows for all
+//    of the CTA's K chunks with one 3-D TMA load (dimensions: bytes of a
+//    chunk, weight row, chunk), which lands as one [16 rows][256 weights] box
+//    per compute warp, into a ring of shared-memory stages (mbarrier
+//    full/empty pairs).  One load per stage keeps the producer's issue time
+//    small; 2-D boxes of one chunk each cost about as much to issue as a
+//    stage takes to arrive.
 //  * Each compute warp owns one 256-weight "chunk" of K for the whole kernel
 //    and keeps the activations of that chunk in registers, already laid out
 //    as tensor-core B fragments in fp16.  Per row tile it decodes the packed
@@ -193,6 +197,32 @@ __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint3
 // rows, column g = part g >> 2 of row g & 3 (the reducer adds columns b and
 // b + 4); NT = 2 holds up to 8 rows with the two parts in the two tiles, both
 // accumulated into one result (so only the first output tile is written).
+// Two consecutive activations as loaded (fp32 pair, or one word of two
+// 16-bit codes) and as fp32.
+template <int XT>
+struct RawPair {
+    using T = uint32_t;
+    __device__ static __forceinline__ T zero() { return 0u; }
+    __device__ static __forceinline__ T load(const void *x, long off) {
+        return __ldg(reinterpret_cast<const uint32_t *>(static_cast<const uint16_t *>(x) + off));
+    }
+    __device__ static __forceinline__ float2 get(T u) {
+        if constexpr (XT == X_F16)
+            return make_float2(f16_bits_to_float(u), f16_bits_to_float(u >> 16));
+        else
+            return make_float2(bf16_bits_to_float(u), bf16_bits_to_float(u >> 16));
+    }
+};
+template <>
+struct RawPair<X_F32> {
+    using T = float2;
+    __device__ static __forceinline__ T zero() { return make_float2(0.f, 0.f); }
+    __device__ static __forceinline__ T load(const void *x, long off) {
+        return __ldg(reinterpret_cast<const float2 *>(static_cast<const float *>(x) + off));
+    }
+    __device__ static __forceinline__ float2 get(T v) { return v; }
+};
+
 template <int XT, int NT>
 struct Q40 {
     static constexpr int P = XFrag<XT>::parts;
@@ -222,6 +252,21 @@ struct Q40 {
         const uint32_t hi = pack_f16x2(a, b);
         if (P == 1 || p == 0) return hi;
         return pack_f16x2(a - f16_bits_to_float(hi), b - f16_bits_to_float(hi >> 16));
+    }
+
+    // The two element pairs of this lane's writer units in block b (zeros for absent rows).
+    __device__ static __forceinline__ void fetch_round(const void *x, int M, int K, long k0, int lane, int b,
+                                                       typename RawPair<XT>::T (&r)[(MERGED ? 4 : (PART_TILES ? 8 : 8 * NT)) / 4][2]) {
+#pragma unroll
+        for (int k = 0; k < (MERGED ? 4 : (PART_TILES ? 8 : 8 * NT)) / 4; ++k) {
+            const int u = lane + 32 * k, m = u >> 3, tu = (u >> 1) & 3, h = u & 1;
+            r[k][0] = r[k][1] = RawPair<XT>::zero();
+            if (m < M) {
+                const long e = (long)m * K + k0 + 32 * b + 16 * h;
+                r[k][0] = RawPair<XT>::load(x, e + cb0(b & 1, tu));
+                r[k][1] = RawPair<XT>::load(x, e + cb2(b & 1, tu));
+            }
+        }
     }
 
     // Activation rows in this pass's column tiles, and writer units per lane:
@@ -282,18 +327,20 @@ struct Q40 {
             const bool part0 = MERGED ? (g < 4) : (PART_TILES ? nt == 0 : true);
             crow[nt] = (part0 && row < M) ? row : -1;
         }
-        // pass 2, one block per round
+        // pass 2, one block per round.  Each round ends in shared-memory stores
+        // and a warp barrier that loads may not pass, so the raw activations of
+        // round b + 2 are requested at the start of round b.
+        using Raw = typename RawPair<XT>::T;
+        Raw raw[3][UPL][2];
+#pragma unroll
+        for (int b = 0; b < 2; ++b) fetch_round(x, M, K, k0, lane, b, raw[b]);
 #pragma unroll
         for (int b = 0; b < 8; ++b) {
+            if (b + 2 < 8) fetch_round(x, M, K, k0, lane, b + 2, raw[(b + 2) % 3]);
 #pragma unroll
             for (int k = 0; k < UPL; ++k) {
                 const int u = lane + 32 * k, m = u >> 3, tu = (u >> 1) & 3, h = u & 1;
-                float2 p = make_float2(0.f, 0.f), q = make_float2(0.f, 0.f);
-                if (m < M) {
-                    const long e = (long)m * K + k0 + 32 * b + 16 * h;
-                    p = load2(x, e + cb0(b & 1, tu));
-                    q = load2(x, e + cb2(b & 1, tu));
-                }
+                float2 p = RawPair<XT>::get(raw[b % 3][k][0]), q = RawPair<XT>::get(raw[b % 3][k][1]);
                 // high-nibble step: x / 16 (exact: a power of two)
                 const float sc = h ? s * 0.0625f : s;
                 p.x *= sc;
@@ -611,10 +658,7 @@ struct OneRow {
             y0 = fmaf(d0, fmaf(S0, 16777216.f, corr[hb]), y0);
             y1 = fmaf(d1, fmaf(S1, 16777216.f, corr[hb]), y1);
         }
-        y0 += __shfl_xor_sync(0xffffffffu, y0, 1);
-        y1 += __shfl_xor_sync(0xffffffffu, y1, 1);
-        y0 += __shfl_xor_sync(0xffffffffu, y0, 2);
-        y1 += __shfl_xor_sync(0xffffffffu, y1, 2);
+        // lane t's share of rows g, g+8 goes to column 2t; the reducer adds the four
         acc[0][0] += y0;
         acc[0][2] += y1;
     }
@@ -984,10 +1028,7 @@ struct OneRowK {
             const float b = fmaf(m1, xsum[1], m0 * xsum[0]);
             y[r] = fmaf(d, a, -dmin * b);
         }
-        y[0] += __shfl_xor_sync(0xffffffffu, y[0], 1);
-        y[1] += __shfl_xor_sync(0xffffffffu, y[1], 1);
-        y[0] += __shfl_xor_sync(0xffffffffu, y[0], 2);
-        y[1] += __shfl_xor_sync(0xffffffffu, y[1], 2);
+        // lane t's share of rows g, g+8 goes to column 2t; the reducer adds the four
         acc[0][0] += y[0];
         acc[0][2] += y[1];
     }
@@ -1079,10 +1120,10 @@ __global__ void __maxnreg__(gemv_max_regs(FMT, XT, NT))
             uint32_t ph = 0;
             for (int tile = rgrp; tile < a.row_tiles; tile += G, ++it) {
                 if (it >= stages && !mbar_wait(&empty[s], ph ^ 1u, a.timeout_ns, DEVERR_GEMV_WAIT)) break;
-                mbar_arrive_expect_tx(&full[s], (uint32_t)(nact * BOX));
-                for (int w = 0; w < nact; ++w)
-                    tma_load_2d(boxes + ((size_t)s * NW + w) * BOX, &wmap, &full[s], (c_begin + w) * (CB / 2),
-                                tile * GEMV_ROWS);
+                // one 3-D box per stage: [chunks of this split][16 rows][chunk bytes]; the last
+                // split's box may run past the last chunk, where it reads zeros (no traffic)
+                mbar_arrive_expect_tx(&full[s], (uint32_t)(a.chunks_per_split * BOX));
+                tma_load_3d(boxes + (size_t)s * NW * BOX, &wmap, &full[s], 0, tile * GEMV_ROWS, c_begin);
                 if (++s == stages) {
                     s = 0;
                     ph ^= 1u;
@@ -1097,28 +1138,78 @@ __global__ void __maxnreg__(gemv_max_regs(FMT, XT, NT))
     }
 
     if (warp == NW + 1) {
-        // ---------------- reducer: y and the workspace only after the preceding work completed
+        // ---------------- reducer: y and the workspace only after the preceding work completed.
+        // Lane (r, half) sums 4-column groups half, half + 2, ... of row r over the
+        // compute warps with 16-byte loads, in warp order (deterministic).
         pdl_wait();
         const int M = a.M, N = a.N;
-        const int nout = GEMV_ROWS * M;  // outputs per tile: 16 rows x M columns
+        constexpr int GPL = OT;   // column groups per lane: 2 * OT groups over two half-warps
+        const int r = lane & 15, half = lane >> 4;
         int s = 0;
         uint32_t ph = 0;
         for (int tile = rgrp; tile < a.row_tiles; tile += G) {
             if (!mbar_wait(&redfull[s], ph, a.timeout_ns, DEVERR_GEMV_WAIT)) break;
-            const uint32_t rs = smem_u32(red) + (uint32_t)(s * NW * RED * 4);
-            for (int o = lane; o < nout; o += 32) {
-                const int r = o % GEMV_ROWS, b = o / GEMV_ROWS;
-                float sum = 0.f;
-                for (int w = 0; w < nact; ++w) {
-                    sum += ldsf(rs + 4 * (w * RED + r * (8 * OT) + b));
-                    if (MERGED) sum += ldsf(rs + 4 * (w * RED + r * (8 * OT) + b + 4));
+            const uint32_t rs = smem_u32(red) + (uint32_t)(s * NW * RED * 4) + (uint32_t)(r * 8 * OT * 4);
+            float4 v[GPL];
+#pragma unroll
+            for (int j = 0; j < GPL; ++j) v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+            // four warps' loads in flight at a time; the sums still run in warp order
+            int w = 0;
+#pragma unroll 1
+            for (; w + 4 <= nact; w += 4) {
+                uint4 u[4][GPL];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < GPL; ++j) u[i][j] = lds128(rs + (uint32_t)((w + i) * RED * 4 + (half + 2 * j) * 16));
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < GPL; ++j) {
+                        v[j].x += __uint_as_float(u[i][j].x);
+                        v[j].y += __uint_as_float(u[i][j].y);
+                        v[j].z += __uint_as_float(u[i][j].z);
+                        v[j].w += __uint_as_float(u[i][j].w);
+                    }
+            }
+#pragma unroll 1
+            for (; w < nact; ++w) {
+#pragma unroll
+                for (int j = 0; j < GPL; ++j) {
+                    const uint4 u = lds128(rs + (uint32_t)(w * RED * 4 + (half + 2 * j) * 16));
+                    v[j].x += __uint_as_float(u.x);
+                    v[j].y += __uint_as_float(u.y);
+                    v[j].z += __uint_as_float(u.z);
+                    v[j].w += __uint_as_float(u.w);
                 }
-                const int row = tile * GEMV_ROWS + r;
-                if (row < N) {
-                    if (S == 1)
-                        a.y[(size_t)b * N + row] = sum;
-                    else
-                        a.partial[((size_t)split * M + b) * N + row] = sum;
+            }
+            if (ONE) {
+                // one-row mappings leave lane t's share of each row in column 2t
+                float t = v[0].x + v[0].z;
+                t += __shfl_xor_sync(0xffffffffu, t, 16);
+                v[0].x = t;
+            } else if (MERGED) {
+                // fp32 parts: column b + 4 holds the lo half of column b
+                v[0].x += __shfl_xor_sync(0xffffffffu, v[0].x, 16);
+                v[0].y += __shfl_xor_sync(0xffffffffu, v[0].y, 16);
+                v[0].z += __shfl_xor_sync(0xffffffffu, v[0].z, 16);
+                v[0].w += __shfl_xor_sync(0xffffffffu, v[0].w, 16);
+            }
+            const int row = tile * GEMV_ROWS + r;
+            if (row < N && (half == 0 || !(ONE || MERGED))) {
+#pragma unroll
+                for (int j = 0; j < GPL; ++j) {
+                    const float o[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int b = 4 * (half + 2 * j) + i;
+                        if (b < M) {
+                            if (S == 1)
+                                a.y[(size_t)b * N + row] = o[i];
+                            else
+                                a.partial[((size_t)split * M + b) * N + row] = o[i];
+                        }
+                    }
                 }
             }
             __syncwarp();
@@ -1132,9 +1223,9 @@ __global__ void __maxnreg__(gemv_max_regs(FMT, XT, NT))
                 old = __shfl_sync(0xffffffffu, old, 0);
                 if (old == (unsigned)(S - 1)) {
                     __threadfence();
-                    for (int o = lane; o < nout; o += 32) {
-                        const int r = o % GEMV_ROWS, b = o / GEMV_ROWS;
-                        const int row = tile * GEMV_ROWS + r;
+                    for (int o = lane; o < GEMV_ROWS * M; o += 32) {
+                        const int rr = o % GEMV_ROWS, b = o / GEMV_ROWS;
+                        const int row = tile * GEMV_ROWS + rr;
                         if (row < N) {
                             float sum = 0.f;
                             for (int sp = 0; sp < S; ++sp) sum += __ldcg(&a.partial[((size_t)sp * M + b) * N + row]);

@@ -157,22 +157,23 @@ extern "C" int lwq_matmul_noalloc(int fmt, const void *Wq, const void *x, float 
     EncodeTiledFn enc = encoder();
     if (!enc) return LWQ_ERR_CUDA;
     const long rb = (long)lwq_row_bytes(fmt, K);
+    const int nchunks = K / 256;
+    const int cps = (nchunks + S - 1) / S;
     CUtensorMap map;
     {
+        // (8-byte word of a chunk, weight row, chunk); one box per stage, as lwq_matmul's
         const int cb = (wf == LWQ_Q8_0) ? 272 : 144;
-        cuuint64_t dims[2] = {(cuuint64_t)(rb / 2), (cuuint64_t)N};
-        cuuint64_t strides[1] = {(cuuint64_t)rb};
-        cuuint32_t box[2] = {(cuuint32_t)(cb / 2), (cuuint32_t)GEMV_ROWS};
-        cuuint32_t estr[2] = {1, 1};
-        if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(Wq), dims, strides, box, estr,
+        cuuint64_t dims[3] = {(cuuint64_t)(cb / 8), (cuuint64_t)N, (cuuint64_t)nchunks};
+        cuuint64_t strides[2] = {(cuuint64_t)rb, (cuuint64_t)cb};
+        cuuint32_t box[3] = {(cuuint32_t)(cb / 8), (cuuint32_t)GEMV_ROWS, (cuuint32_t)cps};
+        cuuint32_t estr[3] = {1, 1, 1};
+        if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, const_cast<void *>(Wq), dims, strides, box, estr,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return LWQ_ERR_CUDA;
     }
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const size_t xelem = (xt == X_F32) ? 4 : 2;
-    const int nchunks = K / 256;
-    const int cps = (nchunks + S - 1) / S;
     for (int m0 = 0; m0 < M; m0 += m_group) {
         const int mg = (M - m0) < m_group ? (M - m0) : m_group;
         if (S > 1 && cudaMemsetAsync(scratch, 0, (size_t)row_tiles * 4, st) != cudaSuccess) return LWQ_ERR_CUDA;
