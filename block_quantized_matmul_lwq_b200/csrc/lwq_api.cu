@@ -123,16 +123,11 @@ bool tc_gemv_eligible(int wf, int xt, long K) {
     return K % 256 == 0;
 }
 
-// Workspace layout: [kCounterBytes of per-row-tile arrival counters][fp32
-// split-K partials].  The counter region has a fixed size so that no call's
-// partials ever overlap another call's counters (counters return to zero at
-// the end of every call).
-constexpr size_t kCounterBytes = 64 * 1024;
-constexpr int kMaxSplitTiles = (int)(kCounterBytes / 4);
-
+// Workspace layout: fp32 split-K partials [S][m_group][N].  Nothing in it
+// needs to start at any particular value.
 size_t splitk_ws(int S, int m, int N) {
     if (S <= 1) return 0;
-    return kCounterBytes + (size_t)S * m * N * 4;
+    return (size_t)S * m * N * 4;
 }
 
 int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Plan *p) {
@@ -189,7 +184,6 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
     while (stages > 2 && gemv_smem(wf, nw, stages, gemv_ot(xt, p->nt)) > kSmemLimit) --stages;
     if (stages < 2 || gemv_smem(wf, nw, stages, gemv_ot(xt, p->nt)) > kSmemLimit) return LWQ_ERR_UNSUPPORTED;
     const int row_tiles = (N + GEMV_ROWS - 1) / GEMV_ROWS;
-    if (S > 1 && row_tiles > kMaxSplitTiles) return LWQ_ERR_UNSUPPORTED;
     int groups = force && force->ctas ? force->ctas / S : sms / S;
     if (groups < 1) groups = 1;
     if (groups > row_tiles) groups = row_tiles;
@@ -444,8 +438,7 @@ int run(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, c
         GemvArgs a;
         a.x = static_cast<const uint8_t *>(x) + (size_t)m0 * K * xelem;
         a.y = y + (size_t)m0 * N;
-        a.counters = static_cast<unsigned *>(ds.ws);
-        a.partial = reinterpret_cast<float *>(static_cast<uint8_t *>(ds.ws) + kCounterBytes);
+        a.partial = static_cast<float *>(ds.ws);
         a.M = mg;
         a.N = N;
         a.K = K;
@@ -461,6 +454,13 @@ int run(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, c
                                          gemv_smem(wf, p.cfg.warps, p.cfg.stages, gemv_ot(xt, nt)), st);
         if (e != cudaSuccess) return LWQ_ERR_CUDA;
         ++launches;
+        if (S > 1) {
+            const long mn = (long)mg * N;
+            e = launch_k(gemv_splitk_sum_kernel, splitk_sum_blocks(mn), 256, 0, st, true,
+                         static_cast<const float *>(a.partial), a.y, S, mn);
+            if (e != cudaSuccess) return LWQ_ERR_CUDA;
+            ++launches;
+        }
     }
     t_last_launches = launches;
     return LWQ_OK;
@@ -515,8 +515,6 @@ int lwq_init(void *d_workspace, size_t bytes) {
     if (rc) return rc;
     if (bytes > 0 && (!d_workspace || !aligned16(d_workspace))) return d_workspace ? LWQ_ERR_MISALIGNED : LWQ_ERR_INVALID_ARG;
     std::lock_guard<std::mutex> lk(g_mu);
-    if (bytes > 0 && cudaMemset(d_workspace, 0, bytes) != cudaSuccess) return LWQ_ERR_CUDA;
-    if (cudaDeviceSynchronize() != cudaSuccess) return LWQ_ERR_CUDA;
     g_dev[dev].ws = bytes ? d_workspace : nullptr;
     g_dev[dev].ws_bytes = bytes;
     g_dev[dev].registered = true;

@@ -33,9 +33,9 @@
 //    lane owns one nibble group (two sub-blocks); the sub-block scales enter
 //    the fp16 A values exactly (sc*q <= 945), the mins through one more MMA.
 //  * A reducer warp sums the compute warps' partials in a fixed order and
-//    writes y, or, with split-K, fp32 partials to the workspace; the last
-//    split to finish a row tile (per-tile arrival counter) adds the splits
-//    in order and writes y.  Results are bitwise deterministic.
+//    writes y, or, with split-K, fp32 partials to the workspace, which a
+//    small follow-up kernel (a programmatic dependent launch) adds in split
+//    order.  Results are bitwise deterministic.
 //
 // This is the matrix-vector half of the co-designed dequantization in
 // "Resumo Tecnico: Llamas na Web", "3. Design de Shader Consciente de
@@ -66,8 +66,7 @@ struct FmtInfo<F_Q4_K> { static constexpr int chunk_bytes = 144; };
 struct GemvArgs {
     const void *x;
     float *y;
-    float *partial;       // [S][M][N] fp32 (split-K only)
-    unsigned *counters;   // [row_tiles] (split-K only), zero between calls
+    float *partial;       // [S][M][N] fp32 (split-K only; gemv_splitk_sum_kernel adds the splits)
     int M, N, K;
     int nchunks;          // K / 256
     int splits;           // S
@@ -1214,28 +1213,6 @@ __global__ void __maxnreg__(gemv_max_regs(FMT, XT, NT))
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
-            if (S > 1) {
-                // deterministic split-K fix-up: the last split to arrive adds all splits in order
-                __threadfence();
-                __syncwarp();
-                unsigned old = 0;
-                if (lane == 0) old = atomicAdd(&a.counters[tile], 1u);
-                old = __shfl_sync(0xffffffffu, old, 0);
-                if (old == (unsigned)(S - 1)) {
-                    __threadfence();
-                    for (int o = lane; o < GEMV_ROWS * M; o += 32) {
-                        const int rr = o % GEMV_ROWS, b = o / GEMV_ROWS;
-                        const int row = tile * GEMV_ROWS + rr;
-                        if (row < N) {
-                            float sum = 0.f;
-                            for (int sp = 0; sp < S; ++sp) sum += __ldcg(&a.partial[((size_t)sp * M + b) * N + row]);
-                            a.y[(size_t)b * N + row] = sum;
-                        }
-                    }
-                    __syncwarp();
-                    if (lane == 0) a.counters[tile] = 0u;
-                }
-            }
             if (++s == stages) {
                 s = 0;
                 ph ^= 1u;
@@ -1283,6 +1260,42 @@ __global__ void __maxnreg__(gemv_max_regs(FMT, XT, NT))
             ph ^= 1u;
         }
     }
+}
+
+// Split-K: y[i] = sum over s (in order) of partial[s][i], i over the M*N
+// outputs of one pass.  Launched as a programmatic dependent of the GEMV: it
+// waits for the GEMV's partials, and lets the next kernel on the stream start.
+static __global__ void __launch_bounds__(256) gemv_splitk_sum_kernel(const float *__restrict__ partial,
+                                                                     float *__restrict__ y, int S, long mn) {
+    if (threadIdx.x == 0) pdl_launch_dependents();
+    pdl_wait();
+    const long stride = (long)gridDim.x * blockDim.x;
+    if ((mn & 3) == 0) {
+        const long n4 = mn >> 2;
+        for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
+            float4 acc = __ldcg(reinterpret_cast<const float4 *>(partial) + i);
+            for (int sp = 1; sp < S; ++sp) {
+                const float4 v = __ldcg(reinterpret_cast<const float4 *>(partial + (long)sp * mn) + i);
+                acc.x += v.x;
+                acc.y += v.y;
+                acc.z += v.z;
+                acc.w += v.w;
+            }
+            reinterpret_cast<float4 *>(y)[i] = acc;
+        }
+    } else {
+        for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < mn; i += stride) {
+            float acc = __ldcg(partial + i);
+            for (int sp = 1; sp < S; ++sp) acc += __ldcg(partial + (long)sp * mn + i);
+            y[i] = acc;
+        }
+    }
+}
+
+inline int splitk_sum_blocks(long mn) {
+    const long n = ((mn & 3) == 0 ? mn / 4 : mn);
+    long b = (n + 255) / 256;
+    return (int)(b < 1 ? 1 : (b > 1184 ? 1184 : b));
 }
 
 }  // namespace lwq

@@ -11,21 +11,18 @@
 // the library is loaded on a device and held until the process exits.
 //
 // Limits and behaviour:
-//  * The scratch is kScratchBytes (4 MiB): 64 KiB of per-row-tile arrival
-//    counters and the rest for fp32 split-K partial sums.  A call whose
-//    configuration needs more (lwq_workspace_size(fmt, M, N, K) bytes) is
-//    rejected with LWQ_ERR_WORKSPACE_TOO_SMALL; so is a call with more row
-//    tiles than the counter region holds.
+//  * The scratch is kScratchBytes (4 MiB) of fp32 split-K partial sums.  A
+//    call whose configuration needs more (lwq_workspace_size(fmt, M, N, K)
+//    bytes) is rejected with LWQ_ERR_WORKSPACE_TOO_SMALL.
 //  * Only the tensor-core GEMV is offered (M <= 16 and the shapes it takes);
 //    other shapes return LWQ_ERR_UNSUPPORTED.
 //  * The device address of the array is looked up once per device, with that
 //    device current, on the first call made on it.  Make that first call
 //    before any stream capture on the device.
 //  * Every call shares the one array and it keeps the previous call's
-//    contents.  Each call clears the counters it uses (an asynchronous memset
-//    on the caller's stream) before its kernels run; partial sums are written
-//    before they are read.  Calls whose kernels overlap on the GPU (different
-//    streams without ordering between them) race on the array.
+//    contents; nothing in it needs to start at any value (partial sums are
+//    written before they are read).  Calls whose kernels overlap on the GPU
+//    (different streams without ordering between them) race on the array.
 //  * Nothing here calls cudaMalloc, cudaFree or any allocating routine.
 //  * A bounded wait that gives up in these kernels sets the device error word
 //    of this file's own module, which lwq_get_device_error does not read; the
@@ -45,7 +42,6 @@ namespace lwq_noalloc {
 using namespace lwq;
 
 constexpr size_t kScratchBytes = 4u << 20;
-constexpr size_t kCounterBytes = 64u << 10;
 constexpr int kMaxDevices = 64;
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 
@@ -148,10 +144,7 @@ extern "C" int lwq_matmul_noalloc(int fmt, const void *Wq, const void *x, float 
     const int m_group = (xt == X_F32) ? (M < 8 ? M : 8) : M;
     const int S = cfg.splits;
     const int row_tiles = (N + GEMV_ROWS - 1) / GEMV_ROWS;
-    if (S > 1) {
-        if ((size_t)row_tiles * 4 > kCounterBytes) return LWQ_ERR_WORKSPACE_TOO_SMALL;
-        if (kCounterBytes + (size_t)S * m_group * N * 4 > kScratchBytes) return LWQ_ERR_WORKSPACE_TOO_SMALL;
-    }
+    if (S > 1 && (size_t)S * m_group * N * 4 > kScratchBytes) return LWQ_ERR_WORKSPACE_TOO_SMALL;
     void *scratch = nullptr;
     if ((rc = scratch_ptr(&scratch))) return rc;
     EncodeTiledFn enc = encoder();
@@ -176,12 +169,10 @@ extern "C" int lwq_matmul_noalloc(int fmt, const void *Wq, const void *x, float 
     const size_t xelem = (xt == X_F32) ? 4 : 2;
     for (int m0 = 0; m0 < M; m0 += m_group) {
         const int mg = (M - m0) < m_group ? (M - m0) : m_group;
-        if (S > 1 && cudaMemsetAsync(scratch, 0, (size_t)row_tiles * 4, st) != cudaSuccess) return LWQ_ERR_CUDA;
         GemvArgs a;
         a.x = static_cast<const uint8_t *>(x) + (size_t)m0 * K * xelem;
         a.y = y + (size_t)m0 * N;
-        a.counters = static_cast<unsigned *>(scratch);
-        a.partial = reinterpret_cast<float *>(static_cast<uint8_t *>(scratch) + kCounterBytes);
+        a.partial = static_cast<float *>(scratch);
         a.M = mg;
         a.N = N;
         a.K = K;
@@ -198,6 +189,22 @@ extern "C" int lwq_matmul_noalloc(int fmt, const void *Wq, const void *x, float 
         cudaError_t e = dispatch(wf, xt, nt, mg == 1, map, a, cfg.ctas, cfg.warps,
                                  smem_bytes(wf, cfg.warps, cfg.stages, ot), st);
         if (e != cudaSuccess) return LWQ_ERR_CUDA;
+        if (S > 1) {
+            // add the splits in order: a programmatic dependent launch after the GEMV
+            const long mn = (long)mg * N;
+            cudaLaunchConfig_t lc = {};
+            lc.gridDim = dim3((unsigned)splitk_sum_blocks(mn));
+            lc.blockDim = dim3(256u);
+            lc.stream = st;
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            at[0].val.programmaticStreamSerializationAllowed = 1;
+            lc.attrs = at;
+            lc.numAttrs = 1;
+            if (cudaLaunchKernelEx(&lc, gemv_splitk_sum_kernel, static_cast<const float *>(a.partial), a.y, S, mn) !=
+                cudaSuccess)
+                return LWQ_ERR_CUDA;
+        }
     }
     return LWQ_OK;
 }

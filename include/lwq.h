@@ -82,8 +82,8 @@ size_t lwq_row_bytes(int fmt, int64_t K);
 
 /* Device workspace bytes that lwq_matmul needs for every call with
  * M <= max_M, N <= max_N, K <= max_K in this format.  The workspace holds the
- * split-K partial sums (fp32) and the per-row-tile arrival counters that the
- * deterministic split-K reduction uses; it is the library's one static arena,
+ * split-K partial sums (fp32), which a follow-up kernel adds in split order
+ * (deterministic); it is the library's one static arena,
  * sized once at start-up ("1. Inferencia Local Eficiente em Memoria",
  * "Alocacao Estatica de Memoria" and "Arena de Buffer de Parametros").
  * Returns 0 for invalid arguments. */
@@ -93,9 +93,9 @@ size_t lwq_workspace_size(int fmt, int max_M, int max_N, int max_K);
  * d_workspace: device pointer, 16-byte aligned (NULL with bytes == 0 is
  * allowed: calls that need no workspace still run).  The library keeps the
  * pointer until lwq_shutdown or the next lwq_init on this device; it never
- * allocates, frees or reads it outside lwq_matmul.  This call zeroes the
- * arrival-counter region with a synchronous cudaMemset, so call it before any
- * stream capture.  Errors: LWQ_ERR_MISALIGNED, LWQ_ERR_CUDA. */
+ * allocates, frees or reads it outside lwq_matmul, and its contents need no
+ * initial value.  No device work is done here.  Errors: LWQ_ERR_MISALIGNED,
+ * LWQ_ERR_INVALID_ARG, LWQ_ERR_CUDA (no current device). */
 int lwq_init(void *d_workspace, size_t bytes);
 
 /* Forget the workspace registered for the current device.  Always LWQ_OK. */
@@ -112,8 +112,10 @@ int lwq_shutdown(void);
  *   stream  a cudaStream_t (NULL = the legacy default stream)
  *
  * Ownership: the caller owns Wq, x, y and the workspace.  The call is
- * asynchronous: it validates the arguments on the host, enqueues one or two
- * kernels on `stream` and returns; it never allocates and never synchronizes
+ * asynchronous: it validates the arguments on the host, enqueues its
+ * kernels on `stream` (one per pass of activation rows, plus a split-K sum
+ * kernel per pass when K is split; lwq_last_launch_count tells how many) and
+ * returns; it never allocates and never synchronizes
  * the host.  Kernel faults surface at the caller's next synchronization, as
  * with any CUDA launch.  Wq, x and y must be 16-byte aligned
  * (LWQ_ERR_MISALIGNED).  Calls that use split-K (see lwq_workspace_size) need
@@ -135,12 +137,11 @@ int lwq_matmul(int fmt, const void *Wq, const void *x, float *y, int M, int N, i
  * Arguments, layouts and results are those of lwq_matmul.  Only the decode
  * GEMV is offered: M <= 16 and the shapes lwq_select_config sends to path 1,
  * else LWQ_ERR_UNSUPPORTED.  A shape whose split-K scratch
- * (lwq_workspace_size bytes) exceeds 4 MiB, or with more than 16384 row tiles
- * of 16 weight rows when split, returns LWQ_ERR_WORKSPACE_TOO_SMALL.  The
- * first call on a device looks up the array's device address (make it before
- * any stream capture).  Calls share the array: each clears its counters on
- * `stream` first, and calls whose kernels overlap on the GPU race.  Nothing
- * is allocated or freed. */
+ * (lwq_workspace_size bytes) exceeds 4 MiB returns LWQ_ERR_WORKSPACE_TOO_SMALL.
+ * The first call on a device looks up the array's device address (make it
+ * before any stream capture).  Calls share the array, which needs no initial
+ * value; calls whose kernels overlap on the GPU race.  Nothing is allocated
+ * or freed. */
 int lwq_matmul_noalloc(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, void *stream);
 
 /* ------------------------------------------------ configuration table

@@ -106,7 +106,7 @@ def test_forced_gemv_configs(dev, w, a, warps, splits, stages):
 
 @pytest.mark.parametrize("w,a,M", [("q4_0", "f32", 1), ("q4_k", "f16", 1), ("q8_0", "f16", 16)])
 def test_split_k_deterministic(dev, w, a, M):
-    """Repeated calls (split-K with arrival counters) give bitwise identical results."""
+    """Repeated calls (split-K: partials added in split order by a follow-up kernel) are bitwise identical."""
     N, K = 300, 11008
     Wq, x = inputs.make_problem(w, a, M, N, K, seed=3)
     assert lwq.lwq_select_config(lwq.fmt_code(w, a), M, N, K).splits > 1

@@ -63,7 +63,7 @@ def test_noalloc_matches_lwq_matmul(dev, w, a, M, N, K):
 
 
 def test_noalloc_back_to_back_shapes(dev):
-    """Different shapes one after another: the second still starts from clean counters."""
+    """Different shapes one after another share the scratch array and both stay correct."""
     for w, a, M, N, K in CASES[::-1]:
         _run_both(dev, w, a, M, N, K, seed=K)
 
