@@ -47,6 +47,37 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # ------------------------------------------------------------------ helpers
 
+def csrc_sha256() -> str:
+    """Hash of the CUDA sources (every .cu/.cuh under the package's csrc/)."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "block_quantized_matmul_lwq_b200", "csrc", "*.cu*"))):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "gemv_tc_kernel_q4_0_f32_11008x4096.md")
+
+
+def profiled_traffic() -> int | None:
+    """DRAM bytes (read + write) of one headline step from the committed ncu summary,
+    or None when the summary is missing or the kernel sources changed since it was taken."""
+    import re
+    try:
+        with open(PROFILE_SUMMARY) as f:
+            text = f.read()
+    except OSError:
+        return None
+    m1 = re.search(r"^traffic_bytes_per_step:\s*(\d+)", text, re.M)
+    m2 = re.search(r"^csrc_sha256:\s*([0-9a-f]{64})", text, re.M)
+    if not (m1 and m2) or m2.group(1) != csrc_sha256():
+        return None
+    return int(m1.group(1))
+
+
 def load_peaks() -> tuple[dict, str]:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -338,34 +369,46 @@ def e2e_workload(lwq, workload: str, dev, steps: int, dist_on: bool):
 
 
 def cpu_baseline(workload: str, budget_s: float = 15.0) -> dict:
-    """The oracle as it stands, on the host cores, over a bounded row sample of one step."""
+    """The oracle as it stands, on the host cores, for about budget_s seconds of CPU work:
+    whole steps repeated when a step is short, else a row sample of one step."""
     import oracle
     calls = step_calls(workload)
     threads = oracle.max_threads()
-    # calibrate on a small row sample, then size the sample to the budget
-    rows = 64
-    t_rows = None
-    total_bytes = 0.0
-    total_s = 0.0
-    for attempt in range(2):
-        total_bytes = 0.0
-        total_s = 0.0
+
+    def make(rows):
+        data = []
         for fmt, act, M, N, K, seed in calls:
             g = inputs.rng(seed)
             n = min(rows, N)
             Wq = inputs.make_weights(fmt, g, n, K)
             x = inputs.activations(inputs.rng(seed + 1000003), M, K, act)
-            t0 = time.perf_counter()
-            oracle.matmul(fmt, Wq, x, act=act)
-            total_s += time.perf_counter() - t0
-            total_bytes += call_bytes(fmt, act, M, n, K)
-        if attempt == 0:
-            t_rows = total_s / rows
-            rows = max(16, int(budget_s / max(t_rows, 1e-9) / 2))
-            rows = min(rows, max(c[3] for c in calls))
+            data.append((fmt, act, M, n, K, Wq, x))
+        return data
+
+    def run(data, reps):
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            for fmt, act, M, n, K, Wq, x in data:
+                oracle.matmul(fmt, Wq, x, act=act)
+        return time.perf_counter() - t0
+
+    full_rows = max(c[3] for c in calls)
+    data = make(64)
+    t_row = run(data, 1) / 64
+    if t_row * full_rows <= budget_s / 4:
+        data = make(full_rows)
+        t_step = run(data, 1)
+        reps = max(1, min(10000, int(budget_s / max(t_step, 1e-9))))
+        sample = f"{reps} repetitions of one whole step (every weight row of every call; fp64 C oracle, OpenMP)"
+    else:
+        rows = max(16, min(full_rows, int(budget_s / max(t_row, 1e-9))))
+        data = make(rows)
+        reps = 1
+        sample = f"first {rows} weight rows of every call of one step (fp64 C oracle, OpenMP)"
+    total_s = run(data, reps)
+    total_bytes = reps * sum(call_bytes(fmt, act, M, n, K) for fmt, act, M, n, K, Wq, x in data)
     return {"value": total_bytes / total_s / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": f"first {rows} weight rows of every call of one step (fp64 C oracle, OpenMP)",
-            "seconds": total_s}
+            "sample": sample, "seconds": round(total_s, 2)}
 
 
 def run_gpu_arm(args):
@@ -403,8 +446,10 @@ def run_gpu_arm(args):
     # roofline: every launch in the timed region is the headline kernel (tensor-core GEMV,
     # Q4_0 x fp32); achieved = algorithmic bytes per step / device time per step on this rank
     achieved = prob.bytes_per_step / (ms_local / args.steps / 1e3) / 1e9
+    traffic = args.traffic if args.traffic is not None else profiled_traffic()
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": args.traffic,
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+                "algorithmic_bytes_per_step": prob.bytes_per_step, "per": "step (three launches: M=1, 4, 8)",
                 "peak_source": peak_src,
                 "kernel": "lwq::gemv_tc_kernel<Q4_0, fp32 x> (M=1 one-row, M=4 one tile, M=8 two tiles)",
                 "per_call_ms": [{"M": p["call"][2], "ms": round(p["ms_mean"], 5),
@@ -536,7 +581,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--reference-budget", type=float, default=60.0)
     ap.add_argument("--traffic", type=float, default=None,
-                    help="ncu dram bytes per launch of the roofline kernel, when measured for this build")
+                    help="ncu DRAM bytes per step of the headline kernels (default: the committed profile "
+                         "summary, when the CUDA sources still match it)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -1,0 +1,104 @@
+"""Multi-rank plumbing of bench.py on CPU: world_size 2 over gloo.
+
+The decode path has no exchange step (every rank runs its own replica), so the
+only cross-rank operations are the timing and byte-count reductions: the
+job's time is the max over ranks and its bytes the sum.  The reference arm
+runs on rank 0 alone.
+"""
+
+from __future__ import annotations
+
+import datetime
+import io
+import multiprocessing as mp
+import os
+import socket
+import sys
+from contextlib import redirect_stdout
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank: int, world: int, port: int, q) -> None:
+    try:
+        sys.path.insert(0, ROOT)
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+        import torch
+        import torch.distributed as dist
+
+        import bench
+
+        dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+        cpu = torch.device("cpu")
+        # each rank "measured" a different time and processed its own bytes
+        t_max = bench.reduce_max(10.0 + rank, True, cpu)
+        b_sum = bench.reduce_sum(1000.0 * (rank + 1), True, cpu)
+        # without torch.distributed both are the identity
+        ident = (bench.reduce_max(3.5, False), bench.reduce_sum(3.5, False))
+        dist.barrier()
+        dist.destroy_process_group()
+        q.put((rank, t_max, b_sum, ident))
+    except Exception as e:  # report, never hang the parent
+        q.put((rank, "error", repr(e), None))
+
+
+@pytest.mark.timeout(180)
+def test_reductions_over_two_gloo_ranks():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=150) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=30)
+        assert p.exitcode == 0
+    for rank, t_max, b_sum, ident in results:
+        assert t_max != "error", b_sum
+        assert t_max == 11.0          # the slowest rank's time
+        assert b_sum == 3000.0        # all ranks' bytes
+        assert ident == (3.5, 3.5)
+
+
+def test_reference_arm_runs_on_rank0_only(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    out = io.StringIO()
+    with redirect_stdout(out):
+        bench.run_reference_arm(bench.parse_args(["--impl", "reference", "--steps", "3", "--warmup", "3"]))
+    assert out.getvalue() == ""
+
+
+def test_warmup_floor():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    with pytest.raises(SystemExit):
+        bench.parse_args(["--warmup", "2"])
+    assert bench.parse_args([]).warmup >= 3
+
+
+def test_profiled_traffic_only_for_matching_sources(tmp_path, monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+
+    p = tmp_path / "summary.md"
+    monkeypatch.setattr(bench, "PROFILE_SUMMARY", str(p))
+    assert bench.profiled_traffic() is None                     # no summary
+    p.write_text(f"traffic_bytes_per_step: 12345\ncsrc_sha256: {bench.csrc_sha256()}\n")
+    assert bench.profiled_traffic() == 12345
+    p.write_text("traffic_bytes_per_step: 12345\ncsrc_sha256: " + "0" * 64 + "\n")
+    assert bench.profiled_traffic() is None                     # kernels changed since the capture
