@@ -370,8 +370,15 @@ int gemm_launch(int wf, int xt, const void *Wq, const void *x, float *y, int M, 
     a.n_wtiles = (N + GEMM_WROWS - 1) / GEMM_WROWS;
     a.n_ttiles = (M + bn - 1) / bn;
     a.bn = bn;
-    a.ab_stages = cfg.stages;
-    a.p_stages = 2;
+    a.a_stages = GEMM_A_STAGES;
+    {
+        // the same ring depths gemm_plan chose (its B ring is the configuration's stage count)
+        lwq_config f = cfg;
+        int nb = 0, np = 0;
+        gemm_rings(gemm_chunk_bytes(wf), bn, &f, &nb, &np);
+        a.b_stages = nb;
+        a.p_stages = np;
+    }
     a.timeout_ns = timeout_ns;
     a.overlap = overlap;
     cudaError_t e;

@@ -45,8 +45,9 @@ struct GemmArgs {
     int n_wtiles;     // ceil(N / 128)
     int n_ttiles;     // ceil(M / BN)
     int bn;           // token tile (UMMA N)
-    int ab_stages;
-    int p_stages;
+    int a_stages;     // dequantized weight k-blocks (produced on chip)
+    int b_stages;     // activation k-blocks (TMA from L2/HBM)
+    int p_stages;     // packed weight chunks (TMA from HBM)
     unsigned long long timeout_ns;
     int overlap;      // host side: launch with programmatic stream serialization
 };
@@ -62,17 +63,17 @@ struct GemmFmt<F_Q4_K> { static constexpr int chunk_bytes = 144; };
 
 __host__ __device__ constexpr size_t gemm_a_bytes() { return (size_t)GEMM_WROWS * 128; }
 __host__ __device__ constexpr size_t gemm_b_bytes(int bn) { return (size_t)bn * 128; }
-// one A+B stage, rounded up to the 1024-byte alignment of 128-byte-swizzle atoms
-__host__ __device__ constexpr size_t gemm_ab_bytes(int bn) { return (gemm_a_bytes() + gemm_b_bytes(bn) + 1023) & ~(size_t)1023; }
+// one B stage, rounded up to the 1024-byte alignment of 128-byte-swizzle atoms (A stages are 16 KB)
+__host__ __device__ constexpr size_t gemm_bstage_bytes(int bn) { return (gemm_b_bytes(bn) + 1023) & ~(size_t)1023; }
 // TMEM columns for two fp32 accumulators of bn columns (a power of two >= 32)
 __host__ __device__ constexpr uint32_t gemm_tmem_cols(int bn) { return 2 * bn <= 128 ? 128u : (2 * bn <= 256 ? 256u : 512u); }
 
-// Shared memory: [ab stages x (A 16 KB | B bn*128 B)] [p stages x 128*CB] [barriers] [tmem addr]
-__host__ __device__ inline size_t gemm_smem_bytes(int cb, int bn, int ab_stages, int p_stages) {
-    size_t s = (size_t)ab_stages * gemm_ab_bytes(bn);
+// Shared memory: [a stages x A 16 KB] [b stages x B bn*128 B] [p stages x 128*CB] [barriers] [tmem addr]
+__host__ __device__ inline size_t gemm_smem_bytes(int cb, int bn, int a_stages, int b_stages, int p_stages) {
+    size_t s = (size_t)a_stages * gemm_a_bytes() + (size_t)b_stages * gemm_bstage_bytes(bn);
     s += (size_t)p_stages * GEMM_WROWS * cb;
     s = (s + 7) & ~(size_t)7;
-    s += (size_t)(2 * ab_stages + 2 * p_stages + 4 + 1) * 8 + 16;
+    s += (size_t)(2 * a_stages + 2 * b_stages + 2 * p_stages + 4 + 1) * 8 + 16;
     return s + 1024;  // slack to align the base to 1024 B
 }
 
@@ -251,7 +252,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     constexpr uint32_t A_BYTES = (uint32_t)gemm_a_bytes();
     const int BN = a.bn;
     const uint32_t B_BYTES = (uint32_t)gemm_b_bytes(BN);
-    const uint32_t AB_BYTES = (uint32_t)gemm_ab_bytes(BN);
+    const uint32_t BS_BYTES = (uint32_t)gemm_bstage_bytes(BN);
     constexpr uint32_t P_BYTES = (uint32_t)GEMM_WROWS * CB;
     const uint32_t TMEM_COLS = gemm_tmem_cols(BN);
     const uint32_t IDESC = umma_idesc_f16(XT == X_F16 ? 0 : 1, GEMM_WROWS, BN);
@@ -260,13 +261,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // 1024-byte aligned base (128-byte swizzle atoms)
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
-    const int S = a.ab_stages, P = a.p_stages;
-    uint8_t *ab = smem;
-    uint8_t *pk = ab + (size_t)S * AB_BYTES;
+    const int SA = a.a_stages, SB = a.b_stages, P = a.p_stages;
+    uint8_t *As = smem;
+    uint8_t *Bs = As + (size_t)SA * A_BYTES;
+    uint8_t *pk = Bs + (size_t)SB * BS_BYTES;
     uint64_t *bars = reinterpret_cast<uint64_t *>(pk + (((size_t)P * P_BYTES + 7) & ~(size_t)7));
-    uint64_t *ab_full = bars, *ab_empty = bars + S;
-    uint64_t *p_full = bars + 2 * S, *p_empty = bars + 2 * S + P;
-    uint64_t *acc_full = bars + 2 * S + 2 * P, *acc_empty = acc_full + 2;
+    uint64_t *a_full = bars, *a_empty = bars + SA;
+    uint64_t *b_full = bars + 2 * SA, *b_empty = bars + 2 * SA + SB;
+    uint64_t *p_full = bars + 2 * SA + 2 * SB, *p_empty = p_full + P;
+    uint64_t *acc_full = p_empty + P, *acc_empty = acc_full + 2;
     uint64_t *mma_done = acc_full + 4;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
 
@@ -275,9 +278,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const int kblocks = a.nchunks * GEMM_KB_PER_CHUNK;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&ab_full[s], 1 + GEMM_DQ_WARPS);
-            mbar_init(&ab_empty[s], 1);
+        for (int s = 0; s < SA; ++s) {
+            mbar_init(&a_full[s], GEMM_DQ_WARPS);
+            mbar_init(&a_empty[s], 1);
+        }
+        for (int s = 0; s < SB; ++s) {
+            mbar_init(&b_full[s], 1);
+            mbar_init(&b_empty[s], 1);
         }
         for (int s = 0; s < P; ++s) {
             mbar_init(&p_full[s], 1);
@@ -301,53 +308,57 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const uint32_t tmem_base = *tmem_holder;
 
     if (warp == 0) {
-        // ------------------------------------------------------ TMA producer
+        // ------------------------------------------------------ TMA producers
+        // Lane 0 streams the packed weight chunks (p ring), lane 1 the activation
+        // k-blocks (ab ring), each as far ahead as its ring allows: a weight chunk
+        // is requested as soon as its slot frees, not behind the activation loads.
         if (lane == 0) {
             tma_prefetch_desc(&wmap);
-            tma_prefetch_desc(&xmap);
-            // ring positions (s, ps) and phase parities tracked incrementally
-            int kbi = 0, ci = 0, s = 0, ps = 0;
-            uint32_t ph = 0, pph = 0;
-            bool ok = true, waited = false;
+            int ci = 0, ps = 0;
+            uint32_t pph = 0;
+            bool ok = true;
             for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
-                const int tt = tile % a.n_ttiles, wt = tile / a.n_ttiles;
-                for (int c = 0; ok && c < a.nchunks; ++c, ++ci) {
-                    if (ci >= P && !(ok = mbar_wait(&p_empty[ps], pph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT)))
-                        break;
+                const int wt = tile / a.n_ttiles;
+                for (int c = 0; c < a.nchunks; ++c, ++ci) {
+                    // Wq only: callers that allow overlap promise it is not written by preceding work
+                    if (ci >= P && !(ok = mbar_wait(&p_empty[ps], pph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
                     mbar_arrive_expect_tx(&p_full[ps], P_BYTES);
                     tma_load_2d(pk + (size_t)ps * P_BYTES, &wmap, &p_full[ps], c * (CB / 2), wt * GEMM_WROWS);
-                    if (!waited) {   // x may be the preceding kernel's output
-                        pdl_wait();
-                        waited = true;
-                    }
                     if (++ps == P) {
                         ps = 0;
                         pph ^= 1u;
                     }
-                    for (int kb = 0; kb < GEMM_KB_PER_CHUNK; ++kb, ++kbi) {
-                        if (kbi >= S && !(ok = mbar_wait(&ab_empty[s], ph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT)))
-                            break;
-                        mbar_arrive_expect_tx(&ab_full[s], B_BYTES);
-                        tma_load_2d(ab + (size_t)s * AB_BYTES + A_BYTES, &xmap, &ab_full[s],
-                                    (c * GEMM_KB_PER_CHUNK + kb) * GEMM_BK, tt * BN);
-                        if (++s == S) {
-                            s = 0;
-                            ph ^= 1u;
-                        }
-                    }
                 }
             }
             // drain: the last loads land before the CTA may exit (runs once; divisions are fine here)
-            for (int j = max(0, kbi - S); j < kbi; ++j)
-                mbar_wait(&ab_full[j % S], (j / S) & 1, a.timeout_ns, DEVERR_GEMM_WAIT);
             for (int j = max(0, ci - P); j < ci; ++j)
                 mbar_wait(&p_full[j % P], (j / P) & 1, a.timeout_ns, DEVERR_GEMM_WAIT);
+        } else if (lane == 1) {
+            tma_prefetch_desc(&xmap);
+            pdl_wait();   // x may be the preceding kernel's output
+            int kbi = 0, s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
+                const int tt = tile % a.n_ttiles;
+                for (int k = 0; k < kblocks; ++k, ++kbi) {
+                    if (kbi >= SB && !(ok = mbar_wait(&b_empty[s], ph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
+                    mbar_arrive_expect_tx(&b_full[s], B_BYTES);
+                    tma_load_2d(Bs + (size_t)s * BS_BYTES, &xmap, &b_full[s], k * GEMM_BK, tt * BN);
+                    if (++s == SB) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            for (int j = max(0, kbi - SB); j < kbi; ++j)
+                mbar_wait(&b_full[j % SB], (j / SB) & 1, a.timeout_ns, DEVERR_GEMM_WAIT);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------- UMMA issuer
         if (lane == 0) {
-            int ti = 0, s = 0;
-            uint32_t ph = 0;
+            int ti = 0, sa = 0, sb = 0;
+            uint32_t pha = 0, phb = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++ti) {
                 const int as = ti & 1;
@@ -356,18 +367,24 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)as * (TMEM_COLS / 2);
                 for (int k = 0; k < kblocks; ++k) {
-                    if (!(ok = mbar_wait(&ab_full[s], ph, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
+                    if (!(ok = mbar_wait(&b_full[sb], phb, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
+                    if (!(ok = mbar_wait(&a_full[sa], pha, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
                     tc_fence_after();
-                    const uint32_t a_addr = smem_u32(ab + (size_t)s * AB_BYTES);
-                    const uint32_t b_addr = a_addr + A_BYTES;
+                    const uint32_t a_addr = smem_u32(As + (size_t)sa * A_BYTES);
+                    const uint32_t b_addr = smem_u32(Bs + (size_t)sb * BS_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < GEMM_BK / 16; ++kk)
                         umma_f16(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32), IDESC,
                                  (k | kk) ? 1u : 0u);
-                    umma_commit(&ab_empty[s]);
-                    if (++s == S) {
-                        s = 0;
-                        ph ^= 1u;
+                    umma_commit(&a_empty[sa]);
+                    umma_commit(&b_empty[sb]);
+                    if (++sa == SA) {
+                        sa = 0;
+                        pha ^= 1u;
+                    }
+                    if (++sb == SB) {
+                        sb = 0;
+                        phb ^= 1u;
                     }
                 }
                 if (!ok) break;
@@ -379,10 +396,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
     } else if (warp < 2 + GEMM_DQ_WARPS) {
         // ------------------------------------------------------ dequantizers
+        // Warp i of the 16 takes weight rows 8i..8i+7 of the tile, all four (h, v) slices of each:
+        // its packed-chunk loads then spread over the shared-memory banks (rows lie 144 bytes apart,
+        // which a warp of 32 rows would fold onto 8 banks), and each quarter-warp's 16-byte stores
+        // (8 rows, one chunk column) fall on distinct swizzled positions.
         const int t = threadIdx.x - 64;          // 0..511
-        const int r = t & (GEMM_WROWS - 1);      // weight row within the tile
-        const int h = (t >> 7) & 1;              // which 32 of the k-block's 64 weights
-        const int v = t >> 8;                    // which 16 of those 32
+        const int r = 8 * (t >> 5) + (t & 7);    // weight row within the tile
+        const int h = (t >> 3) & 1;              // which 32 of the k-block's 64 weights
+        const int v = (t >> 4) & 1;              // which 16 of those 32
         int kbi = 0, s = 0, ps = 0;
         uint32_t ph = 0, pph = 0;
         bool ok = true;
@@ -390,13 +411,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             for (int c = 0; ok && c < a.nchunks; ++c) {
                 if (!(ok = mbar_wait(&p_full[ps], pph, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
                 const uint32_t prow = smem_u32(pk) + (uint32_t)(ps * P_BYTES + r * CB);
-                for (int kb = 0; kb < GEMM_KB_PER_CHUNK; ++kb, ++kbi) {
-                    if (kbi >= S && !(ok = mbar_wait(&ab_empty[s], ph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
-                    Dequant<FMT, XT>::run(prow, kb, h, v, smem_u32(ab + (size_t)s * AB_BYTES), r);
+                // two k-blocks per batch: one proxy fence and one warp barrier for both
+                // (the ring has an even number of stages, so a batch never wraps)
+                for (int kb = 0; kb < GEMM_KB_PER_CHUNK; kb += 2, kbi += 2) {
+                    if (kbi >= SA) {
+                        if (!(ok = mbar_wait(&a_empty[s], ph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
+                        if (!(ok = mbar_wait(&a_empty[s + 1], ph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
+                    }
+                    Dequant<FMT, XT>::run(prow, kb, h, v, smem_u32(As + (size_t)s * A_BYTES), r);
+                    Dequant<FMT, XT>::run(prow, kb + 1, h, v, smem_u32(As + (size_t)(s + 1) * A_BYTES), r);
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&ab_full[s]);
-                    if (++s == S) {
+                    if (lane == 0) {
+                        mbar_arrive(&a_full[s]);
+                        mbar_arrive(&a_full[s + 1]);
+                    }
+                    if ((s += 2) == SA) {
                         s = 0;
                         ph ^= 1u;
                     }
@@ -463,6 +493,23 @@ inline bool gemm_eligible(int wf, int xt, long K) {
 
 inline int gemm_chunk_bytes(int wf) { return wf == LWQ_Q8_0 ? 272 : 144; }
 
+// Ring depths: 4 dequantized A stages (made on chip, two per batch), 3 packed
+// chunk stages (each feeds four k-blocks; 2 when shared memory is short), and
+// as many activation B stages as fit, up to 8 (B tiles arrive from L2/HBM at
+// ~60 bytes per cycle of a busy tensor pipe, so their ring covers the load
+// latency).  A forced stage count fixes the B ring.
+constexpr int GEMM_A_STAGES = 4;   // even: the dequantizers fill two stages per batch
+// B stages (most up to 8, at least 2) and chunk stages (3, else 2) for a tile width.
+inline void gemm_rings(int cb, int bn, const lwq_config *force, int *nb, int *np) {
+    for (int p = 3; p >= 2; --p) {
+        int b = force && force->stages ? force->stages : 8;
+        while (!(force && force->stages) && b > 2 && gemm_smem_bytes(cb, bn, GEMM_A_STAGES, b, p) > 232448) --b;
+        *nb = b;
+        *np = p;
+        if (gemm_smem_bytes(cb, bn, GEMM_A_STAGES, b, p) <= 232448) return;
+    }
+}
+
 inline int gemm_plan(int wf, int xt, int M, int N, int K, const lwq_config *force, int sms, GemmPlan *g) {
     (void)xt;
     (void)K;
@@ -486,21 +533,19 @@ inline int gemm_plan(int wf, int xt, int M, int N, int K, const lwq_config *forc
     }
     if (bn < 32 || bn > 256 || bn % 16) return LWQ_ERR_UNSUPPORTED;
     const int cb = gemm_chunk_bytes(wf);
-    int p_stages = 2;
-    int ab = force && force->stages ? force->stages : 4;
-    const size_t limit = 232448;
-    while (ab > 2 && gemm_smem_bytes(cb, bn, ab, p_stages) > limit) --ab;
-    if (gemm_smem_bytes(cb, bn, ab, p_stages) > limit) return LWQ_ERR_UNSUPPORTED;
+    int nb = 0, np = 0;
+    gemm_rings(cb, bn, force, &nb, &np);
+    if (nb < 2 || gemm_smem_bytes(cb, bn, GEMM_A_STAGES, nb, np) > 232448) return LWQ_ERR_UNSUPPORTED;
     const int tiles = n_wtiles * ((M + bn - 1) / bn);
     int ctas = force && force->ctas ? force->ctas : sms;
     if (ctas > tiles) ctas = tiles;
     if (ctas < 1) ctas = 1;
     g->warps = GEMM_DQ_WARPS;
-    g->stages = ab;
+    g->stages = nb;
     g->ctas = ctas;
     g->tile_n = GEMM_WROWS;
     g->tile_m = bn;
-    g->smem = gemm_smem_bytes(cb, bn, ab, p_stages);
+    g->smem = gemm_smem_bytes(cb, bn, GEMM_A_STAGES, nb, np);
     return LWQ_OK;
 }
 

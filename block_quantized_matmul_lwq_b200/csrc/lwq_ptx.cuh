@@ -65,15 +65,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete is
+// suspended (issuing nothing) until the phase completes or about hint_ns pass.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Suspend-time hint of the waits below: long enough that a waiting warp takes
+// no issue slots from the warps doing the work, short against the bound.
+constexpr uint32_t kWaitHintNs = 20000;
+
 // Wait for the phase with the given parity to complete, for at most
 // timeout_ns nanoseconds.  Returns false (after setting `errbit` in the device
 // error word) when the bound runs out; the caller then stops its loop.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t timeout_ns, unsigned errbit) {
     if (mbar_try_wait(bar, parity)) return true;
-    uint64_t t0 = globaltimer_ns();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 0 && globaltimer_ns() - t0 > timeout_ns) {
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait_hint(bar, parity, kWaitHintNs)) return true;
+        if (globaltimer_ns() - t0 > timeout_ns) {
             set_dev_error(errbit);
             return false;
         }
