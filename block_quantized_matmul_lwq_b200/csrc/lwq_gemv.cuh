@@ -292,17 +292,129 @@ struct Q40 {
         }
     }
 
+    // Activation row of column g in tile nt, and the fp16 part it carries.
+    __device__ static __forceinline__ int col_row(int g, int nt) {
+        return MERGED ? (g & 3) : (PART_TILES ? g : g + 8 * nt);
+    }
+    __device__ static __forceinline__ int col_part(int g, int nt) { return MERGED ? (g >> 2) : (PART_TILES ? nt : 0); }
+
+    // Fast path, one pass with scale 1 (exact whenever the warp's largest |x|
+    // lies in [2^-8, 2^15]: every fp16 value, x / 16 included, stays in range
+    // and tiny elements lose only bits far below the largest's): each lane
+    // builds its own column's fragments straight from its loads (word t of
+    // every block of its row), with no dependence on a maximum first, so all
+    // its loads can be in flight together.  Returns false, leaving the
+    // fragments to be rebuilt, when the range check fails.
+    __device__ __forceinline__ bool load_x_direct(const void *x, int M, int K, long k0, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+        constexpr int LT = PART_TILES ? 1 : NT;   // tiles with distinct rows
+        float mx = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < LT; ++nt) {
+            const int r = col_row(g, nt);
+            const bool live = r < M;
+            const long base = (long)r * K + k0;
+            const bool lo_part = (P == 2 && !PART_TILES && col_part(g, nt) == 1);
+            float bsum[8];
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                bsum[b] = 0.f;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float2 p = make_float2(0.f, 0.f), q = make_float2(0.f, 0.f);
+                    if (live) {
+                        p = load2(x, base + 32 * b + 16 * h + cb0(b & 1, t));
+                        q = load2(x, base + 32 * b + 16 * h + cb2(b & 1, t));
+                    }
+                    mx = fmaxf(mx, fmaxf(fmaxf(fabsf(p.x), fabsf(p.y)), fmaxf(fabsf(q.x), fabsf(q.y))));
+                    const float2 pq = __fadd2_rn(p, q);
+                    bsum[b] += pq.x + pq.y;
+                    if (h) {   // high-nibble step: x / 16 (exact)
+                        p = __fmul2_rn(p, make_float2(0.0625f, 0.0625f));
+                        q = __fmul2_rn(q, make_float2(0.0625f, 0.0625f));
+                    }
+                    if constexpr (P == 1) {
+                        xf[nt][b][h][0] = pack_f16x2(p.x, q.x);
+                        xf[nt][b][h][1] = pack_f16x2(p.y, q.y);
+                    } else {
+                        // hi = the top 11 significant bits (exact in fp16), lo = x - hi
+                        const float2 ph = make_float2(__uint_as_float(__float_as_uint(p.x) & 0xFFFFE000u),
+                                                      __uint_as_float(__float_as_uint(p.y) & 0xFFFFE000u));
+                        const float2 qh = make_float2(__uint_as_float(__float_as_uint(q.x) & 0xFFFFE000u),
+                                                      __uint_as_float(__float_as_uint(q.y) & 0xFFFFE000u));
+                        if constexpr (PART_TILES) {
+                            const float2 pl = __ffma2_rn(ph, make_float2(-1.f, -1.f), p);
+                            const float2 ql = __ffma2_rn(qh, make_float2(-1.f, -1.f), q);
+                            xf[0][b][h][0] = pack_f16x2(ph.x, qh.x);
+                            xf[0][b][h][1] = pack_f16x2(ph.y, qh.y);
+                            xf[1][b][h][0] = pack_f16x2(pl.x, ql.x);
+                            xf[1][b][h][1] = pack_f16x2(pl.y, ql.y);
+                        } else if (lo_part) {
+                            const float2 pl = __ffma2_rn(ph, make_float2(-1.f, -1.f), p);
+                            const float2 ql = __ffma2_rn(qh, make_float2(-1.f, -1.f), q);
+                            xf[nt][b][h][0] = pack_f16x2(pl.x, ql.x);
+                            xf[nt][b][h][1] = pack_f16x2(pl.y, ql.y);
+                        } else {
+                            xf[nt][b][h][0] = pack_f16x2(ph.x, qh.x);
+                            xf[nt][b][h][1] = pack_f16x2(ph.y, qh.y);
+                        }
+                    }
+                }
+                // the block's sum over the four lanes (code words) of this column
+                bsum[b] += __shfl_xor_sync(0xffffffffu, bsum[b], 1);
+                bsum[b] += __shfl_xor_sync(0xffffffffu, bsum[b], 2);
+            }
+            // correction B: sums of blocks (2t, 2t+1) / 64, hi + lo; only part-0 columns carry them
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (j == t) {
+                    s0 = bsum[2 * j];
+                    s1 = bsum[2 * j + 1];
+                }
+            if (!live || col_part(g, nt) != 0) s0 = s1 = 0.f;
+            s0 *= 0.015625f;
+            s1 *= 0.015625f;
+            const uint32_t hh = pack_f16x2(s0, s1);
+            xs[nt][0] = hh;
+            xs[nt][1] = pack_f16x2(s0 - f16_bits_to_float(hh), s1 - f16_bits_to_float(hh >> 16));
+        }
+        if constexpr (PART_TILES) xs[1][0] = xs[1][1] = 0u;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        inv = 1.f;
+        // all-zero activations are exact too; NaN and Inf take the other path
+        return mx == 0.f || (mx >= 0.00390625f && mx <= 32768.f);
+    }
+
     // One block at a time, every lane packs UPL units (each element of the
     // pass's rows once, both fp16 parts) into the warp's staging area, then
     // reads back its own B fragments; the block sums ride along for the offset
     // correction.
+    // Up to 4 fp32 rows, two columns share a row (hi and lo parts), so the
+    // staged path converts each element once; otherwise every lane converts
+    // its own column directly.  Both first try scale 1 in a single pass.
     __device__ __forceinline__ void load_x(const void *x, int M, int K, long k0, int lane, uint32_t stage0,
                                            uint32_t pstride) {
+        if constexpr (MERGED) {
+            if (!load_x_staged<true>(x, M, K, k0, lane, stage0, pstride))
+                load_x_staged<false>(x, M, K, k0, lane, stage0, pstride);
+        } else {
+            if (!load_x_direct(x, M, K, k0, lane)) load_x_staged<false>(x, M, K, k0, lane, stage0, pstride);
+        }
+    }
+
+    // Staged path: one block per round through the staging area.  UNIT: scale
+    // 1 in one pass, returning false when the range check of the direct path
+    // fails; else a per-warp power-of-two scale from a first pass over the chunk.
+    template <bool UNIT>
+    __device__ __forceinline__ bool load_x_staged(const void *x, int M, int K, long k0, int lane, uint32_t stage0,
+                                                  uint32_t pstride) {
         const int g = lane >> 2, t = lane & 3;
         // pass 1: the warp's largest |x|
         float mx = 0.f;
 #pragma unroll
-        for (int k = 0; k < UPL; ++k) {
+        for (int k = 0; k < (UNIT ? 0 : UPL); ++k) {
             const int u = lane + 32 * k, m = u >> 3, tu = (u >> 1) & 3, h = u & 1;
             if (m < M) {
                 const long base = (long)m * K + k0 + 16 * h;
@@ -314,8 +426,11 @@ struct Q40 {
                 }
             }
         }
-        float s;
-        warp_scale<XT>(mx, s, inv);
+        float s = 1.f;
+        if (UNIT)
+            inv = 1.f;
+        else
+            warp_scale<XT>(mx, s, inv);
         // correction sums of blocks (2t, 2t+1) for each tile's column g (part 0 only)
         float cs[NT][2];
         int crow[NT];
@@ -340,6 +455,7 @@ struct Q40 {
             for (int k = 0; k < UPL; ++k) {
                 const int u = lane + 32 * k, m = u >> 3, tu = (u >> 1) & 3, h = u & 1;
                 float2 p = RawPair<XT>::get(raw[b % 3][k][0]), q = RawPair<XT>::get(raw[b % 3][k][1]);
+                if (UNIT) mx = fmaxf(mx, fmaxf(fmaxf(fabsf(p.x), fabsf(p.y)), fmaxf(fabsf(q.x), fabsf(q.y))));
                 // high-nibble step: x / 16 (exact: a power of two)
                 const float sc = h ? s * 0.0625f : s;
                 p.x *= sc;
@@ -384,6 +500,13 @@ struct Q40 {
             const uint32_t hh = pack_f16x2(s0, s1);
             xs[nt][0] = hh;
             xs[nt][1] = pack_f16x2(s0 - f16_bits_to_float(hh), s1 - f16_bits_to_float(hh >> 16));
+        }
+        if constexpr (UNIT) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            return mx == 0.f || (mx >= 0.00390625f && mx <= 32768.f);
+        } else {
+            return true;
         }
     }
 
