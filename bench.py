@@ -512,6 +512,67 @@ def run_gpu_arm(args):
     lwq.lwq_shutdown()
 
 
+def run_sweep(args):
+    """The format x batch sweep: every (format, M, K x N) point timed through lwq_matmul with fp16
+    activations, one JSON line per point (GB/s against HBM for M <= 16, TFLOP/s against bf16 for M > 16)."""
+    import torch
+    import block_quantized_matmul_lwq_b200 as lwq
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    ws_bytes = max(lwq.lwq_workspace_size(lwq.fmt_code(f, "f16"), 1024, n, k)
+                   for f in inputs.SWEEP_FMTS for k, n in inputs.SWEEP_SHAPES_KN)
+    ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    lwq.lwq_init(ws, ws.numel())
+    stream = torch.cuda.Stream(device=dev)
+    for fmt in inputs.SWEEP_FMTS:
+        for K, N in inputs.SWEEP_SHAPES_KN:
+            Wq = inputs.make_weights(fmt, inputs.rng(11), N, K)
+            R = max(3, -(-(4 * L2_BYTES) // Wq.nbytes))
+            base = torch.from_numpy(Wq).to(dev)
+            Ws = [base] + [base.clone() for _ in range(R - 1)]
+            for M in inputs.SWEEP_MS:
+                x = inputs.activations(inputs.rng(12), M, K, "f16")
+                xd = torch.from_numpy(x.view(np.int16)).to(dev)
+                yd = torch.empty((M, N), dtype=torch.float32, device=dev)
+                code = lwq.fmt_code(fmt, "f16") | lwq.LWQ_FLAG_OVERLAP
+                cfg = lwq.lwq_select_config(lwq.fmt_code(fmt, "f16"), M, N, K)
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.stream(stream):
+                    for W in Ws:
+                        lwq.lwq_matmul(code, W, xd, yd, M, N, K, stream=stream)
+                    stream.synchronize()
+                    with torch.cuda.graph(g, stream=stream):
+                        for W in Ws:
+                            lwq.lwq_matmul(code, W, xd, yd, M, N, K, stream=stream)
+                    g.replay()
+                    stream.synchronize()
+                    reps = max(3, min(50, int(2e-3 / max(1e-6, 1e-5 * len(Ws)))))
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    for _ in range(reps):
+                        g.replay()
+                    e1.record(stream)
+                stream.synchronize()
+                ms = e0.elapsed_time(e1) / (reps * len(Ws))
+                rec = {"sweep": True, "fmt": fmt, "act": "f16", "M": M, "K": K, "N": N, "ms": round(ms, 5),
+                       "path": {1: "gemv", 2: "gemm", 3: "simple"}[cfg.path]}
+                if M <= 16:
+                    gbs = call_bytes(fmt, "f16", M, N, K) / (ms / 1e3) / 1e9
+                    rec.update({"GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4)})
+                else:
+                    tf = call_flops(M, N, K) / (ms / 1e3) / 1e12
+                    rec.update({"TFLOP/s": round(tf, 1), "frac_of_bf16": round(tf / peaks["bf16_tflops"], 4)})
+                rec["peak_source"] = peak_src
+                print(json.dumps(rec), flush=True)
+                del g
+            del Ws, base
+    torch.cuda.synchronize(dev)
+    err = lwq.lwq_get_device_error()
+    print(json.dumps({"sweep_done": True, "device_error": err}), flush=True)
+    lwq.lwq_shutdown()
+
+
 def run_reference_arm(args):
     """The oracle (the deliberately slow CPU definition) on the host cores, rank 0 only."""
     rank = int(os.environ.get("RANK", "0"))
@@ -578,6 +639,8 @@ def parse_args(argv=None):
     ap.add_argument("--extra", nargs="*", default=["q8_0_gemv_4096x4096", "q4_k_7b_layer_decode",
                                                    "q4_0_prefill_gemm"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the format x batch sweep instead (one JSON line per point)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--reference-budget", type=float, default=60.0)
     ap.add_argument("--traffic", type=float, default=None,
@@ -593,6 +656,8 @@ def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         run_reference_arm(args)
+    elif args.sweep:
+        run_sweep(args)
     else:
         run_gpu_arm(args)
 

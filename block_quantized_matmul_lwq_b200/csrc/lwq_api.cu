@@ -150,13 +150,13 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
         if (rc) return rc;
         p->cfg.warps = gp.warps;
         p->cfg.stages = gp.stages;
-        p->cfg.splits = 1;
+        p->cfg.splits = gp.splits;
         p->cfg.ctas = gp.ctas;
         p->cfg.tile_n = gp.tile_n;
         p->cfg.tile_m = gp.tile_m;
         p->smem = gp.smem;
         p->m_group = M;
-        p->ws_need = 0;
+        p->ws_need = splitk_ws(gp.splits, M, N);
         return LWQ_OK;
     }
     if (path == 3) {
@@ -334,8 +334,10 @@ cudaError_t launch_gemm_xt(int xt, const CUtensorMap &wm, const CUtensorMap &xm,
     return launch_gemm_tc<FMT, X_BF16>(wm, xm, a, ctas, smem, st);
 }
 
+// Returns the kernels launched (1, or 2 with the split-K sum) through *launches.
 int gemm_launch(int wf, int xt, const void *Wq, const void *x, float *y, int M, int N, int K, long rb,
-                const lwq_config &cfg, size_t smem, unsigned long long timeout_ns, int overlap, cudaStream_t st) {
+                const lwq_config &cfg, size_t smem, unsigned long long timeout_ns, int overlap, float *partial,
+                cudaStream_t st, int *launches) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return LWQ_ERR_CUDA;
     const int cb = gemm_chunk_bytes(wf);
@@ -363,6 +365,9 @@ int gemm_launch(int wf, int xt, const void *Wq, const void *x, float *y, int M, 
     }
     GemmArgs a;
     a.y = y;
+    a.splits = cfg.splits > 1 ? cfg.splits : 1;
+    a.cps = (K / 256 + a.splits - 1) / a.splits;
+    a.partial = partial;
     a.M = M;
     a.N = N;
     a.K = K;
@@ -387,7 +392,17 @@ int gemm_launch(int wf, int xt, const void *Wq, const void *x, float *y, int M, 
     case LWQ_Q8_0: e = launch_gemm_xt<F_Q8_0>(xt, wm, xm, a, cfg.ctas, smem, st); break;
     default: e = launch_gemm_xt<F_Q4_K>(xt, wm, xm, a, cfg.ctas, smem, st); break;
     }
-    return e == cudaSuccess ? LWQ_OK : LWQ_ERR_CUDA;
+    if (e != cudaSuccess) return LWQ_ERR_CUDA;
+    *launches = 1;
+    if (a.splits > 1) {
+        // add the K slices in order: a programmatic dependent launch after the GEMM
+        const long mn = (long)M * N;
+        e = launch_k(gemv_splitk_sum_kernel, splitk_sum_blocks(mn), 256, 0, st, true,
+                     static_cast<const float *>(partial), y, a.splits, mn);
+        if (e != cudaSuccess) return LWQ_ERR_CUDA;
+        *launches = 2;
+    }
+    return LWQ_OK;
 }
 
 int run(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, const lwq_config *force,
@@ -410,9 +425,16 @@ int run(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, c
     int launches = 0;
 
     if (p.cfg.path == 2) {
-        rc = gemm_launch(wf, xt, Wq, x, y, M, N, K, rb, p.cfg, p.smem, kTimeoutNs, overlap, st);
+        DeviceState &ds = g_dev[dev];
+        if (p.ws_need > 0) {
+            if (!ds.registered) return LWQ_ERR_NOT_INITIALIZED;
+            if (ds.ws_bytes < p.ws_need) return LWQ_ERR_WORKSPACE_TOO_SMALL;
+        }
+        int n = 0;
+        rc = gemm_launch(wf, xt, Wq, x, y, M, N, K, rb, p.cfg, p.smem, kTimeoutNs, overlap,
+                         static_cast<float *>(ds.ws), st, &n);
         if (rc) return rc;
-        t_last_launches = 1;
+        t_last_launches = n;
         return LWQ_OK;
     }
     if (p.cfg.path == 3) {
@@ -511,6 +533,15 @@ size_t lwq_workspace_size(int fmt, int max_M, int max_N, int max_K) {
     for (int m = 1; m <= max_M && m <= 16; ++m) {
         Plan p;
         if (make_plan(fmt, m, max_N, max_K, nullptr, sms, &p) == LWQ_OK && p.ws_need > need) need = p.ws_need;
+    }
+    // The GEMM splits K only while its output tiles fill at most half the SMs, into
+    // S <= ceil(sms / tiles) <= K / 1024 slices, so S * tiles <= 1.5 sms and each tile holds at most
+    // 128 x 256 outputs: its partials never exceed 4 * 1.5 * sms * 32768 bytes, nor 4 * (K/1024) * M * N.
+    if (max_M > 16 && (fmt & LWQ_ACT_MASK) != LWQ_ACT_F32) {
+        const size_t by_grid = (size_t)6 * sms * 32768;
+        const size_t by_shape = (size_t)4 * (max_K / 1024) * max_M * max_N;
+        const size_t g = by_grid < by_shape ? by_grid : by_shape;
+        if (g > need) need = g;
     }
     if (need < 256) need = 256;
     return need;

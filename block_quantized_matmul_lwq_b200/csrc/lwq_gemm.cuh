@@ -34,12 +34,15 @@ constexpr int GEMM_EPI_WARPS = 4;
 constexpr int GEMM_THREADS = (2 + GEMM_DQ_WARPS + GEMM_EPI_WARPS) * 32;
 
 struct GemmPlan {
-    int warps, stages, ctas, tile_n, tile_m;
+    int warps, stages, ctas, tile_n, tile_m, splits;
     size_t smem;
 };
 
 struct GemmArgs {
     float *y;
+    float *partial;   // split-K: [splits][M][N] fp32 (gemv_splitk_sum_kernel adds them), else unused
+    int splits;       // K slices per tile (1: write y directly)
+    int cps;          // chunks per K slice
     int M, N, K;
     int nchunks;      // K / 256
     int n_wtiles;     // ceil(N / 128)
@@ -274,8 +277,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_tiles = a.n_wtiles * a.n_ttiles;
-    const int kblocks = a.nchunks * GEMM_KB_PER_CHUNK;
+    // work items: (output tile, K slice); a tile's slices write fp32 partials when K is split
+    const int n_items = a.n_wtiles * a.n_ttiles * a.splits;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < SA; ++s) {
@@ -317,9 +320,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             int ci = 0, ps = 0;
             uint32_t pph = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
+            for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+                const int tile = item / a.splits, ks = item % a.splits;
                 const int wt = tile / a.n_ttiles;
-                for (int c = 0; c < a.nchunks; ++c, ++ci) {
+                const int c0 = ks * a.cps, c1 = min(a.nchunks, c0 + a.cps);
+                for (int c = c0; c < c1; ++c, ++ci) {
                     // Wq only: callers that allow overlap promise it is not written by preceding work
                     if (ci >= P && !(ok = mbar_wait(&p_empty[ps], pph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
                     mbar_arrive_expect_tx(&p_full[ps], P_BYTES);
@@ -339,9 +344,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             int kbi = 0, s = 0;
             uint32_t ph = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
+            for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+                const int tile = item / a.splits, ks = item % a.splits;
                 const int tt = tile % a.n_ttiles;
-                for (int k = 0; k < kblocks; ++k, ++kbi) {
+                const int k0 = ks * a.cps * GEMM_KB_PER_CHUNK;
+                const int k1 = min(a.nchunks, (ks + 1) * a.cps) * GEMM_KB_PER_CHUNK;
+                for (int k = k0; k < k1; ++k, ++kbi) {
                     if (kbi >= SB && !(ok = mbar_wait(&b_empty[s], ph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
                     mbar_arrive_expect_tx(&b_full[s], B_BYTES);
                     tma_load_2d(Bs + (size_t)s * BS_BYTES, &xmap, &b_full[s], k * GEMM_BK, tt * BN);
@@ -360,13 +368,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             int ti = 0, sa = 0, sb = 0;
             uint32_t pha = 0, phb = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++ti) {
+            for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++ti) {
+                const int ks = item % a.splits;
+                const int kbn = (min(a.nchunks, (ks + 1) * a.cps) - ks * a.cps) * GEMM_KB_PER_CHUNK;
                 const int as = ti & 1;
                 if (ti >= 2 && !(ok = mbar_wait(&acc_empty[as], ((ti >> 1) - 1) & 1, a.timeout_ns, DEVERR_GEMM_WAIT)))
                     break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)as * (TMEM_COLS / 2);
-                for (int k = 0; k < kblocks; ++k) {
+                for (int k = 0; k < kbn; ++k) {
                     if (!(ok = mbar_wait(&b_full[sb], phb, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
                     if (!(ok = mbar_wait(&a_full[sa], pha, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
                     tc_fence_after();
@@ -407,8 +417,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         int kbi = 0, s = 0, ps = 0;
         uint32_t ph = 0, pph = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
-            for (int c = 0; ok && c < a.nchunks; ++c) {
+        for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+            const int ks = item % a.splits;
+            const int c0 = ks * a.cps, c1 = min(a.nchunks, c0 + a.cps);
+            for (int c = c0; ok && c < c1; ++c) {
                 if (!(ok = mbar_wait(&p_full[ps], pph, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
                 const uint32_t prow = smem_u32(pk) + (uint32_t)(ps * P_BYTES + r * CB);
                 // two k-blocks per batch: one proxy fence and one warp barrier for both
@@ -445,8 +457,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const int N = a.N, M = a.M;
         int ti = 0;
-        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++ti) {
+        for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++ti) {
+            const int tile = item / a.splits, ks = item % a.splits;
             const int tt = tile % a.n_ttiles, wt = tile / a.n_ttiles;
+            float *out = a.splits > 1 ? a.partial + (size_t)ks * M * N : a.y;
             const int as = ti & 1;
             if (!mbar_wait(&acc_full[as], (ti >> 1) & 1, a.timeout_ns, DEVERR_GEMM_WAIT)) break;
             tc_fence_after();
@@ -468,7 +482,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 if (n < N) {
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        if (j < mcols && m0 + j < M) a.y[(size_t)(m0 + j) * N + n] = __uint_as_float(v[j]);
+                        if (j < mcols && m0 + j < M) out[(size_t)(m0 + j) * N + n] = __uint_as_float(v[j]);
                 }
             }
             tc_fence_before();
@@ -512,19 +526,29 @@ inline void gemm_rings(int cb, int bn, const lwq_config *force, int *nb, int *np
 
 inline int gemm_plan(int wf, int xt, int M, int N, int K, const lwq_config *force, int sms, GemmPlan *g) {
     (void)xt;
-    (void)K;
     const int n_wtiles = (N + GEMM_WROWS - 1) / GEMM_WROWS;
+    const int nchunks = K / 256;
+    // K slices for a tile count: split when the tiles fill at most half the SMs, keeping >= 4 chunks a slice
+    auto slices = [&](long tiles) -> int {
+        if (force && force->splits) return force->splits;
+        if (2 * tiles > sms) return 1;
+        long sp = (sms + tiles - 1) / tiles;
+        if (sp > nchunks / 4) sp = nchunks / 4;
+        return sp < 1 ? 1 : (int)sp;
+    };
     int bn = force && force->tile_m ? force->tile_m : 0;
     if (!bn) {
-        // token tile: the persistent grid runs ceil(tiles / sms) rounds of BN-wide tiles; pick the multiple of 16
-        // that minimizes rounds * (BN + 48) (the constant stands for a tile's decode and pipeline fill overhead),
-        // preferring larger tiles on ties
-        long best = -1;
+        // token tile: the persistent grid runs ceil(items / sms) rounds of work items (a tile's K slice);
+        // an item costs ~ (K / slices) * (BN + 48) (the constant stands for the k-block's decode and
+        // pipeline overhead).  Pick the multiple of 16 with the least rounds * (BN + 48) / slices,
+        // preferring larger tiles on ties.
+        double best = -1;
         const int hi = M < 256 ? ((M + 15) / 16) * 16 : 256;
         for (int c = hi; c >= 32; c -= 16) {
             const long tiles = (long)n_wtiles * ((M + c - 1) / c);
-            const long rounds = (tiles + sms - 1) / sms;
-            const long cost = rounds * (c + 48);
+            const int sp = slices(tiles);
+            const long rounds = (tiles * sp + sms - 1) / sms;
+            const double cost = (double)rounds * (c + 48) / sp;
             if (best < 0 || cost < best) {
                 best = cost;
                 bn = c;
@@ -537,9 +561,15 @@ inline int gemm_plan(int wf, int xt, int M, int N, int K, const lwq_config *forc
     gemm_rings(cb, bn, force, &nb, &np);
     if (nb < 2 || gemm_smem_bytes(cb, bn, GEMM_A_STAGES, nb, np) > 232448) return LWQ_ERR_UNSUPPORTED;
     const int tiles = n_wtiles * ((M + bn - 1) / bn);
+    int splits = slices(tiles);
+    if (splits < 1 || splits > nchunks) return LWQ_ERR_UNSUPPORTED;
+    const int cps = (nchunks + splits - 1) / splits;
+    splits = (nchunks + cps - 1) / cps;   // drop empty slices
+    const int items = tiles * splits;
     int ctas = force && force->ctas ? force->ctas : sms;
-    if (ctas > tiles) ctas = tiles;
+    if (ctas > items) ctas = items;
     if (ctas < 1) ctas = 1;
+    g->splits = splits;
     g->warps = GEMM_DQ_WARPS;
     g->stages = nb;
     g->ctas = ctas;

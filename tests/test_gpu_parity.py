@@ -104,6 +104,20 @@ def test_forced_gemv_configs(dev, w, a, warps, splits, stages):
     check_full(w, a, M, N, K, dev, seed=11, cfg=cfg)
 
 
+@pytest.mark.parametrize("w,a", [("q4_0", "bf16"), ("q4_k", "f16"), ("q8_0", "bf16")])
+@pytest.mark.parametrize("M,N,K,splits", [(40, 300, 2048, 0), (64, 1000, 4096, 0), (96, 130, 3072, 3),
+                                          (33, 257, 4096, 2), (200, 384, 6144, 5)])
+def test_gemm_split_k(dev, w, a, M, N, K, splits):
+    # few output tiles: the GEMM splits K into slices whose fp32 partials a follow-up kernel adds
+    cfg = None
+    if splits:
+        cfg = lwq.lwq_config()
+        cfg.path, cfg.splits = 2, splits
+    else:
+        assert lwq.lwq_select_config(lwq.fmt_code(w, a), M, N, K).splits > 1
+    check_full(w, a, M, N, K, dev, seed=M + N, cfg=cfg)
+
+
 @pytest.mark.parametrize("w,a,M", [("q4_0", "f32", 1), ("q4_k", "f16", 1), ("q8_0", "f16", 16)])
 def test_split_k_deterministic(dev, w, a, M):
     """Repeated calls (split-K: partials added in split order by a follow-up kernel) are bitwise identical."""
