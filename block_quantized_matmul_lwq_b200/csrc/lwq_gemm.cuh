@@ -539,16 +539,16 @@ inline int gemm_plan(int wf, int xt, int M, int N, int K, const lwq_config *forc
     int bn = force && force->tile_m ? force->tile_m : 0;
     if (!bn) {
         // token tile: the persistent grid runs ceil(items / sms) rounds of work items (a tile's K slice);
-        // an item costs ~ (K / slices) * (BN + 48) (the constant stands for the k-block's decode and
-        // pipeline overhead).  Pick the multiple of 16 with the least rounds * (BN + 48) / slices,
-        // preferring larger tiles on ties.
+        // an item costs ~ (K / slices) * (BN + 128) (the constant stands for the k-block's decode and
+        // pipeline overhead, measured to be worth about half a 256-wide MMA).  Pick the multiple of 16
+        // with the least rounds * (BN + 128) / slices, preferring larger tiles on ties.
         double best = -1;
         const int hi = M < 256 ? ((M + 15) / 16) * 16 : 256;
         for (int c = hi; c >= 32; c -= 16) {
             const long tiles = (long)n_wtiles * ((M + c - 1) / c);
             const int sp = slices(tiles);
             const long rounds = (tiles * sp + sms - 1) / sms;
-            const double cost = (double)rounds * (c + 48) / sp;
+            const double cost = (double)rounds * (c + 128) / sp;
             if (best < 0 || cost < best) {
                 best = cost;
                 bn = c;
