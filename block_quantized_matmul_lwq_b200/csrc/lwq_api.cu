@@ -623,3 +623,8 @@ int lwq_last_launch_count(void) { return t_last_launches; }
 int lwq_version(void) { return 0x000100; }
 
 }  // extern "C"
+
+// The allocation-free entry point shares this translation unit, so the whole
+// library is one device module: one copy of each kernel and of the device
+// error word that every bounded wait sets.
+#include "lwq_noalloc.cuh"

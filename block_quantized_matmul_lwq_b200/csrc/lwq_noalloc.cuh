@@ -24,9 +24,14 @@
 //    written before they are read).  Calls whose kernels overlap on the GPU
 //    (different streams without ordering between them) race on the array.
 //  * Nothing here calls cudaMalloc, cudaFree or any allocating routine.
-//  * A bounded wait that gives up in these kernels sets the device error word
-//    of this file's own module, which lwq_get_device_error does not read; the
-//    call's outputs are then not all written.
+//  * A bounded wait that gives up in these kernels sets the library's device
+//    error word, as in lwq_matmul (lwq_get_device_error); the call's outputs
+//    are then not all written.
+//
+// This file is included by lwq_api.cu: the library is a single translation
+// unit, so that the kernels it shares with lwq_matmul and the device error
+// word each exist once.
+#pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -43,7 +48,6 @@ using namespace lwq;
 
 constexpr size_t kScratchBytes = 4u << 20;
 constexpr int kMaxDevices = 64;
-constexpr unsigned long long kTimeoutNs = 2000000000ull;
 
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
@@ -181,7 +185,7 @@ extern "C" int lwq_matmul_noalloc(int fmt, const void *Wq, const void *x, float 
         a.chunks_per_split = cps;
         a.row_tiles = row_tiles;
         a.stages = cfg.stages;
-        a.timeout_ns = kTimeoutNs;
+        a.timeout_ns = lwq::kTimeoutNs;   // the library's 2 s wait bound
         a.overlap = 0;
         // n8 column tiles, as lwq_matmul picks them; fp32 activations keep one output tile
         const int nt = (xt == X_F32) ? ((wf == LWQ_Q4_0 && mg > 4) ? 2 : 1) : (mg <= 8 ? 1 : 2);

@@ -173,7 +173,8 @@ int lwq_matmul_config(int fmt, const void *Wq, const void *x, float *y, int M, i
 const char *lwq_status_string(int status);
 
 /* Device-side error word of the current device: every wait in the kernels
- * (on an mbarrier, a split-K counter or a TMEM handoff) is bounded; a kernel
+ * (on an mbarrier or a TMEM handoff) is bounded, in lwq_matmul and
+ * lwq_matmul_noalloc alike; a kernel
  * that gives up sets a bit here and returns instead of hanging.  The caller
  * must synchronize first.  Returns LWQ_OK, LWQ_ERR_DEVICE_TIMEOUT (and clears
  * the word), or LWQ_ERR_CUDA. */
