@@ -316,16 +316,33 @@ struct Q40 {
             const long base = (long)r * K + k0;
             const bool lo_part = (P == 2 && !PART_TILES && col_part(g, nt) == 1);
             float bsum[8];
+            // The loads of BPP blocks are issued together before any of them is
+            // used: with the fragments already taking 32-64 registers, leaving
+            // the order to the compiler let only a few loads be in flight at a
+            // time, several L2 round trips where one or two suffice.
+            constexpr int BPP = (XT == X_F32) ? 4 : 8;
+            using Raw = typename RawPair<XT>::T;
 #pragma unroll
-            for (int b = 0; b < 8; ++b) {
+            for (int b0 = 0; b0 < 8; b0 += BPP) {
+            Raw rp[BPP][2], rq[BPP][2];
+#pragma unroll
+            for (int bb = 0; bb < BPP; ++bb)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int b = b0 + bb;
+                    rp[bb][h] = rq[bb][h] = RawPair<XT>::zero();
+                    if (live) {
+                        rp[bb][h] = RawPair<XT>::load(x, base + 32 * b + 16 * h + cb0(b & 1, t));
+                        rq[bb][h] = RawPair<XT>::load(x, base + 32 * b + 16 * h + cb2(b & 1, t));
+                    }
+                }
+#pragma unroll
+            for (int bb = 0; bb < BPP; ++bb) {
+                const int b = b0 + bb;
                 bsum[b] = 0.f;
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    float2 p = make_float2(0.f, 0.f), q = make_float2(0.f, 0.f);
-                    if (live) {
-                        p = load2(x, base + 32 * b + 16 * h + cb0(b & 1, t));
-                        q = load2(x, base + 32 * b + 16 * h + cb2(b & 1, t));
-                    }
+                    float2 p = RawPair<XT>::get(rp[bb][h]), q = RawPair<XT>::get(rq[bb][h]);
                     mx = fmaxf(mx, fmaxf(fmaxf(fabsf(p.x), fabsf(p.y)), fmaxf(fabsf(q.x), fabsf(q.y))));
                     const float2 pq = __fadd2_rn(p, q);
                     bsum[b] += pq.x + pq.y;
@@ -363,6 +380,7 @@ struct Q40 {
                 // the block's sum over the four lanes (code words) of this column
                 bsum[b] += __shfl_xor_sync(0xffffffffu, bsum[b], 1);
                 bsum[b] += __shfl_xor_sync(0xffffffffu, bsum[b], 2);
+            }
             }
             // correction B: sums of blocks (2t, 2t+1) / 64, hi + lo; only part-0 columns carry them
             float s0 = 0.f, s1 = 0.f;
@@ -1252,8 +1270,8 @@ __global__ void __maxnreg__(gemv_max_regs(FMT, XT, NT))
                 }
             }
             // drain: every issued stage's load lands before the CTA may exit
-            const int issued = it;
-            for (int j = max(0, issued - stages); j < issued; ++j)
+            const int n_issued = it;
+            for (int j = max(0, n_issued - stages); j < n_issued; ++j)
                 mbar_wait(&full[j % stages], (j / stages) & 1, a.timeout_ns, DEVERR_GEMV_WAIT);
         }
         return;

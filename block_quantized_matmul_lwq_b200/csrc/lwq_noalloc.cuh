@@ -126,11 +126,7 @@ static cudaError_t dispatch(int wf, int xt, int nt, bool one, const CUtensorMap 
     return cudaErrorInvalidValue;
 }
 
-static size_t smem_bytes(int wf, int nw, int stages, int ot) {
-    const int cb = (wf == LWQ_Q8_0) ? 272 : 144;
-    return (size_t)stages * nw * GEMV_ROWS * cb + (size_t)stages * nw * GEMV_ROWS * 8 * ot * 4 +
-           (size_t)3 * stages * 8;
-}
+static size_t smem_bytes(int wf, int nw, int stages, int ot) { return lwq::gemv_smem(wf, nw, stages, ot); }
 
 }  // namespace lwq_noalloc
 
