@@ -256,8 +256,29 @@ class Problem:
         return sum(self.enqueue_call(lwq, i, r, stream) for i in range(len(self.dev_calls)))
 
 
+def replay_steps(graphs, full, n: int, first: int = 0) -> None:
+    """Replay n steps, step i reading weight copy (first + i) mod R: whole
+    rotations (from copy 0) through `full`, which holds all R steps in one
+    graph, and the other steps one graph each."""
+    R = len(graphs)
+    i, c = 0, first % R
+    while i < n:
+        if c == 0 and n - i >= R:
+            full.replay()
+            i += R
+        else:
+            graphs[c].replay()
+            i += 1
+            c = (c + 1) % R
+
+
 def time_workload(lwq, workload: str, dev, steps: int, warmup: int, dist_on: bool, per_call: bool = True):
-    """Device time of `steps` steps (graph-replayed, rotating weights), max over ranks."""
+    """Device time of `steps` steps (graph-replayed, rotating weights), max over ranks.
+
+    The R steps of one weight rotation are captured in one graph, as a decode
+    loop captures its calls: a graph launch costs the device several
+    microseconds and ends the overlap of one call with the next, which one
+    graph per step would add to every step."""
     import torch
     import torch.distributed as dist
     prob = Problem(workload, dev, rotate_min_bytes=4 * L2_BYTES)
@@ -273,10 +294,15 @@ def time_workload(lwq, workload: str, dev, steps: int, warmup: int, dist_on: boo
             with torch.cuda.graph(g, stream=stream):
                 launches_per_step = prob.enqueue_step(lwq, r, stream)
             graphs.append(g)
+        full = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(full, stream=stream):
+            for r in range(prob.R):
+                prob.enqueue_step(lwq, r, stream)
+        full.replay()   # first launch uploads the graph; not a timed or warm-up step
     stream.synchronize()
-    for i in range(warmup):
-        with torch.cuda.stream(stream):
-            graphs[i % prob.R].replay()
+    with torch.cuda.stream(stream):
+        # the warm-up ends on copy R-1, so the timed steps start on the copy read longest ago
+        replay_steps(graphs, full, warmup, first=-warmup)
     stream.synchronize()
     if dist_on:
         dist.barrier()
@@ -284,8 +310,7 @@ def time_workload(lwq, workload: str, dev, steps: int, warmup: int, dist_on: boo
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         start.record(stream)
-        for i in range(steps):
-            graphs[i % prob.R].replay()
+        replay_steps(graphs, full, steps)
         end.record(stream)
     stream.synchronize()
     torch.cuda.synchronize(dev)
@@ -499,7 +524,7 @@ def run_gpu_arm(args):
                        "accumulate": "f32", "M": [1, 4, 8], "N": 11008, "K": 4096, "seed": 0,
                        "l2": f"inputs larger than L2: every call reads its own weight copy, "
                              f"{prob.copies_bytes / 1e6:.0f} MB of copies in rotation",
-                       "parallelism": f"replicas x{world}", "timing": "CUDA graphs of one step, CUDA events",
+                       "parallelism": f"replicas x{world}", "timing": "CUDA graphs of one weight rotation (R steps), CUDA events",
                        "launch": "LWQ_FLAG_OVERLAP: programmatic dependent launches, weights constant"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": lps * args.steps, "clocks": clocks, "workloads": extra,
