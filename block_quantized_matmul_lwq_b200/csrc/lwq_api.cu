@@ -306,6 +306,7 @@ cudaError_t dispatch_simple(int wf, int xt, const uint8_t *W, const void *x, flo
 // The GEMV's view of Wq: 3-D, (8-byte word of a 256-weight chunk, weight row,
 // chunk), strides (row_bytes, chunk_bytes); a box of (all words, 16 rows, cps
 // chunks) lands as cps consecutive [16 rows][chunk] boxes.
+// (8-byte word of a chunk, weight row, chunk): one [cps chunks][16 rows][chunk bytes] box per GEMV stage
 int encode_weight_map(CUtensorMap *map, const void *Wq, int wf, int N, long rb, int cps) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return LWQ_ERR_CUDA;

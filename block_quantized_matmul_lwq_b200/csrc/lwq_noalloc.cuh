@@ -58,23 +58,6 @@ struct DevSlot {
 static DevSlot g_slots[kMaxDevices];
 static std::mutex g_mu;
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encoder() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
 // Device address of g_scratch on the current device (looked up once per device).
 static int scratch_ptr(void **out) {
     int dev = 0;
@@ -147,24 +130,11 @@ extern "C" int lwq_matmul_noalloc(int fmt, const void *Wq, const void *x, float 
     if (S > 1 && (size_t)S * m_group * N * 4 > kScratchBytes) return LWQ_ERR_WORKSPACE_TOO_SMALL;
     void *scratch = nullptr;
     if ((rc = scratch_ptr(&scratch))) return rc;
-    EncodeTiledFn enc = encoder();
-    if (!enc) return LWQ_ERR_CUDA;
     const long rb = (long)lwq_row_bytes(fmt, K);
     const int nchunks = K / 256;
     const int cps = (nchunks + S - 1) / S;
-    CUtensorMap map;
-    {
-        // (8-byte word of a chunk, weight row, chunk); one box per stage, as lwq_matmul's
-        const int cb = (wf == LWQ_Q8_0) ? 272 : 144;
-        cuuint64_t dims[3] = {(cuuint64_t)(cb / 8), (cuuint64_t)N, (cuuint64_t)nchunks};
-        cuuint64_t strides[2] = {(cuuint64_t)rb, (cuuint64_t)cb};
-        cuuint32_t box[3] = {(cuuint32_t)(cb / 8), (cuuint32_t)GEMV_ROWS, (cuuint32_t)cps};
-        cuuint32_t estr[3] = {1, 1, 1};
-        if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, const_cast<void *>(Wq), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return LWQ_ERR_CUDA;
-    }
+    CUtensorMap map;   // one box per stage, as lwq_matmul's
+    if ((rc = lwq::encode_weight_map(&map, Wq, wf, N, rb, cps))) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const size_t xelem = (xt == X_F32) ? 4 : 2;
     for (int m0 = 0; m0 < M; m0 += m_group) {
@@ -183,9 +153,9 @@ extern "C" int lwq_matmul_noalloc(int fmt, const void *Wq, const void *x, float 
         a.stages = cfg.stages;
         a.timeout_ns = lwq::kTimeoutNs;   // the library's 2 s wait bound
         a.overlap = 0;
-        // n8 column tiles, as lwq_matmul picks them; fp32 activations keep one output tile
-        const int nt = (xt == X_F32) ? ((wf == LWQ_Q4_0 && mg > 4) ? 2 : 1) : (mg <= 8 ? 1 : 2);
-        const int ot = (xt == X_F32) ? 1 : nt;
+        // n8 column tiles, as lwq_matmul picks them
+        const int nt = lwq::gemv_nt(wf, xt, mg);
+        const int ot = lwq::gemv_ot(xt, nt);
         cudaError_t e = dispatch(wf, xt, nt, mg == 1, map, a, cfg.ctas, cfg.warps,
                                  smem_bytes(wf, cfg.warps, cfg.stages, ot), st);
         if (e != cudaSuccess) return LWQ_ERR_CUDA;
