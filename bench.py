@@ -89,10 +89,11 @@ def load_peaks() -> tuple[dict, str]:
 
 
 def step_calls(workload: str):
-    """[(fmt, act, M, N, K, seed)] of one step of a workload."""
+    """[(fmt, act, M, N, K, seed)] of one step of a workload.  A tuple seed is a
+    weight of concatenated rows: equal parts, one per seed (see call_weights)."""
     spec = inputs.WORKLOADS[workload]
     calls = []
-    if workload == "q4_k_7b_layer_decode":
+    if workload.startswith("q4_k_7b_layer_decode"):
         for (N, K), seed in zip(spec["shapes"], spec["seeds"]):
             calls.append((spec["fmt"], spec["act"], 1, N, K, seed))
     elif workload == "q4_0_prefill_gemm":
@@ -103,6 +104,21 @@ def step_calls(workload: str):
         for M in spec["Ms"]:
             calls.append((spec["fmt"], spec["act"], M, N, K, spec["seeds"][0]))
     return calls
+
+
+def call_weights(fmt: str, N: int, K: int, seed):
+    """Packed weights of one call: seed s gives make_weights(fmt, rng(s), N, K); a
+    tuple of seeds stacks that many equal row blocks, each generated as its own tensor."""
+    if isinstance(seed, tuple):
+        n = N // len(seed)
+        return np.concatenate([inputs.make_weights(fmt, inputs.rng(s), n, K) for s in seed], axis=0)
+    return inputs.make_weights(fmt, inputs.rng(seed), N, K)
+
+
+def call_activations(act: str, M: int, K: int, seed):
+    """Activations of one call (a fused call takes those of its first part)."""
+    s = seed[0] if isinstance(seed, tuple) else seed
+    return inputs.activations(inputs.rng(s + 1000003), M, K, act)
 
 
 def call_bytes(fmt, act, M, N, K) -> int:
@@ -212,10 +228,9 @@ class Problem:
         for fmt, act, M, N, K, seed in self.calls:
             key = (fmt, N, K, seed)
             if key not in cache:
-                g = inputs.rng(seed)
-                cache[key] = (inputs.make_weights(fmt, g, N, K), g)
-            Wq, _ = cache[key]
-            x = inputs.activations(inputs.rng(seed + 1000003), M, K, act)
+                cache[key] = call_weights(fmt, N, K, seed)
+            Wq = cache[key]
+            x = call_activations(act, M, K, seed)
             self.host.append((Wq, x))
         self.step_weight_bytes = sum(N * inputs.row_bytes(f, K) for f, a, M, N, K, s in self.calls)
         # every call of a step reads its own weight copy; R steps cycle through
@@ -351,9 +366,8 @@ def e2e_workload(lwq, workload: str, dev, steps: int, dist_on: bool):
     calls = step_calls(workload)
     host = []
     for fmt, act, M, N, K, seed in calls:
-        g = inputs.rng(seed)
-        Wq = inputs.make_weights(fmt, g, N, K)
-        x = inputs.activations(inputs.rng(seed + 1000003), M, K, act)
+        Wq = call_weights(fmt, N, K, seed)
+        x = call_activations(act, M, K, seed)
         Wp = torch.from_numpy(Wq).pin_memory()
         xp = torch.from_numpy(x.view(np.int16) if x.dtype == np.uint16 else x).pin_memory()
         yp = torch.empty((M, N), dtype=torch.float32).pin_memory()
@@ -403,10 +417,10 @@ def cpu_baseline(workload: str, budget_s: float = 15.0) -> dict:
     def make(rows):
         data = []
         for fmt, act, M, N, K, seed in calls:
-            g = inputs.rng(seed)
             n = min(rows, N)
-            Wq = inputs.make_weights(fmt, g, n, K)
-            x = inputs.activations(inputs.rng(seed + 1000003), M, K, act)
+            Wq = call_weights(fmt, N, K, seed)[:n] if isinstance(seed, tuple) else \
+                inputs.make_weights(fmt, inputs.rng(seed), n, K)
+            x = call_activations(act, M, K, seed)
             data.append((fmt, act, M, n, K, Wq, x))
         return data
 
@@ -662,7 +676,7 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--extra-steps", type=int, default=400)
     ap.add_argument("--extra", nargs="*", default=["q8_0_gemv_4096x4096", "q4_k_7b_layer_decode",
-                                                   "q4_0_prefill_gemm"])
+                                                   "q4_k_7b_layer_decode_fused", "q4_0_prefill_gemm"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="time the format x batch sweep instead (one JSON line per point)")

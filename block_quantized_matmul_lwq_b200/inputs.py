@@ -182,6 +182,12 @@ WORKLOADS = {
         # (N, K) of q, k, v, o, gate, up, down
         shapes=[(4096, 4096)] * 4 + [(11008, 4096), (11008, 4096), (4096, 11008)],
         seeds=[0, 1, 2, 3, 4, 5, 6]),
+    # the same layer with q, k, v stored as one [12288][row] weight and gate, up as one
+    # [22016][row] weight (rows concatenated in that order): four calls instead of seven
+    "q4_k_7b_layer_decode_fused": dict(
+        fmt="q4_k", act="f16", Ms=[1],
+        shapes=[(12288, 4096), (4096, 4096), (22016, 4096), (4096, 11008)],
+        seeds=[(0, 1, 2), 3, (4, 5), 6]),
     "q4_0_prefill_gemm": dict(fmt="q4_0", act="bf16", Ms=[512, 2048],
                               shapes=[(11008, 4096), (4096, 11008)], seeds=[0, 0]),
 }

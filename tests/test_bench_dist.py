@@ -102,3 +102,24 @@ def test_profiled_traffic_only_for_matching_sources(tmp_path, monkeypatch):
     assert bench.profiled_traffic() == 12345
     p.write_text("traffic_bytes_per_step: 12345\ncsrc_sha256: " + "0" * 64 + "\n")
     assert bench.profiled_traffic() is None                     # kernels changed since the capture
+
+
+def test_fused_layer_is_the_layer_with_rows_concatenated():
+    """The fused Q4_K layer stacks q, k, v and gate, up row-wise: the same weights and bytes in 4 calls, not 7."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+
+    import bench
+
+    plain = bench.step_calls("q4_k_7b_layer_decode")
+    fused = bench.step_calls("q4_k_7b_layer_decode_fused")
+    assert len(plain) == 7 and len(fused) == 4
+    wbytes = lambda calls: sum(N * bench.inputs.row_bytes(f, K) for f, a, M, N, K, s in calls)
+    assert wbytes(plain) == wbytes(fused)
+    # weights generated at reduced K so the check stays fast: stacking commutes with generation
+    f, a, M, N, K, seed = fused[0]
+    K = 256
+    stacked = bench.call_weights(f, N, K, seed)
+    parts = [bench.call_weights(f, N // 3, K, s) for s in seed]
+    assert np.array_equal(stacked, np.concatenate(parts, axis=0))
+    assert stacked.shape == (N, bench.inputs.row_bytes(f, K))

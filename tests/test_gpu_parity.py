@@ -253,3 +253,18 @@ def test_overlap_flag_chains(dev):
         for p_, o_ in zip(plain, over):
             assert np.array_equal(p_, o_)
     assert all(np.all(np.isfinite(p_)) for p_ in plain)
+
+
+@pytest.mark.parametrize("w,a,M", [("q4_k", "f16", 1), ("q4_0", "f32", 4), ("q8_0", "bf16", 8)])
+def test_fused_projections_equal_separate_calls(dev, w, a, M):
+    """One call over weights stacked row-wise (q, k, v in one) gives, bit for bit, the
+    separate calls' outputs side by side: a row's result depends only on its own weights."""
+    K, parts = 4096, (4096, 1024, 1024)
+    Ws = [inputs.make_weights(w, inputs.rng(40 + i), n, K) for i, n in enumerate(parts)]
+    x = inputs.activations(inputs.rng(49), M, K, a)
+    ys = [run_gpu(w, a, Wq, x, M, n, K, dev).cpu().numpy() for Wq, n in zip(Ws, parts)]
+    stacked = np.concatenate(Ws, axis=0)
+    y = run_gpu(w, a, stacked, x, M, sum(parts), K, dev).cpu().numpy()
+    assert np.array_equal(y, np.concatenate(ys, axis=1))
+    y_ref, den = oracle.matmul(w, stacked, x, act=a)
+    assert oracle.normalised_error(y, y_ref, den) <= TOL_GEMV
