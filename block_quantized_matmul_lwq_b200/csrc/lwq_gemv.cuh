@@ -461,18 +461,20 @@ struct Q40 {
         }
         // pass 2, one block per round.  Each round ends in shared-memory stores
         // and a warp barrier that loads may not pass, so the raw activations of
-        // round b + 2 are requested at the start of round b.
+        // round b + PF - 1 are requested at the start of round b: with one unit
+        // per lane all eight rounds' loads are in flight before the first is used.
         using Raw = typename RawPair<XT>::T;
-        Raw raw[3][UPL][2];
+        constexpr int PF = (UPL == 1) ? 8 : 3;
+        Raw raw[PF][UPL][2];
 #pragma unroll
-        for (int b = 0; b < 2; ++b) fetch_round(x, M, K, k0, lane, b, raw[b]);
+        for (int b = 0; b < PF - 1; ++b) fetch_round(x, M, K, k0, lane, b, raw[b]);
 #pragma unroll
         for (int b = 0; b < 8; ++b) {
-            if (b + 2 < 8) fetch_round(x, M, K, k0, lane, b + 2, raw[(b + 2) % 3]);
+            if (b + PF - 1 < 8) fetch_round(x, M, K, k0, lane, b + PF - 1, raw[(b + PF - 1) % PF]);
 #pragma unroll
             for (int k = 0; k < UPL; ++k) {
                 const int u = lane + 32 * k, m = u >> 3, tu = (u >> 1) & 3, h = u & 1;
-                float2 p = RawPair<XT>::get(raw[b % 3][k][0]), q = RawPair<XT>::get(raw[b % 3][k][1]);
+                float2 p = RawPair<XT>::get(raw[b % PF][k][0]), q = RawPair<XT>::get(raw[b % PF][k][1]);
                 if (UNIT) mx = fmaxf(mx, fmaxf(fmaxf(fabsf(p.x), fabsf(p.y)), fmaxf(fabsf(q.x), fabsf(q.y))));
                 // high-nibble step: x / 16 (exact: a power of two)
                 const float sc = h ? s * 0.0625f : s;
