@@ -172,7 +172,12 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
     p->nt = gemv_nt(wf, xt, p->m_group);
     const int nchunks = K / 256;
     const int nw_max = gemv_max_regs(wf, xt, p->nt) == 96 ? 16 : 14;   // register budget (see gemv_tc_kernel)
-    int nw = force && force->warps ? force->warps : (wf == LWQ_Q8_0 ? 8 : nw_max);
+    // Q8_0 chunks are twice as large, so 16 warps leave room for only 2 stages: by
+    // default 8 warps (4 stages, split-K), except where all of K fits one CTA and
+    // there are at most 4 row tiles per SM (4096 x 4096, M = 1: 6.3 -> 5.1 us).
+    const int row_tiles_16 = (N + GEMV_ROWS - 1) / GEMV_ROWS;
+    const int nw_q8 = (nchunks <= nw_max && row_tiles_16 <= 4 * sms) ? nchunks : 8;
+    int nw = force && force->warps ? force->warps : (wf == LWQ_Q8_0 ? nw_q8 : nw_max);
     if (nw > nw_max || nw < 1) return LWQ_ERR_UNSUPPORTED;
     if (nw > nchunks) nw = nchunks;
     int S = force && force->splits ? force->splits : (nchunks + nw - 1) / nw;
