@@ -181,6 +181,27 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
     if (nw > nw_max || nw < 1) return LWQ_ERR_UNSUPPORTED;
     if (nw > nchunks) nw = nchunks;
     int S = force && force->splits ? force->splits : (nchunks + nw - 1) / nw;
+    if (!(force && force->splits) && S > 1) {
+        // K spans several CTAs: up to two more splits than the fewest when that lowers the
+        // busiest CTA's work, tiles x (chunks + 4), the 4 standing for a tile's fixed cost
+        // (its reduction and barrier round trips).  Q4_K, K = 11008, N = 4096: 3 splits leave
+        // a CTA 6 tiles x 15 chunks, 4 splits 7 x 11: 9.9 -> 9.2 us.  Fewer chunks than that
+        // per tile lose (Q8_0, N = 32000, 4 splits of 4 chunks: 24.7 -> 29 us).
+        const int rt = (N + GEMV_ROWS - 1) / GEMV_ROWS;
+        long best = -1;
+        const int s_min = S;
+        for (int s = s_min; s <= s_min + 2; ++s) {
+            const int c = (nchunks + s - 1) / s;
+            const int se = (nchunks + c - 1) / c;   // splits left after dropping empty ones
+            const int g = sms / se;
+            if (g < 1) continue;
+            const long cost = (long)((rt + g - 1) / g) * (c + 4);
+            if (best < 0 || cost < best) {
+                best = cost;
+                S = se;
+            }
+        }
+    }
     if (S < 1) return LWQ_ERR_UNSUPPORTED;
     const int cps = (nchunks + S - 1) / S;
     if (cps > nw) return LWQ_ERR_UNSUPPORTED;  // every chunk of a split needs a warp
