@@ -165,6 +165,61 @@ def matmul_sampled(fmt: str, Wq: np.ndarray, x: np.ndarray, ms, ns, K: int | Non
     return y, den
 
 
+# ------------------------------------------------ int8 activations
+# "Compute Shaders con WebGPU para Inferencia ML" lists quantized arithmetic
+# without runtime dequantization among the reasons to write the kernels by hand,
+# and its quantized matmul scales groups of 32.  The reading implemented here,
+# and by the library under LWQ_FLAG_ACT_I8: each run of 32 activations along K
+# of one row becomes int8 codes q with one fp32 scale d, and the matmul uses
+# x_q = q * d in place of x.  Per block, in fp32 with round-to-nearest-even:
+#   amax = max |x|;  if amax < 2^-100: d = 0 and q = 0;
+#   else d = amax / 127, s = 127 / amax, q = rint(x * s) (clamped to +-127).
+# 16-bit activations are first converted to fp32 (exactly).
+
+ACT_Q8_BLOCK = 32
+ACT_Q8_TINY = np.float32(2.0 ** -100)
+
+
+def activations_f32(x: np.ndarray, act: str | None = None) -> np.ndarray:
+    """Activations as fp32 (f16 and bf16 widen exactly)."""
+    act = _act_of(x, act)
+    x = np.ascontiguousarray(x)
+    if act == "f32":
+        return x.astype(np.float32, copy=False)
+    if act == "f16":
+        return x.view(np.float16).astype(np.float32)
+    return (x.view(np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def quantize_act_q8(x: np.ndarray, act: str | None = None):
+    """(q, d): int8 codes [M][K] and fp32 scales [M][K/32] of the activations."""
+    xf = activations_f32(x, act)
+    M, K = xf.shape
+    if K % ACT_Q8_BLOCK:
+        raise ValueError("K must be a multiple of 32")
+    blk = xf.reshape(M, K // ACT_Q8_BLOCK, ACT_Q8_BLOCK)
+    amax = np.max(np.abs(blk), axis=2)
+    tiny = amax < ACT_Q8_TINY
+    safe = np.where(tiny, np.float32(1), amax)
+    d = np.where(tiny, np.float32(0), amax / np.float32(127)).astype(np.float32)
+    s = np.where(tiny, np.float32(0), np.float32(127) / safe).astype(np.float32)
+    prod = (blk * s[:, :, None]).astype(np.float32)
+    q = np.clip(np.rint(prod), -127, 127).astype(np.int8)
+    return q.reshape(M, K), d
+
+
+def matmul_q8act(fmt: str, Wq: np.ndarray, x: np.ndarray, K: int | None = None, act: str | None = None,
+                 lib=None):
+    """(y, den) in fp64 with the activations replaced by their int8 blocks:
+    y[m,n] = sum_k w[n,k] * q[m,k] * d[m,k/32], den = sum_k |w * q * d|."""
+    q, d = quantize_act_q8(x, act)
+    M, Kx = q.shape
+    K = Kx if K is None else K
+    xq = q.astype(np.float64) * np.repeat(d.astype(np.float64), ACT_Q8_BLOCK, axis=1)
+    W = dequant(fmt, Wq, K, lib=lib).astype(np.float64)
+    return xq @ W.T, np.abs(xq) @ np.abs(W).T
+
+
 def max_threads(lib=None) -> int:
     return (lib or load()).lwq_oracle_max_threads()
 
