@@ -115,14 +115,25 @@ def call_weights(fmt: str, N: int, K: int, seed):
     return inputs.make_weights(fmt, inputs.rng(seed), N, K)
 
 
+def base_act(act: str) -> str:
+    """Activation dtype of a call; "f32:i8" is fp32 activations taken as int8 blocks (LWQ_FLAG_ACT_I8)."""
+    return act.split(":")[0]
+
+
+def call_fmt(lwq, fmt: str, act: str) -> int:
+    """The C ABI's fmt of a call."""
+    code = lwq.fmt_code(fmt, base_act(act))
+    return code | lwq.LWQ_FLAG_ACT_I8 if act.endswith(":i8") else code
+
+
 def call_activations(act: str, M: int, K: int, seed):
     """Activations of one call (a fused call takes those of its first part)."""
     s = seed[0] if isinstance(seed, tuple) else seed
-    return inputs.activations(inputs.rng(s + 1000003), M, K, act)
+    return inputs.activations(inputs.rng(s + 1000003), M, K, base_act(act))
 
 
 def call_bytes(fmt, act, M, N, K) -> int:
-    xe = 4 if act == "f32" else 2
+    xe = 4 if base_act(act) == "f32" else 2
     return N * inputs.row_bytes(fmt, K) + M * K * xe + M * N * 4
 
 
@@ -263,7 +274,7 @@ class Problem:
         W = self.weights[key][(r * self.uses[key] + self.use_index[i]) % len(self.weights[key])]
         # the weight copies are never written while timed, so each call may start
         # streaming its weights while the previous call finishes (LWQ_FLAG_OVERLAP)
-        lwq.lwq_matmul(lwq.fmt_code(fmt, act) | lwq.LWQ_FLAG_OVERLAP, W, xd, yd, M, N, K, stream=stream)
+        lwq.lwq_matmul(call_fmt(lwq, fmt, act) | lwq.LWQ_FLAG_OVERLAP, W, xd, yd, M, N, K, stream=stream)
         return lwq.lwq_last_launch_count()
 
     def enqueue_step(self, lwq, r: int, stream) -> int:
@@ -383,7 +394,7 @@ def e2e_workload(lwq, workload: str, dev, steps: int, dist_on: bool):
         for fmt, act, M, N, K, Wp, xp, yp, Wd, xd, yd in host:
             Wd.copy_(Wp, non_blocking=True)
             xd.copy_(xp, non_blocking=True)
-            lwq.lwq_matmul(lwq.fmt_code(fmt, act), Wd, xd, yd, M, N, K, stream=stream)
+            lwq.lwq_matmul(call_fmt(lwq, fmt, act), Wd, xd, yd, M, N, K, stream=stream)
             yp.copy_(yd, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -469,7 +480,7 @@ def run_gpu_arm(args):
     ws_bytes = 0
     for wl in [HEADLINE] + args.extra:
         for fmt, act, M, N, K, seed in step_calls(wl):
-            ws_bytes = max(ws_bytes, lwq.lwq_workspace_size(lwq.fmt_code(fmt, act), M, N, K))
+            ws_bytes = max(ws_bytes, lwq.lwq_workspace_size(call_fmt(lwq, fmt, act), M, N, K))
     ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
     lwq.lwq_init(ws, ws.numel())
 
@@ -676,7 +687,8 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--extra-steps", type=int, default=400)
     ap.add_argument("--extra", nargs="*", default=["q8_0_gemv_4096x4096", "q4_k_7b_layer_decode",
-                                                   "q4_k_7b_layer_decode_fused", "q4_0_prefill_gemm"])
+                                                   "q4_k_7b_layer_decode_fused", "q4_0_gemv_11008x4096_act_i8",
+                                                   "q4_0_prefill_gemm"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="time the format x batch sweep instead (one JSON line per point)")

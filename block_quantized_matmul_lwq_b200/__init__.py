@@ -21,7 +21,14 @@ LIB_PATH = os.path.join(_HERE, "liblwq.so")
 LWQ_Q8_0, LWQ_Q4_0, LWQ_Q4_K = 1, 2, 3
 LWQ_ACT_F32, LWQ_ACT_F16, LWQ_ACT_BF16 = 0x000, 0x100, 0x200
 LWQ_FLAG_OVERLAP = 0x1000   # weights constant: allow programmatic dependent launch
+LWQ_FLAG_ACT_I8 = 0x2000    # int8 activation blocks of 32 (integer block dot products)
 LWQ_OK = 0
+LWQ_ERR_INVALID_ARG = 1
+LWQ_ERR_UNSUPPORTED = 2
+LWQ_ERR_MISALIGNED = 3
+LWQ_ERR_NOT_INITIALIZED = 4
+LWQ_ERR_WORKSPACE_TOO_SMALL = 5
+LWQ_ERR_CUDA = 6
 LWQ_ERR_DEVICE_TIMEOUT = 7
 STATUS = {0: "LWQ_OK", 1: "LWQ_ERR_INVALID_ARG", 2: "LWQ_ERR_UNSUPPORTED", 3: "LWQ_ERR_MISALIGNED",
           4: "LWQ_ERR_NOT_INITIALIZED", 5: "LWQ_ERR_WORKSPACE_TOO_SMALL", 6: "LWQ_ERR_CUDA",

@@ -84,7 +84,7 @@ int act_code(int fmt) {
 
 int check_fmt_k(int fmt, long K) {
     const int wf = fmt & LWQ_FMT_MASK;
-    if (fmt & ~(LWQ_FMT_MASK | LWQ_ACT_MASK | LWQ_FLAG_OVERLAP)) return LWQ_ERR_UNSUPPORTED;
+    if (fmt & ~(LWQ_FMT_MASK | LWQ_ACT_MASK | LWQ_FLAG_OVERLAP | LWQ_FLAG_ACT_I8)) return LWQ_ERR_UNSUPPORTED;
     if (block_weights(wf) == 0 || act_code(fmt) < 0) return LWQ_ERR_UNSUPPORTED;
     if (K <= 0 || K % block_weights(wf)) return LWQ_ERR_INVALID_ARG;
     return LWQ_OK;
@@ -94,6 +94,7 @@ int check_fmt_k(int fmt, long K) {
 struct Plan {
     lwq_config cfg;
     int nt;          // GEMV n8 tiles (1: <= 8 activation rows per pass, 2: <= 16)
+    bool i8;         // GEMV with int8 activation blocks (LWQ_FLAG_ACT_I8)
     int m_group;     // activation rows per pass
     size_t smem;
     size_t ws_need;  // workspace bytes for one pass
@@ -134,6 +135,11 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
     const int wf = fmt & LWQ_FMT_MASK, xt = act_code(fmt);
     memset(p, 0, sizeof(*p));
     int path = force && force->path ? force->path : 0;
+    if (fmt & LWQ_FLAG_ACT_I8) {
+        // int8 activation blocks: tensor-core GEMV only
+        if (path && path != 1) return LWQ_ERR_UNSUPPORTED;
+        path = 1;
+    }
     if (!path) {
         if (M > 16 && xt != X_F32 && gemm_eligible(wf, xt, K))
             path = 2;
@@ -167,9 +173,11 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
         return LWQ_OK;
     }
     if (path != 1 || !tc_gemv_eligible(wf, xt, K)) return LWQ_ERR_UNSUPPORTED;
-    const int mmax = (xt == X_F32) ? 8 : 16;
+    p->i8 = (fmt & LWQ_FLAG_ACT_I8) != 0;
+    if (p->i8 && (wf != LWQ_Q4_0 || M > 16)) return LWQ_ERR_UNSUPPORTED;
+    const int mmax = (xt == X_F32 || p->i8) ? 8 : 16;   // int8 blocks: one n8 tile of rows per pass
     p->m_group = M < mmax ? M : mmax;
-    p->nt = gemv_nt(wf, xt, p->m_group);
+    p->nt = p->i8 ? 1 : gemv_nt(wf, xt, p->m_group);
     const int nchunks = K / 256;
     const int nw_max = gemv_max_regs(wf, xt, p->nt) == 96 ? 16 : 14;   // register budget (see gemv_tc_kernel)
     // Q8_0 chunks are twice as large, so 16 warps leave room for only 2 stages: by
@@ -269,10 +277,10 @@ cudaError_t ensure_smem(const void *kern, size_t smem) {
     return cudaSuccess;
 }
 
-template <int FMT, int XT, int NT, bool ONE>
+template <int FMT, int XT, int NT, bool ONE, bool I8 = false>
 cudaError_t launch_gemv_tc(const CUtensorMap &map, const GemvArgs &a, int ctas, int nw, size_t smem,
                            cudaStream_t st) {
-    auto kern = gemv_tc_kernel<FMT, XT, NT, ONE>;
+    auto kern = gemv_tc_kernel<FMT, XT, NT, ONE, I8>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), smem);
     if (e != cudaSuccess) return e;
     return launch_k(kern, ctas, (nw + 2) * 32, smem, st, a.overlap != 0, map, a);
@@ -292,8 +300,15 @@ cudaError_t launch_gemv_tc_nt(int nt, bool one, const CUtensorMap &map, const Ge
     return cudaErrorInvalidValue;
 }
 
-cudaError_t dispatch_gemv_tc(int wf, int xt, int nt, bool one, const CUtensorMap &map, const GemvArgs &a, int ctas,
-                             int nw, size_t smem, cudaStream_t st) {
+// i8: int8 activation blocks (Q4_0, one n8 tile)
+cudaError_t dispatch_gemv_tc(int wf, int xt, int nt, bool one, bool i8, const CUtensorMap &map, const GemvArgs &a,
+                             int ctas, int nw, size_t smem, cudaStream_t st) {
+    if (i8) {
+        if (wf != LWQ_Q4_0 || nt != 1) return cudaErrorInvalidValue;
+        if (xt == X_F32) return launch_gemv_tc<F_Q4_0, X_F32, 1, false, true>(map, a, ctas, nw, smem, st);
+        if (xt == X_F16) return launch_gemv_tc<F_Q4_0, X_F16, 1, false, true>(map, a, ctas, nw, smem, st);
+        return launch_gemv_tc<F_Q4_0, X_BF16, 1, false, true>(map, a, ctas, nw, smem, st);
+    }
 #define LWQ_TC(F)                                                                                      \
     if (xt == X_F32) return launch_gemv_tc_nt<F, X_F32>(nt, one, map, a, ctas, nw, smem, st);         \
     if (xt == X_F16) return launch_gemv_tc_nt<F, X_F16>(nt, one, map, a, ctas, nw, smem, st);         \
@@ -508,8 +523,8 @@ int run(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, c
         a.stages = p.cfg.stages;
         a.timeout_ns = kTimeoutNs;
         a.overlap = overlap;
-        const int nt = gemv_nt(wf, xt, mg);
-        cudaError_t e = dispatch_gemv_tc(wf, xt, nt, mg == 1, map, a, p.cfg.ctas, p.cfg.warps,
+        const int nt = p.i8 ? 1 : gemv_nt(wf, xt, mg);
+        cudaError_t e = dispatch_gemv_tc(wf, xt, nt, mg == 1 && !p.i8, p.i8, map, a, p.cfg.ctas, p.cfg.warps,
                                          gemv_smem(wf, p.cfg.warps, p.cfg.stages, gemv_ot(xt, nt)), st);
         if (e != cudaSuccess) return LWQ_ERR_CUDA;
         ++launches;

@@ -174,6 +174,15 @@ __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint3
     mma_f16_16816(d, a, b0, b1, d);
 }
 
+// D = A * B (+0), A 16x32 s8 (row), B 32x8 s8 (col), s32 accumulate.
+__device__ __forceinline__ void imma_s8_16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%10, %10, %10, %10};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0));
+}
+
 // ------------------------------------------------- Q4_0, several activation rows
 // The MMA's N dimension carries activation columns; lane (g, t) of weight
 // rows g, g+8 takes code word t of every block (4 code bytes, 8 weights), and
@@ -588,6 +597,127 @@ struct Q40 {
             mma(cm, ad, xs[o][0], xs[o][1]);
 #pragma unroll
             for (int j = 0; j < 4; ++j) acc[o][j] += fmaf(m[o][j], 16777216.f, -512.f * cm[j]);
+        }
+    }
+};
+
+// ------------------------------------- Q4_0, int8 activation blocks (LWQ_FLAG_ACT_I8)
+// "Quantized arithmetic without runtime dequantization" ("Compute Shaders con
+// WebGPU para Inferencia ML", on why to write the kernels by hand): each run of
+// 32 activations of a row becomes int8 codes q with one fp32 scale d
+// (d = amax/127, q = rint(x * 127/amax); zero below 2^-100), and one
+// mma.m16n8k32 (s8 x s8 -> s32) takes a whole block for 8 activation rows.
+// A Q4_0 code u enters as the signed byte 16(u - 8): a high nibble in place
+// is (byte & 0xF0) ^ 0x80, a low nibble the same after a 4-bit shift.  So the
+// block's integer dot product is 16 * sum (u - 8) q, exact in s32, and
+// y += d_w * (d_x / 16) * C per block in fp32.
+//
+// Lane (g, t) reads code word t of every block, as the fp16 several-row
+// mapping does: byte j of the word is code byte e(t, j), with e(t, j) = 4t + j
+// for odd blocks and (4t - 2 + j) mod 16 for even ones (the even block starts
+// 2 bytes into its word).  Its low nibbles are weights e(t, 0..3) and feed
+// MMA k-slots 4t..4t+3; its high nibbles, weights e(t, .) + 16, feed k-slots
+// 16 + 4t..  The B fragment of the lane (activation row g) holds the
+// activation codes of the same weights in the same slots.
+template <int XT>
+struct Q40I8 {
+    uint32_t xq[8][2];   // [block][k-slots 4t.. / 16+4t..]: int8 codes of activation row g
+    float dx[8][2];      // [block][column 2t, 2t+1]: d_x / 16 of activation rows 2t, 2t+1
+    float inv;           // 1: no activation scale to undo
+
+    __device__ static __forceinline__ int cb0(int hb, int j) { return hb ? 4 * j : (j ? 4 * j - 2 : 14); }
+    __device__ static __forceinline__ int cb2(int hb, int j) { return hb ? 4 * j + 2 : 4 * j; }
+
+    __device__ static __forceinline__ uint32_t pack_s8(int a, int b, int c, int d) {
+        return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8) | ((uint32_t)(c & 0xFF) << 16) |
+               ((uint32_t)d << 24);
+    }
+    __device__ static __forceinline__ int q8(float v, float s) {
+        return max(-127, min(127, __float2int_rn(v * s)));
+    }
+
+    __device__ __forceinline__ void load_x(const void *x, int M, int K, long k0, int lane, uint32_t, uint32_t) {
+        const int g = lane >> 2, t = lane & 3;
+        const bool live = g < M;
+        const long base = (long)g * K + k0;
+        using Raw = typename RawPair<XT>::T;
+        inv = 1.f;
+#pragma unroll
+        for (int b0 = 0; b0 < 8; b0 += 4) {
+            // all loads of four blocks in flight before any is used
+            Raw r[4][4];   // [block][pairs: e(t,0..1), e(t,2..3), +16, +16]
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+                const int b = b0 + bb;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) r[bb][i] = RawPair<XT>::zero();
+                if (live) {
+                    const long e = base + 32 * b;
+                    r[bb][0] = RawPair<XT>::load(x, e + cb0(b & 1, t));
+                    r[bb][1] = RawPair<XT>::load(x, e + cb2(b & 1, t));
+                    r[bb][2] = RawPair<XT>::load(x, e + 16 + cb0(b & 1, t));
+                    r[bb][3] = RawPair<XT>::load(x, e + 16 + cb2(b & 1, t));
+                }
+            }
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+                const int b = b0 + bb;
+                float v[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = RawPair<XT>::get(r[bb][i]);
+                    v[2 * i] = f.x;
+                    v[2 * i + 1] = f.y;
+                }
+                float amax = 0.f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+                // the block's 32 elements of row g lie in lanes 4g .. 4g+3
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+                const bool zero = !(amax >= 7.888609052210118e-31f);   // 2^-100
+                const float d = zero ? 0.f : amax / 127.f;
+                const float sc = zero ? 0.f : 127.f / amax;
+                xq[b][0] = pack_s8(q8(v[0], sc), q8(v[1], sc), q8(v[2], sc), q8(v[3], sc));
+                xq[b][1] = pack_s8(q8(v[4], sc), q8(v[5], sc), q8(v[6], sc), q8(v[7], sc));
+                // columns 2t and 2t+1 carry activation rows 2t, 2t+1 (lanes 8t and 8t+4)
+                dx[b][0] = 0.0625f * __shfl_sync(0xffffffffu, d, 8 * t);
+                dx[b][1] = 0.0625f * __shfl_sync(0xffffffffu, d, 8 * t + 4);
+            }
+        }
+    }
+
+    // tb: this warp's [16 rows][144 B] box.
+    __device__ __forceinline__ void compute(uint32_t tb, float (&acc)[1][4], int lane) const {
+        const int g = lane >> 2, t = lane & 3;
+        const uint32_t r0 = tb + g * 144, r1 = r0 + 8 * 144;   // rows g, g+8
+        const uint32_t sel = t ? 0x3210u : 0x3254u;            // word t of an even block
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const uint32_t pb = 36 * p;
+            const uint32_t w00 = lds32(r0 + pb), w10 = lds32(r1 + pb);             // d(2p), codes
+            const uint32_t w04 = lds32(r0 + pb + 16), w14 = lds32(r1 + pb + 16);   // codes, d(2p+1)
+            uint32_t u[2][2];   // [block of the pair][row]
+            u[0][0] = prmt(lds32(r0 + pb + 4 * t), w04, sel);
+            u[0][1] = prmt(lds32(r1 + pb + 4 * t), w14, sel);
+            u[1][0] = lds32(r0 + pb + 20 + 4 * t);
+            u[1][1] = lds32(r1 + pb + 20 + 4 * t);
+            const float d[2][2] = {{f16_bits_to_float(w00), f16_bits_to_float(w10)},
+                                   {f16_bits_to_float(w04 >> 16), f16_bits_to_float(w14 >> 16)}};
+#pragma unroll
+            for (int hb = 0; hb < 2; ++hb) {
+                const int b = 2 * p + hb;
+                const uint32_t a0 = u[hb][0], a1 = u[hb][1];
+                // signed bytes 16 (u - 8): low nibbles of rows g, g+8, then high nibbles
+                const uint32_t a[4] = {((a0 << 4) & 0xF0F0F0F0u) ^ 0x80808080u, ((a1 << 4) & 0xF0F0F0F0u) ^ 0x80808080u,
+                                       (a0 & 0xF0F0F0F0u) ^ 0x80808080u, (a1 & 0xF0F0F0F0u) ^ 0x80808080u};
+                int c[4];
+                imma_s8_16832(c, a, xq[b][0], xq[b][1]);
+                acc[0][0] = fmaf(d[hb][0] * dx[b][0], (float)c[0], acc[0][0]);
+                acc[0][1] = fmaf(d[hb][0] * dx[b][1], (float)c[1], acc[0][1]);
+                acc[0][2] = fmaf(d[hb][1] * dx[b][0], (float)c[2], acc[0][2]);
+                acc[0][3] = fmaf(d[hb][1] * dx[b][1], (float)c[3], acc[0][3]);
+            }
         }
     }
 };
@@ -1177,7 +1307,7 @@ struct OneRowK {
 };
 
 // FMT x activation type x n8 tiles x one-row mapping
-template <int FMT, int XT, int NT, bool ONE>
+template <int FMT, int XT, int NT, bool ONE, bool I8 = false>
 struct GemvImpl;
 template <int XT, int NT>
 struct GemvImpl<F_Q4_0, XT, NT, false> : Q40<XT, NT> {};
@@ -1191,6 +1321,8 @@ template <int XT, int NT>
 struct GemvImpl<F_Q4_K, XT, NT, false> : Q4K<XT, NT> {};
 template <int XT>
 struct GemvImpl<F_Q4_K, XT, 1, true> : OneRowK<XT> {};
+template <int XT>
+struct GemvImpl<F_Q4_0, XT, 1, false, true> : Q40I8<XT> {};
 
 // ------------------------------------------------------------------ kernel
 // Registers per thread: 96 lets a CTA run 16 compute warps (+ producer and
@@ -1210,7 +1342,7 @@ constexpr int gemv_max_regs(int fmt, int xt, int nt) { return (nt == 1 || (fmt =
 // 128.
 // Shared memory: stages * NW * 16 * CB bytes of packed boxes, stages * NW *
 // 16 * 8NT fp32 partials, then 3 * stages mbarriers.
-template <int FMT, int XT, int NT, bool ONE>
+template <int FMT, int XT, int NT, bool ONE, bool I8 = false>
 __global__ void __maxnreg__(gemv_max_regs(FMT, XT, NT))
     gemv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const GemvArgs a) {
     constexpr int CB = FmtInfo<FMT>::chunk_bytes;
@@ -1218,7 +1350,7 @@ __global__ void __maxnreg__(gemv_max_regs(FMT, XT, NT))
     // fp32 activations keep one output tile (their two fp16 parts are merged
     // before the reducer: in the MMA chain for NT = 2, by the reducer for NT = 1)
     constexpr int OT = (XT == X_F32) ? 1 : NT;
-    constexpr bool MERGED = (XT == X_F32 && NT == 1 && !ONE && FMT == F_Q4_0);
+    constexpr bool MERGED = (XT == X_F32 && NT == 1 && !ONE && !I8 && FMT == F_Q4_0);
     constexpr int RED = GEMV_ROWS * 8 * OT;  // floats per warp per stage
     extern __shared__ __align__(128) uint8_t smem[];
 
@@ -1366,7 +1498,7 @@ __global__ void __maxnreg__(gemv_max_regs(FMT, XT, NT))
 
     // ---------------- compute warps
     if (warp >= nact) return;
-    GemvImpl<FMT, XT, NT, ONE> impl;
+    GemvImpl<FMT, XT, NT, ONE, I8> impl;
     pdl_wait();   // x may be the preceding kernel's output
     // staging for the activation layout: this warp's partial-sum slots of stages 0 and 1,
     // which it first writes after its first tile

@@ -73,42 +73,6 @@ static int scratch_ptr(void **out) {
     return LWQ_OK;
 }
 
-template <int FMT, int XT, int NT, bool ONE>
-static cudaError_t launch(const CUtensorMap &map, const GemvArgs &a, int ctas, int nw, size_t smem,
-                          cudaStream_t st) {
-    auto kern = gemv_tc_kernel<FMT, XT, NT, ONE>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    kern<<<ctas, (nw + 2) * 32, smem, st>>>(map, a);
-    return cudaGetLastError();
-}
-
-template <int FMT, int XT>
-static cudaError_t launch_nt(int nt, bool one, const CUtensorMap &map, const GemvArgs &a, int ctas, int nw,
-                             size_t smem, cudaStream_t st) {
-    if (nt == 1) {
-        if (one) return launch<FMT, XT, 1, true>(map, a, ctas, nw, smem, st);
-        return launch<FMT, XT, 1, false>(map, a, ctas, nw, smem, st);
-    }
-    if constexpr (XT != X_F32 || FMT == F_Q4_0) return launch<FMT, XT, 2, false>(map, a, ctas, nw, smem, st);
-    return cudaErrorInvalidValue;
-}
-
-static cudaError_t dispatch(int wf, int xt, int nt, bool one, const CUtensorMap &map, const GemvArgs &a, int ctas,
-                            int nw, size_t smem, cudaStream_t st) {
-#define LWQ_NA(F)                                                                             \
-    if (xt == X_F32) return launch_nt<F, X_F32>(nt, one, map, a, ctas, nw, smem, st);        \
-    if (xt == X_F16) return launch_nt<F, X_F16>(nt, one, map, a, ctas, nw, smem, st);        \
-    return launch_nt<F, X_BF16>(nt, one, map, a, ctas, nw, smem, st);
-    switch (wf) {
-    case LWQ_Q4_0: { LWQ_NA(F_Q4_0) }
-    case LWQ_Q8_0: { LWQ_NA(F_Q8_0) }
-    case LWQ_Q4_K: { LWQ_NA(F_Q4_K) }
-    }
-#undef LWQ_NA
-    return cudaErrorInvalidValue;
-}
-
 static size_t smem_bytes(int wf, int nw, int stages, int ot) { return lwq::gemv_smem(wf, nw, stages, ot); }
 
 }  // namespace lwq_noalloc
@@ -124,7 +88,8 @@ extern "C" int lwq_matmul_noalloc(int fmt, const void *Wq, const void *x, float 
     if (cfg.path != 1 || M > 16) return LWQ_ERR_UNSUPPORTED;
     const int wf = fmt & LWQ_FMT_MASK;
     const int xt = (fmt & LWQ_ACT_MASK) == LWQ_ACT_F32 ? X_F32 : ((fmt & LWQ_ACT_MASK) == LWQ_ACT_F16 ? X_F16 : X_BF16);
-    const int m_group = (xt == X_F32) ? (M < 8 ? M : 8) : M;
+    const bool i8 = (fmt & LWQ_FLAG_ACT_I8) != 0;
+    const int m_group = (xt == X_F32 || i8) ? (M < 8 ? M : 8) : M;
     const int S = cfg.splits;
     const int row_tiles = (N + GEMV_ROWS - 1) / GEMV_ROWS;
     if (S > 1 && (size_t)S * m_group * N * 4 > kScratchBytes) return LWQ_ERR_WORKSPACE_TOO_SMALL;
@@ -154,9 +119,9 @@ extern "C" int lwq_matmul_noalloc(int fmt, const void *Wq, const void *x, float 
         a.timeout_ns = lwq::kTimeoutNs;   // the library's 2 s wait bound
         a.overlap = 0;
         // n8 column tiles, as lwq_matmul picks them
-        const int nt = lwq::gemv_nt(wf, xt, mg);
+        const int nt = i8 ? 1 : lwq::gemv_nt(wf, xt, mg);
         const int ot = lwq::gemv_ot(xt, nt);
-        cudaError_t e = dispatch(wf, xt, nt, mg == 1, map, a, cfg.ctas, cfg.warps,
+        cudaError_t e = lwq::dispatch_gemv_tc(wf, xt, nt, mg == 1 && !i8, i8, map, a, cfg.ctas, cfg.warps,
                                  smem_bytes(wf, cfg.warps, cfg.stages, ot), st);
         if (e != cudaSuccess) return LWQ_ERR_CUDA;
         if (S > 1) {

@@ -75,6 +75,21 @@ typedef enum {
  * it to complete before reading x or writing y and the workspace.  This hides
  * launch latency between back-to-back calls. */
 #define LWQ_FLAG_OVERLAP 0x1000
+/* Optional flag, or-ed into fmt: int8 activation blocks ("quantized arithmetic
+ * without runtime dequantization", "Compute Shaders con WebGPU para Inferencia
+ * ML").  Each run of 32 activations of a row (K must be a multiple of 256) is
+ * quantized in the kernel to int8 codes q with one fp32 scale d, per block in
+ * fp32 with round-to-nearest-even:
+ *   amax = max |x|;  amax < 2^-100: d = 0, q = 0;  else d = amax / 127,
+ *   q = rint(x * (127 / amax)),
+ * 16-bit activations first widened exactly; and y = x_q * dequant(Wq)^T with
+ * x_q = q * d, the block dot products taken in integers (s8 x s8 -> s32) and
+ * scaled in fp32.  Results differ from the unquantized product by the
+ * activation rounding (max |y - y_exact| / sum |x w| stays below 1e-2 for
+ * N(0,1) activations); against x_q they agree to fp32 rounding.  Supported for
+ * Q4_0 weights, M <= 16 (passes of 8 rows); other formats and M > 16 return
+ * LWQ_ERR_UNSUPPORTED.  Activations must be finite. */
+#define LWQ_FLAG_ACT_I8 0x2000
 
 /* Bytes of one packed row of K weights (K/32*34, K/32*18, K/256*144), or 0
  * when fmt is unknown or K is not a positive multiple of the block size. */

@@ -103,3 +103,21 @@ def test_workspace_size_monotone():
     assert 0 < a <= b
     assert lwq.lwq_workspace_size(fmt, 0, 1, 256) == 0
     assert lwq.lwq_workspace_size(fmt, 1, 1, 100) == 0
+
+
+def test_python_constants_match_the_header():
+    """Every status code and #define of include/lwq.h has the same value in the binding."""
+    import re
+
+    import block_quantized_matmul_lwq_b200 as lwq
+
+    hdr = open(os.path.join(ROOT, "include", "lwq.h")).read()
+    found = 0
+    for name, val in re.findall(r"\b(LWQ_(?:OK|ERR_[A-Z_]+))\s*=\s*(\d+)", hdr):
+        assert getattr(lwq, name) == int(val), name
+        found += 1
+    for name, val in re.findall(r"#define\s+(LWQ_[A-Z0-9_]+)\s+(0x[0-9A-Fa-f]+|\d+)", hdr):
+        if hasattr(lwq, name):
+            assert getattr(lwq, name) == int(val, 0), name
+            found += 1
+    assert found >= 14
