@@ -123,3 +123,45 @@ def test_fused_layer_is_the_layer_with_rows_concatenated():
     parts = [bench.call_weights(f, N // 3, K, s) for s in seed]
     assert np.array_equal(stacked, np.concatenate(parts, axis=0))
     assert stacked.shape == (N, bench.inputs.row_bytes(f, K))
+
+
+class _Graph:
+    def __init__(self, tag, log):
+        self.tag, self.log = tag, log
+
+    def replay(self):
+        self.log.append(self.tag)
+
+
+@pytest.mark.parametrize("R,W,K", [(7, 3, 10), (7, 10, 25), (30, 3, 12), (5, 5, 5), (3, 4, 7), (4, 0, 9)])
+def test_replay_steps_times_exactly_k_steps(R, W, K):
+    """Whole rotations replay one R-step graph, the rest one-step graphs; the warm-up ends on
+    copy R-1, and the timed steps read copies 0, 1, 2, ... in order."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    log = []
+    singles = [_Graph(r, log) for r in range(R)]
+    full = _Graph("full", log)
+    bench.replay_steps(singles, full, W, first=-W)
+    warm = list(log)
+    log.clear()
+    bench.replay_steps(singles, full, K)
+    expand = lambda seq: [c for t in seq for c in (range(R) if t == "full" else [t])]
+    assert expand(warm) == [(R - W + i) % R for i in range(W)]
+    assert expand(log) == [i % R for i in range(K)]
+
+
+def test_int8_workload_codes():
+    sys.path.insert(0, ROOT)
+    import bench
+    import block_quantized_matmul_lwq_b200 as lwq
+
+    calls = bench.step_calls("q4_0_gemv_11008x4096_act_i8")
+    assert [c[2] for c in calls] == [1, 4, 8]
+    f, a, M, N, K, s = calls[0]
+    assert bench.base_act(a) == "f32"
+    assert bench.call_fmt(lwq, f, a) == lwq.fmt_code("q4_0", "f32") | lwq.LWQ_FLAG_ACT_I8
+    assert bench.call_fmt(lwq, f, "f32") == lwq.fmt_code("q4_0", "f32")
+    # the same bytes as the fp32 step: packed weights, fp32 x, fp32 y
+    assert bench.call_bytes(f, a, M, N, K) == bench.call_bytes(f, "f32", M, N, K)
