@@ -44,7 +44,7 @@ typedef enum {
 } lwq_status;
 
 /* ------------------------------------------------- format and dtype codes
- * fmt = weight format | activation dtype.
+ * fmt = weight format | activation dtype [| flags, below].
  *
  * LWQ_Q8_0: 32 weights per 34-byte block: fp16 d (little endian), int8 q[32];
  *           w = d*q.
@@ -119,7 +119,8 @@ int lwq_shutdown(void);
 /*
  * y[M,N] (fp32, row-major) = x[M,K] . dequant(Wq)^T.
  *
- *   fmt     weight format | activation dtype (codes above)
+ *   fmt     weight format | activation dtype, optionally | LWQ_FLAG_OVERLAP
+ *           and | LWQ_FLAG_ACT_I8 (codes above)
  *   Wq      device pointer, N packed rows of lwq_row_bytes(fmt, K) bytes each
  *   x       device pointer, row-major [M][K] in the activation dtype
  *   y       device pointer, row-major [M][N] fp32, fully overwritten
