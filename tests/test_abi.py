@@ -121,3 +121,33 @@ def test_python_constants_match_the_header():
             assert getattr(lwq, name) == int(val, 0), name
             found += 1
     assert found >= 14
+
+
+@pytest.mark.parametrize("w,a,M,N,K,warps,splits,stages", [
+    ("q4_0", "f32", 1, 11008, 4096, 16, 1, 4),     # one-row pass, 4-stage ring
+    ("q4_0", "f32", 4, 11008, 4096, 16, 1, 4),     # one column tile
+    ("q4_0", "f32", 8, 11008, 4096, 16, 1, 3),     # two column tiles: 3-stage ring
+    ("q4_0", "f16", 16, 4096, 4096, 14, 2, 3),     # two tiles of 16-bit rows: 14 warps at 128 registers
+    ("q8_0", "f32", 1, 4096, 4096, 16, 1, 2),      # Q8_0, K in one CTA, few row tiles: a warp per chunk
+    ("q8_0", "f16", 1, 32000, 4096, 8, 2, 4),      # Q8_0, many row tiles: 8 warps, split-K
+    ("q4_k", "f16", 1, 4096, 11008, 16, 4, 4),     # K = 43 chunks: 4 splits balance the CTAs better than 3
+    ("q4_0", "f16", 1, 4096, 14336, 16, 4, 4),     # K = 56 chunks: the fewest splits stay best
+])
+def test_config_table_rules(w, a, M, N, K, warps, splits, stages):
+    """The GEMV rows of the per-shape table chosen from measurements (148 SMs when no GPU is present)."""
+    if lwq.lwq_select_config(lwq.fmt_code("q4_0", "f32"), 1, 11008, 4096).ctas != 148:
+        pytest.skip("a device with another SM count is present")
+    cfg = lwq.lwq_select_config(lwq.fmt_code(w, a), M, N, K)
+    assert (cfg.path, cfg.warps, cfg.splits, cfg.stages) == (1, warps, splits, stages)
+
+
+def test_int8_flag_plan():
+    i8 = lwq.fmt_code("q4_0", "bf16") | lwq.LWQ_FLAG_ACT_I8
+    cfg = lwq.lwq_select_config(i8, 16, 4096, 4096)
+    assert cfg.path == 1
+    # passes of 8 rows: the workspace for M=16 is that of one 8-row pass
+    assert lwq.lwq_workspace_size(i8, 16, 4096, 11008) == lwq.lwq_workspace_size(i8, 8, 4096, 11008)
+    for fmt, M, K in ((lwq.fmt_code("q8_0", "f16") | lwq.LWQ_FLAG_ACT_I8, 1, 4096), (i8, 17, 4096), (i8, 1, 288)):
+        with pytest.raises(lwq.LwqError) as e:
+            lwq.lwq_select_config(fmt, M, 64, K)
+        assert e.value.status == lwq.LWQ_ERR_UNSUPPORTED
