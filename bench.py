@@ -59,23 +59,20 @@ def csrc_sha256() -> str:
     return h.hexdigest()
 
 
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "gemv_tc_kernel_q4_0_f32_11008x4096.md")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
-def profiled_traffic() -> int | None:
-    """DRAM bytes (read + write) of one headline step from the committed ncu summary,
-    or None when the summary is missing or the kernel sources changed since it was taken."""
-    import re
+def profiled_traffic(workload: str) -> int | None:
+    """DRAM bytes (read + write) of one step of `workload`, from the ncu counters recorded in
+    profiles/traffic.json, or None when none are recorded or the CUDA sources changed since."""
     try:
-        with open(PROFILE_SUMMARY) as f:
-            text = f.read()
-    except OSError:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f).get(workload)
+    except (OSError, ValueError):
         return None
-    m1 = re.search(r"^traffic_bytes_per_step:\s*(\d+)", text, re.M)
-    m2 = re.search(r"^csrc_sha256:\s*([0-9a-f]{64})", text, re.M)
-    if not (m1 and m2) or m2.group(1) != csrc_sha256():
+    if not rec or rec.get("csrc_sha256") != csrc_sha256():
         return None
-    return int(m1.group(1))
+    return int(rec["bytes_per_step"])
 
 
 def load_peaks() -> tuple[dict, str]:
@@ -420,7 +417,7 @@ def e2e_workload(lwq, workload: str, dev, steps: int, dist_on: bool):
 
 def cpu_baseline(workload: str, budget_s: float = 15.0) -> dict:
     """The oracle as it stands, on the host cores, for about budget_s seconds of CPU work:
-    whole steps repeated when a step is short, else a row sample of one step."""
+    two thirds with every core (the line's value), one third with one thread."""
     import oracle
     calls = step_calls(workload)
     threads = oracle.max_threads()
@@ -435,30 +432,127 @@ def cpu_baseline(workload: str, budget_s: float = 15.0) -> dict:
             data.append((fmt, act, M, n, K, Wq, x))
         return data
 
-    def run(data, reps):
+    def run(data, reps, nthreads):
         t0 = time.perf_counter()
         for _ in range(reps):
             for fmt, act, M, n, K, Wq, x in data:
-                oracle.matmul(fmt, Wq, x, act=act)
+                oracle.matmul(fmt, Wq, x, act=act, nthreads=nthreads)
         return time.perf_counter() - t0
 
-    full_rows = max(c[3] for c in calls)
-    data = make(64)
-    t_row = run(data, 1) / 64
-    if t_row * full_rows <= budget_s / 4:
-        data = make(full_rows)
-        t_step = run(data, 1)
-        reps = max(1, min(10000, int(budget_s / max(t_step, 1e-9))))
-        sample = f"{reps} repetitions of one whole step (every weight row of every call; fp64 C oracle, OpenMP)"
-    else:
-        rows = max(16, min(full_rows, int(budget_s / max(t_row, 1e-9))))
-        data = make(rows)
-        reps = 1
-        sample = f"first {rows} weight rows of every call of one step (fp64 C oracle, OpenMP)"
-    total_s = run(data, reps)
-    total_bytes = reps * sum(call_bytes(fmt, act, M, n, K) for fmt, act, M, n, K, Wq, x in data)
-    return {"value": total_bytes / total_s / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": sample, "seconds": round(total_s, 2)}
+    def measure(nthreads, budget):
+        full_rows = max(c[3] for c in calls)
+        data = make(64)
+        t_row = run(data, 1, nthreads) / 64
+        if t_row * full_rows <= budget / 4:
+            data = make(full_rows)
+            t_step = run(data, 1, nthreads)
+            reps = max(1, min(10000, int(budget / max(t_step, 1e-9))))
+            sample = f"{reps} repetitions of one whole step (every weight row of every call; fp64 C oracle)"
+        else:
+            rows = max(16, min(full_rows, int(budget / max(t_row, 1e-9))))
+            data = make(rows)
+            reps = 1
+            sample = f"first {rows} weight rows of every call of one step (fp64 C oracle)"
+        total_s = run(data, reps, nthreads)
+        total_bytes = reps * sum(call_bytes(fmt, act, M, n, K) for fmt, act, M, n, K, Wq, x in data)
+        return total_bytes / total_s / 1e9, sample, total_s
+
+    v_all, s_all, t_all = measure(threads, budget_s * 2 / 3)
+    v_one, s_one, t_one = measure(1, budget_s / 3)
+    return {"value": round(v_all, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": s_all + f", OpenMP on {threads} threads", "seconds": round(t_all, 2),
+            "single_thread": {"value": round(v_one, 4), "unit": "GB/s", "cores": 1, "sample": s_one,
+                              "seconds": round(t_one, 2)}}
+
+
+def host_enqueue_cost(lwq, dev, n: int = 10000, batch: int = 200) -> dict:
+    """Host time of one lwq_matmul call (the headline's M=1 call) through the C ABI: median
+    over n calls, timed in batches with the stream drained between batches so that no call
+    waits for room in the launch queue; a no-op call into the library gives the ctypes cost."""
+    import torch
+    fmt, act, M, N, K, seed = step_calls(HEADLINE)[0]
+    W = torch.from_numpy(call_weights(fmt, N, K, seed)).to(dev)
+    x = torch.from_numpy(call_activations(act, M, K, seed)).to(dev)
+    y = torch.empty((M, N), dtype=torch.float32, device=dev)
+    lib = lwq.lib()
+    code = call_fmt(lwq, fmt, act) | lwq.LWQ_FLAG_OVERLAP
+    stream = torch.cuda.Stream(device=dev)
+    sp = stream.cuda_stream
+    args = (code, W.data_ptr(), x.data_ptr(), y.data_ptr(), M, N, K, sp)
+    launches = 0
+    per_call, per_noop = [], []
+    for i in range(-2, n // batch):
+        stream.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(batch):
+            lib.lwq_matmul(*args)
+        t1 = time.perf_counter()
+        launches = lib.lwq_last_launch_count()
+        stream.synchronize()
+        t2 = time.perf_counter()
+        for _ in range(batch):
+            lib.lwq_version()
+        t3 = time.perf_counter()
+        if i >= 0:
+            per_call.append((t1 - t0) / batch * 1e6)
+            per_noop.append((t3 - t2) / batch * 1e6)
+    med, noop = statistics.median(per_call), statistics.median(per_noop)
+    return {"median_us_per_call": round(med, 3), "ctypes_noop_us": round(noop, 3),
+            "library_us_per_call": round(med - noop, 3), "calls": n, "kernels_per_call": launches,
+            "call": {"fmt": fmt, "act": act, "M": M, "N": N, "K": K}}
+
+
+def sweep_points(lwq, dev, peaks: dict, fmts=None, shapes=None, Ms=None) -> list:
+    """The format x batch sweep (fp16 activations, LWQ_FLAG_OVERLAP, rotating weight copies),
+    each point against its binding roofline min(P_tc, BW * I), I = 2MNK / bytes."""
+    import torch
+    fmts = fmts or inputs.SWEEP_FMTS
+    shapes = shapes or inputs.SWEEP_SHAPES_KN
+    Ms = Ms or inputs.SWEEP_MS
+    bw, ptc = peaks["hbm_gbs"] * 1e9, peaks["bf16_tflops"] * 1e12
+    stream = torch.cuda.Stream(device=dev)
+    out = []
+    for fmt in fmts:
+        for K, N in shapes:
+            Wq = inputs.make_weights(fmt, inputs.rng(11), N, K)
+            R = max(3, -(-(4 * L2_BYTES) // Wq.nbytes))
+            base = torch.from_numpy(Wq).to(dev)
+            Ws = [base] + [base.clone() for _ in range(R - 1)]
+            for M in Ms:
+                x = inputs.activations(inputs.rng(12), M, K, "f16")
+                xd = torch.from_numpy(x.view(np.int16)).to(dev)
+                yd = torch.empty((M, N), dtype=torch.float32, device=dev)
+                code = lwq.fmt_code(fmt, "f16") | lwq.LWQ_FLAG_OVERLAP
+                cfg = lwq.lwq_select_config(lwq.fmt_code(fmt, "f16"), M, N, K)
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.stream(stream):
+                    for W in Ws:
+                        lwq.lwq_matmul(code, W, xd, yd, M, N, K, stream=stream)
+                    stream.synchronize()
+                    with torch.cuda.graph(g, stream=stream):
+                        for W in Ws:
+                            lwq.lwq_matmul(code, W, xd, yd, M, N, K, stream=stream)
+                    g.replay()
+                    stream.synchronize()
+                    reps = max(3, min(50, int(2e-3 / max(1e-6, 1e-5 * len(Ws)))))
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    for _ in range(reps):
+                        g.replay()
+                    e1.record(stream)
+                stream.synchronize()
+                ms = e0.elapsed_time(e1) / (reps * len(Ws))
+                nbytes, flops = call_bytes(fmt, "f16", M, N, K), call_flops(M, N, K)
+                t = ms / 1e3
+                attain = min(ptc, bw * flops / nbytes)
+                bound = "hbm" if bw * flops / nbytes < ptc else "tensor"
+                out.append({"fmt": fmt, "M": M, "K": K, "N": N, "ms": round(ms, 5),
+                            "path": {1: "gemv", 2: "gemm", 3: "simple"}[cfg.path],
+                            "GB/s": round(nbytes / t / 1e9, 1), "TFLOP/s": round(flops / t / 1e12, 2),
+                            "bound": bound, "frac": round(flops / t / attain, 4)})
+                del g
+            del Ws, base
+    return out
 
 
 def run_gpu_arm(args):
@@ -481,6 +575,9 @@ def run_gpu_arm(args):
     for wl in [HEADLINE] + args.extra:
         for fmt, act, M, N, K, seed in step_calls(wl):
             ws_bytes = max(ws_bytes, lwq.lwq_workspace_size(call_fmt(lwq, fmt, act), M, N, K))
+    if not args.no_sweep:
+        ws_bytes = max([ws_bytes] + [lwq.lwq_workspace_size(lwq.fmt_code(f, "f16"), max(inputs.SWEEP_MS), n, k)
+                                     for f in inputs.SWEEP_FMTS for k, n in inputs.SWEEP_SHAPES_KN])
     ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
     lwq.lwq_init(ws, ws.numel())
 
@@ -496,12 +593,12 @@ def run_gpu_arm(args):
     # roofline: every launch in the timed region is the headline kernel (tensor-core GEMV,
     # Q4_0 x fp32); achieved = algorithmic bytes per step / device time per step on this rank
     achieved = prob.bytes_per_step / (ms_local / args.steps / 1e3) / 1e9
-    traffic = args.traffic if args.traffic is not None else profiled_traffic()
+    traffic = args.traffic if args.traffic is not None else profiled_traffic(HEADLINE)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
                 "algorithmic_bytes_per_step": prob.bytes_per_step, "per": "step (three launches: M=1, 4, 8)",
                 "peak_source": peak_src,
-                "kernel": "lwq::gemv_tc_kernel<Q4_0, fp32 x> (M=1 one-row, M=4 one tile, M=8 two tiles)",
+                "kernel": "lwq::gemv_kernel<Q4_0, fp32 x> (M=1: one column tile, M=4: two, M=8: three)",
                 "per_call_ms": [{"M": p["call"][2], "ms": round(p["ms_mean"], 5),
                                  "GB/s": round(call_bytes(*p["call"][:5]) / p["ms_mean"] / 1e6, 1)} for p in per]}
 
@@ -532,6 +629,14 @@ def run_gpu_arm(args):
                                      for p in per2]})
         extra[wl] = rec
 
+    host = host_enqueue_cost(lwq, dev) if not args.no_host_cost else None
+    sweep = None
+    if not args.no_sweep:
+        sweep = {"act": "f16", "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"],
+                                         "source": peak_src},
+                 "frac": "achieved / min(P_tc, BW * I), I = 2MNK / (packed W + x + y bytes)",
+                 "points": sweep_points(lwq, dev, peaks)}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(HEADLINE, budget_s=args.cpu_budget)
@@ -542,10 +647,11 @@ def run_gpu_arm(args):
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
-            "config": {"workload": HEADLINE, "weights": "q4_0", "activations": "f32, held as fp16 hi + lo (22 significant bits)",
-                       "mma": "fp16 x fp16 products, f32 accumulation",
+            "config": {"workload": HEADLINE, "weights": "q4_0 (codes q - 8 exact, block scale in fp32)",
+                       "activations": "f32, all 24 significand bits (three exact bf16 parts)",
+                       "mma": "bf16 x bf16 products (exact), f32 accumulation",
                        "accumulate": "f32", "M": [1, 4, 8], "N": 11008, "K": 4096, "seed": 0,
                        "l2": f"inputs larger than L2: every call reads its own weight copy, "
                              f"{prob.copies_bytes / 1e6:.0f} MB of copies in rotation",
@@ -553,6 +659,7 @@ def run_gpu_arm(args):
                        "launch": "LWQ_FLAG_OVERLAP: programmatic dependent launches, weights constant"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": lps * args.steps, "clocks": clocks, "workloads": extra,
+            "host_enqueue": host, "sweep": sweep,
             "device_error": err,
         }
         print(json.dumps(line), flush=True)
@@ -563,8 +670,7 @@ def run_gpu_arm(args):
 
 
 def run_sweep(args):
-    """The format x batch sweep: every (format, M, K x N) point timed through lwq_matmul with fp16
-    activations, one JSON line per point (GB/s against HBM for M <= 16, TFLOP/s against bf16 for M > 16)."""
+    """The format x batch sweep alone: one JSON line per point."""
     import torch
     import block_quantized_matmul_lwq_b200 as lwq
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
@@ -574,49 +680,9 @@ def run_sweep(args):
                    for f in inputs.SWEEP_FMTS for k, n in inputs.SWEEP_SHAPES_KN)
     ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
     lwq.lwq_init(ws, ws.numel())
-    stream = torch.cuda.Stream(device=dev)
-    for fmt in inputs.SWEEP_FMTS:
-        for K, N in inputs.SWEEP_SHAPES_KN:
-            Wq = inputs.make_weights(fmt, inputs.rng(11), N, K)
-            R = max(3, -(-(4 * L2_BYTES) // Wq.nbytes))
-            base = torch.from_numpy(Wq).to(dev)
-            Ws = [base] + [base.clone() for _ in range(R - 1)]
-            for M in inputs.SWEEP_MS:
-                x = inputs.activations(inputs.rng(12), M, K, "f16")
-                xd = torch.from_numpy(x.view(np.int16)).to(dev)
-                yd = torch.empty((M, N), dtype=torch.float32, device=dev)
-                code = lwq.fmt_code(fmt, "f16") | lwq.LWQ_FLAG_OVERLAP
-                cfg = lwq.lwq_select_config(lwq.fmt_code(fmt, "f16"), M, N, K)
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.stream(stream):
-                    for W in Ws:
-                        lwq.lwq_matmul(code, W, xd, yd, M, N, K, stream=stream)
-                    stream.synchronize()
-                    with torch.cuda.graph(g, stream=stream):
-                        for W in Ws:
-                            lwq.lwq_matmul(code, W, xd, yd, M, N, K, stream=stream)
-                    g.replay()
-                    stream.synchronize()
-                    reps = max(3, min(50, int(2e-3 / max(1e-6, 1e-5 * len(Ws)))))
-                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    e0.record(stream)
-                    for _ in range(reps):
-                        g.replay()
-                    e1.record(stream)
-                stream.synchronize()
-                ms = e0.elapsed_time(e1) / (reps * len(Ws))
-                rec = {"sweep": True, "fmt": fmt, "act": "f16", "M": M, "K": K, "N": N, "ms": round(ms, 5),
-                       "path": {1: "gemv", 2: "gemm", 3: "simple"}[cfg.path]}
-                if M <= 16:
-                    gbs = call_bytes(fmt, "f16", M, N, K) / (ms / 1e3) / 1e9
-                    rec.update({"GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4)})
-                else:
-                    tf = call_flops(M, N, K) / (ms / 1e3) / 1e12
-                    rec.update({"TFLOP/s": round(tf, 1), "frac_of_bf16": round(tf / peaks["bf16_tflops"], 4)})
-                rec["peak_source"] = peak_src
-                print(json.dumps(rec), flush=True)
-                del g
-            del Ws, base
+    for rec in sweep_points(lwq, dev, peaks):
+        rec.update({"sweep": True, "act": "f16", "peak_source": peak_src})
+        print(json.dumps(rec), flush=True)
     torch.cuda.synchronize(dev)
     err = lwq.lwq_get_device_error()
     print(json.dumps({"sweep_done": True, "device_error": err}), flush=True)
@@ -690,13 +756,15 @@ def parse_args(argv=None):
                                                    "q4_k_7b_layer_decode_fused", "q4_0_gemv_11008x4096_act_i8",
                                                    "q4_0_prefill_gemm"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true", help="leave the format x batch sweep out of the line")
+    ap.add_argument("--no-host-cost", action="store_true", help="leave the host enqueue timing out")
     ap.add_argument("--sweep", action="store_true",
                     help="time the format x batch sweep instead (one JSON line per point)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--reference-budget", type=float, default=60.0)
     ap.add_argument("--traffic", type=float, default=None,
-                    help="ncu DRAM bytes per step of the headline kernels (default: the committed profile "
-                         "summary, when the CUDA sources still match it)")
+                    help="ncu DRAM bytes per step of the headline kernels (default: profiles/traffic.json, "
+                         "when the CUDA sources still match it)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

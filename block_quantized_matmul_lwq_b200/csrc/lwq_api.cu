@@ -93,36 +93,23 @@ int check_fmt_k(int fmt, long K) {
 // ---------------------------------------------------------- configuration
 struct Plan {
     lwq_config cfg;
-    int nt;          // GEMV n8 tiles (1: <= 8 activation rows per pass, 2: <= 16)
+    int nt;          // GEMV n8 column tiles (activation rows x parts / 8)
     bool i8;         // GEMV with int8 activation blocks (LWQ_FLAG_ACT_I8)
     int m_group;     // activation rows per pass
+    int cps;         // GEMV: chunks of 256 weights per split (the depth of one TMA box)
     size_t smem;
     size_t ws_need;  // workspace bytes for one pass
 };
 
-// packed boxes + fp32 partials + full/empty/reduced mbarriers per stage
-// (ot: output tiles of 8 activation columns; fp32 activations always use one)
-size_t gemv_smem(int wf, int nw, int stages, int ot) {
-    const int cb = (wf == LWQ_Q8_0) ? 272 : 144;
-    return (size_t)stages * nw * GEMV_ROWS * cb + (size_t)stages * nw * GEMV_ROWS * 8 * ot * 4 +
-           (size_t)3 * stages * 8;
+// n8 column tiles of the GEMV for a pass of mg activation rows: each row takes
+// P columns (P = 3 bf16 parts for fp32 activations, else 1), 8 columns per tile.
+inline int gemv_nt(int xt, bool i8, int mg) { return i8 ? 1 : (mg * gemv_parts(xt, i8) + 7) / 8; }
+inline int gemv_chunk_bytes(int wf) { return wf == LWQ_Q8_0 ? 272 : 144; }
+inline size_t gemv_smem(int wf, int cps, int stages, int nt, bool i8, int xt) {
+    return gemv_smem_layout(gemv_chunk_bytes(wf), cps, stages, nt, wf == LWQ_Q4_K, gemv_parts(xt, i8) > 1).total;
 }
 
-// n8 column tiles of the GEMV for a pass of mg activation rows: 16-bit
-// activations, 8 rows per tile; fp32 Q4_0, one tile of 4 rows x 2 fp16 parts
-// up to 4 rows and two tiles (one per part) up to 8; other fp32 formats, one
-// tile (parts in separate MMAs).
-inline int gemv_nt(int wf, int xt, int mg) {
-    if (xt == X_F32) return (wf == LWQ_Q4_0 && mg > 4) ? 2 : 1;
-    return mg <= 8 ? 1 : 2;
-}
-inline int gemv_ot(int xt, int nt) { return xt == X_F32 ? 1 : nt; }
-
-bool tc_gemv_eligible(int wf, int xt, long K) {
-    (void)wf;
-    (void)xt;
-    return K % 256 == 0;
-}
+bool tc_gemv_eligible(long K) { return K % 256 == 0; }
 
 // Workspace layout: fp32 split-K partials [S][m_group][N].  Nothing in it
 // needs to start at any particular value.
@@ -143,7 +130,7 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
     if (!path) {
         if (M > 16 && xt != X_F32 && gemm_eligible(wf, xt, K))
             path = 2;
-        else if (tc_gemv_eligible(wf, xt, K))
+        else if (tc_gemv_eligible(K))
             path = 1;
         else
             path = 3;
@@ -172,63 +159,47 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
         p->cfg.splits = 1;
         return LWQ_OK;
     }
-    if (path != 1 || !tc_gemv_eligible(wf, xt, K)) return LWQ_ERR_UNSUPPORTED;
+    if (path != 1 || !tc_gemv_eligible(K)) return LWQ_ERR_UNSUPPORTED;
     p->i8 = (fmt & LWQ_FLAG_ACT_I8) != 0;
     if (p->i8 && (wf != LWQ_Q4_0 || M > 16)) return LWQ_ERR_UNSUPPORTED;
-    const int mmax = (xt == X_F32 || p->i8) ? 8 : 16;   // int8 blocks: one n8 tile of rows per pass
+    // rows per pass: 8 with fp32 activations (3 parts, 24 columns) or int8 blocks, else 16
+    const int mmax = (xt == X_F32 || p->i8) ? 8 : 16;
     p->m_group = M < mmax ? M : mmax;
-    p->nt = p->i8 ? 1 : gemv_nt(wf, xt, p->m_group);
+    p->nt = gemv_nt(xt, p->i8, p->m_group);
+    const int kw = p->i8 ? 256 : gemv_kw(p->nt);
+    const int wpc = CHUNK / kw;              // compute warps per chunk
+    const int cmax = GEMV_W / wpc;           // chunks a CTA can hold
     const int nchunks = K / 256;
-    const int nw_max = gemv_max_regs(wf, xt, p->nt) == 96 ? 16 : 14;   // register budget (see gemv_tc_kernel)
-    // Q8_0 chunks are twice as large, so 16 warps leave room for only 2 stages: by
-    // default 8 warps (4 stages, split-K), except where all of K fits one CTA and
-    // there are at most 4 row tiles per SM (4096 x 4096, M = 1: 6.3 -> 5.1 us).
-    const int row_tiles_16 = (N + GEMV_ROWS - 1) / GEMV_ROWS;
-    const int nw_q8 = (nchunks <= nw_max && row_tiles_16 <= 4 * sms) ? nchunks : 8;
-    int nw = force && force->warps ? force->warps : (wf == LWQ_Q8_0 ? nw_q8 : nw_max);
-    if (nw > nw_max || nw < 1) return LWQ_ERR_UNSUPPORTED;
-    if (nw > nchunks) nw = nchunks;
-    int S = force && force->splits ? force->splits : (nchunks + nw - 1) / nw;
-    if (!(force && force->splits) && S > 1) {
-        // K spans several CTAs: up to two more splits than the fewest when that lowers the
-        // busiest CTA's work, tiles x (chunks + 4), the 4 standing for a tile's fixed cost
-        // (its reduction and barrier round trips).  Q4_K, K = 11008, N = 4096: 3 splits leave
-        // a CTA 6 tiles x 15 chunks, 4 splits 7 x 11: 9.9 -> 9.2 us.  Fewer chunks than that
-        // per tile lose (Q8_0, N = 32000, 4 splits of 4 chunks: 24.7 -> 29 us).
-        const int rt = (N + GEMV_ROWS - 1) / GEMV_ROWS;
-        long best = -1;
-        const int s_min = S;
-        for (int s = s_min; s <= s_min + 2; ++s) {
-            const int c = (nchunks + s - 1) / s;
-            const int se = (nchunks + c - 1) / c;   // splits left after dropping empty ones
-            const int g = sms / se;
-            if (g < 1) continue;
-            const long cost = (long)((rt + g - 1) / g) * (c + 4);
-            if (best < 0 || cost < best) {
-                best = cost;
-                S = se;
-            }
-        }
+    int cpc = cmax;
+    if (force && force->warps) {
+        if (force->warps < 1 || force->warps > GEMV_W) return LWQ_ERR_UNSUPPORTED;
+        cpc = force->warps / wpc > 0 ? force->warps / wpc : 1;
     }
+    int S = force && force->splits ? force->splits : (nchunks + cpc - 1) / cpc;
     if (S < 1) return LWQ_ERR_UNSUPPORTED;
     const int cps = (nchunks + S - 1) / S;
-    if (cps > nw) return LWQ_ERR_UNSUPPORTED;  // every chunk of a split needs a warp
+    if (cps > cmax) return LWQ_ERR_UNSUPPORTED;  // every chunk of a split needs its warps
     S = (nchunks + cps - 1) / cps;               // drop empty splits
-    // Two-tile passes (16-bit activations, M > 8; fp32, M > 4) run a long
-    // activation prologue while the ring fills; with 3 stages instead of 4
-    // they measured 0.2-0.6 us faster (less weight traffic competing with it).
-    int stages = force && force->stages ? force->stages : (p->nt == 2 ? 3 : 4);
-    while (stages > 2 && gemv_smem(wf, nw, stages, gemv_ot(xt, p->nt)) > kSmemLimit) --stages;
-    if (stages < 2 || gemv_smem(wf, nw, stages, gemv_ot(xt, p->nt)) > kSmemLimit) return LWQ_ERR_UNSUPPORTED;
+    // weight ring: as deep as fits while two CTAs still share an SM (at most 6
+    // stages); a forced depth only has to fit the SM
+    int stages = 6;
+    if (force && force->stages) {
+        stages = force->stages;
+        if (stages < 2 || gemv_smem(wf, cps, stages, p->nt, p->i8, xt) > kSmemLimit) return LWQ_ERR_UNSUPPORTED;
+    } else {
+        while (stages > 2 && gemv_smem(wf, cps, stages, p->nt, p->i8, xt) > GEMV_SMEM_PAIR) --stages;
+    }
     const int row_tiles = (N + GEMV_ROWS - 1) / GEMV_ROWS;
+    // one CTA per SM and call: the other half of each SM is left for the next call
     int groups = force && force->ctas ? force->ctas / S : sms / S;
     if (groups < 1) groups = 1;
     if (groups > row_tiles) groups = row_tiles;
-    p->cfg.warps = nw;
+    p->cps = cps;
+    p->cfg.warps = cps * wpc;
     p->cfg.stages = stages;
     p->cfg.splits = S;
     p->cfg.ctas = S * groups;
-    p->smem = gemv_smem(wf, nw, stages, gemv_ot(xt, p->nt));
+    p->smem = gemv_smem(wf, cps, stages, p->nt, p->i8, xt);
     p->ws_need = splitk_ws(S, p->m_group, N);
     return LWQ_OK;
 }
@@ -277,48 +248,44 @@ cudaError_t ensure_smem(const void *kern, size_t smem) {
     return cudaSuccess;
 }
 
-template <int FMT, int XT, int NT, bool ONE, bool I8 = false>
-cudaError_t launch_gemv_tc(const CUtensorMap &map, const GemvArgs &a, int ctas, int nw, size_t smem,
-                           cudaStream_t st) {
-    auto kern = gemv_tc_kernel<FMT, XT, NT, ONE, I8>;
+template <int FMT, int XT, int NT, bool I8 = false>
+cudaError_t launch_gemv(const CUtensorMap &map, const GemvArgs &a, int ctas, size_t smem, cudaStream_t st) {
+    auto kern = gemv_kernel<FMT, XT, NT, I8>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), smem);
     if (e != cudaSuccess) return e;
-    return launch_k(kern, ctas, (nw + 2) * 32, smem, st, a.overlap != 0, map, a);
+    return launch_k(kern, ctas, GEMV_THREADS, smem, st, a.overlap != 0, map, a);
 }
 
-// NT = n8 column tiles (gemv_nt: 2 for 16-bit activations beyond 8 rows, and
-// for fp32 Q4_0 beyond 4 rows); the
-// one-row mapping serves passes with a single activation row (Q4_0, Q8_0).
+// NT = n8 column tiles: fp32 activations take 1..3 (3 parts per row, 8 rows
+// at most), 16-bit ones 1..2 (16 rows at most); int8 blocks one.
 template <int FMT, int XT>
-cudaError_t launch_gemv_tc_nt(int nt, bool one, const CUtensorMap &map, const GemvArgs &a, int ctas, int nw,
-                              size_t smem, cudaStream_t st) {
-    if (nt == 1) {
-        if (one) return launch_gemv_tc<FMT, XT, 1, true>(map, a, ctas, nw, smem, st);
-        return launch_gemv_tc<FMT, XT, 1, false>(map, a, ctas, nw, smem, st);
+cudaError_t launch_gemv_nt(int nt, const CUtensorMap &map, const GemvArgs &a, int ctas, size_t smem, cudaStream_t st) {
+    if (nt == 1) return launch_gemv<FMT, XT, 1>(map, a, ctas, smem, st);
+    if (nt == 2) return launch_gemv<FMT, XT, 2>(map, a, ctas, smem, st);
+    if constexpr (XT == X_F32) {
+        if (nt == 3) return launch_gemv<FMT, XT, 3>(map, a, ctas, smem, st);
     }
-    if constexpr (XT != X_F32 || FMT == F_Q4_0) return launch_gemv_tc<FMT, XT, 2, false>(map, a, ctas, nw, smem, st);
     return cudaErrorInvalidValue;
 }
 
-// i8: int8 activation blocks (Q4_0, one n8 tile)
-cudaError_t dispatch_gemv_tc(int wf, int xt, int nt, bool one, bool i8, const CUtensorMap &map, const GemvArgs &a,
-                             int ctas, int nw, size_t smem, cudaStream_t st) {
+cudaError_t dispatch_gemv(int wf, int xt, int nt, bool i8, const CUtensorMap &map, const GemvArgs &a, int ctas,
+                          size_t smem, cudaStream_t st) {
     if (i8) {
         if (wf != LWQ_Q4_0 || nt != 1) return cudaErrorInvalidValue;
-        if (xt == X_F32) return launch_gemv_tc<F_Q4_0, X_F32, 1, false, true>(map, a, ctas, nw, smem, st);
-        if (xt == X_F16) return launch_gemv_tc<F_Q4_0, X_F16, 1, false, true>(map, a, ctas, nw, smem, st);
-        return launch_gemv_tc<F_Q4_0, X_BF16, 1, false, true>(map, a, ctas, nw, smem, st);
+        if (xt == X_F32) return launch_gemv<F_Q4_0, X_F32, 1, true>(map, a, ctas, smem, st);
+        if (xt == X_F16) return launch_gemv<F_Q4_0, X_F16, 1, true>(map, a, ctas, smem, st);
+        return launch_gemv<F_Q4_0, X_BF16, 1, true>(map, a, ctas, smem, st);
     }
-#define LWQ_TC(F)                                                                                      \
-    if (xt == X_F32) return launch_gemv_tc_nt<F, X_F32>(nt, one, map, a, ctas, nw, smem, st);         \
-    if (xt == X_F16) return launch_gemv_tc_nt<F, X_F16>(nt, one, map, a, ctas, nw, smem, st);         \
-    return launch_gemv_tc_nt<F, X_BF16>(nt, one, map, a, ctas, nw, smem, st);
+#define LWQ_GV(F)                                                                   \
+    if (xt == X_F32) return launch_gemv_nt<F, X_F32>(nt, map, a, ctas, smem, st);  \
+    if (xt == X_F16) return launch_gemv_nt<F, X_F16>(nt, map, a, ctas, smem, st);  \
+    return launch_gemv_nt<F, X_BF16>(nt, map, a, ctas, smem, st);
     switch (wf) {
-    case LWQ_Q4_0: { LWQ_TC(F_Q4_0) }
-    case LWQ_Q8_0: { LWQ_TC(F_Q8_0) }
-    case LWQ_Q4_K: { LWQ_TC(F_Q4_K) }
+    case LWQ_Q4_0: { LWQ_GV(F_Q4_0) }
+    case LWQ_Q8_0: { LWQ_GV(F_Q8_0) }
+    case LWQ_Q4_K: { LWQ_GV(F_Q4_K) }
     }
-#undef LWQ_TC
+#undef LWQ_GV
     return cudaErrorInvalidValue;
 }
 
@@ -450,6 +417,52 @@ int gemm_launch(int wf, int xt, const void *Wq, const void *x, float *y, int M, 
     return LWQ_OK;
 }
 
+// The GEMV passes of one call (shared by lwq_matmul and lwq_matmul_noalloc):
+// one kernel per pass of m_group activation rows, plus the split-K sum kernel
+// when K is split; `partial` holds that pass's [S][m][N] partial sums.
+int gemv_run(const Plan &p, int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, float *partial,
+             int overlap, cudaStream_t st, int *launches) {
+    const int wf = fmt & LWQ_FMT_MASK, xt = act_code(fmt);
+    const long rb = (long)K / block_weights(wf) * block_bytes(wf);
+    const size_t xelem = (xt == X_F32) ? 4 : 2;
+    const int S = p.cfg.splits;
+    CUtensorMap map;
+    int rc = encode_weight_map(&map, Wq, wf, N, rb, p.cps);
+    if (rc) return rc;
+    int n = 0;
+    for (int m0 = 0; m0 < M; m0 += p.m_group) {
+        const int mg = (M - m0) < p.m_group ? (M - m0) : p.m_group;
+        GemvArgs a;
+        a.x = static_cast<const uint8_t *>(x) + (size_t)m0 * K * xelem;
+        a.y = y + (size_t)m0 * N;
+        a.partial = partial;
+        a.M = mg;
+        a.N = N;
+        a.K = K;
+        a.nchunks = K / 256;
+        a.splits = S;
+        a.cps = p.cps;
+        a.row_tiles = (N + GEMV_ROWS - 1) / GEMV_ROWS;
+        a.wstages = p.cfg.stages;
+        a.timeout_ns = kTimeoutNs;
+        a.overlap = overlap;
+        const int nt = gemv_nt(xt, p.i8, mg);
+        cudaError_t e = dispatch_gemv(wf, xt, nt, p.i8, map, a, p.cfg.ctas,
+                                      gemv_smem(wf, p.cps, p.cfg.stages, nt, p.i8, xt), st);
+        if (e != cudaSuccess) return LWQ_ERR_CUDA;
+        ++n;
+        if (S > 1) {
+            const long mn = (long)mg * N;
+            e = launch_k(gemv_splitk_sum_kernel, splitk_sum_blocks(mn), 256, 0, st, true,
+                         static_cast<const float *>(partial), a.y, S, mn);
+            if (e != cudaSuccess) return LWQ_ERR_CUDA;
+            ++n;
+        }
+    }
+    *launches = n;
+    return LWQ_OK;
+}
+
 int run(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, const lwq_config *force,
         void *stream) {
     t_last_launches = 0;
@@ -501,41 +514,8 @@ int run(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, c
         if (!ds.registered) return LWQ_ERR_NOT_INITIALIZED;
         if (ds.ws_bytes < p.ws_need) return LWQ_ERR_WORKSPACE_TOO_SMALL;
     }
-    const int nchunks = K / 256;
-    const int S = p.cfg.splits;
-    const int cps = (nchunks + S - 1) / S;
-    CUtensorMap map;
-    if ((rc = encode_weight_map(&map, Wq, wf, N, rb, cps))) return rc;
-    const int row_tiles = (N + GEMV_ROWS - 1) / GEMV_ROWS;
-    for (int m0 = 0; m0 < M; m0 += p.m_group) {
-        const int mg = (M - m0) < p.m_group ? (M - m0) : p.m_group;
-        GemvArgs a;
-        a.x = static_cast<const uint8_t *>(x) + (size_t)m0 * K * xelem;
-        a.y = y + (size_t)m0 * N;
-        a.partial = static_cast<float *>(ds.ws);
-        a.M = mg;
-        a.N = N;
-        a.K = K;
-        a.nchunks = nchunks;
-        a.splits = S;
-        a.chunks_per_split = cps;
-        a.row_tiles = row_tiles;
-        a.stages = p.cfg.stages;
-        a.timeout_ns = kTimeoutNs;
-        a.overlap = overlap;
-        const int nt = p.i8 ? 1 : gemv_nt(wf, xt, mg);
-        cudaError_t e = dispatch_gemv_tc(wf, xt, nt, mg == 1 && !p.i8, p.i8, map, a, p.cfg.ctas, p.cfg.warps,
-                                         gemv_smem(wf, p.cfg.warps, p.cfg.stages, gemv_ot(xt, nt)), st);
-        if (e != cudaSuccess) return LWQ_ERR_CUDA;
-        ++launches;
-        if (S > 1) {
-            const long mn = (long)mg * N;
-            e = launch_k(gemv_splitk_sum_kernel, splitk_sum_blocks(mn), 256, 0, st, true,
-                         static_cast<const float *>(a.partial), a.y, S, mn);
-            if (e != cudaSuccess) return LWQ_ERR_CUDA;
-            ++launches;
-        }
-    }
+    rc = gemv_run(p, fmt, Wq, x, y, M, N, K, static_cast<float *>(ds.ws), overlap, st, &launches);
+    if (rc) return rc;
     t_last_launches = launches;
     return LWQ_OK;
 }
@@ -557,6 +537,10 @@ __global__ void selftest_timeout_kernel(unsigned long long timeout_ns) {
 }  // namespace lwq
 
 using namespace lwq;
+
+namespace lwq_noalloc {
+void forget_device(int dev);   // lwq_noalloc.cuh: drop the cached scratch address
+}
 
 extern "C" {
 
@@ -607,8 +591,11 @@ int lwq_init(void *d_workspace, size_t bytes) {
 int lwq_shutdown(void) {
     int dev;
     if (current_device(&dev) == LWQ_OK) {
-        std::lock_guard<std::mutex> lk(g_mu);
-        g_dev[dev] = DeviceState{};
+        {
+            std::lock_guard<std::mutex> lk(g_mu);
+            g_dev[dev] = DeviceState{};
+        }
+        lwq_noalloc::forget_device(dev);
     }
     return LWQ_OK;
 }

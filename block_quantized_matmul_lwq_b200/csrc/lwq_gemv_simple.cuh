@@ -1,6 +1,5 @@
-// Simple GEMV for the shapes the tensor-core paths do not take (K not a
-// multiple of 256 for Q8_0 / Q4_0, Q4_K with fp32 or bf16 activations, and
-// groups of activation rows beyond the fast paths' limits).  One warp per
+// Simple GEMV for the shapes the tensor-core paths do not take: K not a
+// multiple of 256 (only Q8_0 and Q4_0 allow that), at any M.  One warp per
 // weight row; lanes stride over 32-weight units, decode them with byte loads
 // and accumulate in fp32 for up to 16 activation rows; a warp shuffle
 // reduction finishes each output.  Correct for every valid shape, not tuned.

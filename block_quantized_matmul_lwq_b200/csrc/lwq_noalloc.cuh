@@ -18,7 +18,12 @@
 //    other shapes return LWQ_ERR_UNSUPPORTED.
 //  * The device address of the array is looked up once per device, with that
 //    device current, on the first call made on it.  Make that first call
-//    before any stream capture on the device.
+//    before any stream capture on the device.  lwq_shutdown forgets the
+//    address on the current device (call it after a device reset, which can
+//    move the array); the next call looks it up again.
+//  * LWQ_FLAG_OVERLAP is honoured as in lwq_matmul: the kernels then wait for
+//    the preceding work on the stream before they read x or write y or the
+//    scratch.
 //  * Every call shares the one array and it keeps the previous call's
 //    contents; nothing in it needs to start at any value (partial sums are
 //    written before they are read).  Calls whose kernels overlap on the GPU
@@ -73,7 +78,12 @@ static int scratch_ptr(void **out) {
     return LWQ_OK;
 }
 
-static size_t smem_bytes(int wf, int nw, int stages, int ot) { return lwq::gemv_smem(wf, nw, stages, ot); }
+// Drop the cached address of the current device (lwq_shutdown).
+void forget_device(int dev) {
+    if (dev < 0 || dev >= kMaxDevices) return;
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_slots[dev] = DevSlot{};
+}
 
 }  // namespace lwq_noalloc
 
@@ -81,65 +91,18 @@ extern "C" int lwq_matmul_noalloc(int fmt, const void *Wq, const void *x, float 
                                   void *stream) {
     using namespace lwq_noalloc;
     if (!Wq || !x || !y || M <= 0 || N <= 0 || K <= 0) return LWQ_ERR_INVALID_ARG;
-    if (((uintptr_t)Wq | (uintptr_t)x | (uintptr_t)y) & 15u) return LWQ_ERR_MISALIGNED;
-    lwq_config cfg;
-    int rc = lwq_select_config(fmt, M, N, K, &cfg);  // argument checks and the configuration table
+    int rc = lwq::check_fmt_k(fmt, K);
     if (rc) return rc;
-    if (cfg.path != 1 || M > 16) return LWQ_ERR_UNSUPPORTED;
-    const int wf = fmt & LWQ_FMT_MASK;
-    const int xt = (fmt & LWQ_ACT_MASK) == LWQ_ACT_F32 ? X_F32 : ((fmt & LWQ_ACT_MASK) == LWQ_ACT_F16 ? X_F16 : X_BF16);
-    const bool i8 = (fmt & LWQ_FLAG_ACT_I8) != 0;
-    const int m_group = (xt == X_F32 || i8) ? (M < 8 ? M : 8) : M;
-    const int S = cfg.splits;
-    const int row_tiles = (N + GEMV_ROWS - 1) / GEMV_ROWS;
-    if (S > 1 && (size_t)S * m_group * N * 4 > kScratchBytes) return LWQ_ERR_WORKSPACE_TOO_SMALL;
+    if (((uintptr_t)Wq | (uintptr_t)x | (uintptr_t)y) & 15u) return LWQ_ERR_MISALIGNED;
+    int dev = 0;
+    if ((rc = lwq::current_device(&dev))) return rc;
+    lwq::Plan p;
+    if ((rc = lwq::make_plan(fmt, M, N, K, nullptr, lwq::sm_count(dev), &p))) return rc;
+    if (p.cfg.path != 1 || M > 16) return LWQ_ERR_UNSUPPORTED;
+    if (p.ws_need > kScratchBytes) return LWQ_ERR_WORKSPACE_TOO_SMALL;
     void *scratch = nullptr;
     if ((rc = scratch_ptr(&scratch))) return rc;
-    const long rb = (long)lwq_row_bytes(fmt, K);
-    const int nchunks = K / 256;
-    const int cps = (nchunks + S - 1) / S;
-    CUtensorMap map;   // one box per stage, as lwq_matmul's
-    if ((rc = lwq::encode_weight_map(&map, Wq, wf, N, rb, cps))) return rc;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const size_t xelem = (xt == X_F32) ? 4 : 2;
-    for (int m0 = 0; m0 < M; m0 += m_group) {
-        const int mg = (M - m0) < m_group ? (M - m0) : m_group;
-        GemvArgs a;
-        a.x = static_cast<const uint8_t *>(x) + (size_t)m0 * K * xelem;
-        a.y = y + (size_t)m0 * N;
-        a.partial = static_cast<float *>(scratch);
-        a.M = mg;
-        a.N = N;
-        a.K = K;
-        a.nchunks = nchunks;
-        a.splits = S;
-        a.chunks_per_split = cps;
-        a.row_tiles = row_tiles;
-        a.stages = cfg.stages;
-        a.timeout_ns = lwq::kTimeoutNs;   // the library's 2 s wait bound
-        a.overlap = 0;
-        // n8 column tiles, as lwq_matmul picks them
-        const int nt = i8 ? 1 : lwq::gemv_nt(wf, xt, mg);
-        const int ot = lwq::gemv_ot(xt, nt);
-        cudaError_t e = lwq::dispatch_gemv_tc(wf, xt, nt, mg == 1 && !i8, i8, map, a, cfg.ctas, cfg.warps,
-                                 smem_bytes(wf, cfg.warps, cfg.stages, ot), st);
-        if (e != cudaSuccess) return LWQ_ERR_CUDA;
-        if (S > 1) {
-            // add the splits in order: a programmatic dependent launch after the GEMV
-            const long mn = (long)mg * N;
-            cudaLaunchConfig_t lc = {};
-            lc.gridDim = dim3((unsigned)splitk_sum_blocks(mn));
-            lc.blockDim = dim3(256u);
-            lc.stream = st;
-            cudaLaunchAttribute at[1];
-            at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-            at[0].val.programmaticStreamSerializationAllowed = 1;
-            lc.attrs = at;
-            lc.numAttrs = 1;
-            if (cudaLaunchKernelEx(&lc, gemv_splitk_sum_kernel, static_cast<const float *>(a.partial), a.y, S, mn) !=
-                cudaSuccess)
-                return LWQ_ERR_CUDA;
-        }
-    }
-    return LWQ_OK;
+    int launches = 0;
+    return lwq::gemv_run(p, fmt, Wq, x, y, M, N, K, static_cast<float *>(scratch),
+                         (fmt & LWQ_FLAG_OVERLAP) ? 1 : 0, reinterpret_cast<cudaStream_t>(stream), &launches);
 }

@@ -124,17 +124,18 @@ def test_python_constants_match_the_header():
 
 
 @pytest.mark.parametrize("w,a,M,N,K,warps,splits,stages", [
-    ("q4_0", "f32", 1, 11008, 4096, 16, 1, 4),     # one-row pass, 4-stage ring
-    ("q4_0", "f32", 4, 11008, 4096, 16, 1, 4),     # one column tile
-    ("q4_0", "f32", 8, 11008, 4096, 16, 1, 3),     # two column tiles: 3-stage ring
-    ("q4_0", "f16", 16, 4096, 4096, 14, 2, 3),     # two tiles of 16-bit rows: 14 warps at 128 registers
-    ("q8_0", "f32", 1, 4096, 4096, 16, 1, 2),      # Q8_0, K in one CTA, few row tiles: a warp per chunk
-    ("q8_0", "f16", 1, 32000, 4096, 8, 2, 4),      # Q8_0, many row tiles: 8 warps, split-K
-    ("q4_k", "f16", 1, 4096, 11008, 16, 4, 4),     # K = 43 chunks: 4 splits balance the CTAs better than 3
-    ("q4_0", "f16", 1, 4096, 14336, 16, 4, 4),     # K = 56 chunks: the fewest splits stay best
+    ("q4_0", "f32", 1, 11008, 4096, 8, 2, 5),      # 3 columns (fp32 parts): one tile, a chunk per warp, 5 stages
+    ("q4_0", "f32", 4, 11008, 4096, 8, 4, 6),      # 12 columns: two tiles, half a chunk per warp
+    ("q4_0", "f32", 8, 11008, 4096, 8, 4, 6),      # 24 columns: three tiles
+    ("q4_0", "f16", 16, 4096, 4096, 8, 4, 6),      # 16 rows of 16-bit activations: two tiles
+    ("q8_0", "f32", 1, 4096, 4096, 8, 2, 3),       # Q8_0 chunks are twice as large: 3 stages
+    ("q8_0", "f16", 1, 32000, 4096, 8, 2, 3),
+    ("q4_k", "f16", 1, 4096, 11008, 8, 6, 5),      # K = 43 chunks: 6 splits of at most 8
+    ("q4_0", "f16", 1, 4096, 14336, 8, 7, 5),      # K = 56 chunks: 7 splits
 ])
 def test_config_table_rules(w, a, M, N, K, warps, splits, stages):
-    """The GEMV rows of the per-shape table chosen from measurements (148 SMs when no GPU is present)."""
+    """The GEMV rows of the per-shape table (148 SMs when no GPU is present): 8 compute warps, as
+    few splits as their chunks allow, and the deepest ring with which two CTAs still share an SM."""
     if lwq.lwq_select_config(lwq.fmt_code("q4_0", "f32"), 1, 11008, 4096).ctas != 148:
         pytest.skip("a device with another SM count is present")
     cfg = lwq.lwq_select_config(lwq.fmt_code(w, a), M, N, K)

@@ -92,16 +92,19 @@ def test_warmup_floor():
 
 
 def test_profiled_traffic_only_for_matching_sources(tmp_path, monkeypatch):
+    """roofline.traffic comes from profiles/traffic.json only while the CUDA sources match its hash."""
+    import json
     sys.path.insert(0, ROOT)
     import bench
 
-    p = tmp_path / "summary.md"
-    monkeypatch.setattr(bench, "PROFILE_SUMMARY", str(p))
-    assert bench.profiled_traffic() is None                     # no summary
-    p.write_text(f"traffic_bytes_per_step: 12345\ncsrc_sha256: {bench.csrc_sha256()}\n")
-    assert bench.profiled_traffic() == 12345
-    p.write_text("traffic_bytes_per_step: 12345\ncsrc_sha256: " + "0" * 64 + "\n")
-    assert bench.profiled_traffic() is None                     # kernels changed since the capture
+    p = tmp_path / "traffic.json"
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(p))
+    assert bench.profiled_traffic("w") is None                  # no file
+    p.write_text(json.dumps({"w": {"bytes_per_step": 12345, "csrc_sha256": bench.csrc_sha256()}}))
+    assert bench.profiled_traffic("w") == 12345
+    assert bench.profiled_traffic("other") is None              # no record for that workload
+    p.write_text(json.dumps({"w": {"bytes_per_step": 12345, "csrc_sha256": "0" * 64}}))
+    assert bench.profiled_traffic("w") is None                  # kernels changed since the capture
 
 
 def test_fused_layer_is_the_layer_with_rows_concatenated():

@@ -5,6 +5,9 @@ ragged tails; the full workload sizes are checked on sampled outputs (plus
 every tile edge) in the configuration the benchmark times.
 """
 
+import ctypes
+import functools
+
 import numpy as np
 import pytest
 import torch
@@ -32,12 +35,11 @@ def dev():
     del ws
 
 
-FAST = [("q4_0", "f32"), ("q4_0", "f16"), ("q4_0", "bf16"), ("q8_0", "f32"), ("q8_0", "f16"), ("q8_0", "bf16"),
-        ("q4_k", "f16")]
-SIMPLE_ONLY = [("q4_k", "f32"), ("q4_k", "bf16")]
+# every weight format with every activation type (all take the tensor-core GEMV when K % 256 == 0)
+FAST = [(w, a) for w in ("q4_0", "q8_0", "q4_k") for a in ("f32", "f16", "bf16")]
 
 
-@pytest.mark.parametrize("w,a", FAST + SIMPLE_ONLY)
+@pytest.mark.parametrize("w,a", FAST)
 @pytest.mark.parametrize("M,N,K", [(1, 1, 256), (1, 37, 512), (3, 100, 1024), (8, 333, 4096), (5, 61, 2816),
                                    (16, 50, 768), (12, 130, 4352), (1, 17, 6144)])
 def test_small_shapes(dev, w, a, M, N, K):
@@ -45,10 +47,10 @@ def test_small_shapes(dev, w, a, M, N, K):
 
 
 @pytest.mark.parametrize("w,a", FAST)
-@pytest.mark.parametrize("M", [2, 4, 5, 6, 7, 9, 15])
+@pytest.mark.parametrize("M", [2, 3, 4, 5, 6, 7, 8, 9, 15, 16])
 def test_every_column_layout(dev, w, a, M):
-    # row counts at and around the boundaries of the GEMV's column layouts
-    # (fp32: 4 rows x 2 parts in one tile, then one tile per part; 16-bit: 8 rows per tile)
+    # row counts at and around the boundaries of the GEMV's column layouts (fp32: 3 parts per
+    # row, so 1, 2 and 3 tiles of 8 columns at M <= 2, 5 and 8; 16-bit: 8 rows per tile)
     check_full(w, a, M, 45, 1024, dev, seed=100 + M)
 
 
@@ -97,11 +99,17 @@ def test_forced_gemv_configs(dev, w, a, warps, splits, stages):
     cfg = lwq.lwq_config()
     cfg.path, cfg.warps, cfg.splits, cfg.stages = 1, warps, splits, stages
     M, N, K = 5, 211, 3072
-    nchunks = K // 256
-    S = splits or -(-nchunks // warps)
-    if -(-nchunks // S) > warps:
+    Wq, x = inputs.make_problem(w, a, M, N, K, seed=11)
+    Wd, xd = to_device(Wq, dev), to_device(x, dev)
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device=dev)
+    rc = lwq.lib().lwq_matmul_config(lwq.fmt_code(w, a), Wd.data_ptr(), xd.data_ptr(), y.data_ptr(), M, N, K,
+                                     ctypes.byref(cfg), None)
+    if rc == lwq.LWQ_ERR_UNSUPPORTED:
         pytest.skip("configuration leaves a chunk without a warp")
-    check_full(w, a, M, N, K, dev, seed=11, cfg=cfg)
+    assert rc == lwq.LWQ_OK, lwq.lwq_status_string(rc)
+    torch.cuda.synchronize(dev)
+    y_ref, den = oracle.matmul(w, Wq, x, act=a)
+    assert oracle.normalised_error(y.cpu().numpy(), y_ref, den) <= TOL_GEMV
 
 
 @pytest.mark.parametrize("w,a", [("q4_0", "bf16"), ("q4_k", "f16"), ("q8_0", "bf16")])
@@ -156,11 +164,19 @@ def test_q4_0_prefill_gemm(dev, M, N, K):
     check_sampled("q4_0", "bf16", M, N, K, dev, seed=0, count=1500)
 
 
-@pytest.mark.parametrize("w", ["q8_0", "q4_0", "q4_k"])
-@pytest.mark.parametrize("M", [1, 16, 64])
-@pytest.mark.parametrize("K,N", [(4096, 32000), (14336, 4096)])
-def test_sweep_points_sampled(dev, w, M, K, N):
-    check_sampled(w, "f16", M, N, K, dev, seed=M + K, count=600)
+@functools.lru_cache(maxsize=2)
+def _sweep_weights(w, N, K):
+    return inputs.make_weights(w, inputs.rng(11), N, K)
+
+
+@pytest.mark.parametrize("M", inputs.SWEEP_MS)
+@pytest.mark.parametrize("K,N", inputs.SWEEP_SHAPES_KN)
+@pytest.mark.parametrize("w", inputs.SWEEP_FMTS)
+def test_sweep_points_sampled(dev, w, K, N, M):
+    """Every point of the format x batch sweep (fp16 activations), in the configuration the sweep times."""
+    Wq = _sweep_weights(w, N, K)
+    x = inputs.activations(inputs.rng(12 + M), M, K, "f16")
+    check_sampled(w, "f16", M, N, K, dev, seed=M + K, count=400, Wq=Wq, x=x)
 
 
 # ------------------------------------------------------------ error paths

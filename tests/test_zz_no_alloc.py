@@ -4,8 +4,8 @@ Such callers (code that may not call the CUDA allocator, fixed memory pools,
 plugins that receive only input and output pointers) cannot provide the
 workspace that lwq_matmul's split-K needs, so this entry point keeps its
 scratch in a static device array.  These tests call it through the C ABI and
-check its outputs against lwq_matmul's on the same inputs, for two calls in a
-row, with and without split-K.  This file is collected last on purpose.
+check its outputs against lwq_matmul's on the same inputs and against the
+oracle, for two calls in a row.  This file is collected last on purpose.
 """
 
 import numpy as np
@@ -19,8 +19,8 @@ from gpu_util import TOL_GEMV, to_device
 
 pytestmark = pytest.mark.gpu
 
-CASES = [("q4_k", "f16", 1, 4096, 11008),    # split-K (3 splits)
-         ("q4_0", "f32", 4, 11008, 4096),    # no split
+CASES = [("q4_k", "f16", 1, 4096, 11008),    # split-K (6 splits)
+         ("q4_0", "f32", 4, 11008, 4096),    # two column tiles, split-K (4 splits)
          ("q8_0", "f32", 1, 4096, 4096),     # split-K (2 splits)
          ("q4_0", "bf16", 16, 333, 6144)]    # 16 activation rows, split-K, ragged N
 
@@ -49,11 +49,16 @@ def _run_both(dev, w, a, M, N, K, seed):
         outs.append(y)
     torch.cuda.synchronize(dev)
     lwq.lwq_shutdown()
-    _, den = oracle.matmul(w, Wq, x, act=a)
+    y_oracle, den = oracle.matmul(w, Wq, x, act=a)
     ref = y_ref.cpu().numpy()
     for y in outs:
-        err = oracle.normalised_error(y.cpu().numpy(), ref.astype(np.float64), den)
-        assert err <= TOL_GEMV, f"{w}/{a} M={M} N={N} K={K}: {err:.3e}"
+        got = y.cpu().numpy()
+        # against the existing entry point's output on the same inputs ...
+        err = oracle.normalised_error(got, ref.astype(np.float64), den)
+        assert err <= TOL_GEMV, f"{w}/{a} M={M} N={N} K={K}: {err:.3e} against lwq_matmul"
+        # ... and against the oracle itself
+        err = oracle.normalised_error(got, y_oracle, den)
+        assert err <= TOL_GEMV, f"{w}/{a} M={M} N={N} K={K}: {err:.3e} against the oracle"
     return ref, [y.cpu().numpy() for y in outs]
 
 
@@ -72,7 +77,7 @@ def test_noalloc_rejects_oversize_and_other_paths(dev):
     fmt = lwq.fmt_code("q4_0", "f16")
     buf = torch.zeros(64, dtype=torch.float32, device=dev)
     p = buf.data_ptr()
-    # split-K scratch beyond the 4 MiB array: 16 rows x 32000 x K=14336 (4 splits) needs ~8 MiB
+    # split-K scratch beyond the 4 MiB array: 16 rows x 32000 x K=14336 (14 splits) needs ~29 MB
     rc = lwq.lib().lwq_matmul_noalloc(fmt, p, p, p, 16, 32000, 14336, None)
     assert rc == 5, lwq.lwq_status_string(rc)
     # prefill shapes are not offered here
