@@ -105,8 +105,10 @@ struct Plan {
 // P columns (P = 3 bf16 parts for fp32 activations, else 1), 8 columns per tile.
 inline int gemv_nt(int xt, bool i8, int mg) { return i8 ? 1 : (mg * gemv_parts(xt, i8) + 7) / 8; }
 inline int gemv_chunk_bytes(int wf) { return wf == LWQ_Q8_0 ? 272 : 144; }
-inline size_t gemv_smem(int wf, int cps, int stages, int nt, bool i8, int xt) {
-    return gemv_smem_layout(gemv_chunk_bytes(wf), cps, stages, nt, wf == LWQ_Q4_K, gemv_parts(xt, i8) > 1).total;
+inline size_t gemv_smem(int wf, int cps, int stages, int nt, bool i8, int xt, int m) {
+    return gemv_smem_layout(gemv_chunk_bytes(wf), cps, stages, nt, wf == LWQ_Q4_K, gemv_parts(xt, i8), m,
+                            xt == X_F32 ? 4 : 2, i8)
+        .total;
 }
 
 bool tc_gemv_eligible(long K) { return K % 256 == 0; }
@@ -176,21 +178,43 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
         cpc = force->warps / wpc > 0 ? force->warps / wpc : 1;
     }
     int S = force && force->splits ? force->splits : (nchunks + cpc - 1) / cpc;
-    if (S < 1) return LWQ_ERR_UNSUPPORTED;
-    const int cps = (nchunks + S - 1) / S;
-    if (cps > cmax) return LWQ_ERR_UNSUPPORTED;  // every chunk of a split needs its warps
-    S = (nchunks + cps - 1) / cps;               // drop empty splits
-    // weight ring: as deep as fits while two CTAs still share an SM (at most 6
-    // stages); a forced depth only has to fit the SM
-    int stages = 6;
-    if (force && force->stages) {
-        stages = force->stages;
-        if (stages < 2 || gemv_smem(wf, cps, stages, p->nt, p->i8, xt) > kSmemLimit) return LWQ_ERR_UNSUPPORTED;
-    } else {
-        while (stages > 2 && gemv_smem(wf, cps, stages, p->nt, p->i8, xt) > GEMV_SMEM_PAIR) --stages;
+    if (!(force && force->splits) && S > 1) {
+        // K spans several CTAs: up to two more splits than the fewest when that lowers the
+        // busiest CTA's work, tiles x (chunks + 4), the 4 standing for a tile's fixed cost
+        // (its reduction and barrier round trips).  Q4_K, K = 11008, N = 4096: 3 splits leave
+        // a CTA 6 tiles x 15 chunks, 4 splits 7 x 11.
+        const int rt = (N + GEMV_ROWS - 1) / GEMV_ROWS;
+        long best = -1;
+        const int s_min = S;
+        for (int s = s_min; s <= s_min + 2; ++s) {
+            const int c = (nchunks + s - 1) / s;
+            const int se = (nchunks + c - 1) / c;   // splits left after dropping empty ones
+            const int g = sms / se;
+            if (g < 1) continue;
+            const long cost = (long)((rt + g - 1) / g) * (c + 4);
+            if (best < 0 || cost < best) {
+                best = cost;
+                S = se;
+            }
+        }
     }
+    if (S < 1) return LWQ_ERR_UNSUPPORTED;
+    int cps = (nchunks + S - 1) / S;
+    if (cps > cmax) return LWQ_ERR_UNSUPPORTED;  // every chunk of a split needs its warps
+    // weight ring: 4 stages, fewer where shared memory is short (Q8_0 chunks
+    // are twice as large, and the CTA's slice of x is staged too); with 2 stages
+    // still too large, the CTA takes fewer chunks; a forced depth only has to fit
+    const int mg = p->m_group;
+    int stages = force && force->stages ? force->stages : 4;
+    if (!(force && force->stages)) {
+        while (stages > 2 && gemv_smem(wf, cps, stages, p->nt, p->i8, xt, mg) > kSmemLimit) --stages;
+        while (cps > 1 && !(force && force->splits) && gemv_smem(wf, cps, stages, p->nt, p->i8, xt, mg) > kSmemLimit)
+            --cps;
+    }
+    if (stages < 2 || gemv_smem(wf, cps, stages, p->nt, p->i8, xt, mg) > kSmemLimit) return LWQ_ERR_UNSUPPORTED;
+    S = (nchunks + cps - 1) / cps;               // drop empty splits
     const int row_tiles = (N + GEMV_ROWS - 1) / GEMV_ROWS;
-    // one CTA per SM and call: the other half of each SM is left for the next call
+    // one CTA per SM
     int groups = force && force->ctas ? force->ctas / S : sms / S;
     if (groups < 1) groups = 1;
     if (groups > row_tiles) groups = row_tiles;
@@ -199,7 +223,7 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
     p->cfg.stages = stages;
     p->cfg.splits = S;
     p->cfg.ctas = S * groups;
-    p->smem = gemv_smem(wf, cps, stages, p->nt, p->i8, xt);
+    p->smem = gemv_smem(wf, cps, stages, p->nt, p->i8, xt, mg);
     p->ws_need = splitk_ws(S, p->m_group, N);
     return LWQ_OK;
 }
@@ -311,22 +335,71 @@ cudaError_t dispatch_simple(int wf, int xt, const uint8_t *W, const void *x, flo
     return cudaErrorInvalidValue;
 }
 
-// The GEMV's view of Wq: 3-D, (8-byte word of a 256-weight chunk, weight row,
-// chunk), strides (row_bytes, chunk_bytes); a box of (all words, 16 rows, cps
-// chunks) lands as cps consecutive [16 rows][chunk] boxes.
-// (8-byte word of a chunk, weight row, chunk): one [cps chunks][16 rows][chunk bytes] box per GEMV stage
-int encode_weight_map(CUtensorMap *map, const void *Wq, int wf, int N, long rb, int cps) {
+// Tensor maps are encoded on the host for every call.  A map depends only on
+// its arguments, so a small per-thread cache keyed by all of them (address,
+// sizes, strides, box, type, swizzle) returns the same map again for a
+// repeated call, as in a decode loop, without the driver call.
+struct MapReq {
+    void *p;
+    uint32_t dtype, rank, swizzle, pad;
+    cuuint64_t dims[3], strides[2];
+    cuuint32_t box[3], pad2;
+};
+struct MapEntry {
+    MapReq req;
+    CUtensorMap map;
+    bool valid;
+};
+constexpr int kMapCache = 16;
+thread_local MapEntry t_maps[kMapCache];
+thread_local int t_map_next = 0;
+
+int encode_cached(const MapReq &r, CUtensorMap *out) {
+    for (int i = 0; i < kMapCache; ++i)
+        if (t_maps[i].valid && memcmp(&t_maps[i].req, &r, sizeof(MapReq)) == 0) {
+            *out = t_maps[i].map;
+            return LWQ_OK;
+        }
     EncodeTiledFn enc = encode_fn();
     if (!enc) return LWQ_ERR_CUDA;
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(out, (CUtensorMapDataType)r.dtype, r.rank, r.p, r.dims, r.strides, r.box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, (CUtensorMapSwizzle)r.swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return LWQ_ERR_CUDA;
+    MapEntry &e = t_maps[t_map_next];
+    t_map_next = (t_map_next + 1) % kMapCache;
+    e.req = r;
+    e.map = *out;
+    e.valid = true;
+    return LWQ_OK;
+}
+
+MapReq map_req(const void *p, CUtensorMapDataType dtype, int rank, CUtensorMapSwizzle swz) {
+    MapReq r;
+    memset(&r, 0, sizeof(r));   // the padding takes part in the comparison
+    r.p = const_cast<void *>(p);
+    r.dtype = (uint32_t)dtype;
+    r.rank = (uint32_t)rank;
+    r.swizzle = (uint32_t)swz;
+    return r;
+}
+
+// The GEMV's view of Wq: 3-D, (8-byte word of a 256-weight chunk, weight row,
+// chunk), strides (row_bytes, chunk_bytes); a box of (all words, 16 rows, cps
+// chunks) lands as cps consecutive [16 rows][chunk bytes] boxes, one GEMV stage.
+int encode_weight_map(CUtensorMap *map, const void *Wq, int wf, int N, long rb, int cps) {
     const int cb = (wf == LWQ_Q8_0) ? 272 : 144;
-    cuuint64_t dims[3] = {(cuuint64_t)(cb / 8), (cuuint64_t)N, (cuuint64_t)(rb / cb)};
-    cuuint64_t strides[2] = {(cuuint64_t)rb, (cuuint64_t)cb};
-    cuuint32_t box[3] = {(cuuint32_t)(cb / 8), (cuuint32_t)GEMV_ROWS, (cuuint32_t)cps};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, const_cast<void *>(Wq), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? LWQ_OK : LWQ_ERR_CUDA;
+    MapReq r = map_req(Wq, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, CU_TENSOR_MAP_SWIZZLE_NONE);
+    r.dims[0] = (cuuint64_t)(cb / 8);
+    r.dims[1] = (cuuint64_t)N;
+    r.dims[2] = (cuuint64_t)(rb / cb);
+    r.strides[0] = (cuuint64_t)rb;
+    r.strides[1] = (cuuint64_t)cb;
+    r.box[0] = (cuuint32_t)(cb / 8);
+    r.box[1] = (cuuint32_t)GEMV_ROWS;
+    r.box[2] = (cuuint32_t)cps;
+    return encode_cached(r, map);
 }
 
 // ------------------------------------------------------------- prefill GEMM
@@ -350,30 +423,26 @@ cudaError_t launch_gemm_xt(int xt, const CUtensorMap &wm, const CUtensorMap &xm,
 int gemm_launch(int wf, int xt, const void *Wq, const void *x, float *y, int M, int N, int K, long rb,
                 const lwq_config &cfg, size_t smem, unsigned long long timeout_ns, int overlap, float *partial,
                 cudaStream_t st, int *launches) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return LWQ_ERR_CUDA;
     const int cb = gemm_chunk_bytes(wf);
     const int bn = cfg.tile_m;
     CUtensorMap wm, xm;
     {
-        cuuint64_t dims[2] = {(cuuint64_t)(rb / 2), (cuuint64_t)N};
-        cuuint64_t strides[1] = {(cuuint64_t)rb};
-        cuuint32_t box[2] = {(cuuint32_t)(cb / 2), (cuuint32_t)GEMM_WROWS};
-        cuuint32_t estr[2] = {1, 1};
-        if (enc(&wm, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(Wq), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return LWQ_ERR_CUDA;
+        MapReq r = map_req(Wq, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, CU_TENSOR_MAP_SWIZZLE_NONE);
+        r.dims[0] = (cuuint64_t)(rb / 2);
+        r.dims[1] = (cuuint64_t)N;
+        r.strides[0] = (cuuint64_t)rb;
+        r.box[0] = (cuuint32_t)(cb / 2);
+        r.box[1] = (cuuint32_t)GEMM_WROWS;
+        if (encode_cached(r, &wm)) return LWQ_ERR_CUDA;
     }
     {
-        cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
-        cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-        cuuint32_t box[2] = {(cuuint32_t)GEMM_BK, (cuuint32_t)bn};
-        cuuint32_t estr[2] = {1, 1};
-        if (enc(&xm, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(x), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return LWQ_ERR_CUDA;
+        MapReq r = map_req(x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, CU_TENSOR_MAP_SWIZZLE_128B);
+        r.dims[0] = (cuuint64_t)K;
+        r.dims[1] = (cuuint64_t)M;
+        r.strides[0] = (cuuint64_t)K * 2;
+        r.box[0] = (cuuint32_t)GEMM_BK;
+        r.box[1] = (cuuint32_t)bn;
+        if (encode_cached(r, &xm)) return LWQ_ERR_CUDA;
     }
     GemmArgs a;
     a.y = y;
@@ -448,7 +517,7 @@ int gemv_run(const Plan &p, int fmt, const void *Wq, const void *x, float *y, in
         a.overlap = overlap;
         const int nt = gemv_nt(xt, p.i8, mg);
         cudaError_t e = dispatch_gemv(wf, xt, nt, p.i8, map, a, p.cfg.ctas,
-                                      gemv_smem(wf, p.cps, p.cfg.stages, nt, p.i8, xt), st);
+                                      gemv_smem(wf, p.cps, p.cfg.stages, nt, p.i8, xt, mg), st);
         if (e != cudaSuccess) return LWQ_ERR_CUDA;
         ++n;
         if (S > 1) {

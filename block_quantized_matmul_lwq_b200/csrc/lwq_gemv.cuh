@@ -1,17 +1,16 @@
 // Decode GEMV (M <= 16): y[M,N] = x[M,K] . dequant(Wq)^T, exact in x.
 //
 // Design (sm_100a):
-//  * A persistent grid of at most one CTA per SM per call, each small enough
-//    (<= 113 KB of shared memory, 10 warps at <= 96 registers) that two fit
-//    on one SM.  Every CTA triggers its programmatic dependents at once, so
-//    the next call on the stream (launched as a programmatic dependent) can
-//    become resident next to it and stream its own weights while this one
-//    finishes: one call's start-up overlaps the previous call's tail.
+//  * A persistent grid of one CTA per SM per call (16 compute warps, a TMA
+//    producer and a reducer).  Every CTA triggers its programmatic dependents
+//    at once, so the next call on the stream (a programmatic dependent
+//    launch) is scheduled as early as possible and takes each SM as soon as
+//    this call's CTA there exits.
 //  * CTA (split s, row group r) owns a slice of K (split-K factor S) and
 //    walks the 16-row weight tiles r, r+G, r+2G, ...  A producer warp stages,
 //    per tile, the tile's packed rows for all of the CTA's K chunks (256
 //    weights each) with one 3-D TMA load into a ring of shared-memory stages.
-//  * Eight compute warps each own 256 (or 128) weights of the CTA's K slice
+//  * Sixteen compute warps each own 256 (or 128) weights of the CTA's K slice
 //    and keep that slice of x in registers for the whole kernel, laid out as
 //    tensor-core B fragments.  Per tile a warp decodes its packed bytes in
 //    registers straight into A fragments holding the *signed* codes exactly
@@ -54,12 +53,9 @@ enum { X_F32 = 0, X_F16 = 1, X_BF16 = 2 };
 
 constexpr int GEMV_ROWS = 16;                     // weight rows per tile (the MMA's M)
 constexpr int CHUNK = 256;                        // weights per TMA chunk of a row
-constexpr int GEMV_W = 8;                         // compute warps per CTA
+constexpr int GEMV_W = 16;                        // compute warps per CTA
 constexpr int GEMV_THREADS = (GEMV_W + 2) * 32;   // + producer + reducer
 constexpr int GEMV_RSTAGES = 2;                   // depth of the reduction-slot ring
-// Shared memory per CTA such that two CTAs fit on one SM (228 KB, 1 KB
-// reserved per CTA).
-constexpr size_t GEMV_SMEM_PAIR = 115712;
 
 template <int FMT>
 struct FmtInfo;
@@ -86,24 +82,44 @@ struct GemvArgs {
 
 // Activation parts per element: fp32 x is split into three bf16 parts.
 __host__ __device__ constexpr int gemv_parts(int xt, bool i8) { return (xt == X_F32 && !i8) ? 3 : 1; }
-// Weights of K per compute warp: one chunk with one n8 column tile, half a
-// chunk with more (their B fragments take 32 registers per tile and chunk).
-__host__ __device__ constexpr int gemv_kw(int nt) { return nt == 1 ? 256 : 128; }
+// Weights of K per compute warp: one chunk with up to two n8 column tiles,
+// half a chunk with three (their B fragments take 32 registers per tile and
+// chunk).  A whole chunk per warp means fewer, larger tiles per CTA and K up
+// to 4096 in one CTA (no split-K): measured faster at two tiles even with a
+// few registers spilled (fp32, M = 4: 17.2 -> 14.4 us).
+__host__ __device__ constexpr int gemv_kw(int nt) { return nt <= 2 ? 256 : 128; }
+// Floats per row of a reduction slot: the tile's 8 NT columns and 4 of padding,
+// which spreads the rows of a slot over the shared-memory banks.
+__host__ __device__ constexpr int gemv_rs(int nt) { return 8 * nt + 4; }
 
-// Shared-memory layout (bytes): ring | reduction slots | Q4_K x sums | reducer scratch | mbarriers.
+// Padding (16-bit elements) after each row of the activation planes: with K
+// slices of whole chunks it makes the row stride 8 words mod 32, so four rows
+// in a row fall on distinct bank groups (the split planes also swap the two
+// words of each pair in rows 4-7 of every 8, which separates the next four).
+constexpr int GEMV_XPAD = 16;
+
+// Shared-memory layout (bytes): ring | the CTA's slice of x | reduction slots |
+// Q4_K sub-block sums of x | reducer scratch | CTA maximum | mbarriers.
+//  * The slice of x (fp path): P planes [part][activation row][K slice + pad]
+//    of 16-bit values -- the bf16 parts of fp32 x, or 16-bit x as it is.
+//    Int8 activation blocks stage the raw slice [row][K slice].
+//  * The Q4_K sums: [activation row][32-weight sub-block of the slice] fp32.
 struct GemvSmem {
-    size_t stage, ring, red, sx, scratch, bars, total;
+    size_t stage, ring, xs, red, sx, scratch, xmax, bars, total;
 };
 __host__ __device__ inline GemvSmem gemv_smem_layout(int chunk_bytes, int cps, int wstages, int nt, bool q4k,
-                                                     bool parts) {
+                                                     int parts, int m, int xelem, bool i8) {
     GemvSmem s;
     s.stage = (size_t)cps * GEMV_ROWS * chunk_bytes;
     s.ring = (size_t)wstages * s.stage;
-    s.red = (size_t)GEMV_RSTAGES * GEMV_W * GEMV_ROWS * 8 * nt * 4;
-    s.sx = q4k ? (size_t)GEMV_W * 16 * 8 * 4 : 0;
-    s.scratch = parts ? (size_t)GEMV_ROWS * 8 * nt * 4 : 0;
-    s.bars = (size_t)(2 * wstages + 2 * GEMV_RSTAGES) * 8;
-    s.total = s.ring + s.red + s.sx + s.scratch + s.bars;
+    s.xs = i8 ? (size_t)m * cps * CHUNK * xelem : (size_t)parts * m * (cps * CHUNK + GEMV_XPAD) * 2;
+    s.xs = (s.xs + 15) & ~(size_t)15;
+    s.red = (size_t)GEMV_RSTAGES * GEMV_W * GEMV_ROWS * gemv_rs(nt) * 4;
+    s.sx = q4k ? (size_t)m * cps * (CHUNK / 32) * 4 : 0;
+    s.scratch = parts > 1 ? (size_t)GEMV_ROWS * gemv_rs(nt) * 4 : 0;
+    s.xmax = 16 * 4;
+    s.bars = (size_t)(2 * wstages + 2 * GEMV_RSTAGES + 1) * 8;
+    s.total = s.ring + s.xs + s.red + s.sx + s.scratch + s.xmax + s.bars;
     return s;
 }
 
@@ -161,9 +177,18 @@ __device__ __forceinline__ uint32_t q80_pair(uint32_t w) {
 // D = A.B (C = 0) and D += A.B, bf16 or fp16 operands, fp32 accumulate.
 template <bool BF>
 __device__ __forceinline__ void mma_zero(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    const float z[4] = {0.f, 0.f, 0.f, 0.f};
-    if constexpr (BF) mma_bf16_16816(d, a, b0, b1, z);
-    else mma_f16_16816(d, a, b0, b1, z);
+    if constexpr (BF)
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%10,%10,%10,%10};"
+            : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
+    else
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%10,%10,%10,%10};"
+            : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
 }
 template <bool BF>
 __device__ __forceinline__ void mma_acc(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -211,116 +236,241 @@ struct Exact {
     uint32_t xf[NT][NB][2][2];               // [tile][block][step][reg]
     float inv;                               // 1 / the activation scale (a power of two)
 
-    // Two consecutive activations as fp32 (zeros when !live).  Coherent loads
-    // (ld.global.cg), never the read-only path: x may be the output of the
-    // preceding kernel, which can still be running when this one starts, and
-    // read-only loads may be scheduled ahead of the wait for it.
-    __device__ static __forceinline__ float2 ld2(const void *x, long off, bool live) {
-        if (!live) return make_float2(0.f, 0.f);
+    // ---------------------------------------------------------- prologue
+    // The CTA's slice of x is prepared once, by all nact compute warps
+    // together (thread i of nthr), into the part planes in shared memory;
+    // then every warp loads its B fragments from them.  Returns false when a
+    // bounded wait gave up.
+    //  * fp32 x: loaded from global memory (after the wait for the preceding
+    //    kernel), each element once, split into hi / mid / lo bf16 parts.
+    //  * 16-bit x: the reducer's bulk copies stage it in plane 0 as it is.
+    //  * Scale: the CTA's largest |x| far outside [2^-60, 2^60] (and finite)
+    //    scales the slice by a power of two (exact), undone on the results.
+    //  * Q4_K: the sub-block sums S_j of the (scaled) slice go to sx.
+    // Plane rows: row m * P + p holds part p of activation row m (the 8
+    // columns of an n8 tile are 8 consecutive plane rows).  Split planes (fp32
+    // x) swap the words of each word pair in rows r with r & 4 set (bank
+    // spread); staged 16-bit rows lie as copied.
+    struct Slice {
+        uint16_t *xp;    // plane rows [M * P][rs]
+        float *sx;       // Q4_K sums [M][nk / 32]
+        float *xmax;     // 16 per-warp maxima
+        int M, nk, rs;   // rows, K slice, plane row stride (16-bit elements)
+    };
+    __device__ static __forceinline__ int swz(int r) { return (P > 1 && (r & 4)) ? 2 : 0; }   // element offset XOR
+
+    // bf16 bits of the three parts of v (truncations: hi + mid + lo == v)
+    __device__ static __forceinline__ void split3(float v, uint32_t &hi, uint32_t &mid, uint32_t &lo) {
+        const uint32_t h = __float_as_uint(v) & 0xFFFF0000u;
+        const float r = v - __uint_as_float(h);   // exact
+        const uint32_t md = __float_as_uint(r) & 0xFFFF0000u;
+        const float l = r - __uint_as_float(md);  // exact, at most 8 significant bits
+        hi = h >> 16;
+        mid = md >> 16;
+        lo = __float_as_uint(l) >> 16;
+    }
+
+    // CTA-wide maximum of the threads' mx: per-warp maxima in shared memory, one named barrier.
+    __device__ static __forceinline__ float cta_max(float mx, const Slice &S, int nact, int warp, int lane) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) S.xmax[warp] = mx;
+        named_bar_sync(1, nact * 32);
+        float m = 0.f;
+        for (int w = 0; w < nact; ++w) m = fmaxf(m, S.xmax[w]);
+        return m;
+    }
+
+    // Power-of-two scale that puts m in [1, 2), or 1 when m is in range, zero or not finite.
+    __device__ static __forceinline__ float pick_scale(float m, float &inv_out) {
+        inv_out = 1.f;
+        if (!(m > 0.f && m <= 3.0e38f && (m < 8.673617e-19f || m > 1.1529215e18f))) return 1.f;
+        const int e = (int)((__float_as_uint(m) >> 23) & 0xFF) - 127;
+        const int es = e < -126 ? 126 : (e > 126 ? -126 : -e);
+        inv_out = __uint_as_float((uint32_t)(127 - es) << 23);
+        return __uint_as_float((uint32_t)(127 + es) << 23);
+    }
+
+    // Q4_K: the sum of a 32-element sub-block lies in 8 consecutive lanes (4
+    // elements each; a group of 8 lanes is valid or not as a whole).
+    __device__ static __forceinline__ void store_sum(float v, const Slice &S, long e, bool ok, int lane) {
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        if (ok && (lane & 7) == 0) S.sx[e / 32] = v;   // row-major [M][nk/32] == element index / 32
+    }
+
+    // |v| outside [2^-60, 2^60] and not zero (or not finite): the slice needs the power-of-two scale
+    __device__ static __forceinline__ bool out_of_range(float v) {
+        const float a = fabsf(v);
+        return a != 0.f && !(a >= 8.673617e-19f && a <= 1.1529215e18f);
+    }
+
+    // hi / mid / lo bf16 parts of (a, b), each packed as one register (a in the low half)
+    __device__ static __forceinline__ void split_pair(float a, float b, uint32_t &hi, uint32_t &mid, uint32_t &lo) {
+        const uint32_t ha = __float_as_uint(a) & 0xFFFF0000u, hb = __float_as_uint(b) & 0xFFFF0000u;
+        // a - hi and r - mid as packed fp32 FMAs with -1 (exact: the results are representable)
+        const float2 r = __ffma2_rn(make_float2(__uint_as_float(ha), __uint_as_float(hb)), make_float2(-1.f, -1.f),
+                                    make_float2(a, b));
+        const uint32_t ma = __float_as_uint(r.x) & 0xFFFF0000u, mb = __float_as_uint(r.y) & 0xFFFF0000u;
+        const float2 l = __ffma2_rn(make_float2(__uint_as_float(ma), __uint_as_float(mb)), make_float2(-1.f, -1.f), r);
+        hi = prmt(ha, hb, 0x7632u);
+        mid = prmt(ma, mb, 0x7632u);
+        lo = prmt(__float_as_uint(l.x), __float_as_uint(l.y), 0x7632u);
+    }
+
+    __device__ __forceinline__ bool prologue(const GemvArgs &a, const Slice &S, int c_begin, uint64_t *xfull,
+                                             int nact, int warp, int lane, unsigned long long timeout) {
+        const int nthr = nact * 32, tid = warp * 32 + lane;
+        // 4-element units of fp32 x per thread: M * nk / 4 over nact warps with
+        // nact * KW = nk, i.e. 2M with a chunk per warp and M with half a chunk,
+        // M being at most 8 NT / P for this kernel
+        constexpr int VPT = (8 * NT / P) * (KW == CHUNK ? 2 : 1);
+        int *flag = reinterpret_cast<int *>(S.xmax + 15);   // set (to 1) when a rescale is needed
+        inv = 1.f;
         if constexpr (XT == X_F32) {
-            return __ldcg(reinterpret_cast<const float2 *>(static_cast<const float *>(x) + off));
-        } else {
-            const uint32_t u = __ldcg(reinterpret_cast<const unsigned int *>(static_cast<const uint16_t *>(x) + off));
-            if constexpr (XT == X_F16) return make_float2(f16_bits_to_float(u), f16_bits_to_float(u >> 16));
-            else return make_float2(bf16_bits_to_float(u), bf16_bits_to_float(u >> 16));
-        }
-    }
-
-    // Part p of v (already scaled): fp32 hi / mid / lo, each an exact bf16
-    // value; 16-bit activations are their own single part.
-    __device__ static __forceinline__ float part(float v, int p) {
-        if constexpr (P == 1) {
-            return v;
-        } else {
-            const float hi = trunc_bf16(v);
-            const float r = v - hi;   // exact
-            const float mid = trunc_bf16(r);
-            return p == 0 ? hi : (p == 1 ? mid : r - mid);
-        }
-    }
-    // Two values as one packed fp16 (fp16 x: exact conversion) or bf16 (the
-    // top halves of exact bf16 values) register, a in the low half.
-    __device__ static __forceinline__ uint32_t pack(float a, float b) {
-        if constexpr (BF) return prmt(__float_as_uint(a), __float_as_uint(b), 0x7632u);
-        else return pack_f16x2(a, b);
-    }
-
-    // Build the B fragments of this warp's slice of x (chunk starting at
-    // element k0, blocks half*NB ..), each element multiplied by s.  With
-    // Q4_K, writes the sub-block sums S_j of the part-0 columns to sxw
-    // ([16 activation rows][8 floats]).  Returns the lane's largest |x|.
-    __device__ __forceinline__ float build(const void *x, int M, int K, long k0, int half, float s, int lane,
-                                           float *sxw) {
-        const int g = lane >> 2, t = lane & 3;
-        float mx = 0.f;
+            pdl_wait();   // x may be the preceding kernel's output
+            // thread tid takes units tid, tid + nthr, ... in row-major order: (row, unit in row)
+            // advance without divisions
+            const int upr = S.nk / 4, nu = S.M * upr;
+            const int dm = nthr / upr, dk = nthr % upr;
+            int m = tid / upr, k4 = tid % upr;
+            float4 v[VPT];
+            int mk[VPT];   // m << 16 | unit in row
+            bool out = false;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const int c = 8 * nt + g, m = c / P, p = c - m * P;
-            const bool live = m < M;
-            const long row = (long)(live ? m : 0) * K + k0;
-            float ssum[NB];
-            constexpr int BATCH = NB < 4 ? NB : 4;   // blocks whose loads are in flight together
+            for (int j = 0; j < VPT; ++j) {
+                v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+                mk[j] = (m << 16) | k4;
+                if (j * nthr + tid < nu) {
+                    v[j] = __ldcg(reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) + (long)m * a.K +
+                                                                   (long)c_begin * CHUNK + 4 * k4));
+                    out |= out_of_range(v[j].x) | out_of_range(v[j].y) | out_of_range(v[j].z) | out_of_range(v[j].w);
+                }
+                k4 += dk;
+                m += dm;
+                if (k4 >= upr) {
+                    k4 -= upr;
+                    ++m;
+                }
+            }
+            if (out) *flag = 1;
+            // the planes (and Q4_K sums) of the slice scaled by sc
+            auto emit = [&](float sc) {
 #pragma unroll
-            for (int b0 = 0; b0 < NB; b0 += BATCH) {
-                float2 v[BATCH][2][2];
+                for (int j = 0; j < VPT; ++j) {
+                    if (j * nthr >= nu) break;   // uniform across the CTA
+                    const bool ok = j * nthr + tid < nu;
+                    const int mm = mk[j] >> 16, k = 4 * (mk[j] & 0xFFFF);
+                    const float4 w = make_float4(v[j].x * sc, v[j].y * sc, v[j].z * sc, v[j].w * sc);
+                    if constexpr (FMT == F_Q4_K) store_sum((w.x + w.y) + (w.z + w.w), S, (long)mm * S.nk + k, ok, lane);
+                    if (ok) {
+                        uint32_t pr[3][2];
+                        split_pair(w.x, w.y, pr[0][0], pr[1][0], pr[2][0]);
+                        split_pair(w.z, w.w, pr[0][1], pr[1][1], pr[2][1]);
 #pragma unroll
-                for (int bb = 0; bb < BATCH; ++bb)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-#pragma unroll
-                        for (int q = 0; q < 2; ++q)
-                            v[bb][h][q] = ld2(x, row + elem<FMT>(half * NB + b0 + bb, h, t, q), live);
-#pragma unroll
-                for (int bb = 0; bb < BATCH; ++bb) {
-                    const int b = b0 + bb;
-                    ssum[b] = 0.f;
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        float2 e01 = v[bb][h][0], e23 = v[bb][h][1];
-                        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(e01.x), fabsf(e01.y)), fmaxf(fabsf(e23.x), fabsf(e23.y))));
-                        if constexpr (XT != X_F16) {
-                            e01 = __fmul2_rn(e01, make_float2(s, s));
-                            e23 = __fmul2_rn(e23, make_float2(s, s));
+                        for (int q = 0; q < 3; ++q) {
+                            const int r = mm * P + q;
+                            const bool sw = swz(r) != 0;   // words of the pair swapped
+                            *reinterpret_cast<uint2 *>(S.xp + (size_t)r * S.rs + k) =
+                                sw ? make_uint2(pr[q][1], pr[q][0]) : make_uint2(pr[q][0], pr[q][1]);
                         }
-                        if constexpr (FMT == F_Q4_K) ssum[b] += (e01.x + e01.y) + (e23.x + e23.y);
-                        // slots (2t, 2t+1) take bytes 0 and 2, slots (2t+8, 2t+9) bytes 1 and 3
-                        xf[nt][b][h][0] = pack(part(e01.x, p), part(e23.x, p));
-                        xf[nt][b][h][1] = pack(part(e01.y, p), part(e23.y, p));
                     }
                 }
-            }
-            if constexpr (FMT == F_Q4_K) {
+            };
+            emit(1.f);
+            named_bar_sync(1, nthr);
+            if (*flag) {
+                // rare: the largest |x| of the CTA's slice sets a power-of-two scale; split again
+                float mx = 0.f;
 #pragma unroll
-                for (int b = 0; b < NB; ++b) {
-                    float v = ssum[b];
-                    v += __shfl_xor_sync(0xffffffffu, v, 1);
-                    v += __shfl_xor_sync(0xffffffffu, v, 2);
-                    if (t == 0 && p == 0 && live) sxw[m * 8 + b] = v;
+                for (int j = 0; j < VPT; ++j)
+                    mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v[j].x), fabsf(v[j].y)), fmaxf(fabsf(v[j].z), fabsf(v[j].w))));
+                const float sc = pick_scale(cta_max(mx, S, nact, warp, lane), inv);
+                if (sc != 1.f) {
+                    emit(sc);
+                    named_bar_sync(1, nthr);
+                }
+            }
+        } else {
+            if (!mbar_wait(xfull, 0, timeout, DEVERR_GEMV_WAIT)) return false;
+            if constexpr (XT == X_BF16 || FMT == F_Q4_K) {
+                // 4-element units of plane 0 ([m][rs], nk / 4 units per row): the range check
+                // (bf16), a rescale in place when needed (rare), and the Q4_K sums
+                const int upr4 = S.nk / 4, nu4 = S.M * upr4;
+                float sc = 1.f;
+                if constexpr (XT == X_BF16) {
+                    bool out = false;
+                    for (int u = tid; u < nu4; u += nthr) {
+                        const uint2 q = *reinterpret_cast<const uint2 *>(S.xp + (size_t)(u / upr4) * S.rs + 4 * (u % upr4));
+                        out |= out_of_range(bf16_bits_to_float(q.x)) | out_of_range(bf16_bits_to_float(q.x >> 16)) |
+                               out_of_range(bf16_bits_to_float(q.y)) | out_of_range(bf16_bits_to_float(q.y >> 16));
+                    }
+                    if (out) *flag = 1;
+                    named_bar_sync(1, nthr);
+                    if (*flag) {
+                        float mx = 0.f;
+                        for (int u = tid; u < nu4; u += nthr) {
+                            const uint2 q = *reinterpret_cast<const uint2 *>(S.xp + (size_t)(u / upr4) * S.rs + 4 * (u % upr4));
+                            mx = fmaxf(mx, fmaxf(fmaxf(fabsf(bf16_bits_to_float(q.x)), fabsf(bf16_bits_to_float(q.x >> 16))),
+                                                 fmaxf(fabsf(bf16_bits_to_float(q.y)), fabsf(bf16_bits_to_float(q.y >> 16)))));
+                        }
+                        sc = pick_scale(cta_max(mx, S, nact, warp, lane), inv);
+                    }
+                }
+                if (sc != 1.f || FMT == F_Q4_K) {
+                    for (int u0 = 0; u0 < nu4; u0 += nthr) {   // uniform trip count (shuffles inside)
+                        const int u = u0 + tid;
+                        const bool ok = u < nu4;
+                        const int m = ok ? u / upr4 : 0, k = ok ? 4 * (u % upr4) : 0;
+                        uint16_t *p = S.xp + (size_t)m * S.rs + k;
+                        uint2 q = ok ? *reinterpret_cast<const uint2 *>(p) : make_uint2(0u, 0u);
+                        float f[4];
+                        if constexpr (XT == X_F16) {
+                            f[0] = f16_lo(q.x); f[1] = f16_hi(q.x);
+                            f[2] = f16_lo(q.y); f[3] = f16_hi(q.y);
+                        } else {
+                            f[0] = bf16_bits_to_float(q.x) * sc; f[1] = bf16_bits_to_float(q.x >> 16) * sc;
+                            f[2] = bf16_bits_to_float(q.y) * sc; f[3] = bf16_bits_to_float(q.y >> 16) * sc;
+                            if (sc != 1.f && ok)
+                                *reinterpret_cast<uint2 *>(p) =
+                                    make_uint2(prmt(__float_as_uint(f[0]), __float_as_uint(f[1]), 0x7632u),
+                                               prmt(__float_as_uint(f[2]), __float_as_uint(f[3]), 0x7632u));
+                        }
+                        if constexpr (FMT == F_Q4_K) store_sum((f[0] + f[1]) + (f[2] + f[3]), S, (long)m * S.nk + k, ok, lane);
+                    }
+                    named_bar_sync(1, nthr);
                 }
             }
         }
-        return mx;
+        return true;
     }
 
-    __device__ __forceinline__ void load_x(const void *x, int M, int K, long k0, int half, int lane, float *sxw) {
-        float mx = build(x, M, K, k0, half, 1.f, lane, sxw);
-        inv = 1.f;
-        if constexpr (XT != X_F16) {
+    // This warp's B fragments from the planes: the chunk starts at element k0
+    // of the slice, blocks half*NB ..
+    __device__ __forceinline__ void load_frags(const Slice &S, int k0, int half, int lane) {
+        const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            // Far outside [2^-60, 2^60] (and finite): rebuild with the largest
-            // element scaled into [1, 2), so that products and sums stay in
-            // fp32's normal range.  Both scales are exact powers of two.
-            if (mx > 0.f && mx <= 3.0e38f && (mx < 8.673617e-19f || mx > 1.1529215e18f)) {
-                const int e = (int)((__float_as_uint(mx) >> 23) & 0xFF) - 127;
-                const int es = e < -126 ? 126 : (e > 126 ? -126 : -e);
-                const float s = __uint_as_float((uint32_t)(127 + es) << 23);
-                inv = __uint_as_float((uint32_t)(127 - es) << 23);
-                __syncwarp();
-                build(x, M, K, k0, half, s, lane, sxw);
-            }
+        for (int nt = 0; nt < NT; ++nt) {
+            const int c = 8 * nt + g, m = c / P;
+            const bool live = m < S.M;
+            const int r = live ? c : 0;   // plane row m * P + p == column c
+            const uint16_t *row = S.xp + ((size_t)r * S.rs + k0);
+            const int sw = swz(r);
+#pragma unroll
+            for (int b = 0; b < NB; ++b)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t l0 = 0u, l1 = 0u;
+                    if (live) {
+                        l0 = *reinterpret_cast<const uint32_t *>(row + (elem<FMT>(half * NB + b, h, t, 0) ^ sw));
+                        l1 = *reinterpret_cast<const uint32_t *>(row + (elem<FMT>(half * NB + b, h, t, 1) ^ sw));
+                    }
+                    // slots (2t, 2t+1) take bytes 0 and 2, slots (2t+8, 2t+9) bytes 1 and 3
+                    xf[nt][b][h][0] = prmt(l0, l1, 0x5410u);
+                    xf[nt][b][h][1] = prmt(l0, l1, 0x7632u);
+                }
         }
-        __syncwarp();
     }
 
     // One block's chain: d * (A0 . B[step 0] + A1 . B[step 1]) into acc, for
@@ -340,9 +490,10 @@ struct Exact {
     }
 
     // box: this warp's chunk, row 0, in the stage; half: which half of the
-    // chunk (KW = 128); sxw: the warp's x sums (Q4_K).
+    // chunk (KW = 128); sxw: the x sums of this warp's first sub-block, rows
+    // sstride apart (Q4_K).
     __device__ __forceinline__ void compute(uint32_t box, int half, float (&acc)[NT][4], int lane, int M,
-                                            const float *sxw) const {
+                                            const float *sxw, int sstride) const {
         const int g = lane >> 2, t = lane & 3;
         const uint32_t r0 = box + g * CB, r1 = r0 + 8 * CB;   // rows g, g + 8
         if constexpr (FMT == F_Q4_0) {
@@ -357,12 +508,12 @@ struct Exact {
                 {
                     const uint32_t a0[4] = {q40_lo<BF>(e0), q40_lo<BF>(e1), q40_lo<BF>(e0 >> 8), q40_lo<BF>(e1 >> 8)};
                     const uint32_t a1[4] = {q40_hi<BF>(e0), q40_hi<BF>(e1), q40_hi<BF>(e0 >> 8), q40_hi<BF>(e1 >> 8)};
-                    block(a0, a1, 2 * pp, f16_bits_to_float(w0), f16_bits_to_float(w1), acc);
+                    block(a0, a1, 2 * pp, f16_lo(w0), f16_lo(w1), acc);
                 }
                 {
                     const uint32_t a0[4] = {q40_lo<BF>(u0), q40_lo<BF>(u1), q40_lo<BF>(u0 >> 8), q40_lo<BF>(u1 >> 8)};
                     const uint32_t a1[4] = {q40_hi<BF>(u0), q40_hi<BF>(u1), q40_hi<BF>(u0 >> 8), q40_hi<BF>(u1 >> 8)};
-                    block(a0, a1, 2 * pp + 1, f16_bits_to_float(v0 >> 16), f16_bits_to_float(v1 >> 16), acc);
+                    block(a0, a1, 2 * pp + 1, f16_hi(v0), f16_hi(v1), acc);
                 }
             }
         } else if constexpr (FMT == F_Q8_0) {
@@ -385,20 +536,20 @@ struct Exact {
                                             q80_pair<BF>(e[0][1] >> 8)};
                     const uint32_t a1[4] = {q80_pair<BF>(e[1][0]), q80_pair<BF>(e[1][1]), q80_pair<BF>(e[1][0] >> 8),
                                             q80_pair<BF>(e[1][1] >> 8)};
-                    block(a0, a1, 2 * pp, f16_bits_to_float(w0), f16_bits_to_float(w1), acc);
+                    block(a0, a1, 2 * pp, f16_lo(w0), f16_lo(w1), acc);
                 }
                 {
                     const uint32_t a0[4] = {q80_pair<BF>(u[0][0]), q80_pair<BF>(u[0][1]), q80_pair<BF>(u[0][0] >> 8),
                                             q80_pair<BF>(u[0][1] >> 8)};
                     const uint32_t a1[4] = {q80_pair<BF>(u[1][0]), q80_pair<BF>(u[1][1]), q80_pair<BF>(u[1][0] >> 8),
                                             q80_pair<BF>(u[1][1] >> 8)};
-                    block(a0, a1, 2 * pp + 1, f16_bits_to_float(v0 >> 16), f16_bits_to_float(v1 >> 16), acc);
+                    block(a0, a1, 2 * pp + 1, f16_hi(v0), f16_hi(v1), acc);
                 }
             }
         } else {
             // Q4_K: header words d|dmin, scales s[0..3], s[4..7], s[8..11]
             const uint32_t h0 = lds32(r0), h1 = lds32(r1);
-            const float d0 = f16_bits_to_float(h0), d1 = f16_bits_to_float(h1);
+            const float d0 = f16_lo(h0), d1 = f16_lo(h1);
             const float nd0 = d0 * -8388608.f, nd1 = d1 * -8388608.f;   // -2^23 d (exact)
             const uint32_t s10 = lds32(r0 + 4), s11 = lds32(r1 + 4);
             const uint32_t s20 = lds32(r0 + 8), s21 = lds32(r1 + 8);
@@ -444,7 +595,7 @@ struct Exact {
             }
             // mins: y -= dmin * sum_j m_j S_j on the part-0 column of each activation row
             // (sub-blocks 0-3: m = s[j+4] & 63; 4-7: s[j+4] >> 4 | (s[j] >> 6) << 4)
-            const float m0f = f16_bits_to_float(h0 >> 16), m1f = f16_bits_to_float(h1 >> 16);
+            const float m0f = f16_hi(h0), m1f = f16_hi(h1);
             const float nm0 = m0f * -8388608.f, nm1 = m1f * -8388608.f;
             const uint32_t mn0 = half == 0 ? (s20 & 0x3F3F3F3Fu) : (((s30 >> 4) & 0x0F0F0F0Fu) | ((s20 >> 2) & 0x30303030u));
             const uint32_t mn1 = half == 0 ? (s21 & 0x3F3F3F3Fu) : (((s31 >> 4) & 0x0F0F0F0Fu) | ((s21 >> 2) & 0x30303030u));
@@ -463,7 +614,7 @@ struct Exact {
 #pragma unroll
                     for (int b = 0; b < NB; ++b) {
                         const uint32_t mv0 = (NB == 8 && b >= 4) ? mnh0 : mn0, mv1 = (NB == 8 && b >= 4) ? mnh1 : mn1;
-                        const float sj = sxw[m * 8 + b];
+                        const float sj = sxw[m * sstride + b];
                         z0 = fmaf(fmaf(byte_magic(mv0, b & 3), m0f, nm0), sj, z0);   // (dmin * m_j) * S_j
                         z1 = fmaf(fmaf(byte_magic(mv1, b & 3), m1f, nm1), sj, z1);
                     }
@@ -504,8 +655,8 @@ template <int XT>
 struct RawPair {
     using T = uint32_t;
     __device__ static __forceinline__ T zero() { return 0u; }
-    __device__ static __forceinline__ T load(const void *x, long off) {   // coherent: see Exact::ld2
-        return __ldcg(reinterpret_cast<const unsigned int *>(static_cast<const uint16_t *>(x) + off));
+    __device__ static __forceinline__ T load(const void *x, long off) {   // the staged slice of x
+        return *reinterpret_cast<const uint32_t *>(static_cast<const uint16_t *>(x) + off);
     }
     __device__ static __forceinline__ float2 get(T u) {
         if constexpr (XT == X_F16)
@@ -518,8 +669,8 @@ template <>
 struct RawPair<X_F32> {
     using T = float2;
     __device__ static __forceinline__ T zero() { return make_float2(0.f, 0.f); }
-    __device__ static __forceinline__ T load(const void *x, long off) {   // coherent: see Exact::ld2
-        return __ldcg(reinterpret_cast<const float2 *>(static_cast<const float *>(x) + off));
+    __device__ static __forceinline__ T load(const void *x, long off) {   // the staged slice of x
+        return *reinterpret_cast<const float2 *>(static_cast<const float *>(x) + off);
     }
     __device__ static __forceinline__ float2 get(T v) { return v; }
 };
@@ -541,7 +692,20 @@ struct Q40I8 {
         return max(-127, min(127, __float2int_rn(v * s)));
     }
 
-    __device__ __forceinline__ void load_x(const void *x, int M, int K, long k0, int, int lane, float *) {
+    struct Slice {
+        uint8_t *xp;     // the raw slice [M][nk] in shared memory
+        float *sx, *xmax;
+        int M, nk, rs;
+    };
+    __device__ __forceinline__ bool prologue(const GemvArgs &, const Slice &, int, uint64_t *xfull, int, int, int,
+                                             unsigned long long timeout) {
+        return mbar_wait(xfull, 0, timeout, DEVERR_GEMV_WAIT);
+    }
+    __device__ __forceinline__ void load_frags(const Slice &S, int k0, int, int lane) {
+        load_x(S.xp, S.M, S.nk, k0, lane);
+    }
+
+    __device__ __forceinline__ void load_x(const void *x, int M, int K, long k0, int lane) {
         const int g = lane >> 2, t = lane & 3;
         const bool live = g < M;
         const long base = (long)g * K + k0;
@@ -593,7 +757,8 @@ struct Q40I8 {
     }
 
     // box: this warp's [16 rows][144 B] chunk.
-    __device__ __forceinline__ void compute(uint32_t box, int, float (&acc)[1][4], int lane, int, const float *) const {
+    __device__ __forceinline__ void compute(uint32_t box, int, float (&acc)[1][4], int lane, int, const float *,
+                                            int) const {
         const int g = lane >> 2, t = lane & 3;
         const uint32_t r0 = box + g * 144, r1 = r0 + 8 * 144;   // rows g, g+8
         const uint32_t sel = t ? 0x3210u : 0x3254u;            // word t of an even block
@@ -633,18 +798,18 @@ template <int XT>
 struct GemvImpl<F_Q4_0, XT, 1, true> : Q40I8<XT> {};
 
 // ------------------------------------------------------------------ kernel
-// blockDim = GEMV_THREADS: warps 0..7 compute, warp 8 produces (TMA), warp 9
-// reduces.  At most 96 registers per thread, so that two CTAs (two calls)
-// share an SM.  Every wait is bounded; a wait that gives up sets a bit of the
-// device error word and ends its warp's loop.
+// blockDim = GEMV_THREADS: warps 0..15 compute, warp 16 produces (TMA), warp
+// 17 reduces; one CTA per SM (at most 112 registers per thread).  Every wait is
+// bounded; a wait that gives up sets a bit of the device error word and ends
+// its warp's loop.
 template <int FMT, int XT, int NT, bool I8>
-__global__ void __launch_bounds__(GEMV_THREADS, 2)
+__global__ void __launch_bounds__(GEMV_THREADS, 1)
     gemv_kernel(const __grid_constant__ CUtensorMap wmap, const GemvArgs a) {
     constexpr int CB = FmtInfo<FMT>::chunk_bytes;
     constexpr int KW = I8 ? 256 : gemv_kw(NT);
     constexpr int WPC = CHUNK / KW;            // compute warps per chunk
     constexpr int P = gemv_parts(XT, I8);
-    constexpr int RS = 8 * NT;                 // floats per row of a reduction slot
+    constexpr int RS = gemv_rs(NT);            // floats per row of a reduction slot
     extern __shared__ __align__(128) uint8_t smem[];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -657,13 +822,21 @@ __global__ void __launch_bounds__(GEMV_THREADS, 2)
     const int nact = (c_end - c_begin) * WPC;   // compute warps with work (<= GEMV_W)
     const int ws = a.wstages;
 
-    const GemvSmem L = gemv_smem_layout(CB, a.cps, ws, NT, FMT == F_Q4_K, P > 1);
+    constexpr int XE = (XT == X_F32) ? 4 : 2;
+    // the reducer stages x raw with bulk copies, except fp32 x on the fp path (the compute warps split it)
+    constexpr bool STAGE = I8 || XT != X_F32;
+    const GemvSmem L = gemv_smem_layout(CB, a.cps, ws, NT, FMT == F_Q4_K, P, a.M, XE, I8);
     uint8_t *ring = smem;
-    float *red = reinterpret_cast<float *>(smem + L.ring);
-    float *sx = reinterpret_cast<float *>(smem + L.ring + L.red);
-    float *scratch = reinterpret_cast<float *>(smem + L.ring + L.red + L.sx);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.ring + L.red + L.sx + L.scratch);
+    uint8_t *xs = smem + L.ring;
+    float *red = reinterpret_cast<float *>(xs + L.xs);
+    float *sx = reinterpret_cast<float *>(xs + L.xs + L.red);
+    float *scratch = reinterpret_cast<float *>(xs + L.xs + L.red + L.sx);
+    float *xmax = reinterpret_cast<float *>(xs + L.xs + L.red + L.sx + L.scratch);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(xs + L.xs + L.red + L.sx + L.scratch + L.xmax);
     uint64_t *full = bars, *empty = bars + ws, *redfull = bars + 2 * ws, *redempty = bars + 2 * ws + GEMV_RSTAGES;
+    uint64_t *xfull = redempty + GEMV_RSTAGES;
+    const int nk = (c_end - c_begin) * CHUNK;   // elements of K in this CTA's slice
+    const int rs = I8 ? nk : a.cps * CHUNK + GEMV_XPAD;   // row stride of the staged slice (elements)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < ws; ++s) {
@@ -674,7 +847,9 @@ __global__ void __launch_bounds__(GEMV_THREADS, 2)
             mbar_init(&redfull[s], nact > 0 ? nact : 1);
             mbar_init(&redempty[s], 1);
         }
+        mbar_init(xfull, 1);
         fence_mbar_init();
+        reinterpret_cast<int *>(xmax)[15] = 0;   // the activation rescale flag
     }
     __syncthreads();
     // the next kernel on the stream (a programmatic dependent) may become
@@ -714,6 +889,15 @@ __global__ void __launch_bounds__(GEMV_THREADS, 2)
         // the parts of each activation row.
         pdl_wait();
         const int M = a.M, N = a.N;
+        if (STAGE && lane == 0) {
+            // the CTA's slice of x, one bulk copy per activation row, into shared memory
+            mbar_arrive_expect_tx(xfull, (uint32_t)(M * nk * XE));
+            for (int m = 0; m < M; ++m)
+                bulk_load(xs + (size_t)m * rs * XE,
+                          static_cast<const uint8_t *>(a.x) + ((size_t)m * a.K + (size_t)c_begin * CHUNK) * XE,
+                          (uint32_t)(nk * XE), xfull);
+        }
+        __syncwarp();
         const int row = lane & 15;
         int r = 0;
         uint32_t rph = 0;
@@ -778,16 +962,27 @@ __global__ void __launch_bounds__(GEMV_THREADS, 2)
                 rph ^= 1u;
             }
         }
+        // the bulk copies of x land before the CTA may exit
+        if (STAGE) mbar_wait(xfull, 0, a.timeout_ns, DEVERR_GEMV_WAIT);
         return;
     }
 
     // ---------------- compute warps
     if (warp >= nact) return;
     const int ci = warp / WPC, half = warp % WPC;
-    float *sxw = sx + warp * 128;
-    GemvImpl<FMT, XT, NT, I8> impl;
-    pdl_wait();   // x may be the preceding kernel's output
-    impl.load_x(a.x, a.M, a.K, (long)(c_begin + ci) * CHUNK, half, lane, sxw);
+    using Impl = GemvImpl<FMT, XT, NT, I8>;
+    Impl impl;
+    typename Impl::Slice sl;
+    sl.xp = reinterpret_cast<decltype(sl.xp)>(xs);
+    sl.sx = sx;
+    sl.xmax = xmax;
+    sl.M = a.M;
+    sl.nk = nk;
+    sl.rs = rs;
+    if (!impl.prologue(a, sl, c_begin, xfull, nact, warp, lane, a.timeout_ns)) return;
+    impl.load_frags(sl, ci * CHUNK, half, lane);
+    const float *sxw = sx + ci * (CHUNK / 32) + half * (KW / 32);
+    const int sstride = nk / 32;
     const int g = lane >> 2, t = lane & 3;
     int s = 0, r = 0, rit = 0;
     uint32_t ph = 0, rph = 0;
@@ -799,7 +994,7 @@ __global__ void __launch_bounds__(GEMV_THREADS, 2)
 #pragma unroll
             for (int j = 0; j < 4; ++j) acc[nt][j] = 0.f;
         impl.compute(smem_u32(ring) + (uint32_t)((size_t)s * L.stage + (size_t)ci * GEMV_ROWS * CB), half, acc, lane,
-                     a.M, sxw);
+                     a.M, sxw, sstride);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
         if (++s == ws) {

@@ -124,18 +124,18 @@ def test_python_constants_match_the_header():
 
 
 @pytest.mark.parametrize("w,a,M,N,K,warps,splits,stages", [
-    ("q4_0", "f32", 1, 11008, 4096, 8, 2, 5),      # 3 columns (fp32 parts): one tile, a chunk per warp, 5 stages
-    ("q4_0", "f32", 4, 11008, 4096, 8, 4, 6),      # 12 columns: two tiles, half a chunk per warp
-    ("q4_0", "f32", 8, 11008, 4096, 8, 4, 6),      # 24 columns: three tiles
-    ("q4_0", "f16", 16, 4096, 4096, 8, 4, 6),      # 16 rows of 16-bit activations: two tiles
-    ("q8_0", "f32", 1, 4096, 4096, 8, 2, 3),       # Q8_0 chunks are twice as large: 3 stages
-    ("q8_0", "f16", 1, 32000, 4096, 8, 2, 3),
-    ("q4_k", "f16", 1, 4096, 11008, 8, 6, 5),      # K = 43 chunks: 6 splits of at most 8
-    ("q4_0", "f16", 1, 4096, 14336, 8, 7, 5),      # K = 56 chunks: 7 splits
+    ("q4_0", "f32", 1, 11008, 4096, 16, 1, 4),     # 3 columns (fp32 parts): one tile, a chunk per warp, K in one CTA
+    ("q4_0", "f32", 4, 11008, 4096, 16, 1, 2),     # 12 columns: two tiles, still a chunk per warp (2 stages fit)
+    ("q4_0", "f32", 8, 11008, 4096, 16, 2, 4),     # 24 columns: three tiles, half a chunk per warp
+    ("q4_0", "f16", 16, 4096, 4096, 14, 2, 2),     # 16 rows of 16-bit activations: the staged slice limits a CTA to 14 chunks
+    ("q8_0", "f32", 1, 4096, 4096, 16, 1, 2),      # Q8_0 chunks are twice as large: 2 stages
+    ("q8_0", "f16", 1, 32000, 4096, 16, 1, 2),
+    ("q4_k", "f16", 1, 4096, 11008, 11, 4, 4),     # K = 43 chunks: 4 splits of 11 balance the CTAs better than 3
+    ("q4_0", "f16", 1, 4096, 14336, 14, 4, 4),     # K = 56 chunks: 4 splits of 14
 ])
 def test_config_table_rules(w, a, M, N, K, warps, splits, stages):
-    """The GEMV rows of the per-shape table (148 SMs when no GPU is present): 8 compute warps, as
-    few splits as their chunks allow, and the deepest ring with which two CTAs still share an SM."""
+    """The GEMV rows of the per-shape table (148 SMs when no GPU is present): up to 16 compute warps,
+    the split count from the per-CTA work model, and a 4-stage ring where shared memory allows."""
     if lwq.lwq_select_config(lwq.fmt_code("q4_0", "f32"), 1, 11008, 4096).ctas != 148:
         pytest.skip("a device with another SM count is present")
     cfg = lwq.lwq_select_config(lwq.fmt_code(w, a), M, N, K)
