@@ -2,7 +2,7 @@
 //
 // Design (sm_100a):
 //  * A persistent grid of one CTA per SM per call (16 compute warps, a TMA
-//    producer and a reducer).  Every CTA triggers its programmatic dependents
+//    producer and two reducers).  Every CTA triggers its programmatic dependents
 //    at once, so the next call on the stream (a programmatic dependent
 //    launch) is scheduled as early as possible and takes each SM as soon as
 //    this call's CTA there exits.
@@ -31,7 +31,7 @@
 //  * Q4_K: per 32-weight sub-block j, y += (d * sc_j) * (sum q x) in fp32
 //    (d * sc_j is exact in fp32), and once per tile y -= dmin * sum_j m_j S_j
 //    with S_j the sub-block sums of x, which the warp keeps in shared memory.
-//  * A reducer warp sums the compute warps' partial tiles in a fixed order
+//  * Two reducer warps (8 rows each) sum the compute warps' partial tiles in a fixed order
 //    and the parts of each activation row, and writes y, or, with split-K,
 //    fp32 partials to the workspace, which a small follow-up kernel (a
 //    programmatic dependent launch) adds in split order.  Results are
@@ -54,7 +54,8 @@ enum { X_F32 = 0, X_F16 = 1, X_BF16 = 2 };
 constexpr int GEMV_ROWS = 16;                     // weight rows per tile (the MMA's M)
 constexpr int CHUNK = 256;                        // weights per TMA chunk of a row
 constexpr int GEMV_W = 16;                        // compute warps per CTA
-constexpr int GEMV_THREADS = (GEMV_W + 2) * 32;   // + producer + reducer
+constexpr int GEMV_RED = 2;                       // reducer warps (rows 8j .. 8j + 7 each)
+constexpr int GEMV_THREADS = (GEMV_W + 1 + GEMV_RED) * 32;   // + producer + reducers
 constexpr int GEMV_RSTAGES = 2;                   // depth of the reduction-slot ring
 
 template <int FMT>
@@ -798,8 +799,9 @@ template <int XT>
 struct GemvImpl<F_Q4_0, XT, 1, true> : Q40I8<XT> {};
 
 // ------------------------------------------------------------------ kernel
-// blockDim = GEMV_THREADS: warps 0..15 compute, warp 16 produces (TMA), warp
-// 17 reduces; one CTA per SM (at most 112 registers per thread).  Every wait is
+// blockDim = GEMV_THREADS: warps 0..15 compute, warp 16 produces (TMA), warps
+// 17 and 18 reduce; one CTA per SM (at most 96 registers per thread: 19 warps
+// over four 16K-register sub-partitions).  Every wait is
 // bounded; a wait that gives up sets a bit of the device error word and ends
 // its warp's loop.
 template <int FMT, int XT, int NT, bool I8>
@@ -845,7 +847,7 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1)
         }
         for (int s = 0; s < GEMV_RSTAGES; ++s) {
             mbar_init(&redfull[s], nact > 0 ? nact : 1);
-            mbar_init(&redempty[s], 1);
+            mbar_init(&redempty[s], GEMV_RED);
         }
         mbar_init(xfull, 1);
         fence_mbar_init();
@@ -882,14 +884,16 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1)
         return;
     }
 
-    if (warp == GEMV_W + 1) {
-        // ---------------- reducer: touches y and the workspace only after the
-        // preceding work has completed.  Lane (row, column group cg) sums the
-        // compute warps' 4-column groups in warp order (deterministic), then
-        // the parts of each activation row.
+    if (warp > GEMV_W) {
+        // ---------------- reducers: touch y and the workspace only after the
+        // preceding work has completed.  Reducer j takes rows 8j .. 8j + 7 of
+        // each tile; lane (row, column group) sums the compute warps' 4-column
+        // groups in warp order (deterministic), then the parts of each
+        // activation row.
+        const int j = warp - GEMV_W - 1;
         pdl_wait();
         const int M = a.M, N = a.N;
-        if (STAGE && lane == 0) {
+        if (j == 0 && STAGE && lane == 0) {
             // the CTA's slice of x, one bulk copy per activation row, into shared memory
             mbar_arrive_expect_tx(xfull, (uint32_t)(M * nk * XE));
             for (int m = 0; m < M; ++m)
@@ -898,58 +902,50 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1)
                           (uint32_t)(nk * XE), xfull);
         }
         __syncwarp();
-        const int row = lane & 15;
+        const int row = 8 * j + (lane & 7), cgl = lane >> 3;
+        float *dst = (S == 1) ? a.y : a.partial + (size_t)split * M * N;
         int r = 0;
         uint32_t rph = 0;
         for (int tile = rgrp; tile < a.row_tiles; tile += G) {
             if (!mbar_wait(&redfull[r], rph, a.timeout_ns, DEVERR_GEMV_WAIT)) break;
             const uint32_t rs0 = smem_u32(red) + (uint32_t)(r * GEMV_W * GEMV_ROWS * RS * 4);
             const int n = tile * GEMV_ROWS + row;
-            float *dst = (S == 1) ? a.y : a.partial + (size_t)split * M * N;
 #pragma unroll
-            for (int k = 0; k < NT; ++k) {
-                const int cg = (lane >> 4) + 2 * k;
-                const uint32_t addr = rs0 + (uint32_t)((row * RS + 4 * cg) * 4);
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                int w = 0;
-#pragma unroll 1
-                for (; w + 4 <= nact; w += 4) {
-                    uint4 u[4];
+            for (int k = 0; k < (2 * NT + 3) / 4; ++k) {
+                const int cg = cgl + 4 * k;
+                if (cg < 2 * NT) {
+                    const uint32_t addr = rs0 + (uint32_t)((row * RS + 4 * cg) * 4);
+                    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                    // all of the warps' loads in flight at once, summed in warp order
+                    uint4 u[GEMV_W];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) u[i] = lds128(addr + (uint32_t)((w + i) * GEMV_ROWS * RS * 4));
+                    for (int w = 0; w < GEMV_W; ++w)
+                        u[w] = w < nact ? lds128(addr + (uint32_t)(w * GEMV_ROWS * RS * 4)) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        v.x += __uint_as_float(u[i].x);
-                        v.y += __uint_as_float(u[i].y);
-                        v.z += __uint_as_float(u[i].z);
-                        v.w += __uint_as_float(u[i].w);
+                    for (int w = 0; w < GEMV_W; ++w) {
+                        v.x += __uint_as_float(u[w].x);
+                        v.y += __uint_as_float(u[w].y);
+                        v.z += __uint_as_float(u[w].z);
+                        v.w += __uint_as_float(u[w].w);
                     }
-                }
-#pragma unroll 1
-                for (; w < nact; ++w) {
-                    const uint4 u = lds128(addr + (uint32_t)(w * GEMV_ROWS * RS * 4));
-                    v.x += __uint_as_float(u.x);
-                    v.y += __uint_as_float(u.y);
-                    v.z += __uint_as_float(u.z);
-                    v.w += __uint_as_float(u.w);
-                }
-                if constexpr (P == 1) {
-                    // column = activation row
-                    const float o[4] = {v.x, v.y, v.z, v.w};
-                    if (n < N) {
+                    if constexpr (P == 1) {
+                        // column = activation row
+                        const float o[4] = {v.x, v.y, v.z, v.w};
+                        if (n < N) {
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            if (4 * cg + i < M) dst[(size_t)(4 * cg + i) * N + n] = o[i];
+                            for (int i = 0; i < 4; ++i)
+                                if (4 * cg + i < M) dst[(size_t)(4 * cg + i) * N + n] = o[i];
+                        }
+                    } else {
+                        st_shared_v4(smem_u32(scratch) + (uint32_t)((row * RS + 4 * cg) * 4), __float_as_uint(v.x),
+                                     __float_as_uint(v.y), __float_as_uint(v.z), __float_as_uint(v.w));
                     }
-                } else {
-                    st_shared_v4(smem_u32(scratch) + (uint32_t)((row * RS + 4 * cg) * 4), __float_as_uint(v.x),
-                                 __float_as_uint(v.y), __float_as_uint(v.z), __float_as_uint(v.w));
                 }
             }
             if constexpr (P > 1) {
                 __syncwarp();
-                for (int o = lane; o < GEMV_ROWS * M; o += 32) {
-                    const int rr = o & 15, m = o >> 4, nn = tile * GEMV_ROWS + rr;
+                for (int o = lane; o < 8 * M; o += 32) {
+                    const int rr = 8 * j + (o & 7), m = o >> 3, nn = tile * GEMV_ROWS + rr;
                     const float *sp = scratch + rr * RS + m * P;
                     const float val = (sp[0] + sp[1]) + sp[2];
                     if (nn < N) dst[(size_t)m * N + nn] = val;
@@ -963,7 +959,7 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1)
             }
         }
         // the bulk copies of x land before the CTA may exit
-        if (STAGE) mbar_wait(xfull, 0, a.timeout_ns, DEVERR_GEMV_WAIT);
+        if (j == 0 && STAGE) mbar_wait(xfull, 0, a.timeout_ns, DEVERR_GEMV_WAIT);
         return;
     }
 
