@@ -338,22 +338,28 @@ struct Exact {
             int m = tid / upr, k4 = tid % upr;
             float4 v[VPT];
             int mk[VPT];   // m << 16 | unit in row
-            bool out = false;
+            // every load is issued before any value is used, so they are all in flight
+            // at once; a unit past the end reloads the thread's first unit (always one of
+            // the slice: M * nk / 4 >= nthr) and is zeroed below
+            const float *xb = static_cast<const float *>(a.x) + (long)c_begin * CHUNK;
+            const long first = (long)m * a.K + 4 * k4;
 #pragma unroll
             for (int j = 0; j < VPT; ++j) {
-                v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
                 mk[j] = (m << 16) | k4;
-                if (j * nthr + tid < nu) {
-                    v[j] = __ldcg(reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) + (long)m * a.K +
-                                                                   (long)c_begin * CHUNK + 4 * k4));
-                    out |= out_of_range(v[j].x) | out_of_range(v[j].y) | out_of_range(v[j].z) | out_of_range(v[j].w);
-                }
+                const bool ok = j * nthr + tid < nu;
+                v[j] = __ldcg(reinterpret_cast<const float4 *>(xb + (ok ? (long)m * a.K + 4 * k4 : first)));
                 k4 += dk;
                 m += dm;
                 if (k4 >= upr) {
                     k4 -= upr;
                     ++m;
                 }
+            }
+            bool out = false;
+#pragma unroll
+            for (int j = 0; j < VPT; ++j) {
+                if (j * nthr + tid >= nu) v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+                out |= out_of_range(v[j].x) | out_of_range(v[j].y) | out_of_range(v[j].z) | out_of_range(v[j].w);
             }
             if (out) *flag = 1;
             // the planes (and Q4_K sums) of the slice scaled by sc
@@ -462,11 +468,12 @@ struct Exact {
             for (int b = 0; b < NB; ++b)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    uint32_t l0 = 0u, l1 = 0u;
-                    if (live) {
-                        l0 = *reinterpret_cast<const uint32_t *>(row + (elem<FMT>(half * NB + b, h, t, 0) ^ sw));
-                        l1 = *reinterpret_cast<const uint32_t *>(row + (elem<FMT>(half * NB + b, h, t, 1) ^ sw));
-                    }
+                    // unconditional loads (a dead column reads plane row 0), zeroed after:
+                    // no load waits behind a branch on the previous one
+                    uint32_t l0 = *reinterpret_cast<const uint32_t *>(row + (elem<FMT>(half * NB + b, h, t, 0) ^ sw));
+                    uint32_t l1 = *reinterpret_cast<const uint32_t *>(row + (elem<FMT>(half * NB + b, h, t, 1) ^ sw));
+                    l0 = live ? l0 : 0u;
+                    l1 = live ? l1 : 0u;
                     // slots (2t, 2t+1) take bytes 0 and 2, slots (2t+8, 2t+9) bytes 1 and 3
                     xf[nt][b][h][0] = prmt(l0, l1, 0x5410u);
                     xf[nt][b][h][1] = prmt(l0, l1, 0x7632u);
@@ -709,7 +716,7 @@ struct Q40I8 {
     __device__ __forceinline__ void load_x(const void *x, int M, int K, long k0, int lane) {
         const int g = lane >> 2, t = lane & 3;
         const bool live = g < M;
-        const long base = (long)g * K + k0;
+        const long base = (live ? (long)g * K : 0L) + k0;   // a dead column reads row 0, zeroed below
         using Raw = typename RawPair<XT>::T;
         inv = 1.f;
 #pragma unroll
@@ -719,15 +726,17 @@ struct Q40I8 {
 #pragma unroll
             for (int bb = 0; bb < 4; ++bb) {
                 const int b = b0 + bb;
+                const long e = base + 32 * b;
+                r[bb][0] = RawPair<XT>::load(x, e + cb0(b & 1, t));
+                r[bb][1] = RawPair<XT>::load(x, e + cb2(b & 1, t));
+                r[bb][2] = RawPair<XT>::load(x, e + 16 + cb0(b & 1, t));
+                r[bb][3] = RawPair<XT>::load(x, e + 16 + cb2(b & 1, t));
+            }
+            if (!live) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) r[bb][i] = RawPair<XT>::zero();
-                if (live) {
-                    const long e = base + 32 * b;
-                    r[bb][0] = RawPair<XT>::load(x, e + cb0(b & 1, t));
-                    r[bb][1] = RawPair<XT>::load(x, e + cb2(b & 1, t));
-                    r[bb][2] = RawPair<XT>::load(x, e + 16 + cb0(b & 1, t));
-                    r[bb][3] = RawPair<XT>::load(x, e + 16 + cb2(b & 1, t));
-                }
+                for (int bb = 0; bb < 4; ++bb)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) r[bb][i] = RawPair<XT>::zero();
             }
 #pragma unroll
             for (int bb = 0; bb < 4; ++bb) {
@@ -868,6 +877,10 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1)
             uint32_t ph = 0;
             for (int tile = rgrp; tile < a.row_tiles; tile += G, ++it) {
                 if (it >= ws && !mbar_wait(&empty[s], ph ^ 1u, a.timeout_ns, DEVERR_GEMV_WAIT)) break;
+                // first pass through the ring: one stage in flight at a time, so that the
+                // first stage (and the prologue's activation loads) are not queued behind
+                // every SM's whole ring of weight requests
+                if (it > 0 && it < ws && !mbar_wait(&full[it - 1], 0u, a.timeout_ns, DEVERR_GEMV_WAIT)) break;
                 // one 3-D box per stage: [chunks of this split][16 rows][chunk bytes]; the
                 // last split's box may run past the last chunk, where it reads zeros
                 mbar_arrive_expect_tx(&full[s], (uint32_t)L.stage);
