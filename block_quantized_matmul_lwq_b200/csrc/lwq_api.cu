@@ -403,20 +403,24 @@ int encode_weight_map(CUtensorMap *map, const void *Wq, int wf, int N, long rb, 
 }
 
 // ------------------------------------------------------------- prefill GEMM
-template <int FMT, int XT>
+template <int FMT, int XT, int H>
 cudaError_t launch_gemm_tc(const CUtensorMap &wm, const CUtensorMap &xm, const GemmArgs &a, int ctas, size_t smem,
                            cudaStream_t st) {
-    auto kern = gemm_tc_kernel<FMT, XT>;
+    auto kern = gemm_tc_kernel<FMT, XT, H>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), smem);
     if (e != cudaSuccess) return e;
     return launch_k(kern, ctas, GEMM_THREADS, smem, st, a.overlap != 0, wm, xm, a);
 }
 
+// h = 128-row halves of a weight tile
 template <int FMT>
-cudaError_t launch_gemm_xt(int xt, const CUtensorMap &wm, const CUtensorMap &xm, const GemmArgs &a, int ctas,
+cudaError_t launch_gemm_xt(int xt, int h, const CUtensorMap &wm, const CUtensorMap &xm, const GemmArgs &a, int ctas,
                            size_t smem, cudaStream_t st) {
-    if (xt == X_F16) return launch_gemm_tc<FMT, X_F16>(wm, xm, a, ctas, smem, st);
-    return launch_gemm_tc<FMT, X_BF16>(wm, xm, a, ctas, smem, st);
+    if (xt == X_F16)
+        return h == 2 ? launch_gemm_tc<FMT, X_F16, 2>(wm, xm, a, ctas, smem, st)
+                      : launch_gemm_tc<FMT, X_F16, 1>(wm, xm, a, ctas, smem, st);
+    return h == 2 ? launch_gemm_tc<FMT, X_BF16, 2>(wm, xm, a, ctas, smem, st)
+                  : launch_gemm_tc<FMT, X_BF16, 1>(wm, xm, a, ctas, smem, st);
 }
 
 // Returns the kernels launched (1, or 2 with the split-K sum) through *launches.
@@ -453,15 +457,17 @@ int gemm_launch(int wf, int xt, const void *Wq, const void *x, float *y, int M, 
     a.N = N;
     a.K = K;
     a.nchunks = K / 256;
-    a.n_wtiles = (N + GEMM_WROWS - 1) / GEMM_WROWS;
+    const int h = cfg.tile_n / GEMM_WROWS;   // 128-row halves of a weight tile
+    if (h != 1 && h != 2) return LWQ_ERR_UNSUPPORTED;
+    a.n_wtiles = (N + cfg.tile_n - 1) / cfg.tile_n;
     a.n_ttiles = (M + bn - 1) / bn;
     a.bn = bn;
-    a.a_stages = GEMM_A_STAGES;
     {
         // the same ring depths gemm_plan chose (its B ring is the configuration's stage count)
         lwq_config f = cfg;
-        int nb = 0, np = 0;
-        gemm_rings(gemm_chunk_bytes(wf), bn, &f, &nb, &np);
+        int na = 0, nb = 0, np = 0;
+        if (!gemm_rings(gemm_chunk_bytes(wf), bn, h, &f, &na, &nb, &np)) return LWQ_ERR_UNSUPPORTED;
+        a.a_stages = na;
         a.b_stages = nb;
         a.p_stages = np;
     }
@@ -469,9 +475,9 @@ int gemm_launch(int wf, int xt, const void *Wq, const void *x, float *y, int M, 
     a.overlap = overlap;
     cudaError_t e;
     switch (wf) {
-    case LWQ_Q4_0: e = launch_gemm_xt<F_Q4_0>(xt, wm, xm, a, cfg.ctas, smem, st); break;
-    case LWQ_Q8_0: e = launch_gemm_xt<F_Q8_0>(xt, wm, xm, a, cfg.ctas, smem, st); break;
-    default: e = launch_gemm_xt<F_Q4_K>(xt, wm, xm, a, cfg.ctas, smem, st); break;
+    case LWQ_Q4_0: e = launch_gemm_xt<F_Q4_0>(xt, h, wm, xm, a, cfg.ctas, smem, st); break;
+    case LWQ_Q8_0: e = launch_gemm_xt<F_Q8_0>(xt, h, wm, xm, a, cfg.ctas, smem, st); break;
+    default: e = launch_gemm_xt<F_Q4_K>(xt, h, wm, xm, a, cfg.ctas, smem, st); break;
     }
     if (e != cudaSuccess) return LWQ_ERR_CUDA;
     *launches = 1;

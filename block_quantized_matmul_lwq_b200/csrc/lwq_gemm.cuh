@@ -8,16 +8,20 @@
 // per MMA, so the decode work per flop shrinks with the token tile.
 //
 // Roles (one persistent CTA per SM, warp-specialized):
-//   warp 0      TMA producer: packed weight chunks [128 rows][256 weights]
+//   warp 0      TMA producer: packed weight chunks [128 or 256 rows][256 weights]
 //               and activation tiles [BN tokens][64 k] (128-byte swizzle)
 //   warp 1      TMEM allocator and single-thread UMMA issuer
 //   warps 2..17 dequantizers: packed chunk -> bf16/fp16 weight tile
-//               [128 rows][64 k] in the UMMA K-major 128-byte-swizzle layout
+//               [128 rows][64 k] per half in the UMMA K-major 128-byte-swizzle layout
 //   warps 18-21 epilogue: TMEM -> registers -> y (fp32), coalesced along N
-// UMMA shape: M = 128 weight rows, N = BN tokens (a multiple of 16 from 32
-// to 256, chosen per shape to balance the persistent grid's waves), K = 16;
-// accumulators double-buffered in TMEM so the epilogue of one tile overlaps
-// the main loop of the next.  Every wait is bounded (device error word).
+// Weight tile: 128 rows (one UMMA per K step) or 256 rows (two, one per
+// 128-row half, sharing the activation tile: half the L2 traffic of
+// activations per flop, which bounds the 128-row tiles).  UMMA shape: M = 128
+// weight rows, N = BN tokens (a multiple of 16 from 32 to 256), K = 16.  The
+// tile pair is chosen per shape from a model of the persistent grid's rounds
+// and a tile's shared-memory, tensor and L2 time.  Accumulators are
+// double-buffered in TMEM where two fit (the epilogue of one tile overlaps
+// the main loop of the next).  Every wait is bounded (device error word).
 #pragma once
 
 #include "../../include/lwq.h"
@@ -68,13 +72,19 @@ __host__ __device__ constexpr size_t gemm_a_bytes() { return (size_t)GEMM_WROWS 
 __host__ __device__ constexpr size_t gemm_b_bytes(int bn) { return (size_t)bn * 128; }
 // one B stage, rounded up to the 1024-byte alignment of 128-byte-swizzle atoms (A stages are 16 KB)
 __host__ __device__ constexpr size_t gemm_bstage_bytes(int bn) { return (gemm_b_bytes(bn) + 1023) & ~(size_t)1023; }
-// TMEM columns for two fp32 accumulators of bn columns (a power of two >= 32)
-__host__ __device__ constexpr uint32_t gemm_tmem_cols(int bn) { return 2 * bn <= 128 ? 128u : (2 * bn <= 256 ? 256u : 512u); }
+// Accumulator buffers: two (the epilogue of one tile overlaps the main loop of
+// the next) when both fit the 512 TMEM columns, else one.
+__host__ __device__ constexpr int gemm_nbuf(int h, int bn) { return 2 * h * bn <= 512 ? 2 : 1; }
+// TMEM columns allocated: a power of two >= 32 holding nbuf x h accumulators of bn fp32 columns
+__host__ __device__ constexpr uint32_t gemm_tmem_cols(int h, int bn) {
+    const int need = gemm_nbuf(h, bn) * h * bn;
+    return need <= 32 ? 32u : (need <= 64 ? 64u : (need <= 128 ? 128u : (need <= 256 ? 256u : 512u)));
+}
 
-// Shared memory: [a stages x A 16 KB] [b stages x B bn*128 B] [p stages x 128*CB] [barriers] [tmem addr]
-__host__ __device__ inline size_t gemm_smem_bytes(int cb, int bn, int a_stages, int b_stages, int p_stages) {
-    size_t s = (size_t)a_stages * gemm_a_bytes() + (size_t)b_stages * gemm_bstage_bytes(bn);
-    s += (size_t)p_stages * GEMM_WROWS * cb;
+// Shared memory: [a stages x h x A 16 KB] [b stages x B bn*128 B] [p stages x h*128*CB] [barriers] [tmem addr]
+__host__ __device__ inline size_t gemm_smem_bytes(int cb, int bn, int h, int a_stages, int b_stages, int p_stages) {
+    size_t s = (size_t)a_stages * h * gemm_a_bytes() + (size_t)b_stages * gemm_bstage_bytes(bn);
+    s += (size_t)p_stages * h * GEMM_WROWS * cb;
     s = (s + 7) & ~(size_t)7;
     s += (size_t)(2 * a_stages + 2 * b_stages + 2 * p_stages + 4 + 1) * 8 + 16;
     return s + 1024;  // slack to align the base to 1024 B
@@ -247,17 +257,29 @@ struct Dequant<F_Q4_K, XT> {
 };
 
 // -------------------------------------------------------------------- kernel
-template <int FMT, int XT>
+// H = 128-row halves of a weight tile (1 or 2).  With H = 2 the tile is 256
+// weight rows: two UMMAs per K step (one per half, into two accumulators)
+// share each activation tile, so activations stream from L2 once per 256
+// weight rows instead of once per 128.
+template <int FMT, int XT, int H>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap,
                    const GemmArgs a) {
     constexpr int CB = GemmFmt<FMT>::chunk_bytes;
-    constexpr uint32_t A_BYTES = (uint32_t)gemm_a_bytes();
+    constexpr uint32_t AH_BYTES = (uint32_t)gemm_a_bytes();       // one half's k-block tile
+    constexpr uint32_t A_BYTES = H * AH_BYTES;
+    constexpr uint32_t PH_BYTES = (uint32_t)GEMM_WROWS * CB;      // one half's packed chunk
+    constexpr uint32_t P_BYTES = H * PH_BYTES;
+    constexpr int WR = H * GEMM_WROWS;                            // weight rows per tile
+    // dequantized k-blocks per batch (one proxy fence and warp barrier per batch):
+    // two when the A ring has 4 stages, one with the 2-stage ring of 256-row tiles
+    constexpr int BATCH = H == 1 ? 2 : 1;
     const int BN = a.bn;
     const uint32_t B_BYTES = (uint32_t)gemm_b_bytes(BN);
     const uint32_t BS_BYTES = (uint32_t)gemm_bstage_bytes(BN);
-    constexpr uint32_t P_BYTES = (uint32_t)GEMM_WROWS * CB;
-    const uint32_t TMEM_COLS = gemm_tmem_cols(BN);
+    const int NBUF = gemm_nbuf(H, BN);
+    const uint32_t TMEM_COLS = gemm_tmem_cols(H, BN);
+    const uint32_t BUF_COLS = TMEM_COLS / (uint32_t)NBUF;          // columns per accumulator buffer
     const uint32_t IDESC = umma_idesc_f16(XT == X_F16 ? 0 : 1, GEMM_WROWS, BN);
 
     extern __shared__ uint8_t smem_raw[];
@@ -328,7 +350,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     // Wq only: callers that allow overlap promise it is not written by preceding work
                     if (ci >= P && !(ok = mbar_wait(&p_empty[ps], pph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
                     mbar_arrive_expect_tx(&p_full[ps], P_BYTES);
-                    tma_load_2d(pk + (size_t)ps * P_BYTES, &wmap, &p_full[ps], c * (CB / 2), wt * GEMM_WROWS);
+#pragma unroll
+                    for (int hh = 0; hh < H; ++hh)   // rows past N read zeros
+                        tma_load_2d(pk + (size_t)ps * P_BYTES + hh * PH_BYTES, &wmap, &p_full[ps], c * (CB / 2),
+                                    wt * WR + hh * GEMM_WROWS);
                     if (++ps == P) {
                         ps = 0;
                         pph ^= 1u;
@@ -371,11 +396,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++ti) {
                 const int ks = item % a.splits;
                 const int kbn = (min(a.nchunks, (ks + 1) * a.cps) - ks * a.cps) * GEMM_KB_PER_CHUNK;
-                const int as = ti & 1;
-                if (ti >= 2 && !(ok = mbar_wait(&acc_empty[as], ((ti >> 1) - 1) & 1, a.timeout_ns, DEVERR_GEMM_WAIT)))
+                const int as = ti % NBUF, use = ti / NBUF;   // buffer, and how often it was used before
+                if (use >= 1 && !(ok = mbar_wait(&acc_empty[as], (uint32_t)((use - 1) & 1), a.timeout_ns, DEVERR_GEMM_WAIT)))
                     break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)as * (TMEM_COLS / 2);
+                const uint32_t d_tmem = tmem_base + (uint32_t)as * BUF_COLS;
                 for (int k = 0; k < kbn; ++k) {
                     if (!(ok = mbar_wait(&b_full[sb], phb, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
                     if (!(ok = mbar_wait(&a_full[sa], pha, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
@@ -384,8 +409,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     const uint32_t b_addr = smem_u32(Bs + (size_t)sb * BS_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < GEMM_BK / 16; ++kk)
-                        umma_f16(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32), IDESC,
-                                 (k | kk) ? 1u : 0u);
+#pragma unroll
+                        for (int hh = 0; hh < H; ++hh)   // half hh accumulates at columns hh * BN of the buffer
+                            umma_f16(d_tmem + (uint32_t)(hh * BN), umma_desc_sw128(a_addr + hh * AH_BYTES + kk * 32),
+                                     umma_desc_sw128(b_addr + kk * 32), IDESC, (k | kk) ? 1u : 0u);
                     umma_commit(&a_empty[sa]);
                     umma_commit(&b_empty[sb]);
                     if (++sa == SA) {
@@ -406,12 +433,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
     } else if (warp < 2 + GEMM_DQ_WARPS) {
         // ------------------------------------------------------ dequantizers
-        // Warp i of the 16 takes weight rows 8i..8i+7 of the tile, all four (h, v) slices of each:
+        // Warp i of the 16 takes weight rows 8i..8i+7 of each half, all four (h, v) slices of each:
         // its packed-chunk loads then spread over the shared-memory banks (rows lie 144 bytes apart,
         // which a warp of 32 rows would fold onto 8 banks), and each quarter-warp's 16-byte stores
         // (8 rows, one chunk column) fall on distinct swizzled positions.
         const int t = threadIdx.x - 64;          // 0..511
-        const int r = 8 * (t >> 5) + (t & 7);    // weight row within the tile
+        const int r = 8 * (t >> 5) + (t & 7);    // weight row within the half
         const int h = (t >> 3) & 1;              // which 32 of the k-block's 64 weights
         const int v = (t >> 4) & 1;              // which 16 of those 32
         int kbi = 0, s = 0, ps = 0;
@@ -423,22 +450,27 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             for (int c = c0; ok && c < c1; ++c) {
                 if (!(ok = mbar_wait(&p_full[ps], pph, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
                 const uint32_t prow = smem_u32(pk) + (uint32_t)(ps * P_BYTES + r * CB);
-                // two k-blocks per batch: one proxy fence and one warp barrier for both
-                // (the ring has an even number of stages, so a batch never wraps)
-                for (int kb = 0; kb < GEMM_KB_PER_CHUNK; kb += 2, kbi += 2) {
+                // BATCH k-blocks per batch; the A ring's depth is a multiple of BATCH, so a batch never wraps
+                for (int kb = 0; kb < GEMM_KB_PER_CHUNK; kb += BATCH, kbi += BATCH) {
                     if (kbi >= SA) {
-                        if (!(ok = mbar_wait(&a_empty[s], ph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
-                        if (!(ok = mbar_wait(&a_empty[s + 1], ph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
+#pragma unroll
+                        for (int j = 0; j < BATCH; ++j)
+                            if (ok && !(ok = mbar_wait(&a_empty[s + j], ph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
+                        if (!ok) break;
                     }
-                    Dequant<FMT, XT>::run(prow, kb, h, v, smem_u32(As + (size_t)s * A_BYTES), r);
-                    Dequant<FMT, XT>::run(prow, kb + 1, h, v, smem_u32(As + (size_t)(s + 1) * A_BYTES), r);
+#pragma unroll
+                    for (int j = 0; j < BATCH; ++j)
+#pragma unroll
+                        for (int hh = 0; hh < H; ++hh)
+                            Dequant<FMT, XT>::run(prow + hh * PH_BYTES, kb + j, h, v,
+                                                  smem_u32(As + (size_t)(s + j) * A_BYTES + hh * AH_BYTES), r);
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        mbar_arrive(&a_full[s]);
-                        mbar_arrive(&a_full[s + 1]);
+#pragma unroll
+                        for (int j = 0; j < BATCH; ++j) mbar_arrive(&a_full[s + j]);
                     }
-                    if ((s += 2) == SA) {
+                    if ((s += BATCH) == SA) {
                         s = 0;
                         ph ^= 1u;
                     }
@@ -461,28 +493,31 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             const int tile = item / a.splits, ks = item % a.splits;
             const int tt = tile % a.n_ttiles, wt = tile / a.n_ttiles;
             float *out = a.splits > 1 ? a.partial + (size_t)ks * M * N : a.y;
-            const int as = ti & 1;
-            if (!mbar_wait(&acc_full[as], (ti >> 1) & 1, a.timeout_ns, DEVERR_GEMM_WAIT)) break;
+            const int as = ti % NBUF, use = ti / NBUF;
+            if (!mbar_wait(&acc_full[as], (uint32_t)(use & 1), a.timeout_ns, DEVERR_GEMM_WAIT)) break;
             tc_fence_after();
-            const int n = wt * GEMM_WROWS + q * 32 + lane;
-            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)as * (TMEM_COLS / 2);
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 32) {
-                uint32_t v[32];
-                if (BN - c0 >= 32) {
-                    tmem_ld_32x32b_x32(taddr + c0, v);
-                } else {
-                    tmem_ld_32x32b_x16(taddr + c0, *reinterpret_cast<uint32_t(*)[16]>(v));
+            for (int hh = 0; hh < H; ++hh) {
+                const int n = wt * WR + hh * GEMM_WROWS + q * 32 + lane;
+                const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)as * BUF_COLS + (uint32_t)(hh * BN);
+#pragma unroll 1
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    uint32_t v[32];
+                    if (BN - c0 >= 32) {
+                        tmem_ld_32x32b_x32(taddr + c0, v);
+                    } else {
+                        tmem_ld_32x32b_x16(taddr + c0, *reinterpret_cast<uint32_t(*)[16]>(v));
 #pragma unroll
-                    for (int j = 16; j < 32; ++j) v[j] = 0u;
-                }
-                tmem_wait_ld();
-                const int m0 = tt * BN + c0;
-                const int mcols = min(32, BN - c0);
-                if (n < N) {
+                        for (int j = 16; j < 32; ++j) v[j] = 0u;
+                    }
+                    tmem_wait_ld();
+                    const int m0 = tt * BN + c0;
+                    const int mcols = min(32, BN - c0);
+                    if (n < N) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (j < mcols && m0 + j < M) out[(size_t)(m0 + j) * N + n] = __uint_as_float(v[j]);
+                        for (int j = 0; j < 32; ++j)
+                            if (j < mcols && m0 + j < M) out[(size_t)(m0 + j) * N + n] = __uint_as_float(v[j]);
+                    }
                 }
             }
             tc_fence_before();
@@ -507,27 +542,49 @@ inline bool gemm_eligible(int wf, int xt, long K) {
 
 inline int gemm_chunk_bytes(int wf) { return wf == LWQ_Q8_0 ? 272 : 144; }
 
-// Ring depths: 4 dequantized A stages (made on chip, two per batch), 3 packed
-// chunk stages (each feeds four k-blocks; 2 when shared memory is short), and
-// as many activation B stages as fit, up to 8 (B tiles arrive from L2/HBM at
-// ~60 bytes per cycle of a busy tensor pipe, so their ring covers the load
-// latency).  A forced stage count fixes the B ring.
-constexpr int GEMM_A_STAGES = 4;   // even: the dequantizers fill two stages per batch
-// B stages (most up to 8, at least 2) and chunk stages (3, else 2) for a tile width.
-inline void gemm_rings(int cb, int bn, const lwq_config *force, int *nb, int *np) {
-    for (int p = 3; p >= 2; --p) {
+// Ring depths.  128-row tiles: 4 dequantized A stages (made on chip, two per
+// batch), 3 packed chunk stages (each feeds four k-blocks; 2 when shared
+// memory is short), and as many activation B stages as fit, up to 8 (B tiles
+// arrive from L2 at ~60 bytes per cycle of a busy tensor pipe, so their ring
+// covers the load latency).  256-row tiles: 2 A stages (one per batch) and 2
+// chunk stages, the rest for B.  A forced stage count fixes the B ring.
+constexpr int GEMM_A_STAGES = 4;   // 128-row tiles; even: the dequantizers fill two stages per batch
+inline int gemm_a_stages(int h) { return h == 1 ? GEMM_A_STAGES : 2; }
+inline bool gemm_rings(int cb, int bn, int h, const lwq_config *force, int *na, int *nb, int *np) {
+    *na = gemm_a_stages(h);
+    for (int p = h == 1 ? 3 : 2; p >= 2; --p) {
         int b = force && force->stages ? force->stages : 8;
-        while (!(force && force->stages) && b > 2 && gemm_smem_bytes(cb, bn, GEMM_A_STAGES, b, p) > 232448) --b;
+        while (!(force && force->stages) && b > 2 && gemm_smem_bytes(cb, bn, h, *na, b, p) > 232448) --b;
         *nb = b;
         *np = p;
-        if (gemm_smem_bytes(cb, bn, GEMM_A_STAGES, b, p) <= 232448) return;
+        if (gemm_smem_bytes(cb, bn, h, *na, b, p) <= 232448) return true;
     }
+    return false;
+}
+
+// Modelled time (ns) of one k-block (64 of K) of a tile on one SM, the
+// slowest of: shared-memory traffic at 128 B per cycle (the UMMAs' operand
+// reads, the TMA writes of activations and packed weights, the dequantizers'
+// reads and writes), the tensor pipe at this machine's measured bf16 rate per
+// SM, the activation stream from L2 at its measured aggregate share, and the
+// B ring's cover of the L2 latency.
+inline double gemm_kblock_ns(int cb, int bn, int h, int nb) {
+    const double smem = h * (16384.0 + bn * 128.0) + bn * 128.0 + h * 128.0 * cb / 4.0 * 2.0 + h * 16384.0;
+    const double t_smem = smem / 243.0;        // 128 B/clk at 1.9 GHz
+    const double t_mma = h * bn * 1.46;        // 2*128*bn*64 flops at 11.2 TFLOP/s
+    const double t_l2 = bn * 128.0 / 81.0;     // ~12 TB/s over 148 SMs
+    const double t_lat = 1000.0 / nb;          // ~1 us of L2 latency over nb stages
+    double t = t_smem;
+    if (t_mma > t) t = t_mma;
+    if (t_l2 > t) t = t_l2;
+    if (t_lat > t) t = t_lat;
+    return t;
 }
 
 inline int gemm_plan(int wf, int xt, int M, int N, int K, const lwq_config *force, int sms, GemmPlan *g) {
     (void)xt;
-    const int n_wtiles = (N + GEMM_WROWS - 1) / GEMM_WROWS;
     const int nchunks = K / 256;
+    const int cb = gemm_chunk_bytes(wf);
     // K slices for a tile count: split when the tiles fill at most half the SMs, keeping >= 4 chunks a slice
     auto slices = [&](long tiles) -> int {
         if (force && force->splits) return force->splits;
@@ -536,31 +593,38 @@ inline int gemm_plan(int wf, int xt, int M, int N, int K, const lwq_config *forc
         if (sp > nchunks / 4) sp = nchunks / 4;
         return sp < 1 ? 1 : (int)sp;
     };
-    int bn = force && force->tile_m ? force->tile_m : 0;
-    if (!bn) {
-        // token tile: the persistent grid runs ceil(items / sms) rounds of work items (a tile's K slice);
-        // an item costs ~ (K / slices) * (BN + 128) (the constant stands for the k-block's decode and
-        // pipeline overhead, measured to be worth about half a 256-wide MMA).  Pick the multiple of 16
-        // with the least rounds * (BN + 128) / slices, preferring larger tiles on ties.
-        double best = -1;
-        const int hi = M < 256 ? ((M + 15) / 16) * 16 : 256;
-        for (int c = hi; c >= 32; c -= 16) {
-            const long tiles = (long)n_wtiles * ((M + c - 1) / c);
+    if (force && force->tile_n && force->tile_n != 128 && force->tile_n != 256) return LWQ_ERR_UNSUPPORTED;
+    if (force && force->tile_m && (force->tile_m < 32 || force->tile_m > 256 || force->tile_m % 16))
+        return LWQ_ERR_UNSUPPORTED;
+    // weight tile (128 or 256 rows) and token tile (a multiple of 16 from 32 to 256): the least
+    // modelled time, rounds of the persistent grid x the time of one work item (a tile's K slice)
+    double best = -1;
+    int bh = 0, bn = 0;
+    for (int h = 1; h <= 2; ++h) {
+        if (force && force->tile_n && force->tile_n != 128 * h) continue;
+        const int hi = force && force->tile_m ? force->tile_m : (M < 256 ? ((M + 15) / 16) * 16 : 256);
+        const int lo = force && force->tile_m ? force->tile_m : 32;
+        for (int c = hi; c >= lo; c -= 16) {
+            int na = 0, nb = 0, np = 0;
+            if (!gemm_rings(cb, c, h, force, &na, &nb, &np)) continue;
+            const long tiles = (long)((N + 128 * h - 1) / (128 * h)) * ((M + c - 1) / c);
             const int sp = slices(tiles);
             const long rounds = (tiles * sp + sms - 1) / sms;
-            const double cost = (double)rounds * (c + 128) / sp;
-            if (best < 0 || cost < best) {
+            const double kbs = (double)((nchunks + sp - 1) / sp) * GEMM_KB_PER_CHUNK;
+            double item = kbs * gemm_kblock_ns(cb, c, h, nb) + 1500.0;
+            if (gemm_nbuf(h, c) == 1 && rounds > 1) item += h * c * 512.0 / 100.0;   // epilogue not overlapped
+            const double cost = (double)rounds * item;
+            if (best < 0 || cost < best * 0.999) {
                 best = cost;
+                bh = h;
                 bn = c;
             }
         }
     }
-    if (bn < 32 || bn > 256 || bn % 16) return LWQ_ERR_UNSUPPORTED;
-    const int cb = gemm_chunk_bytes(wf);
-    int nb = 0, np = 0;
-    gemm_rings(cb, bn, force, &nb, &np);
-    if (nb < 2 || gemm_smem_bytes(cb, bn, GEMM_A_STAGES, nb, np) > 232448) return LWQ_ERR_UNSUPPORTED;
-    const int tiles = n_wtiles * ((M + bn - 1) / bn);
+    if (!bh) return LWQ_ERR_UNSUPPORTED;
+    int na = 0, nb = 0, np = 0;
+    if (!gemm_rings(cb, bn, bh, force, &na, &nb, &np) || nb < 2) return LWQ_ERR_UNSUPPORTED;
+    const int tiles = ((N + 128 * bh - 1) / (128 * bh)) * ((M + bn - 1) / bn);
     int splits = slices(tiles);
     if (splits < 1 || splits > nchunks) return LWQ_ERR_UNSUPPORTED;
     const int cps = (nchunks + splits - 1) / splits;
@@ -573,9 +637,9 @@ inline int gemm_plan(int wf, int xt, int M, int N, int K, const lwq_config *forc
     g->warps = GEMM_DQ_WARPS;
     g->stages = nb;
     g->ctas = ctas;
-    g->tile_n = GEMM_WROWS;
+    g->tile_n = 128 * bh;
     g->tile_m = bn;
-    g->smem = gemm_smem_bytes(cb, bn, GEMM_A_STAGES, nb, np);
+    g->smem = gemm_smem_bytes(cb, bn, bh, na, nb, np);
     return LWQ_OK;
 }
 

@@ -169,7 +169,8 @@ typedef struct {
     int stages;      /* pipeline depth (shared-memory ring stages) */
     int splits;      /* GEMV: split-K factor (1 = none) */
     int ctas;        /* CTAs launched (persistent grid) */
-    int tile_n;      /* GEMM: output columns per tile (weights rows) */
+    int tile_n;      /* GEMM: output columns per tile (weight rows): 128, or 256 as two
+                        128-row halves sharing each activation tile */
     int tile_m;      /* GEMM: output rows per tile (activation rows) */
     int reserved[5];
 } lwq_config;

@@ -142,6 +142,34 @@ def test_config_table_rules(w, a, M, N, K, warps, splits, stages):
     assert (cfg.path, cfg.warps, cfg.splits, cfg.stages) == (1, warps, splits, stages)
 
 
+@pytest.mark.parametrize("w,a,M,N,K,tile_n,tile_m,ctas", [
+    # 256 weight rows x 176 tokens: 43 x 3 = 129 tiles, one round (measured 52 us; 128 x 176 took 70 us)
+    ("q4_0", "bf16", 512, 11008, 4096, 256, 176, 129),
+    # 256 x 240: 16 x 9 = 144 tiles, one round (measured 157 us; 128 x 256, two rounds, 172 us)
+    ("q4_0", "bf16", 2048, 4096, 11008, 256, 240, 144),
+])
+def test_gemm_table_rules(w, a, M, N, K, tile_n, tile_m, ctas):
+    """The GEMM rows of the per-shape table (148 SMs when no GPU is present): the weight and token tiles
+    with the least modelled time, rounds of the persistent grid x the time of one tile."""
+    if lwq.lwq_select_config(lwq.fmt_code("q4_0", "f32"), 1, 11008, 4096).ctas != 148:
+        pytest.skip("a device with another SM count is present")
+    cfg = lwq.lwq_select_config(lwq.fmt_code(w, a), M, N, K)
+    assert (cfg.path, cfg.tile_n, cfg.tile_m, cfg.ctas, cfg.splits) == (2, tile_n, tile_m, ctas, 1)
+
+
+def test_gemm_tile_choices_are_valid():
+    """Every GEMM row of the sweep has a 128- or 256-row weight tile and a token tile that is a
+    multiple of 16 in [32, 256]."""
+    for w in ("q8_0", "q4_0", "q4_k"):
+        for K, N in ((4096, 4096), (4096, 14336), (14336, 4096), (4096, 32000)):
+            for M in (17, 64, 256, 1024):
+                cfg = lwq.lwq_select_config(lwq.fmt_code(w, "f16"), M, N, K)
+                assert cfg.path == 2
+                assert cfg.tile_n in (128, 256)
+                assert 32 <= cfg.tile_m <= 256 and cfg.tile_m % 16 == 0
+                assert cfg.stages >= 2 and cfg.splits >= 1 and 1 <= cfg.ctas <= 148
+
+
 def test_int8_flag_plan():
     i8 = lwq.fmt_code("q4_0", "bf16") | lwq.LWQ_FLAG_ACT_I8
     cfg = lwq.lwq_select_config(i8, 16, 4096, 4096)

@@ -126,6 +126,26 @@ def test_gemm_split_k(dev, w, a, M, N, K, splits):
     check_full(w, a, M, N, K, dev, seed=M + N, cfg=cfg)
 
 
+GEMM_256_CASES = [
+    (40, 300, 2048, 48, 0, 0),        # N ends inside the second half of the only weight tile
+    (130, 1000, 1024, 64, 0, 3),      # two accumulator buffers (2 x 2 x 64 columns), several tiles per CTA
+    (300, 700, 1536, 176, 0, 2),      # one accumulator buffer, the epilogue before the next tile's MMAs
+    (96, 513, 3072, 96, 3, 0),        # K slices: fp32 partials added by the follow-up kernel
+    (257, 256, 512, 256, 0, 1)]       # widest token tile, one CTA walks both token tiles
+
+
+# Q8_0's packed chunks of 256 rows (2 x 68 KB) leave room for token tiles up to 96 only
+@pytest.mark.parametrize("w,a,M,N,K,bn,splits,ctas",
+                         [(w, a) + c for w, a in [("q4_0", "bf16"), ("q4_k", "f16"), ("q4_0", "f16")]
+                          for c in GEMM_256_CASES] +
+                         [("q8_0", "bf16", 130, 1000, 1024, 64, 0, 3), ("q8_0", "f16", 96, 513, 3072, 96, 3, 0)])
+def test_gemm_256_row_tiles(dev, w, a, M, N, K, bn, splits, ctas):
+    """256-row weight tiles (two UMMAs per K step share the activation tile) against the oracle."""
+    cfg = lwq.lwq_config()
+    cfg.path, cfg.tile_n, cfg.tile_m, cfg.splits, cfg.ctas = 2, 256, bn, splits, ctas
+    check_full(w, a, M, N, K, dev, seed=M + N + bn, cfg=cfg)
+
+
 @pytest.mark.parametrize("w,a,M", [("q4_0", "f32", 1), ("q4_k", "f16", 1), ("q8_0", "f16", 16)])
 def test_split_k_deterministic(dev, w, a, M):
     """Repeated calls (split-K: partials added in split order by a follow-up kernel) are bitwise identical."""
