@@ -16,6 +16,12 @@ Quantizacao"):
   nibble; the weight is ``(nibble-8)*d``.
 * Q4_K -- 256 weights per 144-byte superblock: fp16 ``d``, fp16 ``dmin``,
   12 bytes holding eight 6-bit (scale, min) pairs, 128 bytes of nibbles.
+* Q6_K -- 256 weights per 210-byte superblock: 128 bytes of low nibbles, 64
+  bytes of 2-bit high parts, 16 int8 scales (one per 16 weights), fp16 ``d``.
+* Q5_K -- 256 weights per 176-byte superblock: fp16 ``d``, fp16 ``dmin``, the
+  12 scale/min bytes of Q4_K, 32 bytes of fifth bits, 128 bytes of nibbles.
+* Q2_K -- 256 weights per 84-byte superblock: 16 bytes of 4-bit (scale, min)
+  pairs, 64 bytes of 2-bit codes, fp16 ``d``, fp16 ``dmin``.
 
 Draw order for one tensor: a fresh ``numpy.random.default_rng(seed)``
 (PCG64) draws the weight tensor first (row-major [N][K]) and then the
@@ -28,8 +34,8 @@ import numpy as np
 
 QK = 32          # weights per Q8_0 / Q4_0 block
 QK_K = 256       # weights per Q4_K superblock
-BLOCK_BYTES = {"q8_0": 34, "q4_0": 18, "q4_k": 144}
-BLOCK_WEIGHTS = {"q8_0": QK, "q4_0": QK, "q4_k": QK_K}
+BLOCK_BYTES = {"q8_0": 34, "q4_0": 18, "q4_k": 144, "q6_k": 210, "q5_k": 176, "q2_k": 84}
+BLOCK_WEIGHTS = {"q8_0": QK, "q4_0": QK, "q4_k": QK_K, "q6_k": QK_K, "q5_k": QK_K, "q2_k": QK_K}
 
 
 def row_bytes(fmt: str, K: int) -> int:
@@ -130,6 +136,77 @@ def random_q4_k(g: np.random.Generator, N: int, K: int) -> np.ndarray:
     return out.reshape(N, nb * 144)
 
 
+def _superblocks(fmt: str, K: int) -> int:
+    if K % QK_K:
+        raise ValueError(f"{fmt} needs K % 256 == 0")
+    return K // QK_K
+
+
+def random_q6_k(g: np.random.Generator, N: int, K: int) -> np.ndarray:
+    """Random Q6_K bytes [N][K/256*210].
+
+    d ~ U(0, 0.01) drawn in fp32 and rounded to fp16; the 16 int8 scales,
+    the 128 low-nibble bytes and the 64 high-bit bytes are uniform random
+    bytes (uniform 6-bit codes and int8 scales).  Draw order: d[N][nb],
+    scale bytes[N][nb][16], low bytes[N][nb][128], high bytes[N][nb][64].
+    Layout: low bytes at 0, high bytes at 128, scales at 192, d at 208.
+    """
+    nb = _superblocks("q6_k", K)
+    d = g.uniform(0.0, 0.01, size=(N, nb)).astype(np.float32)
+    sc = g.integers(0, 256, size=(N, nb, 16), dtype=np.uint8)
+    ql = g.integers(0, 256, size=(N, nb, 128), dtype=np.uint8)
+    qh = g.integers(0, 256, size=(N, nb, 64), dtype=np.uint8)
+    out = np.empty((N, nb, 210), dtype=np.uint8)
+    out[..., 0:128] = ql
+    out[..., 128:192] = qh
+    out[..., 192:208] = sc
+    out[..., 208:210] = _f16_bits(d).view(np.uint8).reshape(N, nb, 2)
+    return out.reshape(N, nb * 210)
+
+
+def random_q5_k(g: np.random.Generator, N: int, K: int) -> np.ndarray:
+    """Random Q5_K bytes [N][K/256*176].
+
+    d and dmin ~ U(0, 0.01) rounded to fp16; scale/min, fifth-bit and nibble
+    bytes uniform.  Draw order: d[N][nb], dmin[N][nb], scale bytes[N][nb][12],
+    fifth-bit bytes[N][nb][32], nibble bytes[N][nb][128].  Layout: d at 0,
+    dmin at 2, scales at 4, fifth bits at 16, nibbles at 48.
+    """
+    nb = _superblocks("q5_k", K)
+    d = g.uniform(0.0, 0.01, size=(N, nb)).astype(np.float32)
+    dmin = g.uniform(0.0, 0.01, size=(N, nb)).astype(np.float32)
+    sc = g.integers(0, 256, size=(N, nb, 12), dtype=np.uint8)
+    qh = g.integers(0, 256, size=(N, nb, 32), dtype=np.uint8)
+    qs = g.integers(0, 256, size=(N, nb, 128), dtype=np.uint8)
+    out = np.empty((N, nb, 176), dtype=np.uint8)
+    out[..., 0:2] = _f16_bits(d).view(np.uint8).reshape(N, nb, 2)
+    out[..., 2:4] = _f16_bits(dmin).view(np.uint8).reshape(N, nb, 2)
+    out[..., 4:16] = sc
+    out[..., 16:48] = qh
+    out[..., 48:176] = qs
+    return out.reshape(N, nb * 176)
+
+
+def random_q2_k(g: np.random.Generator, N: int, K: int) -> np.ndarray:
+    """Random Q2_K bytes [N][K/256*84].
+
+    d and dmin ~ U(0, 0.01) rounded to fp16; scale/min bytes and code bytes
+    uniform.  Draw order: d[N][nb], dmin[N][nb], scale bytes[N][nb][16], code
+    bytes[N][nb][64].  Layout: scales at 0, codes at 16, d at 80, dmin at 82.
+    """
+    nb = _superblocks("q2_k", K)
+    d = g.uniform(0.0, 0.01, size=(N, nb)).astype(np.float32)
+    dmin = g.uniform(0.0, 0.01, size=(N, nb)).astype(np.float32)
+    sc = g.integers(0, 256, size=(N, nb, 16), dtype=np.uint8)
+    qs = g.integers(0, 256, size=(N, nb, 64), dtype=np.uint8)
+    out = np.empty((N, nb, 84), dtype=np.uint8)
+    out[..., 0:16] = sc
+    out[..., 16:80] = qs
+    out[..., 80:82] = _f16_bits(d).view(np.uint8).reshape(N, nb, 2)
+    out[..., 82:84] = _f16_bits(dmin).view(np.uint8).reshape(N, nb, 2)
+    return out.reshape(N, nb * 84)
+
+
 def activations(g: np.random.Generator, M: int, K: int, act: str) -> np.ndarray:
     """x ~ N(0,1) drawn in fp32 [M][K], then stored in ``act``.
 
@@ -162,6 +239,12 @@ def make_weights(fmt: str, g: np.random.Generator, N: int, K: int) -> np.ndarray
         return quantize_q4_0(normal_weights(g, N, K))
     if fmt == "q4_k":
         return random_q4_k(g, N, K)
+    if fmt == "q6_k":
+        return random_q6_k(g, N, K)
+    if fmt == "q5_k":
+        return random_q5_k(g, N, K)
+    if fmt == "q2_k":
+        return random_q2_k(g, N, K)
     raise ValueError(fmt)
 
 

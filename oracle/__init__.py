@@ -21,7 +21,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "lwq_oracle.c")
 _LIB = os.path.join(_HERE, "liblwq_oracle.so")
 
-FMT = {"q8_0": 1, "q4_0": 2, "q4_k": 3}
+FMT = {"q8_0": 1, "q4_0": 2, "q4_k": 3, "q6_k": 4, "q5_k": 5, "q2_k": 6}
 ACT = {"f32": 0, "f16": 1, "bf16": 2}
 
 CFLAGS = ["-O2", "-fopenmp", "-ffp-contract=off", "-shared", "-fPIC", "-std=c11"]

@@ -32,6 +32,21 @@
  *         Nibbles: 4 groups g of 32 bytes; element 64g+l = qs[32g+l] & 15
  *         (sub-block 2g) and element 64g+32+l = qs[32g+l] >> 4 (sub-block
  *         2g+1), l < 32.  w = d*sc_j*q - dmin*m_j for element in sub-block j.
+ *   Q6_K: superblock of 256 weights, 210 bytes: ql[128] (low 4 bits of the
+ *         6-bit codes), qh[64] (high 2 bits), int8 sc[16] (one scale per 16
+ *         weights), fp16 d last.  Element e = 128n + 32g + l (n < 2, g < 4,
+ *         l < 32): low bits = nibble (g >> 1) of ql[64n + 32(g & 1) + l]
+ *         (0 = low, 1 = high), high bits = bits 2g, 2g+1 of qh[32n + l];
+ *         q = low | high << 4 in [0, 64); w = d * sc[e / 16] * (q - 32).
+ *   Q5_K: superblock of 256 weights, 176 bytes: fp16 d, fp16 dmin, s[12]
+ *         (scales and mins packed as for Q4_K), qh[32], qs[128].  Element
+ *         e = 64g + 32h + l (g < 4, h < 2, l < 32): low bits = nibble h of
+ *         qs[32g + l], fifth bit = bit 2g + h of qh[l]; sub-block j = 2g + h;
+ *         w = d*sc_j*q - dmin*m_j.
+ *   Q2_K: superblock of 256 weights, 84 bytes: s[16] (per 16 weights: scale
+ *         in the low nibble, min in the high nibble), qs[64], fp16 d, fp16
+ *         dmin.  Element e = 128n + 32j + l (n < 2, j < 4, l < 32): q = bits
+ *         2j, 2j+1 of qs[32n + l]; w = d*(s[e/16] & 15)*q - dmin*(s[e/16] >> 4).
  *
  * Activations x are fp32, fp16 or bf16 codes; each is decoded exactly from
  * its IEEE-754 bit fields.
@@ -52,6 +67,9 @@
 #define OR_Q8_0 1
 #define OR_Q4_0 2
 #define OR_Q4_K 3
+#define OR_Q6_K 4
+#define OR_Q5_K 5
+#define OR_Q2_K 6
 #define OR_ACT_F32 0
 #define OR_ACT_F16 1
 #define OR_ACT_BF16 2
@@ -92,7 +110,10 @@ long lwq_oracle_block_weights(int fmt) {
     switch (fmt) {
     case OR_Q8_0: return 32;
     case OR_Q4_0: return 32;
-    case OR_Q4_K: return 256;
+    case OR_Q4_K:
+    case OR_Q6_K:
+    case OR_Q5_K:
+    case OR_Q2_K: return 256;
     default: return -1;
     }
 }
@@ -102,6 +123,9 @@ long lwq_oracle_block_bytes(int fmt) {
     case OR_Q8_0: return 34;
     case OR_Q4_0: return 18;
     case OR_Q4_K: return 144;
+    case OR_Q6_K: return 210;
+    case OR_Q5_K: return 176;
+    case OR_Q2_K: return 84;
     default: return -1;
     }
 }
@@ -163,6 +187,46 @@ static void decode_q4_k(const uint8_t *b, float *w) {
     }
 }
 
+static void decode_q6_k(const uint8_t *b, float *w) {
+    const uint8_t *ql = b, *qh = b + 128;
+    const int8_t *sc = (const int8_t *)(b + 192);
+    double d = lwq_oracle_f16(rd16(b + 208));
+    for (int e = 0; e < 256; e++) {
+        int n = e / 128, g = (e % 128) / 32, l = e % 32;
+        int low = (ql[64 * n + 32 * (g & 1) + l] >> (4 * (g >> 1))) & 15;
+        int high = (qh[32 * n + l] >> (2 * g)) & 3;
+        int q = low | (high << 4);
+        /* d (11 bits) * sc (8) * (q - 32) (6): exact in fp64 and in fp32 */
+        w[e] = (float)(d * (double)sc[e / 16] * (double)(q - 32));
+    }
+}
+
+static void decode_q5_k(const uint8_t *b, float *w) {
+    double d = lwq_oracle_f16(rd16(b));
+    double dmin = lwq_oracle_f16(rd16(b + 2));
+    const uint8_t *s = b + 4, *qh = b + 16, *qs = b + 48;
+    for (int e = 0; e < 256; e++) {
+        int g = e / 64, h = (e % 64) / 32, l = e % 32;
+        int q = ((qs[32 * g + l] >> (4 * h)) & 15) | (((qh[l] >> (2 * g + h)) & 1) << 4);
+        int sc, m;
+        lwq_oracle_q4k_scale_min(s, 2 * g + h, &sc, &m);
+        /* d*sc*q (<= 22 significant bits) and dmin*m (<= 17) exact in fp64, as for Q4_K */
+        w[e] = (float)(d * (double)sc * (double)q - dmin * (double)m);
+    }
+}
+
+static void decode_q2_k(const uint8_t *b, float *w) {
+    const uint8_t *s = b, *qs = b + 16;
+    double d = lwq_oracle_f16(rd16(b + 80));
+    double dmin = lwq_oracle_f16(rd16(b + 82));
+    for (int e = 0; e < 256; e++) {
+        int n = e / 128, j = (e % 128) / 32, l = e % 32;
+        int q = (qs[32 * n + l] >> (2 * j)) & 3;
+        int sc = s[e / 16] & 15, m = s[e / 16] >> 4;
+        w[e] = (float)(d * (double)sc * (double)q - dmin * (double)m);
+    }
+}
+
 /* Decode one packed row of K weights into fp32.  Returns 0, or -1 on bad args. */
 int lwq_oracle_dequant_row(int fmt, const uint8_t *row, long K, float *out) {
     long bw = lwq_oracle_block_weights(fmt);
@@ -171,9 +235,14 @@ int lwq_oracle_dequant_row(int fmt, const uint8_t *row, long K, float *out) {
     for (long blk = 0; blk < K / bw; blk++) {
         const uint8_t *b = row + blk * bb;
         float *w = out + blk * bw;
-        if (fmt == OR_Q8_0) decode_q8_0(b, w);
-        else if (fmt == OR_Q4_0) decode_q4_0(b, w);
-        else decode_q4_k(b, w);
+        switch (fmt) {
+        case OR_Q8_0: decode_q8_0(b, w); break;
+        case OR_Q4_0: decode_q4_0(b, w); break;
+        case OR_Q4_K: decode_q4_k(b, w); break;
+        case OR_Q6_K: decode_q6_k(b, w); break;
+        case OR_Q5_K: decode_q5_k(b, w); break;
+        default: decode_q2_k(b, w); break;
+        }
     }
     return 0;
 }

@@ -103,6 +103,45 @@ def indep_decode(fmt: str, Wq: np.ndarray, K: int) -> np.ndarray:
         q = np.stack([qs & 15, qs >> 4], axis=3).reshape(N, K // 256, 8, 32)  # sub-block j = 2g + half
         w = d[..., None, None] * sc[..., None] * q - dmin[..., None, None] * mn[..., None]
         return w.reshape(N, K)
+    if fmt == "q6_k":
+        b = W.reshape(N, K // 256, 210)
+        d = indep_f16(b[..., 208:210].copy().view(np.uint16)[..., 0])
+        sc = b[..., 192:208].view(np.int8).astype(np.float64)              # [N][nb][16]
+        ql = b[..., 0:128].reshape(N, K // 256, 2, 2, 32).astype(np.int64)  # [half][ql quarter][l]
+        qh = b[..., 128:192].reshape(N, K // 256, 2, 1, 32).astype(np.int64)
+        low = np.concatenate([ql & 15, ql >> 4], axis=3)                   # [half][g = 2*nibble + quarter][l]
+        high = (qh >> (2 * np.arange(4)[None, None, None, :, None])) & 3
+        q = (low | (high << 4)).reshape(N, K // 256, 256).astype(np.float64) - 32.0
+        return (d[..., None] * np.repeat(sc, 16, axis=-1) * q).reshape(N, K)
+    if fmt == "q5_k":
+        b = W.reshape(N, K // 256, 176)
+        d = indep_f16(b[..., 0:2].copy().view(np.uint16)[..., 0])
+        dmin = indep_f16(b[..., 2:4].copy().view(np.uint16)[..., 0])
+        s = b[..., 4:16].astype(np.int64)
+        sc = np.empty(s.shape[:-1] + (8,), dtype=np.int64)
+        mn = np.empty_like(sc)
+        sc[..., :4] = s[..., 0:4] & 63
+        mn[..., :4] = s[..., 4:8] & 63
+        sc[..., 4:] = (s[..., 8:12] & 15) | ((s[..., 0:4] >> 6) << 4)
+        mn[..., 4:] = (s[..., 8:12] >> 4) | ((s[..., 4:8] >> 6) << 4)
+        qh = b[..., 16:48].astype(np.int64)                                # [N][nb][32]
+        qs = b[..., 48:176].reshape(N, K // 256, 4, 32).astype(np.int64)
+        nib = np.stack([qs & 15, qs >> 4], axis=3)                         # [g][h][l]
+        bit = np.stack([(qh[..., None, :] >> (2 * np.arange(4)[:, None] + h)) & 1 for h in (0, 1)], axis=3)
+        q = (nib | (bit << 4)).reshape(N, K // 256, 8, 32)                 # sub-block j = 2g + h
+        w = d[..., None, None] * sc[..., None] * q - dmin[..., None, None] * mn[..., None]
+        return w.reshape(N, K)
+    if fmt == "q2_k":
+        b = W.reshape(N, K // 256, 84)
+        s = b[..., 0:16].astype(np.int64)
+        d = indep_f16(b[..., 80:82].copy().view(np.uint16)[..., 0])
+        dmin = indep_f16(b[..., 82:84].copy().view(np.uint16)[..., 0])
+        qs = b[..., 16:80].reshape(N, K // 256, 2, 1, 32).astype(np.int64)
+        q = ((qs >> (2 * np.arange(4)[None, None, None, :, None])) & 3).reshape(N, K // 256, 256)
+        scale = np.repeat(s & 15, 16, axis=-1)
+        mins = np.repeat(s >> 4, 16, axis=-1)
+        w = d[..., None] * scale * q - dmin[..., None] * mins
+        return w.reshape(N, K)
     raise ValueError(fmt)
 
 
@@ -207,7 +246,7 @@ def pin_roundtrip_q4_0(lib):
 def pin_bruteforce_one_block(lib):
     """K = one block, N, M <= 3: oracle y equals Python-loop sums over an independent decode."""
     g = np.random.default_rng(99)
-    for fmt, K in (("q8_0", 32), ("q4_0", 32), ("q4_k", 256)):
+    for fmt, K in (("q8_0", 32), ("q4_0", 32), ("q4_k", 256), ("q6_k", 256), ("q5_k", 256), ("q2_k", 256)):
         for act in ("f32", "f16", "bf16"):
             for M, N in ((1, 1), (2, 3), (3, 2)):
                 Wq = inputs.make_weights(fmt, g, N, K)
@@ -232,7 +271,7 @@ def pin_bruteforce_one_block(lib):
 def pin_library_matmul(lib):
     """Oracle y equals torch.matmul (fp64) of the independently decoded W, to 1e-12 relative to den."""
     g = np.random.default_rng(5)
-    for fmt, K in (("q8_0", 512), ("q4_0", 512), ("q4_k", 512)):
+    for fmt, K in (("q8_0", 512), ("q4_0", 512), ("q4_k", 512), ("q6_k", 512), ("q5_k", 512), ("q2_k", 512)):
         for act in ("f32", "f16", "bf16"):
             M, N = 5, 37
             Wq = inputs.make_weights(fmt, g, N, K)
@@ -289,12 +328,18 @@ def pin_zero_denominator(lib):
     Wq = inputs.make_weights("q4_k", np.random.default_rng(4), N, 256)
     y, den = oracle.matmul("q4_k", Wq, np.zeros((2, 256), dtype=np.float16), lib=lib)
     assert np.all(y == 0) and np.all(den == 0)
+    # Q6_K: every code 32 (low nibbles 0, high bits 2) is zero whatever the scales and d
+    blk = np.asarray(inputs.make_weights("q6_k", np.random.default_rng(5), N, 512)).reshape(N, 2, 210).copy()
+    blk[..., 0:128] = 0
+    blk[..., 128:192] = 0xAA
+    y, den = oracle.matmul("q6_k", blk.reshape(N, -1), np.random.default_rng(6).standard_normal((2, 512)).astype(np.float32), lib=lib)
+    assert np.all(y == 0) and np.all(den == 0)
 
 
 def pin_sampled_equals_full(lib):
     """The sampled entry point returns bit-identical values to the full product."""
     g = np.random.default_rng(21)
-    for fmt, K in (("q8_0", 256), ("q4_0", 288), ("q4_k", 512)):
+    for fmt, K in (("q8_0", 256), ("q4_0", 288), ("q4_k", 512), ("q6_k", 768), ("q5_k", 512), ("q2_k", 256)):
         M, N = 3, 23
         Wq = inputs.make_weights(fmt, g, N, K)
         x = inputs.activations(g, M, K, "f16")
@@ -310,8 +355,11 @@ def pin_row_bytes(lib):
     for fmt, K, rb in (("q8_0", 4096, 4352), ("q4_0", 4096, 2304), ("q4_k", 4096, 2304),
                        ("q4_0", 11008, 6192), ("q4_k", 11008, 6192), ("q8_0", 14336, 15232)):
         assert lib.lwq_oracle_row_bytes(oracle.FMT[fmt], K) == rb
+    for fmt, K, rb in (("q6_k", 4096, 3360), ("q6_k", 11008, 9030), ("q5_k", 4096, 2816), ("q2_k", 4096, 1344)):
+        assert lib.lwq_oracle_row_bytes(oracle.FMT[fmt], K) == rb
     assert lib.lwq_oracle_row_bytes(oracle.FMT["q4_k"], 128) == -1
     assert lib.lwq_oracle_row_bytes(oracle.FMT["q4_0"], 48) == -1
+    assert lib.lwq_oracle_row_bytes(oracle.FMT["q6_k"], 288) == -1
 
 
 ALL_PINS = [pin_hand_blocks, pin_f16_exhaustive, pin_bf16_exhaustive, pin_q4k_scale_roundtrip,

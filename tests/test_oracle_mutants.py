@@ -25,7 +25,25 @@ MUTANTS = {
     "q4_k_min_high_bits": ("*m = (s[j + 4] >> 4) | ((s[j] >> 6) << 4);", "*m = (s[j + 4] >> 4);"),
     "q4_k_group_halves": ("int qlo = qs[32 * g + l] & 15;\n            int qhi = qs[32 * g + l] >> 4;",
                           "int qlo = qs[32 * g + l] >> 4;\n            int qhi = qs[32 * g + l] & 15;"),
-    "q4_k_dmin_is_d": ("double dmin = lwq_oracle_f16(rd16(b + 2));", "double dmin = lwq_oracle_f16(rd16(b));"),
+    "q4_k_dmin_is_d": ("double dmin = lwq_oracle_f16(rd16(b + 2));\n    const uint8_t *s = b + 4;\n    const uint8_t *qs",
+                       "double dmin = lwq_oracle_f16(rd16(b));\n    const uint8_t *s = b + 4;\n    const uint8_t *qs"),
+    "q5_k_dmin_is_d": ("double dmin = lwq_oracle_f16(rd16(b + 2));\n    const uint8_t *s = b + 4, *qh",
+                       "double dmin = lwq_oracle_f16(rd16(b));\n    const uint8_t *s = b + 4, *qh"),
+    "q6_k_no_offset": ("(double)sc[e / 16] * (double)(q - 32)", "(double)sc[e / 16] * (double)(q)"),
+    "q6_k_high_shift": ("int high = (qh[32 * n + l] >> (2 * g)) & 3;", "int high = (qh[32 * n + l] >> g) & 3;"),
+    "q6_k_low_quarter": ("ql[64 * n + 32 * (g & 1) + l] >> (4 * (g >> 1))", "ql[64 * n + 32 * (g >> 1) + l] >> (4 * (g & 1))"),
+    "q6_k_scale_per_32": ("(double)sc[e / 16] * (double)(q - 32)", "(double)sc[e / 32] * (double)(q - 32)"),
+    "q6_k_d_offset": ("double d = lwq_oracle_f16(rd16(b + 208));", "double d = lwq_oracle_f16(rd16(b + 206));"),
+    "q6_k_unsigned_scale": ("const int8_t *sc = (const int8_t *)(b + 192);", "const uint8_t *sc = (const uint8_t *)(b + 192);"),
+    "q5_k_fifth_bit_index": ("(((qh[l] >> (2 * g + h)) & 1) << 4)", "(((qh[l] >> (g + 4 * h)) & 1) << 4)"),
+    "q5_k_no_fifth_bit": ("| (((qh[l] >> (2 * g + h)) & 1) << 4)", ""),
+    "q5_k_swapped_arrays": ("*qh = b + 16, *qs = b + 48;", "*qh = b + 144, *qs = b + 16;"),
+    "q5_k_min_sign": ("(double)q - dmin * (double)m);\n    }\n}\n\nstatic void decode_q2_k",
+                      "(double)q + dmin * (double)m);\n    }\n}\n\nstatic void decode_q2_k"),
+    "q2_k_min_nibble": ("m = s[e / 16] >> 4;", "m = s[e / 16] & 15;"),
+    "q2_k_field_shift": ("int q = (qs[32 * n + l] >> (2 * j)) & 3;", "int q = (qs[32 * n + l] >> j) & 3;"),
+    "q2_k_d_is_dmin": ("double d = lwq_oracle_f16(rd16(b + 80));", "double d = lwq_oracle_f16(rd16(b + 82));"),
+    "q2_k_half_stride": ("int q = (qs[32 * n + l] >> (2 * j)) & 3;", "int q = (qs[16 * n + l] >> (2 * j)) & 3;"),
     "f16_bias": ("v = ldexp((double)(1024 + f), e - 25);", "v = ldexp((double)(1024 + f), e - 24);"),
     "f16_subnormal": ("v = ldexp((double)f, -24);", "v = ldexp((double)(1024 + f), -24);"),
     "bf16_bias": ("v = ldexp((double)(128 + f), e - 134);", "v = ldexp((double)(128 + f), e - 133);"),
