@@ -18,7 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblwq.so")
 
 # codes (include/lwq.h)
-LWQ_Q8_0, LWQ_Q4_0, LWQ_Q4_K = 1, 2, 3
+LWQ_Q8_0, LWQ_Q4_0, LWQ_Q4_K, LWQ_Q6_K, LWQ_Q5_K, LWQ_Q2_K = 1, 2, 3, 4, 5, 6
 LWQ_ACT_F32, LWQ_ACT_F16, LWQ_ACT_BF16 = 0x000, 0x100, 0x200
 LWQ_FLAG_OVERLAP = 0x1000   # weights constant: allow programmatic dependent launch
 LWQ_FLAG_ACT_I8 = 0x2000    # int8 activation blocks of 32 (integer block dot products)
@@ -33,7 +33,8 @@ LWQ_ERR_DEVICE_TIMEOUT = 7
 STATUS = {0: "LWQ_OK", 1: "LWQ_ERR_INVALID_ARG", 2: "LWQ_ERR_UNSUPPORTED", 3: "LWQ_ERR_MISALIGNED",
           4: "LWQ_ERR_NOT_INITIALIZED", 5: "LWQ_ERR_WORKSPACE_TOO_SMALL", 6: "LWQ_ERR_CUDA",
           7: "LWQ_ERR_DEVICE_TIMEOUT"}
-WEIGHT_FORMATS = {"q8_0": LWQ_Q8_0, "q4_0": LWQ_Q4_0, "q4_k": LWQ_Q4_K}
+WEIGHT_FORMATS = {"q8_0": LWQ_Q8_0, "q4_0": LWQ_Q4_0, "q4_k": LWQ_Q4_K, "q6_k": LWQ_Q6_K, "q5_k": LWQ_Q5_K,
+                  "q2_k": LWQ_Q2_K}
 ACT_DTYPES = {"f32": LWQ_ACT_F32, "f16": LWQ_ACT_F16, "bf16": LWQ_ACT_BF16}
 
 # every symbol the header declares
@@ -123,7 +124,7 @@ def _check(rc: int, where: str) -> int:
 
 
 def fmt_code(weights: str, act: str) -> int:
-    """``fmt`` for the C ABI from names: weights in q8_0/q4_0/q4_k, act in f32/f16/bf16."""
+    """``fmt`` for the C ABI from names: weights in q8_0/q4_0/q4_k/q6_k/q5_k/q2_k, act in f32/f16/bf16."""
     return WEIGHT_FORMATS[weights] | ACT_DTYPES[act]
 
 

@@ -71,8 +71,28 @@ int sm_count(int dev) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int block_weights(int wf) { return wf == LWQ_Q4_K ? 256 : (wf == LWQ_Q8_0 || wf == LWQ_Q4_0 ? 32 : 0); }
-int block_bytes(int wf) { return wf == LWQ_Q4_K ? 144 : (wf == LWQ_Q8_0 ? 34 : (wf == LWQ_Q4_0 ? 18 : 0)); }
+int block_weights(int wf) {
+    switch (wf) {
+    case LWQ_Q8_0:
+    case LWQ_Q4_0: return 32;
+    case LWQ_Q4_K:
+    case LWQ_Q6_K:
+    case LWQ_Q5_K:
+    case LWQ_Q2_K: return 256;
+    default: return 0;
+    }
+}
+int block_bytes(int wf) {
+    switch (wf) {
+    case LWQ_Q8_0: return 34;
+    case LWQ_Q4_0: return 18;
+    case LWQ_Q4_K: return 144;
+    case LWQ_Q6_K: return 210;
+    case LWQ_Q5_K: return 176;
+    case LWQ_Q2_K: return 84;
+    default: return 0;
+    }
+}
 int act_code(int fmt) {
     switch (fmt & LWQ_ACT_MASK) {
     case LWQ_ACT_F32: return X_F32;
@@ -104,14 +124,19 @@ struct Plan {
 // n8 column tiles of the GEMV for a pass of mg activation rows: each row takes
 // P columns (P = 3 bf16 parts for fp32 activations, else 1), 8 columns per tile.
 inline int gemv_nt(int xt, bool i8, int mg) { return i8 ? 1 : (mg * gemv_parts(xt, i8) + 7) / 8; }
-inline int gemv_chunk_bytes(int wf) { return wf == LWQ_Q8_0 ? 272 : 144; }
+inline int gemv_chunk_bytes(int wf) { return wf == LWQ_Q8_0 ? 272 : (wf == LWQ_Q5_K ? 176 : 144); }
 inline size_t gemv_smem(int wf, int cps, int stages, int nt, bool i8, int xt, int m) {
-    return gemv_smem_layout(gemv_chunk_bytes(wf), cps, stages, nt, wf == LWQ_Q4_K, gemv_parts(xt, i8), m,
+    return gemv_smem_layout(gemv_chunk_bytes(wf), cps, stages, nt, wf == LWQ_Q4_K || wf == LWQ_Q5_K,
+                            gemv_parts(xt, i8), m,
                             xt == X_F32 ? 4 : 2, i8)
         .total;
 }
 
-bool tc_gemv_eligible(long K) { return K % 256 == 0; }
+// Formats with a tensor-core GEMV decoder (their packed rows are 16-byte
+// multiples, as the weight stream's tensor map needs); the others take the
+// simple kernel.
+bool tc_gemv_format(int wf) { return wf == LWQ_Q8_0 || wf == LWQ_Q4_0 || wf == LWQ_Q4_K || wf == LWQ_Q5_K; }
+bool tc_gemv_eligible(int wf, long K) { return tc_gemv_format(wf) && K % 256 == 0; }
 
 // Workspace layout: fp32 split-K partials [S][m_group][N].  Nothing in it
 // needs to start at any particular value.
@@ -132,7 +157,7 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
     if (!path) {
         if (M > 16 && xt != X_F32 && gemm_eligible(wf, xt, K))
             path = 2;
-        else if (tc_gemv_eligible(K))
+        else if (tc_gemv_eligible(wf, K))
             path = 1;
         else
             path = 3;
@@ -161,7 +186,7 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
         p->cfg.splits = 1;
         return LWQ_OK;
     }
-    if (path != 1 || !tc_gemv_eligible(K)) return LWQ_ERR_UNSUPPORTED;
+    if (path != 1 || !tc_gemv_eligible(wf, K)) return LWQ_ERR_UNSUPPORTED;
     p->i8 = (fmt & LWQ_FLAG_ACT_I8) != 0;
     if (p->i8 && (wf != LWQ_Q4_0 || M > 16)) return LWQ_ERR_UNSUPPORTED;
     // rows per pass: 8 with fp32 activations (3 parts, 24 columns) or int8 blocks, else 16
@@ -308,6 +333,7 @@ cudaError_t dispatch_gemv(int wf, int xt, int nt, bool i8, const CUtensorMap &ma
     case LWQ_Q4_0: { LWQ_GV(F_Q4_0) }
     case LWQ_Q8_0: { LWQ_GV(F_Q8_0) }
     case LWQ_Q4_K: { LWQ_GV(F_Q4_K) }
+    case LWQ_Q5_K: { LWQ_GV(F_Q5_K) }
     }
 #undef LWQ_GV
     return cudaErrorInvalidValue;
@@ -330,6 +356,9 @@ cudaError_t dispatch_simple(int wf, int xt, const uint8_t *W, const void *x, flo
     case LWQ_Q8_0: { LWQ_SIMPLE(F_Q8_0) }
     case LWQ_Q4_0: { LWQ_SIMPLE(F_Q4_0) }
     case LWQ_Q4_K: { LWQ_SIMPLE(F_Q4_K) }
+    case LWQ_Q6_K: { LWQ_SIMPLE(F_Q6_K) }
+    case LWQ_Q5_K: { LWQ_SIMPLE(F_Q5_K) }
+    case LWQ_Q2_K: { LWQ_SIMPLE(F_Q2_K) }
     }
 #undef LWQ_SIMPLE
     return cudaErrorInvalidValue;
@@ -389,7 +418,7 @@ MapReq map_req(const void *p, CUtensorMapDataType dtype, int rank, CUtensorMapSw
 // chunk), strides (row_bytes, chunk_bytes); a box of (all words, 16 rows, cps
 // chunks) lands as cps consecutive [16 rows][chunk bytes] boxes, one GEMV stage.
 int encode_weight_map(CUtensorMap *map, const void *Wq, int wf, int N, long rb, int cps) {
-    const int cb = (wf == LWQ_Q8_0) ? 272 : 144;
+    const int cb = gemv_chunk_bytes(wf);
     MapReq r = map_req(Wq, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, CU_TENSOR_MAP_SWIZZLE_NONE);
     r.dims[0] = (cuuint64_t)(cb / 8);
     r.dims[1] = (cuuint64_t)N;
@@ -477,6 +506,7 @@ int gemm_launch(int wf, int xt, const void *Wq, const void *x, float *y, int M, 
     switch (wf) {
     case LWQ_Q4_0: e = launch_gemm_xt<F_Q4_0>(xt, h, wm, xm, a, cfg.ctas, smem, st); break;
     case LWQ_Q8_0: e = launch_gemm_xt<F_Q8_0>(xt, h, wm, xm, a, cfg.ctas, smem, st); break;
+    case LWQ_Q5_K: e = launch_gemm_xt<F_Q5_K>(xt, h, wm, xm, a, cfg.ctas, smem, st); break;
     default: e = launch_gemm_xt<F_Q4_K>(xt, h, wm, xm, a, cfg.ctas, smem, st); break;
     }
     if (e != cudaSuccess) return LWQ_ERR_CUDA;

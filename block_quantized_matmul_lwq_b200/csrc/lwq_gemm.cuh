@@ -67,6 +67,8 @@ template <>
 struct GemmFmt<F_Q8_0> { static constexpr int chunk_bytes = 272; };
 template <>
 struct GemmFmt<F_Q4_K> { static constexpr int chunk_bytes = 144; };
+template <>
+struct GemmFmt<F_Q5_K> { static constexpr int chunk_bytes = 176; };
 
 __host__ __device__ constexpr size_t gemm_a_bytes() { return (size_t)GEMM_WROWS * 128; }
 __host__ __device__ constexpr size_t gemm_b_bytes(int bn) { return (size_t)bn * 128; }
@@ -246,6 +248,49 @@ struct Dequant<F_Q4_K, XT> {
             for (int i = 0; i < 8; ++i) {
                 const uint32_t byte = (qw[2 * c + (i >> 2)] >> (8 * (i & 3) + sh)) & 15u;
                 f[i] = fmaf(ds, __uint_as_float(0x4B000000u | byte) - 8388608.0f, -dm);
+            }
+            uint32_t o[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+                o[p] = (XT == X_F16) ? pack_f16x2(f[2 * p], f[2 * p + 1]) : pack_bf16x2(f[2 * p], f[2 * p + 1]);
+            st_shared_v4(a_base + sw128_chunk_offset(r, 4 * h + 2 * v + c), o[0], o[1], o[2], o[3]);
+        }
+    }
+};
+
+// Q5_K: as Q4_K, with the nibbles at 48 and a fifth bit per code: bit j of
+// qh[l] for element l of sub-block j's 32 (qh[32] at 16).
+template <int XT>
+struct Dequant<F_Q5_K, XT> {
+    static __device__ __forceinline__ void run(uint32_t prow, int kb, int h, int v, uint32_t a_base, int r) {
+        const uint4 hd = lds128(prow);
+        const uint4 qv = lds128(prow + 48 + 32 * kb + 16 * v);
+        const uint4 hv = lds128(prow + 16 + 16 * v);
+        const int j = 2 * kb + h;
+        const uint32_t s0 = hd.y, s1 = hd.z, s2 = hd.w;
+        uint32_t scw, mw;
+        if (j < 4) {
+            scw = s0 & 0x3F3F3F3Fu;
+            mw = s1 & 0x3F3F3F3Fu;
+        } else {
+            scw = (s2 & 0x0F0F0F0Fu) | ((s0 >> 2) & 0x30303030u);
+            mw = ((s2 >> 4) & 0x0F0F0F0Fu) | ((s1 >> 2) & 0x30303030u);
+        }
+        const int sc = (scw >> (8 * (j & 3))) & 63, m = (mw >> (8 * (j & 3))) & 63;
+        const float ds = f16_bits_to_float(hd.x) * (float)sc;           // exact in fp32
+        const float dm = f16_bits_to_float(hd.x >> 16) * (float)m;      // exact in fp32
+        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+        const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+        const uint32_t sh = 4u * h;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            float f[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t bsh = 8 * (i & 3);
+                const uint32_t q = ((qw[2 * c + (i >> 2)] >> (bsh + sh)) & 15u) |
+                                   (((hw[2 * c + (i >> 2)] >> (bsh + j)) & 1u) << 4);
+                f[i] = fmaf(ds, __uint_as_float(0x4B000000u | q) - 8388608.0f, -dm);
             }
             uint32_t o[4];
 #pragma unroll
@@ -535,12 +580,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 }
 
 // ---------------------------------------------------------------- host side
+// Formats with a tcgen05 GEMM decoder; their packed rows are 16-byte multiples.
+inline bool gemm_format(int wf) { return wf == LWQ_Q8_0 || wf == LWQ_Q4_0 || wf == LWQ_Q4_K || wf == LWQ_Q5_K; }
 inline bool gemm_eligible(int wf, int xt, long K) {
-    (void)wf;
-    return (xt == X_F16 || xt == X_BF16) && K % 256 == 0;
+    return gemm_format(wf) && (xt == X_F16 || xt == X_BF16) && K % 256 == 0;
 }
 
-inline int gemm_chunk_bytes(int wf) { return wf == LWQ_Q8_0 ? 272 : 144; }
+inline int gemm_chunk_bytes(int wf) { return wf == LWQ_Q8_0 ? 272 : (wf == LWQ_Q5_K ? 176 : 144); }
 
 // Ring depths.  128-row tiles: 4 dequantized A stages (made on chip, two per
 // batch), 3 packed chunk stages (each feeds four k-blocks; 2 when shared

@@ -48,7 +48,7 @@
 
 namespace lwq {
 
-enum { F_Q8_0 = 1, F_Q4_0 = 2, F_Q4_K = 3 };
+enum { F_Q8_0 = 1, F_Q4_0 = 2, F_Q4_K = 3, F_Q6_K = 4, F_Q5_K = 5, F_Q2_K = 6 };
 enum { X_F32 = 0, X_F16 = 1, X_BF16 = 2 };
 
 constexpr int GEMV_ROWS = 16;                     // weight rows per tile (the MMA's M)
@@ -66,6 +66,10 @@ template <>
 struct FmtInfo<F_Q4_0> { static constexpr int chunk_bytes = 144; };
 template <>
 struct FmtInfo<F_Q4_K> { static constexpr int chunk_bytes = 144; };
+template <>
+struct FmtInfo<F_Q5_K> { static constexpr int chunk_bytes = 176; };
+// formats with a per-sub-block min (the S_j sums of x enter the result)
+__host__ __device__ constexpr bool fmt_has_min(int fmt) { return fmt == F_Q4_K || fmt == F_Q5_K; }
 
 struct GemvArgs {
     const void *x;
@@ -166,6 +170,12 @@ __device__ __forceinline__ uint32_t q4k_hi(uint32_t w) {   // high nibbles, unsi
     if constexpr (BF) return hfma2_bf16(and_or(w >> 4, 0x000F000Fu, B2_MAGIC), B2_ONE, B2_M128);
     else return hfma2_f16(and_or(w, 0x00F000F0u, H2_MAGIC), H2_SIXTEENTH, H2_M64);
 }
+// Q5_K: the 5-bit codes of bytes 0 and 2, unsigned.
+template <bool BF>
+__device__ __forceinline__ uint32_t q5k_pair(uint32_t v) {
+    if constexpr (BF) return hfma2_bf16(and_or(v, 0x001F001Fu, B2_MAGIC), B2_ONE, B2_M128);
+    else return hfma2_f16(and_or(v, 0x001F001Fu, H2_MAGIC), H2_ONE, H2_M1024);
+}
 // Q8_0: the int8 codes of bytes 0 and 2.  fp16: (1024 + (q + 128)) - 1152.
 // bf16 has room for 7 bits only: (128 + (q & 127)) plus -128 or -256 from the
 // sign bit, which lands on the exponent bit of 0xC300 (0xC380 is -256).
@@ -223,7 +233,7 @@ __device__ __forceinline__ float byte_magic(uint32_t v, int jj) {
 //    the last two code bytes of the block in its place (one PRMT).
 template <int FMT>
 __device__ __forceinline__ int elem(int bb, int h, int t, int q) {
-    if (FMT == F_Q4_K || (bb & 1)) return 32 * bb + 16 * h + 4 * t + 2 * q;
+    if (FMT == F_Q4_K || FMT == F_Q5_K || FMT == F_Q6_K || (bb & 1)) return 32 * bb + 16 * h + 4 * t + 2 * q;
     if (FMT == F_Q4_0) return 32 * bb + 16 * h + ((4 * t - 2 + 2 * q) & 15);
     return 32 * bb + ((16 * h + 4 * t - 2 + 2 * q) & 31);
 }
@@ -370,7 +380,7 @@ struct Exact {
                     const bool ok = j * nthr + tid < nu;
                     const int mm = mk[j] >> 16, k = 4 * (mk[j] & 0xFFFF);
                     const float4 w = make_float4(v[j].x * sc, v[j].y * sc, v[j].z * sc, v[j].w * sc);
-                    if constexpr (FMT == F_Q4_K) store_sum((w.x + w.y) + (w.z + w.w), S, (long)mm * S.nk + k, ok, lane);
+                    if constexpr (fmt_has_min(FMT)) store_sum((w.x + w.y) + (w.z + w.w), S, (long)mm * S.nk + k, ok, lane);
                     if (ok) {
                         uint32_t pr[3][2];
                         split_pair(w.x, w.y, pr[0][0], pr[1][0], pr[2][0]);
@@ -401,7 +411,7 @@ struct Exact {
             }
         } else {
             if (!mbar_wait(xfull, 0, timeout, DEVERR_GEMV_WAIT)) return false;
-            if constexpr (XT == X_BF16 || FMT == F_Q4_K) {
+            if constexpr (XT == X_BF16 || fmt_has_min(FMT)) {
                 // 4-element units of plane 0 ([m][rs], nk / 4 units per row): the range check
                 // (bf16), a rescale in place when needed (rare), and the Q4_K sums
                 const int upr4 = S.nk / 4, nu4 = S.M * upr4;
@@ -425,7 +435,7 @@ struct Exact {
                         sc = pick_scale(cta_max(mx, S, nact, warp, lane), inv);
                     }
                 }
-                if (sc != 1.f || FMT == F_Q4_K) {
+                if (sc != 1.f || fmt_has_min(FMT)) {
                     for (int u0 = 0; u0 < nu4; u0 += nthr) {   // uniform trip count (shuffles inside)
                         const int u = u0 + tid;
                         const bool ok = u < nu4;
@@ -444,7 +454,7 @@ struct Exact {
                                     make_uint2(prmt(__float_as_uint(f[0]), __float_as_uint(f[1]), 0x7632u),
                                                prmt(__float_as_uint(f[2]), __float_as_uint(f[3]), 0x7632u));
                         }
-                        if constexpr (FMT == F_Q4_K) store_sum((f[0] + f[1]) + (f[2] + f[3]), S, (long)m * S.nk + k, ok, lane);
+                        if constexpr (fmt_has_min(FMT)) store_sum((f[0] + f[1]) + (f[2] + f[3]), S, (long)m * S.nk + k, ok, lane);
                     }
                     named_bar_sync(1, nthr);
                 }
@@ -555,7 +565,10 @@ struct Exact {
                 }
             }
         } else {
-            // Q4_K: header words d|dmin, scales s[0..3], s[4..7], s[8..11]
+            // Q4_K and Q5_K: header words d|dmin, scales s[0..3], s[4..7], s[8..11];
+            // Q5_K's fifth bits (qh[32]) follow at 16 and its nibbles at 48
+            constexpr bool K5 = FMT == F_Q5_K;
+            constexpr uint32_t QS = K5 ? 48u : 16u;
             const uint32_t h0 = lds32(r0), h1 = lds32(r1);
             const float d0 = f16_lo(h0), d1 = f16_lo(h1);
             const float nd0 = d0 * -8388608.f, nd1 = d1 * -8388608.f;   // -2^23 d (exact)
@@ -571,14 +584,23 @@ struct Exact {
                 sch0 = (s30 & 0x0F0F0F0Fu) | ((s10 >> 2) & 0x30303030u);
                 sch1 = (s31 & 0x0F0F0F0Fu) | ((s11 >> 2) & 0x30303030u);
             }
+            // Q5_K: qh bytes of elements 16h + 4t .. 16h + 4t + 3 of every group (bit 2g + nibble)
+            uint32_t hq0[2] = {0u, 0u}, hq1[2] = {0u, 0u};
+            if constexpr (K5) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    hq0[h] = lds32(r0 + 16 + 16 * h + 4 * t);
+                    hq1[h] = lds32(r1 + 16 + 16 * h + 4 * t);
+                }
+            }
 #pragma unroll
             for (int gq = 0; gq < NB / 2; ++gq) {
                 const int grp = half * (NB / 2) + gq;
                 uint32_t c0[2], c1[2];
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    c0[h] = lds32(r0 + 16 + 32 * grp + 16 * h + 4 * t);
-                    c1[h] = lds32(r1 + 16 + 32 * grp + 16 * h + 4 * t);
+                    c0[h] = lds32(r0 + QS + 32 * grp + 16 * h + 4 * t);
+                    c1[h] = lds32(r1 + QS + 32 * grp + 16 * h + 4 * t);
                 }
 #pragma unroll
                 for (int hi = 0; hi < 2; ++hi) {
@@ -586,7 +608,21 @@ struct Exact {
                     const uint32_t sv0 = (NB == 8 && b >= 4) ? sch0 : sc0, sv1 = (NB == 8 && b >= 4) ? sch1 : sc1;
                     const float s0 = fmaf(byte_magic(sv0, b & 3), d0, nd0);   // d * sc (exact)
                     const float s1 = fmaf(byte_magic(sv1, b & 3), d1, nd1);
-                    if (hi == 0) {
+                    if constexpr (K5) {
+                        // 5-bit codes, one per byte: nibble hi of the code byte | bit 2 grp + hi of qh << 4
+                        const int sh = 2 * grp + hi;
+                        uint32_t v0[2], v1[2];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            v0[h] = ((c0[h] >> (4 * hi)) & 0x0F0F0F0Fu) | (((hq0[h] >> sh) & 0x01010101u) << 4);
+                            v1[h] = ((c1[h] >> (4 * hi)) & 0x0F0F0F0Fu) | (((hq1[h] >> sh) & 0x01010101u) << 4);
+                        }
+                        const uint32_t a0[4] = {q5k_pair<BF>(v0[0]), q5k_pair<BF>(v1[0]), q5k_pair<BF>(v0[0] >> 8),
+                                                q5k_pair<BF>(v1[0] >> 8)};
+                        const uint32_t a1[4] = {q5k_pair<BF>(v0[1]), q5k_pair<BF>(v1[1]), q5k_pair<BF>(v0[1] >> 8),
+                                                q5k_pair<BF>(v1[1] >> 8)};
+                        block(a0, a1, b, s0, s1, acc);
+                    } else if (hi == 0) {
                         const uint32_t a0[4] = {q4k_lo<BF>(c0[0]), q4k_lo<BF>(c1[0]), q4k_lo<BF>(c0[0] >> 8),
                                                 q4k_lo<BF>(c1[0] >> 8)};
                         const uint32_t a1[4] = {q4k_lo<BF>(c0[1]), q4k_lo<BF>(c1[1]), q4k_lo<BF>(c0[1] >> 8),
@@ -836,7 +872,7 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1)
     constexpr int XE = (XT == X_F32) ? 4 : 2;
     // the reducer stages x raw with bulk copies, except fp32 x on the fp path (the compute warps split it)
     constexpr bool STAGE = I8 || XT != X_F32;
-    const GemvSmem L = gemv_smem_layout(CB, a.cps, ws, NT, FMT == F_Q4_K, P, a.M, XE, I8);
+    const GemvSmem L = gemv_smem_layout(CB, a.cps, ws, NT, fmt_has_min(FMT), P, a.M, XE, I8);
     uint8_t *ring = smem;
     uint8_t *xs = smem + L.ring;
     float *red = reinterpret_cast<float *>(xs + L.xs);

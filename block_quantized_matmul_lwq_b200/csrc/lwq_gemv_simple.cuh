@@ -1,5 +1,6 @@
 // Simple GEMV for the shapes the tensor-core paths do not take: K not a
-// multiple of 256 (only Q8_0 and Q4_0 allow that), at any M.  One warp per
+// multiple of 256 (only Q8_0 and Q4_0 allow that), and K-quant rows whose
+// byte stride is not a multiple of 16 (Q6_K, Q2_K), at any M.  One warp per
 // weight row; lanes stride over 32-weight units, decode them with byte loads
 // and accumulate in fp32 for up to 16 activation rows; a warp shuffle
 // reduction finishes each output.  Correct for every valid shape, not tuned.
@@ -37,6 +38,53 @@ __device__ __forceinline__ void decode_unit(const uint8_t *row, int u, float (&w
             const int v = b[2 + i];
             w[i] = d * (float)((v & 15) - 8);
             w[i + 16] = d * (float)((v >> 4) - 8);
+        }
+    } else if constexpr (FMT == F_Q6_K) {
+        // unit u: elements 32j .. 32j+31 of superblock u/8 (j = u%8 = 4n + g)
+        const uint8_t *b = row + (size_t)(u >> 3) * 210;
+        const int j = u & 7, n = j >> 2, g = j & 3;
+        const float d = f16_bits_to_float(ld_u16(b + 208));
+        const uint8_t *ql = b + 64 * n + 32 * (g & 1), *qh = b + 128 + 32 * n;
+        const int8_t *sc = reinterpret_cast<const int8_t *>(b + 192);
+        const float s0 = d * (float)sc[2 * j], s1 = d * (float)sc[2 * j + 1];   // exact in fp32
+#pragma unroll
+        for (int l = 0; l < 32; ++l) {
+            const int q = ((ql[l] >> (4 * (g >> 1))) & 15) | (((qh[l] >> (2 * g)) & 3) << 4);
+            w[l] = (l < 16 ? s0 : s1) * (float)(q - 32);                          // exact in fp32
+        }
+    } else if constexpr (FMT == F_Q5_K) {
+        const uint8_t *b = row + (size_t)(u >> 3) * 176;
+        const int j = u & 7, g = j >> 1, h = j & 1;   // sub-block j
+        const float d = f16_bits_to_float(ld_u16(b));
+        const float dmin = f16_bits_to_float(ld_u16(b + 2));
+        const uint8_t *s = b + 4;
+        int sc, m;
+        if (j < 4) {
+            sc = s[j] & 63;
+            m = s[j + 4] & 63;
+        } else {
+            sc = (s[j + 4] & 15) | ((s[j - 4] >> 6) << 4);
+            m = (s[j + 4] >> 4) | ((s[j] >> 6) << 4);
+        }
+        const float ds = d * (float)sc, dm = dmin * (float)m;  // both exact in fp32
+        const uint8_t *qh = b + 16, *qs = b + 48 + 32 * g;
+#pragma unroll
+        for (int l = 0; l < 32; ++l)
+            w[l] = fmaf(ds, (float)(((qs[l] >> (4 * h)) & 15) | (((qh[l] >> (2 * g + h)) & 1) << 4)), -dm);
+    } else if constexpr (FMT == F_Q2_K) {
+        // unit u: elements 32j .. 32j+31 of superblock u/8 (j = 4n + field)
+        const uint8_t *b = row + (size_t)(u >> 3) * 84;
+        const int j = u & 7, n = j >> 2, f = j & 3;
+        const float d = f16_bits_to_float(ld_u16(b + 80));
+        const float dmin = f16_bits_to_float(ld_u16(b + 82));
+        const uint8_t *qs = b + 16 + 32 * n;
+        const int s0 = b[2 * j], s1 = b[2 * j + 1];
+        const float ds0 = d * (float)(s0 & 15), dm0 = dmin * (float)(s0 >> 4);   // exact in fp32
+        const float ds1 = d * (float)(s1 & 15), dm1 = dmin * (float)(s1 >> 4);
+#pragma unroll
+        for (int l = 0; l < 32; ++l) {
+            const float q = (float)((qs[l] >> (2 * f)) & 3);
+            w[l] = l < 16 ? fmaf(ds0, q, -dm0) : fmaf(ds1, q, -dm1);
         }
     } else {
         const uint8_t *b = row + (size_t)(u >> 3) * 144;

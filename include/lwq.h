@@ -57,11 +57,30 @@ typedef enum {
  *           m_j = (s[j+4]>>4)|((s[j]>>6)<<4)), 128 bytes of nibbles in 4
  *           groups of 32 (group g: low nibbles are sub-block 2g, high
  *           nibbles sub-block 2g+1); w = d*sc_j*q - dmin*m_j.
+ * More K-quant formats of the same family ("Resumo Tecnico: Llamas na Web"
+ * names q4_k_m, which mixes Q4_K and Q6_K tensors, and q2_k, without their
+ * layouts; these are the llama.cpp layouts of those names):
+ * LWQ_Q6_K: 256 weights per 210-byte superblock: ql[128] (low 4 bits of the
+ *           6-bit codes), qh[64] (high 2 bits), int8 sc[16] (one scale per 16
+ *           weights), fp16 d.  Element 128n+32g+l (n<2, g<4, l<32) takes
+ *           nibble g>>1 of ql[64n+32(g&1)+l] and bits 2g, 2g+1 of qh[32n+l];
+ *           w = d*sc[e/16]*(q - 32).
+ * LWQ_Q5_K: 256 weights per 176-byte superblock: fp16 d, fp16 dmin, the 12
+ *           scale/min bytes of Q4_K, qh[32], qs[128].  Element 64g+32h+l
+ *           takes nibble h of qs[32g+l] and (as bit 4) bit 2g+h of qh[l];
+ *           w = d*sc_j*q - dmin*m_j, j = 2g+h.
+ * LWQ_Q2_K: 256 weights per 84-byte superblock: s[16] (per 16 weights: scale
+ *           in the low nibble, min in the high nibble), qs[64], fp16 d, fp16
+ *           dmin.  Element 128n+32j+l takes bits 2j, 2j+1 of qs[32n+l];
+ *           w = d*(s[e/16]&15)*q - dmin*(s[e/16]>>4).
  * Activations x: fp32, fp16 or bf16, row-major [M][K].
  */
 #define LWQ_Q8_0 1
 #define LWQ_Q4_0 2
 #define LWQ_Q4_K 3
+#define LWQ_Q6_K 4
+#define LWQ_Q5_K 5
+#define LWQ_Q2_K 6
 #define LWQ_FMT_MASK 0xFF
 #define LWQ_ACT_F32 0x000
 #define LWQ_ACT_F16 0x100
@@ -91,7 +110,8 @@ typedef enum {
  * LWQ_ERR_UNSUPPORTED.  Activations must be finite. */
 #define LWQ_FLAG_ACT_I8 0x2000
 
-/* Bytes of one packed row of K weights (K/32*34, K/32*18, K/256*144), or 0
+/* Bytes of one packed row of K weights (K/32*34, K/32*18, K/256*144,
+ * K/256*210, K/256*176, K/256*84), or 0
  * when fmt is unknown or K is not a positive multiple of the block size. */
 size_t lwq_row_bytes(int fmt, int64_t K);
 

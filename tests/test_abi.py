@@ -8,6 +8,7 @@ import re
 import pytest
 
 import block_quantized_matmul_lwq_b200 as lwq
+from block_quantized_matmul_lwq_b200 import inputs
 from block_quantized_matmul_lwq_b200 import build as lwq_build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -168,6 +169,19 @@ def test_gemm_tile_choices_are_valid():
                 assert cfg.tile_n in (128, 256)
                 assert 32 <= cfg.tile_m <= 256 and cfg.tile_m % 16 == 0
                 assert cfg.stages >= 2 and cfg.splits >= 1 and 1 <= cfg.ctas <= 148
+
+
+def test_more_kquant_formats_routing_and_row_bytes():
+    """Q5_K takes the tensor-core paths; Q6_K and Q2_K (rows not 16-byte multiples in general)
+    the simple kernel, at any M; row bytes follow the superblock sizes 176, 210 and 84."""
+    for M, path in ((1, 1), (16, 1), (17, 2), (512, 2)):
+        assert lwq.lwq_select_config(lwq.fmt_code("q5_k", "f16"), M, 4096, 4096).path == path
+    for w in ("q6_k", "q2_k"):
+        for M in (1, 16, 17, 512):
+            assert lwq.lwq_select_config(lwq.fmt_code(w, "f16"), M, 4096, 4096).path == 3
+    for w, K, rb in (("q6_k", 4096, 3360), ("q6_k", 11008, 9030), ("q5_k", 4096, 2816), ("q2_k", 11008, 3612)):
+        assert lwq.lwq_row_bytes(lwq.fmt_code(w, "f16"), K) == rb == inputs.row_bytes(w, K)
+    assert lwq.lwq_row_bytes(lwq.fmt_code("q6_k", "f16"), 288) == 0
 
 
 def test_int8_flag_plan():

@@ -1,0 +1,94 @@
+"""More K-quant formats (Q5_K, Q6_K, Q2_K) on the GPU against the oracle.
+
+Q5_K has tensor-core decoders (the GEMV and the tcgen05 GEMM); Q6_K and Q2_K
+rows are 210 and 84 bytes per superblock, so their rows are not 16-byte
+multiples in general and the simple kernel takes them.  Every case is scored
+element by element against the oracle on the same seeded inputs.
+"""
+
+import ctypes
+
+import pytest
+import torch
+
+import block_quantized_matmul_lwq_b200 as lwq
+from gpu_util import check_full, check_sampled
+
+pytestmark = pytest.mark.gpu
+
+WS_BYTES = 256 << 20
+ACTS = ("f32", "f16", "bf16")
+
+
+@pytest.fixture(scope="module")
+def dev():
+    d = torch.device("cuda:0")
+    torch.cuda.set_device(d)
+    ws = torch.zeros(WS_BYTES, dtype=torch.uint8, device=d)
+    lwq.lwq_init(ws, WS_BYTES)
+    yield d
+    torch.cuda.synchronize(d)
+    assert lwq.lwq_get_device_error() == lwq.LWQ_OK
+    lwq.lwq_shutdown()
+    del ws
+
+
+@pytest.mark.parametrize("w", ["q5_k", "q6_k", "q2_k"])
+@pytest.mark.parametrize("a", ACTS)
+@pytest.mark.parametrize("M,N,K", [(1, 1, 256), (1, 37, 512), (3, 100, 1024), (8, 333, 4096), (5, 61, 2816),
+                                   (16, 50, 768), (12, 130, 4352), (1, 17, 6144)])
+def test_small_shapes(dev, w, a, M, N, K):
+    check_full(w, a, M, N, K, dev, seed=M * 1000 + N + K)
+
+
+@pytest.mark.parametrize("a", ACTS)
+@pytest.mark.parametrize("M", [2, 3, 4, 5, 6, 7, 8, 9, 15, 16])
+def test_q5_k_every_column_layout(dev, a, M):
+    assert lwq.lwq_select_config(lwq.fmt_code("q5_k", a), M, 45, 1024).path == 1
+    check_full("q5_k", a, M, 45, 1024, dev, seed=200 + M)
+
+
+@pytest.mark.parametrize("w", ["q5_k", "q6_k", "q2_k"])
+def test_7b_layer_shapes(dev, w):
+    """The 7B layer's three projection shapes at M = 1 with fp16 activations, every output."""
+    for N, K in ((4096, 4096), (11008, 4096), (4096, 11008)):
+        check_full(w, "f16", 1, N, K, dev, seed=N + K)
+
+
+@pytest.mark.parametrize("w,a", [("q5_k", "bf16"), ("q5_k", "f16"), ("q6_k", "bf16"), ("q2_k", "f16")])
+@pytest.mark.parametrize("M,N,K", [(40, 300, 2048), (130, 1000, 1024), (300, 700, 1536)])
+def test_prefill_shapes(dev, w, a, M, N, K):
+    check_full(w, a, M, N, K, dev, seed=M + N)
+
+
+def test_q5_k_prefill_gemm_sampled(dev):
+    """Q5_K at the prefill shape (tcgen05 GEMM, 256-row tiles), sampled outputs."""
+    M, N, K = 512, 11008, 4096
+    cfg = lwq.lwq_select_config(lwq.fmt_code("q5_k", "bf16"), M, N, K)
+    assert cfg.path == 2
+    check_sampled("q5_k", "bf16", M, N, K, dev, seed=7, count=2000)
+
+
+@pytest.mark.parametrize("tile_n,bn,splits", [(128, 64, 0), (256, 96, 0), (256, 48, 3), (128, 176, 2)])
+def test_q5_k_forced_gemm_tiles(dev, tile_n, bn, splits):
+    cfg = lwq.lwq_config()
+    cfg.path, cfg.tile_n, cfg.tile_m, cfg.splits = 2, tile_n, bn, splits
+    check_full("q5_k", "f16", 150, 520, 3072, dev, seed=tile_n + bn, cfg=cfg)
+
+
+def test_q5_k_split_k_gemv(dev):
+    """Small N, long K: the GEMV splits K over CTAs and a follow-up kernel adds the partials."""
+    fmt = lwq.fmt_code("q5_k", "f32")
+    assert lwq.lwq_select_config(fmt, 4, 300, 11008).splits > 1
+    check_full("q5_k", "f32", 4, 300, 11008, dev, seed=5)
+
+
+def test_forced_path_without_decoder_is_refused(dev):
+    """Forcing the tensor-core GEMV on a format without its decoder returns LWQ_ERR_UNSUPPORTED."""
+    cfg = lwq.lwq_config()
+    cfg.path = 1
+    buf = torch.zeros(64, dtype=torch.float32, device="cuda:0")
+    p = buf.data_ptr()
+    rc = lwq.lib().lwq_matmul_config(lwq.fmt_code("q6_k", "f16"), p, p, p, 1, 16, 256, ctypes.byref(cfg), None)
+    assert rc == lwq.LWQ_ERR_UNSUPPORTED
+
