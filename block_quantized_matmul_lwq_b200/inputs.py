@@ -256,6 +256,23 @@ def make_problem(fmt: str, act: str, M: int, N: int, K: int, seed: int = 0):
     return Wq, x
 
 
+def attention_problem(B: int, H: int, Hkv: int, Lmax: int, D: int, act: str, seed: int = 0, lens=None):
+    """Decode-attention inputs from one seeded stream: q [B][H][D], then the key cache and the
+    value cache [B][Hkv][Lmax][D], all ~ N(0, 1) drawn in fp32 and stored in ``act`` (fp16, or
+    bf16 codes).  Sequence lengths: ``lens`` as given, else Lmax for every sequence."""
+    g = rng(seed)
+
+    def draw(shape):
+        a = g.standard_normal(shape, dtype=np.float32)
+        return np.ascontiguousarray(a.astype(np.float16)) if act == "f16" else f32_to_bf16_bits(a)
+
+    q = draw((B, H, D))
+    k = draw((B, Hkv, Lmax, D))
+    v = draw((B, Hkv, Lmax, D))
+    lens = np.full(B, Lmax, dtype=np.int32) if lens is None else np.asarray(lens, dtype=np.int32)
+    return q, k, v, lens
+
+
 # The workloads, by what they are (format, activation dtype, shapes, seed).
 WORKLOADS = {
     "q8_0_gemv_4096x4096": dict(fmt="q8_0", act="f32", Ms=[1], shapes=[(4096, 4096)], seeds=[0]),

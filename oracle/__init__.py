@@ -59,6 +59,9 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.lwq_oracle_matmul_sampled.argtypes = [c.c_int, c.c_int, c.c_void_p, c.c_void_p, c.c_long,
                                               c.c_long, c.c_long, c.c_void_p, c.c_void_p, c.c_long,
                                               c.c_void_p, c.c_void_p, c.c_int]
+    lib.lwq_oracle_attention.restype = c.c_int
+    lib.lwq_oracle_attention.argtypes = [c.c_int, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_long, c.c_long,
+                                         c.c_long, c.c_long, c.c_long, c.c_double, c.c_void_p, c.c_void_p]
     lib.lwq_oracle_max_threads.restype = c.c_int
     lib.lwq_oracle_max_threads.argtypes = []
     return lib
@@ -218,6 +221,27 @@ def matmul_q8act(fmt: str, Wq: np.ndarray, x: np.ndarray, K: int | None = None, 
     xq = q.astype(np.float64) * np.repeat(d.astype(np.float64), ACT_Q8_BLOCK, axis=1)
     W = dequant(fmt, Wq, K, lib=lib).astype(np.float64)
     return xq @ W.T, np.abs(xq) @ np.abs(W).T
+
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, lens, scale: float, act: str | None = None, lib=None):
+    """Decode attention (see ``lwq_oracle_attention``): q [B][H][D], k/v [B][Hkv][Lmax][D] as fp16
+    arrays or bf16 codes (uint16), lens [B].  Returns (out, den), fp64 [B][H][D]."""
+    lib = lib or load()
+    if act is None:
+        act = "f16" if q.dtype == np.float16 else "bf16"
+    B, H, D = q.shape
+    Hkv, Lmax = k.shape[1], k.shape[2]
+    lens = np.ascontiguousarray(np.asarray(lens, dtype=np.int32))
+    q16 = np.ascontiguousarray(q).view(np.uint16)
+    k16 = np.ascontiguousarray(k).view(np.uint16)
+    v16 = np.ascontiguousarray(v).view(np.uint16)
+    out = np.empty((B, H, D), dtype=np.float64)
+    den = np.empty((B, H, D), dtype=np.float64)
+    rc = lib.lwq_oracle_attention(ACT[act], _ptr(q16), _ptr(k16), _ptr(v16), _ptr(lens), B, H, Hkv, Lmax, D,
+                                  float(scale), _ptr(out), _ptr(den))
+    if rc:
+        raise ValueError("bad attention arguments")
+    return out, den
 
 
 def max_threads(lib=None) -> int:

@@ -364,3 +364,75 @@ int lwq_oracle_max_threads(void) {
     return 1;
 #endif
 }
+
+/*
+ * Decode attention (one query per sequence and head) -- the plain definition
+ * behind "Compute Shaders con WebGPU para Inferencia ML", "El Mecanismo de
+ * Atencion": scores s_j = scale * (q . k_j), weights p_j = softmax(s)_j,
+ * out = sum_j p_j v_j.  The page fuses the softmax into the pass over the keys
+ * with a running maximum (online softmax); that reaches this same result up to
+ * rounding, so the oracle is the definition written out, in fp64:
+ *
+ *   m = max_j s_j;  p_j = exp(s_j - m);  out[d] = (sum_j p_j v_j[d]) / (sum_j p_j)
+ *   den[d] = (sum_j p_j |v_j[d]|) / (sum_j p_j)      (the error scale)
+ *
+ * Layouts (16-bit codes of dtype act: OR_ACT_F16 or OR_ACT_BF16):
+ *   q   [B][H][D]
+ *   k,v [B][Hkv][Lmax][D]   (key j of sequence b and kv head g at [b][g][j])
+ *   out, den [B][H][D] fp64
+ * Query head h reads kv head h / (H / Hkv).  Sequence b has len[b] keys
+ * (1 <= len[b] <= Lmax).  Returns 0, or -1 on bad arguments.
+ */
+int lwq_oracle_attention(int act, const uint16_t *q, const uint16_t *k, const uint16_t *v, const int *len,
+                         long B, long H, long Hkv, long Lmax, long D, double scale, double *out, double *den) {
+    if ((act != OR_ACT_F16 && act != OR_ACT_BF16) || B <= 0 || H <= 0 || Hkv <= 0 || H % Hkv || Lmax <= 0 ||
+        D <= 0)
+        return -1;
+    for (long b = 0; b < B; b++)
+        if (len[b] < 1 || len[b] > Lmax) return -1;
+    long G = H / Hkv;
+    int fail = 0;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static) reduction(| : fail)
+#endif
+    for (long bh = 0; bh < B * H; bh++) {
+        long b = bh / H, h = bh % H, g = h / G;
+        long n = len[b];
+        double *s = (double *)malloc(sizeof(double) * (size_t)n);
+        if (!s) {
+            fail = 1;
+            continue;
+        }
+        const uint16_t *qh = q + (b * H + h) * D;
+        const uint16_t *kb = k + (b * Hkv + g) * Lmax * D;
+        const uint16_t *vb = v + (b * Hkv + g) * Lmax * D;
+        double m = -INFINITY;
+        for (long j = 0; j < n; j++) {
+            double dot = 0.0;
+            for (long d = 0; d < D; d++) {
+                double qd = act == OR_ACT_F16 ? lwq_oracle_f16(qh[d]) : lwq_oracle_bf16(qh[d]);
+                double kd = act == OR_ACT_F16 ? lwq_oracle_f16(kb[j * D + d]) : lwq_oracle_bf16(kb[j * D + d]);
+                dot += qd * kd;
+            }
+            s[j] = scale * dot;
+            if (s[j] > m) m = s[j];
+        }
+        double sum = 0.0;
+        for (long j = 0; j < n; j++) {
+            s[j] = exp(s[j] - m);
+            sum += s[j];
+        }
+        for (long d = 0; d < D; d++) {
+            double acc = 0.0, acc_abs = 0.0;
+            for (long j = 0; j < n; j++) {
+                double vd = act == OR_ACT_F16 ? lwq_oracle_f16(vb[j * D + d]) : lwq_oracle_bf16(vb[j * D + d]);
+                acc += s[j] * vd;
+                acc_abs += s[j] * fabs(vd);
+            }
+            out[(b * H + h) * D + d] = acc / sum;
+            if (den) den[(b * H + h) * D + d] = acc_abs / sum;
+        }
+        free(s);
+    }
+    return fail ? -1 : 0;
+}

@@ -12,6 +12,8 @@ from __future__ import annotations
 
 import os
 
+import math
+
 import numpy as np
 import torch
 
@@ -362,6 +364,104 @@ def pin_row_bytes(lib):
     assert lib.lwq_oracle_row_bytes(oracle.FMT["q6_k"], 288) == -1
 
 
+# ------------------------------------------------------ decode attention pins
+
+def _f16(a):
+    return np.asarray(a, dtype=np.float16)
+
+
+def pin_attn_one_key(lib):
+    """One key: its softmax weight is 1, so out is that key's value row exactly (den its |row|)."""
+    q, k, v, _ = inputs.attention_problem(2, 4, 2, 5, 16, "f16", seed=1)
+    out, den = oracle.attention(q, k, v, [1, 1], 0.25, lib=lib)
+    for b in range(2):
+        for h in range(4):
+            np.testing.assert_array_equal(out[b, h], v[b, h // 2, 0].astype(np.float64))
+            np.testing.assert_array_equal(den[b, h], np.abs(v[b, h // 2, 0].astype(np.float64)))
+
+
+def pin_attn_zero_query_is_mean(lib):
+    """q = 0 makes every score 0: out is the plain mean of the value rows of the sequence."""
+    q, k, v, _ = inputs.attention_problem(1, 2, 1, 9, 8, "f16", seed=2)
+    q[:] = 0
+    out, _ = oracle.attention(q, k, v, [7], 0.3, lib=lib)
+    ref = v[0, 0, :7].astype(np.float64).mean(axis=0)
+    assert np.allclose(out[0, 0], ref, rtol=0, atol=1e-15)
+
+
+def pin_attn_two_keys(lib):
+    """Scores 0 and s: out = (v0 + e^s v1) / (1 + e^s)."""
+    D = 4
+    q = np.zeros((1, 1, D), dtype=np.float16)
+    q[0, 0, 0] = 1.0
+    k = np.zeros((1, 1, 2, D), dtype=np.float16)
+    k[0, 0, 1, 0] = 1.0986328125          # an fp16 value near ln 3
+    v = _f16([[[[1, 2, -3, 0.5], [5, -6, 7, 0.25]]]])
+    out, _ = oracle.attention(q, k, v, [2], 1.0, lib=lib)
+    r = math.exp(1.0986328125)
+    ref = (v[0, 0, 0].astype(np.float64) + r * v[0, 0, 1].astype(np.float64)) / (1 + r)
+    assert np.allclose(out[0, 0], ref, rtol=1e-15, atol=0)
+
+
+def pin_attn_dominant_key(lib):
+    """A score 1000 above every other one takes all the weight (exp(-1000) is 0 in fp64), and
+    the maximum is subtracted first (exp(1000) would overflow)."""
+    q, k, v, _ = inputs.attention_problem(1, 1, 1, 6, 8, "f16", seed=3)
+    q[:] = 0
+    q[0, 0, 0] = 1.0
+    k[0, 0, :, 0] = 0
+    k[0, 0, 4, 0] = 1000.0
+    out, _ = oracle.attention(q, k, v, [6], 1.0, lib=lib)
+    np.testing.assert_array_equal(out[0, 0], v[0, 0, 4].astype(np.float64))
+
+
+def pin_attn_gqa_heads(lib):
+    """Query head h reads kv head h / (H / Hkv): value rows all 2^g in kv head g give out = 2^g."""
+    q, k, v, _ = inputs.attention_problem(2, 6, 3, 5, 8, "bf16", seed=4)
+    for g in range(3):
+        v[:, g] = inputs.f32_to_bf16_bits(np.full((2, 5, 8), 2.0 ** g, dtype=np.float32))
+    out, _ = oracle.attention(q, k, v, [5, 3], 0.5, act="bf16", lib=lib)
+    for h in range(6):
+        assert np.all(out[:, h] == 2.0 ** (h // 2)), h
+
+
+def pin_attn_linear_in_v(lib):
+    """out is linear in the value rows (small halves: the sums of two caches are exact in fp16)."""
+    g = np.random.default_rng(5)
+    q, k, _, _ = inputs.attention_problem(1, 2, 2, 11, 8, "f16", seed=5)
+    v1 = _f16(g.integers(-8, 9, size=(1, 2, 11, 8)) / 2)
+    v2 = _f16(g.integers(-8, 9, size=(1, 2, 11, 8)) / 2)
+    o1, _ = oracle.attention(q, k, v1, [11], 0.35, lib=lib)
+    o2, _ = oracle.attention(q, k, v2, [11], 0.35, lib=lib)
+    o12, _ = oracle.attention(q, k, _f16(v1.astype(np.float32) + v2.astype(np.float32)), [11], 0.35, lib=lib)
+    assert np.allclose(o12, o1 + o2, rtol=0, atol=1e-13)
+
+
+def pin_attn_length_respected(lib):
+    """Keys past a sequence's length change nothing."""
+    q, k, v, _ = inputs.attention_problem(2, 2, 2, 12, 8, "f16", seed=6)
+    out, _ = oracle.attention(q, k, v, [5, 12], 0.4, lib=lib)
+    k2, v2 = k.copy(), v.copy()
+    k2[0, :, 5:] = 60000.0
+    v2[0, :, 5:] = -60000.0
+    out2, _ = oracle.attention(q, k2, v2, [5, 12], 0.4, lib=lib)
+    np.testing.assert_array_equal(out, out2)
+
+
+def pin_attn_logsumexp_bruteforce(lib):
+    """Tiny case against Python floats in the log-sum-exp form: out = sum_j exp(s_j - lse) v_j."""
+    q, k, v, _ = inputs.attention_problem(1, 2, 1, 3, 4, "f16", seed=7)
+    scale = 0.7
+    out, _ = oracle.attention(q, k, v, [3], scale, lib=lib)
+    for h in range(2):
+        s = [scale * sum(float(q[0, h, d]) * float(k[0, 0, j, d]) for d in range(4)) for j in range(3)]
+        lse = math.log(sum(math.exp(x) for x in s))
+        ref = [sum(math.exp(s[j] - lse) * float(v[0, 0, j, d]) for j in range(3)) for d in range(4)]
+        assert np.allclose(out[0, h], ref, rtol=1e-13, atol=1e-15)
+
+
 ALL_PINS = [pin_hand_blocks, pin_f16_exhaustive, pin_bf16_exhaustive, pin_q4k_scale_roundtrip,
             pin_roundtrip_q8_0, pin_roundtrip_q4_0, pin_bruteforce_one_block, pin_library_matmul,
-            pin_linearity, pin_zero_denominator, pin_sampled_equals_full, pin_row_bytes]
+            pin_linearity, pin_zero_denominator, pin_sampled_equals_full, pin_row_bytes,
+            pin_attn_one_key, pin_attn_zero_query_is_mean, pin_attn_two_keys, pin_attn_dominant_key,
+            pin_attn_gqa_heads, pin_attn_linear_in_v, pin_attn_length_respected, pin_attn_logsumexp_bruteforce]

@@ -44,6 +44,14 @@ MUTANTS = {
     "q2_k_field_shift": ("int q = (qs[32 * n + l] >> (2 * j)) & 3;", "int q = (qs[32 * n + l] >> j) & 3;"),
     "q2_k_d_is_dmin": ("double d = lwq_oracle_f16(rd16(b + 80));", "double d = lwq_oracle_f16(rd16(b + 82));"),
     "q2_k_half_stride": ("int q = (qs[32 * n + l] >> (2 * j)) & 3;", "int q = (qs[16 * n + l] >> (2 * j)) & 3;"),
+    "attn_no_scale": ("s[j] = scale * dot;", "s[j] = dot;"),
+    "attn_no_max": ("s[j] = exp(s[j] - m);", "s[j] = exp(s[j]);"),
+    "attn_gqa_modulo": ("long b = bh / H, h = bh % H, g = h / G;", "long b = bh / H, h = bh % H, g = h % Hkv;"),
+    "attn_values_are_keys": ("const uint16_t *vb = v + (b * Hkv + g) * Lmax * D;",
+                             "const uint16_t *vb = k + (b * Hkv + g) * Lmax * D;"),
+    "attn_mean_not_softmax": ("out[(b * H + h) * D + d] = acc / sum;", "out[(b * H + h) * D + d] = acc / (double)n;"),
+    "attn_ignores_len": ("long n = len[b];", "long n = Lmax;"),
+    "attn_den_no_abs": ("acc_abs += s[j] * fabs(vd);", "acc_abs += s[j] * vd;"),
     "f16_bias": ("v = ldexp((double)(1024 + f), e - 25);", "v = ldexp((double)(1024 + f), e - 24);"),
     "f16_subnormal": ("v = ldexp((double)f, -24);", "v = ldexp((double)(1024 + f), -24);"),
     "bf16_bias": ("v = ldexp((double)(128 + f), e - 134);", "v = ldexp((double)(128 + f), e - 133);"),
