@@ -40,7 +40,8 @@ ACT_DTYPES = {"f32": LWQ_ACT_F32, "f16": LWQ_ACT_F16, "bf16": LWQ_ACT_BF16}
 # every symbol the header declares
 EXPORTS = ["lwq_row_bytes", "lwq_workspace_size", "lwq_init", "lwq_shutdown", "lwq_matmul",
            "lwq_select_config", "lwq_matmul_config", "lwq_status_string", "lwq_get_device_error",
-           "lwq_selftest_timeout", "lwq_last_launch_count", "lwq_version", "lwq_matmul_noalloc"]
+           "lwq_selftest_timeout", "lwq_last_launch_count", "lwq_version", "lwq_matmul_noalloc",
+           "lwq_attention_workspace_size", "lwq_attention_decode"]
 
 
 class LwqError(RuntimeError):
@@ -80,6 +81,10 @@ def _load() -> ctypes.CDLL:
     lib.lwq_last_launch_count.restype, lib.lwq_last_launch_count.argtypes = i, []
     lib.lwq_version.restype, lib.lwq_version.argtypes = i, []
     lib.lwq_matmul_noalloc.restype, lib.lwq_matmul_noalloc.argtypes = i, [i, vp, vp, vp, i, i, i, vp]
+    lib.lwq_attention_workspace_size.restype = c.c_size_t
+    lib.lwq_attention_workspace_size.argtypes = [i, i, i, i, i]
+    lib.lwq_attention_decode.restype = i
+    lib.lwq_attention_decode.argtypes = [i, vp, vp, vp, vp, vp, i, i, i, i, i, c.c_float, vp]
     return lib
 
 
@@ -184,3 +189,14 @@ def lwq_matmul_noalloc(fmt: int, Wq, x, y, M: int, N: int, K: int, stream=None) 
     """lwq_matmul for callers that cannot allocate: no workspace, static 4 MiB scratch (see include/lwq.h)."""
     _check(_lib.lwq_matmul_noalloc(fmt, _ptr(Wq), _ptr(x), _ptr(y), M, N, K, _stream(stream)),
            "lwq_matmul_noalloc")
+
+
+def lwq_attention_workspace_size(B: int, H: int, Hkv: int, Lmax: int, D: int) -> int:
+    return _lib.lwq_attention_workspace_size(B, H, Hkv, Lmax, D)
+
+
+def lwq_attention_decode(act: int, q, k, v, seq_lens, out, B: int, H: int, Hkv: int, Lmax: int, D: int,
+                         scale: float, stream=None) -> None:
+    """Decode attention through the C ABI (act: LWQ_ACT_F16 or LWQ_ACT_BF16; seq_lens may be None)."""
+    _check(_lib.lwq_attention_decode(act, _ptr(q), _ptr(k), _ptr(v), _ptr(seq_lens), _ptr(out), B, H, Hkv, Lmax, D,
+                                     float(scale), _stream(stream)), "lwq_attention_decode")

@@ -18,6 +18,7 @@
 #include "lwq_gemm.cuh"
 #include "lwq_gemv.cuh"
 #include "lwq_gemv_simple.cuh"
+#include "lwq_attn.cuh"
 
 namespace lwq {
 namespace {
@@ -625,6 +626,40 @@ int run(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, c
     return LWQ_OK;
 }
 
+// ------------------------------------------------------- decode attention
+template <int XT, int D, int G>
+cudaError_t launch_attn(const AttnArgs &a, cudaStream_t st) {
+    attn_split_kernel<XT, D, G><<<dim3((unsigned)a.S, (unsigned)a.Hkv, (unsigned)a.B), ATTN_WARPS * 32, 0, st>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || a.S == 1) return e;
+    // the splits' merge: a programmatic dependent launch that waits for the split kernel
+    return launch_k(attn_combine_kernel<D>, a.B * a.H, D, 0, st, true, (const float *)a.part, a.out, a.S);
+}
+
+template <int XT, int D>
+cudaError_t launch_attn_g(int G, const AttnArgs &a, cudaStream_t st) {
+    switch (G) {
+    case 1: return launch_attn<XT, D, 1>(a, st);
+    case 2: return launch_attn<XT, D, 2>(a, st);
+    case 4: return launch_attn<XT, D, 4>(a, st);
+    case 8: return launch_attn<XT, D, 8>(a, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+size_t attn_ws_bytes(int B, int H, int S, int D) { return S > 1 ? (size_t)B * H * S * (D + 2) * 4 : 0; }
+
+int attn_check(int dtype, int B, int H, int Hkv, int Lmax, int D) {
+    if (B <= 0 || H <= 0 || Hkv <= 0 || Lmax <= 0 || D <= 0) return LWQ_ERR_INVALID_ARG;
+    if (dtype != LWQ_ACT_F16 && dtype != LWQ_ACT_BF16) return LWQ_ERR_UNSUPPORTED;
+    if (D != 64 && D != 128) return LWQ_ERR_UNSUPPORTED;
+    if (H % Hkv) return LWQ_ERR_INVALID_ARG;
+    const int G = H / Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return LWQ_ERR_UNSUPPORTED;
+    if (B > 65535 || Hkv > 65535) return LWQ_ERR_UNSUPPORTED;
+    return LWQ_OK;
+}
+
 __global__ void selftest_timeout_kernel(unsigned long long timeout_ns) {
     __shared__ uint64_t bar;
     if (threadIdx.x == 0) {
@@ -756,6 +791,59 @@ int lwq_selftest_timeout(unsigned timeout_us, void *stream) {
 }
 
 int lwq_last_launch_count(void) { return t_last_launches; }
+
+size_t lwq_attention_workspace_size(int B, int H, int Hkv, int Lmax, int D) {
+    if (attn_check(LWQ_ACT_F16, B, H, Hkv, Lmax, D)) return 0;
+    int dev = 0, sms = 148;
+    if (current_device(&dev) == LWQ_OK) sms = sm_count(dev);
+    int S = 1, chunk = 0;
+    attn_splits(B, Hkv, Lmax, sms, &S, &chunk);
+    return attn_ws_bytes(B, H, S, D);
+}
+
+int lwq_attention_decode(int dtype, const void *q, const void *k, const void *v, const int32_t *seq_lens, float *out,
+                         int B, int H, int Hkv, int Lmax, int D, float scale, void *stream) {
+    t_last_launches = 0;
+    if (!q || !k || !v || !out) return LWQ_ERR_INVALID_ARG;
+    int rc = attn_check(dtype, B, H, Hkv, Lmax, D);
+    if (rc) return rc;
+    if (!isfinite(scale)) return LWQ_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+        return LWQ_ERR_MISALIGNED;
+    int dev;
+    if ((rc = current_device(&dev))) return rc;
+    AttnArgs a;
+    a.q = static_cast<const uint16_t *>(q);
+    a.k = static_cast<const uint16_t *>(k);
+    a.v = static_cast<const uint16_t *>(v);
+    a.lens = seq_lens;
+    a.out = out;
+    a.B = B;
+    a.H = H;
+    a.Hkv = Hkv;
+    a.Lmax = Lmax;
+    a.qscale = scale * 1.4426950408889634f;   // log2(e): the kernels take exponentials as exp2
+    attn_splits(B, Hkv, Lmax, sm_count(dev), &a.S, &a.chunk);
+    DeviceState &ds = g_dev[dev];
+    a.part = nullptr;
+    const size_t need = attn_ws_bytes(B, H, a.S, D);
+    if (need > 0) {
+        if (!ds.registered) return LWQ_ERR_NOT_INITIALIZED;
+        if (ds.ws_bytes < need) return LWQ_ERR_WORKSPACE_TOO_SMALL;
+        a.part = static_cast<float *>(ds.ws);
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int G = H / Hkv;
+    cudaError_t e;
+    if (dtype == LWQ_ACT_F16)
+        e = D == 64 ? launch_attn_g<X_F16, 64>(G, a, st) : launch_attn_g<X_F16, 128>(G, a, st);
+    else
+        e = D == 64 ? launch_attn_g<X_BF16, 64>(G, a, st) : launch_attn_g<X_BF16, 128>(G, a, st);
+    if (e != cudaSuccess) return LWQ_ERR_CUDA;
+    t_last_launches = a.S > 1 ? 2 : 1;
+    return LWQ_OK;
+}
 
 int lwq_version(void) { return 0x000100; }
 

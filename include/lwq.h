@@ -204,6 +204,32 @@ int lwq_select_config(int fmt, int M, int N, int K, lwq_config *cfg);
 int lwq_matmul_config(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K,
                       const lwq_config *cfg, void *stream);
 
+/* ------------------------------------------------------ decode attention
+ * One query token per sequence and head against that sequence's key/value
+ * cache, the softmax fused into the one pass over the keys ("Compute Shaders
+ * con WebGPU para Inferencia ML", "El Mecanismo de Atencion": scores
+ * q.k / sqrt(head_dim), a running maximum and sum, the weighted values
+ * accumulated in the same pass):
+ *   s_j = scale * (q . k_j),  out = sum_{j < len} softmax(s)_j v_j.
+ * dtype: LWQ_ACT_F16 or LWQ_ACT_BF16, the type of q, k and v.
+ * q [B][H][D]; k, v [B][Hkv][Lmax][D] (the caches, key j of sequence b and kv
+ * head g at [b][g][j]); out [B][H][D] fp32; all row-major device arrays,
+ * 16-byte aligned.  Query head h reads kv head h / (H / Hkv); H / Hkv must be
+ * 1, 2, 4 or 8, and D 64 or 128.  seq_lens: device array of B int32 lengths
+ * (a length outside [1, Lmax] is clamped into it), or NULL for Lmax each.
+ * scale: usually 1 / sqrt(D).  Long sequences are split over several CTAs
+ * whose partial results a second kernel merges; the partials live in the
+ * workspace registered with lwq_init (the static arena that "Llamas na Web",
+ * "Alocacao Estatica de Memoria", sizes at start-up for FlashAttention-style
+ * scratch), lwq_attention_workspace_size bytes.  Errors: LWQ_ERR_INVALID_ARG
+ * (a size <= 0, H not a multiple of Hkv, NULL q/k/v/out, non-finite scale),
+ * LWQ_ERR_UNSUPPORTED (dtype, D, H / Hkv), LWQ_ERR_MISALIGNED,
+ * LWQ_ERR_NOT_INITIALIZED / LWQ_ERR_WORKSPACE_TOO_SMALL (split partials),
+ * LWQ_ERR_CUDA.  The library allocates nothing and does not synchronize. */
+size_t lwq_attention_workspace_size(int B, int H, int Hkv, int Lmax, int D);
+int lwq_attention_decode(int dtype, const void *q, const void *k, const void *v, const int32_t *seq_lens, float *out,
+                         int B, int H, int Hkv, int Lmax, int D, float scale, void *stream);
+
 /* ------------------------------------------------ errors and diagnostics */
 
 /* Static description of a status code. */
