@@ -81,6 +81,40 @@ __device__ __forceinline__ void transpose_reduce(float (&val)[V], int lane) {
     for (int bit = 16 >> K; bit > 0; bit >>= 1) val[0] += __shfl_xor_sync(0xffffffffu, val[0], bit);
 }
 
+// Asynchronous global -> shared copies of 4 or 8 bytes (cp.async), grouped;
+// a thread reads back only what it copied itself, after waiting for its group.
+template <int BYTES>
+__device__ __forceinline__ void cp_async(uint32_t dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(dst), "l"(src), "n"(BYTES) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// E 16-bit elements of a row, already in shared memory, as fp32.
+template <int XT, int E>
+__device__ __forceinline__ void smem_row(uint32_t addr, float (&f)[E]) {
+    uint32_t w[E / 2];
+    if constexpr (E == 4) {
+        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(addr));
+    } else {
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w[0]) : "r"(addr));
+    }
+#pragma unroll
+    for (int i = 0; i < E / 2; ++i) {
+        if constexpr (XT == X_F16) {
+            const float2 v = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
+            f[2 * i] = v.x;
+            f[2 * i + 1] = v.y;
+        } else {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
+}
+
+constexpr int ATTN_RING = 4;   // steps of K and V rows in flight per warp (shared-memory ring)
+
 struct AttnArgs {
     const uint16_t *q, *k, *v;
     const int *lens;     // [B] or null (every sequence Lmax long)
@@ -118,13 +152,59 @@ __global__ void __launch_bounds__(ATTN_WARPS * 32) attn_split_kernel(const AttnA
     const uint16_t *kb = a.k + ((size_t)b * a.Hkv + g) * (size_t)a.Lmax * D + E * lane;
     const uint16_t *vb = a.v + ((size_t)b * a.Hkv + g) * (size_t)a.Lmax * D + E * lane;
 
-    for (int jg = j0 + ATTN_U * warp; jg < j1; jg += ATTN_U * ATTN_WARPS) {
-        float kf[ATTN_U][E], vf[ATTN_U][E];
+    // Each warp streams its steps (4 keys' K and V rows) through a ring of
+    // ATTN_RING shared-memory stages with cp.async: several steps are in flight
+    // without holding registers.  Lane i copies, and later reads, bytes
+    // [2E i, 2E i + 2E) of each row.  Stage layout: [key u][K, V][lane][E].
+    constexpr int STRIDE = ATTN_U * ATTN_WARPS;
+    constexpr uint32_t ROWB = 2 * D, STAGEB = ATTN_U * 2 * ROWB;
+    // the ring, later reused for the warps' merge
+    // one query head per kv head (G = 1): the direct loads keep HBM busy without the ring (measured
+    // 0.98 of peak against 0.81 with it); with G > 1 the per-step math is longer and the ring's
+    // deeper stream pays
+    constexpr bool RING = G > 1;
+    constexpr uint32_t RINGB = RING ? ATTN_WARPS * ATTN_RING * STAGEB : 0;
+    constexpr uint32_t MERGEB = (2 * ATTN_WARPS * G + ATTN_WARPS * G * D) * 4;
+    __shared__ __align__(16) uint8_t smraw[RINGB > MERGEB ? RINGB : MERGEB];
+    const uint32_t ring0 = (uint32_t)__cvta_generic_to_shared(smraw) + (uint32_t)warp * ATTN_RING * STAGEB + 2 * E * lane;
+    const int jfirst = j0 + ATTN_U * warp;
+    const int nsteps = jfirst < j1 ? (j1 - jfirst + STRIDE - 1) / STRIDE : 0;
+    auto issue = [&](int i) {   // step i of this warp into stage i % ATTN_RING (an empty group past the end)
+        if (i < nsteps) {
+            const uint32_t st = ring0 + (uint32_t)(i % ATTN_RING) * STAGEB;
+            const int jg = jfirst + i * STRIDE;
 #pragma unroll
-        for (int u = 0; u < ATTN_U; ++u) {
-            const int j = min(jg + u, j1 - 1);   // a key past the split reloads the last one (masked below)
-            load_row<XT, E>(kb + (size_t)j * D, kf[u]);
-            load_row<XT, E>(vb + (size_t)j * D, vf[u]);
+            for (int u = 0; u < ATTN_U; ++u) {
+                const int j = min(jg + u, j1 - 1);   // a key past the split reloads the last one (masked below)
+                cp_async<2 * E>(st + (2 * u) * ROWB, kb + (size_t)j * D);
+                cp_async<2 * E>(st + (2 * u + 1) * ROWB, vb + (size_t)j * D);
+            }
+        }
+        cp_async_commit();
+    };
+    if constexpr (RING) {
+#pragma unroll
+        for (int i = 0; i < ATTN_RING - 1; ++i) issue(i);
+    }
+    for (int i = 0; i < nsteps; ++i) {
+        const int jg = jfirst + i * STRIDE;
+        float kf[ATTN_U][E], vf[ATTN_U][E];
+        if constexpr (RING) {
+            issue(i + ATTN_RING - 1);
+            cp_async_wait<ATTN_RING - 1>();   // step i's group has landed
+            const uint32_t st = ring0 + (uint32_t)(i % ATTN_RING) * STAGEB;
+#pragma unroll
+            for (int u = 0; u < ATTN_U; ++u) {
+                smem_row<XT, E>(st + (2 * u) * ROWB, kf[u]);
+                smem_row<XT, E>(st + (2 * u + 1) * ROWB, vf[u]);
+            }
+        } else {
+#pragma unroll
+            for (int u = 0; u < ATTN_U; ++u) {
+                const int j = min(jg + u, j1 - 1);   // a key past the split reloads the last one (masked below)
+                load_row<XT, E>(kb + (size_t)j * D, kf[u]);
+                load_row<XT, E>(vb + (size_t)j * D, vf[u]);
+            }
         }
         // the G x U dot products: lane partials, summed over the warp together
         constexpr int V = G * ATTN_U;
@@ -168,7 +248,11 @@ __global__ void __launch_bounds__(ATTN_WARPS * 32) attn_split_kernel(const AttnA
     }
 
     // merge the warps: per head the largest running maximum, the others rescaled to it
-    __shared__ float sm[ATTN_WARPS][G], sl[ATTN_WARPS][G], sacc[ATTN_WARPS][G][D];
+    // (every warp's copies have landed and been read: the ring's space is free after the barrier)
+    __syncthreads();
+    float(*sm)[G] = reinterpret_cast<float(*)[G]>(smraw);
+    float(*sl)[G] = reinterpret_cast<float(*)[G]>(smraw + ATTN_WARPS * G * 4);
+    float(*sacc)[G][D] = reinterpret_cast<float(*)[G][D]>(smraw + 2 * ATTN_WARPS * G * 4);
 #pragma unroll
     for (int h = 0; h < G; ++h) {
         if (lane == 0) {
