@@ -11,7 +11,9 @@ loop), so each kernel may begin streaming its weights while the previous one
 drains; the end-to-end leg, whose weights are copied in every step, does not
 use it.  The other
 workloads (Q8_0 4096x4096, the Q4_K 7B decode layer and the Q4_0 prefill
-GEMMs) are measured in the same run and reported under "workloads".
+GEMMs) are measured in the same run and reported under "workloads"; the
+decode-attention workloads (the pages' 512-token example and 7B-shaped
+batches) under "attention".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lwq|reference]
 
@@ -555,6 +557,43 @@ def sweep_points(lwq, dev, peaks: dict, fmts=None, shapes=None, Ms=None) -> list
     return out
 
 
+def time_attention(lwq, dev, name: str, reps: int, peaks: dict) -> dict:
+    """Decode attention through the C ABI: CUDA events around ``reps`` calls, the caches rotated
+    over copies that together exceed 4x L2 (every call streams its K and V from HBM)."""
+    import torch
+    spec = inputs.ATTENTION_WORKLOADS[name]
+    B, H, Hkv, L, D = spec["B"], spec["H"], spec["Hkv"], spec["L"], spec["D"]
+    q, k, v, lens = inputs.attention_problem(B, H, Hkv, L, D, spec["act"], seed=0)
+    dq = torch.from_numpy(q).to(dev)
+    cache_bytes = 2 * k.nbytes
+    copies = max(1, -(-4 * L2_BYTES // cache_bytes))
+    ks = [torch.from_numpy(k).to(dev)]
+    vs = [torch.from_numpy(v).to(dev)]
+    for _ in range(copies - 1):
+        ks.append(ks[0].clone())
+        vs.append(vs[0].clone())
+    out = torch.empty((B, H, D), dtype=torch.float32, device=dev)
+    code = lwq.LWQ_ACT_F16 if spec["act"] == "f16" else lwq.LWQ_ACT_BF16
+    scale = D ** -0.5
+    n = max(reps, 3 * copies)
+    for i in range(3):
+        lwq.lwq_attention_decode(code, dq, ks[i % copies], vs[i % copies], None, out, B, H, Hkv, L, D, scale)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(n):
+        lwq.lwq_attention_decode(code, dq, ks[i % copies], vs[i % copies], None, out, B, H, Hkv, L, D, scale)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    us = e0.elapsed_time(e1) * 1e3 / n
+    nbytes = cache_bytes + q.nbytes + out.numel() * 4
+    gbs = nbytes / us / 1e3
+    return {"shape": {"B": B, "H": H, "Hkv": Hkv, "L": L, "D": D, "dtype": spec["act"]}, "calls": n,
+            "us_per_call": round(us, 2), "launches_per_call": lwq.lwq_last_launch_count(),
+            "bytes_per_call": int(nbytes), "value": round(gbs, 1), "unit": "GB/s",
+            "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4), "cache_copies": copies}
+
+
 def run_gpu_arm(args):
     import torch
     import torch.distributed as dist
@@ -629,6 +668,11 @@ def run_gpu_arm(args):
                                      for p in per2]})
         extra[wl] = rec
 
+    attention = None
+    if not args.no_attention:
+        attention = {name: time_attention(lwq, dev, name, args.extra_steps, peaks)
+                     for name in inputs.ATTENTION_WORKLOADS}
+
     host = host_enqueue_cost(lwq, dev) if not args.no_host_cost else None
     sweep = None
     if not args.no_sweep:
@@ -658,7 +702,7 @@ def run_gpu_arm(args):
                        "parallelism": f"replicas x{world}", "timing": "CUDA graphs of one weight rotation (R steps), CUDA events",
                        "launch": "LWQ_FLAG_OVERLAP: programmatic dependent launches, weights constant"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": lps * args.steps, "clocks": clocks, "workloads": extra,
+            "gpu_launches": lps * args.steps, "clocks": clocks, "workloads": extra, "attention": attention,
             "host_enqueue": host, "sweep": sweep,
             "device_error": err,
         }
@@ -758,6 +802,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="leave the format x batch sweep out of the line")
     ap.add_argument("--no-host-cost", action="store_true", help="leave the host enqueue timing out")
+    ap.add_argument("--no-attention", action="store_true", help="leave the decode-attention workloads out")
     ap.add_argument("--sweep", action="store_true",
                     help="time the format x batch sweep instead (one JSON line per point)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)

@@ -294,6 +294,17 @@ WORKLOADS = {
                               shapes=[(11008, 4096), (4096, 11008)], seeds=[0, 0]),
 }
 
+# Decode attention workloads: one query token per sequence against its key/value cache.
+#  * the pages' example ("Compute Shaders con WebGPU para Inferencia ML", "El Mecanismo de
+#    Atencion"): 512 tokens, 12 heads, head dimension 64;
+#  * a 7B-shaped decode batch: 16 sequences of 4096 cached tokens, 32 heads of 128, each with
+#    its own kv head (multi-head) or 4 query heads per kv head (grouped).
+ATTENTION_WORKLOADS = {
+    "attention_decode_page": dict(B=1, H=12, Hkv=12, L=512, D=64, act="f16"),
+    "attention_decode_7b_mha": dict(B=16, H=32, Hkv=32, L=4096, D=128, act="f16"),
+    "attention_decode_7b_gqa": dict(B=16, H=32, Hkv=8, L=4096, D=128, act="f16"),
+}
+
 SWEEP_FMTS = ["q8_0", "q4_0", "q4_k"]
 SWEEP_MS = [1, 2, 4, 8, 16, 64, 256, 1024]
 SWEEP_SHAPES_KN = [(4096, 4096), (4096, 14336), (14336, 4096), (4096, 32000)]
