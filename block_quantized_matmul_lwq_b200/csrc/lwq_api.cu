@@ -189,7 +189,9 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
     }
     if (path != 1 || !tc_gemv_eligible(wf, K)) return LWQ_ERR_UNSUPPORTED;
     p->i8 = (fmt & LWQ_FLAG_ACT_I8) != 0;
-    if (p->i8 && (wf != LWQ_Q4_0 || M > 16)) return LWQ_ERR_UNSUPPORTED;
+    // int8 activation blocks: Q4_0 and Q8_0 weights, any M (passes of 8 rows; every pass streams
+    // the weights again, so a prefill-sized M reads them M / 8 times)
+    if (p->i8 && wf != LWQ_Q4_0 && wf != LWQ_Q8_0) return LWQ_ERR_UNSUPPORTED;
     // rows per pass: 8 with fp32 activations (3 parts, 24 columns) or int8 blocks, else 16
     const int mmax = (xt == X_F32 || p->i8) ? 8 : 16;
     p->m_group = M < mmax ? M : mmax;
@@ -321,10 +323,18 @@ cudaError_t launch_gemv_nt(int nt, const CUtensorMap &map, const GemvArgs &a, in
 cudaError_t dispatch_gemv(int wf, int xt, int nt, bool i8, const CUtensorMap &map, const GemvArgs &a, int ctas,
                           size_t smem, cudaStream_t st) {
     if (i8) {
-        if (wf != LWQ_Q4_0 || nt != 1) return cudaErrorInvalidValue;
-        if (xt == X_F32) return launch_gemv<F_Q4_0, X_F32, 1, true>(map, a, ctas, smem, st);
-        if (xt == X_F16) return launch_gemv<F_Q4_0, X_F16, 1, true>(map, a, ctas, smem, st);
-        return launch_gemv<F_Q4_0, X_BF16, 1, true>(map, a, ctas, smem, st);
+        if (nt != 1) return cudaErrorInvalidValue;
+        if (wf == LWQ_Q4_0) {
+            if (xt == X_F32) return launch_gemv<F_Q4_0, X_F32, 1, true>(map, a, ctas, smem, st);
+            if (xt == X_F16) return launch_gemv<F_Q4_0, X_F16, 1, true>(map, a, ctas, smem, st);
+            return launch_gemv<F_Q4_0, X_BF16, 1, true>(map, a, ctas, smem, st);
+        }
+        if (wf == LWQ_Q8_0) {
+            if (xt == X_F32) return launch_gemv<F_Q8_0, X_F32, 1, true>(map, a, ctas, smem, st);
+            if (xt == X_F16) return launch_gemv<F_Q8_0, X_F16, 1, true>(map, a, ctas, smem, st);
+            return launch_gemv<F_Q8_0, X_BF16, 1, true>(map, a, ctas, smem, st);
+        }
+        return cudaErrorInvalidValue;
     }
 #define LWQ_GV(F)                                                                   \
     if (xt == X_F32) return launch_gemv_nt<F, X_F32>(nt, map, a, ctas, smem, st);  \

@@ -719,22 +719,29 @@ struct RawPair<X_F32> {
     __device__ static __forceinline__ float2 get(T v) { return v; }
 };
 
-template <int XT>
+// Q8_0 weights take the same path with their int8 codes as they are: lane t
+// holds codes 4t..4t+3 and 16+4t..16+4t+3 of each block (the even block of a
+// pair starts 2 bytes into a word: two words and a PRMT), the activations in
+// the same natural order, and y += d_w * d_x * C.
+template <int XT, int FMT = F_Q4_0>
 struct Q40I8 {
+    static constexpr bool Q8 = FMT == F_Q8_0;
+    static constexpr int CB = FmtInfo<FMT>::chunk_bytes;
     uint32_t xq[8][2];   // [block][k-slots 4t.. / 16+4t..]: int8 codes of activation row g
-    float dx[8][2];      // [block][column 2t, 2t+1]: d_x / 16 of activation rows 2t, 2t+1
+    float dx[8][2];      // [block][column 2t, 2t+1]: d_x (Q4_0: d_x / 16) of activation rows 2t, 2t+1
     float inv;           // 1: no activation scale to undo
 
-    __device__ static __forceinline__ int cb0(int hb, int j) { return hb ? 4 * j : (j ? 4 * j - 2 : 14); }
-    __device__ static __forceinline__ int cb2(int hb, int j) { return hb ? 4 * j + 2 : 4 * j; }
+    // activation element of k-slot pair (4t, 4t+1) and (4t+2, 4t+3) of block parity hb
+    __device__ static __forceinline__ int cb0(int hb, int j) { return (Q8 || hb) ? 4 * j : (j ? 4 * j - 2 : 14); }
+    __device__ static __forceinline__ int cb2(int hb, int j) { return (Q8 || hb) ? 4 * j + 2 : 4 * j; }
 
     __device__ static __forceinline__ uint32_t pack_s8(int a, int b, int c, int d) {
         return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8) | ((uint32_t)(c & 0xFF) << 16) |
                ((uint32_t)d << 24);
     }
-    __device__ static __forceinline__ int q8(float v, float s) {
-        return max(-127, min(127, __float2int_rn(v * s)));
-    }
+    // |v| <= amax and s = RN(127 / amax), so |v s| rounds to at most 127 (1 + 2^-23) < 127.5:
+    // the code never leaves [-127, 127] and needs no clamp
+    __device__ static __forceinline__ int q8(float v, float s) { return __float2int_rn(v * s); }
 
     struct Slice {
         uint8_t *xp;     // the raw slice [M][nk] in shared memory
@@ -796,17 +803,49 @@ struct Q40I8 {
                 xq[b][0] = pack_s8(q8(v[0], sc), q8(v[1], sc), q8(v[2], sc), q8(v[3], sc));
                 xq[b][1] = pack_s8(q8(v[4], sc), q8(v[5], sc), q8(v[6], sc), q8(v[7], sc));
                 // columns 2t and 2t+1 carry activation rows 2t, 2t+1 (lanes 8t and 8t+4)
-                dx[b][0] = 0.0625f * __shfl_sync(0xffffffffu, d, 8 * t);
-                dx[b][1] = 0.0625f * __shfl_sync(0xffffffffu, d, 8 * t + 4);
+                constexpr float DS = Q8 ? 1.f : 0.0625f;   // Q4_0 codes enter as 16 (u - 8)
+                dx[b][0] = DS * __shfl_sync(0xffffffffu, d, 8 * t);
+                dx[b][1] = DS * __shfl_sync(0xffffffffu, d, 8 * t + 4);
             }
         }
     }
 
-    // box: this warp's [16 rows][144 B] chunk.
+    // box: this warp's [16 rows][CB] chunk.
     __device__ __forceinline__ void compute(uint32_t box, int, float (&acc)[1][4], int lane, int, const float *,
                                             int) const {
         const int g = lane >> 2, t = lane & 3;
-        const uint32_t r0 = box + g * 144, r1 = r0 + 8 * 144;   // rows g, g+8
+        const uint32_t r0 = box + g * CB, r1 = r0 + 8 * CB;   // rows g, g+8
+        if constexpr (Q8) {
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const uint32_t pb = 68 * p;   // the block pair: d(2p) codes(2p) | d(2p+1) codes(2p+1)
+                const uint32_t w00 = lds32(r0 + pb), w10 = lds32(r1 + pb);             // d(2p)
+                const uint32_t w08 = lds32(r0 + pb + 32), w18 = lds32(r1 + pb + 32);   // d(2p+1) in the high half
+                uint32_t u[2][2][2];   // [block of the pair][row][codes 4t.. / 16+4t..]
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t o = pb + 16 * h + 4 * t;
+                    u[0][0][h] = prmt(lds32(r0 + o), lds32(r0 + o + 4), 0x5432u);
+                    u[0][1][h] = prmt(lds32(r1 + o), lds32(r1 + o + 4), 0x5432u);
+                    u[1][0][h] = lds32(r0 + o + 36);
+                    u[1][1][h] = lds32(r1 + o + 36);
+                }
+                const float d[2][2] = {{f16_bits_to_float(w00), f16_bits_to_float(w10)},
+                                       {f16_bits_to_float(w08 >> 16), f16_bits_to_float(w18 >> 16)}};
+#pragma unroll
+                for (int hb = 0; hb < 2; ++hb) {
+                    const int b = 2 * p + hb;
+                    const uint32_t a[4] = {u[hb][0][0], u[hb][1][0], u[hb][0][1], u[hb][1][1]};
+                    int c[4];
+                    imma_s8_16832(c, a, xq[b][0], xq[b][1]);
+                    acc[0][0] = fmaf(d[hb][0] * dx[b][0], (float)c[0], acc[0][0]);
+                    acc[0][1] = fmaf(d[hb][0] * dx[b][1], (float)c[1], acc[0][1]);
+                    acc[0][2] = fmaf(d[hb][1] * dx[b][0], (float)c[2], acc[0][2]);
+                    acc[0][3] = fmaf(d[hb][1] * dx[b][1], (float)c[3], acc[0][3]);
+                }
+            }
+            return;
+        }
         const uint32_t sel = t ? 0x3210u : 0x3254u;            // word t of an even block
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
@@ -842,6 +881,8 @@ template <int FMT, int XT, int NT, bool I8>
 struct GemvImpl : Exact<FMT, XT, NT, gemv_kw(NT)> {};
 template <int XT>
 struct GemvImpl<F_Q4_0, XT, 1, true> : Q40I8<XT> {};
+template <int XT>
+struct GemvImpl<F_Q8_0, XT, 1, true> : Q40I8<XT, F_Q8_0> {};
 
 // ------------------------------------------------------------------ kernel
 // blockDim = GEMV_THREADS: warps 0..15 compute, warp 16 produces (TMA), warps

@@ -1,5 +1,5 @@
-"""GPU parity of the int8-activation GEMV (LWQ_FLAG_ACT_I8) against the oracle's
-definition (oracle.quantize_act_q8 / matmul_q8act).
+"""GPU parity of the int8-activation GEMV (LWQ_FLAG_ACT_I8; Q4_0 and Q8_0 weights)
+against the oracle's definition (oracle.quantize_act_q8 / matmul_q8act).
 
 The activation codes are integer decisions taken in fp32 on both sides with the
 same operations, so they must agree exactly; what remains is fp32 rounding of
@@ -35,8 +35,8 @@ def dev():
     assert lwq.lwq_get_device_error() == lwq.LWQ_OK
 
 
-def run_i8(a, Wq, x, M, N, K, dev, noalloc=False):
-    fmt = lwq.fmt_code("q4_0", a) | lwq.LWQ_FLAG_ACT_I8
+def run_i8(a, Wq, x, M, N, K, dev, noalloc=False, w="q4_0"):
+    fmt = lwq.fmt_code(w, a) | lwq.LWQ_FLAG_ACT_I8
     Wd, xd = to_device(Wq, dev), to_device(x, dev)
     y = torch.full((M, N), float("nan"), dtype=torch.float32, device=dev)
     if noalloc:
@@ -47,21 +47,34 @@ def run_i8(a, Wq, x, M, N, K, dev, noalloc=False):
     return y.cpu().numpy()
 
 
-def check(a, M, N, K, dev, seed, noalloc=False, x=None):
-    Wq, x0 = inputs.make_problem("q4_0", a, M, N, K, seed=seed)
+def check(a, M, N, K, dev, seed, noalloc=False, x=None, w="q4_0"):
+    Wq, x0 = inputs.make_problem(w, a, M, N, K, seed=seed)
     x = x0 if x is None else x
-    y = run_i8(a, Wq, x, M, N, K, dev, noalloc=noalloc)
-    y_ref, den = oracle.matmul_q8act("q4_0", Wq, x, act=a)
+    y = run_i8(a, Wq, x, M, N, K, dev, noalloc=noalloc, w=w)
+    y_ref, den = oracle.matmul_q8act(w, Wq, x, act=a)
     err = oracle.normalised_error(y, y_ref, den)
     assert err <= TOL_I8, f"{a} M={M} N={N} K={K}: err {err:.3e} > {TOL_I8}"
     return y, Wq, x
 
 
+@pytest.mark.parametrize("w", ["q4_0", "q8_0"])
 @pytest.mark.parametrize("a", ["f32", "f16", "bf16"])
 @pytest.mark.parametrize("M,N,K", [(1, 211, 3072), (2, 1000, 4096), (5, 47, 11008), (8, 300, 4096),
                                    (9, 130, 2048), (16, 64, 4352)])
-def test_parity(dev, a, M, N, K):
-    check(a, M, N, K, dev, seed=M * 31 + K)
+def test_parity(dev, w, a, M, N, K):
+    check(a, M, N, K, dev, seed=M * 31 + K, w=w)
+
+
+@pytest.mark.parametrize("w", ["q4_0", "q8_0"])
+@pytest.mark.parametrize("M", [17, 40, 130])
+def test_many_rows_in_passes(dev, w, M):
+    """M > 16: passes of 8 activation rows, each streaming the weights."""
+    check("bf16", M, 300, 2048, dev, seed=M, w=w)
+
+
+def test_q8_0_gemv_4096x4096(dev):
+    """Q8_0 4096 x 4096 at M = 1 with int8 activation blocks, every output."""
+    check("f32", 1, 4096, 4096, dev, seed=0, w="q8_0")
 
 
 def test_headline_shape_against_exact_product(dev):
@@ -94,7 +107,7 @@ def test_noalloc_and_deterministic(dev):
     assert oracle.normalised_error(ys[0], y_ref, den) <= TOL_I8
 
 
-@pytest.mark.parametrize("w,M,K", [("q8_0", 1, 4096), ("q4_k", 1, 4096), ("q4_0", 17, 4096), ("q4_0", 1, 288)])
+@pytest.mark.parametrize("w,M,K", [("q4_k", 1, 4096), ("q5_k", 1, 4096), ("q6_k", 1, 4096), ("q4_0", 1, 288)])
 def test_unsupported(dev, w, M, K):
     fmt = lwq.fmt_code(w, "f16") | lwq.LWQ_FLAG_ACT_I8
     N = 64
