@@ -125,7 +125,10 @@ struct Plan {
 // n8 column tiles of the GEMV for a pass of mg activation rows: each row takes
 // P columns (P = 3 bf16 parts for fp32 activations, else 1), 8 columns per tile.
 inline int gemv_nt(int xt, bool i8, int mg) { return i8 ? 1 : (mg * gemv_parts(xt, i8) + 7) / 8; }
-inline int gemv_chunk_bytes(int wf) { return wf == LWQ_Q8_0 ? 272 : (wf == LWQ_Q5_K ? 176 : 144); }
+// bytes of one row of a chunk in a GEMV stage (Q6_K: its 240-byte box, see FmtInfo)
+inline int gemv_chunk_bytes(int wf) {
+    return wf == LWQ_Q8_0 ? 272 : (wf == LWQ_Q5_K ? 176 : (wf == LWQ_Q6_K ? 240 : 144));
+}
 inline size_t gemv_smem(int wf, int cps, int stages, int nt, bool i8, int xt, int m) {
     return gemv_smem_layout(gemv_chunk_bytes(wf), cps, stages, nt, wf == LWQ_Q4_K || wf == LWQ_Q5_K,
                             gemv_parts(xt, i8), m,
@@ -137,7 +140,12 @@ inline size_t gemv_smem(int wf, int cps, int stages, int nt, bool i8, int xt, in
 // multiples, as the weight stream's tensor map needs); the others take the
 // simple kernel.
 bool tc_gemv_format(int wf) { return wf == LWQ_Q8_0 || wf == LWQ_Q4_0 || wf == LWQ_Q4_K || wf == LWQ_Q5_K; }
-bool tc_gemv_eligible(int wf, long K) { return tc_gemv_format(wf) && K % 256 == 0; }
+// Q6_K rows are 210 bytes per superblock: the tensor map needs a 16-byte row
+// stride, so K a multiple of 2048 (8 superblocks)
+bool tc_gemv_eligible(int wf, long K) {
+    if (wf == LWQ_Q6_K) return K % 2048 == 0;
+    return tc_gemv_format(wf) && K % 256 == 0;
+}
 
 // Workspace layout: fp32 split-K partials [S][m_group][N].  Nothing in it
 // needs to start at any particular value.
@@ -345,6 +353,7 @@ cudaError_t dispatch_gemv(int wf, int xt, int nt, bool i8, const CUtensorMap &ma
     case LWQ_Q8_0: { LWQ_GV(F_Q8_0) }
     case LWQ_Q4_K: { LWQ_GV(F_Q4_K) }
     case LWQ_Q5_K: { LWQ_GV(F_Q5_K) }
+    case LWQ_Q6_K: { LWQ_GV(F_Q6_K) }
     }
 #undef LWQ_GV
     return cudaErrorInvalidValue;
@@ -429,6 +438,16 @@ MapReq map_req(const void *p, CUtensorMapDataType dtype, int rank, CUtensorMapSw
 // chunk), strides (row_bytes, chunk_bytes); a box of (all words, 16 rows, cps
 // chunks) lands as cps consecutive [16 rows][chunk bytes] boxes, one GEMV stage.
 int encode_weight_map(CUtensorMap *map, const void *Wq, int wf, int N, long rb, int cps) {
+    if (wf == LWQ_Q6_K) {
+        // [N rows][rb / 2 words] with a box of [16 rows][120 words], one per chunk
+        MapReq r = map_req(Wq, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, CU_TENSOR_MAP_SWIZZLE_NONE);
+        r.dims[0] = (cuuint64_t)(rb / 2);
+        r.dims[1] = (cuuint64_t)N;
+        r.strides[0] = (cuuint64_t)rb;
+        r.box[0] = 120;
+        r.box[1] = (cuuint32_t)GEMV_ROWS;
+        return encode_cached(r, map);
+    }
     const int cb = gemv_chunk_bytes(wf);
     MapReq r = map_req(Wq, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, CU_TENSOR_MAP_SWIZZLE_NONE);
     r.dims[0] = (cuuint64_t)(cb / 8);

@@ -68,6 +68,11 @@ template <>
 struct FmtInfo<F_Q4_K> { static constexpr int chunk_bytes = 144; };
 template <>
 struct FmtInfo<F_Q5_K> { static constexpr int chunk_bytes = 176; };
+// Q6_K superblocks are 210 bytes, not a 16-byte multiple: each chunk is its own
+// TMA box of 120 16-bit words (240 bytes) starting at the 16-byte boundary at
+// or below the superblock, which lies 2 * ((105 c) & 7) bytes into the box.
+template <>
+struct FmtInfo<F_Q6_K> { static constexpr int chunk_bytes = 240; };
 // formats with a per-sub-block min (the S_j sums of x enter the result)
 __host__ __device__ constexpr bool fmt_has_min(int fmt) { return fmt == F_Q4_K || fmt == F_Q5_K; }
 
@@ -170,6 +175,12 @@ __device__ __forceinline__ uint32_t q4k_hi(uint32_t w) {   // high nibbles, unsi
     if constexpr (BF) return hfma2_bf16(and_or(w >> 4, 0x000F000Fu, B2_MAGIC), B2_ONE, B2_M128);
     else return hfma2_f16(and_or(w, 0x00F000F0u, H2_MAGIC), H2_SIXTEENTH, H2_M64);
 }
+// Q6_K: the 6-bit codes of bytes 0 and 2, minus 32.
+template <bool BF>
+__device__ __forceinline__ uint32_t q6k_pair(uint32_t v) {
+    if constexpr (BF) return hfma2_bf16(and_or(v, 0x003F003Fu, B2_MAGIC), B2_ONE, 0xC320C320u);   // 128 + v - 160
+    else return hfma2_f16(and_or(v, 0x003F003Fu, H2_MAGIC), H2_ONE, 0xE420E420u);                 // 1024 + v - 1056
+}
 // Q5_K: the 5-bit codes of bytes 0 and 2, unsigned.
 template <bool BF>
 __device__ __forceinline__ uint32_t q5k_pair(uint32_t v) {
@@ -246,6 +257,7 @@ struct Exact {
     static constexpr int CB = FmtInfo<FMT>::chunk_bytes;
     uint32_t xf[NT][NB][2][2];               // [tile][block][step][reg]
     float inv;                               // 1 / the activation scale (a power of two)
+    uint32_t q6o = 0;                        // Q6_K: byte offset of the superblock in its chunk box
 
     // ---------------------------------------------------------- prologue
     // The CTA's slice of x is prepared once, by all nact compute warps
@@ -507,6 +519,65 @@ struct Exact {
         }
     }
 
+    // Q6_K: 32-bit word at byte q6o + off of a row (q6o even; MIS: q6o = 2 mod 4,
+    // the word straddles two aligned words)
+    template <bool MIS>
+    __device__ __forceinline__ uint32_t q6w(uint32_t row, uint32_t off) const {
+        if constexpr (MIS) return prmt(lds32(row + q6o - 2 + off), lds32(row + q6o + 2 + off), 0x5432u);
+        else return lds32(row + q6o + off);
+    }
+    // Q6_K (210-byte superblock = the warp's chunk; with KW = 128 the warp takes
+    // half `half` of it).  For half n and l0 in {0, 16}, lane t's words
+    // A = ql[64n + l0 + 4t], B = ql[64n + 32 + l0 + 4t] and H = qh[32n + l0 + 4t]
+    // give the 6-bit codes of elements 16j + 4t .. 16j + 4t + 3 of the four
+    // sub-blocks j = 8n + 2g + l0/16 (g = 0..3: low nibbles of A, of B, high
+    // nibbles of A, of B; high bits 2g, 2g+1 of H).  A sub-block of 16 weights has
+    // one int8 scale: one MMA step, then y += d * sc_j * C.
+    template <bool MIS>
+    __device__ __forceinline__ void compute_q6(uint32_t r0, uint32_t r1, int half, float (&acc)[NT][4], int t) const {
+        const float d0 = f16_lo(q6w<MIS>(r0, 208)), d1 = f16_lo(q6w<MIS>(r1, 208));
+        constexpr int NH = NB / 4;                                    // halves of the superblock: 2 or 1
+#pragma unroll
+        for (int hh = 0; hh < NH; ++hh) {
+            const int n = NH == 2 ? hh : half;
+            // int8 scales of sub-blocks 8n .. 8n + 7, biased by 128 (so a byte is an unsigned magic)
+            const uint32_t sa0 = q6w<MIS>(r0, 192 + 8 * n) ^ 0x80808080u, sb0 = q6w<MIS>(r0, 196 + 8 * n) ^ 0x80808080u;
+            const uint32_t sa1 = q6w<MIS>(r1, 192 + 8 * n) ^ 0x80808080u, sb1 = q6w<MIS>(r1, 196 + 8 * n) ^ 0x80808080u;
+#pragma unroll
+            for (int lq = 0; lq < 2; ++lq) {
+                const uint32_t l0 = 16 * lq;
+                const uint32_t A0 = q6w<MIS>(r0, 64 * n + l0 + 4 * t), A1 = q6w<MIS>(r1, 64 * n + l0 + 4 * t);
+                const uint32_t B0 = q6w<MIS>(r0, 64 * n + 32 + l0 + 4 * t), B1 = q6w<MIS>(r1, 64 * n + 32 + l0 + 4 * t);
+                const uint32_t H0 = q6w<MIS>(r0, 128 + 32 * n + l0 + 4 * t), H1 = q6w<MIS>(r1, 128 + 32 * n + l0 + 4 * t);
+#pragma unroll
+                for (int g6 = 0; g6 < 4; ++g6) {
+                    auto code = [&](uint32_t A, uint32_t B, uint32_t H) {
+                        const uint32_t lo = ((g6 & 1) ? B : A) >> (4 * (g6 >> 1));
+                        const uint32_t hi = g6 == 0 ? (H << 4) : g6 == 1 ? (H << 2) : g6 == 2 ? H : (H >> 2);
+                        return (lo & 0x0F0F0F0Fu) | (hi & 0x30303030u);
+                    };
+                    const uint32_t v0 = code(A0, B0, H0), v1 = code(A1, B1, H1);
+                    const int j = 2 * g6 + lq;                 // sub-block within half n (0..7)
+                    // sc_j = (2^23 + (sc + 128)) - (2^23 + 128), exact; d * sc_j has <= 19 bits: exact
+                    const float s0 = (byte_magic(j < 4 ? sa0 : sb0, j & 3) - 8388736.f) * d0;
+                    const float s1 = (byte_magic(j < 4 ? sa1 : sb1, j & 3) - 8388736.f) * d1;
+                    const uint32_t a[4] = {q6k_pair<BF>(v0), q6k_pair<BF>(v1), q6k_pair<BF>(v0 >> 8),
+                                           q6k_pair<BF>(v1 >> 8)};
+                    const int jl = 8 * hh + j;                 // sub-block of this warp: block jl / 2, step jl % 2
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        float c[4];
+                        mma_zero<BF>(c, a, xf[nt][jl >> 1][jl & 1][0], xf[nt][jl >> 1][jl & 1][1]);
+                        acc[nt][0] = fmaf(s0, c[0], acc[nt][0]);
+                        acc[nt][1] = fmaf(s0, c[1], acc[nt][1]);
+                        acc[nt][2] = fmaf(s1, c[2], acc[nt][2]);
+                        acc[nt][3] = fmaf(s1, c[3], acc[nt][3]);
+                    }
+                }
+            }
+        }
+    }
+
     // box: this warp's chunk, row 0, in the stage; half: which half of the
     // chunk (KW = 128); sxw: the x sums of this warp's first sub-block, rows
     // sstride apart (Q4_K).
@@ -534,6 +605,9 @@ struct Exact {
                     block(a0, a1, 2 * pp + 1, f16_hi(v0), f16_hi(v1), acc);
                 }
             }
+        } else if constexpr (FMT == F_Q6_K) {
+            if (q6o & 2) compute_q6<true>(r0, r1, half, acc, t);
+            else compute_q6<false>(r0, r1, half, acc, t);
         } else if constexpr (FMT == F_Q8_0) {
 #pragma unroll
             for (int pp = 0; pp < NB / 2; ++pp) {
@@ -961,7 +1035,15 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1)
                 // one 3-D box per stage: [chunks of this split][16 rows][chunk bytes]; the
                 // last split's box may run past the last chunk, where it reads zeros
                 mbar_arrive_expect_tx(&full[s], (uint32_t)L.stage);
-                tma_load_3d(ring + (size_t)s * L.stage, &wmap, &full[s], 0, tile * GEMV_ROWS, c_begin);
+                if constexpr (FMT == F_Q6_K) {
+                    // one 2-D box per chunk, [16 rows][120 words] from the 16-byte boundary at or
+                    // below the superblock (chunks past the end read zeros)
+                    for (int ci = 0; ci < a.cps; ++ci)
+                        tma_load_2d(ring + (size_t)s * L.stage + (size_t)ci * GEMV_ROWS * CB, &wmap, &full[s],
+                                    (105 * (c_begin + ci)) & ~7, tile * GEMV_ROWS);
+                } else {
+                    tma_load_3d(ring + (size_t)s * L.stage, &wmap, &full[s], 0, tile * GEMV_ROWS, c_begin);
+                }
                 if (++s == ws) {
                     s = 0;
                     ph ^= 1u;
@@ -1067,6 +1149,7 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1)
     sl.rs = rs;
     if (!impl.prologue(a, sl, c_begin, xfull, nact, warp, lane, a.timeout_ns)) return;
     impl.load_frags(sl, ci * CHUNK, half, lane);
+    if constexpr (FMT == F_Q6_K && !I8) impl.q6o = 2u * (uint32_t)((105 * (c_begin + ci)) & 7);
     const float *sxw = sx + ci * (CHUNK / 32) + half * (KW / 32);
     const int sstride = nk / 32;
     const int g = lane >> 2, t = lane & 3;

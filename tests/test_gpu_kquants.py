@@ -1,8 +1,9 @@
 """More K-quant formats (Q5_K, Q6_K, Q2_K) on the GPU against the oracle.
 
-Q5_K has tensor-core decoders (the GEMV and the tcgen05 GEMM); Q6_K and Q2_K
-rows are 210 and 84 bytes per superblock, so their rows are not 16-byte
-multiples in general and the simple kernel takes them.  Every case is scored
+Q5_K has tensor-core decoders (the GEMV and the tcgen05 GEMM).  Q6_K and Q2_K
+superblocks are 210 and 84 bytes, so their rows are not 16-byte multiples in
+general: Q6_K takes the tensor-core GEMV when K is a multiple of 2048 and the
+simple kernel otherwise; Q2_K always takes the simple kernel.  Every case is scored
 element by element against the oracle on the same seeded inputs.
 """
 
@@ -46,6 +47,23 @@ def test_small_shapes(dev, w, a, M, N, K):
 def test_q5_k_every_column_layout(dev, a, M):
     assert lwq.lwq_select_config(lwq.fmt_code("q5_k", a), M, 45, 1024).path == 1
     check_full("q5_k", a, M, 45, 1024, dev, seed=200 + M)
+
+
+@pytest.mark.parametrize("a", ACTS)
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 6, 8, 9, 16])
+@pytest.mark.parametrize("K", [2048, 6144])
+def test_q6_k_tensor_core_gemv(dev, a, M, K):
+    """Q6_K rows of whole 16-byte multiples (K % 2048 == 0): per-chunk TMA boxes whose superblock
+    starts 0..14 bytes in (both word alignments), every column layout, ragged N."""
+    assert lwq.lwq_select_config(lwq.fmt_code("q6_k", a), M, 45, K).path == 1
+    check_full("q6_k", a, M, 45, K, dev, seed=300 + M + K)
+
+
+@pytest.mark.parametrize("warps,splits,stages", [(1, 0, 2), (3, 0, 2), (8, 2, 3), (4, 3, 2)])
+def test_q6_k_forced_gemv_configs(dev, warps, splits, stages):
+    cfg = lwq.lwq_config()
+    cfg.path, cfg.warps, cfg.splits, cfg.stages = 1, warps, splits, stages
+    check_full("q6_k", "f16", 3, 100, 4096, dev, seed=warps + splits, cfg=cfg)
 
 
 @pytest.mark.parametrize("w", ["q5_k", "q6_k", "q2_k"])
