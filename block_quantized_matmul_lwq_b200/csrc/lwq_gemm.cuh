@@ -69,6 +69,10 @@ template <>
 struct GemmFmt<F_Q4_K> { static constexpr int chunk_bytes = 144; };
 template <>
 struct GemmFmt<F_Q5_K> { static constexpr int chunk_bytes = 176; };
+// Q6_K: a 240-byte box per row and superblock, from the 16-byte boundary at or
+// below the 210-byte superblock (which starts 2 * ((105 c) & 7) bytes in)
+template <>
+struct GemmFmt<F_Q6_K> { static constexpr int chunk_bytes = 240; };
 
 __host__ __device__ constexpr size_t gemm_a_bytes() { return (size_t)GEMM_WROWS * 128; }
 __host__ __device__ constexpr size_t gemm_b_bytes(int bn) { return (size_t)bn * 128; }
@@ -301,6 +305,53 @@ struct Dequant<F_Q5_K, XT> {
     }
 };
 
+// 16 bytes at a 2-byte-aligned shared address (5 aligned words and PRMTs when
+// the address is 2 mod 4).
+__device__ __forceinline__ uint4 lds128_a2(uint32_t addr) {
+    const uint32_t b = addr & ~3u;
+    const uint32_t w0 = lds32(b), w1 = lds32(b + 4), w2 = lds32(b + 8), w3 = lds32(b + 12);
+    if (!(addr & 2)) return make_uint4(w0, w1, w2, w3);
+    const uint32_t w4 = lds32(b + 16);
+    return make_uint4(prmt(w0, w1, 0x5432u), prmt(w1, w2, 0x5432u), prmt(w2, w3, 0x5432u), prmt(w3, w4, 0x5432u));
+}
+
+// Q6_K: k-block kb = sub-blocks 4kb .. 4kb+3 of 16 weights; (h, v) takes
+// sub-block j = 4kb + 2h + v, whose codes are nibble g>>1 of
+// ql[64n + 32(g&1) + 16(j&1) + i] and bits 2g, 2g+1 of qh[32n + 16(j&1) + i]
+// (n = j/8, g = (j/2)%4, i < 16), scale int8 sc[j], w = d * sc * (q - 32),
+// exact in fp32 and rounded once to the 16-bit type.  prow: the row's
+// superblock (2-byte aligned).
+template <int XT>
+struct Dequant<F_Q6_K, XT> {
+    static __device__ __forceinline__ void run(uint32_t prow, int kb, int h, int v, uint32_t a_base, int r) {
+        const int j = 4 * kb + 2 * h + v, n = j >> 3, g = (j >> 1) & 3, l0 = 16 * (j & 1);
+        const uint4 qlv = lds128_a2(prow + 64 * n + 32 * (g & 1) + l0);
+        const uint4 qhv = lds128_a2(prow + 128 + 32 * n + l0);
+        const uint32_t dw = lds32((prow + 208) & ~3u), sw = lds32((prow + 192 + j) & ~3u);
+        const float d = f16_bits_to_float(((prow + 208) & 2) ? (dw >> 16) : dw);
+        const int sc = (int)(int8_t)(sw >> (8 * ((prow + 192 + j) & 3)));
+        const float ds = d * (float)sc;   // exact in fp32
+        const uint32_t ql[4] = {qlv.x, qlv.y, qlv.z, qlv.w}, qh[4] = {qhv.x, qhv.y, qhv.z, qhv.w};
+        const uint32_t ls = 4u * (g >> 1), hs = 2u * g;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            float f[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t bsh = 8 * (i & 3);
+                const uint32_t q = ((ql[2 * c + (i >> 2)] >> (bsh + ls)) & 15u) |
+                                   (((qh[2 * c + (i >> 2)] >> (bsh + hs)) & 3u) << 4);
+                f[i] = ds * (float)((int)q - 32);   // exact
+            }
+            uint32_t o[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+                o[p] = (XT == X_F16) ? pack_f16x2(f[2 * p], f[2 * p + 1]) : pack_bf16x2(f[2 * p], f[2 * p + 1]);
+            st_shared_v4(a_base + sw128_chunk_offset(r, 4 * h + 2 * v + c), o[0], o[1], o[2], o[3]);
+        }
+    }
+};
+
 // -------------------------------------------------------------------- kernel
 // H = 128-row halves of a weight tile (1 or 2).  With H = 2 the tile is 256
 // weight rows: two UMMAs per K step (one per half, into two accumulators)
@@ -395,9 +446,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     // Wq only: callers that allow overlap promise it is not written by preceding work
                     if (ci >= P && !(ok = mbar_wait(&p_empty[ps], pph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
                     mbar_arrive_expect_tx(&p_full[ps], P_BYTES);
+                    // Q6_K: the box starts at the 16-byte boundary at or below the superblock
+                    const int x0 = FMT == F_Q6_K ? (105 * c) & ~7 : c * (CB / 2);
 #pragma unroll
                     for (int hh = 0; hh < H; ++hh)   // rows past N read zeros
-                        tma_load_2d(pk + (size_t)ps * P_BYTES + hh * PH_BYTES, &wmap, &p_full[ps], c * (CB / 2),
+                        tma_load_2d(pk + (size_t)ps * P_BYTES + hh * PH_BYTES, &wmap, &p_full[ps], x0,
                                     wt * WR + hh * GEMM_WROWS);
                     if (++ps == P) {
                         ps = 0;
@@ -494,7 +547,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             const int c0 = ks * a.cps, c1 = min(a.nchunks, c0 + a.cps);
             for (int c = c0; ok && c < c1; ++c) {
                 if (!(ok = mbar_wait(&p_full[ps], pph, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
-                const uint32_t prow = smem_u32(pk) + (uint32_t)(ps * P_BYTES + r * CB);
+                // (Q6_K: the superblock lies 2 * ((105 c) & 7) bytes into its box)
+                const uint32_t prow = smem_u32(pk) + (uint32_t)(ps * P_BYTES + r * CB) +
+                                      (FMT == F_Q6_K ? 2u * (uint32_t)((105 * c) & 7) : 0u);
                 // BATCH k-blocks per batch; the A ring's depth is a multiple of BATCH, so a batch never wraps
                 for (int kb = 0; kb < GEMM_KB_PER_CHUNK; kb += BATCH, kbi += BATCH) {
                     if (kbi >= SA) {
@@ -580,13 +635,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 }
 
 // ---------------------------------------------------------------- host side
-// Formats with a tcgen05 GEMM decoder; their packed rows are 16-byte multiples.
-inline bool gemm_format(int wf) { return wf == LWQ_Q8_0 || wf == LWQ_Q4_0 || wf == LWQ_Q4_K || wf == LWQ_Q5_K; }
+// Formats with a tcgen05 GEMM decoder; their packed rows must be 16-byte
+// multiples (the weight tensor map's row stride): Q6_K needs K % 2048 == 0.
+inline bool gemm_format(int wf) {
+    return wf == LWQ_Q8_0 || wf == LWQ_Q4_0 || wf == LWQ_Q4_K || wf == LWQ_Q5_K || wf == LWQ_Q6_K;
+}
 inline bool gemm_eligible(int wf, int xt, long K) {
-    return gemm_format(wf) && (xt == X_F16 || xt == X_BF16) && K % 256 == 0;
+    return gemm_format(wf) && (xt == X_F16 || xt == X_BF16) && K % (wf == LWQ_Q6_K ? 2048 : 256) == 0;
 }
 
-inline int gemm_chunk_bytes(int wf) { return wf == LWQ_Q8_0 ? 272 : (wf == LWQ_Q5_K ? 176 : 144); }
+// bytes of one row of a packed chunk in a stage (Q6_K: its 240-byte box)
+inline int gemm_chunk_bytes(int wf) {
+    return wf == LWQ_Q8_0 ? 272 : (wf == LWQ_Q5_K ? 176 : (wf == LWQ_Q6_K ? 240 : 144));
+}
 
 // Ring depths.  128-row tiles: 4 dequantized A stages (made on chip, two per
 // batch), 3 packed chunk stages (each feeds four k-blocks; 2 when shared

@@ -59,6 +59,25 @@ def test_q6_k_tensor_core_gemv(dev, a, M, K):
     check_full("q6_k", a, M, 45, K, dev, seed=300 + M + K)
 
 
+@pytest.mark.parametrize("a", ["bf16", "f16"])
+@pytest.mark.parametrize("M,N,K,tile_n", [(40, 300, 2048, 0), (130, 1000, 4096, 0), (200, 520, 6144, 128),
+                                          (64, 700, 4096, 256)])
+def test_q6_k_gemm(dev, a, M, N, K, tile_n):
+    """Q6_K on the tcgen05 GEMM (K a multiple of 2048): per-superblock boxes at both word alignments."""
+    cfg = None
+    if tile_n:
+        cfg = lwq.lwq_config()
+        cfg.path, cfg.tile_n = 2, tile_n
+    assert lwq.lwq_select_config(lwq.fmt_code("q6_k", a), M, N, K).path == 2
+    check_full("q6_k", a, M, N, K, dev, seed=M + K, cfg=cfg)
+
+
+def test_q6_k_prefill_gemm_sampled(dev):
+    M, N, K = 512, 11008, 4096
+    assert lwq.lwq_select_config(lwq.fmt_code("q6_k", "bf16"), M, N, K).path == 2
+    check_sampled("q6_k", "bf16", M, N, K, dev, seed=9, count=2000)
+
+
 @pytest.mark.parametrize("warps,splits,stages", [(1, 0, 2), (3, 0, 2), (8, 2, 3), (4, 3, 2)])
 def test_q6_k_forced_gemv_configs(dev, warps, splits, stages):
     cfg = lwq.lwq_config()
