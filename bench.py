@@ -805,6 +805,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-attention", action="store_true", help="leave the decode-attention workloads out")
     ap.add_argument("--sweep", action="store_true",
                     help="time the format x batch sweep instead (one JSON line per point)")
+    ap.add_argument("--case", default=None,
+                    help="time one workload alone (a name from inputs.WORKLOADS or inputs.ATTENTION_WORKLOADS) "
+                         "and print its own JSON line: a small command for profilers")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--reference-budget", type=float, default=60.0)
     ap.add_argument("--traffic", type=float, default=None,
@@ -816,12 +819,38 @@ def parse_args(argv=None):
     return args
 
 
+def run_case(args):
+    """One workload alone, on one GPU (the command the ncu captures under profiles/ run)."""
+    import torch
+    import block_quantized_matmul_lwq_b200 as lwq
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, _ = load_peaks()
+    if args.case in inputs.ATTENTION_WORKLOADS:
+        spec = inputs.ATTENTION_WORKLOADS[args.case]
+        need = lwq.lwq_attention_workspace_size(spec["B"], spec["H"], spec["Hkv"], spec["L"], spec["D"])
+        ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
+        lwq.lwq_init(ws, ws.numel())
+        rec = time_attention(lwq, dev, args.case, args.steps, peaks)
+    else:
+        need = max(lwq.lwq_workspace_size(call_fmt(lwq, f, a), M, N, K) for f, a, M, N, K, _ in step_calls(args.case))
+        ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
+        lwq.lwq_init(ws, ws.numel())
+        prob, ms_local, ms, lps, per = time_workload(lwq, args.case, dev, args.steps, args.warmup, False)
+        rec = {"ms_per_step": round(ms / args.steps, 5), "launches_per_step": lps,
+               "per_call_ms": [round(p["ms_mean"], 5) for p in per]}
+    print(json.dumps({"case": args.case, **rec}), flush=True)
+    lwq.lwq_shutdown()
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         run_reference_arm(args)
     elif args.sweep:
         run_sweep(args)
+    elif args.case:
+        run_case(args)
     else:
         run_gpu_arm(args)
 
