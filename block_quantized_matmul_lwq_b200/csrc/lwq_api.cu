@@ -735,9 +735,9 @@ size_t lwq_workspace_size(int fmt, int max_M, int max_N, int max_K) {
     }
     // The GEMM splits K only while its output tiles fill at most half the SMs, into
     // S <= ceil(sms / tiles) <= K / 1024 slices, so S * tiles <= 1.5 sms and each tile holds at most
-    // 128 x 256 outputs: its partials never exceed 4 * 1.5 * sms * 32768 bytes, nor 4 * (K/1024) * M * N.
+    // 256 x 256 outputs: its partials never exceed 4 * 1.5 * sms * 65536 bytes, nor 4 * (K/1024) * M * N.
     if (max_M > 16 && (fmt & LWQ_ACT_MASK) != LWQ_ACT_F32) {
-        const size_t by_grid = (size_t)6 * sms * 32768;
+        const size_t by_grid = (size_t)6 * sms * 65536;
         const size_t by_shape = (size_t)4 * (max_K / 1024) * max_M * max_N;
         const size_t g = by_grid < by_shape ? by_grid : by_shape;
         if (g > need) need = g;

@@ -189,6 +189,20 @@ def test_more_kquant_formats_routing_and_row_bytes():
     assert lwq.lwq_row_bytes(lwq.fmt_code("q6_k", "f16"), 288) == 0
 
 
+def test_workspace_size_covers_smaller_shapes():
+    """lwq_workspace_size(fmt, max_M, N, K) covers every M <= max_M: the split-K partials of each
+    sweep point (splits x rows of a pass x N fp32) fit the size taken at the sweep's largest M."""
+    for w in inputs.SWEEP_FMTS:
+        for K, N in inputs.SWEEP_SHAPES_KN:
+            fmt = lwq.fmt_code(w, "f16")
+            top = lwq.lwq_workspace_size(fmt, max(inputs.SWEEP_MS), N, K)
+            for M in list(range(1, 40)) + inputs.SWEEP_MS:
+                c = lwq.lwq_select_config(fmt, M, N, K)
+                rows = M if c.path == 2 else min(M, 16)
+                need = c.splits * rows * N * 4 if c.splits > 1 else 0
+                assert need <= top, (w, K, N, M, need, top)
+
+
 def test_int8_flag_plan():
     i8 = lwq.fmt_code("q4_0", "bf16") | lwq.LWQ_FLAG_ACT_I8
     cfg = lwq.lwq_select_config(i8, 16, 4096, 4096)
