@@ -659,7 +659,17 @@ int run(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, c
 // ------------------------------------------------------- decode attention
 template <int XT, int D, int G>
 cudaError_t launch_attn(const AttnArgs &a, cudaStream_t st) {
-    attn_split_kernel<XT, D, G><<<dim3((unsigned)a.S, (unsigned)a.Hkv, (unsigned)a.B), ATTN_WARPS * 32, 0, st>>>(a);
+    const dim3 grid((unsigned)a.S, (unsigned)a.Hkv, (unsigned)a.B);
+    if constexpr (G == 1) {
+        attn_split_kernel<XT, D, G><<<grid, ATTN_WARPS * 32, 0, st>>>(a);
+    } else {
+        // grouped heads: the tensor-core pass (its K/V ring is dynamic shared memory)
+        auto kern = attn_split_tc_kernel<XT, D, G>;
+        constexpr size_t smem = attn_tc_smem<D>();
+        cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), smem);
+        if (e != cudaSuccess) return e;
+        kern<<<grid, ATTN_WARPS * 32, smem, st>>>(a);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || a.S == 1) return e;
     // the splits' merge: a programmatic dependent launch that waits for the split kernel
@@ -827,7 +837,7 @@ size_t lwq_attention_workspace_size(int B, int H, int Hkv, int Lmax, int D) {
     int dev = 0, sms = 148;
     if (current_device(&dev) == LWQ_OK) sms = sm_count(dev);
     int S = 1, chunk = 0;
-    attn_splits(B, Hkv, Lmax, sms, &S, &chunk);
+    attn_splits(B, H, Hkv, Lmax, sms, &S, &chunk);
     return attn_ws_bytes(B, H, S, D);
 }
 
@@ -854,7 +864,7 @@ int lwq_attention_decode(int dtype, const void *q, const void *k, const void *v,
     a.Hkv = Hkv;
     a.Lmax = Lmax;
     a.qscale = scale * 1.4426950408889634f;   // log2(e): the kernels take exponentials as exp2
-    attn_splits(B, Hkv, Lmax, sm_count(dev), &a.S, &a.chunk);
+    attn_splits(B, H, Hkv, Lmax, sm_count(dev), &a.S, &a.chunk);
     DeviceState &ds = g_dev[dev];
     a.part = nullptr;
     const size_t need = attn_ws_bytes(B, H, a.S, D);
