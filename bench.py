@@ -481,8 +481,11 @@ def host_enqueue_cost(lwq, dev, n: int = 10000, batch: int = 200) -> dict:
     stream = torch.cuda.Stream(device=dev)
     sp = stream.cuda_stream
     args = (code, W.data_ptr(), x.data_ptr(), y.data_ptr(), M, N, K, sp)
+    import ctypes
+    cfg = lwq.lwq_config()
+    plan_args = (code, M, N, K, ctypes.byref(cfg))
     launches = 0
-    per_call, per_noop = [], []
+    per_call, per_noop, per_plan = [], [], []
     for i in range(-2, n // batch):
         stream.synchronize()
         t0 = time.perf_counter()
@@ -495,12 +498,20 @@ def host_enqueue_cost(lwq, dev, n: int = 10000, batch: int = 200) -> dict:
         for _ in range(batch):
             lib.lwq_version()
         t3 = time.perf_counter()
+        for _ in range(batch):
+            lib.lwq_select_config(*plan_args)
+        t4 = time.perf_counter()
         if i >= 0:
             per_call.append((t1 - t0) / batch * 1e6)
             per_noop.append((t3 - t2) / batch * 1e6)
-    med, noop = statistics.median(per_call), statistics.median(per_noop)
+            per_plan.append((t4 - t3) / batch * 1e6)
+    med, noop, plan = statistics.median(per_call), statistics.median(per_noop), statistics.median(per_plan)
+    # the library's own host work per call: argument checks and the tile choice (lwq_select_config
+    # runs the same checks and planner); the rest of a call is the cached tensor-map lookup and the
+    # CUDA launch itself
     return {"median_us_per_call": round(med, 3), "ctypes_noop_us": round(noop, 3),
-            "library_us_per_call": round(med - noop, 3), "calls": n, "kernels_per_call": launches,
+            "library_us_per_call": round(med - noop, 3), "dispatch_us_per_call": round(plan - noop, 3),
+            "calls": n, "kernels_per_call": launches,
             "call": {"fmt": fmt, "act": act, "M": M, "N": N, "K": K}}
 
 

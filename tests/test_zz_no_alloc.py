@@ -19,10 +19,12 @@ from gpu_util import TOL_GEMV, to_device
 
 pytestmark = pytest.mark.gpu
 
-CASES = [("q4_k", "f16", 1, 4096, 11008),    # split-K (6 splits)
-         ("q4_0", "f32", 4, 11008, 4096),    # two column tiles, split-K (4 splits)
-         ("q8_0", "f32", 1, 4096, 4096),     # split-K (2 splits)
-         ("q4_0", "bf16", 16, 333, 6144)]    # 16 activation rows, split-K, ragged N
+CASES = [("q4_k", "f16", 1, 4096, 11008),    # split-K
+         ("q4_0", "f32", 4, 11008, 4096),    # two column tiles
+         ("q8_0", "f32", 1, 4096, 4096),
+         ("q4_0", "bf16", 16, 333, 6144),    # 16 activation rows, split-K, ragged N
+         ("q6_k", "f16", 2, 500, 8192),      # per-superblock boxes, split-K
+         ("q5_k", "bf16", 3, 300, 4096)]
 
 
 @pytest.fixture(scope="module")
