@@ -313,7 +313,7 @@ cudaError_t launch_gemv(const CUtensorMap &map, const GemvArgs &a, int ctas, siz
     auto kern = gemv_kernel<FMT, XT, NT, I8>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), smem);
     if (e != cudaSuccess) return e;
-    return launch_k(kern, ctas, GEMV_THREADS, smem, st, a.overlap != 0, map, a);
+    return launch_k(kern, ctas, gemv_threads(FMT, NT), smem, st, a.overlap != 0, map, a);
 }
 
 // NT = n8 column tiles: fp32 activations take 1..3 (3 parts per row, 8 rows

@@ -54,8 +54,15 @@ enum { X_F32 = 0, X_F16 = 1, X_BF16 = 2 };
 constexpr int GEMV_ROWS = 16;                     // weight rows per tile (the MMA's M)
 constexpr int CHUNK = 256;                        // weights per TMA chunk of a row
 constexpr int GEMV_W = 16;                        // compute warps per CTA
-constexpr int GEMV_RED = 2;                       // reducer warps (rows 8j .. 8j + 7 each)
-constexpr int GEMV_THREADS = (GEMV_W + 1 + GEMV_RED) * 32;   // + producer + reducers
+// Reducer warps: two (rows 8j .. 8j + 7 each), or four (rows 4j .. 4j + 3) for
+// the one-scale formats at three n8 tiles (fp32 x with 6..8 activation rows),
+// where the reduction is then the longest stage of a tile.  Four reducers make
+// 21 warps, which caps every thread at 80 registers: the K-quant decoders spill
+// there and lose more than the shorter reduction gains.
+__host__ __device__ constexpr int gemv_red(int fmt, int nt) {
+    return nt == 3 && (fmt == F_Q4_0 || fmt == F_Q8_0) ? 4 : 2;
+}
+__host__ __device__ constexpr int gemv_threads(int fmt, int nt) { return (GEMV_W + 1 + gemv_red(fmt, nt)) * 32; }
 constexpr int GEMV_RSTAGES = 2;                   // depth of the reduction-slot ring
 
 template <int FMT>
@@ -959,19 +966,20 @@ template <int XT>
 struct GemvImpl<F_Q8_0, XT, 1, true> : Q40I8<XT, F_Q8_0> {};
 
 // ------------------------------------------------------------------ kernel
-// blockDim = GEMV_THREADS: warps 0..15 compute, warp 16 produces (TMA), warps
-// 17 and 18 reduce; one CTA per SM (at most 96 registers per thread: 19 warps
-// over four 16K-register sub-partitions).  Every wait is
+// blockDim = gemv_threads(FMT, NT): warps 0..15 compute, warp 16 produces (TMA), the
+// rest reduce; one CTA per SM (at most 96 registers per thread with 19 warps
+// over four 16K-register sub-partitions, 80 with 21).  Every wait is
 // bounded; a wait that gives up sets a bit of the device error word and ends
 // its warp's loop.
 template <int FMT, int XT, int NT, bool I8>
-__global__ void __launch_bounds__(GEMV_THREADS, 1)
+__global__ void __launch_bounds__(gemv_threads(FMT, NT), 1)
     gemv_kernel(const __grid_constant__ CUtensorMap wmap, const GemvArgs a) {
     constexpr int CB = FmtInfo<FMT>::chunk_bytes;
     constexpr int KW = I8 ? 256 : gemv_kw(NT);
     constexpr int WPC = CHUNK / KW;            // compute warps per chunk
     constexpr int P = gemv_parts(XT, I8);
     constexpr int RS = gemv_rs(NT);            // floats per row of a reduction slot
+    constexpr int RED = gemv_red(FMT, NT);
     extern __shared__ __align__(128) uint8_t smem[];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1007,7 +1015,7 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1)
         }
         for (int s = 0; s < GEMV_RSTAGES; ++s) {
             mbar_init(&redfull[s], nact > 0 ? nact : 1);
-            mbar_init(&redempty[s], GEMV_RED);
+            mbar_init(&redempty[s], RED);
         }
         mbar_init(xfull, 1);
         fence_mbar_init();
@@ -1058,9 +1066,9 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1)
 
     if (warp > GEMV_W) {
         // ---------------- reducers: touch y and the workspace only after the
-        // preceding work has completed.  Reducer j takes rows 8j .. 8j + 7 of
-        // each tile; lane (row, column group) sums the compute warps' 4-column
-        // groups in warp order (deterministic), then the parts of each
+        // preceding work has completed.  Reducer j takes RR rows of each tile
+        // from row RR j; lane (row, column group) sums the compute warps'
+        // 4-column groups in warp order (deterministic), then the parts of each
         // activation row.
         const int j = warp - GEMV_W - 1;
         pdl_wait();
@@ -1074,7 +1082,8 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1)
                           (uint32_t)(nk * XE), xfull);
         }
         __syncwarp();
-        const int row = 8 * j + (lane & 7), cgl = lane >> 3;
+        constexpr int RR = GEMV_ROWS / RED, NCG = 32 / RR;   // rows per reducer, column groups in parallel
+        const int row = RR * j + (lane % RR), cgl = lane / RR;
         float *dst = (S == 1) ? a.y : a.partial + (size_t)split * M * N;
         int r = 0;
         uint32_t rph = 0;
@@ -1083,8 +1092,8 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1)
             const uint32_t rs0 = smem_u32(red) + (uint32_t)(r * GEMV_W * GEMV_ROWS * RS * 4);
             const int n = tile * GEMV_ROWS + row;
 #pragma unroll
-            for (int k = 0; k < (2 * NT + 3) / 4; ++k) {
-                const int cg = cgl + 4 * k;
+            for (int k = 0; k < (2 * NT + NCG - 1) / NCG; ++k) {
+                const int cg = cgl + NCG * k;
                 if (cg < 2 * NT) {
                     const uint32_t addr = rs0 + (uint32_t)((row * RS + 4 * cg) * 4);
                     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1116,8 +1125,8 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1)
             }
             if constexpr (P > 1) {
                 __syncwarp();
-                for (int o = lane; o < 8 * M; o += 32) {
-                    const int rr = 8 * j + (o & 7), m = o >> 3, nn = tile * GEMV_ROWS + rr;
+                for (int o = lane; o < RR * M; o += 32) {
+                    const int rr = RR * j + (o % RR), m = o / RR, nn = tile * GEMV_ROWS + rr;
                     const float *sp = scratch + rr * RS + m * P;
                     const float val = (sp[0] + sp[1]) + sp[2];
                     if (nn < N) dst[(size_t)m * N + nn] = val;
