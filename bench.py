@@ -92,11 +92,10 @@ def step_calls(workload: str):
     weight of concatenated rows: equal parts, one per seed (see call_weights)."""
     spec = inputs.WORKLOADS[workload]
     calls = []
-    if workload.startswith("q4_k_7b_layer_decode"):
-        for (N, K), seed in zip(spec["shapes"], spec["seeds"]):
-            calls.append((spec["fmt"], spec["act"], 1, N, K, seed))
-    elif workload == "q4_0_prefill_gemm":
-        for M, (N, K), seed in zip(spec["Ms"], spec["shapes"], spec["seeds"]):
+    if len(spec["shapes"]) > 1:
+        # one call per shape (a single M serves every shape)
+        Ms = spec["Ms"] if len(spec["Ms"]) == len(spec["shapes"]) else spec["Ms"] * len(spec["shapes"])
+        for M, (N, K), seed in zip(Ms, spec["shapes"], spec["seeds"]):
             calls.append((spec["fmt"], spec["act"], M, N, K, seed))
     else:
         (N, K), = spec["shapes"]
@@ -112,6 +111,11 @@ def call_weights(fmt: str, N: int, K: int, seed):
         n = N // len(seed)
         return np.concatenate([inputs.make_weights(fmt, inputs.rng(s), n, K) for s in seed], axis=0)
     return inputs.make_weights(fmt, inputs.rng(seed), N, K)
+
+
+def call_path(lwq, fmt: str, act: str, M: int, N: int, K: int) -> str:
+    """The kernel family the library picks for a call."""
+    return {1: "gemv", 2: "gemm", 3: "simple"}[lwq.lwq_select_config(call_fmt(lwq, fmt, act), M, N, K).path]
 
 
 def base_act(act: str) -> str:
@@ -662,7 +666,7 @@ def run_gpu_arm(args):
         p2, _, ms2, lps2, per2 = time_workload(lwq, wl, dev, args.extra_steps, 3, dist_on)
         rec = {"steps": args.extra_steps, "ms_per_step": round(ms2 / args.extra_steps, 5),
                "launches_per_step": lps2}
-        if wl == "q4_0_prefill_gemm":
+        if wl.endswith("prefill_gemm"):
             tflops = p2.flops_per_step * args.extra_steps / (ms2 / 1e3) / 1e12
             rec.update({"value": round(tflops, 2), "unit": "TFLOP/s",
                         "frac_of_bf16_peak": round(tflops / peaks["bf16_tflops"], 4),
@@ -675,7 +679,8 @@ def run_gpu_arm(args):
             rec.update({"value": round(gbs, 1), "unit": "GB/s", "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
                         "per_call": [{"M": p["call"][2], "N": p["call"][3], "K": p["call"][4],
                                       "ms": round(p["ms_mean"], 5),
-                                      "GB/s": round(call_bytes(*p["call"][:5]) / p["ms_mean"] / 1e6, 1)}
+                                      "GB/s": round(call_bytes(*p["call"][:5]) / p["ms_mean"] / 1e6, 1),
+                                      "path": call_path(lwq, *p["call"][:5])}
                                      for p in per2]})
         extra[wl] = rec
 
@@ -809,7 +814,9 @@ def parse_args(argv=None):
     ap.add_argument("--extra-steps", type=int, default=400)
     ap.add_argument("--extra", nargs="*", default=["q8_0_gemv_4096x4096", "q4_k_7b_layer_decode",
                                                    "q4_k_7b_layer_decode_fused", "q4_0_gemv_11008x4096_act_i8",
-                                                   "q4_0_prefill_gemm"])
+                                                   "q4_0_prefill_gemm", "q6_k_7b_layer_decode",
+                                                   "q5_k_7b_layer_decode", "q2_k_7b_layer_decode",
+                                                   "q6_k_prefill_gemm", "q5_k_prefill_gemm"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="leave the format x batch sweep out of the line")
     ap.add_argument("--no-host-cost", action="store_true", help="leave the host enqueue timing out")

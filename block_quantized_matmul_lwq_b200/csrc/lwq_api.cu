@@ -127,23 +127,27 @@ struct Plan {
 inline int gemv_nt(int xt, bool i8, int mg) { return i8 ? 1 : (mg * gemv_parts(xt, i8) + 7) / 8; }
 // bytes of one row of a chunk in a GEMV stage (Q6_K: its 240-byte box, see FmtInfo)
 inline int gemv_chunk_bytes(int wf) {
-    return wf == LWQ_Q8_0 ? 272 : (wf == LWQ_Q5_K ? 176 : (wf == LWQ_Q6_K ? 240 : 144));
+    return wf == LWQ_Q8_0 ? 272 : (wf == LWQ_Q5_K ? 176 : (wf == LWQ_Q6_K ? 240 : (wf == LWQ_Q2_K ? 84 : 144)));
 }
 inline size_t gemv_smem(int wf, int cps, int stages, int nt, bool i8, int xt, int m) {
-    return gemv_smem_layout(gemv_chunk_bytes(wf), cps, stages, nt, wf == LWQ_Q4_K || wf == LWQ_Q5_K,
-                            gemv_parts(xt, i8), m,
-                            xt == X_F32 ? 4 : 2, i8)
+    // the library's format codes equal the kernels' (LWQ_Q8_0 == F_Q8_0, ...)
+    return gemv_smem_layout(gemv_chunk_bytes(wf), cps, stages, nt, fmt_sums(wf), gemv_parts(xt, i8), m,
+                            xt == X_F32 ? 4 : 2, i8, fmt_row_slots(wf))
         .total;
 }
 
 // Formats with a tensor-core GEMV decoder (their packed rows are 16-byte
 // multiples, as the weight stream's tensor map needs); the others take the
 // simple kernel.
-bool tc_gemv_format(int wf) { return wf == LWQ_Q8_0 || wf == LWQ_Q4_0 || wf == LWQ_Q4_K || wf == LWQ_Q5_K; }
+bool tc_gemv_format(int wf) {
+    return wf == LWQ_Q8_0 || wf == LWQ_Q4_0 || wf == LWQ_Q4_K || wf == LWQ_Q5_K || wf == LWQ_Q2_K;
+}
 // Q6_K rows are 210 bytes per superblock: the tensor map needs a 16-byte row
-// stride, so K a multiple of 2048 (8 superblocks)
-bool tc_gemv_eligible(int wf, long K) {
+// stride, so K a multiple of 2048 (8 superblocks).  Q2_K streams row slots of
+// the flat matrix, whose tensor map needs the whole matrix to be 16-byte units.
+bool tc_gemv_eligible(int wf, long N, long K) {
     if (wf == LWQ_Q6_K) return K % 2048 == 0;
+    if (wf == LWQ_Q2_K) return K % 256 == 0 && (N * (K / 256) * 84) % 16 == 0;
     return tc_gemv_format(wf) && K % 256 == 0;
 }
 
@@ -166,7 +170,7 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
     if (!path) {
         if (M > 16 && xt != X_F32 && gemm_eligible(wf, xt, K))
             path = 2;
-        else if (tc_gemv_eligible(wf, K))
+        else if (tc_gemv_eligible(wf, N, K))
             path = 1;
         else
             path = 3;
@@ -195,7 +199,7 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
         p->cfg.splits = 1;
         return LWQ_OK;
     }
-    if (path != 1 || !tc_gemv_eligible(wf, K)) return LWQ_ERR_UNSUPPORTED;
+    if (path != 1 || !tc_gemv_eligible(wf, N, K)) return LWQ_ERR_UNSUPPORTED;
     p->i8 = (fmt & LWQ_FLAG_ACT_I8) != 0;
     // int8 activation blocks: Q4_0 and Q8_0 weights, any M (passes of 8 rows; every pass streams
     // the weights again, so a prefill-sized M reads them M / 8 times)
@@ -354,6 +358,7 @@ cudaError_t dispatch_gemv(int wf, int xt, int nt, bool i8, const CUtensorMap &ma
     case LWQ_Q4_K: { LWQ_GV(F_Q4_K) }
     case LWQ_Q5_K: { LWQ_GV(F_Q5_K) }
     case LWQ_Q6_K: { LWQ_GV(F_Q6_K) }
+    case LWQ_Q2_K: { LWQ_GV(F_Q2_K) }
     }
 #undef LWQ_GV
     return cudaErrorInvalidValue;
@@ -438,6 +443,17 @@ MapReq map_req(const void *p, CUtensorMapDataType dtype, int rank, CUtensorMapSw
 // chunk), strides (row_bytes, chunk_bytes); a box of (all words, 16 rows, cps
 // chunks) lands as cps consecutive [16 rows][chunk bytes] boxes, one GEMV stage.
 int encode_weight_map(CUtensorMap *map, const void *Wq, int wf, int N, long rb, int cps) {
+    if (wf == LWQ_Q2_K) {
+        // row slots: the flat matrix as [N rb / 16 units][16 bytes], a box of whole units
+        // covering one row's slice of a split and up to 7 units before it
+        MapReq r = map_req(Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, CU_TENSOR_MAP_SWIZZLE_NONE);
+        r.dims[0] = 16;
+        r.dims[1] = (cuuint64_t)((long)N * rb / 16);
+        r.strides[0] = 16;
+        r.box[0] = 16;
+        r.box[1] = (cuuint32_t)gemv_slot_units(84, cps);
+        return encode_cached(r, map);
+    }
     if (wf == LWQ_Q6_K) {
         // [N rows][rb / 2 words] with a box of [16 rows][120 words], one per chunk
         MapReq r = map_req(Wq, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, CU_TENSOR_MAP_SWIZZLE_NONE);

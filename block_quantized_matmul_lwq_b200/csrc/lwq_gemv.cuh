@@ -80,8 +80,31 @@ struct FmtInfo<F_Q5_K> { static constexpr int chunk_bytes = 176; };
 // or below the superblock, which lies 2 * ((105 c) & 7) bytes into the box.
 template <>
 struct FmtInfo<F_Q6_K> { static constexpr int chunk_bytes = 240; };
-// formats with a per-sub-block min (the S_j sums of x enter the result)
-__host__ __device__ constexpr bool fmt_has_min(int fmt) { return fmt == F_Q4_K || fmt == F_Q5_K; }
+// Q2_K superblocks are 84 bytes: a row of K = 11008 (3612 bytes) is not a
+// 16-byte multiple, so no tensor map can take the rows as its second
+// dimension.  Its weights stream as row slots instead (fmt_row_slots).
+template <>
+struct FmtInfo<F_Q2_K> { static constexpr int chunk_bytes = 84; };
+// Formats with a per-sub-block min (the S_j sums of x enter the result), and
+// the number of those sums per 256-weight chunk (sub-blocks of 32 or 16).
+__host__ __device__ constexpr int fmt_sums(int fmt) {
+    return (fmt == F_Q4_K || fmt == F_Q5_K) ? 8 : (fmt == F_Q2_K ? 16 : 0);
+}
+__host__ __device__ constexpr bool fmt_has_min(int fmt) { return fmt_sums(fmt) > 0; }
+// Row slots: the weight matrix is read as one flat array of 16-byte units (a
+// tensor map of [bytes / 16][16]); per stage, row r of the tile is one box of
+// whole units into its own 128-byte aligned slot, starting r mod 8 units before
+// the unit that holds the row's first byte of the split.  The slice then lies
+// 16 (r mod 8) + ((n rb + 84 c) mod 16) bytes into the slot -- the second term
+// 0, 4, 8 or 12, so 32-bit words stay aligned -- and the 8 rows that a warp's
+// lane groups read at once fall on distinct bank quads.
+__host__ __device__ constexpr bool fmt_row_slots(int fmt) { return fmt == F_Q2_K; }
+__host__ __device__ constexpr int gemv_slot_units(int chunk_bytes, int cps) {   // units per row box
+    return (chunk_bytes * cps + 12 + 15) / 16 + 7;
+}
+__host__ __device__ constexpr int gemv_slot_bytes(int chunk_bytes, int cps) {   // slot stride
+    return (16 * gemv_slot_units(chunk_bytes, cps) + 127) / 128 * 128;
+}
 
 struct GemvArgs {
     const void *x;
@@ -120,19 +143,22 @@ constexpr int GEMV_XPAD = 16;
 //  * The slice of x (fp path): P planes [part][activation row][K slice + pad]
 //    of 16-bit values -- the bf16 parts of fp32 x, or 16-bit x as it is.
 //    Int8 activation blocks stage the raw slice [row][K slice].
-//  * The Q4_K sums: [activation row][32-weight sub-block of the slice] fp32.
+//  * The K-quant sums: [activation row][sub-block of the slice] fp32 (sub-blocks
+//    of 32 weights; Q2_K: 16).
 struct GemvSmem {
-    size_t stage, ring, xs, red, sx, scratch, xmax, bars, total;
+    size_t stage, slot, tx, ring, xs, red, sx, scratch, xmax, bars, total;   // tx: bytes a stage's loads bring
 };
-__host__ __device__ inline GemvSmem gemv_smem_layout(int chunk_bytes, int cps, int wstages, int nt, bool q4k,
-                                                     int parts, int m, int xelem, bool i8) {
+__host__ __device__ inline GemvSmem gemv_smem_layout(int chunk_bytes, int cps, int wstages, int nt, int sums,
+                                                     int parts, int m, int xelem, bool i8, bool slots) {
     GemvSmem s;
-    s.stage = (size_t)cps * GEMV_ROWS * chunk_bytes;
+    s.slot = slots ? (size_t)gemv_slot_bytes(chunk_bytes, cps) : 0;
+    s.stage = slots ? GEMV_ROWS * s.slot : (size_t)cps * GEMV_ROWS * chunk_bytes;
+    s.tx = slots ? (size_t)GEMV_ROWS * 16 * gemv_slot_units(chunk_bytes, cps) : s.stage;
     s.ring = (size_t)wstages * s.stage;
     s.xs = i8 ? (size_t)m * cps * CHUNK * xelem : (size_t)parts * m * (cps * CHUNK + GEMV_XPAD) * 2;
     s.xs = (s.xs + 15) & ~(size_t)15;
     s.red = (size_t)GEMV_RSTAGES * GEMV_W * GEMV_ROWS * gemv_rs(nt) * 4;
-    s.sx = q4k ? (size_t)m * cps * (CHUNK / 32) * 4 : 0;
+    s.sx = (size_t)m * cps * sums * 4;
     s.scratch = parts > 1 ? (size_t)GEMV_ROWS * gemv_rs(nt) * 4 : 0;
     s.xmax = 16 * 4;
     s.bars = (size_t)(2 * wstages + 2 * GEMV_RSTAGES + 1) * 8;
@@ -194,6 +220,12 @@ __device__ __forceinline__ uint32_t q5k_pair(uint32_t v) {
     if constexpr (BF) return hfma2_bf16(and_or(v, 0x001F001Fu, B2_MAGIC), B2_ONE, B2_M128);
     else return hfma2_f16(and_or(v, 0x001F001Fu, H2_MAGIC), H2_ONE, H2_M1024);
 }
+// Q2_K: the 2-bit codes in bits 0-1 of bytes 0 and 2, unsigned.
+template <bool BF>
+__device__ __forceinline__ uint32_t q2k_pair(uint32_t v) {
+    if constexpr (BF) return hfma2_bf16(and_or(v, 0x00030003u, B2_MAGIC), B2_ONE, B2_M128);
+    else return hfma2_f16(and_or(v, 0x00030003u, H2_MAGIC), H2_ONE, H2_M1024);
+}
 // Q8_0: the int8 codes of bytes 0 and 2.  fp16: (1024 + (q + 128)) - 1152.
 // bf16 has room for 7 bits only: (128 + (q & 127)) plus -128 or -256 from the
 // sign bit, which lands on the exponent bit of 0xC300 (0xC380 is -256).
@@ -251,7 +283,8 @@ __device__ __forceinline__ float byte_magic(uint32_t v, int jj) {
 //    the last two code bytes of the block in its place (one PRMT).
 template <int FMT>
 __device__ __forceinline__ int elem(int bb, int h, int t, int q) {
-    if (FMT == F_Q4_K || FMT == F_Q5_K || FMT == F_Q6_K || (bb & 1)) return 32 * bb + 16 * h + 4 * t + 2 * q;
+    if (FMT == F_Q4_K || FMT == F_Q5_K || FMT == F_Q6_K || FMT == F_Q2_K || (bb & 1))
+        return 32 * bb + 16 * h + 4 * t + 2 * q;
     if (FMT == F_Q4_0) return 32 * bb + 16 * h + ((4 * t - 2 + 2 * q) & 15);
     return 32 * bb + ((16 * h + 4 * t - 2 + 2 * q) & 31);
 }
@@ -265,6 +298,7 @@ struct Exact {
     uint32_t xf[NT][NB][2][2];               // [tile][block][step][reg]
     float inv;                               // 1 / the activation scale (a power of two)
     uint32_t q6o = 0;                        // Q6_K: byte offset of the superblock in its chunk box
+    uint32_t q2r0 = 0, q2r1 = 0;             // Q2_K: the superblock in rows g and g + 8 of the stage
 
     // ---------------------------------------------------------- prologue
     // The CTA's slice of x is prepared once, by all nact compute warps
@@ -323,11 +357,16 @@ struct Exact {
 
     // Q4_K: the sum of a 32-element sub-block lies in 8 consecutive lanes (4
     // elements each; a group of 8 lanes is valid or not as a whole).
+    // Q2_K: of a 16-element sub-block, in 4 consecutive lanes.
     __device__ static __forceinline__ void store_sum(float v, const Slice &S, long e, bool ok, int lane) {
         v += __shfl_xor_sync(0xffffffffu, v, 1);
         v += __shfl_xor_sync(0xffffffffu, v, 2);
-        v += __shfl_xor_sync(0xffffffffu, v, 4);
-        if (ok && (lane & 7) == 0) S.sx[e / 32] = v;   // row-major [M][nk/32] == element index / 32
+        if constexpr (FMT == F_Q2_K) {
+            if (ok && (lane & 3) == 0) S.sx[e / 16] = v;   // row-major [M][nk/16] == element index / 16
+        } else {
+            v += __shfl_xor_sync(0xffffffffu, v, 4);
+            if (ok && (lane & 7) == 0) S.sx[e / 32] = v;   // row-major [M][nk/32] == element index / 32
+        }
     }
 
     // |v| outside [2^-60, 2^60] and not zero (or not finite): the slice needs the power-of-two scale
@@ -585,6 +624,78 @@ struct Exact {
         }
     }
 
+    // Q2_K (84-byte superblock = the warp's chunk; with KW = 128 the warp takes
+    // half `half` of it).  Rows g and g + 8 lie at box + q2r0 and box + q2r1
+    // (row slots).  Sub-block 8n + 2j + h (16 weights: elements 128n + 32j +
+    // 16h ..) has its codes in bits 2j, 2j+1 of qs[32n + 16h ..]: lane t's word
+    // qs[32n + 16h + 4t ..] gives elements 4t .. 4t + 3 of it, bytes 0 and 2
+    // shifted by 2j into the even pair, bytes 1 and 3 by 2j + 8 into the odd
+    // one.  One MMA step per sub-block, then y += d * sc * C; the mins enter
+    // once per tile, y -= dmin * sum m S over the part-0 columns.
+    __device__ __forceinline__ void compute_q2(uint32_t box, int half, float (&acc)[NT][4], int t, int M,
+                                               const float *sxw, int sstride) const {
+        const uint32_t r0 = box + q2r0, r1 = box + q2r1;
+        const uint32_t h0 = lds32(r0 + 80), h1 = lds32(r1 + 80);   // d | dmin
+        const float d0 = f16_lo(h0), d1 = f16_lo(h1);
+        const float nd0 = d0 * -8388608.f, nd1 = d1 * -8388608.f;   // -2^23 d (exact)
+        constexpr int NH = NB / 4;                                    // halves of the superblock: 2 or 1
+        uint32_t sc[NH][2][2];                                        // [half][row][word]: s[8n .. 8n + 7]
+#pragma unroll
+        for (int hh = 0; hh < NH; ++hh) {
+            const int n = NH == 2 ? hh : half;
+            sc[hh][0][0] = lds32(r0 + 8 * n);
+            sc[hh][0][1] = lds32(r0 + 8 * n + 4);
+            sc[hh][1][0] = lds32(r1 + 8 * n);
+            sc[hh][1][1] = lds32(r1 + 8 * n + 4);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t W0 = lds32(r0 + 16 + 32 * n + 16 * h + 4 * t);
+                const uint32_t W1 = lds32(r1 + 16 + 32 * n + 16 * h + 4 * t);
+                const uint32_t V0 = W0 >> 8, V1 = W1 >> 8;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int sb = 2 * j + h;   // scale byte of the sub-block in s[8n ..]
+                    const float s0 = fmaf(byte_magic(sc[hh][0][sb >> 2] & 0x0F0F0F0Fu, sb & 3), d0, nd0);   // d * sc
+                    const float s1 = fmaf(byte_magic(sc[hh][1][sb >> 2] & 0x0F0F0F0Fu, sb & 3), d1, nd1);
+                    const uint32_t a[4] = {q2k_pair<BF>(W0 >> (2 * j)), q2k_pair<BF>(W1 >> (2 * j)),
+                                           q2k_pair<BF>(V0 >> (2 * j)), q2k_pair<BF>(V1 >> (2 * j))};
+                    const int bl = 4 * hh + j;   // the warp's 32-element block: step h of it
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        float c[4];
+                        mma_zero<BF>(c, a, xf[nt][bl][h][0], xf[nt][bl][h][1]);
+                        acc[nt][0] = fmaf(s0, c[0], acc[nt][0]);
+                        acc[nt][1] = fmaf(s0, c[1], acc[nt][1]);
+                        acc[nt][2] = fmaf(s1, c[2], acc[nt][2]);
+                        acc[nt][3] = fmaf(s1, c[3], acc[nt][3]);
+                    }
+                }
+            }
+        }
+        // mins: the warp's sub-blocks q = 0 .. 2 NB - 1 in element order are s bytes
+        // 8n + q (n = the warp's first half), sums sxw[m * sstride + q]
+        const float m0f = f16_hi(h0), m1f = f16_hi(h1);
+        const float nm0 = m0f * -8388608.f, nm1 = m1f * -8388608.f;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c = 8 * nt + 2 * t + cc, m = c / P;
+                if (c - m * P != 0 || m >= M) continue;
+                float z0 = 0.f, z1 = 0.f;
+#pragma unroll
+                for (int q = 0; q < 2 * NB; ++q) {
+                    const uint32_t w0 = (sc[q >> 3][0][(q >> 2) & 1] >> 4) & 0x0F0F0F0Fu;
+                    const uint32_t w1 = (sc[q >> 3][1][(q >> 2) & 1] >> 4) & 0x0F0F0F0Fu;
+                    const float sj = sxw[m * sstride + q];
+                    z0 = fmaf(fmaf(byte_magic(w0, q & 3), m0f, nm0), sj, z0);   // (dmin * m) * S
+                    z1 = fmaf(fmaf(byte_magic(w1, q & 3), m1f, nm1), sj, z1);
+                }
+                acc[nt][cc] -= z0;
+                acc[nt][2 + cc] -= z1;
+            }
+    }
+
     // box: this warp's chunk, row 0, in the stage; half: which half of the
     // chunk (KW = 128); sxw: the x sums of this warp's first sub-block, rows
     // sstride apart (Q4_K).
@@ -612,6 +723,8 @@ struct Exact {
                     block(a0, a1, 2 * pp + 1, f16_hi(v0), f16_hi(v1), acc);
                 }
             }
+        } else if constexpr (FMT == F_Q2_K) {
+            compute_q2(box, half, acc, t, M, sxw, sstride);
         } else if constexpr (FMT == F_Q6_K) {
             if (q6o & 2) compute_q6<true>(r0, r1, half, acc, t);
             else compute_q6<false>(r0, r1, half, acc, t);
@@ -995,7 +1108,7 @@ __global__ void __launch_bounds__(gemv_threads(FMT, NT), 1)
     constexpr int XE = (XT == X_F32) ? 4 : 2;
     // the reducer stages x raw with bulk copies, except fp32 x on the fp path (the compute warps split it)
     constexpr bool STAGE = I8 || XT != X_F32;
-    const GemvSmem L = gemv_smem_layout(CB, a.cps, ws, NT, fmt_has_min(FMT), P, a.M, XE, I8);
+    const GemvSmem L = gemv_smem_layout(CB, a.cps, ws, NT, fmt_sums(FMT), P, a.M, XE, I8, fmt_row_slots(FMT));
     uint8_t *ring = smem;
     uint8_t *xs = smem + L.ring;
     float *red = reinterpret_cast<float *>(xs + L.xs);
@@ -1042,8 +1155,19 @@ __global__ void __launch_bounds__(gemv_threads(FMT, NT), 1)
                 if (it > 0 && it < ws && !mbar_wait(&full[it - 1], 0u, a.timeout_ns, DEVERR_GEMV_WAIT)) break;
                 // one 3-D box per stage: [chunks of this split][16 rows][chunk bytes]; the
                 // last split's box may run past the last chunk, where it reads zeros
-                mbar_arrive_expect_tx(&full[s], (uint32_t)L.stage);
-                if constexpr (FMT == F_Q6_K) {
+                mbar_arrive_expect_tx(&full[s], (uint32_t)L.tx);
+                if constexpr (fmt_row_slots(FMT)) {
+                    // one box per row of the tile: whole 16-byte units from r mod 8 units before
+                    // the one holding the row's first byte of this split (rows past the end
+                    // read zeros; row 0, the only one that could start before the matrix, starts
+                    // at its own unit)
+                    const long rb = (long)a.nchunks * CB;
+                    for (int r = 0; r < GEMV_ROWS; ++r) {
+                        const long b0 = (long)(tile * GEMV_ROWS + r) * rb + (long)c_begin * CB;
+                        tma_load_2d(ring + (size_t)s * L.stage + (size_t)r * L.slot, &wmap, &full[s], 0,
+                                    (int)((b0 >> 4) - (r & 7)));
+                    }
+                } else if constexpr (FMT == F_Q6_K) {
                     // one 2-D box per chunk, [16 rows][120 words] from the 16-byte boundary at or
                     // below the superblock (chunks past the end read zeros)
                     for (int ci = 0; ci < a.cps; ++ci)
@@ -1159,8 +1283,9 @@ __global__ void __launch_bounds__(gemv_threads(FMT, NT), 1)
     if (!impl.prologue(a, sl, c_begin, xfull, nact, warp, lane, a.timeout_ns)) return;
     impl.load_frags(sl, ci * CHUNK, half, lane);
     if constexpr (FMT == F_Q6_K && !I8) impl.q6o = 2u * (uint32_t)((105 * (c_begin + ci)) & 7);
-    const float *sxw = sx + ci * (CHUNK / 32) + half * (KW / 32);
-    const int sstride = nk / 32;
+    constexpr int SUB = FMT == F_Q2_K ? 16 : 32;   // weights per sum of x
+    const float *sxw = sx + ci * (CHUNK / SUB) + half * (KW / SUB);
+    const int sstride = nk / SUB;
     const int g = lane >> 2, t = lane & 3;
     int s = 0, r = 0, rit = 0;
     uint32_t ph = 0, rph = 0;
@@ -1171,8 +1296,18 @@ __global__ void __launch_bounds__(gemv_threads(FMT, NT), 1)
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int j = 0; j < 4; ++j) acc[nt][j] = 0.f;
-        impl.compute(smem_u32(ring) + (uint32_t)((size_t)s * L.stage + (size_t)ci * GEMV_ROWS * CB), half, acc, lane,
-                     a.M, sxw, sstride);
+        uint32_t box;
+        if constexpr (fmt_row_slots(FMT)) {
+            // rows g and g + 8 of the tile: their slots, the slice's offset in them, this warp's chunk
+            const long rb = (long)a.nchunks * CB;
+            const long b0 = (long)(tile * GEMV_ROWS + g) * rb + (long)c_begin * CB, b1 = b0 + 8 * rb;
+            impl.q2r0 = (uint32_t)(g * L.slot + 16 * g) + (uint32_t)(b0 & 15) + (uint32_t)(ci * CB);
+            impl.q2r1 = (uint32_t)((g + 8) * L.slot + 16 * g) + (uint32_t)(b1 & 15) + (uint32_t)(ci * CB);
+            box = smem_u32(ring) + (uint32_t)((size_t)s * L.stage);
+        } else {
+            box = smem_u32(ring) + (uint32_t)((size_t)s * L.stage + (size_t)ci * GEMV_ROWS * CB);
+        }
+        impl.compute(box, half, acc, lane, a.M, sxw, sstride);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
         if (++s == ws) {

@@ -292,6 +292,19 @@ WORKLOADS = {
     "q4_0_gemv_11008x4096_act_i8": dict(fmt="q4_0", act="f32:i8", Ms=[1, 4, 8], shapes=[(11008, 4096)], seeds=[0]),
     "q4_0_prefill_gemm": dict(fmt="q4_0", act="bf16", Ms=[512, 2048],
                               shapes=[(11008, 4096), (4096, 11008)], seeds=[0, 0]),
+    # the other K-quant formats over the same 7B layer (fp16 activations, one token)
+    "q6_k_7b_layer_decode": dict(fmt="q6_k", act="f16", Ms=[1],
+                                 shapes=[(4096, 4096)] * 4 + [(11008, 4096), (11008, 4096), (4096, 11008)],
+                                 seeds=[0, 1, 2, 3, 4, 5, 6]),
+    "q5_k_7b_layer_decode": dict(fmt="q5_k", act="f16", Ms=[1],
+                                 shapes=[(4096, 4096)] * 4 + [(11008, 4096), (11008, 4096), (4096, 11008)],
+                                 seeds=[0, 1, 2, 3, 4, 5, 6]),
+    "q2_k_7b_layer_decode": dict(fmt="q2_k", act="f16", Ms=[1],
+                                 shapes=[(4096, 4096)] * 4 + [(11008, 4096), (11008, 4096), (4096, 11008)],
+                                 seeds=[0, 1, 2, 3, 4, 5, 6]),
+    # and their prefill GEMM at the up-projection shape (bf16 activations, 512 tokens)
+    "q6_k_prefill_gemm": dict(fmt="q6_k", act="bf16", Ms=[512], shapes=[(11008, 4096)], seeds=[0]),
+    "q5_k_prefill_gemm": dict(fmt="q5_k", act="bf16", Ms=[512], shapes=[(11008, 4096)], seeds=[0]),
 }
 
 # Decode attention workloads: one query token per sequence against its key/value cache.

@@ -3,8 +3,10 @@
 Q5_K has tensor-core decoders (the GEMV and the tcgen05 GEMM).  Q6_K and Q2_K
 superblocks are 210 and 84 bytes, so their rows are not 16-byte multiples in
 general: Q6_K takes the tensor-core GEMV when K is a multiple of 2048 and the
-simple kernel otherwise; Q2_K always takes the simple kernel.  Every case is scored
-element by element against the oracle on the same seeded inputs.
+simple kernel otherwise; Q2_K takes the tensor-core GEMV, its rows streamed as
+slots of the flat matrix, whenever the whole matrix is a 16-byte multiple (N * K
+/ 256 * 84), else the simple kernel.  Every case is scored element by element
+against the oracle on the same seeded inputs.
 """
 
 import ctypes
@@ -76,6 +78,32 @@ def test_q6_k_prefill_gemm_sampled(dev):
     M, N, K = 512, 11008, 4096
     assert lwq.lwq_select_config(lwq.fmt_code("q6_k", "bf16"), M, N, K).path == 2
     check_sampled("q6_k", "bf16", M, N, K, dev, seed=9, count=2000)
+
+
+@pytest.mark.parametrize("a", ACTS)
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 6, 8, 9, 16])
+@pytest.mark.parametrize("K", [256, 1024, 4352, 11008])
+def test_q2_k_tensor_core_gemv(dev, a, M, K):
+    """Q2_K row slots: 44 rows (a 16-byte multiple whatever K), slices that start 0, 4, 8 or 12
+    bytes into their slot, every column layout, a ragged last row tile, split-K at K = 11008."""
+    assert lwq.lwq_select_config(lwq.fmt_code("q2_k", a), M, 44, K).path == 1
+    check_full("q2_k", a, M, 44, K, dev, seed=400 + M + K)
+
+
+@pytest.mark.parametrize("warps,splits,stages", [(1, 0, 2), (3, 0, 2), (8, 2, 3), (4, 3, 2), (16, 0, 4)])
+def test_q2_k_forced_gemv_configs(dev, warps, splits, stages):
+    cfg = lwq.lwq_config()
+    cfg.path, cfg.warps, cfg.splits, cfg.stages = 1, warps, splits, stages
+    check_full("q2_k", "f32", 5, 120, 4352, dev, seed=warps + splits, cfg=cfg)
+
+
+def test_q2_k_routing(dev):
+    """Q2_K takes the tensor-core GEMV when N * row bytes is a 16-byte multiple, else the simple kernel."""
+    f = lwq.fmt_code("q2_k", "f16")
+    assert lwq.lwq_select_config(f, 1, 4096, 11008).path == 1
+    assert lwq.lwq_select_config(f, 1, 37, 11008).path == 3      # 37 x 3612 bytes
+    assert lwq.lwq_select_config(f, 1, 37, 4096).path == 1       # 1344-byte rows
+    check_full("q2_k", "f16", 2, 37, 11008, dev, seed=3)
 
 
 @pytest.mark.parametrize("warps,splits,stages", [(1, 0, 2), (3, 0, 2), (8, 2, 3), (4, 3, 2)])
