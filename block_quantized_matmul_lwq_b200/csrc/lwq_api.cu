@@ -126,13 +126,23 @@ struct Plan {
 // P columns (P = 3 bf16 parts for fp32 activations, else 1), 8 columns per tile.
 inline int gemv_nt(int xt, bool i8, int mg) { return i8 ? 1 : (mg * gemv_parts(xt, i8) + 7) / 8; }
 // bytes of one row of a chunk in a GEMV stage (Q6_K: its 240-byte box, see FmtInfo)
-inline int gemv_chunk_bytes(int wf) {
-    return wf == LWQ_Q8_0 ? 272 : (wf == LWQ_Q5_K ? 176 : (wf == LWQ_Q6_K ? 240 : (wf == LWQ_Q2_K ? 84 : 144)));
+// The GEMV kernel format of a call: the library's format codes equal the
+// kernels' (LWQ_Q8_0 == F_Q8_0, ...), except Q6_K rows that are not 16-byte
+// multiples, which stream as row slots (F_Q6_KS).
+inline int gemv_kfmt(int wf, long K) { return (wf == LWQ_Q6_K && K % 2048 != 0) ? F_Q6_KS : wf; }
+inline int gemv_chunk_bytes(int kf) {
+    switch (kf) {
+    case F_Q8_0: return 272;
+    case F_Q5_K: return 176;
+    case F_Q6_K: return 240;
+    case F_Q6_KS: return 210;
+    case F_Q2_K: return 84;
+    default: return 144;
+    }
 }
-inline size_t gemv_smem(int wf, int cps, int stages, int nt, bool i8, int xt, int m) {
-    // the library's format codes equal the kernels' (LWQ_Q8_0 == F_Q8_0, ...)
-    return gemv_smem_layout(gemv_chunk_bytes(wf), cps, stages, nt, fmt_sums(wf), gemv_parts(xt, i8), m,
-                            xt == X_F32 ? 4 : 2, i8, fmt_row_slots(wf))
+inline size_t gemv_smem(int kf, int cps, int stages, int nt, bool i8, int xt, int m) {
+    return gemv_smem_layout(gemv_chunk_bytes(kf), cps, stages, nt, fmt_sums(kf), gemv_parts(xt, i8), m,
+                            xt == X_F32 ? 4 : 2, i8, fmt_row_slots(kf))
         .total;
 }
 
@@ -140,15 +150,17 @@ inline size_t gemv_smem(int wf, int cps, int stages, int nt, bool i8, int xt, in
 // multiples, as the weight stream's tensor map needs); the others take the
 // simple kernel.
 bool tc_gemv_format(int wf) {
-    return wf == LWQ_Q8_0 || wf == LWQ_Q4_0 || wf == LWQ_Q4_K || wf == LWQ_Q5_K || wf == LWQ_Q2_K;
+    return wf == LWQ_Q8_0 || wf == LWQ_Q4_0 || wf == LWQ_Q4_K || wf == LWQ_Q5_K || wf == LWQ_Q2_K || wf == LWQ_Q6_K;
 }
-// Q6_K rows are 210 bytes per superblock: the tensor map needs a 16-byte row
-// stride, so K a multiple of 2048 (8 superblocks).  Q2_K streams row slots of
+// Q6_K rows are 210 bytes per superblock: with K a multiple of 2048 (8
+// superblocks) they are 16-byte multiples and a tensor map takes them as its
+// rows; otherwise, like Q2_K's 84-byte superblocks, they stream as row slots of
 // the flat matrix, whose tensor map needs the whole matrix to be 16-byte units.
 bool tc_gemv_eligible(int wf, long N, long K) {
-    if (wf == LWQ_Q6_K) return K % 2048 == 0;
-    if (wf == LWQ_Q2_K) return K % 256 == 0 && (N * (K / 256) * 84) % 16 == 0;
-    return tc_gemv_format(wf) && K % 256 == 0;
+    if (K % 256 != 0) return false;
+    if (wf == LWQ_Q6_K) return K % 2048 == 0 || (N * (K / 256) * 210) % 16 == 0;
+    if (wf == LWQ_Q2_K) return (N * (K / 256) * 84) % 16 == 0;
+    return tc_gemv_format(wf);
 }
 
 // Workspace layout: fp32 split-K partials [S][m_group][N].  Nothing in it
@@ -247,11 +259,11 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
     const int mg = p->m_group;
     int stages = force && force->stages ? force->stages : 4;
     if (!(force && force->stages)) {
-        while (stages > 2 && gemv_smem(wf, cps, stages, p->nt, p->i8, xt, mg) > kSmemLimit) --stages;
-        while (cps > 1 && !(force && force->splits) && gemv_smem(wf, cps, stages, p->nt, p->i8, xt, mg) > kSmemLimit)
+        while (stages > 2 && gemv_smem(gemv_kfmt(wf, K), cps, stages, p->nt, p->i8, xt, mg) > kSmemLimit) --stages;
+        while (cps > 1 && !(force && force->splits) && gemv_smem(gemv_kfmt(wf, K), cps, stages, p->nt, p->i8, xt, mg) > kSmemLimit)
             --cps;
     }
-    if (stages < 2 || gemv_smem(wf, cps, stages, p->nt, p->i8, xt, mg) > kSmemLimit) return LWQ_ERR_UNSUPPORTED;
+    if (stages < 2 || gemv_smem(gemv_kfmt(wf, K), cps, stages, p->nt, p->i8, xt, mg) > kSmemLimit) return LWQ_ERR_UNSUPPORTED;
     S = (nchunks + cps - 1) / cps;               // drop empty splits
     const int row_tiles = (N + GEMV_ROWS - 1) / GEMV_ROWS;
     // one CTA per SM
@@ -263,7 +275,7 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
     p->cfg.stages = stages;
     p->cfg.splits = S;
     p->cfg.ctas = S * groups;
-    p->smem = gemv_smem(wf, cps, stages, p->nt, p->i8, xt, mg);
+    p->smem = gemv_smem(gemv_kfmt(wf, K), cps, stages, p->nt, p->i8, xt, mg);
     p->ws_need = splitk_ws(S, p->m_group, N);
     return LWQ_OK;
 }
@@ -357,7 +369,10 @@ cudaError_t dispatch_gemv(int wf, int xt, int nt, bool i8, const CUtensorMap &ma
     case LWQ_Q8_0: { LWQ_GV(F_Q8_0) }
     case LWQ_Q4_K: { LWQ_GV(F_Q4_K) }
     case LWQ_Q5_K: { LWQ_GV(F_Q5_K) }
-    case LWQ_Q6_K: { LWQ_GV(F_Q6_K) }
+    case LWQ_Q6_K: {
+        if (a.K % 2048 != 0) { LWQ_GV(F_Q6_KS) }
+        LWQ_GV(F_Q6_K)
+    }
     case LWQ_Q2_K: { LWQ_GV(F_Q2_K) }
     }
 #undef LWQ_GV
@@ -442,8 +457,9 @@ MapReq map_req(const void *p, CUtensorMapDataType dtype, int rank, CUtensorMapSw
 // The GEMV's view of Wq: 3-D, (8-byte word of a 256-weight chunk, weight row,
 // chunk), strides (row_bytes, chunk_bytes); a box of (all words, 16 rows, cps
 // chunks) lands as cps consecutive [16 rows][chunk bytes] boxes, one GEMV stage.
-int encode_weight_map(CUtensorMap *map, const void *Wq, int wf, int N, long rb, int cps) {
-    if (wf == LWQ_Q2_K) {
+int encode_weight_map(CUtensorMap *map, const void *Wq, int wf, int N, long K, long rb, int cps) {
+    const int kf = gemv_kfmt(wf, K);
+    if (fmt_row_slots(kf)) {
         // row slots: the flat matrix as [N rb / 16 units][16 bytes], a box of whole units
         // covering one row's slice of a split and up to 7 units before it
         MapReq r = map_req(Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -451,7 +467,7 @@ int encode_weight_map(CUtensorMap *map, const void *Wq, int wf, int N, long rb, 
         r.dims[1] = (cuuint64_t)((long)N * rb / 16);
         r.strides[0] = 16;
         r.box[0] = 16;
-        r.box[1] = (cuuint32_t)gemv_slot_units(84, cps);
+        r.box[1] = (cuuint32_t)gemv_slot_units(gemv_chunk_bytes(kf), cps);
         return encode_cached(r, map);
     }
     if (wf == LWQ_Q6_K) {
@@ -464,7 +480,7 @@ int encode_weight_map(CUtensorMap *map, const void *Wq, int wf, int N, long rb, 
         r.box[1] = (cuuint32_t)GEMV_ROWS;
         return encode_cached(r, map);
     }
-    const int cb = gemv_chunk_bytes(wf);
+    const int cb = gemv_chunk_bytes(kf);
     MapReq r = map_req(Wq, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, CU_TENSOR_MAP_SWIZZLE_NONE);
     r.dims[0] = (cuuint64_t)(cb / 8);
     r.dims[1] = (cuuint64_t)N;
@@ -579,7 +595,7 @@ int gemv_run(const Plan &p, int fmt, const void *Wq, const void *x, float *y, in
     const size_t xelem = (xt == X_F32) ? 4 : 2;
     const int S = p.cfg.splits;
     CUtensorMap map;
-    int rc = encode_weight_map(&map, Wq, wf, N, rb, p.cps);
+    int rc = encode_weight_map(&map, Wq, wf, N, K, rb, p.cps);
     if (rc) return rc;
     int n = 0;
     for (int m0 = 0; m0 < M; m0 += p.m_group) {
@@ -600,7 +616,7 @@ int gemv_run(const Plan &p, int fmt, const void *Wq, const void *x, float *y, in
         a.overlap = overlap;
         const int nt = gemv_nt(xt, p.i8, mg);
         cudaError_t e = dispatch_gemv(wf, xt, nt, p.i8, map, a, p.cfg.ctas,
-                                      gemv_smem(wf, p.cps, p.cfg.stages, nt, p.i8, xt, mg), st);
+                                      gemv_smem(gemv_kfmt(wf, K), p.cps, p.cfg.stages, nt, p.i8, xt, mg), st);
         if (e != cudaSuccess) return LWQ_ERR_CUDA;
         ++n;
         if (S > 1) {

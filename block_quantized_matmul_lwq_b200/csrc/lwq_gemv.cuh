@@ -48,7 +48,8 @@
 
 namespace lwq {
 
-enum { F_Q8_0 = 1, F_Q4_0 = 2, F_Q4_K = 3, F_Q6_K = 4, F_Q5_K = 5, F_Q2_K = 6 };
+// F_Q6_KS: Q6_K rows that are not 16-byte multiples, streamed as row slots
+enum { F_Q8_0 = 1, F_Q4_0 = 2, F_Q4_K = 3, F_Q6_K = 4, F_Q5_K = 5, F_Q2_K = 6, F_Q6_KS = 7 };
 enum { X_F32 = 0, X_F16 = 1, X_BF16 = 2 };
 
 constexpr int GEMV_ROWS = 16;                     // weight rows per tile (the MMA's M)
@@ -85,6 +86,8 @@ struct FmtInfo<F_Q6_K> { static constexpr int chunk_bytes = 240; };
 // dimension.  Its weights stream as row slots instead (fmt_row_slots).
 template <>
 struct FmtInfo<F_Q2_K> { static constexpr int chunk_bytes = 84; };
+template <>
+struct FmtInfo<F_Q6_KS> { static constexpr int chunk_bytes = 210; };
 // Formats with a per-sub-block min (the S_j sums of x enter the result), and
 // the number of those sums per 256-weight chunk (sub-blocks of 32 or 16).
 __host__ __device__ constexpr int fmt_sums(int fmt) {
@@ -95,12 +98,13 @@ __host__ __device__ constexpr bool fmt_has_min(int fmt) { return fmt_sums(fmt) >
 // tensor map of [bytes / 16][16]); per stage, row r of the tile is one box of
 // whole units into its own 128-byte aligned slot, starting r mod 8 units before
 // the unit that holds the row's first byte of the split.  The slice then lies
-// 16 (r mod 8) + ((n rb + 84 c) mod 16) bytes into the slot -- the second term
-// 0, 4, 8 or 12, so 32-bit words stay aligned -- and the 8 rows that a warp's
-// lane groups read at once fall on distinct bank quads.
-__host__ __device__ constexpr bool fmt_row_slots(int fmt) { return fmt == F_Q2_K; }
+// 16 (r mod 8) + ((n rb + cb c) mod 16) bytes into the slot, and the 8 rows
+// that a warp's lane groups read at once fall on distinct bank quads.  The
+// second term is 0, 4, 8 or 12 for Q2_K (cb = 84), so its 32-bit words stay
+// aligned; Q6_K (cb = 210) may start 2 bytes off a word.
+__host__ __device__ constexpr bool fmt_row_slots(int fmt) { return fmt == F_Q2_K || fmt == F_Q6_KS; }
 __host__ __device__ constexpr int gemv_slot_units(int chunk_bytes, int cps) {   // units per row box
-    return (chunk_bytes * cps + 12 + 15) / 16 + 7;
+    return (chunk_bytes * cps + 15 + 15) / 16 + 7;
 }
 __host__ __device__ constexpr int gemv_slot_bytes(int chunk_bytes, int cps) {   // slot stride
     return (16 * gemv_slot_units(chunk_bytes, cps) + 127) / 128 * 128;
@@ -283,7 +287,7 @@ __device__ __forceinline__ float byte_magic(uint32_t v, int jj) {
 //    the last two code bytes of the block in its place (one PRMT).
 template <int FMT>
 __device__ __forceinline__ int elem(int bb, int h, int t, int q) {
-    if (FMT == F_Q4_K || FMT == F_Q5_K || FMT == F_Q6_K || FMT == F_Q2_K || (bb & 1))
+    if (FMT == F_Q4_K || FMT == F_Q5_K || FMT == F_Q6_K || FMT == F_Q6_KS || FMT == F_Q2_K || (bb & 1))
         return 32 * bb + 16 * h + 4 * t + 2 * q;
     if (FMT == F_Q4_0) return 32 * bb + 16 * h + ((4 * t - 2 + 2 * q) & 15);
     return 32 * bb + ((16 * h + 4 * t - 2 + 2 * q) & 31);
@@ -298,7 +302,7 @@ struct Exact {
     uint32_t xf[NT][NB][2][2];               // [tile][block][step][reg]
     float inv;                               // 1 / the activation scale (a power of two)
     uint32_t q6o = 0;                        // Q6_K: byte offset of the superblock in its chunk box
-    uint32_t q2r0 = 0, q2r1 = 0;             // Q2_K: the superblock in rows g and g + 8 of the stage
+    uint32_t sr0 = 0, sr1 = 0;               // row slots: the superblock in rows g and g + 8 of the stage
 
     // ---------------------------------------------------------- prologue
     // The CTA's slice of x is prepared once, by all nact compute warps
@@ -567,10 +571,21 @@ struct Exact {
 
     // Q6_K: 32-bit word at byte q6o + off of a row (q6o even; MIS: q6o = 2 mod 4,
     // the word straddles two aligned words)
-    template <bool MIS>
+    // Q6_K: 32-bit word at byte off of a superblock.  MIS 0 / 1: the superblock
+    // starts q6o bytes into the row's chunk box, q6o = 0 / 2 mod 4 (one load, or
+    // two aligned loads and a PRMT); MIS 2 (row slots): row is the superblock's
+    // own address, even, with each row's alignment its own (two loads and a PRMT
+    // whose selector follows the row).
+    template <int MIS>
     __device__ __forceinline__ uint32_t q6w(uint32_t row, uint32_t off) const {
-        if constexpr (MIS) return prmt(lds32(row + q6o - 2 + off), lds32(row + q6o + 2 + off), 0x5432u);
-        else return lds32(row + q6o + off);
+        if constexpr (MIS == 2) {
+            const uint32_t a = (row + off) & ~3u;
+            return prmt(lds32(a), lds32(a + 4), (row & 2) ? 0x5432u : 0x3210u);
+        } else if constexpr (MIS == 1) {
+            return prmt(lds32(row + q6o - 2 + off), lds32(row + q6o + 2 + off), 0x5432u);
+        } else {
+            return lds32(row + q6o + off);
+        }
     }
     // Q6_K (210-byte superblock = the warp's chunk; with KW = 128 the warp takes
     // half `half` of it).  For half n and l0 in {0, 16}, lane t's words
@@ -579,7 +594,7 @@ struct Exact {
     // sub-blocks j = 8n + 2g + l0/16 (g = 0..3: low nibbles of A, of B, high
     // nibbles of A, of B; high bits 2g, 2g+1 of H).  A sub-block of 16 weights has
     // one int8 scale: one MMA step, then y += d * sc_j * C.
-    template <bool MIS>
+    template <int MIS>
     __device__ __forceinline__ void compute_q6(uint32_t r0, uint32_t r1, int half, float (&acc)[NT][4], int t) const {
         const float d0 = f16_lo(q6w<MIS>(r0, 208)), d1 = f16_lo(q6w<MIS>(r1, 208));
         constexpr int NH = NB / 4;                                    // halves of the superblock: 2 or 1
@@ -625,7 +640,7 @@ struct Exact {
     }
 
     // Q2_K (84-byte superblock = the warp's chunk; with KW = 128 the warp takes
-    // half `half` of it).  Rows g and g + 8 lie at box + q2r0 and box + q2r1
+    // half `half` of it).  Rows g and g + 8 lie at box + sr0 and box + sr1
     // (row slots).  Sub-block 8n + 2j + h (16 weights: elements 128n + 32j +
     // 16h ..) has its codes in bits 2j, 2j+1 of qs[32n + 16h ..]: lane t's word
     // qs[32n + 16h + 4t ..] gives elements 4t .. 4t + 3 of it, bytes 0 and 2
@@ -634,7 +649,7 @@ struct Exact {
     // once per tile, y -= dmin * sum m S over the part-0 columns.
     __device__ __forceinline__ void compute_q2(uint32_t box, int half, float (&acc)[NT][4], int t, int M,
                                                const float *sxw, int sstride) const {
-        const uint32_t r0 = box + q2r0, r1 = box + q2r1;
+        const uint32_t r0 = box + sr0, r1 = box + sr1;
         const uint32_t h0 = lds32(r0 + 80), h1 = lds32(r1 + 80);   // d | dmin
         const float d0 = f16_lo(h0), d1 = f16_lo(h1);
         const float nd0 = d0 * -8388608.f, nd1 = d1 * -8388608.f;   // -2^23 d (exact)
@@ -725,9 +740,11 @@ struct Exact {
             }
         } else if constexpr (FMT == F_Q2_K) {
             compute_q2(box, half, acc, t, M, sxw, sstride);
+        } else if constexpr (FMT == F_Q6_KS) {
+            compute_q6<2>(box + sr0, box + sr1, half, acc, t);
         } else if constexpr (FMT == F_Q6_K) {
-            if (q6o & 2) compute_q6<true>(r0, r1, half, acc, t);
-            else compute_q6<false>(r0, r1, half, acc, t);
+            if (q6o & 2) compute_q6<1>(r0, r1, half, acc, t);
+            else compute_q6<0>(r0, r1, half, acc, t);
         } else if constexpr (FMT == F_Q8_0) {
 #pragma unroll
             for (int pp = 0; pp < NB / 2; ++pp) {
@@ -1301,8 +1318,8 @@ __global__ void __launch_bounds__(gemv_threads(FMT, NT), 1)
             // rows g and g + 8 of the tile: their slots, the slice's offset in them, this warp's chunk
             const long rb = (long)a.nchunks * CB;
             const long b0 = (long)(tile * GEMV_ROWS + g) * rb + (long)c_begin * CB, b1 = b0 + 8 * rb;
-            impl.q2r0 = (uint32_t)(g * L.slot + 16 * g) + (uint32_t)(b0 & 15) + (uint32_t)(ci * CB);
-            impl.q2r1 = (uint32_t)((g + 8) * L.slot + 16 * g) + (uint32_t)(b1 & 15) + (uint32_t)(ci * CB);
+            impl.sr0 = (uint32_t)(g * L.slot + 16 * g) + (uint32_t)(b0 & 15) + (uint32_t)(ci * CB);
+            impl.sr1 = (uint32_t)((g + 8) * L.slot + 16 * g) + (uint32_t)(b1 & 15) + (uint32_t)(ci * CB);
             box = smem_u32(ring) + (uint32_t)((size_t)s * L.stage);
         } else {
             box = smem_u32(ring) + (uint32_t)((size_t)s * L.stage + (size_t)ci * GEMV_ROWS * CB);

@@ -172,17 +172,18 @@ def test_gemm_tile_choices_are_valid():
 
 
 def test_more_kquant_formats_routing_and_row_bytes():
-    """Q5_K takes the tensor-core paths; Q6_K the tensor-core paths when its rows are 16-byte
-    multiples (K a multiple of 2048), else the simple kernel; Q2_K the tensor-core GEMV (row slots)
-    when the matrix is a 16-byte multiple, at any M, else the simple kernel; row bytes follow the
-    superblock sizes 176, 210 and 84."""
+    """Q5_K takes the tensor-core paths; Q6_K the tensor-core GEMV (row slots where its rows are not
+    16-byte multiples) and, with K a multiple of 2048, the tcgen05 GEMM; Q2_K the tensor-core GEMV
+    (row slots) at any M; both fall back to the simple kernel only when the whole matrix is not a
+    16-byte multiple; row bytes follow the superblock sizes 176, 210 and 84."""
     for M, path in ((1, 1), (16, 1), (17, 2), (512, 2)):
         assert lwq.lwq_select_config(lwq.fmt_code("q5_k", "f16"), M, 4096, 4096).path == path
-    for M, K, path in ((1, 4096, 1), (16, 14336, 1), (1, 11008, 3), (8, 2816, 3), (17, 4096, 1), (40, 11008, 3)):
+    for M, K, path in ((1, 4096, 1), (16, 14336, 1), (1, 11008, 1), (8, 2816, 1), (17, 4096, 1), (40, 11008, 1)):
         assert lwq.lwq_select_config(lwq.fmt_code("q6_k", "f32"), M, 4096, K).path == path
-    # 16-bit activations, M > 16: the tcgen05 GEMM where the rows allow it
+    assert lwq.lwq_select_config(lwq.fmt_code("q6_k", "f32"), 1, 4095, 11008).path == 3   # 4095 x 9030 bytes
+    # 16-bit activations, M > 16: the tcgen05 GEMM where the rows allow it, else the GEMV in passes
     assert lwq.lwq_select_config(lwq.fmt_code("q6_k", "bf16"), 17, 4096, 4096).path == 2
-    assert lwq.lwq_select_config(lwq.fmt_code("q6_k", "bf16"), 512, 4096, 11008).path == 3
+    assert lwq.lwq_select_config(lwq.fmt_code("q6_k", "bf16"), 512, 4096, 11008).path == 1
     for M in (1, 16, 17, 512):
         assert lwq.lwq_select_config(lwq.fmt_code("q2_k", "f16"), M, 4096, 4096).path == 1
         assert lwq.lwq_select_config(lwq.fmt_code("q2_k", "f16"), M, 4096, 11008).path == 1

@@ -2,11 +2,11 @@
 
 Q5_K has tensor-core decoders (the GEMV and the tcgen05 GEMM).  Q6_K and Q2_K
 superblocks are 210 and 84 bytes, so their rows are not 16-byte multiples in
-general: Q6_K takes the tensor-core GEMV when K is a multiple of 2048 and the
-simple kernel otherwise; Q2_K takes the tensor-core GEMV, its rows streamed as
-slots of the flat matrix, whenever the whole matrix is a 16-byte multiple (N * K
-/ 256 * 84), else the simple kernel.  Every case is scored element by element
-against the oracle on the same seeded inputs.
+general.  Q6_K rows of K a multiple of 2048 are, and take per-chunk TMA boxes
+(and the tcgen05 GEMM); other Q6_K rows, and every Q2_K row, stream as slots of
+the flat matrix whenever the whole matrix is a 16-byte multiple, else take the
+simple kernel.  Every case is scored element by element against the oracle on
+the same seeded inputs.
 """
 
 import ctypes
@@ -90,6 +90,23 @@ def test_q2_k_tensor_core_gemv(dev, a, M, K):
     check_full("q2_k", a, M, 44, K, dev, seed=400 + M + K)
 
 
+@pytest.mark.parametrize("a", ACTS)
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 6, 8, 9, 16])
+@pytest.mark.parametrize("K", [256, 2816, 4352, 11008])
+def test_q6_k_row_slot_gemv(dev, a, M, K):
+    """Q6_K rows that are not 16-byte multiples: row slots whose superblocks start at either word
+    alignment, row by row, every column layout, a ragged last row tile, split-K at K = 11008."""
+    assert lwq.lwq_select_config(lwq.fmt_code("q6_k", a), M, 56, K).path == 1
+    check_full("q6_k", a, M, 56, K, dev, seed=500 + M + K)
+
+
+@pytest.mark.parametrize("warps,splits,stages", [(1, 0, 2), (3, 0, 2), (8, 2, 3), (4, 3, 2), (16, 0, 4)])
+def test_q6_k_row_slot_forced_configs(dev, warps, splits, stages):
+    cfg = lwq.lwq_config()
+    cfg.path, cfg.warps, cfg.splits, cfg.stages = 1, warps, splits, stages
+    check_full("q6_k", "bf16", 3, 72, 4352, dev, seed=warps + splits, cfg=cfg)
+
+
 @pytest.mark.parametrize("warps,splits,stages", [(1, 0, 2), (3, 0, 2), (8, 2, 3), (4, 3, 2), (16, 0, 4)])
 def test_q2_k_forced_gemv_configs(dev, warps, splits, stages):
     cfg = lwq.lwq_config()
@@ -149,11 +166,13 @@ def test_q5_k_split_k_gemv(dev):
 
 
 def test_forced_path_without_decoder_is_refused(dev):
-    """Forcing the tensor-core GEMV on a format without its decoder returns LWQ_ERR_UNSUPPORTED."""
+    """Forcing the tensor-core GEMV where its weight stream cannot go (a Q6_K or Q2_K matrix that is
+    not a whole number of 16-byte units) returns LWQ_ERR_UNSUPPORTED before anything runs."""
     cfg = lwq.lwq_config()
     cfg.path = 1
-    buf = torch.zeros(64, dtype=torch.float32, device="cuda:0")
+    buf = torch.zeros(1024, dtype=torch.float32, device="cuda:0")
     p = buf.data_ptr()
-    rc = lwq.lib().lwq_matmul_config(lwq.fmt_code("q6_k", "f16"), p, p, p, 1, 16, 256, ctypes.byref(cfg), None)
-    assert rc == lwq.LWQ_ERR_UNSUPPORTED
+    for w, N in (("q6_k", 15), ("q2_k", 1), ("q2_k", 5)):   # 15 x 210, 84, 5 x 84 bytes
+        rc = lwq.lib().lwq_matmul_config(lwq.fmt_code(w, "f16"), p, p, p, 1, N, 256, ctypes.byref(cfg), None)
+        assert rc == lwq.LWQ_ERR_UNSUPPORTED, w
 
