@@ -18,6 +18,12 @@
  *            warp-level MMAs, split-K partials reduced deterministically;
  *   M >  16  prefill GEMM: packed tiles staged by TMA, dequantized to
  *            bf16/fp16 in shared memory, tcgen05 MMAs accumulating in TMEM.
+ * Q6_K rows that are not 16-byte multiples (K not a multiple of 2048) and Q2_K
+ * rows stream into the GEMV as slots of the flat matrix (whole 16-byte units
+ * per row), which needs N * lwq_row_bytes(fmt, K) to be a multiple of 16; they
+ * have no tcgen05 GEMM, so M > 16 runs the GEMV over groups of rows.  Shapes
+ * no tensor-core path takes (K not a multiple of 256, or such a matrix that is
+ * not a whole number of 16-byte units) run a simple GEMV kernel.
  *
  * Everything is plain C: pointers and sizes, no C++ or framework types.
  */
@@ -145,7 +151,7 @@ int lwq_shutdown(void);
  *   Wq      device pointer, N packed rows of lwq_row_bytes(fmt, K) bytes each
  *   x       device pointer, row-major [M][K] in the activation dtype
  *   y       device pointer, row-major [M][N] fp32, fully overwritten
- *   M, N, K sizes (> 0); K a multiple of 32 (Q8_0, Q4_0) or 256 (Q4_K)
+ *   M, N, K sizes (> 0); K a multiple of 32 (Q8_0, Q4_0) or 256 (K-quants)
  *   stream  a cudaStream_t (NULL = the legacy default stream)
  *
  * Ownership: the caller owns Wq, x, y and the workspace.  The call is
