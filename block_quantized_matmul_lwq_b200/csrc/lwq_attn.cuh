@@ -470,7 +470,9 @@ __global__ void __launch_bounds__(D) attn_combine_kernel(const float *__restrict
     out[bh * D + d] = A / L;
 }
 
-// Splits of the sequence (each at least 256 keys, a multiple of 16).
+// Splits of the sequence (each at least 64 keys, a multiple of 16).  A small
+// problem (few sequences and heads) thus still spreads over many CTAs: each
+// warp's chain of dependent key steps, not bandwidth, sets its time.
 //  * One query head per kv head: enough CTAs for ~4 per SM (up to ~9 are
 //    resident: many short waves).
 //  * Grouped heads (the tensor-core pass, 2 CTAs resident per SM): the split
@@ -479,7 +481,7 @@ __global__ void __launch_bounds__(D) attn_combine_kernel(const float *__restrict
 //    costs a whole wave.
 inline void attn_splits(int B, int H, int Hkv, int Lmax, int sms, int *S, int *chunk) {
     const long pairs = (long)B * Hkv;
-    const long smax = (Lmax + 255) / 256;
+    const long smax = (Lmax + 63) / 64;
     long best_s = 1;
     if (H == Hkv) {
         best_s = (4L * sms + pairs - 1) / pairs;

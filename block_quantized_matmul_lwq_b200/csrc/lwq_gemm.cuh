@@ -179,6 +179,27 @@ struct Dequant<F_Q4_0, XT> {
     }
 };
 
+// Codes to the 16-bit type, 8 at a time: n0 and n1 hold one code per
+// byte (codes 0-3 and 4-7).  Byte b becomes the fp32 2^23 + code (one PRMT
+// with the exponent byte 0x4B), then, two at a time with packed fp32
+// arithmetic, (2^23 + code) + off (exact: code + off) and w = s * that + c,
+// rounded once to fp32 as fmaf(s, code + off, c) would be; then each pair is
+// rounded once to the 16-bit type.
+template <int XT>
+__device__ __forceinline__ void kq_codes_to_chunk(uint32_t n0, uint32_t n1, float s, float off, float c, uint32_t (&o)[4]) {
+    const float2 s2 = make_float2(s, s), c2 = make_float2(c, c), off2 = make_float2(off, off);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const uint32_t nw = (p < 2) ? n0 : n1;
+        const uint32_t b = 2u * (uint32_t)(p & 1);
+        const float2 fq = make_float2(__uint_as_float(prmt(nw, 0x4B000000u, 0x7440u + b)),
+                                      __uint_as_float(prmt(nw, 0x4B000000u, 0x7441u + b)));
+        const float2 t = __fadd2_rn(fq, off2);   // exact
+        const float2 w = __ffma2_rn(s2, t, c2);
+        o[p] = (XT == X_F16) ? pack_f16x2(w.x, w.y) : pack_bf16x2(w.x, w.y);
+    }
+}
+
 // Q8_0: k-block kb = blocks 2kb (h=0) and 2kb+1 (h=1); codes 16v..16v+15
 // of the block become output chunks 4h+2v and 4h+2v+1.
 template <int XT>
@@ -205,17 +226,8 @@ struct Dequant<F_Q8_0, XT> {
                 o[2] = hmul2_f16(hfma2_f16(prmt(q1, 0x6400u, 0x5150u), H2_ONE, H2_M1152), d2);
                 o[3] = hmul2_f16(hfma2_f16(prmt(q1, 0x6400u, 0x5352u), H2_ONE, H2_M1152), d2);
             } else {
-                const float bias = 8388736.0f;  // 2^23 + 128
-                float f[8];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    f[i] = (__uint_as_float(prmt(q0, 0x4B000000u, 0x7440u + i)) - bias) * d;
-                    f[4 + i] = (__uint_as_float(prmt(q1, 0x4B000000u, 0x7440u + i)) - bias) * d;
-                }
-                o[0] = pack_bf16x2(f[0], f[1]);
-                o[1] = pack_bf16x2(f[2], f[3]);
-                o[2] = pack_bf16x2(f[4], f[5]);
-                o[3] = pack_bf16x2(f[6], f[7]);
+                // (2^23 + (q + 128)) - (2^23 + 128) = q, then d * q rounded once
+                kq_codes_to_chunk<XT>(q0, q1, d, -8388736.0f, -0.0f, o);
             }
             st_shared_v4(a_base + sw128_chunk_offset(r, 4 * h + 2 * v + c), o[0], o[1], o[2], o[3]);
         }
@@ -247,16 +259,10 @@ struct Dequant<F_Q4_K, XT> {
         const uint32_t sh = 4u * h;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-            float f[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint32_t byte = (qw[2 * c + (i >> 2)] >> (8 * (i & 3) + sh)) & 15u;
-                f[i] = fmaf(ds, __uint_as_float(0x4B000000u | byte) - 8388608.0f, -dm);
-            }
+            // w = ds * q - dm, q the nibbles h of the 8 bytes
             uint32_t o[4];
-#pragma unroll
-            for (int p = 0; p < 4; ++p)
-                o[p] = (XT == X_F16) ? pack_f16x2(f[2 * p], f[2 * p + 1]) : pack_bf16x2(f[2 * p], f[2 * p + 1]);
+            kq_codes_to_chunk<XT>((qw[2 * c] >> sh) & 0x0F0F0F0Fu, (qw[2 * c + 1] >> sh) & 0x0F0F0F0Fu, ds,
+                                  -8388608.0f, -dm, o);
             st_shared_v4(a_base + sw128_chunk_offset(r, 4 * h + 2 * v + c), o[0], o[1], o[2], o[3]);
         }
     }
@@ -288,18 +294,13 @@ struct Dequant<F_Q5_K, XT> {
         const uint32_t sh = 4u * h;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-            float f[8];
+            // q = nibble h | (bit j of the qh byte) << 4, four bytes at a time
+            uint32_t n[2];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint32_t bsh = 8 * (i & 3);
-                const uint32_t q = ((qw[2 * c + (i >> 2)] >> (bsh + sh)) & 15u) |
-                                   (((hw[2 * c + (i >> 2)] >> (bsh + j)) & 1u) << 4);
-                f[i] = fmaf(ds, __uint_as_float(0x4B000000u | q) - 8388608.0f, -dm);
-            }
+            for (int w = 0; w < 2; ++w)
+                n[w] = ((qw[2 * c + w] >> sh) & 0x0F0F0F0Fu) | (((hw[2 * c + w] >> j) << 4) & 0x10101010u);
             uint32_t o[4];
-#pragma unroll
-            for (int p = 0; p < 4; ++p)
-                o[p] = (XT == X_F16) ? pack_f16x2(f[2 * p], f[2 * p + 1]) : pack_bf16x2(f[2 * p], f[2 * p + 1]);
+            kq_codes_to_chunk<XT>(n[0], n[1], ds, -8388608.0f, -dm, o);
             st_shared_v4(a_base + sw128_chunk_offset(r, 4 * h + 2 * v + c), o[0], o[1], o[2], o[3]);
         }
     }
@@ -335,18 +336,13 @@ struct Dequant<F_Q6_K, XT> {
         const uint32_t ls = 4u * (g >> 1), hs = 2u * g;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-            float f[8];
+            // q = nibble g>>1 of the ql byte | bits 2g, 2g+1 of the qh byte << 4; w = ds * (q - 32), exact
+            uint32_t n[2];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint32_t bsh = 8 * (i & 3);
-                const uint32_t q = ((ql[2 * c + (i >> 2)] >> (bsh + ls)) & 15u) |
-                                   (((qh[2 * c + (i >> 2)] >> (bsh + hs)) & 3u) << 4);
-                f[i] = ds * (float)((int)q - 32);   // exact
-            }
+            for (int w = 0; w < 2; ++w)
+                n[w] = ((ql[2 * c + w] >> ls) & 0x0F0F0F0Fu) | (((qh[2 * c + w] >> hs) << 4) & 0x30303030u);
             uint32_t o[4];
-#pragma unroll
-            for (int p = 0; p < 4; ++p)
-                o[p] = (XT == X_F16) ? pack_f16x2(f[2 * p], f[2 * p + 1]) : pack_bf16x2(f[2 * p], f[2 * p + 1]);
+            kq_codes_to_chunk<XT>(n[0], n[1], ds, -8388640.0f, -0.0f, o);   // + (-0): ds * t exactly, signed zeros too
             st_shared_v4(a_base + sw128_chunk_offset(r, 4 * h + 2 * v + c), o[0], o[1], o[2], o[3]);
         }
     }
