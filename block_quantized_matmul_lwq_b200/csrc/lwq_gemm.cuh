@@ -158,11 +158,13 @@ struct Dequant;
 template <int XT>
 struct Dequant<F_Q4_0, XT> {
     static __device__ __forceinline__ void run(uint32_t prow, int kb, int h, int v, uint32_t a_base, int r) {
-        // block 2kb+h starts at byte 36kb + 18h; its nibbles at +2, so bytes 8v..8v+7 are at 36kb+18h+2+8v
-        const uint32_t w = prow + 4 * (9 * kb + 4 * h + 2 * v);   // word-aligned start (2 bytes early when h=0)
-        const uint32_t W0 = lds32(w), W1 = lds32(w + 4), W2 = lds32(w + 8);
-        const uint32_t s = h ? 32u : 16u;
-        const uint32_t q0 = __funnelshift_rc(W0, W1, s), q1 = __funnelshift_rc(W1, W2, s);
+        // block 2kb+h starts at byte 36kb + 18h; its nibbles at +2, so bytes 8v..8v+7 are at 36kb+18h+2+8v:
+        // word 9kb+2v, 2 bytes in (h=0), or exactly word 9kb+5+2v (h=1).  Rows lie 36 words apart, so a
+        // warp's h=0 lanes read even banks and its h=1 lanes odd ones: no two lanes of a load share a bank
+        // (the third load of an h=1 lane repeats its first)
+        const uint32_t w = prow + 4 * (9 * kb + 2 * v + (h ? 5 : 0));
+        const uint32_t W0 = lds32(w), W1 = lds32(w + 4), W2 = lds32(h ? w : w + 8);
+        const uint32_t q0 = h ? W0 : __funnelshift_r(W0, W1, 16), q1 = h ? W1 : __funnelshift_r(W1, W2, 16);
         const uint32_t dw = lds32(prow + 4 * (9 * kb + 4 * h));
         const float d = f16_bits_to_float(h ? (dw >> 16) : dw);
         uint32_t dh2, dl2;
