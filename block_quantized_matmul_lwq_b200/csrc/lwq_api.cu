@@ -265,6 +265,15 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
     }
     if (stages < 2 || gemv_smem(gemv_kfmt(wf, K), cps, stages, p->nt, p->i8, xt, mg) > kSmemLimit) return LWQ_ERR_UNSUPPORTED;
     S = (nchunks + cps - 1) / cps;               // drop empty splits
+    if (!(force && force->splits)) {
+        // even splits: shared memory that limited a CTA to cps chunks (K = 4096, 16 rows of 16-bit
+        // x: 14) would otherwise leave the last split a remainder (2), and its CTAs idle beside the
+        // others; the smaller slice may also leave room for more weight stages
+        cps = (nchunks + S - 1) / S;
+        if (!(force && force->stages))
+            while (stages < 4 && gemv_smem(gemv_kfmt(wf, K), cps, stages + 1, p->nt, p->i8, xt, mg) <= kSmemLimit)
+                ++stages;
+    }
     const int row_tiles = (N + GEMV_ROWS - 1) / GEMV_ROWS;
     // one CTA per SM
     int groups = force && force->ctas ? force->ctas / S : sms / S;
