@@ -829,6 +829,7 @@ def parse_args(argv=None):
                     help="steps of each prefill GEMM workload (about a second, so the clocks settle)")
     ap.add_argument("--extra", nargs="*", default=["q8_0_gemv_4096x4096", "q4_k_7b_layer_decode",
                                                    "q4_k_7b_layer_decode_fused", "q4_0_gemv_11008x4096_act_i8",
+                                                   "q4_k_7b_layer_decode_act_i8",
                                                    "q4_0_prefill_gemm", "q6_k_7b_layer_decode",
                                                    "q5_k_7b_layer_decode", "q2_k_7b_layer_decode",
                                                    "q6_k_prefill_gemm", "q5_k_prefill_gemm"])

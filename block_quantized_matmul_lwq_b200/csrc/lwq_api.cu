@@ -213,9 +213,9 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
     }
     if (path != 1 || !tc_gemv_eligible(wf, N, K)) return LWQ_ERR_UNSUPPORTED;
     p->i8 = (fmt & LWQ_FLAG_ACT_I8) != 0;
-    // int8 activation blocks: Q4_0 and Q8_0 weights, any M (passes of 8 rows; every pass streams
+    // int8 activation blocks: Q4_0, Q8_0 and Q4_K weights, any M (passes of 8 rows; every pass streams
     // the weights again, so a prefill-sized M reads them M / 8 times)
-    if (p->i8 && wf != LWQ_Q4_0 && wf != LWQ_Q8_0) return LWQ_ERR_UNSUPPORTED;
+    if (p->i8 && wf != LWQ_Q4_0 && wf != LWQ_Q8_0 && wf != LWQ_Q4_K) return LWQ_ERR_UNSUPPORTED;
     // rows per pass: 8 with fp32 activations (3 parts, 24 columns) or int8 blocks, else 16
     const int mmax = (xt == X_F32 || p->i8) ? 8 : 16;
     p->m_group = M < mmax ? M : mmax;
@@ -366,6 +366,11 @@ cudaError_t dispatch_gemv(int wf, int xt, int nt, bool i8, const CUtensorMap &ma
             if (xt == X_F32) return launch_gemv<F_Q8_0, X_F32, 1, true>(map, a, ctas, smem, st);
             if (xt == X_F16) return launch_gemv<F_Q8_0, X_F16, 1, true>(map, a, ctas, smem, st);
             return launch_gemv<F_Q8_0, X_BF16, 1, true>(map, a, ctas, smem, st);
+        }
+        if (wf == LWQ_Q4_K) {
+            if (xt == X_F32) return launch_gemv<F_Q4_K, X_F32, 1, true>(map, a, ctas, smem, st);
+            if (xt == X_F16) return launch_gemv<F_Q4_K, X_F16, 1, true>(map, a, ctas, smem, st);
+            return launch_gemv<F_Q4_K, X_BF16, 1, true>(map, a, ctas, smem, st);
         }
         return cudaErrorInvalidValue;
     }

@@ -937,14 +937,15 @@ struct RawPair<X_F32> {
 template <int XT, int FMT = F_Q4_0>
 struct Q40I8 {
     static constexpr bool Q8 = FMT == F_Q8_0;
+    static constexpr bool QK = FMT == F_Q4_K;   // Q4_K: unsigned codes, sub-block scale and min
     static constexpr int CB = FmtInfo<FMT>::chunk_bytes;
     uint32_t xq[8][2];   // [block][k-slots 4t.. / 16+4t..]: int8 codes of activation row g
     float dx[8][2];      // [block][column 2t, 2t+1]: d_x (Q4_0: d_x / 16) of activation rows 2t, 2t+1
     float inv;           // 1: no activation scale to undo
 
     // activation element of k-slot pair (4t, 4t+1) and (4t+2, 4t+3) of block parity hb
-    __device__ static __forceinline__ int cb0(int hb, int j) { return (Q8 || hb) ? 4 * j : (j ? 4 * j - 2 : 14); }
-    __device__ static __forceinline__ int cb2(int hb, int j) { return (Q8 || hb) ? 4 * j + 2 : 4 * j; }
+    __device__ static __forceinline__ int cb0(int hb, int j) { return (Q8 || QK || hb) ? 4 * j : (j ? 4 * j - 2 : 14); }
+    __device__ static __forceinline__ int cb2(int hb, int j) { return (Q8 || QK || hb) ? 4 * j + 2 : 4 * j; }
 
     __device__ static __forceinline__ uint32_t pack_s8(int a, int b, int c, int d) {
         return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8) | ((uint32_t)(c & 0xFF) << 16) |
@@ -1014,7 +1015,7 @@ struct Q40I8 {
                 xq[b][0] = pack_s8(q8(v[0], sc), q8(v[1], sc), q8(v[2], sc), q8(v[3], sc));
                 xq[b][1] = pack_s8(q8(v[4], sc), q8(v[5], sc), q8(v[6], sc), q8(v[7], sc));
                 // columns 2t and 2t+1 carry activation rows 2t, 2t+1 (lanes 8t and 8t+4)
-                constexpr float DS = Q8 ? 1.f : 0.0625f;   // Q4_0 codes enter as 16 (u - 8)
+                constexpr float DS = (Q8 || QK) ? 1.f : 0.0625f;   // Q4_0 codes enter as 16 (u - 8)
                 dx[b][0] = DS * __shfl_sync(0xffffffffu, d, 8 * t);
                 dx[b][1] = DS * __shfl_sync(0xffffffffu, d, 8 * t + 4);
             }
@@ -1026,6 +1027,46 @@ struct Q40I8 {
                                             int) const {
         const int g = lane >> 2, t = lane & 3;
         const uint32_t r0 = box + g * CB, r1 = r0 + 8 * CB;   // rows g, g+8
+        if constexpr (QK) {
+            // Q4_K superblock: sub-block b (32 weights) takes nibble b & 1 of qs[32 (b / 2) ..]; its
+            // codes u enter as they are (0..15), so C = sum u q_x, and a second MMA with A = 1
+            // gives the code sums Q = sum q_x of each activation row:
+            //   y += d_x (d sc_b C - dmin m_b Q)
+            const uint32_t h0 = lds32(r0), h1 = lds32(r1);                 // d | dmin
+            const float d0 = f16_lo(h0), d1 = f16_lo(h1), n0 = -f16_hi(h0), n1 = -f16_hi(h1);
+            const uint32_t s10 = lds32(r0 + 4), s11 = lds32(r1 + 4), s20 = lds32(r0 + 8), s21 = lds32(r1 + 8);
+            const uint32_t s30 = lds32(r0 + 12), s31 = lds32(r1 + 12);
+            // 6-bit scales and mins, one per byte: sub-blocks 0-3 and 4-7
+            const uint32_t sc[2][2] = {{s10 & 0x3F3F3F3Fu, (s30 & 0x0F0F0F0Fu) | ((s10 >> 2) & 0x30303030u)},
+                                       {s11 & 0x3F3F3F3Fu, (s31 & 0x0F0F0F0Fu) | ((s11 >> 2) & 0x30303030u)}};
+            const uint32_t mn[2][2] = {{s20 & 0x3F3F3F3Fu, ((s30 >> 4) & 0x0F0F0F0Fu) | ((s20 >> 2) & 0x30303030u)},
+                                       {s21 & 0x3F3F3F3Fu, ((s31 >> 4) & 0x0F0F0F0Fu) | ((s21 >> 2) & 0x30303030u)}};
+            const uint32_t ones[4] = {0x01010101u, 0x01010101u, 0x01010101u, 0x01010101u};
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) {
+                const uint32_t o = 16u + 32u * (uint32_t)gq + 4u * (uint32_t)t;
+                const uint32_t lo0 = lds32(r0 + o), lo1 = lds32(r1 + o), hi0 = lds32(r0 + o + 16), hi1 = lds32(r1 + o + 16);
+#pragma unroll
+                for (int hb = 0; hb < 2; ++hb) {
+                    const int b = 2 * gq + hb;
+                    const int sh = 4 * hb;
+                    const uint32_t a[4] = {(lo0 >> sh) & 0x0F0F0F0Fu, (lo1 >> sh) & 0x0F0F0F0Fu,
+                                           (hi0 >> sh) & 0x0F0F0F0Fu, (hi1 >> sh) & 0x0F0F0F0Fu};
+                    int c[4], q[4];
+                    imma_s8_16832(c, a, xq[b][0], xq[b][1]);
+                    imma_s8_16832(q, ones, xq[b][0], xq[b][1]);
+                    const float s0 = d0 * (float)((sc[0][b >> 2] >> (8 * (b & 3))) & 0xFFu);   // exact
+                    const float s1 = d1 * (float)((sc[1][b >> 2] >> (8 * (b & 3))) & 0xFFu);
+                    const float m0 = n0 * (float)((mn[0][b >> 2] >> (8 * (b & 3))) & 0xFFu);
+                    const float m1 = n1 * (float)((mn[1][b >> 2] >> (8 * (b & 3))) & 0xFFu);
+                    acc[0][0] = fmaf(dx[b][0], fmaf(s0, (float)c[0], m0 * (float)q[0]), acc[0][0]);
+                    acc[0][1] = fmaf(dx[b][1], fmaf(s0, (float)c[1], m0 * (float)q[1]), acc[0][1]);
+                    acc[0][2] = fmaf(dx[b][0], fmaf(s1, (float)c[2], m1 * (float)q[2]), acc[0][2]);
+                    acc[0][3] = fmaf(dx[b][1], fmaf(s1, (float)c[3], m1 * (float)q[3]), acc[0][3]);
+                }
+            }
+            return;
+        }
         if constexpr (Q8) {
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
@@ -1094,6 +1135,8 @@ template <int XT>
 struct GemvImpl<F_Q4_0, XT, 1, true> : Q40I8<XT> {};
 template <int XT>
 struct GemvImpl<F_Q8_0, XT, 1, true> : Q40I8<XT, F_Q8_0> {};
+template <int XT>
+struct GemvImpl<F_Q4_K, XT, 1, true> : Q40I8<XT, F_Q4_K> {};
 
 // ------------------------------------------------------------------ kernel
 // blockDim = gemv_threads(FMT, NT): warps 0..15 compute, warp 16 produces (TMA), the

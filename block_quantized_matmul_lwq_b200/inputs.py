@@ -290,6 +290,11 @@ WORKLOADS = {
         seeds=[(0, 1, 2), 3, (4, 5), 6]),
     # the headline decode step with int8 activation blocks (LWQ_FLAG_ACT_I8)
     "q4_0_gemv_11008x4096_act_i8": dict(fmt="q4_0", act="f32:i8", Ms=[1, 4, 8], shapes=[(11008, 4096)], seeds=[0]),
+    # the Q4_K layer with its fp16 activations taken as int8 blocks
+    "q4_k_7b_layer_decode_act_i8": dict(
+        fmt="q4_k", act="f16:i8", Ms=[1],
+        shapes=[(4096, 4096)] * 4 + [(11008, 4096), (11008, 4096), (4096, 11008)],
+        seeds=[0, 1, 2, 3, 4, 5, 6]),
     "q4_0_prefill_gemm": dict(fmt="q4_0", act="bf16", Ms=[512, 2048],
                               shapes=[(11008, 4096), (4096, 11008)], seeds=[0, 0]),
     # the other K-quant formats over the same 7B layer (fp16 activations, one token)

@@ -112,7 +112,7 @@ typedef enum {
  * scaled in fp32.  Results differ from the unquantized product by the
  * activation rounding (max |y - y_exact| / sum |x w| stays below 1e-2 for
  * N(0,1) activations); against x_q they agree to fp32 rounding.  Supported for
- * Q4_0 and Q8_0 weights at any M, in passes of 8 activation rows (each pass
+ * Q4_0, Q8_0 and Q4_K weights at any M, in passes of 8 activation rows (each pass
  * streams the weights: a prefill-sized M reads them M/8 times); other formats
  * return LWQ_ERR_UNSUPPORTED.  Activations must be finite. */
 #define LWQ_FLAG_ACT_I8 0x2000

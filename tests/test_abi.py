@@ -216,7 +216,8 @@ def test_int8_flag_plan():
     assert lwq.lwq_workspace_size(i8, 16, 4096, 11008) == lwq.lwq_workspace_size(i8, 8, 4096, 11008)
     assert lwq.lwq_select_config(i8, 17, 4096, 4096).path == 1              # M > 16: GEMV passes of 8 rows
     assert lwq.lwq_select_config(lwq.fmt_code("q8_0", "f16") | lwq.LWQ_FLAG_ACT_I8, 1, 4096, 4096).path == 1
-    for fmt, M, K in ((lwq.fmt_code("q4_k", "f16") | lwq.LWQ_FLAG_ACT_I8, 1, 4096), (i8, 1, 288)):
+    assert lwq.lwq_select_config(lwq.fmt_code("q4_k", "f16") | lwq.LWQ_FLAG_ACT_I8, 1, 4096, 4096).path == 1
+    for fmt, M, K in ((lwq.fmt_code("q6_k", "f16") | lwq.LWQ_FLAG_ACT_I8, 1, 4096), (i8, 1, 288)):
         with pytest.raises(lwq.LwqError) as e:
             lwq.lwq_select_config(fmt, M, 64, K)
         assert e.value.status == lwq.LWQ_ERR_UNSUPPORTED

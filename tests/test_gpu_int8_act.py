@@ -1,4 +1,4 @@
-"""GPU parity of the int8-activation GEMV (LWQ_FLAG_ACT_I8; Q4_0 and Q8_0 weights)
+"""GPU parity of the int8-activation GEMV (LWQ_FLAG_ACT_I8; Q4_0, Q8_0 and Q4_K weights)
 against the oracle's definition (oracle.quantize_act_q8 / matmul_q8act).
 
 The activation codes are integer decisions taken in fp32 on both sides with the
@@ -57,7 +57,7 @@ def check(a, M, N, K, dev, seed, noalloc=False, x=None, w="q4_0"):
     return y, Wq, x
 
 
-@pytest.mark.parametrize("w", ["q4_0", "q8_0"])
+@pytest.mark.parametrize("w", ["q4_0", "q8_0", "q4_k"])
 @pytest.mark.parametrize("a", ["f32", "f16", "bf16"])
 @pytest.mark.parametrize("M,N,K", [(1, 211, 3072), (2, 1000, 4096), (5, 47, 11008), (8, 300, 4096),
                                    (9, 130, 2048), (16, 64, 4352)])
@@ -65,7 +65,7 @@ def test_parity(dev, w, a, M, N, K):
     check(a, M, N, K, dev, seed=M * 31 + K, w=w)
 
 
-@pytest.mark.parametrize("w", ["q4_0", "q8_0"])
+@pytest.mark.parametrize("w", ["q4_0", "q8_0", "q4_k"])
 @pytest.mark.parametrize("M", [17, 40, 130])
 def test_many_rows_in_passes(dev, w, M):
     """M > 16: passes of 8 activation rows, each streaming the weights."""
@@ -75,6 +75,12 @@ def test_many_rows_in_passes(dev, w, M):
 def test_q8_0_gemv_4096x4096(dev):
     """Q8_0 4096 x 4096 at M = 1 with int8 activation blocks, every output."""
     check("f32", 1, 4096, 4096, dev, seed=0, w="q8_0")
+
+
+def test_q4_k_7b_layer_shapes(dev):
+    """Q4_K at the 7B layer's three shapes, fp16 activations as int8 blocks, every output (split-K at K = 11008)."""
+    for N, K in ((4096, 4096), (11008, 4096), (4096, 11008)):
+        check("f16", 1, N, K, dev, seed=N + K, w="q4_k")
 
 
 def test_headline_shape_against_exact_product(dev):
@@ -107,7 +113,7 @@ def test_noalloc_and_deterministic(dev):
     assert oracle.normalised_error(ys[0], y_ref, den) <= TOL_I8
 
 
-@pytest.mark.parametrize("w,M,K", [("q4_k", 1, 4096), ("q5_k", 1, 4096), ("q6_k", 1, 4096), ("q4_0", 1, 288)])
+@pytest.mark.parametrize("w,M,K", [("q2_k", 1, 4096), ("q5_k", 1, 4096), ("q6_k", 1, 4096), ("q4_0", 1, 288)])
 def test_unsupported(dev, w, M, K):
     fmt = lwq.fmt_code(w, "f16") | lwq.LWQ_FLAG_ACT_I8
     N = 64
