@@ -832,7 +832,7 @@ def parse_args(argv=None):
                                                    "q4_k_7b_layer_decode_act_i8",
                                                    "q4_0_prefill_gemm", "q6_k_7b_layer_decode",
                                                    "q5_k_7b_layer_decode", "q2_k_7b_layer_decode",
-                                                   "q6_k_prefill_gemm", "q5_k_prefill_gemm"])
+                                                   "q6_k_prefill_gemm", "q5_k_prefill_gemm", "q2_k_prefill_gemm"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="leave the format x batch sweep out of the line")
     ap.add_argument("--no-host-cost", action="store_true", help="leave the host enqueue timing out")

@@ -584,6 +584,7 @@ int gemm_launch(int wf, int xt, const void *Wq, const void *x, float *y, int M, 
     case LWQ_Q8_0: e = launch_gemm_xt<F_Q8_0>(xt, h, wm, xm, a, cfg.ctas, smem, st); break;
     case LWQ_Q5_K: e = launch_gemm_xt<F_Q5_K>(xt, h, wm, xm, a, cfg.ctas, smem, st); break;
     case LWQ_Q6_K: e = launch_gemm_xt<F_Q6_K>(xt, h, wm, xm, a, cfg.ctas, smem, st); break;
+    case LWQ_Q2_K: e = launch_gemm_xt<F_Q2_K>(xt, h, wm, xm, a, cfg.ctas, smem, st); break;
     default: e = launch_gemm_xt<F_Q4_K>(xt, h, wm, xm, a, cfg.ctas, smem, st); break;
     }
     if (e != cudaSuccess) return LWQ_ERR_CUDA;

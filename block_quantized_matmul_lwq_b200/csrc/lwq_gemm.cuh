@@ -73,6 +73,11 @@ struct GemmFmt<F_Q5_K> { static constexpr int chunk_bytes = 176; };
 // below the 210-byte superblock (which starts 2 * ((105 c) & 7) bytes in)
 template <>
 struct GemmFmt<F_Q6_K> { static constexpr int chunk_bytes = 240; };
+// Q2_K: a 96-byte box per row and superblock, from the 16-byte boundary at or
+// below the 84-byte superblock (which starts 2 * ((42 c) & 7) bytes in: 0, 4, 8
+// or 12, so its words stay aligned); rows of 16-byte multiples need K % 1024 == 0
+template <>
+struct GemmFmt<F_Q2_K> { static constexpr int chunk_bytes = 96; };
 
 __host__ __device__ constexpr size_t gemm_a_bytes() { return (size_t)GEMM_WROWS * 128; }
 __host__ __device__ constexpr size_t gemm_b_bytes(int bn) { return (size_t)bn * 128; }
@@ -350,6 +355,32 @@ struct Dequant<F_Q6_K, XT> {
     }
 };
 
+// Q2_K: k-block kb = elements 64kb .. 64kb+63 of the superblock; (h, v) takes the
+// 16-weight sub-block 4kb + 2h + v, elements 128n + 32j + 16v + i (n = kb/2,
+// j = 2(kb & 1) + h, i < 16), whose codes are bits 2j, 2j+1 of qs[32n + 16v + i]
+// (qs at 16), scale and min the nibbles of s[4kb + 2h + v]; w = d sc q - dmin m,
+// rounded once.  prow: the row's superblock (4-byte aligned).
+template <int XT>
+struct Dequant<F_Q2_K, XT> {
+    static __device__ __forceinline__ void run(uint32_t prow, int kb, int h, int v, uint32_t a_base, int r) {
+        const int n = kb >> 1, j = 2 * (kb & 1) + h, sb = 4 * kb + 2 * h + v;
+        const uint32_t dw = lds32(prow + 80);                       // d | dmin
+        const uint32_t sbyte = (lds32(prow + (uint32_t)(sb & ~3)) >> (8 * (sb & 3))) & 0xFFu;
+        const float ds = f16_bits_to_float(dw) * (float)(sbyte & 15u);           // exact in fp32
+        const float dm = f16_bits_to_float(dw >> 16) * (float)(sbyte >> 4);      // exact in fp32
+        const uint32_t q = prow + 16u + 32u * (uint32_t)n + 16u * (uint32_t)v;
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] = (lds32(q + 4 * i) >> (2 * j)) & 0x03030303u;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            uint32_t o[4];
+            kq_codes_to_chunk<XT>(w[2 * c], w[2 * c + 1], ds, -8388608.0f, -dm, o);
+            st_shared_v4(a_base + sw128_chunk_offset(r, 4 * h + 2 * v + c), o[0], o[1], o[2], o[3]);
+        }
+    }
+};
+
 // -------------------------------------------------------------------- kernel
 // H = 128-row halves of a weight tile (1 or 2).  With H = 2 the tile is 256
 // weight rows: two UMMAs per K step (one per half, into two accumulators)
@@ -444,8 +475,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     // Wq only: callers that allow overlap promise it is not written by preceding work
                     if (ci >= P && !(ok = mbar_wait(&p_empty[ps], pph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
                     mbar_arrive_expect_tx(&p_full[ps], P_BYTES);
-                    // Q6_K: the box starts at the 16-byte boundary at or below the superblock
-                    const int x0 = FMT == F_Q6_K ? (105 * c) & ~7 : c * (CB / 2);
+                    // Q6_K, Q2_K: the box starts at the 16-byte boundary at or below the superblock
+                    const int x0 = FMT == F_Q6_K ? (105 * c) & ~7 : (FMT == F_Q2_K ? (42 * c) & ~7 : c * (CB / 2));
 #pragma unroll
                     for (int hh = 0; hh < H; ++hh)   // rows past N read zeros
                         tma_load_2d(pk + (size_t)ps * P_BYTES + hh * PH_BYTES, &wmap, &p_full[ps], x0,
@@ -545,9 +576,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             const int c0 = ks * a.cps, c1 = min(a.nchunks, c0 + a.cps);
             for (int c = c0; ok && c < c1; ++c) {
                 if (!(ok = mbar_wait(&p_full[ps], pph, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
-                // (Q6_K: the superblock lies 2 * ((105 c) & 7) bytes into its box)
+                // (Q6_K, Q2_K: the superblock lies 2 * ((105 c) & 7), 2 * ((42 c) & 7) bytes into its box)
                 const uint32_t prow = smem_u32(pk) + (uint32_t)(ps * P_BYTES + r * CB) +
-                                      (FMT == F_Q6_K ? 2u * (uint32_t)((105 * c) & 7) : 0u);
+                                      (FMT == F_Q6_K ? 2u * (uint32_t)((105 * c) & 7)
+                                                     : (FMT == F_Q2_K ? 2u * (uint32_t)((42 * c) & 7) : 0u));
                 // BATCH k-blocks per batch; the A ring's depth is a multiple of BATCH, so a batch never wraps
                 for (int kb = 0; kb < GEMM_KB_PER_CHUNK; kb += BATCH, kbi += BATCH) {
                     if (kbi >= SA) {
@@ -636,15 +668,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // Formats with a tcgen05 GEMM decoder; their packed rows must be 16-byte
 // multiples (the weight tensor map's row stride): Q6_K needs K % 2048 == 0.
 inline bool gemm_format(int wf) {
-    return wf == LWQ_Q8_0 || wf == LWQ_Q4_0 || wf == LWQ_Q4_K || wf == LWQ_Q5_K || wf == LWQ_Q6_K;
+    return wf == LWQ_Q8_0 || wf == LWQ_Q4_0 || wf == LWQ_Q4_K || wf == LWQ_Q5_K || wf == LWQ_Q6_K || wf == LWQ_Q2_K;
 }
+// rows that a tensor map can take: Q6_K (210-byte superblocks) needs K % 2048, Q2_K (84) K % 1024
 inline bool gemm_eligible(int wf, int xt, long K) {
-    return gemm_format(wf) && (xt == X_F16 || xt == X_BF16) && K % (wf == LWQ_Q6_K ? 2048 : 256) == 0;
+    const long kmul = wf == LWQ_Q6_K ? 2048 : (wf == LWQ_Q2_K ? 1024 : 256);
+    return gemm_format(wf) && (xt == X_F16 || xt == X_BF16) && K % kmul == 0;
 }
 
-// bytes of one row of a packed chunk in a stage (Q6_K: its 240-byte box)
+// bytes of one row of a packed chunk in a stage (Q6_K, Q2_K: their 240- and 96-byte boxes)
 inline int gemm_chunk_bytes(int wf) {
-    return wf == LWQ_Q8_0 ? 272 : (wf == LWQ_Q5_K ? 176 : (wf == LWQ_Q6_K ? 240 : 144));
+    return wf == LWQ_Q8_0 ? 272 : (wf == LWQ_Q5_K ? 176 : (wf == LWQ_Q6_K ? 240 : (wf == LWQ_Q2_K ? 96 : 144)));
 }
 
 // Ring depths.  128-row tiles: 4 dequantized A stages (made on chip, two per

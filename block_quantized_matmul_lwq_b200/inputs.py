@@ -310,6 +310,7 @@ WORKLOADS = {
     # and their prefill GEMM at the up-projection shape (bf16 activations, 512 tokens)
     "q6_k_prefill_gemm": dict(fmt="q6_k", act="bf16", Ms=[512], shapes=[(11008, 4096)], seeds=[0]),
     "q5_k_prefill_gemm": dict(fmt="q5_k", act="bf16", Ms=[512], shapes=[(11008, 4096)], seeds=[0]),
+    "q2_k_prefill_gemm": dict(fmt="q2_k", act="bf16", Ms=[512], shapes=[(11008, 4096)], seeds=[0]),
 }
 
 # Decode attention workloads: one query token per sequence against its key/value cache.

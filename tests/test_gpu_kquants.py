@@ -74,6 +74,26 @@ def test_q6_k_gemm(dev, a, M, N, K, tile_n):
     check_full("q6_k", a, M, N, K, dev, seed=M + K, cfg=cfg)
 
 
+@pytest.mark.parametrize("a", ["bf16", "f16"])
+@pytest.mark.parametrize("M,N,K,tile_n", [(40, 300, 1024, 0), (130, 1000, 4096, 0), (200, 520, 3072, 128),
+                                          (64, 700, 4096, 256), (17, 96, 2048, 0)])
+def test_q2_k_gemm(dev, a, M, N, K, tile_n):
+    """Q2_K on the tcgen05 GEMM (K a multiple of 1024): per-superblock 96-byte boxes whose superblock
+    starts 0, 4, 8 or 12 bytes in."""
+    cfg = None
+    if tile_n:
+        cfg = lwq.lwq_config()
+        cfg.path, cfg.tile_n = 2, tile_n
+    assert lwq.lwq_select_config(lwq.fmt_code("q2_k", a), M, N, K).path == 2
+    check_full("q2_k", a, M, N, K, dev, seed=M + K + 1, cfg=cfg)
+
+
+def test_q2_k_prefill_gemm_sampled(dev):
+    M, N, K = 512, 11008, 4096
+    assert lwq.lwq_select_config(lwq.fmt_code("q2_k", "bf16"), M, N, K).path == 2
+    check_sampled("q2_k", "bf16", M, N, K, dev, seed=19, count=2000)
+
+
 def test_q6_k_prefill_gemm_sampled(dev):
     M, N, K = 512, 11008, 4096
     assert lwq.lwq_select_config(lwq.fmt_code("q6_k", "bf16"), M, N, K).path == 2
