@@ -180,7 +180,7 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
         path = 1;
     }
     if (!path) {
-        if (M > 16 && xt != X_F32 && gemm_eligible(wf, xt, K))
+        if (M > 16 && xt != X_F32 && gemm_eligible(wf, xt, N, K))
             path = 2;
         else if (tc_gemv_eligible(wf, N, K))
             path = 1;
@@ -189,7 +189,7 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
     }
     p->cfg.path = path;
     if (path == 2) {
-        if (!gemm_eligible(wf, xt, K)) return LWQ_ERR_UNSUPPORTED;
+        if (!gemm_eligible(wf, xt, N, K)) return LWQ_ERR_UNSUPPORTED;
         GemmPlan gp;
         int rc = gemm_plan(wf, xt, M, N, K, force, sms, &gp);
         if (rc) return rc;
@@ -534,8 +534,19 @@ int gemm_launch(int wf, int xt, const void *Wq, const void *x, float *y, int M, 
                 cudaStream_t st, int *launches) {
     const int cb = gemm_chunk_bytes(wf);
     const int bn = cfg.tile_m;
+    const bool slots = gemm_row_slots(wf, K);
     CUtensorMap wm, xm;
-    {
+    if (slots) {
+        // row slots copy without a tensor map; the kernel's map argument is then this flat view
+        // of the matrix as 16-byte units, which it does not read
+        MapReq r = map_req(Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, CU_TENSOR_MAP_SWIZZLE_NONE);
+        r.dims[0] = 16;
+        r.dims[1] = (cuuint64_t)((long)N * rb / 16);
+        r.strides[0] = 16;
+        r.box[0] = 16;
+        r.box[1] = 1;
+        if (encode_cached(r, &wm)) return LWQ_ERR_CUDA;
+    } else {
         MapReq r = map_req(Wq, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, CU_TENSOR_MAP_SWIZZLE_NONE);
         r.dims[0] = (cuuint64_t)(rb / 2);
         r.dims[1] = (cuuint64_t)N;
@@ -578,6 +589,9 @@ int gemm_launch(int wf, int xt, const void *Wq, const void *x, float *y, int M, 
     }
     a.timeout_ns = timeout_ns;
     a.overlap = overlap;
+    a.slots = slots ? 1 : 0;
+    a.wq = Wq;
+    a.row_bytes = rb;
     cudaError_t e;
     switch (wf) {
     case LWQ_Q4_0: e = launch_gemm_xt<F_Q4_0>(xt, h, wm, xm, a, cfg.ctas, smem, st); break;

@@ -57,6 +57,13 @@ struct GemmArgs {
     int p_stages;     // packed weight chunks (TMA from HBM)
     unsigned long long timeout_ns;
     int overlap;      // host side: launch with programmatic stream serialization
+    // Q6_K and Q2_K rows that are not 16-byte multiples: row slots.  Each row's superblock of
+    // a chunk is its own bulk copy (cp.async.bulk, no tensor map) of the 16-byte units that hold
+    // it, into the row's place in the stage (chunk_bytes apart), so the superblock starts
+    // (n rb + sb c) mod 16 bytes in.  Rows past N copy row N - 1 (their outputs are not stored).
+    int slots;
+    const void *wq;   // the packed weights (row slots only)
+    long row_bytes;   // rb
 };
 
 template <int FMT>
@@ -462,7 +469,55 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         // Lane 0 streams the packed weight chunks (p ring), lane 1 the activation
         // k-blocks (ab ring), each as far ahead as its ring allows: a weight chunk
         // is requested as soon as its slot frees, not behind the activation loads.
-        if (lane == 0) {
+        // Row slots: lanes 0 and 2..31 share a stage's row copies (lane 0 waits
+        // and arrives for them).
+        bool slot_lane = false;
+        if constexpr (FMT == F_Q6_K || FMT == F_Q2_K) slot_lane = a.slots && lane != 1;
+        if (slot_lane) {
+            constexpr int SBB = FMT == F_Q6_K ? 210 : 84;   // superblock bytes
+            constexpr unsigned MASK = 0xFFFFFFFDu;          // every lane but 1
+            const int li = lane == 0 ? 0 : lane - 1;        // 0..30
+            const uint8_t *wq = static_cast<const uint8_t *>(a.wq);
+            int ci = 0, ps = 0;
+            uint32_t pph = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+                const int tile = item / a.splits, ks = item % a.splits;
+                const int wt = tile / a.n_ttiles;
+                const int c0 = ks * a.cps, c1 = min(a.nchunks, c0 + a.cps);
+                for (int c = c0; ok && c < c1; ++c, ++ci) {
+                    if (lane == 0 && ci >= P) ok = mbar_wait(&p_empty[ps], pph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT);
+                    ok = __shfl_sync(MASK, ok, 0);
+                    if (!ok) break;
+                    // bytes of the stage's copies, then lane 0 arrives expecting them, then the copies
+                    uint32_t bytes = 0;
+                    for (int rr = li; rr < WR; rr += 31) {
+                        const long n = min(wt * WR + rr, a.N - 1);
+                        const uint32_t o = (uint32_t)((n * a.row_bytes + (long)SBB * c) & 15);
+                        bytes += (o + SBB + 15) & ~15u;
+                    }
+                    bytes = __reduce_add_sync(MASK, bytes);
+                    if (lane == 0) mbar_arrive_expect_tx(&p_full[ps], bytes);
+                    __syncwarp(MASK);
+                    for (int rr = li; rr < WR; rr += 31) {
+                        const long n = min(wt * WR + rr, a.N - 1);
+                        const long b0 = n * a.row_bytes + (long)SBB * c;
+                        const uint32_t o = (uint32_t)(b0 & 15);
+                        bulk_load(pk + (size_t)ps * P_BYTES + (size_t)(rr / GEMM_WROWS) * PH_BYTES +
+                                      (size_t)(rr % GEMM_WROWS) * CB,
+                                  wq + (b0 - o), (o + SBB + 15) & ~15u, &p_full[ps]);
+                    }
+                    if (++ps == P) {
+                        ps = 0;
+                        pph ^= 1u;
+                    }
+                }
+            }
+            // drain: the last copies land before the CTA may exit
+            if (lane == 0)
+                for (int j = max(0, ci - P); j < ci; ++j)
+                    mbar_wait(&p_full[j % P], (j / P) & 1, a.timeout_ns, DEVERR_GEMM_WAIT);
+        } else if (lane == 0) {
             tma_prefetch_desc(&wmap);
             int ci = 0, ps = 0;
             uint32_t pph = 0;
@@ -573,13 +628,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         bool ok = true;
         for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
             const int ks = item % a.splits;
+            const int wt = item / a.splits / a.n_ttiles;
             const int c0 = ks * a.cps, c1 = min(a.nchunks, c0 + a.cps);
             for (int c = c0; ok && c < c1; ++c) {
                 if (!(ok = mbar_wait(&p_full[ps], pph, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
-                // (Q6_K, Q2_K: the superblock lies 2 * ((105 c) & 7), 2 * ((42 c) & 7) bytes into its box)
-                const uint32_t prow = smem_u32(pk) + (uint32_t)(ps * P_BYTES + r * CB) +
-                                      (FMT == F_Q6_K ? 2u * (uint32_t)((105 * c) & 7)
-                                                     : (FMT == F_Q2_K ? 2u * (uint32_t)((42 * c) & 7) : 0u));
+                // (Q6_K, Q2_K: the superblock lies 2 * ((105 c) & 7), 2 * ((42 c) & 7) bytes into its box, or
+                // with row slots (n rb + sb c) mod 16 bytes into its place)
+                uint32_t off = FMT == F_Q6_K ? 2u * (uint32_t)((105 * c) & 7)
+                                             : (FMT == F_Q2_K ? 2u * (uint32_t)((42 * c) & 7) : 0u);
+                if constexpr (FMT == F_Q6_K || FMT == F_Q2_K) {
+                    if (a.slots) {
+                        const long n = min(wt * WR + r, a.N - 1);
+                        off = (uint32_t)((n * a.row_bytes + (long)(FMT == F_Q6_K ? 210 : 84) * c) & 15);
+                    }
+                }
+                const uint32_t prow = smem_u32(pk) + (uint32_t)(ps * P_BYTES + r * CB) + off;
                 // BATCH k-blocks per batch; the A ring's depth is a multiple of BATCH, so a batch never wraps
                 for (int kb = 0; kb < GEMM_KB_PER_CHUNK; kb += BATCH, kbi += BATCH) {
                     if (kbi >= SA) {
@@ -670,10 +733,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 inline bool gemm_format(int wf) {
     return wf == LWQ_Q8_0 || wf == LWQ_Q4_0 || wf == LWQ_Q4_K || wf == LWQ_Q5_K || wf == LWQ_Q6_K || wf == LWQ_Q2_K;
 }
-// rows that a tensor map can take: Q6_K (210-byte superblocks) needs K % 2048, Q2_K (84) K % 1024
-inline bool gemm_eligible(int wf, int xt, long K) {
-    const long kmul = wf == LWQ_Q6_K ? 2048 : (wf == LWQ_Q2_K ? 1024 : 256);
-    return gemm_format(wf) && (xt == X_F16 || xt == X_BF16) && K % kmul == 0;
+// Q6_K (210-byte superblocks) and Q2_K (84) rows are 16-byte multiples, which a tensor map can take
+// as its rows, when K % 2048 and K % 1024 == 0; other K stream as row slots (GemmArgs::slots), whose
+// copies need the whole matrix to be 16-byte units
+inline bool gemm_row_slots(int wf, long K) {
+    return (wf == LWQ_Q6_K && K % 2048 != 0) || (wf == LWQ_Q2_K && K % 1024 != 0);
+}
+inline bool gemm_eligible(int wf, int xt, long N, long K) {
+    if (!gemm_format(wf) || (xt != X_F16 && xt != X_BF16) || K % 256 != 0) return false;
+    if (gemm_row_slots(wf, K)) return (N * (K / 256) * (wf == LWQ_Q6_K ? 210 : 84)) % 16 == 0;
+    return true;
 }
 
 // bytes of one row of a packed chunk in a stage (Q6_K, Q2_K: their 240- and 96-byte boxes)

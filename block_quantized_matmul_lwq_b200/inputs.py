@@ -307,10 +307,14 @@ WORKLOADS = {
     "q2_k_7b_layer_decode": dict(fmt="q2_k", act="f16", Ms=[1],
                                  shapes=[(4096, 4096)] * 4 + [(11008, 4096), (11008, 4096), (4096, 11008)],
                                  seeds=[0, 1, 2, 3, 4, 5, 6]),
-    # and their prefill GEMM at the up-projection shape (bf16 activations, 512 tokens)
-    "q6_k_prefill_gemm": dict(fmt="q6_k", act="bf16", Ms=[512], shapes=[(11008, 4096)], seeds=[0]),
-    "q5_k_prefill_gemm": dict(fmt="q5_k", act="bf16", Ms=[512], shapes=[(11008, 4096)], seeds=[0]),
-    "q2_k_prefill_gemm": dict(fmt="q2_k", act="bf16", Ms=[512], shapes=[(11008, 4096)], seeds=[0]),
+    # and their prefill GEMM at the up- and down-projection shapes (bf16 activations, 512 tokens; the
+    # down projection's Q6_K and Q2_K rows are not 16-byte multiples and stream as row slots)
+    "q6_k_prefill_gemm": dict(fmt="q6_k", act="bf16", Ms=[512, 512], shapes=[(11008, 4096), (4096, 11008)],
+                              seeds=[0, 0]),
+    "q5_k_prefill_gemm": dict(fmt="q5_k", act="bf16", Ms=[512, 512], shapes=[(11008, 4096), (4096, 11008)],
+                              seeds=[0, 0]),
+    "q2_k_prefill_gemm": dict(fmt="q2_k", act="bf16", Ms=[512, 512], shapes=[(11008, 4096), (4096, 11008)],
+                              seeds=[0, 0]),
 }
 
 # Decode attention workloads: one query token per sequence against its key/value cache.

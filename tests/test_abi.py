@@ -173,11 +173,10 @@ def test_gemm_tile_choices_are_valid():
 
 
 def test_more_kquant_formats_routing_and_row_bytes():
-    """Q5_K takes the tensor-core paths; Q6_K the tensor-core GEMV (row slots where its rows are not
-    16-byte multiples) and, with K a multiple of 2048, the tcgen05 GEMM; Q2_K the tensor-core GEMV
-    (row slots) and, with K a multiple of 1024, the tcgen05 GEMM; both fall back to the simple kernel
-    only when the whole matrix is not a 16-byte multiple; row bytes follow the superblock sizes 176,
-    210 and 84."""
+    """Q5_K takes the tensor-core paths; Q6_K and Q2_K the tensor-core GEMV and the tcgen05 GEMM too,
+    their rows streamed as row slots where they are not 16-byte multiples; they fall back to the
+    simple kernel (any M) only when the whole matrix is not a 16-byte multiple; row bytes follow the
+    superblock sizes 176, 210 and 84."""
     for M, path in ((1, 1), (16, 1), (17, 2), (512, 2)):
         assert lwq.lwq_select_config(lwq.fmt_code("q5_k", "f16"), M, 4096, 4096).path == path
     for M, K, path in ((1, 4096, 1), (16, 14336, 1), (1, 11008, 1), (8, 2816, 1), (17, 4096, 1), (40, 11008, 1)):
@@ -185,11 +184,12 @@ def test_more_kquant_formats_routing_and_row_bytes():
     assert lwq.lwq_select_config(lwq.fmt_code("q6_k", "f32"), 1, 4095, 11008).path == 3   # 4095 x 9030 bytes
     # 16-bit activations, M > 16: the tcgen05 GEMM where the rows allow it, else the GEMV in passes
     assert lwq.lwq_select_config(lwq.fmt_code("q6_k", "bf16"), 17, 4096, 4096).path == 2
-    assert lwq.lwq_select_config(lwq.fmt_code("q6_k", "bf16"), 512, 4096, 11008).path == 1
+    assert lwq.lwq_select_config(lwq.fmt_code("q6_k", "bf16"), 512, 4096, 11008).path == 2   # row slots
+    assert lwq.lwq_select_config(lwq.fmt_code("q6_k", "bf16"), 512, 4095, 11008).path == 3   # not 16-byte units
     for M in (1, 16, 17, 512):
         # the tcgen05 GEMM for M > 16 when the rows are 16-byte multiples (K % 1024 == 0)
         assert lwq.lwq_select_config(lwq.fmt_code("q2_k", "f16"), M, 4096, 4096).path == (1 if M <= 16 else 2)
-        assert lwq.lwq_select_config(lwq.fmt_code("q2_k", "f16"), M, 4096, 11008).path == 1
+        assert lwq.lwq_select_config(lwq.fmt_code("q2_k", "f16"), M, 4096, 11008).path == (1 if M <= 16 else 2)
         assert lwq.lwq_select_config(lwq.fmt_code("q2_k", "f16"), M, 4097, 11008).path == 3
     for w, K, rb in (("q6_k", 4096, 3360), ("q6_k", 11008, 9030), ("q5_k", 4096, 2816), ("q2_k", 11008, 3612)):
         assert lwq.lwq_row_bytes(lwq.fmt_code(w, "f16"), K) == rb == inputs.row_bytes(w, K)

@@ -88,6 +88,29 @@ def test_q2_k_gemm(dev, a, M, N, K, tile_n):
     check_full("q2_k", a, M, N, K, dev, seed=M + K + 1, cfg=cfg)
 
 
+@pytest.mark.parametrize("w", ["q6_k", "q2_k"])
+@pytest.mark.parametrize("a", ["bf16", "f16"])
+@pytest.mark.parametrize("M,N,K,tile_n,splits", [(40, 48, 2816, 0, 0), (130, 296, 4352, 0, 0), (64, 520, 11008, 256, 0),
+                                                 (200, 136, 1536, 128, 3), (17, 264, 11008, 0, 0)])
+def test_row_slot_gemm(dev, w, a, M, N, K, tile_n, splits):
+    """Q6_K and Q2_K rows that are not 16-byte multiples on the tcgen05 GEMM: one bulk copy per row and
+    superblock, superblocks starting at every 2-byte (Q6_K) or 4-byte (Q2_K) offset, rows past N."""
+    cfg = None
+    if tile_n or splits:
+        cfg = lwq.lwq_config()
+        cfg.path, cfg.tile_n, cfg.splits = 2, tile_n, splits
+    assert lwq.lwq_select_config(lwq.fmt_code(w, a), M, N, K).path == 2
+    check_full(w, a, M, N, K, dev, seed=M + N + K, cfg=cfg)
+
+
+@pytest.mark.parametrize("w", ["q6_k", "q2_k"])
+def test_row_slot_prefill_down_projection(dev, w):
+    """The 7B down projection (K = 11008) at 512 tokens, sampled outputs plus every tile edge."""
+    M, N, K = 512, 4096, 11008
+    assert lwq.lwq_select_config(lwq.fmt_code(w, "bf16"), M, N, K).path == 2
+    check_sampled(w, "bf16", M, N, K, dev, seed=23, count=2000)
+
+
 def test_q2_k_prefill_gemm_sampled(dev):
     M, N, K = 512, 11008, 4096
     assert lwq.lwq_select_config(lwq.fmt_code("q2_k", "bf16"), M, N, K).path == 2
