@@ -19,11 +19,9 @@
  *   M >  16  prefill GEMM: packed tiles staged by TMA, dequantized to
  *            bf16/fp16 in shared memory, tcgen05 MMAs accumulating in TMEM.
  * Q6_K rows that are not 16-byte multiples (K not a multiple of 2048) and Q2_K
- * rows stream into the GEMV as slots of the flat matrix (whole 16-byte units
- * per row), which needs N * lwq_row_bytes(fmt, K) to be a multiple of 16.  The
- * tcgen05 GEMM takes Q6_K with K a multiple of 2048 and Q2_K with K a multiple
- * of 1024; other Q6_K and Q2_K shapes with M > 16 run the GEMV over groups of
- * rows.  Shapes
+ * rows (K not a multiple of 1024) stream as slots of the flat matrix (whole
+ * 16-byte units per row) into both paths, which needs N * lwq_row_bytes(fmt,
+ * K) to be a multiple of 16.  Shapes
  * no tensor-core path takes (K not a multiple of 256, or such a matrix that is
  * not a whole number of 16-byte units) run a simple GEMV kernel.
  *
