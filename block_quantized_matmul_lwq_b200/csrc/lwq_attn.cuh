@@ -84,13 +84,6 @@ __device__ __forceinline__ void transpose_reduce(float (&val)[V], int lane) {
 
 // Asynchronous global -> shared copies (cp.async) of 4, 8 or 16 bytes, grouped
 // per thread; a warp barrier after the wait makes them visible to the warp.
-template <int BYTES>
-__device__ __forceinline__ void cp_async(uint32_t dst, const void *src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(dst), "l"(src), "n"(BYTES) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 struct AttnArgs {
     const uint16_t *q, *k, *v;

@@ -57,10 +57,11 @@ struct GemmArgs {
     int p_stages;     // packed weight chunks (TMA from HBM)
     unsigned long long timeout_ns;
     int overlap;      // host side: launch with programmatic stream serialization
-    // Q6_K and Q2_K rows that are not 16-byte multiples: row slots.  Each row's superblock of
-    // a chunk is its own bulk copy (cp.async.bulk, no tensor map) of the 16-byte units that hold
-    // it, into the row's place in the stage (chunk_bytes apart), so the superblock starts
-    // (n rb + sb c) mod 16 bytes in.  Rows past N copy row N - 1 (their outputs are not stored).
+    // Q6_K and Q2_K rows that are not 16-byte multiples: row slots.  The dequantizer warps
+    // fetch their own rows: each row's superblock of a chunk is copied as the 16-byte units that
+    // hold it (cp.async, 16 bytes per thread and copy) into the row's place in the stage
+    // (chunk_bytes apart), so the superblock starts (n rb + sb c) mod 16 bytes in.  Rows past N
+    // copy row N - 1 (their outputs are not stored).
     int slots;
     const void *wq;   // the packed weights (row slots only)
     long row_bytes;   // rb
@@ -469,55 +470,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         // Lane 0 streams the packed weight chunks (p ring), lane 1 the activation
         // k-blocks (ab ring), each as far ahead as its ring allows: a weight chunk
         // is requested as soon as its slot frees, not behind the activation loads.
-        // Row slots: lanes 0 and 2..31 share a stage's row copies (lane 0 waits
-        // and arrives for them).
-        bool slot_lane = false;
-        if constexpr (FMT == F_Q6_K || FMT == F_Q2_K) slot_lane = a.slots && lane != 1;
-        if (slot_lane) {
-            constexpr int SBB = FMT == F_Q6_K ? 210 : 84;   // superblock bytes
-            constexpr unsigned MASK = 0xFFFFFFFDu;          // every lane but 1
-            const int li = lane == 0 ? 0 : lane - 1;        // 0..30
-            const uint8_t *wq = static_cast<const uint8_t *>(a.wq);
-            int ci = 0, ps = 0;
-            uint32_t pph = 0;
-            bool ok = true;
-            for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
-                const int tile = item / a.splits, ks = item % a.splits;
-                const int wt = tile / a.n_ttiles;
-                const int c0 = ks * a.cps, c1 = min(a.nchunks, c0 + a.cps);
-                for (int c = c0; ok && c < c1; ++c, ++ci) {
-                    if (lane == 0 && ci >= P) ok = mbar_wait(&p_empty[ps], pph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT);
-                    ok = __shfl_sync(MASK, ok, 0);
-                    if (!ok) break;
-                    // bytes of the stage's copies, then lane 0 arrives expecting them, then the copies
-                    uint32_t bytes = 0;
-                    for (int rr = li; rr < WR; rr += 31) {
-                        const long n = min(wt * WR + rr, a.N - 1);
-                        const uint32_t o = (uint32_t)((n * a.row_bytes + (long)SBB * c) & 15);
-                        bytes += (o + SBB + 15) & ~15u;
-                    }
-                    bytes = __reduce_add_sync(MASK, bytes);
-                    if (lane == 0) mbar_arrive_expect_tx(&p_full[ps], bytes);
-                    __syncwarp(MASK);
-                    for (int rr = li; rr < WR; rr += 31) {
-                        const long n = min(wt * WR + rr, a.N - 1);
-                        const long b0 = n * a.row_bytes + (long)SBB * c;
-                        const uint32_t o = (uint32_t)(b0 & 15);
-                        bulk_load(pk + (size_t)ps * P_BYTES + (size_t)(rr / GEMM_WROWS) * PH_BYTES +
-                                      (size_t)(rr % GEMM_WROWS) * CB,
-                                  wq + (b0 - o), (o + SBB + 15) & ~15u, &p_full[ps]);
-                    }
-                    if (++ps == P) {
-                        ps = 0;
-                        pph ^= 1u;
-                    }
-                }
-            }
-            // drain: the last copies land before the CTA may exit
-            if (lane == 0)
-                for (int j = max(0, ci - P); j < ci; ++j)
-                    mbar_wait(&p_full[j % P], (j / P) & 1, a.timeout_ns, DEVERR_GEMM_WAIT);
-        } else if (lane == 0) {
+        // With row slots the dequantizer warps fetch the weights themselves (lane 0 idles).
+        bool slot_mode = false;
+        if constexpr (FMT == F_Q6_K || FMT == F_Q2_K) slot_mode = a.slots != 0;
+        if (lane == 0 && !slot_mode) {
             tma_prefetch_desc(&wmap);
             int ci = 0, ps = 0;
             uint32_t pph = 0;
@@ -626,53 +582,101 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         int kbi = 0, s = 0, ps = 0;
         uint32_t ph = 0, pph = 0;
         bool ok = true;
-        for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
-            const int ks = item % a.splits;
-            const int wt = item / a.splits / a.n_ttiles;
-            const int c0 = ks * a.cps, c1 = min(a.nchunks, c0 + a.cps);
-            for (int c = c0; ok && c < c1; ++c) {
-                if (!(ok = mbar_wait(&p_full[ps], pph, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
-                // (Q6_K, Q2_K: the superblock lies 2 * ((105 c) & 7), 2 * ((42 c) & 7) bytes into its box, or
-                // with row slots (n rb + sb c) mod 16 bytes into its place)
-                uint32_t off = FMT == F_Q6_K ? 2u * (uint32_t)((105 * c) & 7)
-                                             : (FMT == F_Q2_K ? 2u * (uint32_t)((42 * c) & 7) : 0u);
-                if constexpr (FMT == F_Q6_K || FMT == F_Q2_K) {
-                    if (a.slots) {
-                        const long n = min(wt * WR + r, a.N - 1);
-                        off = (uint32_t)((n * a.row_bytes + (long)(FMT == F_Q6_K ? 210 : 84) * c) & 15);
-                    }
-                }
-                const uint32_t prow = smem_u32(pk) + (uint32_t)(ps * P_BYTES + r * CB) + off;
-                // BATCH k-blocks per batch; the A ring's depth is a multiple of BATCH, so a batch never wraps
-                for (int kb = 0; kb < GEMM_KB_PER_CHUNK; kb += BATCH, kbi += BATCH) {
-                    if (kbi >= SA) {
-#pragma unroll
-                        for (int j = 0; j < BATCH; ++j)
-                            if (ok && !(ok = mbar_wait(&a_empty[s + j], ph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
-                        if (!ok) break;
-                    }
+        // the four k-blocks of one packed chunk (row r's superblock at prow)
+        auto dequant_chunk = [&](uint32_t prow) {
+            // BATCH k-blocks per batch; the A ring's depth is a multiple of BATCH, so a batch never wraps
+            for (int kb = 0; kb < GEMM_KB_PER_CHUNK; kb += BATCH, kbi += BATCH) {
+                if (kbi >= SA) {
 #pragma unroll
                     for (int j = 0; j < BATCH; ++j)
+                        if (ok && !(ok = mbar_wait(&a_empty[s + j], ph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
+                    if (!ok) break;
+                }
 #pragma unroll
-                        for (int hh = 0; hh < H; ++hh)
-                            Dequant<FMT, XT>::run(prow + hh * PH_BYTES, kb + j, h, v,
-                                                  smem_u32(As + (size_t)(s + j) * A_BYTES + hh * AH_BYTES), r);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
+                for (int j = 0; j < BATCH; ++j)
 #pragma unroll
-                        for (int j = 0; j < BATCH; ++j) mbar_arrive(&a_full[s + j]);
+                    for (int hh = 0; hh < H; ++hh)
+                        Dequant<FMT, XT>::run(prow + hh * PH_BYTES, kb + j, h, v,
+                                              smem_u32(As + (size_t)(s + j) * A_BYTES + hh * AH_BYTES), r);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+#pragma unroll
+                    for (int j = 0; j < BATCH; ++j) mbar_arrive(&a_full[s + j]);
+                }
+                if ((s += BATCH) == SA) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+        };
+        bool slot_mode = false;
+        if constexpr (FMT == F_Q6_K || FMT == F_Q2_K) slot_mode = a.slots != 0;
+        if (slot_mode) {
+            if constexpr (FMT == F_Q6_K || FMT == F_Q2_K) {
+                // Row slots: this warp's rows (8 of each half) are fetched by the warp itself, P - 1
+                // chunks ahead along the CTA's (item, chunk) sequence, with 16-byte cp.async: a warp
+                // reads only its own rows, so a warp barrier orders the copies and the reads.
+                constexpr int SBB = FMT == F_Q6_K ? 210 : 84;           // superblock bytes
+                constexpr int UMAX = (SBB + 15 + 15) / 16;              // 16-byte units a row's copy may take
+                const uint8_t *wq = static_cast<const uint8_t *>(a.wq);
+                const int w8 = 8 * (t >> 5);                            // the warp's first row
+                int f_item = blockIdx.x, f_c = (blockIdx.x % a.splits) * a.cps;
+                auto fetch = [&](int slot) {
+                    if (f_item < n_items) {
+                        const int wt_f = f_item / a.splits / a.n_ttiles;
+                        for (int idx = lane; idx < 8 * H * UMAX; idx += 32) {
+                            const int rw = idx / UMAX, u = idx % UMAX;
+                            const int hh = rw >> 3, rr = w8 + (rw & 7);
+                            const long n = min(wt_f * WR + hh * GEMM_WROWS + rr, a.N - 1);
+                            const long b0 = n * a.row_bytes + (long)SBB * f_c;
+                            const int o = (int)(b0 & 15);
+                            if (u < (o + SBB + 15) / 16)
+                                cp_async_cg16(smem_u32(pk) + (uint32_t)(slot * P_BYTES + hh * PH_BYTES + rr * CB + 16 * u),
+                                              wq + (b0 - o) + 16 * u);
+                        }
+                        const int c1_f = min(a.nchunks, (f_item % a.splits) * a.cps + a.cps);
+                        if (++f_c >= c1_f) {
+                            f_item += gridDim.x;
+                            f_c = (f_item % a.splits) * a.cps;
+                        }
                     }
-                    if ((s += BATCH) == SA) {
-                        s = 0;
-                        ph ^= 1u;
+                    cp_async_commit();   // an empty group past the end keeps the counting uniform
+                };
+                for (int j = 0; j < P - 1; ++j) fetch(j);
+                int seq = 0;
+                for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+                    const int ks = item % a.splits;
+                    const int wt = item / a.splits / a.n_ttiles;
+                    const int c0 = ks * a.cps, c1 = min(a.nchunks, c0 + a.cps);
+                    for (int c = c0; ok && c < c1; ++c, ++seq) {
+                        fetch((seq + P - 1) % P);   // the slot the previous chunk freed
+                        cp_async_wait_n(P - 1);     // this chunk's copies (this thread's) have landed
+                        __syncwarp();               // ... and every lane's
+                        const long n = min(wt * WR + r, a.N - 1);
+                        const uint32_t off = (uint32_t)((n * a.row_bytes + (long)SBB * c) & 15);
+                        dequant_chunk(smem_u32(pk) + (uint32_t)((seq % P) * P_BYTES + r * CB) + off);
+                        __syncwarp();               // every lane is done with the slot before it is refilled
                     }
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&p_empty[ps]);
-                if (++ps == P) {
-                    ps = 0;
-                    pph ^= 1u;
+                cp_async_wait<0>();                 // no copy still lands after the warp is done
+            }
+        } else {
+            for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+                const int ks = item % a.splits;
+                const int c0 = ks * a.cps, c1 = min(a.nchunks, c0 + a.cps);
+                for (int c = c0; ok && c < c1; ++c) {
+                    if (!(ok = mbar_wait(&p_full[ps], pph, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
+                    // (Q6_K, Q2_K: the superblock lies 2 * ((105 c) & 7), 2 * ((42 c) & 7) bytes into its box)
+                    const uint32_t off = FMT == F_Q6_K ? 2u * (uint32_t)((105 * c) & 7)
+                                                       : (FMT == F_Q2_K ? 2u * (uint32_t)((42 * c) & 7) : 0u);
+                    dequant_chunk(smem_u32(pk) + (uint32_t)(ps * P_BYTES + r * CB) + off);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&p_empty[ps]);
+                    if (++ps == P) {
+                        ps = 0;
+                        pph ^= 1u;
+                    }
                 }
             }
         }
