@@ -625,15 +625,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 auto fetch = [&](int slot) {
                     if (f_item < n_items) {
                         const int wt_f = f_item / a.splits / a.n_ttiles;
-                        for (int idx = lane; idx < 8 * H * UMAX; idx += 32) {
-                            const int rw = idx / UMAX, u = idx % UMAX;
-                            const int hh = rw >> 3, rr = w8 + (rw & 7);
+                        // lane: row (lane >> 2) of the warp's 8 in each half, units (lane & 3) + 4 i of it
+#pragma unroll
+                        for (int hh = 0; hh < H; ++hh) {
+                            const int rr = w8 + (lane >> 2);
                             const long n = min(wt_f * WR + hh * GEMM_WROWS + rr, a.N - 1);
                             const long b0 = n * a.row_bytes + (long)SBB * f_c;
                             const int o = (int)(b0 & 15);
-                            if (u < (o + SBB + 15) / 16)
-                                cp_async_cg16(smem_u32(pk) + (uint32_t)(slot * P_BYTES + hh * PH_BYTES + rr * CB + 16 * u),
-                                              wq + (b0 - o) + 16 * u);
+                            const int units = (o + SBB + 15) / 16;
+                            const uint8_t *src = wq + (b0 - o);
+                            const uint32_t dst = smem_u32(pk) + (uint32_t)(slot * P_BYTES + hh * PH_BYTES + rr * CB);
+#pragma unroll
+                            for (int i = 0; i < (UMAX + 3) / 4; ++i) {
+                                const int u = (lane & 3) + 4 * i;
+                                if (u < units) cp_async_cg16(dst + 16 * u, src + 16 * u);
+                            }
                         }
                         const int c1_f = min(a.nchunks, (f_item % a.splits) * a.cps + a.cps);
                         if (++f_c >= c1_f) {
