@@ -230,6 +230,10 @@ __device__ __forceinline__ uint32_t q2k_pair(uint32_t v) {
     if constexpr (BF) return hfma2_bf16(and_or(v, 0x00030003u, B2_MAGIC), B2_ONE, B2_M128);
     else return hfma2_f16(and_or(v, 0x00030003u, H2_MAGIC), H2_ONE, H2_M1024);
 }
+// Q4_K / Q5_K: two 6-bit mins (bits 0-5 of each half) as exact bf16 values.
+__device__ __forceinline__ uint32_t min6_pair_bf16(uint32_t v) {
+    return hfma2_bf16(and_or(v, 0x003F003Fu, B2_MAGIC), B2_ONE, B2_M128);
+}
 // Q8_0: the int8 codes of bytes 0 and 2.  fp16: (1024 + (q + 128)) - 1152.
 // bf16 has room for 7 bits only: (128 + (q & 127)) plus -128 or -256 from the
 // sign bit, which lands on the exponent bit of 0xC300 (0xC380 is -256).
@@ -849,9 +853,12 @@ struct Exact {
                 }
             }
             // mins: y -= dmin * sum_j m_j S_j on the part-0 column of each activation row
-            // (sub-blocks 0-3: m = s[j+4] & 63; 4-7: s[j+4] >> 4 | (s[j] >> 6) << 4)
+            // (sub-blocks 0-3: m = s[j+4] & 63; 4-7: s[j+4] >> 4 | (s[j] >> 6) << 4), on the tensor
+            // cores: C = A B with A = the mins of rows g, g + 8 at k-slots 2t, 2t + 1 (the warp's
+            // sub-blocks 2t, 2t + 1; slots 8-15 empty) and B = the sums S of column g's activation
+            // row as three exact bf16 parts (zero on the other parts' columns); products exact,
+            // fp32 sums.  bf16 MMAs whatever the activation type (S needs fp32's exponent range).
             const float m0f = f16_hi(h0), m1f = f16_hi(h1);
-            const float nm0 = m0f * -8388608.f, nm1 = m1f * -8388608.f;
             const uint32_t mn0 = half == 0 ? (s20 & 0x3F3F3F3Fu) : (((s30 >> 4) & 0x0F0F0F0Fu) | ((s20 >> 2) & 0x30303030u));
             const uint32_t mn1 = half == 0 ? (s21 & 0x3F3F3F3Fu) : (((s31 >> 4) & 0x0F0F0F0Fu) | ((s21 >> 2) & 0x30303030u));
             uint32_t mnh0 = 0, mnh1 = 0;
@@ -859,23 +866,30 @@ struct Exact {
                 mnh0 = ((s30 >> 4) & 0x0F0F0F0Fu) | ((s20 >> 2) & 0x30303030u);
                 mnh1 = ((s31 >> 4) & 0x0F0F0F0Fu) | ((s21 >> 2) & 0x30303030u);
             }
+            const bool kin = 2 * t < NB;                          // k-slots 2t, 2t+1 hold sub-blocks of this warp
+            const uint32_t msel = (t & 1) ? 0x4342u : 0x4140u;    // bytes 2t, 2t+1 (mod 4) to halves 0 and 1
+            const uint32_t w0 = (NB == 8 && t >= 2) ? mnh0 : mn0, w1 = (NB == 8 && t >= 2) ? mnh1 : mn1;
+            const uint32_t am[4] = {kin ? min6_pair_bf16(prmt(w0, 0u, msel)) : 0u,
+                                    kin ? min6_pair_bf16(prmt(w1, 0u, msel)) : 0u, 0u, 0u};
+            const int g = lane >> 2;
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int c = 8 * nt + 2 * t + cc, m = c / P;
-                    if (c - m * P != 0 || m >= M) continue;
-                    float z0 = 0.f, z1 = 0.f;
-#pragma unroll
-                    for (int b = 0; b < NB; ++b) {
-                        const uint32_t mv0 = (NB == 8 && b >= 4) ? mnh0 : mn0, mv1 = (NB == 8 && b >= 4) ? mnh1 : mn1;
-                        const float sj = sxw[m * sstride + b];
-                        z0 = fmaf(fmaf(byte_magic(mv0, b & 3), m0f, nm0), sj, z0);   // (dmin * m_j) * S_j
-                        z1 = fmaf(fmaf(byte_magic(mv1, b & 3), m1f, nm1), sj, z1);
-                    }
-                    acc[nt][cc] -= z0;
-                    acc[nt][2 + cc] -= z1;
-                }
+            for (int nt = 0; nt < NT; ++nt) {
+                const int c = 8 * nt + g, m = c / P;
+                const bool live = kin && (c - m * P == 0) && m < M;
+                const float2 sv = live ? *reinterpret_cast<const float2 *>(sxw + m * sstride + 2 * t)
+                                       : make_float2(0.f, 0.f);
+                uint32_t ph0, pm0, pl0, ph1, pm1, pl1;
+                split3(sv.x, ph0, pm0, pl0);
+                split3(sv.y, ph1, pm1, pl1);
+                float cz[4];
+                mma_zero<true>(cz, am, ph0 | (ph1 << 16), 0u);
+                mma_acc<true>(cz, am, pm0 | (pm1 << 16), 0u);
+                mma_acc<true>(cz, am, pl0 | (pl1 << 16), 0u);
+                acc[nt][0] = fmaf(-m0f, cz[0], acc[nt][0]);
+                acc[nt][1] = fmaf(-m0f, cz[1], acc[nt][1]);
+                acc[nt][2] = fmaf(-m1f, cz[2], acc[nt][2]);
+                acc[nt][3] = fmaf(-m1f, cz[3], acc[nt][3]);
+            }
         }
     }
 };
