@@ -651,7 +651,7 @@ struct Exact {
     // shifted by 2j into the even pair, bytes 1 and 3 by 2j + 8 into the odd
     // one.  One MMA step per sub-block, then y += d * sc * C; the mins enter
     // once per tile, y -= dmin * sum m S over the part-0 columns.
-    __device__ __forceinline__ void compute_q2(uint32_t box, int half, float (&acc)[NT][4], int t, int M,
+    __device__ __forceinline__ void compute_q2(uint32_t box, int half, float (&acc)[NT][4], int g, int t, int M,
                                                const float *sxw, int sstride) const {
         const uint32_t r0 = box + sr0, r1 = box + sr1;
         const uint32_t h0 = lds32(r0 + 80), h1 = lds32(r1 + 80);   // d | dmin
@@ -691,28 +691,45 @@ struct Exact {
                 }
             }
         }
-        // mins: the warp's sub-blocks q = 0 .. 2 NB - 1 in element order are s bytes
-        // 8n + q (n = the warp's first half), sums sxw[m * sstride + q]
+        // mins: the warp's sub-blocks q = 0 .. 2 NB - 1 in element order are s bytes 8n + q (n =
+        // the warp's first half), sums sxw[m * sstride + q].  y -= dmin * sum_q m_q S_q on the tensor
+        // cores: k-slot q holds sub-block q (A: the 4-bit mins of rows g, g + 8; B: S of column g's
+        // activation row as three exact bf16 parts, zero on the other parts' columns).
         const float m0f = f16_hi(h0), m1f = f16_hi(h1);
-        const float nm0 = m0f * -8388608.f, nm1 = m1f * -8388608.f;
+        const uint32_t msel = (t & 1) ? 0x4342u : 0x4140u;   // bytes 2t, 2t+1 (mod 4) to halves 0 and 1
+        uint32_t am[4];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+        for (int hi = 0; hi < 2; ++hi) {   // k-slots 2t, 2t+1 (hi = 0) and 2t+8, 2t+9 (hi = 1)
+            const bool kin = hi == 0 || NB == 8;
+            am[2 * hi] = kin ? min6_pair_bf16(prmt((sc[hi & (NH - 1)][0][t >> 1] >> 4) & 0x0F0F0F0Fu, 0u, msel)) : 0u;
+            am[2 * hi + 1] = kin ? min6_pair_bf16(prmt((sc[hi & (NH - 1)][1][t >> 1] >> 4) & 0x0F0F0F0Fu, 0u, msel)) : 0u;
+        }
 #pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const int c = 8 * nt + 2 * t + cc, m = c / P;
-                if (c - m * P != 0 || m >= M) continue;
-                float z0 = 0.f, z1 = 0.f;
+        for (int nt = 0; nt < NT; ++nt) {
+            const int c = 8 * nt + g, m = c / P;
+            const bool live = (c - m * P == 0) && m < M;
+            uint32_t b[2][3];   // [k-slot half][part]
 #pragma unroll
-                for (int q = 0; q < 2 * NB; ++q) {
-                    const uint32_t w0 = (sc[q >> 3][0][(q >> 2) & 1] >> 4) & 0x0F0F0F0Fu;
-                    const uint32_t w1 = (sc[q >> 3][1][(q >> 2) & 1] >> 4) & 0x0F0F0F0Fu;
-                    const float sj = sxw[m * sstride + q];
-                    z0 = fmaf(fmaf(byte_magic(w0, q & 3), m0f, nm0), sj, z0);   // (dmin * m) * S
-                    z1 = fmaf(fmaf(byte_magic(w1, q & 3), m1f, nm1), sj, z1);
-                }
-                acc[nt][cc] -= z0;
-                acc[nt][2 + cc] -= z1;
+            for (int hi = 0; hi < 2; ++hi) {
+                const bool kin = live && (hi == 0 || NB == 8);
+                const float2 sv = kin ? *reinterpret_cast<const float2 *>(sxw + m * sstride + 2 * t + 8 * hi)
+                                      : make_float2(0.f, 0.f);
+                uint32_t h0p, m0p, l0p, h1p, m1p, l1p;
+                split3(sv.x, h0p, m0p, l0p);
+                split3(sv.y, h1p, m1p, l1p);
+                b[hi][0] = h0p | (h1p << 16);
+                b[hi][1] = m0p | (m1p << 16);
+                b[hi][2] = l0p | (l1p << 16);
             }
+            float cz[4];
+            mma_zero<true>(cz, am, b[0][0], b[1][0]);
+            mma_acc<true>(cz, am, b[0][1], b[1][1]);
+            mma_acc<true>(cz, am, b[0][2], b[1][2]);
+            acc[nt][0] = fmaf(-m0f, cz[0], acc[nt][0]);
+            acc[nt][1] = fmaf(-m0f, cz[1], acc[nt][1]);
+            acc[nt][2] = fmaf(-m1f, cz[2], acc[nt][2]);
+            acc[nt][3] = fmaf(-m1f, cz[3], acc[nt][3]);
+        }
     }
 
     // box: this warp's chunk, row 0, in the stage; half: which half of the
@@ -743,7 +760,7 @@ struct Exact {
                 }
             }
         } else if constexpr (FMT == F_Q2_K) {
-            compute_q2(box, half, acc, t, M, sxw, sstride);
+            compute_q2(box, half, acc, g, t, M, sxw, sstride);
         } else if constexpr (FMT == F_Q6_KS) {
             compute_q6<2>(box + sr0, box + sr1, half, acc, t);
         } else if constexpr (FMT == F_Q6_K) {
