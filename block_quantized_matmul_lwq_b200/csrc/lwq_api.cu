@@ -146,9 +146,8 @@ inline size_t gemv_smem(int kf, int cps, int stages, int nt, bool i8, int xt, in
         .total;
 }
 
-// Formats with a tensor-core GEMV decoder (their packed rows are 16-byte
-// multiples, as the weight stream's tensor map needs); the others take the
-// simple kernel.
+// Formats with a tensor-core GEMV decoder (all of them); tc_gemv_eligible adds
+// the shape conditions of their weight streams.
 bool tc_gemv_format(int wf) {
     return wf == LWQ_Q8_0 || wf == LWQ_Q4_0 || wf == LWQ_Q4_K || wf == LWQ_Q5_K || wf == LWQ_Q2_K || wf == LWQ_Q6_K;
 }

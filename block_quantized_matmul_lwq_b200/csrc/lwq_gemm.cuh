@@ -738,8 +738,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 }
 
 // ---------------------------------------------------------------- host side
-// Formats with a tcgen05 GEMM decoder; their packed rows must be 16-byte
-// multiples (the weight tensor map's row stride): Q6_K needs K % 2048 == 0.
+// Formats with a tcgen05 GEMM decoder (all of them); gemm_eligible adds the
+// conditions of their weight streams.
 inline bool gemm_format(int wf) {
     return wf == LWQ_Q8_0 || wf == LWQ_Q4_0 || wf == LWQ_Q4_K || wf == LWQ_Q5_K || wf == LWQ_Q6_K || wf == LWQ_Q2_K;
 }

@@ -2,19 +2,21 @@
 //
 // Design (sm_100a):
 //  * A persistent grid of one CTA per SM per call (16 compute warps, a TMA
-//    producer and two reducers).  Every CTA triggers its programmatic dependents
+//    producer and two or four reducers).  Every CTA triggers its programmatic dependents
 //    at once, so the next call on the stream (a programmatic dependent
 //    launch) is scheduled as early as possible and takes each SM as soon as
 //    this call's CTA there exits.
 //  * CTA (split s, row group r) owns a slice of K (split-K factor S) and
 //    walks the 16-row weight tiles r, r+G, r+2G, ...  A producer warp stages,
 //    per tile, the tile's packed rows for all of the CTA's K chunks (256
-//    weights each) with one 3-D TMA load into a ring of shared-memory stages.
+//    weights each) with one 3-D TMA load into a ring of shared-memory stages
+//    (Q6_K: one 2-D box per chunk; row slots: one box per row).
 //  * Sixteen compute warps each own 256 (or 128) weights of the CTA's K slice
 //    and keep that slice of x in registers for the whole kernel, laid out as
 //    tensor-core B fragments.  Per tile a warp decodes its packed bytes in
-//    registers straight into A fragments holding the *signed* codes exactly
-//    (q - 8 for Q4_0, q for Q8_0, the unsigned nibble for Q4_K) and runs one
+//    registers straight into A fragments holding the codes exactly (q - 8 for
+//    Q4_0, q for Q8_0, q - 32 for Q6_K, the unsigned code for Q4_K, Q5_K and
+//    Q2_K) and runs one
 //    two-step mma.sync chain per 32-weight block, then adds d_block * chain
 //    into its fp32 accumulators.  A code of zero weight therefore contributes
 //    exactly nothing, however large the activation it meets.
@@ -28,10 +30,12 @@
 //    and bf16 x whose largest element in a warp's slice is far outside
 //    [2^-60, 2^60] are scaled by a power of two first (exact), and the scale
 //    is undone on the fp32 results.
-//  * Q4_K: per 32-weight sub-block j, y += (d * sc_j) * (sum q x) in fp32
+//  * Q4_K (Q5_K, Q2_K): per sub-block j, y += (d * sc_j) * (sum q x) in fp32
 //    (d * sc_j is exact in fp32), and once per tile y -= dmin * sum_j m_j S_j
-//    with S_j the sub-block sums of x, which the warp keeps in shared memory.
-//  * Two reducer warps (8 rows each) sum the compute warps' partial tiles in a fixed order
+//    with S_j the sub-block sums of x (kept in shared memory), as three bf16
+//    MMAs with S split into exact parts.
+//  * Two reducer warps (8 rows each; four of 4 rows for Q4_0 and Q8_0 at three
+//    column tiles) sum the compute warps' partial tiles in a fixed order
 //    and the parts of each activation row, and writes y, or, with split-K,
 //    fp32 partials to the workspace, which a small follow-up kernel (a
 //    programmatic dependent launch) adds in split order.  Results are

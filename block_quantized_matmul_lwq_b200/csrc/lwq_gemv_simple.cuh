@@ -1,6 +1,7 @@
 // Simple GEMV for the shapes the tensor-core paths do not take: K not a
-// multiple of 256 (only Q8_0 and Q4_0 allow that), and K-quant rows whose
-// byte stride is not a multiple of 16 (Q6_K, Q2_K), at any M.  One warp per
+// multiple of 256 (only Q8_0 and Q4_0 allow that), and Q6_K or Q2_K matrices
+// that are not a whole number of 16-byte units (N * row bytes; their row
+// slots need it), at any M.  One warp per
 // weight row; lanes stride over 32-weight units, decode them with byte loads
 // and accumulate in fp32 for up to 16 activation rows; a warp shuffle
 // reduction finishes each output.  Correct for every valid shape, not tuned.
