@@ -1003,8 +1003,69 @@ struct Q40I8 {
         load_x(S.xp, S.M, S.nk, k0, lane);
     }
 
+    // One block of one activation row: lanes 4G .. 4G+3 (t = lane & 3) take its 32
+    // elements, 8 each at the k-slots of their B fragment; returns the lane's two
+    // code words and the block's scale d.
+    __device__ static __forceinline__ void quant_block(const void *x, long e, int hb, int t, uint32_t &q0,
+                                                       uint32_t &q1, float &d) {
+        using Raw = typename RawPair<XT>::T;
+        const Raw r0 = RawPair<XT>::load(x, e + cb0(hb, t)), r1 = RawPair<XT>::load(x, e + cb2(hb, t));
+        const Raw r2 = RawPair<XT>::load(x, e + 16 + cb0(hb, t)), r3 = RawPair<XT>::load(x, e + 16 + cb2(hb, t));
+        const float2 f0 = RawPair<XT>::get(r0), f1 = RawPair<XT>::get(r1), f2 = RawPair<XT>::get(r2),
+                     f3 = RawPair<XT>::get(r3);
+        const float v[8] = {f0.x, f0.y, f1.x, f1.y, f2.x, f2.y, f3.x, f3.y};
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        const bool zero = !(amax >= 7.888609052210118e-31f);   // 2^-100
+        d = zero ? 0.f : amax / 127.f;
+        const float sc = zero ? 0.f : 127.f / amax;
+        q0 = pack_s8(q8(v[0], sc), q8(v[1], sc), q8(v[2], sc), q8(v[3], sc));
+        q1 = pack_s8(q8(v[4], sc), q8(v[5], sc), q8(v[6], sc), q8(v[7], sc));
+    }
+
     __device__ __forceinline__ void load_x(const void *x, int M, int K, long k0, int lane) {
         const int g = lane >> 2, t = lane & 3;
+        constexpr float DSF = (Q8 || QK) ? 1.f : 0.0625f;   // Q4_0 codes enter as 16 (u - 8)
+        if (M <= 4) {
+            // Few rows: lane group G quantizes block G of every row (M blocks in a row of
+            // dependent steps instead of 8), then the codes move to the lanes whose B
+            // fragments hold them (row g, block b: group b's result for row g) and the
+            // scales to the lanes whose columns they scale (rows 2t, 2t + 1).
+            inv = 1.f;
+            uint32_t tq[4][2];
+            float td[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (j < M) quant_block(x, (long)j * K + k0 + 32 * g, g & 1, t, tq[j][0], tq[j][1], td[j]);
+                else tq[j][0] = tq[j][1] = 0u, td[j] = 0.f;
+            }
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                uint32_t q0 = 0u, q1 = 0u;
+                float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (j >= M) break;   // uniform
+                    const uint32_t a0 = __shfl_sync(0xffffffffu, tq[j][0], 4 * b + t);
+                    const uint32_t a1 = __shfl_sync(0xffffffffu, tq[j][1], 4 * b + t);
+                    const float dj = __shfl_sync(0xffffffffu, td[j], 4 * b);
+                    if (g == j) {
+                        q0 = a0;
+                        q1 = a1;
+                    }
+                    if (2 * t == j) d0 = dj;
+                    if (2 * t + 1 == j) d1 = dj;
+                }
+                xq[b][0] = q0;
+                xq[b][1] = q1;
+                dx[b][0] = DSF * d0;
+                dx[b][1] = DSF * d1;
+            }
+            return;
+        }
         const bool live = g < M;
         const long base = (live ? (long)g * K : 0L) + k0;   // a dead column reads row 0, zeroed below
         using Raw = typename RawPair<XT>::T;
