@@ -24,7 +24,9 @@ CASES = [("q4_k", "f16", 1, 4096, 11008),    # split-K
          ("q8_0", "f32", 1, 4096, 4096),
          ("q4_0", "bf16", 16, 333, 6144),    # 16 activation rows, split-K, ragged N
          ("q6_k", "f16", 2, 500, 8192),      # per-superblock boxes, split-K
-         ("q5_k", "bf16", 3, 300, 4096)]
+         ("q5_k", "bf16", 3, 300, 4096),
+         ("q6_k", "bf16", 2, 96, 11008),     # row slots (9030-byte rows), split-K
+         ("q2_k", "f32", 3, 120, 11008)]     # row slots (3612-byte rows)
 
 
 @pytest.fixture(scope="module")
