@@ -638,6 +638,9 @@ def run_gpu_arm(args):
     if not args.no_sweep:
         ws_bytes = max([ws_bytes] + [lwq.lwq_workspace_size(lwq.fmt_code(f, "f16"), max(inputs.SWEEP_MS), n, k)
                                      for f in inputs.SWEEP_FMTS for k, n in inputs.SWEEP_SHAPES_KN])
+    if not args.no_attention:
+        ws_bytes = max([ws_bytes] + [lwq.lwq_attention_workspace_size(s["B"], s["H"], s["Hkv"], s["L"], s["D"])
+                                     for s in inputs.ATTENTION_WORKLOADS.values()])
     ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
     lwq.lwq_init(ws, ws.numel())
 
