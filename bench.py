@@ -480,7 +480,8 @@ def cpu_baseline(workload: str, budget_s: float = 15.0) -> dict:
 def host_enqueue_cost(lwq, dev, n: int = 10000, batch: int = 200) -> dict:
     """Host time of one lwq_matmul call (the headline's M=1 call) through the C ABI: median
     over n calls, timed in batches with the stream drained between batches so that no call
-    waits for room in the launch queue; a no-op call into the library gives the ctypes cost."""
+    waits for room in the launch queue; the same calls with M = 0, which the first argument check
+    refuses, give what ctypes costs for each signature."""
     import torch
     fmt, act, M, N, K, seed = step_calls(HEADLINE)[0]
     W = torch.from_numpy(call_weights(fmt, N, K, seed)).to(dev)
@@ -494,8 +495,12 @@ def host_enqueue_cost(lwq, dev, n: int = 10000, batch: int = 200) -> dict:
     import ctypes
     cfg = lwq.lwq_config()
     plan_args = (code, M, N, K, ctypes.byref(cfg))
+    # the same entry points with the same arguments except M = 0, refused by their first check:
+    # what ctypes itself costs for each signature
+    call0_args = (code, W.data_ptr(), x.data_ptr(), y.data_ptr(), 0, N, K, sp)
+    plan0_args = (code, 0, N, K, ctypes.byref(cfg))
     launches = 0
-    per_call, per_noop, per_plan = [], [], []
+    per_call, per_call0, per_plan, per_plan0 = [], [], [], []
     for i in range(-2, n // batch):
         stream.synchronize()
         t0 = time.perf_counter()
@@ -506,21 +511,26 @@ def host_enqueue_cost(lwq, dev, n: int = 10000, batch: int = 200) -> dict:
         stream.synchronize()
         t2 = time.perf_counter()
         for _ in range(batch):
-            lib.lwq_version()
+            lib.lwq_matmul(*call0_args)
         t3 = time.perf_counter()
         for _ in range(batch):
             lib.lwq_select_config(*plan_args)
         t4 = time.perf_counter()
+        for _ in range(batch):
+            lib.lwq_select_config(*plan0_args)
+        t5 = time.perf_counter()
         if i >= 0:
             per_call.append((t1 - t0) / batch * 1e6)
-            per_noop.append((t3 - t2) / batch * 1e6)
+            per_call0.append((t3 - t2) / batch * 1e6)
             per_plan.append((t4 - t3) / batch * 1e6)
-    med, noop, plan = statistics.median(per_call), statistics.median(per_noop), statistics.median(per_plan)
-    # the library's own host work per call: argument checks and the tile choice (lwq_select_config
-    # runs the same checks and planner); the rest of a call is the cached tensor-map lookup and the
-    # CUDA launch itself
-    return {"median_us_per_call": round(med, 3), "ctypes_noop_us": round(noop, 3),
-            "library_us_per_call": round(med - noop, 3), "dispatch_us_per_call": round(plan - noop, 3),
+            per_plan0.append((t5 - t4) / batch * 1e6)
+    med, call0 = statistics.median(per_call), statistics.median(per_call0)
+    plan, plan0 = statistics.median(per_plan), statistics.median(per_plan0)
+    # the library's own host work per call (argument checks, the tile choice, the cached tensor-map
+    # lookup and the CUDA launch), and of it the checks and the tile choice alone (lwq_select_config
+    # runs the same checks and planner), each less its refused call's cost
+    return {"median_us_per_call": round(med, 3), "ctypes_us_per_call": round(call0, 3),
+            "library_us_per_call": round(med - call0, 3), "dispatch_us_per_call": round(plan - plan0, 3),
             "calls": n, "kernels_per_call": launches,
             "call": {"fmt": fmt, "act": act, "M": M, "N": N, "K": K}}
 
