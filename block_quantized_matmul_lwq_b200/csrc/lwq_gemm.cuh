@@ -9,11 +9,13 @@
 //
 // Roles (one persistent CTA per SM, warp-specialized):
 //   warp 0      TMA producer: packed weight chunks [128 or 256 rows][256 weights]
-//               and activation tiles [BN tokens][64 k] (128-byte swizzle)
 //   warp 1      TMEM allocator and single-thread UMMA issuer
 //   warps 2..17 dequantizers: packed chunk -> bf16/fp16 weight tile
 //               [128 rows][64 k] per half in the UMMA K-major 128-byte-swizzle layout
 //   warps 18-21 epilogue: TMEM -> registers -> y (fp32), coalesced along N
+//   warp 22     TMA producer: activation tiles [BN tokens][64 k] (128-byte swizzle)
+//               (a warp of its own: two producers in one warp's lanes delayed each
+//               other's requests while one of them waited)
 // Weight tile: 128 rows (one UMMA per K step) or 256 rows (two, one per
 // 128-row half, sharing the activation tile: half the L2 traffic of
 // activations per flop, which bounds the 128-row tiles).  UMMA shape: M = 128
@@ -35,7 +37,8 @@ constexpr int GEMM_BK = 64;           // k per k-block (one 128-byte swizzle ato
 constexpr int GEMM_KB_PER_CHUNK = 4;  // k-blocks per packed 256-weight chunk
 constexpr int GEMM_DQ_WARPS = 16;
 constexpr int GEMM_EPI_WARPS = 4;
-constexpr int GEMM_THREADS = (2 + GEMM_DQ_WARPS + GEMM_EPI_WARPS) * 32;
+constexpr int GEMM_THREADS = (3 + GEMM_DQ_WARPS + GEMM_EPI_WARPS) * 32;
+constexpr int GEMM_ACT_WARP = 2 + GEMM_DQ_WARPS + GEMM_EPI_WARPS;
 
 struct GemmPlan {
     int warps, stages, ctas, tile_n, tile_m, splits;
@@ -466,11 +469,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const uint32_t tmem_base = *tmem_holder;
 
     if (warp == 0) {
-        // ------------------------------------------------------ TMA producers
-        // Lane 0 streams the packed weight chunks (p ring), lane 1 the activation
-        // k-blocks (ab ring), each as far ahead as its ring allows: a weight chunk
-        // is requested as soon as its slot frees, not behind the activation loads.
-        // With row slots the dequantizer warps fetch the weights themselves (lane 0 idles).
+        // ------------------------------------------------ TMA producer: weights
+        // Lane 0 streams the packed weight chunks (p ring) as far ahead as the ring
+        // allows: a chunk is requested as soon as its slot frees.  The activation
+        // k-blocks have their own producer warp (GEMM_ACT_WARP), so neither
+        // producer's waits hold up the other's requests.  With row slots the
+        // dequantizer warps fetch the weights themselves (this warp idles).
         bool slot_mode = false;
         if constexpr (FMT == F_Q6_K || FMT == F_Q2_K) slot_mode = a.slots != 0;
         if (lane == 0 && !slot_mode) {
@@ -501,29 +505,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             // drain: the last loads land before the CTA may exit (runs once; divisions are fine here)
             for (int j = max(0, ci - P); j < ci; ++j)
                 mbar_wait(&p_full[j % P], (j / P) & 1, a.timeout_ns, DEVERR_GEMM_WAIT);
-        } else if (lane == 1) {
-            tma_prefetch_desc(&xmap);
-            pdl_wait();   // x may be the preceding kernel's output
-            int kbi = 0, s = 0;
-            uint32_t ph = 0;
-            bool ok = true;
-            for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
-                const int tile = item / a.splits, ks = item % a.splits;
-                const int tt = tile % a.n_ttiles;
-                const int k0 = ks * a.cps * GEMM_KB_PER_CHUNK;
-                const int k1 = min(a.nchunks, (ks + 1) * a.cps) * GEMM_KB_PER_CHUNK;
-                for (int k = k0; k < k1; ++k, ++kbi) {
-                    if (kbi >= SB && !(ok = mbar_wait(&b_empty[s], ph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
-                    mbar_arrive_expect_tx(&b_full[s], B_BYTES);
-                    tma_load_2d(Bs + (size_t)s * BS_BYTES, &xmap, &b_full[s], k * GEMM_BK, tt * BN);
-                    if (++s == SB) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
-                }
-            }
-            for (int j = max(0, kbi - SB); j < kbi; ++j)
-                mbar_wait(&b_full[j % SB], (j / SB) & 1, a.timeout_ns, DEVERR_GEMM_WAIT);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------- UMMA issuer
@@ -568,6 +549,33 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             // every issued MMA completes before TMEM is released
             umma_commit(mma_done);
             mbar_wait(mma_done, 0, a.timeout_ns, DEVERR_GEMM_WAIT);
+        }
+    } else if (warp == GEMM_ACT_WARP) {
+        // --------------------------------------------- TMA producer: activations
+        // Lane 0 streams the activation k-blocks (b ring) as far ahead as it allows.
+        if (lane == 0) {
+            tma_prefetch_desc(&xmap);
+            pdl_wait();   // x may be the preceding kernel's output
+            int kbi = 0, s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+                const int tile = item / a.splits, ks = item % a.splits;
+                const int tt = tile % a.n_ttiles;
+                const int k0 = ks * a.cps * GEMM_KB_PER_CHUNK;
+                const int k1 = min(a.nchunks, (ks + 1) * a.cps) * GEMM_KB_PER_CHUNK;
+                for (int k = k0; k < k1; ++k, ++kbi) {
+                    if (kbi >= SB && !(ok = mbar_wait(&b_empty[s], ph ^ 1u, a.timeout_ns, DEVERR_GEMM_WAIT))) break;
+                    mbar_arrive_expect_tx(&b_full[s], B_BYTES);
+                    tma_load_2d(Bs + (size_t)s * BS_BYTES, &xmap, &b_full[s], k * GEMM_BK, tt * BN);
+                    if (++s == SB) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            for (int j = max(0, kbi - SB); j < kbi; ++j)
+                mbar_wait(&b_full[j % SB], (j / SB) & 1, a.timeout_ns, DEVERR_GEMM_WAIT);
         }
     } else if (warp < 2 + GEMM_DQ_WARPS) {
         // ------------------------------------------------------ dequantizers
