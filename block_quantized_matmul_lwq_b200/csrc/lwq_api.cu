@@ -732,8 +732,10 @@ cudaError_t launch_attn(const AttnArgs &a, cudaStream_t st) {
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || a.S == 1) return e;
-    // the splits' merge: a programmatic dependent launch that waits for the split kernel
-    return launch_k(attn_combine_kernel<D>, a.B * a.H, D, 0, st, true, (const float *)a.part, a.out, a.S);
+    // the splits' merge: a programmatic dependent launch that waits for the split kernel; a CTA per
+    // (sequence, head) and 32 columns
+    return launch_k(attn_combine_kernel<D>, a.B * a.H * (D / 32), 32 * attn_combine_warps(a.S), 0, st, true,
+                    (const float *)a.part, a.out, a.S);
 }
 
 template <int XT, int D>

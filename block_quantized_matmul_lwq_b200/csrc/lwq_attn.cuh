@@ -442,25 +442,73 @@ __global__ void __launch_bounds__(ATTN_WARPS * 32) attn_split_tc_kernel(const At
     pdl_launch_dependents();
 }
 
-// out[b][h][d] from the S partial results of (b, h): rescale each split to the
-// largest maximum, add in split order, divide by the total weight.
+// out[b][h][d] from the S partial results of (b, h).  A CTA takes one (b, h)
+// and 32 of its D columns (lane = column) with NG = ceil(S / 8) warps (at most
+// 16): warp j takes slots j, j + NG, ... in order with 8 slots' loads in
+// flight, keeping a running maximum and rescaling its weight and weighted
+// values when the maximum grows (an empty split, m = -inf, adds nothing); the
+// warps' results are then rescaled to the largest maximum, added in warp order
+// and divided by the total weight.  S alone fixes the order of every addition.
+// (One thread walking all S splits, twice, made the merge of a long sequence's
+// 32 splits cost more than a tenth of the call.)
+constexpr int ATTN_COMBINE_U = 8;
+inline int attn_combine_warps(int S) {
+    const int ng = (S + ATTN_COMBINE_U - 1) / ATTN_COMBINE_U;
+    return ng < 1 ? 1 : (ng > 16 ? 16 : ng);
+}
 template <int D>
-__global__ void __launch_bounds__(D) attn_combine_kernel(const float *__restrict__ part, float *__restrict__ out,
-                                                          int S) {
+__global__ void __launch_bounds__(512) attn_combine_kernel(const float *__restrict__ part, float *__restrict__ out,
+                                                            int S) {
+    constexpr int U = ATTN_COMBINE_U;
+    __shared__ float gm[16], gl[16], ga[16][32];
     pdl_wait();
-    const size_t bh = blockIdx.x;
-    const int d = threadIdx.x;
+    const int NG = blockDim.x >> 5;
+    const size_t bh = blockIdx.x / (D / 32);
+    const int j = threadIdx.x >> 5, c = threadIdx.x & 31, d = 32 * (blockIdx.x % (D / 32)) + c;
     const float *p = part + bh * S * (D + 2);
-    float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, __ldcg(p + (size_t)s * (D + 2)));
-    float L = 0.f, A = 0.f;
-    for (int s = 0; s < S; ++s) {
-        const float *ps = p + (size_t)s * (D + 2);
-        const float f = exp2f(__ldcg(ps) - M);   // 0 for an empty split
-        L = fmaf(__ldcg(ps + 1), f, L);
-        A = fmaf(__ldcg(ps + 2 + d), f, A);
+    float M = -INFINITY, L = 0.f, A = 0.f;
+    for (int s0 = j; s0 < S; s0 += NG * U) {
+        float mv[U], lv[U], av[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {   // a slot past S reads slot 0 and is skipped below
+            const int s = s0 + u * NG;
+            const float *ps = p + (size_t)(s < S ? s : 0) * (D + 2);
+            mv[u] = s < S ? __ldcg(ps) : -INFINITY;
+            lv[u] = __ldcg(ps + 1);
+            av[u] = __ldcg(ps + 2 + d);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (mv[u] == -INFINITY) continue;
+            const float mn = fmaxf(M, mv[u]);
+            const float fo = exp2f(M - mn), fn = exp2f(mv[u] - mn);   // fo = 0 while M = -inf
+            L = fmaf(L, fo, lv[u] * fn);
+            A = fmaf(A, fo, av[u] * fn);
+            M = mn;
+        }
     }
-    out[bh * D + d] = A / L;
+    if (NG == 1) {   // split 0 holds key 0: M is finite
+        out[bh * D + d] = A / L;
+        return;
+    }
+    if (c == 0) {
+        gm[j] = M;
+        gl[j] = L;
+    }
+    ga[j][c] = A;
+    __syncthreads();
+    if (j == 0) {   // warp 0 holds split 0: Mt is finite
+        float Mt = -INFINITY;
+        for (int g = 0; g < NG; ++g) Mt = fmaxf(Mt, gm[g]);
+        float Lt = 0.f, At = 0.f;
+        for (int g = 0; g < NG; ++g) {
+            if (gm[g] == -INFINITY) continue;
+            const float f = exp2f(gm[g] - Mt);
+            Lt = fmaf(gl[g], f, Lt);
+            At = fmaf(ga[g][c], f, At);
+        }
+        out[bh * D + d] = At / Lt;
+    }
 }
 
 // Splits of the sequence (each at least 64 keys, a multiple of 16).  A small
