@@ -519,13 +519,19 @@ __global__ void __launch_bounds__(512) attn_combine_kernel(const float *__restri
 //  * Grouped heads (the tensor-core pass, 2 CTAs resident per SM): the split
 //    count with the least modelled time, waves x (keys per split + 128), the
 //    128 standing for a CTA's ramp; a last wave that leaves most SMs idle
-//    costs a whole wave.
+//    costs a whole wave.  With 8 or fewer (sequence, kv head) pairs, one CTA
+//    per SM instead (splits = SMs / pairs).
 inline void attn_splits(int B, int H, int Hkv, int Lmax, int sms, int *S, int *chunk) {
     const long pairs = (long)B * Hkv;
     const long smax = (Lmax + 63) / 64;
     long best_s = 1;
     if (H == Hkv) {
         best_s = (4L * sms + pairs - 1) / pairs;
+    } else if (pairs <= 8) {
+        // few (sequence, kv head) pairs, i.e. long sequences: one CTA per SM.  Two per SM on half the keys each
+        // measured slower (1 x 32768 keys, 8 kv heads: 18 splits 28.9 us, 37 splits 30.9 us; 2 x 16384, 4 kv
+        // heads: 20.5 and 22.3 us): the SM's bandwidth is shared, and the merge has twice the splits.
+        best_s = sms / pairs;
     } else {
         const long slots = 2L * sms;
         double best = -1.0;
