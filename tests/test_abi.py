@@ -223,3 +223,19 @@ def test_int8_flag_plan():
         with pytest.raises(lwq.LwqError) as e:
             lwq.lwq_select_config(fmt, M, 64, K)
         assert e.value.status == lwq.LWQ_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("B,H,Hkv,L,D,splits", [
+    (1, 32, 8, 32768, 128, 18),   # 8 (sequence, kv head) pairs: one CTA per SM, 148 // 8 splits
+    (2, 32, 4, 16384, 128, 18),
+    (2, 8, 4, 300, 64, 5),        # at most one split per 64 keys
+    (4, 32, 8, 8192, 128, 9),     # 32 pairs: the wave model (288 CTAs, two per SM)
+    (16, 32, 8, 4096, 128, 2),
+    (64, 32, 8, 2048, 128, 1),    # enough pairs: no split, no workspace
+    (16, 32, 32, 4096, 128, 2),   # one query head per kv head: about four CTAs per SM
+])
+def test_attention_split_plan(B, H, Hkv, L, D, splits):
+    """The decode-attention work division, read back through the workspace it needs ([B][H][S][D + 2] fp32
+    partials when the keys are split).  Without a GPU the planner takes a B200's 148 SMs."""
+    ws = lwq.lwq_attention_workspace_size(B, H, Hkv, L, D)
+    assert ws == (B * H * splits * (D + 2) * 4 if splits > 1 else 0)
