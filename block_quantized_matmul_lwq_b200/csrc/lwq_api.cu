@@ -118,6 +118,7 @@ struct Plan {
     bool i8;         // GEMV with int8 activation blocks (LWQ_FLAG_ACT_I8)
     int m_group;     // activation rows per pass
     int cps;         // GEMV: chunks of 256 weights per split (the depth of one TMA box)
+    int kw;          // GEMV: weights of K per compute warp and chunk at nt column tiles (256 or 128)
     size_t smem;
     size_t ws_need;  // workspace bytes for one pass
 };
@@ -278,8 +279,14 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
     int groups = force && force->ctas ? force->ctas / S : sms / S;
     if (groups < 1) groups = 1;
     if (groups > row_tiles) groups = row_tiles;
+    // Two column tiles whose K slice is 8 chunks or fewer (16-bit x with 9..16 rows, or fp32 x with 4 or 5 rows
+    // where the staged slice leaves room for no more): half a chunk per warp, so that all 16 compute warps
+    // work and each holds half the B fragments.  A warp per chunk left 8 warps idle and spilled registers.
+    int kwe = kw;
+    if (!p->i8 && p->nt == 2 && kw == CHUNK && 2 * cps <= GEMV_W && !(force && force->warps)) kwe = CHUNK / 2;
+    p->kw = kwe;
     p->cps = cps;
-    p->cfg.warps = cps * wpc;
+    p->cfg.warps = cps * (CHUNK / kwe);
     p->cfg.stages = stages;
     p->cfg.splits = S;
     p->cfg.ctas = S * groups;
@@ -332,28 +339,32 @@ cudaError_t ensure_smem(const void *kern, size_t smem) {
     return cudaSuccess;
 }
 
-template <int FMT, int XT, int NT, bool I8 = false>
+template <int FMT, int XT, int NT, bool I8 = false, int KW = (I8 ? 256 : gemv_kw(NT))>
 cudaError_t launch_gemv(const CUtensorMap &map, const GemvArgs &a, int ctas, size_t smem, cudaStream_t st) {
-    auto kern = gemv_kernel<FMT, XT, NT, I8>;
+    auto kern = gemv_kernel<FMT, XT, NT, I8, KW>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), smem);
     if (e != cudaSuccess) return e;
     return launch_k(kern, ctas, gemv_threads(FMT, NT), smem, st, a.overlap != 0, map, a);
 }
 
 // NT = n8 column tiles: fp32 activations take 1..3 (3 parts per row, 8 rows
-// at most), 16-bit ones 1..2 (16 rows at most); int8 blocks one.
+// at most), 16-bit ones 1..2 (16 rows at most); int8 blocks one.  kw: the
+// plan's K per warp and chunk at two tiles (128 or 256).
 template <int FMT, int XT>
-cudaError_t launch_gemv_nt(int nt, const CUtensorMap &map, const GemvArgs &a, int ctas, size_t smem, cudaStream_t st) {
+cudaError_t launch_gemv_nt(int nt, int kw, const CUtensorMap &map, const GemvArgs &a, int ctas, size_t smem,
+                           cudaStream_t st) {
     if (nt == 1) return launch_gemv<FMT, XT, 1>(map, a, ctas, smem, st);
-    if (nt == 2) return launch_gemv<FMT, XT, 2>(map, a, ctas, smem, st);
+    if (nt == 2)
+        return kw == CHUNK / 2 ? launch_gemv<FMT, XT, 2, false, CHUNK / 2>(map, a, ctas, smem, st)
+                               : launch_gemv<FMT, XT, 2>(map, a, ctas, smem, st);
     if constexpr (XT == X_F32) {
         if (nt == 3) return launch_gemv<FMT, XT, 3>(map, a, ctas, smem, st);
     }
     return cudaErrorInvalidValue;
 }
 
-cudaError_t dispatch_gemv(int wf, int xt, int nt, bool i8, const CUtensorMap &map, const GemvArgs &a, int ctas,
-                          size_t smem, cudaStream_t st) {
+cudaError_t dispatch_gemv(int wf, int xt, int nt, int kw, bool i8, const CUtensorMap &map, const GemvArgs &a,
+                          int ctas, size_t smem, cudaStream_t st) {
     if (i8) {
         if (nt != 1) return cudaErrorInvalidValue;
         if (wf == LWQ_Q4_0) {
@@ -373,10 +384,10 @@ cudaError_t dispatch_gemv(int wf, int xt, int nt, bool i8, const CUtensorMap &ma
         }
         return cudaErrorInvalidValue;
     }
-#define LWQ_GV(F)                                                                   \
-    if (xt == X_F32) return launch_gemv_nt<F, X_F32>(nt, map, a, ctas, smem, st);  \
-    if (xt == X_F16) return launch_gemv_nt<F, X_F16>(nt, map, a, ctas, smem, st);  \
-    return launch_gemv_nt<F, X_BF16>(nt, map, a, ctas, smem, st);
+#define LWQ_GV(F)                                                                       \
+    if (xt == X_F32) return launch_gemv_nt<F, X_F32>(nt, kw, map, a, ctas, smem, st);  \
+    if (xt == X_F16) return launch_gemv_nt<F, X_F16>(nt, kw, map, a, ctas, smem, st);  \
+    return launch_gemv_nt<F, X_BF16>(nt, kw, map, a, ctas, smem, st);
     switch (wf) {
     case LWQ_Q4_0: { LWQ_GV(F_Q4_0) }
     case LWQ_Q8_0: { LWQ_GV(F_Q8_0) }
@@ -643,7 +654,8 @@ int gemv_run(const Plan &p, int fmt, const void *Wq, const void *x, float *y, in
         a.timeout_ns = kTimeoutNs;
         a.overlap = overlap;
         const int nt = gemv_nt(xt, p.i8, mg);
-        cudaError_t e = dispatch_gemv(wf, xt, nt, p.i8, map, a, p.cfg.ctas,
+        const int kw = nt == p.nt ? p.kw : gemv_kw(nt);   // a last, shorter pass may take fewer tiles
+        cudaError_t e = dispatch_gemv(wf, xt, nt, kw, p.i8, map, a, p.cfg.ctas,
                                       gemv_smem(gemv_kfmt(wf, K), p.cps, p.cfg.stages, nt, p.i8, xt, mg), st);
         if (e != cudaSuccess) return LWQ_ERR_CUDA;
         ++n;

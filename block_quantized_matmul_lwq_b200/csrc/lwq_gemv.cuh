@@ -134,7 +134,9 @@ __host__ __device__ constexpr int gemv_parts(int xt, bool i8) { return (xt == X_
 // half a chunk with three (their B fragments take 32 registers per tile and
 // chunk).  A whole chunk per warp means fewer, larger tiles per CTA and K up
 // to 4096 in one CTA (no split-K): measured faster at two tiles even with a
-// few registers spilled (fp32, M = 4: 17.2 -> 14.4 us).
+// few registers spilled (fp32, M = 4: 17.2 -> 14.4 us).  The planner takes
+// half a chunk at two tiles too when a CTA's K slice has 8 chunks or fewer,
+// which a warp per chunk would leave to half the warps.
 __host__ __device__ constexpr int gemv_kw(int nt) { return nt <= 2 ? 256 : 128; }
 // Floats per row of a reduction slot: the tile's 8 NT columns and 4 of padding,
 // which spreads the rows of a slot over the shared-memory banks.
@@ -705,6 +707,8 @@ struct Exact {
 #pragma unroll
         for (int hi = 0; hi < 2; ++hi) {   // k-slots 2t, 2t+1 (hi = 0) and 2t+8, 2t+9 (hi = 1)
             const bool kin = hi == 0 || NB == 8;
+            // (the lane's word index puts sc in local memory; a select in its place measured slower:
+            // 11008 x 4096 at M = 1, 12.7 -> 13.4 us, and M = 9..12, 4-7 %)
             am[2 * hi] = kin ? min6_pair_bf16(prmt((sc[hi & (NH - 1)][0][t >> 1] >> 4) & 0x0F0F0F0Fu, 0u, msel)) : 0u;
             am[2 * hi + 1] = kin ? min6_pair_bf16(prmt((sc[hi & (NH - 1)][1][t >> 1] >> 4) & 0x0F0F0F0Fu, 0u, msel)) : 0u;
         }
@@ -1225,14 +1229,15 @@ struct Q40I8 {
     }
 };
 
-template <int FMT, int XT, int NT, bool I8>
-struct GemvImpl : Exact<FMT, XT, NT, gemv_kw(NT)> {};
+// KW: weights of K per compute warp and chunk (256: a warp per chunk; 128: two)
+template <int FMT, int XT, int NT, bool I8, int KW = (I8 ? 256 : gemv_kw(NT))>
+struct GemvImpl : Exact<FMT, XT, NT, KW> {};
 template <int XT>
-struct GemvImpl<F_Q4_0, XT, 1, true> : Q40I8<XT> {};
+struct GemvImpl<F_Q4_0, XT, 1, true, 256> : Q40I8<XT> {};
 template <int XT>
-struct GemvImpl<F_Q8_0, XT, 1, true> : Q40I8<XT, F_Q8_0> {};
+struct GemvImpl<F_Q8_0, XT, 1, true, 256> : Q40I8<XT, F_Q8_0> {};
 template <int XT>
-struct GemvImpl<F_Q4_K, XT, 1, true> : Q40I8<XT, F_Q4_K> {};
+struct GemvImpl<F_Q4_K, XT, 1, true, 256> : Q40I8<XT, F_Q4_K> {};
 
 // ------------------------------------------------------------------ kernel
 // blockDim = gemv_threads(FMT, NT): warps 0..15 compute, warp 16 produces (TMA), the
@@ -1240,11 +1245,10 @@ struct GemvImpl<F_Q4_K, XT, 1, true> : Q40I8<XT, F_Q4_K> {};
 // over four 16K-register sub-partitions, 80 with 21).  Every wait is
 // bounded; a wait that gives up sets a bit of the device error word and ends
 // its warp's loop.
-template <int FMT, int XT, int NT, bool I8>
+template <int FMT, int XT, int NT, bool I8, int KW = (I8 ? 256 : gemv_kw(NT))>
 __global__ void __launch_bounds__(gemv_threads(FMT, NT), 1)
     gemv_kernel(const __grid_constant__ CUtensorMap wmap, const GemvArgs a) {
     constexpr int CB = FmtInfo<FMT>::chunk_bytes;
-    constexpr int KW = I8 ? 256 : gemv_kw(NT);
     constexpr int WPC = CHUNK / KW;            // compute warps per chunk
     constexpr int P = gemv_parts(XT, I8);
     constexpr int RS = gemv_rs(NT);            // floats per row of a reduction slot
@@ -1427,7 +1431,7 @@ __global__ void __launch_bounds__(gemv_threads(FMT, NT), 1)
     // ---------------- compute warps
     if (warp >= nact) return;
     const int ci = warp / WPC, half = warp % WPC;
-    using Impl = GemvImpl<FMT, XT, NT, I8>;
+    using Impl = GemvImpl<FMT, XT, NT, I8, KW>;
     Impl impl;
     typename Impl::Slice sl;
     sl.xp = reinterpret_cast<decltype(sl.xp)>(xs);

@@ -128,8 +128,11 @@ def test_python_constants_match_the_header():
     ("q4_0", "f32", 1, 11008, 4096, 16, 1, 4),     # 3 columns (fp32 parts): one tile, a chunk per warp, K in one CTA
     ("q4_0", "f32", 4, 11008, 4096, 16, 1, 2),     # 12 columns: two tiles, still a chunk per warp (2 stages fit)
     ("q4_0", "f32", 8, 11008, 4096, 16, 2, 4),     # 24 columns: three tiles, half a chunk per warp
-    ("q4_0", "f16", 16, 4096, 4096, 8, 2, 4),      # 16 rows of 16-bit activations: the staged slice limits a CTA to
-                                                   # 14 chunks, so 2 splits, evened out to 8 chunks with room for 4 stages
+    ("q4_0", "f16", 16, 4096, 4096, 16, 2, 4),     # 16 rows of 16-bit activations: the staged slice limits a CTA to
+                                                   # 14 chunks, so 2 splits, evened out to 8 chunks with room for 4
+                                                   # stages, and half a chunk per warp so that all 16 warps work
+    ("q8_0", "f32", 4, 4096, 4096, 16, 2, 4),      # Q8_0, fp32 x, 4 rows: 8 chunks a CTA, half a chunk per warp
+    ("q4_0", "f16", 12, 4096, 4096, 16, 1, 2),     # 12 rows: 16 chunks fit, a chunk per warp
     ("q8_0", "f32", 1, 4096, 4096, 16, 1, 2),      # Q8_0 chunks are twice as large: 2 stages
     ("q8_0", "f16", 1, 32000, 4096, 16, 1, 2),
     ("q4_k", "f16", 1, 4096, 11008, 11, 4, 4),     # K = 43 chunks: 4 splits of 11 balance the CTAs better than 3

@@ -304,3 +304,25 @@ def test_fused_projections_equal_separate_calls(dev, w, a, M):
     assert np.array_equal(y, np.concatenate(ys, axis=1))
     y_ref, den = oracle.matmul(w, stacked, x, act=a)
     assert oracle.normalised_error(y, y_ref, den) <= TOL_GEMV
+
+
+# Two column tiles with a K slice of 8 chunks or fewer: half a chunk of K per warp (all 16 compute warps work).
+HALF_CHUNK_CASES = [
+    ("q4_0", "f16", 16, 300, 4096), ("q4_0", "bf16", 9, 257, 2048), ("q4_0", "f32", 4, 130, 2048),
+    ("q8_0", "f16", 12, 300, 4096), ("q8_0", "f32", 4, 211, 4096), ("q8_0", "bf16", 16, 64, 1024),
+    ("q4_k", "f16", 16, 300, 4096), ("q4_k", "bf16", 10, 129, 2048), ("q4_k", "f32", 5, 96, 2048),
+    ("q5_k", "f16", 12, 300, 4096), ("q5_k", "f32", 4, 211, 4096), ("q5_k", "bf16", 16, 33, 1024),
+    ("q6_k", "f16", 9, 300, 4096), ("q6_k", "f32", 4, 160, 4096), ("q6_k", "bf16", 16, 136, 4352),
+    ("q2_k", "f16", 16, 300, 4096), ("q2_k", "f32", 3, 96, 2048), ("q2_k", "bf16", 11, 160, 2048),
+]
+
+
+@pytest.mark.parametrize("w,a,M,N,K", HALF_CHUNK_CASES)
+def test_half_chunk_warps(dev, w, a, M, N, K):
+    """The two-tile GEMV with half a chunk of K per warp, every format, against the oracle (Q6_K with K = 4352
+    and Q2_K stream as row slots); the plan must be the one under test."""
+    cfg = lwq.lwq_select_config(lwq.fmt_code(w, a), M, N, K)
+    nchunks = K // 256
+    cps = -(-nchunks // cfg.splits)
+    assert cfg.path == 1 and cps <= 8 and cfg.warps == 2 * cps, cfg.as_dict()
+    check_full(w, a, M, N, K, dev, seed=M + N + K)
