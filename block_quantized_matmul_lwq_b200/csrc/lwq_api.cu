@@ -220,7 +220,13 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
     const int mmax = (xt == X_F32 || p->i8) ? 8 : 16;
     p->m_group = M < mmax ? M : mmax;
     p->nt = gemv_nt(xt, p->i8, p->m_group);
-    const int kw = p->i8 ? 256 : gemv_kw(p->nt);
+    // K per warp and chunk: gemv_kw, except the K-quants at two tiles with K <= 4096, which take half a chunk:
+    // their decoders spill with a whole chunk's B fragments (68-132 bytes), and two K splits of half chunks
+    // measured faster than one of whole chunks (M = 9..12 of 16-bit x, M = 3, 4 of fp32 x: Q4_K 1.06-1.16x,
+    // Q2_K up to 1.12x, none slower).  At K = 11008 the same choice was mixed (0.89-1.17x).
+    const bool kq = wf == LWQ_Q4_K || wf == LWQ_Q5_K || wf == LWQ_Q6_K || wf == LWQ_Q2_K;
+    const bool half = p->nt == 2 && kq && K <= 4096 && !(force && force->warps);
+    const int kw = p->i8 ? 256 : (half ? CHUNK / 2 : gemv_kw(p->nt));
     const int wpc = CHUNK / kw;              // compute warps per chunk
     const int cmax = GEMV_W / wpc;           // chunks a CTA can hold
     const int nchunks = K / 256;
