@@ -301,6 +301,19 @@ int make_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, Pl
     return LWQ_OK;
 }
 
+// A GEMV plan whose split-K partials exceed the `have` bytes of workspace (none registered: 0) gives way to
+// the plan with a warp per chunk, where that one needs no more: the K-quants' half chunks split K where a warp
+// per chunk would not, and a call that fits without them still runs.  Forced configurations are kept.
+int fit_plan(int fmt, int M, int N, int K, const lwq_config *force, int sms, size_t have, Plan *p) {
+    if (force || p->cfg.path != 1 || p->ws_need <= have) return LWQ_OK;
+    lwq_config whole = {};
+    whole.path = 1;
+    whole.warps = GEMV_W;
+    Plan q;
+    if (make_plan(fmt, M, N, K, &whole, sms, &q) == LWQ_OK && q.ws_need <= have) *p = q;
+    return LWQ_OK;
+}
+
 // --------------------------------------------------------------- launches
 // Launch on `st`; with `overlap`, as a programmatic dependent launch, so that
 // the kernel may start (and prefetch weights) before the preceding kernel on
@@ -691,6 +704,7 @@ int run(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, c
     const int overlap = (fmt & LWQ_FLAG_OVERLAP) ? 1 : 0;
     Plan p;
     if ((rc = make_plan(fmt, M, N, K, force, sm_count(dev), &p))) return rc;
+    fit_plan(fmt, M, N, K, force, sm_count(dev), g_dev[dev].registered ? g_dev[dev].ws_bytes : 0, &p);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const long rb = (long)K / block_weights(wf) * block_bytes(wf);
     const size_t xelem = (xt == X_F32) ? 4 : 2;

@@ -98,6 +98,7 @@ extern "C" int lwq_matmul_noalloc(int fmt, const void *Wq, const void *x, float 
     if ((rc = lwq::current_device(&dev))) return rc;
     lwq::Plan p;
     if ((rc = lwq::make_plan(fmt, M, N, K, nullptr, lwq::sm_count(dev), &p))) return rc;
+    lwq::fit_plan(fmt, M, N, K, nullptr, lwq::sm_count(dev), kScratchBytes, &p);
     if (p.cfg.path != 1 || M > 16) return LWQ_ERR_UNSUPPORTED;
     if (p.ws_need > kScratchBytes) return LWQ_ERR_WORKSPACE_TOO_SMALL;
     void *scratch = nullptr;

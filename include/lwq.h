@@ -164,7 +164,11 @@ int lwq_shutdown(void);
  * (LWQ_ERR_MISALIGNED).  Calls that use split-K (see lwq_workspace_size) need
  * a registered workspace (LWQ_ERR_NOT_INITIALIZED,
  * LWQ_ERR_WORKSPACE_TOO_SMALL); calls sharing one workspace must be ordered
- * (one stream, or events), since their partial sums share the arena.
+ * (one stream, or events), since their partial sums share the arena.  A GEMV
+ * call whose chosen plan splits K but finds too little workspace takes the
+ * plan with a warp per chunk of K instead when that one needs no more (the
+ * K-quants with 9..16 rows of 16-bit x or 3..5 of fp32 x and K <= 4096), so it
+ * runs as it would with no workspace; lwq_workspace_size covers the faster plan.
  * M > 16 with fp32 activations runs the GEMV path over groups of rows of x.
  */
 int lwq_matmul(int fmt, const void *Wq, const void *x, float *y, int M, int N, int K, void *stream);

@@ -235,6 +235,29 @@ def test_workspace_errors(dev):
 dev_ws_keepalive = []
 
 
+def test_plan_without_split_when_workspace_is_short(dev):
+    """The fastest plan splits K (Q4_K, two tiles, half chunks) but no workspace is registered: the call takes
+    the plan with a warp per chunk, which needs none, and stays correct."""
+    w, a, M, N, K = "q4_k", "f16", 12, 300, 4096
+    fmt = lwq.fmt_code(w, a)
+    assert lwq.lwq_select_config(fmt, M, N, K).splits == 2
+    Wq, x = inputs.make_problem(w, a, M, N, K, seed=9)
+    Wd, xd = to_device(Wq, dev), to_device(x, dev)
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device=dev)
+    lwq.lwq_shutdown()
+    try:
+        rc = lwq.lib().lwq_matmul(fmt, Wd.data_ptr(), xd.data_ptr(), y.data_ptr(), M, N, K, None)
+        assert rc == lwq.LWQ_OK, lwq.lwq_status_string(rc)
+        assert lwq.lwq_last_launch_count() == 1   # no split-K sum
+        torch.cuda.synchronize(dev)
+    finally:
+        ws = torch.zeros(WS_BYTES, dtype=torch.uint8, device=dev)
+        lwq.lwq_init(ws, WS_BYTES)
+        dev_ws_keepalive.append(ws)
+    y_ref, den = oracle.matmul(w, Wq, x, act=a)
+    assert oracle.normalised_error(y.cpu().numpy(), y_ref, den) <= TOL_GEMV
+
+
 def test_bounded_wait_reports_timeout(dev):
     """A wait on an mbarrier that nothing arrives at ends after its bound and reports."""
     torch.cuda.synchronize(dev)
