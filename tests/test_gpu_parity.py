@@ -240,7 +240,7 @@ def test_plan_without_split_when_workspace_is_short(dev):
     the plan with a warp per chunk, which needs none, and stays correct."""
     w, a, M, N, K = "q4_k", "f16", 12, 300, 4096
     fmt = lwq.fmt_code(w, a)
-    assert lwq.lwq_select_config(fmt, M, N, K).splits == 2
+    assert lwq.lwq_select_config(fmt, M, N, K).splits > 1
     Wq, x = inputs.make_problem(w, a, M, N, K, seed=9)
     Wd, xd = to_device(Wq, dev), to_device(x, dev)
     y = torch.full((M, N), float("nan"), dtype=torch.float32, device=dev)
