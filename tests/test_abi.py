@@ -242,3 +242,25 @@ def test_attention_split_plan(B, H, Hkv, L, D, splits):
     partials when the keys are split).  Without a GPU the planner takes a B200's 148 SMs."""
     ws = lwq.lwq_attention_workspace_size(B, H, Hkv, L, D)
     assert ws == (B * H * splits * (D + 2) * 4 if splits > 1 else 0)
+
+
+@pytest.mark.parametrize("w", ["q4_0", "q8_0", "q4_k", "q5_k", "q6_k", "q2_k"])
+@pytest.mark.parametrize("a", ["f32", "f16", "bf16"])
+def test_gemv_warps_per_chunk(w, a):
+    """The GEMV plan's K per warp, read back as warps / chunks per CTA: half a chunk (two warps per chunk) at
+    three column tiles, and at two when a CTA's K slice has 8 chunks or fewer or a K-quant has K <= 4096;
+    otherwise a warp per chunk.  Never more than 16 compute warps."""
+    kq = w in ("q4_k", "q5_k", "q6_k", "q2_k")
+    fmt = lwq.fmt_code(w, a)
+    parts, mmax = (3, 8) if a == "f32" else (1, 16)
+    for M in range(1, 17):
+        for N, K in ((4096, 4096), (4096, 2048), (11008, 4096), (4096, 11008), (300, 1024), (4096, 14336)):
+            cfg = lwq.lwq_select_config(fmt, M, N, K)
+            if cfg.path != 1:
+                continue
+            cps = -(-(K // 256) // cfg.splits)
+            wpc, rem = divmod(cfg.warps, cps)
+            assert rem == 0 and wpc in (1, 2) and cfg.warps <= 16, (M, N, K, cfg.as_dict())
+            nt = -(-min(M, mmax) * parts // 8)
+            half = nt == 3 or (nt == 2 and (cps <= 8 or (kq and K <= 4096)))
+            assert (wpc == 2) == half, (M, N, K, cfg.as_dict())
